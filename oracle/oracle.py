@@ -1,0 +1,221 @@
+"""ctypes front end of the fp64 C oracle (``sa_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` import this module; the library itself never
+does.  The oracle shares no code with the CUDA path.  The method it follows
+is the CSA / HCA hybrid attention of "DeepSeek-V4: Towards Highly Efficient
+Million-Token Context Intelligence Review", section 3-2 (2) "Hybrid attention
+with CSA and HCA" (component table); the readings of what that section leaves
+open are listed in the header of ``sa_oracle.c``.
+
+All bf16 tensors are passed as numpy ``uint16`` bit patterns, e4m3 tensors as
+``uint8`` codes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sa_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (no CUDA involved)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".{os.getpid()}.tmp"
+        subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB_PATH)
+        P = ctypes.c_void_p
+        i64, i32, dbl = ctypes.c_int64, ctypes.c_int32, ctypes.c_double
+        L.or_bf16_to_double.argtypes = [ctypes.c_uint16]
+        L.or_bf16_to_double.restype = dbl
+        L.or_bf16_from_double.argtypes = [dbl]
+        L.or_bf16_from_double.restype = ctypes.c_uint16
+        L.or_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        L.or_e4m3_to_double.restype = dbl
+        L.or_e4m3_from_double_satfinite.argtypes = [dbl]
+        L.or_e4m3_from_double_satfinite.restype = ctypes.c_uint8
+        L.or_compress.argtypes = [P, i64, ctypes.c_int, ctypes.c_int, P]
+        L.or_compress.restype = i64
+        L.or_fp8_quantize.argtypes = [P, i64, ctypes.c_int, P, P]
+        L.or_fp8_quantize.restype = None
+        L.or_index_scores.argtypes = [P, P, i64, ctypes.c_int, P]
+        L.or_index_scores.restype = None
+        L.or_topk.argtypes = [P, i64, i32, P]
+        L.or_topk.restype = i32
+        L.or_attention.argtypes = [P, ctypes.c_int, ctypes.c_int, P, P, P, P, ctypes.c_int, P, i64, dbl, P, P, P]
+        L.or_attention.restype = None
+        L.or_hybrid_query.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, i64,
+                                      ctypes.c_int, P, P, P, P, P, i64,
+                                      ctypes.c_int, P, P, P, P, i64, ctypes.c_int, i32, dbl,
+                                      P, P, P, P, P, P]
+        L.or_hybrid_query.restype = None
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data
+
+
+# -- number formats ---------------------------------------------------------
+
+def bf16_to_double(bits: int) -> float:
+    return lib().or_bf16_to_double(int(bits))
+
+
+def bf16_from_double(x: float) -> int:
+    return int(lib().or_bf16_from_double(float(x)))
+
+
+def e4m3_to_double(code: int) -> float:
+    return lib().or_e4m3_to_double(int(code))
+
+
+def e4m3_from_double(x: float) -> int:
+    return int(lib().or_e4m3_from_double_satfinite(float(x)))
+
+
+def bf16_array_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Decode an array of bf16 bit patterns through the oracle's codec."""
+    table = np.array([lib().or_bf16_to_double(i) for i in range(65536)], dtype=np.float64)
+    return table[np.asarray(bits, dtype=np.uint16)]
+
+
+def e4m3_array_to_f64(codes: np.ndarray) -> np.ndarray:
+    table = np.array([lib().or_e4m3_to_double(i) for i in range(256)], dtype=np.float64)
+    return table[np.asarray(codes, dtype=np.uint8)]
+
+
+# -- the method ---------------------------------------------------------------
+
+def compress(x: np.ndarray, m: int) -> np.ndarray:
+    """O1: x [L][d] uint16 -> [L // m][d] uint16 (mean of each complete block)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    L, d = x.shape
+    out = np.zeros((L // m, d), dtype=np.uint16)
+    n = lib().or_compress(_p(x), L, d, m, _p(out))
+    assert n == L // m
+    return out
+
+
+def fp8_quantize(xc: np.ndarray):
+    """O2: xc [n][d] uint16 -> (codes [n][d] uint8, scales [ceil(n/64)] float32)."""
+    xc = np.ascontiguousarray(xc, dtype=np.uint16)
+    n, d = xc.shape
+    codes = np.zeros((n, d), dtype=np.uint8)
+    scales = np.zeros(((n + 63) // 64,), dtype=np.float32)
+    lib().or_fp8_quantize(_p(xc), n, d, _p(codes), _p(scales))
+    return codes, scales
+
+
+def index_scores(qI: np.ndarray, Ic: np.ndarray) -> np.ndarray:
+    """O3: qI [dI] uint16, Ic [n][dI] uint16 -> fp32 scores [n]."""
+    qI = np.ascontiguousarray(qI, dtype=np.uint16)
+    Ic = np.ascontiguousarray(Ic, dtype=np.uint16)
+    n, dI = Ic.shape
+    s = np.zeros((n,), dtype=np.float32)
+    lib().or_index_scores(_p(qI), _p(Ic), n, dI, _p(s))
+    return s
+
+
+def topk(s: np.ndarray, k: int, n_visible: int | None = None):
+    """O4: returns (idx [k] int32 ascending, -1 padded; count)."""
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    nv = s.shape[0] if n_visible is None else n_visible
+    idx = np.zeros((k,), dtype=np.int32)
+    cnt = lib().or_topk(_p(s), nv, k, _p(idx))
+    return idx, int(cnt)
+
+
+def attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, rows, scale: float,
+              k_scales: np.ndarray | None = None, v_scales: np.ndarray | None = None,
+              return_p: bool = False):
+    """O5: q [H][d] uint16; K, V [N][d] uint16 (bf16) or uint8 (e4m3 + scales).
+
+    Returns (out [H][d] f64, lse [H] f64[, p [H][nrows] f64]).
+    """
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    H, d = q.shape
+    fp8 = K.dtype == np.uint8
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+    out = np.zeros((H, d), dtype=np.float64)
+    lse = np.zeros((H,), dtype=np.float64)
+    p = np.zeros((H, max(rows.shape[0], 1)), dtype=np.float64) if return_p else None
+    K = np.ascontiguousarray(K)
+    V = np.ascontiguousarray(V)
+    ks = None if k_scales is None else np.ascontiguousarray(k_scales, dtype=np.float32)
+    vs = None if v_scales is None else np.ascontiguousarray(v_scales, dtype=np.float32)
+    lib().or_attention(_p(q), H, d, _p(K), _p(ks), _p(V), _p(vs), int(fp8), _p(rows), rows.shape[0],
+                       float(scale), _p(out), _p(lse), _p(p))
+    if return_p:
+        return out, lse, p[:, :rows.shape[0]]
+    return out, lse
+
+
+class CompressedSeq:
+    """One sequence's compressed caches as the oracle builds them (O1 + O2)."""
+
+    def __init__(self, K, V, KI, m_csa=4, m_hca=128, fp8=False):
+        self.fp8 = fp8
+        self.m_csa, self.m_hca = m_csa, m_hca
+        ck, cv = compress(K, m_csa), compress(V, m_csa)
+        hk, hv = compress(K, m_hca), compress(V, m_hca)
+        self.cidx = compress(KI, m_csa)
+        self.n_csa, self.n_hca = ck.shape[0], hk.shape[0]
+        self.ck_bf16, self.cv_bf16, self.hk_bf16, self.hv_bf16 = ck, cv, hk, hv
+        if fp8:
+            self.ck, self.cks = fp8_quantize(ck)
+            self.cv, self.cvs = fp8_quantize(cv)
+            self.hk, self.hks = fp8_quantize(hk)
+            self.hv, self.hvs = fp8_quantize(hv)
+        else:
+            self.ck, self.cv, self.hk, self.hv = ck, cv, hk, hv
+            self.cks = self.cvs = self.hks = self.hvs = None
+
+
+def hybrid_query(cs: CompressedSeq, q: np.ndarray, qI: np.ndarray, t: int, k: int, scale: float):
+    """O6 for one query at token position t.  Returns a dict of results."""
+    L = lib()
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    qI = np.ascontiguousarray(qI, dtype=np.uint16)
+    H, d = q.shape
+    dI = qI.shape[0]
+    idx = np.zeros((k,), dtype=np.int32)
+    cnt = np.zeros((1,), dtype=np.int32)
+    oc = np.zeros((H, d)); lc = np.zeros((H,))
+    oh = np.zeros((H, d)); lh = np.zeros((H,))
+
+    def c(a):
+        return None if a is None else np.ascontiguousarray(a)
+    ck, cks, cv, cvs = c(cs.ck), c(cs.cks), c(cs.cv), c(cs.cvs)
+    hk, hks, hv, hvs = c(cs.hk), c(cs.hks), c(cs.hv), c(cs.hvs)
+    cidx = c(cs.cidx)
+    # keep 1-element dummies so that empty caches still pass valid pointers
+    dummy16 = np.zeros((1,), dtype=np.uint16)
+    L.or_hybrid_query(_p(q), _p(qI), H, d, dI, int(t),
+                      cs.m_csa, _p(ck if ck.size else dummy16), _p(cks), _p(cv if cv.size else dummy16), _p(cvs),
+                      _p(cidx if cidx.size else dummy16), cs.n_csa,
+                      cs.m_hca, _p(hk if hk.size else dummy16), _p(hks), _p(hv if hv.size else dummy16), _p(hvs),
+                      cs.n_hca, int(cs.fp8), int(k), float(scale),
+                      _p(idx), _p(cnt), _p(oc), _p(lc), _p(oh), _p(lh))
+    return {"idx": idx, "cnt": int(cnt[0]), "out_csa": oc, "lse_csa": lc, "out_hca": oh, "lse_hca": lh}
