@@ -1,0 +1,421 @@
+#!/usr/bin/env python
+"""Throughput of the CSA + HCA hybrid-attention decode step on B200.
+
+One step = one hybrid_attn_decode call (indexer scores + exact top-k + CSA
+attention over the chosen entries + HCA attention over all entries) for every
+sequence of the batch, caches already compressed and resident in HBM.  The
+default workload is decode at 1M tokens of context: B=4, 64 query heads, one
+shared KV head, head_dim 128, CSA m=4 top-k 2048, HCA m=128, bf16 N(0,1)
+inputs from a fixed seed.  Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the fp64 CPU oracle on the same workload
+
+Under torchrun every rank runs its own batch of independent sequences (weak
+scaling, no collective on the data path); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_attention_pool_b200 import configs, synth  # noqa: E402
+
+DEFAULT_WORKLOAD = "decode_b4_t1m_h64_k2048"
+METRIC = "hybrid-attn decode tokens/s @1M ctx; achieved HBM GB/s (% of peak), 1 B200"
+SCALE = float(np.float32(1.0 / math.sqrt(128.0)))
+L2_FLUSH_BYTES = 512 << 20  # > 126 MB L2, written between timed steps
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "sparse_attention_pool_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """dram bytes per launch from the committed ncu summary, if it still matches the sources."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    r = rec.get(f"{kernel}@{workload}")
+    if not r or r.get("source_hash") != kernel_source_hash():
+        return None
+    return r.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = f"/tmp/sa_clocks_{os.getpid()}.csv"
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if not self.proc or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def decode_bytes(w, lengths):
+    """Algorithmic HBM bytes of one decode step and of its indexer score kernel."""
+    bkv = 1 if w.fp8 else 2
+    step = 0
+    score = 0
+    for L in lengths:
+        nc, nh = int(L) // w.m_csa, int(L) // w.m_hca
+        sel = min(w.topk, nc)
+        step += nc * 128 + sel * 2 * 128 * bkv + nh * 2 * 128 * bkv + w.H * 256 + 128 + 2 * w.H * 256
+        if w.fp8:
+            step += sel * 8 + ((nh + 63) // 64) * 8
+        score += nc * 128 + nc * 4  # read the indexer keys, write one 32-bit key per entry
+    return step, score
+
+
+def make_inputs(w, rank):
+    seed = synth.BASE_SEED + w.index + 7919 * rank
+    B, L = w.B, w.L
+    if w.L_min is not None:
+        lengths = synth.ragged_lengths(seed, B, w.L_min, w.L)
+    else:
+        lengths = np.full((B,), L, dtype=np.int32)
+    K = synth.normal_bf16(seed, "k", (B, L, 128))
+    V = synth.normal_bf16(seed, "v", (B, L, 128))
+    KI = synth.normal_bf16(seed, "kidx", (B, L, 64))
+    q = synth.normal_bf16(seed, "q", (B, w.H, 128))
+    qI = synth.normal_bf16(seed, "qidx", (B, 64))
+    return lengths, K, V, KI, q, qI
+
+
+def to_bf16_tensor(a, dev):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+
+# ---------------------------------------------------------------- our arm ---
+
+def run_ours(args, w, rank, world, dev):
+    import torch
+    import torch.distributed as dist
+
+    import sparse_attention_pool_b200 as S
+    from sparse_attention_pool_b200 import _lib
+
+    lengths, K, V, KI, q_h, qI_h = make_inputs(w, rank)
+    t_gen = time.time()
+    Kd, Vd, KId = to_bf16_tensor(K, dev), to_bf16_tensor(V, dev), to_bf16_tensor(KI, dev)
+    lens = torch.from_numpy(lengths).to(dev)
+    csa = S.alloc_cache(w.B, w.L // w.m_csa, w.m_csa, fp8=w.fp8, with_kidx=True, device=dev)
+    hca = S.alloc_cache(w.B, w.L // w.m_hca, w.m_hca, fp8=w.fp8, device=dev)
+    S.csa_compress(Kd, Vd, KId, lens, csa)
+    S.hca_compress(Kd, Vd, lens, hca)
+    torch.cuda.synchronize()
+    del Kd, Vd, KId
+    torch.cuda.empty_cache()
+    q = to_bf16_tensor(q_h, dev)
+    qI = to_bf16_tensor(qI_h, dev)
+    B, H, k = w.B, w.H, w.topk
+    ws = S.alloc_workspace(S.workspace_size(S.SA_OP_HYBRID_DECODE, B, 1, H, csa.Ncap, hca.Ncap, k), device=dev)
+    out_c = torch.empty(B, H, 128, dtype=torch.bfloat16, device=dev)
+    out_h = torch.empty_like(out_c)
+    lse_c = torch.empty(B, H, dtype=torch.float32, device=dev)
+    lse_h = torch.empty_like(lse_c)
+    idx = torch.empty(B, k, dtype=torch.int32, device=dev)
+    cnt = torch.empty(B, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    L = _lib.lib()
+
+    def step():
+        S.hybrid_attn_decode(q, qI, csa, hca, k, ws, scale=SCALE, out_csa=out_c, out_hca=out_h, lse_csa=lse_c,
+                             lse_hca=lse_h, idx_out=idx, cnt_out=cnt)
+
+    # stage events around the indexer score kernel (captured into the graph)
+    ev_s0 = torch.cuda.Event(enable_timing=True)
+    ev_s1 = torch.cuda.Event(enable_timing=True)
+    L.sa_set_stage_events(_lib.SA_STAGE_INDEX_SCORE, ev_s0.cuda_event, ev_s1.cuda_event)
+    step()  # eager first call: one-time kernel attributes
+    torch.cuda.synchronize()
+    S.read_device_status()
+    n0 = L.sa_launch_count()
+    step()
+    torch.cuda.synchronize()
+    launches_per_step = int(L.sa_launch_count() - n0)
+
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        flush.zero_()
+        graph.replay()
+    torch.cuda.synchronize()
+
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    step_ms, score_ms = [], []
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for i in range(args.steps):
+            flush.zero_()  # untimed: evict the caches from L2
+            ev0[i].record(stream)
+            graph.replay()
+            ev1[i].record(stream)
+            ev1[i].synchronize()
+            step_ms.append(ev0[i].elapsed_time(ev1[i]))
+            score_ms.append(ev_s0.elapsed_time(ev_s1))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    S.read_device_status()
+
+    # end to end through the public API: pinned host q / q_idx in, outputs back out
+    q_pin = torch.from_numpy(np.ascontiguousarray(q_h).view(np.int16)).pin_memory()
+    qi_pin = torch.from_numpy(np.ascontiguousarray(qI_h).view(np.int16)).pin_memory()
+    oc_pin = torch.empty(B, H, 128, dtype=torch.int16).pin_memory()
+    oh_pin = torch.empty_like(oc_pin).pin_memory()
+    lc_pin = torch.empty(B, H, dtype=torch.float32).pin_memory()
+    lh_pin = torch.empty_like(lc_pin).pin_memory()
+    q_dev = torch.empty(B, H, 128, dtype=torch.int16, device=dev)
+    qi_dev = torch.empty(B, 64, dtype=torch.int16, device=dev)
+    h2d = q_pin.numel() * 2 + qi_pin.numel() * 2
+    d2h = oc_pin.numel() * 2 * 2 + lc_pin.numel() * 4 * 2
+    e2e_ms = []
+    L.sa_set_stage_events(_lib.SA_STAGE_INDEX_SCORE, None, None)
+    if world > 1:
+        dist.barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        ev0[i].record(stream)
+        q_dev.copy_(q_pin, non_blocking=True)
+        qi_dev.copy_(qi_pin, non_blocking=True)
+        S.hybrid_attn_decode(q_dev.view(torch.bfloat16), qi_dev.view(torch.bfloat16), csa, hca, k, ws, scale=SCALE,
+                             out_csa=out_c, out_hca=out_h, lse_csa=lse_c, lse_hca=lse_h, idx_out=idx, cnt_out=cnt)
+        oc_pin.copy_(out_c.view(torch.int16), non_blocking=True)
+        oh_pin.copy_(out_h.view(torch.int16), non_blocking=True)
+        lc_pin.copy_(lse_c, non_blocking=True)
+        lh_pin.copy_(lse_h, non_blocking=True)
+        ev1[i].record(stream)
+        ev1[i].synchronize()
+        e2e_ms.append(ev0[i].elapsed_time(ev1[i]))
+    e2e_total = sum(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = float(t.item())
+    S.read_device_status()
+    del graph
+
+    tokens = B * world * args.steps
+    value = tokens / (total_ms / 1e3)
+    step_bytes, score_bytes = decode_bytes(w, lengths)
+    peak, peak_kind = measured_peaks()
+    score_avg = statistics.mean(score_ms)
+    achieved = score_bytes / (score_avg / 1e3) / 1e9
+    step_gbs = step_bytes / (total_ms / args.steps / 1e3) / 1e9
+    result = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if not w.fp8 else "fp8e4m3-kv/bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B_per_gpu": B, "context": int(w.L), "heads": H, "head_dim": 128,
+                   "csa_m": w.m_csa, "topk": k, "hca_m": w.m_hca, "kv_dtype": "e4m3" if w.fp8 else "bf16",
+                   "parallelism": f"replicas x{world} (independent sequences)",
+                   "l2": "flushed between timed steps (512 MB memset)", "launch": "CUDA graph replay"},
+        "hbm": {"step_bytes": step_bytes, "step_gbs": step_gbs, "step_frac": step_gbs / peak,
+                "step_frac_of_8tbs": step_gbs / 8000.0},
+        "roofline": {"kernel": "score_decode_kernel", "bound": "hbm", "achieved": achieved, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                     "bytes_per_launch": score_bytes, "avg_launch_ms": score_avg,
+                     "traffic": recorded_traffic("score_decode_kernel", w.name)},
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": {"value": tokens / (e2e_total / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "api": "hybrid_attn_decode (eager) + pinned-host copies"},
+        "clocks": clk.summary(),
+        "setup_s": round(time.time() - t_gen, 1),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, lengths, K, V, KI, q_h, qI_h, budget_s=args.cpu_budget)
+    return result
+
+
+# ----------------------------------------------------------- oracle (CPU) ---
+
+def oracle_decode_one(w, lengths, K, V, KI, q_h, qI_h, b):
+    """One decode token of sequence b on the fp64 oracle; returns (seconds, setup seconds)."""
+    from oracle import oracle as O
+    t0 = time.time()
+    Lb = int(lengths[b])
+    cs = O.CompressedSeq(K[b, :Lb], V[b, :Lb], KI[b, :Lb], m_csa=w.m_csa, m_hca=w.m_hca, fp8=w.fp8)
+    setup = time.time() - t0
+    t1 = time.perf_counter()
+    O.hybrid_query(cs, q_h[b], qI_h[b], t=Lb, k=w.topk, scale=SCALE)
+    return time.perf_counter() - t1, setup, cs
+
+
+def cpu_baseline(w, lengths, K, V, KI, q_h, qI_h, budget_s=20.0):
+    from oracle import oracle as O
+    el, setup, cs = oracle_decode_one(w, lengths, K, V, KI, q_h, qI_h, 0)
+    times = [el]
+    t_end = time.time() + max(0.0, budget_s - el)
+    while time.time() < t_end and len(times) < 8:
+        t1 = time.perf_counter()
+        O.hybrid_query(cs, q_h[0], qI_h[0], t=int(lengths[0]), k=w.topk, scale=SCALE)
+        times.append(time.perf_counter() - t1)
+    return {"value": len(times) / sum(times), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{len(times)} decode token(s) of sequence 0 ({int(lengths[0])} tokens of context) on the "
+                      f"single-threaded fp64 C oracle, caches pre-built by the oracle ({setup:.1f} s, untimed)"}
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return None
+    lengths, K, V, KI, q_h, qI_h = make_inputs(w, 0)
+    from oracle import oracle as O
+    cs = {}
+    times = []
+    for i in range(args.warmup + args.steps):
+        b = i % w.B
+        if b not in cs:
+            Lb = int(lengths[b])
+            cs[b] = O.CompressedSeq(K[b, :Lb], V[b, :Lb], KI[b, :Lb], m_csa=w.m_csa, m_hca=w.m_hca, fp8=w.fp8)
+        t1 = time.perf_counter()
+        O.hybrid_query(cs[b], q_h[b], qI_h[b], t=int(lengths[b]), k=w.topk, scale=SCALE)
+        el = time.perf_counter() - t1
+        if i >= args.warmup:
+            times.append(el)
+    total = sum(times)
+    value = len(times) / total
+    sample = (f"each step: one decode token of one sequence (sequences 0..{w.B - 1} in turn) on the "
+              f"single-threaded fp64 C oracle; caches built by the oracle, untimed")
+    return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total / len(times) * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "B_per_gpu": w.B, "context": int(w.L), "heads": w.H, "topk": w.topk},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=[x.name for x in configs.WORKLOADS])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = configs.BY_NAME[args.workload]
+    if w.mode != "decode":
+        ap.error("bench.py times decode workloads; prefill is checked by the tests")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, w, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    try:
+        res = run_ours(args, w, rank, world, dev)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

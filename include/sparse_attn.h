@@ -1,0 +1,212 @@
+/*
+ * sparse_attn.h -- C ABI of libsparse_attn.so: CSA + HCA hybrid attention on
+ * one NVIDIA B200 (sm_100a).
+ *
+ * The method is the hybrid attention of "DeepSeek-V4: Towards Highly Efficient
+ * Million-Token Context Intelligence Review" (dimensionstp.github.io),
+ * section 3-2 (2) "Hybrid attention with CSA and HCA":
+ *   - CSA (compressed sparse attention) pools every 4 tokens of K/V into one
+ *     compressed entry, scores every entry with an indexer, keeps the top-k
+ *     entries and attends over them only;
+ *   - HCA (heavily compressed attention) pools every 128 tokens into one entry
+ *     and attends densely over all entries;
+ *   - the layers interleave the two, so one "hybrid" step returns both outputs;
+ *   - compressed KV may be stored in FP8 (the "Mixed KV storage" row).
+ * Where the page leaves the arithmetic open, this library implements:
+ *   pooling  = fp64 sum of each aligned, complete block of m tokens in
+ *              ascending token order, times 1/m, rounded once to bf16 (RNE);
+ *              an incomplete tail block is not compressed;
+ *   fp8      = e4m3 codes, one fp32 scale per 64 consecutive entries,
+ *              scale = fp32(amax / 448) (1 when amax == 0),
+ *              code = e4m3_rne_satfinite(fp32(x / scale));
+ *   score    = fp32( fp64 sum over i = 0..63, ascending, of q_idx[i]*kidx[j][i] ),
+ *              -0 -> +0; one 64-dim indexer query per token, shared by heads;
+ *   top-k    = the k entries with the largest (score, -index); indices are
+ *              returned in ascending order, padded with -1;
+ *   attention= per head softmax(scale * q . K^T) V over the chosen entries,
+ *              fp32 accumulation, bf16 output (RNE), fp32 natural-log lse;
+ *              scale = 1/sqrt(128) when 0 is passed; an empty set gives a
+ *              zero output and lse = -inf;
+ *   causality= a query at token position t sees entry c iff (c + 1) * m <= t;
+ *              in decode the query follows the cached tokens, t = length.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; each must
+ *     be 16-byte aligned.  bf16 tensors are raw IEEE bfloat16, e4m3 tensors
+ *     are raw OCP FP8 E4M3 ("fn") bytes.  Layouts are dense, row-major, in
+ *     the order written next to each argument.
+ *   - The library never allocates, frees or synchronises device memory; all
+ *     work is queued on `stream` (a cudaStream_t passed as void*, NULL = the
+ *     legacy default stream) and returns before it runs.
+ *   - Argument errors are detected on the host before anything is launched
+ *     and return a non-zero sa_status; sa_last_error() then gives the reason.
+ *   - Errors that only the device can see (a length above its capacity, a
+ *     bounded wait that ran out) never trap: kernels record them in a
+ *     per-device status word and carry on with clamped values.
+ *     sa_read_device_status() reports and clears it.
+ *   - head_dim d must be 128 and the indexer dim d_idx 64.  H is 1..128.
+ *   - Results are deterministic run to run and do not depend on the batch a
+ *     sequence is in (the split of every reduction is fixed per sequence).
+ */
+#ifndef SPARSE_ATTN_H
+#define SPARSE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SA_ABI_VERSION 1
+
+typedef enum {
+    SA_OK = 0,
+    SA_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, bad size or shape      */
+    SA_ERR_UNSUPPORTED = 2,  /* a valid request this build does not implement      */
+    SA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than sa_workspace_size */
+    SA_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch, memset, ...)   */
+    SA_ERR_TIMEOUT = 5,      /* device status: a bounded wait ran out              */
+    SA_ERR_DEVICE = 6        /* device status: a length exceeded its capacity, ... */
+} sa_status;
+
+typedef enum { SA_BF16 = 0, SA_FP8_E4M3 = 1 } sa_kv_dtype;
+
+/* Raw (uncompressed) tokens of B sequences, padded to Lcap tokens each. */
+typedef struct {
+    const void* k;         /* [B][Lcap][d] bf16                                   */
+    const void* v;         /* [B][Lcap][d] bf16                                   */
+    const void* kidx;      /* [B][Lcap][d_idx] bf16 indexer keys (CSA), or NULL   */
+    const int32_t* len;    /* device [B]: tokens of each sequence, 0..Lcap        */
+    int32_t B, Lcap, d, d_idx;
+} sa_raw;
+
+/* A compressed cache (CSA: m = 4 with indexer keys; HCA: m = 128 without). */
+typedef struct {
+    void* k;               /* [B][Ncap][d] bf16, or e4m3 codes                     */
+    void* v;               /* [B][Ncap][d] bf16, or e4m3 codes                     */
+    float* k_scale;        /* [B][ceil(Ncap/64)] fp32 when dtype == SA_FP8_E4M3     */
+    float* v_scale;        /* same for v; both NULL for bf16                        */
+    void* kidx;            /* [B][Ncap][d_idx] bf16 (needed by the CSA indexer)     */
+    int32_t* n;            /* device [B]: complete entries per sequence             */
+    int32_t B, Ncap, d, d_idx;
+    int32_t m;             /* tokens per entry: a power of two, 1..1024            */
+    int32_t dtype;         /* sa_kv_dtype                                           */
+} sa_cache;
+
+/* Operation codes for sa_workspace_size. */
+typedef enum {
+    SA_OP_INDEX_TOPK = 1,
+    SA_OP_SPARSE_ATTN = 2,
+    SA_OP_DENSE_ATTN = 3,
+    SA_OP_HYBRID_DECODE = 4,
+    SA_OP_HYBRID_PREFILL = 5
+} sa_op;
+
+/* Compression, section 3-2 (2) component table, CSA row ("every 4 tokens ->
+ * 1 compressed entry").  Pools raw k, v and kidx of every sequence into
+ * `out` (out->m tokens per entry, normally 4) and writes out->n[b] =
+ * floor(len[b] / m).  Needs out->kidx != NULL and raw->kidx != NULL.
+ * Entries at or beyond n[b] are left untouched.  fp8 caches also get their
+ * per-64-entry scales.  Requires out->Ncap >= Lcap / m.                       */
+sa_status csa_compress(const sa_raw* raw, const sa_cache* out, void* stream);
+
+/* Compression, HCA row ("every 128 tokens -> 1 compressed entry"): as
+ * csa_compress for k and v only (kidx ignored); out->m is normally 128.      */
+sa_status hca_compress(const sa_raw* raw, const sa_cache* out, void* stream);
+
+/* CSA indexer + top-k, section 3-2 (2) (CSA "sparse top-k selection") and
+ * 3-2 (4) ("CSA indexer QK path").
+ *   q_idx [B][Tq][d_idx] bf16: indexer queries.
+ *   q_pos [B][Tq] int32 device token positions, or NULL for decode (Tq must
+ *         then be 1 and every complete entry is visible).
+ *   idx   [B][Tq][k] int32 out: chosen entries, ascending, -1 padded.
+ *   cnt   [B][Tq] int32 out: min(k, visible entries).
+ * ws / ws_bytes: scratch of at least sa_workspace_size(SA_OP_INDEX_TOPK, ...).
+ * k: 1..65536.                                                               */
+sa_status csa_index_topk(const void* q_idx, int32_t Tq, const int32_t* q_pos,
+                         const sa_cache* csa, int32_t k, int32_t* idx, int32_t* cnt,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* CSA attention over the chosen entries, section 3-2 (2) (CSA attends over
+ * the selected entries only).
+ *   q   [B][Tq][H][d] bf16; idx / cnt as produced by csa_index_topk (an index
+ *       outside 0..n[b]-1 is skipped and flagged in the device status).
+ *   out [B][Tq][H][d] bf16; lse [B][Tq][H] fp32 or NULL.                     */
+sa_status csa_sparse_attn(const void* q, int32_t Tq, int32_t H, const sa_cache* csa,
+                          const int32_t* idx, const int32_t* cnt, int32_t k, float scale,
+                          void* out, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* HCA dense attention over every visible entry, section 3-2 (2) (HCA keeps
+ * dense attention, no selection).  q_pos as in csa_index_topk (NULL = decode,
+ * all n[b] entries visible).  Shapes as csa_sparse_attn.                     */
+sa_status hca_dense_attn(const void* q, int32_t Tq, int32_t H, const int32_t* q_pos,
+                         const sa_cache* hca, float scale, void* out, float* lse,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* One decode step of both branches for B sequences (one new query each):
+ * indexer + top-k + CSA attention, and HCA attention.
+ *   q [B][H][d] bf16, q_idx [B][d_idx] bf16.
+ *   out_csa, out_hca [B][H][d] bf16; lse_csa, lse_hca [B][H] fp32 or NULL.
+ *   idx_out [B][k] / cnt_out [B] int32, or NULL to keep them in the workspace. */
+sa_status hybrid_attn_decode(const void* q, const void* q_idx, int32_t H,
+                             const sa_cache* csa, const sa_cache* hca, int32_t k, float scale,
+                             void* out_csa, void* out_hca, float* lse_csa, float* lse_hca,
+                             int32_t* idx_out, int32_t* cnt_out,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* Causal prefill of both branches: T queries per sequence at token positions
+ * 0..T-1 over caches compressed from those same tokens.
+ *   q [B][T][H][d] bf16, q_idx [B][T][d_idx] bf16.
+ *   out_csa, out_hca [B][T][H][d] bf16; lse_* [B][T][H] fp32 or NULL.
+ *   idx_out [B][T][k] and cnt_out [B][T] int32 are required.                  */
+sa_status hybrid_attn_prefill(const void* q, const void* q_idx, int32_t T, int32_t H,
+                              const sa_cache* csa, const sa_cache* hca, int32_t k, float scale,
+                              void* out_csa, void* out_hca, float* lse_csa, float* lse_hca,
+                              int32_t* idx_out, int32_t* cnt_out,
+                              void* ws, size_t ws_bytes, void* stream);
+
+/* Bytes of scratch an operation needs (0 on invalid sizes).  Ncap_csa /
+ * Ncap_hca are the capacities of the two caches (pass 0 for one that the
+ * operation does not use).  The scratch must be device memory, 256-byte
+ * aligned, zeroed once before its first use; calls sharing one scratch
+ * buffer must be ordered on one stream.                                      */
+size_t sa_workspace_size(int32_t op, int32_t B, int32_t Tq, int32_t H,
+                         int32_t Ncap_csa, int32_t Ncap_hca, int32_t k);
+
+/* Synchronises `stream`, reads the device status word that every kernel of
+ * the library records its device-side anomalies in (one word per device,
+ * shared by all callers in the process), clears it, and returns SA_OK,
+ * SA_ERR_TIMEOUT or SA_ERR_DEVICE.                                           */
+sa_status sa_read_device_status(void* stream);
+
+/* Text for the last non-OK status returned on the calling host thread.      */
+const char* sa_last_error(void);
+
+/* SA_ABI_VERSION of the loaded library.                                      */
+int32_t sa_abi_version(void);
+
+/* Stages of a decode step, for sa_set_stage_events.                          */
+typedef enum {
+    SA_STAGE_INDEX_SCORE = 0,  /* indexer score kernel (streams the indexer keys) */
+    SA_STAGE_TOPK_SELECT = 1,  /* threshold search + ordered selection kernels    */
+    SA_STAGE_CSA_ATTN = 2,     /* CSA attention (+ its split merge)                */
+    SA_STAGE_HCA_ATTN = 3,     /* HCA attention (+ its split merge)                */
+    SA_NUM_STAGES = 4
+} sa_stage;
+
+/* Tracing hook: while set, every decode-path call made on the calling host
+ * thread records `before` and `after` (cudaEvent_t passed as void*) on its
+ * stream immediately around the kernels of `stage`.  NULL, NULL switches the
+ * stage off.  The events are the caller's; the library only records them.   */
+sa_status sa_set_stage_events(int32_t stage, void* before, void* after);
+
+/* Number of kernels this library has launched from the calling host thread
+ * since the process started (a diagnostic counter; memsets are not kernels). */
+uint64_t sa_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSE_ATTN_H */

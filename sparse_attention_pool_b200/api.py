@@ -1,0 +1,186 @@
+"""Thin Python binding of libsparse_attn.so.
+
+Every function here only marshals torch tensors (device memory owned by the
+caller) into the C ABI of include/sparse_attn.h and raises on a non-OK
+status; every step of the computation runs in the library's CUDA kernels.
+Function names follow the C entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+from ._lib import SaCache, SaRaw, check, lib
+
+D, D_IDX = 128, 64
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, dtype, name):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise TypeError(f"{name}: must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    return t
+
+
+@dataclass
+class Cache:
+    """A compressed KV cache (caller-owned device tensors) and its descriptor."""
+    k: torch.Tensor
+    v: torch.Tensor
+    n: torch.Tensor
+    m: int
+    kidx: torch.Tensor | None = None
+    k_scale: torch.Tensor | None = None
+    v_scale: torch.Tensor | None = None
+
+    @property
+    def B(self):
+        return self.k.shape[0]
+
+    @property
+    def Ncap(self):
+        return self.k.shape[1]
+
+    @property
+    def fp8(self):
+        return self.k.dtype == torch.uint8
+
+    def struct(self) -> SaCache:
+        return SaCache(_ptr(self.k), _ptr(self.v), _ptr(self.k_scale), _ptr(self.v_scale), _ptr(self.kidx),
+                       _ptr(self.n), self.B, self.Ncap, D, D_IDX, self.m,
+                       _lib.SA_FP8_E4M3 if self.fp8 else _lib.SA_BF16)
+
+
+def alloc_cache(B: int, Ncap: int, m: int, *, fp8: bool = False, with_kidx: bool = False,
+                device="cuda") -> Cache:
+    kv_dtype = torch.uint8 if fp8 else torch.bfloat16
+    nG = (Ncap + 63) // 64
+    return Cache(
+        k=torch.zeros(B, Ncap, D, dtype=kv_dtype, device=device),
+        v=torch.zeros(B, Ncap, D, dtype=kv_dtype, device=device),
+        n=torch.zeros(B, dtype=torch.int32, device=device),
+        m=m,
+        kidx=torch.zeros(B, Ncap, D_IDX, dtype=torch.bfloat16, device=device) if with_kidx else None,
+        k_scale=torch.zeros(B, max(nG, 1), dtype=torch.float32, device=device) if fp8 else None,
+        v_scale=torch.zeros(B, max(nG, 1), dtype=torch.float32, device=device) if fp8 else None,
+    )
+
+
+def _raw(k, v, kidx, lengths):
+    _need(k, torch.bfloat16, "k")
+    _need(v, torch.bfloat16, "v")
+    _need(lengths, torch.int32, "lengths")
+    if kidx is not None:
+        _need(kidx, torch.bfloat16, "kidx")
+    B, Lcap = k.shape[0], k.shape[1]
+    return SaRaw(_ptr(k), _ptr(v), _ptr(kidx), _ptr(lengths), B, Lcap, D, D_IDX)
+
+
+def csa_compress(k, v, kidx, lengths, cache: Cache, stream=None):
+    raw = _raw(k, v, kidx, lengths)
+    cs = cache.struct()
+    check("csa_compress", lib().csa_compress(ctypes.byref(raw), ctypes.byref(cs), _stream(stream)))
+
+
+def hca_compress(k, v, lengths, cache: Cache, stream=None):
+    raw = _raw(k, v, None, lengths)
+    cs = cache.struct()
+    check("hca_compress", lib().hca_compress(ctypes.byref(raw), ctypes.byref(cs), _stream(stream)))
+
+
+def workspace_size(op: int, B: int, Tq: int, H: int, Ncap_csa: int, Ncap_hca: int, k: int) -> int:
+    return int(lib().sa_workspace_size(op, B, Tq, H, Ncap_csa, Ncap_hca, k))
+
+
+def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """Zeroed scratch; torch's allocator returns 512-byte aligned blocks."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def csa_index_topk(q_idx, csa: Cache, k: int, ws, *, q_pos=None, idx=None, cnt=None, stream=None):
+    _need(q_idx, torch.bfloat16, "q_idx")
+    B = csa.B
+    Tq = 1 if q_pos is None else q_idx.shape[1]
+    if idx is None:
+        idx = torch.empty(B, Tq, k, dtype=torch.int32, device=q_idx.device)
+    if cnt is None:
+        cnt = torch.empty(B, Tq, dtype=torch.int32, device=q_idx.device)
+    cs = csa.struct()
+    check("csa_index_topk", lib().csa_index_topk(_ptr(q_idx), Tq, _ptr(q_pos), ctypes.byref(cs), k, _ptr(idx),
+                                                 _ptr(cnt), _ptr(ws), ws.numel(), _stream(stream)))
+    return idx, cnt
+
+
+def csa_sparse_attn(q, csa: Cache, idx, cnt, k: int, ws, *, scale=0.0, out=None, lse=None, stream=None):
+    _need(q, torch.bfloat16, "q")
+    B, Tq, H = q.shape[0], (q.shape[1] if q.dim() == 4 else 1), q.shape[-2]
+    if out is None:
+        out = torch.empty_like(q)
+    cs = csa.struct()
+    check("csa_sparse_attn", lib().csa_sparse_attn(_ptr(q), Tq, H, ctypes.byref(cs), _ptr(idx), _ptr(cnt), k,
+                                                   float(scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                                   _stream(stream)))
+    return out
+
+
+def hca_dense_attn(q, hca: Cache, ws, *, q_pos=None, scale=0.0, out=None, lse=None, stream=None):
+    _need(q, torch.bfloat16, "q")
+    Tq, H = (q.shape[1] if q.dim() == 4 else 1), q.shape[-2]
+    if out is None:
+        out = torch.empty_like(q)
+    cs = hca.struct()
+    check("hca_dense_attn", lib().hca_dense_attn(_ptr(q), Tq, H, _ptr(q_pos), ctypes.byref(cs), float(scale),
+                                                 _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def hybrid_attn_decode(q, q_idx, csa: Cache, hca: Cache, k: int, ws, *, scale=0.0, out_csa=None, out_hca=None,
+                       lse_csa=None, lse_hca=None, idx_out=None, cnt_out=None, stream=None):
+    """q [B][H][128] bf16, q_idx [B][64] bf16 -> (out_csa, out_hca) [B][H][128] bf16."""
+    _need(q, torch.bfloat16, "q")
+    _need(q_idx, torch.bfloat16, "q_idx")
+    H = q.shape[1]
+    out_csa = torch.empty_like(q) if out_csa is None else out_csa
+    out_hca = torch.empty_like(q) if out_hca is None else out_hca
+    c, h = csa.struct(), hca.struct()
+    check("hybrid_attn_decode",
+          lib().hybrid_attn_decode(_ptr(q), _ptr(q_idx), H, ctypes.byref(c), ctypes.byref(h), k, float(scale),
+                                   _ptr(out_csa), _ptr(out_hca), _ptr(lse_csa), _ptr(lse_hca), _ptr(idx_out),
+                                   _ptr(cnt_out), _ptr(ws), ws.numel(), _stream(stream)))
+    return out_csa, out_hca
+
+
+def hybrid_attn_prefill(q, q_idx, csa: Cache, hca: Cache, k: int, ws, idx_out, cnt_out, *, scale=0.0,
+                        out_csa=None, out_hca=None, lse_csa=None, lse_hca=None, stream=None):
+    """q [B][T][H][128] bf16, q_idx [B][T][64] bf16; idx_out [B][T][k], cnt_out [B][T] int32."""
+    _need(q, torch.bfloat16, "q")
+    _need(q_idx, torch.bfloat16, "q_idx")
+    T, H = q.shape[1], q.shape[2]
+    out_csa = torch.empty_like(q) if out_csa is None else out_csa
+    out_hca = torch.empty_like(q) if out_hca is None else out_hca
+    c, h = csa.struct(), hca.struct()
+    check("hybrid_attn_prefill",
+          lib().hybrid_attn_prefill(_ptr(q), _ptr(q_idx), T, H, ctypes.byref(c), ctypes.byref(h), k, float(scale),
+                                    _ptr(out_csa), _ptr(out_hca), _ptr(lse_csa), _ptr(lse_hca), _ptr(idx_out),
+                                    _ptr(cnt_out), _ptr(ws), ws.numel(), _stream(stream)))
+    return out_csa, out_hca
+
+
+def read_device_status(stream=None):
+    """Synchronises the stream and raises if a kernel recorded a device-side anomaly."""
+    check("sa_read_device_status", lib().sa_read_device_status(_stream(stream)))

@@ -1,0 +1,389 @@
+// attn.cuh -- softmax attention of H query heads (one shared KV head) over a
+// list of compressed entries: the CSA branch over the top-k entries
+// (gathered rows) and the HCA branch over every visible entry (contiguous
+// rows), "DeepSeek-V4 ... Review", section 3-2 (2) component table.
+//
+// out_h = sum_j softmax_j(scale * q_h . K_j) V_j,  lse_h = log sum_j exp(.)
+//
+// One CTA handles one query (all H heads: M = 16 rows per warp) and one split
+// of its entry list, 64 entries per tile, double-buffered with cp.async into
+// XOR-swizzled shared memory.  QK^T and PV run on bf16 tensor-core MMAs with
+// fp32 accumulation (flash-decoding: online softmax in registers, P re-used
+// from the S accumulators).  An fp8 cache is widened to bf16 in shared memory
+// (every e4m3 value is exact in bf16); its per-64-entry scales multiply the S
+// columns (K) and the P columns (V) in fp32.  With one split the CTA writes
+// the bf16 output directly; otherwise it writes a normalised fp32 partial and
+// its lse, merged by attn_combine_kernel in a fixed order (deterministic and
+// independent of the batch: the split size depends only on the entry count).
+#pragma once
+#include "sa_common.cuh"
+
+namespace sa {
+
+constexpr int kTileN = 64;  // entries per tile
+
+struct AttnArgs {
+    const uint16_t* q;   // [BQ][H][128], BQ = B * Tq
+    const void* K;       // [B][Ncap][128] bf16 or e4m3
+    const void* V;
+    const float* ks;     // [B][nG] (fp8)
+    const float* vs;
+    const int32_t* n;    // [B]
+    const int32_t* idx;  // gather: [BQ][kmax]
+    const int32_t* cnt;  // gather: [BQ]
+    const int32_t* pos;  // dense: [BQ] token positions, or NULL (all n[b] visible)
+    int Tq, H, Ncap, nG, kmax, m;
+    float scale_log2;    // softmax scale * log2(e)
+    int tiles_per_split, splits;
+    float* part_o;       // [BQ][splits][H][128]
+    float* part_lse;     // [BQ][splits][H]
+    uint16_t* out;       // [BQ][H][128]
+    float* lse;          // [BQ][H] or NULL
+};
+
+__device__ __forceinline__ uint32_t swz(int r, int chunk) {  // byte offset in a [rows][128] bf16 tile
+    return (uint32_t)(r * 256 + ((chunk ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <int NW, bool GATHER, bool FP8>
+struct AttnSmem {
+    static constexpr int kQBytes = NW * 16 * 256;
+    static constexpr int kKVBytes = kTileN * 256;                 // one bf16 tile
+    static constexpr int kStageRaw = FP8 ? kTileN * 128 : kKVBytes;  // one raw tile (K or V)
+    static constexpr int kQ = 0;
+    static constexpr int kRaw = kQ + kQBytes;                      // [2 stages][K, V] raw tiles
+    static constexpr int kConv = kRaw + 2 * 2 * kStageRaw;         // fp8: widened K, V tiles
+    static constexpr int kMeta = kConv + (FP8 ? 2 * kKVBytes : 0);  // [2][64] valid + (fp8) scales
+    static constexpr int kTotal = kMeta + 2 * kTileN * 4 * 3;
+};
+
+template <int NW, bool GATHER, bool FP8>
+__global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
+    using L = AttnSmem<NW, GATHER, FP8>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int split = blockIdx.x, bq = blockIdx.y;
+    const int b = bq / a.Tq;
+    int nb = a.n[b];
+    if (nb < 0 || nb > a.Ncap) {
+        if (tid == 0 && split == 0) flag(DEV_LEN);
+        nb = nb < 0 ? 0 : a.Ncap;
+    }
+    // number of list positions for this query
+    int R;
+    if (GATHER) {
+        R = a.cnt[bq];
+        if (R < 0 || R > a.kmax) {
+            if (tid == 0 && split == 0) flag(DEV_LEN);
+            R = R < 0 ? 0 : a.kmax;
+        }
+    } else {
+        R = nb;
+        if (a.pos) {
+            const int t = a.pos[bq];
+            if (t < 0) {
+                if (tid == 0 && split == 0) flag(DEV_POS);
+                R = 0;
+            } else {
+                R = min(R, t / a.m);
+            }
+        }
+    }
+    const int p_begin = split * a.tiles_per_split * kTileN;
+    const int p_end = min(R, p_begin + a.tiles_per_split * kTileN);
+    const int ntiles = p_end > p_begin ? (p_end - p_begin + kTileN - 1) / kTileN : 0;
+
+    uint8_t* sQ = smem + L::kQ;
+    uint8_t* sRaw = smem + L::kRaw;
+    uint8_t* sConv = smem + L::kConv;
+    int* sValid = reinterpret_cast<int*>(smem + L::kMeta);           // [2][64]
+    float* sKs = reinterpret_cast<float*>(sValid + 2 * kTileN);       // [2][64]
+    float* sVs = sKs + 2 * kTileN;                                    // [2][64]
+
+    const uint16_t* qp = a.q + (size_t)bq * a.H * 128;
+    // Q tile: rows >= H are zero
+    for (int c = tid; c < NW * 16 * 16; c += NW * 32) {
+        const int r = c >> 4, ch = c & 15;
+        cp_async16_zfill(sQ + swz(r, ch), qp + (size_t)min(r, a.H - 1) * 128 + ch * 8, r < a.H);
+    }
+    cp_async_commit();
+
+    const uint8_t* Kb = reinterpret_cast<const uint8_t*>(a.K);
+    const uint8_t* Vb = reinterpret_cast<const uint8_t*>(a.V);
+    const int rowBytes = FP8 ? 128 : 256;
+    const size_t seqBase = (size_t)b * a.Ncap * rowBytes;
+
+    auto load_tile = [&](int tile, int stage) {
+        const int p0 = p_begin + tile * kTileN;
+        uint8_t* rk = sRaw + (stage * 2 + 0) * L::kStageRaw;
+        uint8_t* rv = sRaw + (stage * 2 + 1) * L::kStageRaw;
+        constexpr int cpr = FP8 ? 8 : 16;  // 16-byte chunks per row
+        for (int c = tid; c < kTileN * cpr; c += NW * 32) {
+            const int r = c / cpr, ch = c % cpr;
+            const int p = p0 + r;
+            int j = p;
+            bool ok = p < p_end;
+            if (GATHER && ok) {
+                j = a.idx[(size_t)bq * a.kmax + p];
+                if (j < 0 || j >= nb) {
+                    ok = false;
+                    if (ch == 0) flag(DEV_INDEX);
+                }
+            }
+            const size_t off = seqBase + (size_t)(ok ? j : 0) * rowBytes + ch * 16;
+            const uint32_t doff = FP8 ? (uint32_t)(r * 128 + ch * 16) : swz(r, ch);
+            cp_async16_zfill(rk + doff, Kb + off, ok);
+            cp_async16_zfill(rv + doff, Vb + off, ok);
+            if (ch == 0) {
+                sValid[stage * kTileN + r] = ok;
+                if (FP8) {
+                    const int g = ok ? j / 64 : 0;
+                    sKs[stage * kTileN + r] = ok ? a.ks[(size_t)b * a.nG + g] : 0.f;
+                    sVs[stage * kTileN + r] = ok ? a.vs[(size_t)b * a.nG + g] : 0.f;
+                }
+            }
+        }
+    };
+
+    if (ntiles > 0) load_tile(0, 0);
+    cp_async_commit();
+
+    // per-thread state: rows r0 = lane/4 and r1 = lane/4 + 8 of this warp's 16 heads
+    float o[16][4];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
+    uint32_t qf[8][4];
+
+    cp_async_wait<1>();  // Q landed
+    __syncthreads();
+    {
+        const uint32_t qbase = smem_u32(sQ);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            const int r = warp * 16 + (lane & 15);
+            const int ch = kk * 2 + (lane >> 4);
+            ldsm_x4(qbase + swz(r, ch), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
+        }
+    }
+
+    for (int t = 0; t < ntiles; ++t) {
+        const int stage = t & 1;
+        if (t + 1 < ntiles) load_tile(t + 1, stage ^ 1);
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();
+
+        const uint8_t* tk;
+        const uint8_t* tv;
+        if (FP8) {
+            // widen e4m3 codes to bf16 (exact), into swizzled tiles
+            const uint8_t* rk = sRaw + (stage * 2 + 0) * L::kStageRaw;
+            const uint8_t* rv = sRaw + (stage * 2 + 1) * L::kStageRaw;
+            uint8_t* ck = sConv;
+            uint8_t* cv = sConv + L::kKVBytes;
+            for (int c = tid; c < kTileN * 16; c += NW * 32) {  // 8 codes -> one 16-byte bf16 chunk
+                const int r = c >> 4, ch = c & 15;
+                const uint2 wk = *reinterpret_cast<const uint2*>(rk + r * 128 + ch * 8);
+                const uint2 wv = *reinterpret_cast<const uint2*>(rv + r * 128 + ch * 8);
+                uint4 ok4, ov4;
+                uint32_t* okp = &ok4.x;
+                uint32_t* ovp = &ov4.x;
+                const uint32_t kw[2] = {wk.x, wk.y}, vw[2] = {wv.x, wv.y};
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        okp[h * 2 + e] = pack_bf16x2(e4m3_to_f32((kw[h] >> (16 * e)) & 0xFF),
+                                                     e4m3_to_f32((kw[h] >> (16 * e + 8)) & 0xFF));
+                        ovp[h * 2 + e] = pack_bf16x2(e4m3_to_f32((vw[h] >> (16 * e)) & 0xFF),
+                                                     e4m3_to_f32((vw[h] >> (16 * e + 8)) & 0xFF));
+                    }
+                *reinterpret_cast<uint4*>(ck + swz(r, ch)) = ok4;
+                *reinterpret_cast<uint4*>(cv + swz(r, ch)) = ov4;
+            }
+            __syncthreads();
+            tk = ck;
+            tv = cv;
+        } else {
+            tk = sRaw + (stage * 2 + 0) * L::kStageRaw;
+            tv = sRaw + (stage * 2 + 1) * L::kStageRaw;
+        }
+
+        // S = Q K^T : 16 rows x 64 entries per warp
+        float s[8][4];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+        const uint32_t kbase = smem_u32(tk);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {  // pairs of 8-entry n-tiles
+                const int r = np * 16 + (lane & 7) + ((lane >> 4) << 3);
+                const int ch = kk * 2 + ((lane >> 3) & 1);
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(kbase + swz(r, ch), b0, b1, b2, b3);
+                mma16816(s[2 * np], qf[kk], b0, b1);
+                mma16816(s[2 * np + 1], qf[kk], b2, b3);
+            }
+        }
+        // scales, masking, online softmax (log2 domain)
+        const int* valid = sValid + stage * kTileN;
+        float tmax[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int col = j * 8 + (lane & 3) * 2 + (e & 1);
+                float v = s[j][e];
+                if (FP8) v *= sKs[stage * kTileN + col];
+                v = valid[col] ? v * a.scale_log2 : -INFINITY;
+                s[j][e] = v;
+                tmax[e >> 1] = fmaxf(tmax[e >> 1], v);
+            }
+        float alpha[2], mnew[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            tmax[h] = fmaxf(tmax[h], __shfl_xor_sync(0xFFFFFFFFu, tmax[h], 1));
+            tmax[h] = fmaxf(tmax[h], __shfl_xor_sync(0xFFFFFFFFu, tmax[h], 2));
+            mnew[h] = fmaxf(mrow[h], tmax[h]);
+            alpha[h] = (mnew[h] == -INFINITY) ? 1.f : exp2f(mrow[h] - mnew[h]);
+            mrow[h] = mnew[h];
+        }
+        float lsum[2] = {0.f, 0.f};
+        uint32_t pf[4][4];  // P as bf16 A fragments, 4 k-steps of 16 entries
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float p[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float mm = mnew[e >> 1];
+                p[e] = (mm == -INFINITY) ? 0.f : exp2f(s[j][e] - mm);
+                lsum[e >> 1] += p[e];
+                if (FP8) p[e] *= sVs[stage * kTileN + j * 8 + (lane & 3) * 2 + (e & 1)];
+            }
+            pf[j >> 1][(j & 1) * 2 + 0] = pack_bf16x2(p[0], p[1]);
+            pf[j >> 1][(j & 1) * 2 + 1] = pack_bf16x2(p[2], p[3]);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) lrow[h] = lrow[h] * alpha[h] + lsum[h];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            o[i][0] *= alpha[0];
+            o[i][1] *= alpha[0];
+            o[i][2] *= alpha[1];
+            o[i][3] *= alpha[1];
+        }
+        // O += P V
+        const uint32_t vbase = smem_u32(tv);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            // pf[kk] = {a0, a1, a2, a3} in mma order: rows r0/r1 x entries 16kk + {0..7, 8..15}
+            const uint32_t af[4] = {pf[kk][0], pf[kk][1], pf[kk][2], pf[kk][3]};
+#pragma unroll
+            for (int dp = 0; dp < 8; ++dp) {  // pairs of 8-dim n-tiles
+                const int r = kk * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+                const int ch = dp * 2 + (lane >> 4);
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(vbase + swz(r, ch), b0, b1, b2, b3);
+                mma16816(o[2 * dp], af, b0, b1);
+                mma16816(o[2 * dp + 1], af, b2, b3);
+            }
+        }
+        __syncthreads();  // this stage's buffers are reloaded next iteration
+    }
+    cp_async_wait<0>();
+
+    // finish: row sums across the 4 lanes of a row
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        lrow[h] += __shfl_xor_sync(0xFFFFFFFFu, lrow[h], 1);
+        lrow[h] += __shfl_xor_sync(0xFFFFFFFFu, lrow[h], 2);
+    }
+    const float kLn2 = 0.6931471805599453f;
+    float inv[2], lse_r[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const bool empty = !(lrow[h] > 0.f);
+        inv[h] = empty ? 0.f : 1.f / lrow[h];
+        lse_r[h] = empty ? -INFINITY : (mrow[h] + __log2f(lrow[h])) * kLn2;
+    }
+    const int hr[2] = {warp * 16 + (lane >> 2), warp * 16 + (lane >> 2) + 8};
+    if (a.splits == 1) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            if (hr[h] >= a.H) continue;
+            uint16_t* op = a.out + ((size_t)bq * a.H + hr[h]) * 128;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int d = i * 8 + (lane & 3) * 2;
+                *reinterpret_cast<uint32_t*>(op + d) = pack_bf16x2(o[i][2 * h] * inv[h], o[i][2 * h + 1] * inv[h]);
+            }
+            if (a.lse && (lane & 3) == 0) a.lse[(size_t)bq * a.H + hr[h]] = lse_r[h];
+        }
+    } else {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            if (hr[h] >= a.H) continue;
+            float* op = a.part_o + (((size_t)bq * a.splits + split) * a.H + hr[h]) * 128;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int d = i * 8 + (lane & 3) * 2;
+                *reinterpret_cast<float2*>(op + d) = make_float2(o[i][2 * h] * inv[h], o[i][2 * h + 1] * inv[h]);
+            }
+            if ((lane & 3) == 0) a.part_lse[((size_t)bq * a.splits + split) * a.H + hr[h]] = lse_r[h];
+        }
+    }
+}
+
+// Merge the split partials of every (query, head) in split order.
+__global__ void __launch_bounds__(256) attn_combine_kernel(const float* part_o, const float* part_lse, int splits,
+                                                           int H, uint16_t* out, float* lse) {
+    const int bq = blockIdx.y;
+    const int h = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (h >= H) return;
+    const float* pl = part_lse + (size_t)bq * splits * H + h;
+    float M = -INFINITY;
+    for (int s = 0; s < splits; ++s) M = fmaxf(M, pl[(size_t)s * H]);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float wsum = 0.f;
+    if (M != -INFINITY) {
+        for (int s = 0; s < splits; ++s) {
+            const float ls = pl[(size_t)s * H];
+            if (ls == -INFINITY) continue;
+            const float w = __expf(ls - M);
+            const float4 v = *reinterpret_cast<const float4*>(part_o + (((size_t)bq * splits + s) * H + h) * 128 +
+                                                              lane * 4);
+            acc.x += w * v.x;
+            acc.y += w * v.y;
+            acc.z += w * v.z;
+            acc.w += w * v.w;
+            wsum += w;
+        }
+    }
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    uint16_t* op = out + ((size_t)bq * H + h) * 128 + lane * 4;
+    *reinterpret_cast<uint2*>(op) = make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
+    if (lse && lane == 0) lse[(size_t)bq * H + h] = wsum > 0.f ? M + __logf(wsum) : -INFINITY;
+}
+
+}  // namespace sa

@@ -1,0 +1,632 @@
+// sparse_attn.cu -- the C ABI of libsparse_attn.so (declared in
+// include/sparse_attn.h): argument checks, workspace layout and the launch
+// sequence of every operation.  All device code lives in the *.cuh files
+// included below, compiled as one translation unit for sm_100a.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/sparse_attn.h"
+#include "attn.cuh"
+#include "compress.cuh"
+#include "sa_common.cuh"
+#include "topk_decode.cuh"
+#include "topk_prefill.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+thread_local uint64_t g_launches = 0;
+thread_local cudaEvent_t g_stage_ev[SA_NUM_STAGES][2] = {};
+
+inline void stage_mark(int stage, int which, cudaStream_t st) {
+    if (g_stage_ev[stage][which]) cudaEventRecord(g_stage_ev[stage][which], st);
+}
+
+sa_status fail(sa_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+#define SA_CHECK(cond, ...)                                  \
+    do {                                                     \
+        if (!(cond)) return fail(SA_ERR_INVALID_ARG, __VA_ARGS__); \
+    } while (0)
+
+#define SA_LAUNCHED()                                                                          \
+    do {                                                                                       \
+        cudaError_t e_ = cudaGetLastError();                                                   \
+        if (e_ != cudaSuccess) return fail(SA_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e_)); \
+        ++g_launches;                                                                          \
+    } while (0)
+
+#define SA_CUDA(call)                                                                              \
+    do {                                                                                           \
+        cudaError_t e_ = (call);                                                                   \
+        if (e_ != cudaSuccess) return fail(SA_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+    } while (0)
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+int num_sms() {
+    static int sms[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return 148;
+    if (!sms[dev]) {
+        int v = 0;
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        sms[dev] = v > 0 ? v : 148;
+    }
+    return sms[dev];
+}
+
+sa_status check_cache(const sa_cache* c, bool need_kidx, const char* what) {
+    SA_CHECK(c != nullptr, "%s: cache descriptor is NULL", what);
+    SA_CHECK(c->B >= 1 && c->B <= 65535, "%s: B=%d outside 1..65535", what, c->B);
+    SA_CHECK(c->Ncap >= 0 && c->Ncap <= (1 << 24), "%s: Ncap=%d outside 0..2^24", what, c->Ncap);
+    SA_CHECK(c->d == 128, "%s: head dim d=%d (only 128 is supported)", what, c->d);
+    SA_CHECK(c->m >= 1 && c->m <= 1024 && (c->m & (c->m - 1)) == 0, "%s: m=%d is not a power of two in 1..1024",
+             what, c->m);
+    SA_CHECK(c->dtype == SA_BF16 || c->dtype == SA_FP8_E4M3, "%s: dtype=%d", what, c->dtype);
+    SA_CHECK(c->k && c->v && c->n, "%s: k, v and n must be non-NULL", what);
+    SA_CHECK(aligned16(c->k) && aligned16(c->v) && aligned16(c->n), "%s: k, v, n must be 16-byte aligned", what);
+    if (c->dtype == SA_FP8_E4M3) {
+        SA_CHECK(c->k_scale && c->v_scale, "%s: fp8 cache needs k_scale and v_scale", what);
+        SA_CHECK(aligned16(c->k_scale) && aligned16(c->v_scale), "%s: scales must be 16-byte aligned", what);
+    }
+    if (need_kidx) {
+        SA_CHECK(c->kidx != nullptr, "%s: CSA cache needs indexer keys (kidx)", what);
+        SA_CHECK(c->d_idx == 64, "%s: indexer dim d_idx=%d (only 64 is supported)", what, c->d_idx);
+        SA_CHECK(aligned16(c->kidx), "%s: kidx must be 16-byte aligned", what);
+    }
+    return SA_OK;
+}
+
+inline int ilog2(int v) {
+    int r = 0;
+    while ((1 << r) < v) ++r;
+    return r;
+}
+
+// --------------------------------------------------------------- TMA map --
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// Indexer keys [B][Ncap][64] bf16 as a 3-D tensor map, box 64 x kScRows x 1, 128B swizzle.
+sa_status make_ic_map(CUtensorMap* map, const void* kidx, int B, int Ncap) {
+    auto enc = get_encode();
+    if (!enc) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    cuuint64_t dims[3] = {64, (cuuint64_t)Ncap, (cuuint64_t)B};
+    cuuint64_t strides[2] = {128, (cuuint64_t)Ncap * 128};
+    cuuint32_t box[3] = {64, (cuuint32_t)sa::kScRows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(kidx), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return SA_OK;
+}
+
+// ------------------------------------------------------- workspace layout --
+struct TopkDecodeWs {
+    size_t zero_off, zero_bytes, keys, cand_key, cand_idx, bitmap, idx, cnt, total;
+    int Wcap;
+};
+
+TopkDecodeWs topk_decode_layout(int B, int Ncap, int k, bool own_idx) {
+    TopkDecodeWs w{};
+    w.Wcap = ((Ncap + 31) / 32 + 1) & ~1;
+    size_t o = 256;  // bytes 0..255 are reserved
+    w.zero_off = o;
+    w.zero_bytes = up256((size_t)B * sa::kBins * 4 * 2 + (size_t)B * 4);
+    o += w.zero_bytes;
+    w.keys = o;
+    o += up256((size_t)B * Ncap * 4);
+    w.cand_key = o;
+    o += up256((size_t)B * Ncap * 4);
+    w.cand_idx = o;
+    o += up256((size_t)B * Ncap * 4);
+    w.bitmap = o;
+    o += up256((size_t)B * w.Wcap * 4);
+    w.idx = o;
+    if (own_idx) o += up256((size_t)B * k * 4);
+    w.cnt = o;
+    if (own_idx) o += up256((size_t)B * 4);
+    w.total = o;
+    return w;
+}
+
+// Split rule of the attention kernels: depends only on the list capacity, never
+// on the batch, so a sequence's result does not depend on its batch-mates.
+struct Split {
+    int tps, splits;
+};
+Split attn_split(int rows_cap, bool prefill) {
+    const int tiles = cdiv(rows_cap > 0 ? rows_cap : 1, sa::kTileN);
+    if (prefill) return {tiles, 1};
+    const int tps = cdiv(tiles, 32);
+    return {tps, cdiv(tiles, tps)};
+}
+
+size_t attn_partial_bytes(long long BQ, int splits, int H) {
+    if (splits <= 1) return 0;
+    return up256((size_t)BQ * splits * H * 128 * 4) + up256((size_t)BQ * splits * H * 4);
+}
+
+// ------------------------------------------------------------ launchers ----
+template <int NW, bool G, bool F>
+sa_status launch_attn_t(const sa::AttnArgs& a, dim3 grid, cudaStream_t st) {
+    using L = sa::AttnSmem<NW, G, F>;
+    static bool init = false;
+    if (!init) {
+        SA_CUDA(cudaFuncSetAttribute(sa::attn_split_kernel<NW, G, F>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     L::kTotal));
+        init = true;
+    }
+    sa::attn_split_kernel<NW, G, F><<<grid, NW * 32, L::kTotal, st>>>(a);
+    SA_LAUNCHED();
+    return SA_OK;
+}
+
+sa_status launch_attn(const sa::AttnArgs& a, bool gather, bool fp8, long long BQ, cudaStream_t st) {
+    dim3 grid(a.splits, (unsigned)BQ);
+    if (BQ > 2147483647LL) return fail(SA_ERR_INVALID_ARG, "too many queries");
+    const bool big = a.H > 64;
+    if (!big) {
+        if (gather) return fp8 ? launch_attn_t<4, true, true>(a, grid, st) : launch_attn_t<4, true, false>(a, grid, st);
+        return fp8 ? launch_attn_t<4, false, true>(a, grid, st) : launch_attn_t<4, false, false>(a, grid, st);
+    }
+    if (gather) return fp8 ? launch_attn_t<8, true, true>(a, grid, st) : launch_attn_t<8, true, false>(a, grid, st);
+    return fp8 ? launch_attn_t<8, false, true>(a, grid, st) : launch_attn_t<8, false, false>(a, grid, st);
+}
+
+sa_status launch_combine(const float* po, const float* pl, int splits, int H, long long BQ, uint16_t* out, float* lse,
+                         cudaStream_t st) {
+    dim3 grid(cdiv(H, 8), (unsigned)BQ);
+    sa::attn_combine_kernel<<<grid, 256, 0, st>>>(po, pl, splits, H, out, lse);
+    SA_LAUNCHED();
+    return SA_OK;
+}
+
+// Shared body of csa_sparse_attn / hca_dense_attn / the hybrid calls.
+sa_status run_attn(const void* q, int Tq, int H, const sa_cache* c, bool gather, const int32_t* idx,
+                   const int32_t* cnt, int kmax, const int32_t* pos, float scale, void* out, float* lse, void* ws,
+                   size_t ws_off, cudaStream_t st) {
+    const long long BQ = (long long)c->B * Tq;
+    const bool prefill = (Tq > 1) || (pos != nullptr);
+    const Split sp = attn_split(gather ? kmax : c->Ncap, prefill);
+    sa::AttnArgs a{};
+    a.q = static_cast<const uint16_t*>(q);
+    a.K = c->k;
+    a.V = c->v;
+    a.ks = c->k_scale;
+    a.vs = c->v_scale;
+    a.n = c->n;
+    a.idx = idx;
+    a.cnt = cnt;
+    a.pos = pos;
+    a.Tq = Tq;
+    a.H = H;
+    a.Ncap = c->Ncap;
+    a.nG = (c->Ncap + 63) / 64;
+    a.kmax = kmax;
+    a.m = c->m;
+    const float s = scale == 0.f ? 1.0f / sqrtf(128.0f) : scale;
+    a.scale_log2 = s * 1.4426950408889634f;
+    a.tiles_per_split = sp.tps;
+    a.splits = sp.splits;
+    a.out = static_cast<uint16_t*>(out);
+    a.lse = lse;
+    if (sp.splits > 1) {
+        uint8_t* base = static_cast<uint8_t*>(ws) + ws_off;
+        a.part_o = reinterpret_cast<float*>(base);
+        a.part_lse = reinterpret_cast<float*>(base + up256((size_t)BQ * sp.splits * H * 128 * 4));
+    }
+    sa_status r = launch_attn(a, gather, c->dtype == SA_FP8_E4M3, BQ, st);
+    if (r != SA_OK) return r;
+    if (sp.splits > 1) return launch_combine(a.part_o, a.part_lse, sp.splits, H, BQ, a.out, lse, st);
+    return SA_OK;
+}
+
+sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* idx, int32_t* cnt, void* ws,
+                          const TopkDecodeWs& w, cudaStream_t st) {
+    const int B = c->B, Ncap = c->Ncap;
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    sa::TopkDecodeArgs a{};
+    a.q_idx = static_cast<const uint16_t*>(q_idx);
+    a.n = c->n;
+    a.keys = reinterpret_cast<uint32_t*>(base + w.keys);
+    a.hist1 = reinterpret_cast<uint32_t*>(base + w.zero_off);
+    a.hist2 = a.hist1 + (size_t)B * sa::kBins;
+    a.cand_cnt = a.hist2 + (size_t)B * sa::kBins;
+    a.cand_key = reinterpret_cast<uint32_t*>(base + w.cand_key);
+    a.cand_idx = reinterpret_cast<int32_t*>(base + w.cand_idx);
+    a.bitmap = reinterpret_cast<uint32_t*>(base + w.bitmap);
+    a.idx = idx;
+    a.cnt = cnt;
+    a.Ncap = Ncap;
+    a.Wcap = w.Wcap;
+    a.k = k;
+    // rows per CTA: about three CTAs per SM over the whole batch, whole tiles
+    const long long target = (long long)num_sms() * 3;
+    long long chunk = ((long long)B * Ncap + target - 1) / target;
+    chunk = ((chunk + sa::kScRows - 1) / sa::kScRows) * sa::kScRows;
+    if (chunk < sa::kScRows) chunk = sa::kScRows;
+    a.chunk = (int)chunk;
+    const int nchunks = Ncap > 0 ? cdiv(Ncap, chunk) : 1;
+
+    SA_CUDA(cudaMemsetAsync(base + w.zero_off, 0, w.zero_bytes, st));
+    if (Ncap > 0) {
+        CUtensorMap map;
+        sa_status r = make_ic_map(&map, c->kidx, B, Ncap);
+        if (r != SA_OK) return r;
+        const size_t smem = sa::kScStages * sa::kScTileBytes + sa::kBins * 4 + sa::kScStages * 8 + 1024;
+        static bool init = false;
+        if (!init) {
+            SA_CUDA(cudaFuncSetAttribute(sa::score_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem));
+            init = true;
+        }
+        stage_mark(SA_STAGE_INDEX_SCORE, 0, st);
+        sa::score_decode_kernel<<<dim3(nchunks, B), sa::kScThreads, smem, st>>>(map, a);
+        SA_LAUNCHED();
+        stage_mark(SA_STAGE_INDEX_SCORE, 1, st);
+        stage_mark(SA_STAGE_TOPK_SELECT, 0, st);
+        sa::topk_filter_kernel<<<dim3(nchunks, B), sa::kFiltThreads, 0, st>>>(a);
+        SA_LAUNCHED();
+    }
+    else stage_mark(SA_STAGE_TOPK_SELECT, 0, st);
+    sa::topk_resolve_kernel<<<B, sa::kResThreads, 0, st>>>(a);
+    SA_LAUNCHED();
+    stage_mark(SA_STAGE_TOPK_SELECT, 1, st);
+    return SA_OK;
+}
+
+sa_status check_ws(void* ws, size_t have, size_t need) {
+    if (need == 0) return SA_OK;
+    if (!ws) return fail(SA_ERR_WORKSPACE, "workspace is NULL but %zu bytes are needed", need);
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(SA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+    if (have < need) return fail(SA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", have, need);
+    return SA_OK;
+}
+
+// ---------------------------------------------------------------- prefill --
+constexpr int kPrefillQB = 1024;  // queries per score block
+
+inline int keys_stride(int Ncap) { return std::max(1, cdiv(Ncap, sa::kPsE)) * sa::kPsE; }
+
+size_t prefill_pos_off() { return 256; }
+size_t prefill_keys_off(int B, int T) { return 256 + up256((size_t)B * T * 4); }
+
+size_t prefill_topk_bytes(int B, int T, int Ncap, int k) {
+    (void)k;
+    const int qb = std::min(T, kPrefillQB);
+    return prefill_keys_off(B, T) + up256((size_t)qb * keys_stride(Ncap) * 4);
+}
+
+const int32_t* prefill_positions(void* ws, int B, int T, cudaStream_t st) {
+    int32_t* pos = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + prefill_pos_off());
+    const long long total = (long long)B * T;
+    sa::fill_positions_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(pos, B, T);
+    if (cudaGetLastError() != cudaSuccess) return nullptr;
+    ++g_launches;
+    return pos;
+}
+
+sa_status run_topk_prefill(const void* q_idx, int Tq, const int32_t* pos, const sa_cache* c, int k, int32_t* idx,
+                           int32_t* cnt, void* ws, cudaStream_t st) {
+    sa::TopkPrefillArgs a{};
+    a.q_idx = static_cast<const uint16_t*>(q_idx);
+    a.kidx = static_cast<const uint16_t*>(c->kidx);
+    a.pos = pos;
+    a.n = c->n;
+    a.keys = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + prefill_keys_off(c->B, Tq));
+    a.idx = idx;
+    a.cnt = cnt;
+    a.Tq = Tq;
+    a.Ncap = c->Ncap;
+    a.KS = keys_stride(c->Ncap);
+    a.k = k;
+    a.log2m = ilog2(c->m);
+    static bool init = false;
+    if (!init) {
+        SA_CUDA(cudaFuncSetAttribute(sa::score_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     sa::kPsSmem));
+        SA_CUDA(cudaFuncSetAttribute(sa::select_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     sa::kSelSmemKeys * 4));
+        init = true;
+    }
+    const int etiles = std::max(1, cdiv(c->Ncap, sa::kPsE));
+    for (int b = 0; b < c->B; ++b) {
+        for (int t0 = 0; t0 < Tq; t0 += kPrefillQB) {
+            a.b = b;
+            a.t0 = t0;
+            a.qb = std::min(kPrefillQB, Tq - t0);
+            if (c->Ncap > 0) {
+                sa::score_prefill_kernel<<<dim3(etiles, cdiv(a.qb, sa::kPsQ)), sa::kPsThreads, sa::kPsSmem, st>>>(a);
+                SA_LAUNCHED();
+            }
+            sa::select_prefill_kernel<<<a.qb, sa::kSelThreads, sa::kSelSmemKeys * 4, st>>>(a);
+            SA_LAUNCHED();
+        }
+    }
+    return SA_OK;
+}
+
+}  // namespace
+
+// =========================================================== public ABI ====
+extern "C" {
+
+int32_t sa_abi_version(void) { return SA_ABI_VERSION; }
+
+uint64_t sa_launch_count(void) { return g_launches; }
+
+sa_status sa_set_stage_events(int32_t stage, void* before, void* after) {
+    SA_CHECK(stage >= 0 && stage < SA_NUM_STAGES, "sa_set_stage_events: stage=%d", stage);
+    SA_CHECK((before == nullptr) == (after == nullptr), "sa_set_stage_events: give both events or neither");
+    g_stage_ev[stage][0] = static_cast<cudaEvent_t>(before);
+    g_stage_ev[stage][1] = static_cast<cudaEvent_t>(after);
+    return SA_OK;
+}
+
+const char* sa_last_error(void) { return g_err; }
+
+static sa_status compress_common(const sa_raw* raw, const sa_cache* out, void* stream, bool csa) {
+    const char* what = csa ? "csa_compress" : "hca_compress";
+    SA_CHECK(raw != nullptr, "%s: raw descriptor is NULL", what);
+    sa_status r = check_cache(out, csa, what);
+    if (r != SA_OK) return r;
+    SA_CHECK(raw->B == out->B, "%s: raw B=%d but cache B=%d", what, raw->B, out->B);
+    SA_CHECK(raw->d == 128, "%s: raw d=%d (only 128)", what, raw->d);
+    SA_CHECK(raw->Lcap >= 0, "%s: Lcap=%d", what, raw->Lcap);
+    SA_CHECK(raw->k && raw->v && raw->len, "%s: raw k, v, len must be non-NULL", what);
+    SA_CHECK(aligned16(raw->k) && aligned16(raw->v) && aligned16(raw->len), "%s: raw pointers must be 16-byte aligned",
+             what);
+    SA_CHECK((long long)out->Ncap >= (long long)raw->Lcap / out->m, "%s: Ncap=%d < Lcap/m=%d", what, out->Ncap,
+             raw->Lcap / out->m);
+    if (csa) {
+        SA_CHECK(raw->kidx != nullptr && aligned16(raw->kidx), "%s: raw kidx must be non-NULL and aligned", what);
+        SA_CHECK(raw->d_idx == 64, "%s: raw d_idx=%d (only 64)", what, raw->d_idx);
+    }
+    sa::CompressArgs a{};
+    a.src[0] = static_cast<const uint16_t*>(raw->k);
+    a.src[1] = static_cast<const uint16_t*>(raw->v);
+    a.src[2] = csa ? static_cast<const uint16_t*>(raw->kidx) : nullptr;
+    a.dst[0] = out->k;
+    a.dst[1] = out->v;
+    a.dst[2] = csa ? out->kidx : nullptr;
+    a.scale[0] = out->k_scale;
+    a.scale[1] = out->v_scale;
+    a.dims[0] = 128;
+    a.dims[1] = 128;
+    a.dims[2] = 64;
+    a.ntensors = csa ? 3 : 2;
+    a.len = raw->len;
+    a.n_out = out->n;
+    a.Lcap = raw->Lcap;
+    a.Ncap = out->Ncap;
+    a.nG = (out->Ncap + 63) / 64;
+    a.m = out->m;
+    a.log2m = ilog2(out->m);
+    a.fp8 = out->dtype == SA_FP8_E4M3;
+    const int groups = std::max(1, cdiv(raw->Lcap / out->m, 64));
+    sa::compress_kernel<<<dim3(groups, raw->B), sa::kCompThreads, 0, static_cast<cudaStream_t>(stream)>>>(a);
+    SA_LAUNCHED();
+    return SA_OK;
+}
+
+sa_status csa_compress(const sa_raw* raw, const sa_cache* out, void* stream) {
+    return compress_common(raw, out, stream, true);
+}
+
+sa_status hca_compress(const sa_raw* raw, const sa_cache* out, void* stream) {
+    return compress_common(raw, out, stream, false);
+}
+
+size_t sa_workspace_size(int32_t op, int32_t B, int32_t Tq, int32_t H, int32_t Ncap_csa, int32_t Ncap_hca,
+                         int32_t k) {
+    if (B < 1 || Tq < 1 || H < 1 || H > 128 || Ncap_csa < 0 || Ncap_hca < 0 || k < 0) return 0;
+    const long long BQ = (long long)B * Tq;
+    const bool prefill = Tq > 1;
+    switch (op) {
+        case SA_OP_INDEX_TOPK:
+            if (k < 1) return 0;
+            if (prefill) return prefill_topk_bytes(B, Tq, Ncap_csa, k);
+            return topk_decode_layout(B, Ncap_csa, k, false).total;
+        case SA_OP_SPARSE_ATTN: {
+            if (k < 1) return 0;
+            Split s = attn_split(k, prefill);
+            return 256 + attn_partial_bytes(BQ, s.splits, H);
+        }
+        case SA_OP_DENSE_ATTN: {
+            Split s = attn_split(Ncap_hca, prefill);
+            return 256 + attn_partial_bytes(BQ, s.splits, H);
+        }
+        case SA_OP_HYBRID_DECODE: {
+            if (k < 1 || Tq != 1) return 0;
+            TopkDecodeWs w = topk_decode_layout(B, Ncap_csa, k, true);
+            Split sc = attn_split(k, false), sh = attn_split(Ncap_hca, false);
+            return w.total + attn_partial_bytes(BQ, sc.splits, H) + attn_partial_bytes(BQ, sh.splits, H);
+        }
+        case SA_OP_HYBRID_PREFILL:
+            if (k < 1) return 0;
+            return prefill_topk_bytes(B, Tq, Ncap_csa, k);
+        default:
+            return 0;
+    }
+}
+
+sa_status sa_read_device_status(void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    SA_CUDA(cudaStreamSynchronize(st));
+    uint32_t v = 0, zero = 0;
+    SA_CUDA(cudaMemcpyFromSymbol(&v, sa::g_status, sizeof(v)));
+    SA_CUDA(cudaMemcpyToSymbol(sa::g_status, &zero, sizeof(zero)));
+    if (v & sa::DEV_TIMEOUT) return fail(SA_ERR_TIMEOUT, "device status 0x%x: a bounded wait ran out", v);
+    if (v) return fail(SA_ERR_DEVICE, "device status 0x%x (2: length/count out of range, 4: bad index, 8: bad position)", v);
+    return SA_OK;
+}
+
+static sa_status check_common_q(const void* q, int H, const char* what) {
+    SA_CHECK(q != nullptr && aligned16(q), "%s: q must be non-NULL and 16-byte aligned", what);
+    SA_CHECK(H >= 1 && H <= 128, "%s: H=%d outside 1..128", what, H);
+    return SA_OK;
+}
+
+sa_status csa_index_topk(const void* q_idx, int32_t Tq, const int32_t* q_pos, const sa_cache* csa, int32_t k,
+                         int32_t* idx, int32_t* cnt, void* ws, size_t ws_bytes, void* stream) {
+    sa_status r = check_cache(csa, true, "csa_index_topk");
+    if (r != SA_OK) return r;
+    SA_CHECK(q_idx && aligned16(q_idx), "csa_index_topk: q_idx must be non-NULL and 16-byte aligned");
+    SA_CHECK(idx && cnt && aligned16(idx) && aligned16(cnt), "csa_index_topk: idx/cnt must be non-NULL and aligned");
+    SA_CHECK(k >= 1 && k <= 65536, "csa_index_topk: k=%d outside 1..65536", k);
+    SA_CHECK(Tq >= 1, "csa_index_topk: Tq=%d", Tq);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (q_pos == nullptr) {
+        SA_CHECK(Tq == 1, "csa_index_topk: decode (q_pos == NULL) needs Tq == 1, got %d", Tq);
+        TopkDecodeWs w = topk_decode_layout(csa->B, csa->Ncap, k, false);
+        r = check_ws(ws, ws_bytes, w.total);
+        if (r != SA_OK) return r;
+        return run_topk_decode(q_idx, csa, k, idx, cnt, ws, w, st);
+    }
+    SA_CHECK(aligned16(q_pos), "csa_index_topk: q_pos must be 16-byte aligned");
+    r = check_ws(ws, ws_bytes, prefill_topk_bytes(csa->B, Tq, csa->Ncap, k));
+    if (r != SA_OK) return r;
+    return run_topk_prefill(q_idx, Tq, q_pos, csa, k, idx, cnt, ws, st);
+}
+
+sa_status csa_sparse_attn(const void* q, int32_t Tq, int32_t H, const sa_cache* csa, const int32_t* idx,
+                          const int32_t* cnt, int32_t k, float scale, void* out, float* lse, void* ws,
+                          size_t ws_bytes, void* stream) {
+    sa_status r = check_cache(csa, false, "csa_sparse_attn");
+    if (r != SA_OK) return r;
+    r = check_common_q(q, H, "csa_sparse_attn");
+    if (r != SA_OK) return r;
+    SA_CHECK(Tq >= 1, "csa_sparse_attn: Tq=%d", Tq);
+    SA_CHECK(k >= 1 && k <= 65536, "csa_sparse_attn: k=%d outside 1..65536", k);
+    SA_CHECK(idx && cnt && aligned16(idx) && aligned16(cnt), "csa_sparse_attn: idx/cnt must be non-NULL and aligned");
+    SA_CHECK(out && aligned16(out), "csa_sparse_attn: out must be non-NULL and 16-byte aligned");
+    SA_CHECK(!lse || aligned16(lse), "csa_sparse_attn: lse must be 16-byte aligned");
+    SA_CHECK(std::isfinite(scale) && scale >= 0.f, "csa_sparse_attn: scale must be finite and >= 0");
+    r = check_ws(ws, ws_bytes, sa_workspace_size(SA_OP_SPARSE_ATTN, csa->B, Tq, H, csa->Ncap, 0, k));
+    if (r != SA_OK) return r;
+    return run_attn(q, Tq, H, csa, true, idx, cnt, k, nullptr, scale, out, lse, ws, 256,
+                    static_cast<cudaStream_t>(stream));
+}
+
+sa_status hca_dense_attn(const void* q, int32_t Tq, int32_t H, const int32_t* q_pos, const sa_cache* hca, float scale,
+                         void* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+    sa_status r = check_cache(hca, false, "hca_dense_attn");
+    if (r != SA_OK) return r;
+    r = check_common_q(q, H, "hca_dense_attn");
+    if (r != SA_OK) return r;
+    SA_CHECK(Tq >= 1, "hca_dense_attn: Tq=%d", Tq);
+    SA_CHECK(q_pos != nullptr || Tq == 1, "hca_dense_attn: decode (q_pos == NULL) needs Tq == 1");
+    SA_CHECK(!q_pos || aligned16(q_pos), "hca_dense_attn: q_pos must be 16-byte aligned");
+    SA_CHECK(out && aligned16(out), "hca_dense_attn: out must be non-NULL and 16-byte aligned");
+    SA_CHECK(!lse || aligned16(lse), "hca_dense_attn: lse must be 16-byte aligned");
+    SA_CHECK(std::isfinite(scale) && scale >= 0.f, "hca_dense_attn: scale must be finite and >= 0");
+    const bool prefill = (Tq > 1) || q_pos;
+    const Split sp = attn_split(hca->Ncap, prefill);
+    r = check_ws(ws, ws_bytes, 256 + attn_partial_bytes((long long)hca->B * Tq, sp.splits, H));
+    if (r != SA_OK) return r;
+    return run_attn(q, Tq, H, hca, false, nullptr, nullptr, 0, q_pos, scale, out, lse, ws, 256,
+                    static_cast<cudaStream_t>(stream));
+}
+
+sa_status hybrid_attn_decode(const void* q, const void* q_idx, int32_t H, const sa_cache* csa, const sa_cache* hca,
+                             int32_t k, float scale, void* out_csa, void* out_hca, float* lse_csa, float* lse_hca,
+                             int32_t* idx_out, int32_t* cnt_out, void* ws, size_t ws_bytes, void* stream) {
+    sa_status r = check_cache(csa, true, "hybrid_attn_decode(csa)");
+    if (r != SA_OK) return r;
+    r = check_cache(hca, false, "hybrid_attn_decode(hca)");
+    if (r != SA_OK) return r;
+    r = check_common_q(q, H, "hybrid_attn_decode");
+    if (r != SA_OK) return r;
+    SA_CHECK(csa->B == hca->B, "hybrid_attn_decode: csa B=%d != hca B=%d", csa->B, hca->B);
+    SA_CHECK(q_idx && aligned16(q_idx), "hybrid_attn_decode: q_idx must be non-NULL and aligned");
+    SA_CHECK(k >= 1 && k <= 65536, "hybrid_attn_decode: k=%d outside 1..65536", k);
+    SA_CHECK(out_csa && out_hca && aligned16(out_csa) && aligned16(out_hca), "hybrid_attn_decode: outputs must be aligned");
+    SA_CHECK((!lse_csa || aligned16(lse_csa)) && (!lse_hca || aligned16(lse_hca)), "hybrid_attn_decode: lse alignment");
+    SA_CHECK((idx_out == nullptr) == (cnt_out == nullptr), "hybrid_attn_decode: give both idx_out and cnt_out or neither");
+    SA_CHECK((!idx_out || aligned16(idx_out)) && (!cnt_out || aligned16(cnt_out)), "hybrid_attn_decode: idx/cnt alignment");
+    SA_CHECK(std::isfinite(scale) && scale >= 0.f, "hybrid_attn_decode: scale must be finite and >= 0");
+    const size_t need = sa_workspace_size(SA_OP_HYBRID_DECODE, csa->B, 1, H, csa->Ncap, hca->Ncap, k);
+    r = check_ws(ws, ws_bytes, need);
+    if (r != SA_OK) return r;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    TopkDecodeWs w = topk_decode_layout(csa->B, csa->Ncap, k, true);
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + w.idx);
+    int32_t* cnt = cnt_out ? cnt_out : reinterpret_cast<int32_t*>(base + w.cnt);
+    r = run_topk_decode(q_idx, csa, k, idx, cnt, ws, w, st);
+    if (r != SA_OK) return r;
+    const Split sc = attn_split(k, false);
+    stage_mark(SA_STAGE_CSA_ATTN, 0, st);
+    r = run_attn(q, 1, H, csa, true, idx, cnt, k, nullptr, scale, out_csa, lse_csa, ws, w.total, st);
+    if (r != SA_OK) return r;
+    stage_mark(SA_STAGE_CSA_ATTN, 1, st);
+    stage_mark(SA_STAGE_HCA_ATTN, 0, st);
+    r = run_attn(q, 1, H, hca, false, nullptr, nullptr, 0, nullptr, scale, out_hca, lse_hca, ws,
+                 w.total + attn_partial_bytes(csa->B, sc.splits, H), st);
+    if (r != SA_OK) return r;
+    stage_mark(SA_STAGE_HCA_ATTN, 1, st);
+    return SA_OK;
+}
+
+sa_status hybrid_attn_prefill(const void* q, const void* q_idx, int32_t T, int32_t H, const sa_cache* csa,
+                              const sa_cache* hca, int32_t k, float scale, void* out_csa, void* out_hca,
+                              float* lse_csa, float* lse_hca, int32_t* idx_out, int32_t* cnt_out, void* ws,
+                              size_t ws_bytes, void* stream) {
+    sa_status r = check_cache(csa, true, "hybrid_attn_prefill(csa)");
+    if (r != SA_OK) return r;
+    r = check_cache(hca, false, "hybrid_attn_prefill(hca)");
+    if (r != SA_OK) return r;
+    r = check_common_q(q, H, "hybrid_attn_prefill");
+    if (r != SA_OK) return r;
+    SA_CHECK(csa->B == hca->B, "hybrid_attn_prefill: csa B=%d != hca B=%d", csa->B, hca->B);
+    SA_CHECK(T >= 1, "hybrid_attn_prefill: T=%d", T);
+    SA_CHECK(q_idx && aligned16(q_idx), "hybrid_attn_prefill: q_idx must be non-NULL and aligned");
+    SA_CHECK(k >= 1 && k <= 65536, "hybrid_attn_prefill: k=%d outside 1..65536", k);
+    SA_CHECK(out_csa && out_hca && aligned16(out_csa) && aligned16(out_hca), "hybrid_attn_prefill: outputs must be aligned");
+    SA_CHECK((!lse_csa || aligned16(lse_csa)) && (!lse_hca || aligned16(lse_hca)), "hybrid_attn_prefill: lse alignment");
+    SA_CHECK(idx_out && cnt_out && aligned16(idx_out) && aligned16(cnt_out),
+             "hybrid_attn_prefill: idx_out and cnt_out are required and must be aligned");
+    SA_CHECK(std::isfinite(scale) && scale >= 0.f, "hybrid_attn_prefill: scale must be finite and >= 0");
+    r = check_ws(ws, ws_bytes, sa_workspace_size(SA_OP_HYBRID_PREFILL, csa->B, T, H, csa->Ncap, hca->Ncap, k));
+    if (r != SA_OK) return r;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // positions 0..T-1 for every sequence live in the workspace
+    const int32_t* pos = prefill_positions(ws, csa->B, T, st);
+    if (!pos) return fail(SA_ERR_CUDA, "could not write query positions");
+    r = run_topk_prefill(q_idx, T, pos, csa, k, idx_out, cnt_out, ws, st);
+    if (r != SA_OK) return r;
+    r = run_attn(q, T, H, csa, true, idx_out, cnt_out, k, pos, scale, out_csa, lse_csa, ws, 0, st);
+    if (r != SA_OK) return r;
+    return run_attn(q, T, H, hca, false, nullptr, nullptr, 0, pos, scale, out_hca, lse_hca, ws, 0, st);
+}
+
+}  // extern "C"

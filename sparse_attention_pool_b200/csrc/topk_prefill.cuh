@@ -1,0 +1,254 @@
+// topk_prefill.cuh -- CSA indexer scores and exact top-k for many queries at
+// once (causal prefill), "DeepSeek-V4 ... Review", section 3-2 (2) and 3-2 (4).
+//
+// Query q at token position t sees entries c with (c + 1) * m <= t.  Scores
+// are the same exact quantity as in decode (fp64 FMA chain in ascending i,
+// rounded once to fp32).  Two kernels per block of queries:
+//   1. score_prefill_kernel -- a register-tiled fp64 "GEMM": each CTA scores 64
+//      queries x 128 entries.  The queries are staged as fp64 (q * 2^768), the
+//      keys as packed bf16 pairs that each thread widens exactly (scaled-bf16
+//      bit placement) right before use; every thread owns 4 x 8 independent
+//      FMA chains.  Keys land in a [QB][KS] scratch block.
+//   2. select_prefill_kernel -- one CTA per query: loads the query's visible
+//      keys into shared memory, radix-selects the k-th largest (11/11/10-bit
+//      digits), keeps ties at the threshold by lowest index, and writes the
+//      chosen indices in ascending order with an ordered block compaction.
+#pragma once
+#include "sa_common.cuh"
+#include "topk_decode.cuh"
+
+namespace sa {
+
+constexpr int kPsQ = 64;         // queries per score tile
+constexpr int kPsE = 128;        // entries per score tile
+constexpr int kPsThreads = 256;  // 16 x 16 threads, 4 queries x 8 entries each
+constexpr int kPsSmem = 64 * kPsQ * 8 + 32 * kPsE * 4;  // fp64 queries + packed key pairs
+constexpr int kSelThreads = 1024;
+constexpr int kSelSmemKeys = 48 * 1024;  // keys held in shared memory (192 KB)
+
+struct TopkPrefillArgs {
+    const uint16_t* q_idx;  // [B][Tq][64]
+    const uint16_t* kidx;   // [B][Ncap][64]
+    const int32_t* pos;     // [B][Tq]
+    const int32_t* n;       // [B]
+    uint32_t* keys;         // [QB][KS] scratch for this block of queries
+    int32_t* idx;           // [B][Tq][k]
+    int32_t* cnt;           // [B][Tq]
+    int Tq, Ncap, KS, k, log2m;
+    int b, t0, qb;          // this launch: sequence b, queries t0 .. t0+qb-1
+};
+
+__device__ __forceinline__ int visible_entries(const TopkPrefillArgs& a, int t) {
+    int nb = a.n[a.b];
+    if (nb < 0 || nb > a.Ncap) {
+        flag(DEV_LEN);
+        nb = nb < 0 ? 0 : a.Ncap;
+    }
+    int p = a.pos[(size_t)a.b * a.Tq + t];
+    if (p < 0) {
+        flag(DEV_POS);
+        p = 0;
+    }
+    return min(nb, p >> a.log2m);
+}
+
+__global__ void __launch_bounds__(kPsThreads, 2) score_prefill_kernel(TopkPrefillArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    double* sQ = reinterpret_cast<double*>(smem);                        // [64 dims][64 queries]
+    uint32_t* sK = reinterpret_cast<uint32_t*>(smem + 64 * kPsQ * 8);    // [32 dim pairs][128 entries]
+    __shared__ int s_maxvis;
+
+    const int tid = threadIdx.x;
+    const int e0 = blockIdx.x * kPsE;
+    const int ql0 = blockIdx.y * kPsQ;  // first query of the tile, local to the block
+    if (tid == 0) s_maxvis = 0;
+    __syncthreads();
+    if (tid < kPsQ && ql0 + tid < a.qb) atomicMax(&s_maxvis, visible_entries(a, a.t0 + ql0 + tid));
+    __syncthreads();
+    if (e0 >= s_maxvis) return;  // no query of this tile sees these entries
+
+    {  // queries: q * 2^768 as fp64, dim-major
+        const int ql = tid & 63;
+        const bool ok = ql0 + ql < a.qb;
+        const uint4* src = reinterpret_cast<const uint4*>(a.q_idx + ((size_t)a.b * a.Tq + a.t0 + ql0 + ql) * 64);
+        for (int c = tid >> 6; c < 8; c += kPsThreads / 64) {
+            const uint4 w = ok ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                sQ[(8 * c + 2 * u) * kPsQ + ql] = (double)bf16lo_f32(ws[u]) * 0x1p768;
+                sQ[(8 * c + 2 * u + 1) * kPsQ + ql] = (double)bf16hi_f32(ws[u]) * 0x1p768;
+            }
+        }
+    }
+    {  // keys: packed bf16 pairs, [dim pair][entry]
+        const int e = tid & 127;
+        const bool ok = e0 + e < a.Ncap;
+        const uint4* src = reinterpret_cast<const uint4*>(a.kidx + ((size_t)a.b * a.Ncap + e0 + e) * 64);
+        for (int c = tid >> 7; c < 8; c += kPsThreads / 128) {
+            const uint4 w = ok ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+            sK[(4 * c + 0) * kPsE + e] = w.x;
+            sK[(4 * c + 1) * kPsE + e] = w.y;
+            sK[(4 * c + 2) * kPsE + e] = w.z;
+            sK[(4 * c + 3) * kPsE + e] = w.w;
+        }
+    }
+    __syncthreads();
+
+    const int tq = tid >> 4, te = tid & 15;
+    double acc[4][8];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 8; ++v) acc[u][v] = 0.0;
+
+#pragma unroll 2
+    for (int i2 = 0; i2 < 32; ++i2) {
+        const uint4 k0 = *reinterpret_cast<const uint4*>(sK + i2 * kPsE + te * 4);
+        const uint4 k1 = *reinterpret_cast<const uint4*>(sK + i2 * kPsE + 64 + te * 4);
+        const uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // dim 2*i2 + h, ascending
+            const double2 qa = *reinterpret_cast<const double2*>(sQ + (2 * i2 + h) * kPsQ + tq * 4);
+            const double2 qb = *reinterpret_cast<const double2*>(sQ + (2 * i2 + h) * kPsQ + tq * 4 + 2);
+            const double qv[4] = {qa.x, qa.y, qb.x, qb.y};
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                const double kd = h ? bf16hi_scaled(kw[v]) : bf16lo_scaled(kw[v]);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) acc[u][v] = fma(qv[u], kd, acc[u][v]);
+            }
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int ql = ql0 + tq * 4 + u;
+        if (ql >= a.qb) continue;
+        uint32_t* row = a.keys + (size_t)ql * a.KS + e0;
+        uint4 lo, hi;
+        lo.x = score_key(__double2float_rn(acc[u][0] * 0x1p128));
+        lo.y = score_key(__double2float_rn(acc[u][1] * 0x1p128));
+        lo.z = score_key(__double2float_rn(acc[u][2] * 0x1p128));
+        lo.w = score_key(__double2float_rn(acc[u][3] * 0x1p128));
+        hi.x = score_key(__double2float_rn(acc[u][4] * 0x1p128));
+        hi.y = score_key(__double2float_rn(acc[u][5] * 0x1p128));
+        hi.z = score_key(__double2float_rn(acc[u][6] * 0x1p128));
+        hi.w = score_key(__double2float_rn(acc[u][7] * 0x1p128));
+        *reinterpret_cast<uint4*>(row + te * 4) = lo;       // KS is a multiple of 128: in bounds
+        *reinterpret_cast<uint4*>(row + 64 + te * 4) = hi;
+    }
+}
+
+// Warp-aggregated shared-memory histogram increment (many equal bins).
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool valid) {
+    const uint32_t b = valid ? bin : 0xFFFFFFFFu;
+    const uint32_t peers = __match_any_sync(0xFFFFFFFFu, b);
+    const int leader = __ffs(peers) - 1;
+    if (valid && (int)(threadIdx.x & 31) == leader) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+}
+
+__global__ void __launch_bounds__(kSelThreads, 1) select_prefill_kernel(TopkPrefillArgs a) {
+    extern __shared__ __align__(16) uint32_t skeys[];  // [kSelSmemKeys]
+    __shared__ uint32_t hist[kBins];
+    __shared__ uint32_t sh32[32];
+    __shared__ int res[2];
+    const int ql = blockIdx.x;
+    const int t = a.t0 + ql;
+    const int k = a.k;
+    const int nv = visible_entries(a, t);
+    int32_t* idx = a.idx + ((size_t)a.b * a.Tq + t) * k;
+    if (nv <= k) {
+        for (int i = threadIdx.x; i < k; i += blockDim.x) idx[i] = i < nv ? i : -1;
+        if (threadIdx.x == 0) a.cnt[(size_t)a.b * a.Tq + t] = nv;
+        return;
+    }
+    const uint32_t* grow = a.keys + (size_t)ql * a.KS;
+    const uint32_t* kp = grow;
+    if (nv <= kSelSmemKeys) {
+        const int n4 = (nv + 3) >> 2;  // rows are 16-byte aligned (KS multiple of 128)
+        for (int i = threadIdx.x; i < n4; i += blockDim.x)
+            reinterpret_cast<uint4*>(skeys)[i] = reinterpret_cast<const uint4*>(grow)[i];
+        kp = skeys;
+    }
+    const int nround = (nv + blockDim.x - 1) / blockDim.x * blockDim.x;  // whole warps iterate together
+
+    // digit 1
+    for (int i = threadIdx.x; i < kBins; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int j = threadIdx.x; j < nround; j += blockDim.x) {
+        const bool v = j < nv;
+        hist_add(hist, v ? kp[j] >> 21 : 0u, v);
+    }
+    __syncthreads();
+    int d1, d2, d3;
+    uint32_t above;
+    find_digit_desc<kBins>(hist, (uint32_t)k, sh32, &d1, &above, res);
+    const uint32_t K1 = (uint32_t)k - above;
+    // digit 2
+    for (int i = threadIdx.x; i < kBins; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int j = threadIdx.x; j < nround; j += blockDim.x) {
+        const uint32_t key = j < nv ? kp[j] : 0u;
+        const bool v = j < nv && (int)(key >> 21) == d1;
+        hist_add(hist, (key >> 10) & (kBins - 1), v);
+    }
+    __syncthreads();
+    find_digit_desc<kBins>(hist, K1, sh32, &d2, &above, res);
+    const uint32_t K2 = K1 - above;
+    // digit 3
+    const uint32_t pre = ((uint32_t)d1 << 11) | (uint32_t)d2;
+    for (int i = threadIdx.x; i < kBinsLow; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int j = threadIdx.x; j < nround; j += blockDim.x) {
+        const uint32_t key = j < nv ? kp[j] : 0u;
+        const bool v = j < nv && (key >> 10) == pre;
+        hist_add(hist, key & (kBinsLow - 1), v);
+    }
+    __syncthreads();
+    find_digit_desc<kBinsLow>(hist, K2, sh32, &d3, &above, res);
+    const uint32_t r = K2 - above;
+    const uint32_t nties = hist[d3 < 0 ? 0 : d3];
+    __syncthreads();
+    if ((d1 | d2 | d3) < 0 && threadIdx.x == 0) flag(DEV_LEN);  // inconsistent: cannot happen
+    const uint32_t T = (pre << 10) | (uint32_t)d3;
+
+    // lowest-index tie-break: the r-th tie in index order
+    int jmax = 0x7FFFFFFF;
+    if (r < nties) {
+        uint32_t running = 0;
+        for (int j0 = 0; j0 < nround; j0 += blockDim.x) {
+            const int j = j0 + threadIdx.x;
+            const bool tie = j < nv && kp[j] == T;
+            uint32_t tot;
+            const uint32_t before = running + block_exclusive_scan(tie ? 1u : 0u, sh32, &tot);
+            if (tie && before + 1 == r) res[0] = j;
+            running += tot;
+            if (running >= r) break;  // uniform: every thread sees the same running
+        }
+        __syncthreads();
+        jmax = res[0];
+        __syncthreads();
+    }
+    // ordered compaction of the selection
+    uint32_t running = 0;
+    for (int j0 = 0; j0 < nround; j0 += blockDim.x) {
+        const int j = j0 + threadIdx.x;
+        const uint32_t key = j < nv ? kp[j] : 0u;
+        const bool sel = j < nv && (key > T || (key == T && j <= jmax));
+        uint32_t tot;
+        const uint32_t p = running + block_exclusive_scan(sel ? 1u : 0u, sh32, &tot);
+        if (sel && p < (uint32_t)k) idx[p] = j;
+        running += tot;
+    }
+    if (threadIdx.x == 0) {
+        if (running != (uint32_t)k) flag(DEV_LEN);  // cannot happen
+        a.cnt[(size_t)a.b * a.Tq + t] = k;
+    }
+}
+
+__global__ void fill_positions_kernel(int32_t* pos, int B, int T) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < (long long)B * T) pos[i] = (int32_t)(i % T);
+}
+
+}  // namespace sa

@@ -1,0 +1,124 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every
+symbol the header declares, sizes workspaces, and rejects bad arguments on
+the host before anything is launched (no compute call is made here)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_attention_pool_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sparse_attn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return _lib.lib()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", text)) - {"sizeof"})
+
+
+def test_exports_every_header_symbol(L):
+    names = header_functions()
+    assert set(names) == set(_lib.EXPORTS)
+    for n in names:
+        assert hasattr(L, n), n
+    assert L.sa_abi_version() == 1
+
+
+def test_workspace_sizes(L):
+    ws = L.sa_workspace_size
+    assert ws(_lib.SA_OP_HYBRID_DECODE, 4, 1, 64, 262144, 8192, 2048) > 4 * 262144 * 12
+    assert ws(_lib.SA_OP_HYBRID_DECODE, 4, 2, 64, 262144, 8192, 2048) == 0   # decode is one query per sequence
+    assert ws(_lib.SA_OP_INDEX_TOPK, 1, 1, 8, 1024, 0, 0) == 0               # k = 0 is invalid
+    assert ws(99, 1, 1, 8, 1024, 0, 64) == 0
+    assert ws(_lib.SA_OP_SPARSE_ATTN, 1, 1, 129, 1024, 0, 64) == 0           # H > 128
+    # batch scales the decode workspace linearly, per sequence independent of the batch
+    a = ws(_lib.SA_OP_INDEX_TOPK, 1, 1, 64, 16384, 0, 512)
+    b = ws(_lib.SA_OP_INDEX_TOPK, 8, 1, 64, 16384, 0, 512)
+    assert a > 0 and b > 7 * (a - 1024)
+    assert ws(_lib.SA_OP_HYBRID_PREFILL, 1, 131072, 64, 32768, 1024, 2048) >= 1024 * 32768 * 4
+
+
+FAKE = 0x10000          # aligned, never dereferenced: every call below fails validation first
+
+
+def _cache(**kw):
+    c = _lib.SaCache(FAKE, FAKE, None, None, FAKE, FAKE, 1, 1024, 128, 64, 4, _lib.SA_BF16)
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+def _raw(**kw):
+    r = _lib.SaRaw(FAKE, FAKE, FAKE, FAKE, 1, 4096, 128, 64)
+    for k, v in kw.items():
+        setattr(r, k, v)
+    return r
+
+
+@pytest.mark.parametrize("raw_kw,cache_kw,frag", [
+    ({}, {"d": 64}, "head dim"),
+    ({}, {"m": 3}, "power of two"),
+    ({}, {"m": 2048}, "power of two"),
+    ({}, {"dtype": 7}, "dtype"),
+    ({}, {"kidx": None}, "kidx"),
+    ({}, {"k": FAKE + 4}, "aligned"),
+    ({}, {"dtype": _lib.SA_FP8_E4M3}, "k_scale"),
+    ({"kidx": None}, {}, "kidx"),
+    ({"B": 2}, {}, "B=2"),
+    ({"Lcap": 8192}, {}, "Ncap"),
+    ({"d": 256}, {}, "raw d"),
+])
+def test_compress_rejects_bad_arguments(L, raw_kw, cache_kw, frag):
+    r, c = _raw(**raw_kw), _cache(**cache_kw)
+    st = L.csa_compress(ctypes.byref(r), ctypes.byref(c), None)
+    assert st == _lib.SA_ERR_INVALID_ARG
+    assert frag in L.sa_last_error().decode()
+
+
+def test_null_descriptors(L):
+    assert L.csa_compress(None, None, None) == _lib.SA_ERR_INVALID_ARG
+    c = _cache()
+    assert L.hca_compress(None, ctypes.byref(c), None) == _lib.SA_ERR_INVALID_ARG
+    assert "raw descriptor" in L.sa_last_error().decode()
+
+
+def test_topk_and_attention_reject_bad_arguments(L):
+    c = _cache()
+    P = ctypes.c_void_p
+    # k out of range
+    assert L.csa_index_topk(P(FAKE), 1, None, ctypes.byref(c), 0, P(FAKE), P(FAKE), P(FAKE), 1 << 30, None) == 1
+    # decode with Tq > 1
+    assert L.csa_index_topk(P(FAKE), 2, None, ctypes.byref(c), 8, P(FAKE), P(FAKE), P(FAKE), 1 << 30, None) == 1
+    # workspace too small
+    st = L.csa_index_topk(P(FAKE), 1, None, ctypes.byref(c), 8, P(FAKE), P(FAKE), P(FAKE), 16, None)
+    assert st == _lib.SA_ERR_WORKSPACE and "workspace" in L.sa_last_error().decode()
+    # misaligned workspace
+    st = L.csa_index_topk(P(FAKE), 1, None, ctypes.byref(c), 8, P(FAKE), P(FAKE), P(FAKE + 16), 1 << 30, None)
+    assert st == _lib.SA_ERR_WORKSPACE
+    # H out of range, negative scale, NaN scale
+    assert L.csa_sparse_attn(P(FAKE), 1, 0, ctypes.byref(c), P(FAKE), P(FAKE), 8, 0.0, P(FAKE), None, P(FAKE),
+                             1 << 30, None) == 1
+    assert L.hca_dense_attn(P(FAKE), 1, 8, None, ctypes.byref(c), -1.0, P(FAKE), None, P(FAKE), 1 << 30, None) == 1
+    assert L.hca_dense_attn(P(FAKE), 1, 8, None, ctypes.byref(c), float("nan"), P(FAKE), None, P(FAKE), 1 << 30,
+                            None) == 1
+    # prefill needs idx_out / cnt_out
+    h = _cache(m=128, kidx=None)
+    assert L.hybrid_attn_prefill(P(FAKE), P(FAKE), 16, 8, ctypes.byref(c), ctypes.byref(h), 8, 0.0, P(FAKE),
+                                 P(FAKE), None, None, None, None, P(FAKE), 1 << 30, None) == 1
+    assert "idx_out" in L.sa_last_error().decode()
+    # mismatched batches
+    h2 = _cache(m=128, kidx=None, B=2)
+    assert L.hybrid_attn_decode(P(FAKE), P(FAKE), 8, ctypes.byref(c), ctypes.byref(h2), 8, 0.0, P(FAKE), P(FAKE),
+                                None, None, None, None, P(FAKE), 1 << 30, None) == 1
+    assert "B=" in L.sa_last_error().decode()
