@@ -22,6 +22,7 @@ import hashlib
 import json
 import math
 import os
+import signal
 import statistics
 import subprocess
 import sys
@@ -37,7 +38,7 @@ from sparse_attention_pool_b200 import configs, synth  # noqa: E402
 DEFAULT_WORKLOAD = "decode_b4_t1m_h64_k2048"
 METRIC = "hybrid-attn decode tokens/s @1M ctx; achieved HBM GB/s (% of peak), 1 B200"
 SCALE = float(np.float32(1.0 / math.sqrt(128.0)))
-L2_FLUSH_BYTES = 512 << 20  # > 126 MB L2, written between timed steps
+L2_FLUSH_BYTES = 512 << 20  # > 126 MB L2: written, then read, between timed steps
 
 
 def measured_peaks():
@@ -85,22 +86,40 @@ class ClockSampler:
 
     def __enter__(self):
         try:
-            self.fh = open(self.path, "w")
+            # -f writes every sample straight to the file (stdout to a file would be block-buffered)
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+                                          "--format=csv,noheader,nounits", "-lms", "100", "-f", self.path],
+                                         stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
 
+    def lines(self):
+        try:
+            with open(self.path) as f:
+                return sum(1 for _ in f)
+        except OSError:
+            return 0
+
+    def keep_busy(self, work, min_samples, max_s=10.0):
+        """Run untimed work until the sampler has written `min_samples` more lines."""
+        if not self.proc:
+            return
+        import torch
+        start, t0 = self.lines(), time.time()
+        while self.lines() < start + min_samples and time.time() - t0 < max_s:
+            for _ in range(20):
+                work()
+            torch.cuda.synchronize()
+
     def __exit__(self, *exc):
         if self.proc:
-            self.proc.terminate()
+            self.proc.send_signal(signal.SIGINT)
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-            self.fh.close()
+                self.proc.wait()
 
     def summary(self):
         if not self.proc or not os.path.exists(self.path):
@@ -191,17 +210,30 @@ def run_ours(args, w, rank, world, dev):
     idx = torch.empty(B, k, dtype=torch.int32, device=dev)
     cnt = torch.empty(B, dtype=torch.int32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_sink = torch.empty(1, dtype=torch.int64, device=dev)
     stream = torch.cuda.current_stream()
+
+    def flush_l2():
+        # Writing a buffer larger than L2 evicts the step's data; reading it back
+        # then leaves L2 holding clean lines, so the timed step pays no write-back
+        # of the flush itself.
+        flush.fill_(1)
+        flush_sink.copy_(flush.view(torch.int64).sum())
     L = _lib.lib()
 
     def step():
         S.hybrid_attn_decode(q, qI, csa, hca, k, ws, scale=SCALE, out_csa=out_c, out_hca=out_h, lse_csa=lse_c,
                              lse_hca=lse_h, idx_out=idx, cnt_out=cnt)
 
-    # stage events around the indexer score kernel (captured into the graph)
-    ev_s0 = torch.cuda.Event(enable_timing=True)
-    ev_s1 = torch.cuda.Event(enable_timing=True)
-    L.sa_set_stage_events(_lib.SA_STAGE_INDEX_SCORE, ev_s0.cuda_event, ev_s1.cuda_event)
+    # events around every stage of the step (captured into the graph as record nodes)
+    stage_names = ["index_score", "topk_select", "csa_attn", "hca_attn"]
+    stage_ev = []
+    for si in range(len(stage_names)):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)  # creates the events; the library re-records them around the stage
+        e1.record(stream)
+        L.sa_set_stage_events(si, e0.cuda_event, e1.cuda_event)
+        stage_ev.append((e0, e1))
     step()  # eager first call: one-time kernel attributes
     torch.cuda.synchronize()
     S.read_device_status()
@@ -215,25 +247,30 @@ def run_ours(args, w, rank, world, dev):
         step()
     torch.cuda.synchronize()
     for _ in range(args.warmup):
-        flush.zero_()
+        flush_l2()
         graph.replay()
     torch.cuda.synchronize()
 
     ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    step_ms, score_ms = [], []
+    step_ms = []
+    stage_ms = [[] for _ in stage_names]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
+        clk.keep_busy(lambda: (flush_l2(), graph.replay()), min_samples=3)  # clocks under load first
         for i in range(args.steps):
-            flush.zero_()  # untimed: evict the caches from L2
+            flush_l2()  # untimed: evict the caches from L2
             ev0[i].record(stream)
             graph.replay()
             ev1[i].record(stream)
             ev1[i].synchronize()
             step_ms.append(ev0[i].elapsed_time(ev1[i]))
-            score_ms.append(ev_s0.elapsed_time(ev_s1))
+            for si, (e0, e1) in enumerate(stage_ev):
+                stage_ms[si].append(e0.elapsed_time(e1))
+        clk.keep_busy(lambda: (flush_l2(), graph.replay()), min_samples=2)
+    score_ms = stage_ms[0]
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -256,11 +293,12 @@ def run_ours(args, w, rank, world, dev):
     h2d = q_pin.numel() * 2 + qi_pin.numel() * 2
     d2h = oc_pin.numel() * 2 * 2 + lc_pin.numel() * 4 * 2
     e2e_ms = []
-    L.sa_set_stage_events(_lib.SA_STAGE_INDEX_SCORE, None, None)
+    for si in range(len(stage_names)):
+        L.sa_set_stage_events(si, None, None)
     if world > 1:
         dist.barrier()
     for i in range(args.steps):
-        flush.zero_()
+        flush_l2()
         ev0[i].record(stream)
         q_dev.copy_(q_pin, non_blocking=True)
         qi_dev.copy_(qi_pin, non_blocking=True)
@@ -304,13 +342,14 @@ def run_ours(args, w, rank, world, dev):
         "config": {"workload": w.name, "B_per_gpu": B, "context": int(w.L), "heads": H, "head_dim": 128,
                    "csa_m": w.m_csa, "topk": k, "hca_m": w.m_hca, "kv_dtype": "e4m3" if w.fp8 else "bf16",
                    "parallelism": f"replicas x{world} (independent sequences)",
-                   "l2": "flushed between timed steps (512 MB memset)", "launch": "CUDA graph replay"},
+                   "l2": "flushed between timed steps: 512 MB written then read back (clean L2)", "launch": "CUDA graph replay"},
         "hbm": {"step_bytes": step_bytes, "step_gbs": step_gbs, "step_frac": step_gbs / peak,
                 "step_frac_of_8tbs": step_gbs / 8000.0},
         "roofline": {"kernel": "score_decode_kernel", "bound": "hbm", "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                      "bytes_per_launch": score_bytes, "avg_launch_ms": score_avg,
                      "traffic": recorded_traffic("score_decode_kernel", w.name)},
+        "stages_ms": {n: statistics.mean(v) for n, v in zip(stage_names, stage_ms)},
         "gpu_launches": launches_per_step * args.steps,
         "e2e": {"value": tokens / (e2e_total / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "api": "hybrid_attn_decode (eager) + pinned-host copies"},

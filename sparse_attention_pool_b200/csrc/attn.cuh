@@ -63,21 +63,22 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-template <int NW, bool GATHER, bool FP8>
+template <int NW, bool GATHER, bool FP8, int ST>
 struct AttnSmem {
     static constexpr int kQBytes = NW * 16 * 256;
     static constexpr int kKVBytes = kTileN * 256;                 // one bf16 tile
     static constexpr int kStageRaw = FP8 ? kTileN * 128 : kKVBytes;  // one raw tile (K or V)
     static constexpr int kQ = 0;
-    static constexpr int kRaw = kQ + kQBytes;                      // [2 stages][K, V] raw tiles
-    static constexpr int kConv = kRaw + 2 * 2 * kStageRaw;         // fp8: widened K, V tiles
-    static constexpr int kMeta = kConv + (FP8 ? 2 * kKVBytes : 0);  // [2][64] valid + (fp8) scales
-    static constexpr int kTotal = kMeta + 2 * kTileN * 4 * 3;
+    static constexpr int kRaw = kQ + kQBytes;                      // [ST stages][K, V] raw tiles
+    static constexpr int kConv = kRaw + ST * 2 * kStageRaw;        // fp8: widened K, V tiles
+    static constexpr int kMeta = kConv + (FP8 ? 2 * kKVBytes : 0);  // [ST][64] valid + (fp8) scales
+    static constexpr int kTotal = kMeta + ST * kTileN * 4 * 3;
 };
 
-template <int NW, bool GATHER, bool FP8>
+// ST = pipeline stages: ST - 1 tiles are in flight while one is computed.
+template <int NW, bool GATHER, bool FP8, int ST>
 __global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
-    using L = AttnSmem<NW, GATHER, FP8>;
+    using L = AttnSmem<NW, GATHER, FP8, ST>;
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int split = blockIdx.x, bq = blockIdx.y;
@@ -114,9 +115,9 @@ __global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
     uint8_t* sQ = smem + L::kQ;
     uint8_t* sRaw = smem + L::kRaw;
     uint8_t* sConv = smem + L::kConv;
-    int* sValid = reinterpret_cast<int*>(smem + L::kMeta);           // [2][64]
-    float* sKs = reinterpret_cast<float*>(sValid + 2 * kTileN);       // [2][64]
-    float* sVs = sKs + 2 * kTileN;                                    // [2][64]
+    int* sValid = reinterpret_cast<int*>(smem + L::kMeta);           // [ST][64]
+    float* sKs = reinterpret_cast<float*>(sValid + ST * kTileN);      // [ST][64]
+    float* sVs = sKs + ST * kTileN;                                   // [ST][64]
 
     const uint16_t* qp = a.q + (size_t)bq * a.H * 128;
     // Q tile: rows >= H are zero
@@ -131,40 +132,49 @@ __global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
     const int rowBytes = FP8 ? 128 : 256;
     const size_t seqBase = (size_t)b * a.Ncap * rowBytes;
 
+    // each thread copies CPT 16-byte chunks of one row; a gathered row costs one index load
+    constexpr int cpr = FP8 ? 8 : 16;            // 16-byte chunks per row
+    constexpr int TPR = (NW * 32) / kTileN;      // threads per row
+    constexpr int CPT = cpr / TPR;               // chunks per thread
+    static_assert(TPR >= 1 && CPT >= 1 && CPT * TPR == cpr, "tile mapping");
     auto load_tile = [&](int tile, int stage) {
         const int p0 = p_begin + tile * kTileN;
         uint8_t* rk = sRaw + (stage * 2 + 0) * L::kStageRaw;
         uint8_t* rv = sRaw + (stage * 2 + 1) * L::kStageRaw;
-        constexpr int cpr = FP8 ? 8 : 16;  // 16-byte chunks per row
-        for (int c = tid; c < kTileN * cpr; c += NW * 32) {
-            const int r = c / cpr, ch = c % cpr;
-            const int p = p0 + r;
-            int j = p;
-            bool ok = p < p_end;
-            if (GATHER && ok) {
-                j = a.idx[(size_t)bq * a.kmax + p];
-                if (j < 0 || j >= nb) {
-                    ok = false;
-                    if (ch == 0) flag(DEV_INDEX);
-                }
+        const int r = tid / TPR, c0 = (tid % TPR) * CPT;
+        const int p = p0 + r;
+        int j = p;
+        bool ok = p < p_end;
+        if (GATHER && ok) {
+            j = a.idx[(size_t)bq * a.kmax + p];
+            if (j < 0 || j >= nb) {
+                ok = false;
+                if (c0 == 0) flag(DEV_INDEX);
             }
-            const size_t off = seqBase + (size_t)(ok ? j : 0) * rowBytes + ch * 16;
+        }
+        const size_t rowOff = seqBase + (size_t)(ok ? j : 0) * rowBytes;
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) {
+            const int ch = c0 + c;
             const uint32_t doff = FP8 ? (uint32_t)(r * 128 + ch * 16) : swz(r, ch);
-            cp_async16_zfill(rk + doff, Kb + off, ok);
-            cp_async16_zfill(rv + doff, Vb + off, ok);
-            if (ch == 0) {
-                sValid[stage * kTileN + r] = ok;
-                if (FP8) {
-                    const int g = ok ? j / 64 : 0;
-                    sKs[stage * kTileN + r] = ok ? a.ks[(size_t)b * a.nG + g] : 0.f;
-                    sVs[stage * kTileN + r] = ok ? a.vs[(size_t)b * a.nG + g] : 0.f;
-                }
+            cp_async16_zfill(rk + doff, Kb + rowOff + ch * 16, ok);
+            cp_async16_zfill(rv + doff, Vb + rowOff + ch * 16, ok);
+        }
+        if (c0 == 0) {
+            sValid[stage * kTileN + r] = ok;
+            if (FP8) {
+                const int g = ok ? j / 64 : 0;
+                sKs[stage * kTileN + r] = ok ? a.ks[(size_t)b * a.nG + g] : 0.f;
+                sVs[stage * kTileN + r] = ok ? a.vs[(size_t)b * a.nG + g] : 0.f;
             }
         }
     };
 
-    if (ntiles > 0) load_tile(0, 0);
-    cp_async_commit();
+#pragma unroll
+    for (int s = 0; s < ST - 1; ++s) {
+        if (s < ntiles) load_tile(s, s);
+        cp_async_commit();
+    }
 
     // per-thread state: rows r0 = lane/4 and r1 = lane/4 + 8 of this warp's 16 heads
     float o[16][4];
@@ -173,24 +183,21 @@ __global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
     float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
     uint32_t qf[8][4];
 
-    cp_async_wait<1>();  // Q landed
-    __syncthreads();
-    {
-        const uint32_t qbase = smem_u32(sQ);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            const int r = warp * 16 + (lane & 15);
-            const int ch = kk * 2 + (lane >> 4);
-            ldsm_x4(qbase + swz(r, ch), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
-        }
-    }
-
     for (int t = 0; t < ntiles; ++t) {
-        const int stage = t & 1;
-        if (t + 1 < ntiles) load_tile(t + 1, stage ^ 1);
+        const int stage = t % ST;
+        if (t + ST - 1 < ntiles) load_tile(t + ST - 1, (t + ST - 1) % ST);
         cp_async_commit();
-        cp_async_wait<1>();
+        cp_async_wait<ST - 1>();  // Q (first group) and tile t have landed
         __syncthreads();
+        if (t == 0) {
+            const uint32_t qbase = smem_u32(sQ);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const int r = warp * 16 + (lane & 15);
+                const int ch = kk * 2 + (lane >> 4);
+                ldsm_x4(qbase + swz(r, ch), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
+            }
+        }
 
         const uint8_t* tk;
         const uint8_t* tv;
@@ -354,25 +361,31 @@ __global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
     }
 }
 
-// Merge the split partials of every (query, head) in split order.
-__global__ void __launch_bounds__(256) attn_combine_kernel(const float* part_o, const float* part_lse, int splits,
-                                                           int H, uint16_t* out, float* lse) {
-    const int bq = blockIdx.y;
-    const int h = blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (h >= H) return;
+// Merge the split partials of one (query, head): one CTA of 8 warps, warp w
+// owns splits w, w+8, ...; every load is issued up front, the sums are then
+// reduced across warps in a fixed order (deterministic).
+constexpr int kCombThreads = 256;
+
+__global__ void __launch_bounds__(kCombThreads) attn_combine_kernel(const float* part_o, const float* part_lse,
+                                                                    int splits, int H, uint16_t* out, float* lse) {
+    __shared__ float4 red[kCombThreads / 32][32];
+    __shared__ float wred[kCombThreads / 32];
+    const int bh = blockIdx.x;  // bq * H + h
+    const int bq = bh / H, h = bh - bq * H;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const float* pl = part_lse + (size_t)bq * splits * H + h;
     float M = -INFINITY;
-    for (int s = 0; s < splits; ++s) M = fmaxf(M, pl[(size_t)s * H]);
+    for (int s = lane; s < splits; s += 32) M = fmaxf(M, pl[(size_t)s * H]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float wsum = 0.f;
     if (M != -INFINITY) {
-        for (int s = 0; s < splits; ++s) {
+        for (int s = warp; s < splits; s += kCombThreads / 32) {
             const float ls = pl[(size_t)s * H];
-            if (ls == -INFINITY) continue;
-            const float w = __expf(ls - M);
-            const float4 v = *reinterpret_cast<const float4*>(part_o + (((size_t)bq * splits + s) * H + h) * 128 +
-                                                              lane * 4);
+            const float w = ls == -INFINITY ? 0.f : __expf(ls - M);
+            const float4 v =
+                *reinterpret_cast<const float4*>(part_o + (((size_t)bq * splits + s) * H + h) * 128 + lane * 4);
             acc.x += w * v.x;
             acc.y += w * v.y;
             acc.z += w * v.z;
@@ -380,10 +393,25 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* part_o, 
             wsum += w;
         }
     }
-    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-    uint16_t* op = out + ((size_t)bq * H + h) * 128 + lane * 4;
-    *reinterpret_cast<uint2*>(op) = make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
-    if (lse && lane == 0) lse[(size_t)bq * H + h] = wsum > 0.f ? M + __logf(wsum) : -INFINITY;
+    red[warp][lane] = acc;
+    if (lane == 0) wred[warp] = wsum;
+    __syncthreads();
+    if (warp == 0) {
+        float4 t = red[0][lane];
+        float ws = wred[0];
+#pragma unroll
+        for (int w = 1; w < kCombThreads / 32; ++w) {
+            t.x += red[w][lane].x;
+            t.y += red[w][lane].y;
+            t.z += red[w][lane].z;
+            t.w += red[w][lane].w;
+            ws += wred[w];
+        }
+        const float inv = ws > 0.f ? 1.f / ws : 0.f;
+        uint16_t* op = out + ((size_t)bq * H + h) * 128 + lane * 4;
+        *reinterpret_cast<uint2*>(op) = make_uint2(pack_bf16x2(t.x * inv, t.y * inv), pack_bf16x2(t.z * inv, t.w * inv));
+        if (lse && lane == 0) lse[(size_t)bq * H + h] = ws > 0.f ? M + __logf(ws) : -INFINITY;
+    }
 }
 
 }  // namespace sa

@@ -25,8 +25,17 @@ thread_local char g_err[512] = "";
 thread_local uint64_t g_launches = 0;
 thread_local cudaEvent_t g_stage_ev[SA_NUM_STAGES][2] = {};
 
+// Inside a stream capture the record must become a graph node of its own
+// (an "external" record), so that replays re-record the event.
 inline void stage_mark(int stage, int which, cudaStream_t st) {
-    if (g_stage_ev[stage][which]) cudaEventRecord(g_stage_ev[stage][which], st);
+    cudaEvent_t ev = g_stage_ev[stage][which];
+    if (!ev) return;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(st, &cs);
+    if (cs == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal);
+    else
+        cudaEventRecord(ev, st);
 }
 
 sa_status fail(sa_status s, const char* fmt, ...) {
@@ -131,23 +140,46 @@ sa_status make_ic_map(CUtensorMap* map, const void* kidx, int B, int Ncap) {
 
 // ------------------------------------------------------- workspace layout --
 struct TopkDecodeWs {
-    size_t zero_off, zero_bytes, keys, cand_key, cand_idx, bitmap, idx, cnt, total;
-    int Wcap;
+    size_t hist, done, keys, emax, cand_key, cand_idx, amb_key, amb_idx, cand_cnt, in_cnt, bitmap, idx, cnt, total;
+    int maxchunks, Wcap;
 };
 
+// Rows per score CTA: about three CTAs per SM over the whole batch, whole tiles.
+int score_chunk(int B, int Ncap) {
+    const long long target = (long long)num_sms() * 3;
+    long long chunk = ((long long)B * Ncap + target - 1) / target;
+    chunk = ((chunk + sa::kScRows - 1) / sa::kScRows) * sa::kScRows;
+    return (int)std::max<long long>(chunk, sa::kScRows);
+}
+
+// [reserved 256 B][histograms][keys][per-chunk max error][candidate slots key/idx]
+// [band key/idx][per-chunk counts][bitmap][idx][cnt]
 TopkDecodeWs topk_decode_layout(int B, int Ncap, int k, bool own_idx) {
     TopkDecodeWs w{};
+    w.maxchunks = std::max(1, cdiv(Ncap, sa::kScRows));
     w.Wcap = ((Ncap + 31) / 32 + 1) & ~1;
-    size_t o = 256;  // bytes 0..255 are reserved
-    w.zero_off = o;
-    w.zero_bytes = up256((size_t)B * sa::kBins * 4 * 2 + (size_t)B * 4);
-    o += w.zero_bytes;
+    size_t o = 256;
+    w.hist = o;  // histograms and tickets are zeroed together before every call
+    o += (size_t)B * sa::kBins * 4;
+    w.done = o;
+    o += up256((size_t)B * 4);
+    const size_t col = up256((size_t)B * Ncap * 4);
     w.keys = o;
-    o += up256((size_t)B * Ncap * 4);
+    o += col;
+    w.emax = o;
+    o += up256((size_t)B * w.maxchunks * 4);
     w.cand_key = o;
-    o += up256((size_t)B * Ncap * 4);
+    o += col;
     w.cand_idx = o;
-    o += up256((size_t)B * Ncap * 4);
+    o += col;
+    w.amb_key = o;
+    o += col;
+    w.amb_idx = o;
+    o += col;
+    w.cand_cnt = o;
+    o += up256((size_t)B * w.maxchunks * 4);
+    w.in_cnt = o;
+    o += up256((size_t)B * w.maxchunks * 4);
     w.bitmap = o;
     o += up256((size_t)B * w.Wcap * 4);
     w.idx = o;
@@ -176,37 +208,64 @@ size_t attn_partial_bytes(long long BQ, int splits, int H) {
 }
 
 // ------------------------------------------------------------ launchers ----
-template <int NW, bool G, bool F>
+template <int NW, bool G, bool F, int ST>
 sa_status launch_attn_t(const sa::AttnArgs& a, dim3 grid, cudaStream_t st) {
-    using L = sa::AttnSmem<NW, G, F>;
+    using L = sa::AttnSmem<NW, G, F, ST>;
     static bool init = false;
     if (!init) {
-        SA_CUDA(cudaFuncSetAttribute(sa::attn_split_kernel<NW, G, F>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        SA_CUDA(cudaFuncSetAttribute(sa::attn_split_kernel<NW, G, F, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      L::kTotal));
         init = true;
     }
-    sa::attn_split_kernel<NW, G, F><<<grid, NW * 32, L::kTotal, st>>>(a);
+    sa::attn_split_kernel<NW, G, F, ST><<<grid, NW * 32, L::kTotal, st>>>(a);
     SA_LAUNCHED();
     return SA_OK;
 }
 
+template <int NW, int ST>
+sa_status launch_attn_nw(const sa::AttnArgs& a, bool gather, bool fp8, dim3 grid, cudaStream_t st) {
+    if (gather) return fp8 ? launch_attn_t<NW, true, true, ST>(a, grid, st) : launch_attn_t<NW, true, false, ST>(a, grid, st);
+    return fp8 ? launch_attn_t<NW, false, true, ST>(a, grid, st) : launch_attn_t<NW, false, false, ST>(a, grid, st);
+}
+
+// Splits of up to 4 tiles keep all of them in flight (4 stages); longer
+// lists (prefill) stream through a 2-stage pipeline.
 sa_status launch_attn(const sa::AttnArgs& a, bool gather, bool fp8, long long BQ, cudaStream_t st) {
-    dim3 grid(a.splits, (unsigned)BQ);
     if (BQ > 2147483647LL) return fail(SA_ERR_INVALID_ARG, "too many queries");
-    const bool big = a.H > 64;
-    if (!big) {
-        if (gather) return fp8 ? launch_attn_t<4, true, true>(a, grid, st) : launch_attn_t<4, true, false>(a, grid, st);
-        return fp8 ? launch_attn_t<4, false, true>(a, grid, st) : launch_attn_t<4, false, false>(a, grid, st);
-    }
-    if (gather) return fp8 ? launch_attn_t<8, true, true>(a, grid, st) : launch_attn_t<8, true, false>(a, grid, st);
-    return fp8 ? launch_attn_t<8, false, true>(a, grid, st) : launch_attn_t<8, false, false>(a, grid, st);
+    dim3 grid(a.splits, (unsigned)BQ);
+    const bool deep = a.tiles_per_split >= 2 && a.tiles_per_split <= 4;
+    if (a.H <= 64) return deep ? launch_attn_nw<4, 4>(a, gather, fp8, grid, st) : launch_attn_nw<4, 2>(a, gather, fp8, grid, st);
+    return deep ? launch_attn_nw<8, 4>(a, gather, fp8, grid, st) : launch_attn_nw<8, 2>(a, gather, fp8, grid, st);
 }
 
 sa_status launch_combine(const float* po, const float* pl, int splits, int H, long long BQ, uint16_t* out, float* lse,
                          cudaStream_t st) {
-    dim3 grid(cdiv(H, 8), (unsigned)BQ);
-    sa::attn_combine_kernel<<<grid, 256, 0, st>>>(po, pl, splits, H, out, lse);
+    if (BQ * H > 2147483647LL) return fail(SA_ERR_INVALID_ARG, "too many queries");
+    sa::attn_combine_kernel<<<(unsigned)(BQ * H), sa::kCombThreads, 0, st>>>(po, pl, splits, H, out, lse);
     SA_LAUNCHED();
+    return SA_OK;
+}
+
+// A side stream (per host thread and device) on which the HCA branch of a
+// hybrid decode step runs concurrently with the CSA chain.  Created by the
+// first hybrid call on a device, which should precede any stream capture.
+struct SideStream {
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+thread_local SideStream g_side[64];
+
+sa_status side_stream(SideStream** out) {
+    int dev = 0;
+    SA_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) return fail(SA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+    SideStream& ss = g_side[dev];
+    if (!ss.s) {
+        SA_CUDA(cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking));
+        SA_CUDA(cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming));
+        SA_CUDA(cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming));
+    }
+    *out = &ss;
     return SA_OK;
 }
 
@@ -250,55 +309,60 @@ sa_status run_attn(const void* q, int Tq, int H, const sa_cache* c, bool gather,
     return SA_OK;
 }
 
+// The indexer + top-k of a decode step: the score kernel (the HBM stream) and
+// the cluster selection kernel.  `between` runs after the score kernel is
+// queued (the hybrid step forks its HCA branch there).
+template <typename F>
 sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* idx, int32_t* cnt, void* ws,
-                          const TopkDecodeWs& w, cudaStream_t st) {
+                          const TopkDecodeWs& w, cudaStream_t st, F&& between) {
     const int B = c->B, Ncap = c->Ncap;
     uint8_t* base = static_cast<uint8_t*>(ws);
     sa::TopkDecodeArgs a{};
     a.q_idx = static_cast<const uint16_t*>(q_idx);
+    a.kidx = static_cast<const uint16_t*>(c->kidx);
     a.n = c->n;
     a.keys = reinterpret_cast<uint32_t*>(base + w.keys);
-    a.hist1 = reinterpret_cast<uint32_t*>(base + w.zero_off);
-    a.hist2 = a.hist1 + (size_t)B * sa::kBins;
-    a.cand_cnt = a.hist2 + (size_t)B * sa::kBins;
+    a.hist1 = reinterpret_cast<uint32_t*>(base + w.hist);
+    a.emax_part = reinterpret_cast<float*>(base + w.emax);
     a.cand_key = reinterpret_cast<uint32_t*>(base + w.cand_key);
     a.cand_idx = reinterpret_cast<int32_t*>(base + w.cand_idx);
+    a.amb_key = reinterpret_cast<uint32_t*>(base + w.amb_key);
+    a.amb_idx = reinterpret_cast<int32_t*>(base + w.amb_idx);
+    a.cand_cnt = reinterpret_cast<uint32_t*>(base + w.cand_cnt);
+    a.in_cnt = reinterpret_cast<uint32_t*>(base + w.in_cnt);
     a.bitmap = reinterpret_cast<uint32_t*>(base + w.bitmap);
+    a.done = reinterpret_cast<uint32_t*>(base + w.done);
     a.idx = idx;
     a.cnt = cnt;
     a.Ncap = Ncap;
     a.Wcap = w.Wcap;
     a.k = k;
-    // rows per CTA: about three CTAs per SM over the whole batch, whole tiles
-    const long long target = (long long)num_sms() * 3;
-    long long chunk = ((long long)B * Ncap + target - 1) / target;
-    chunk = ((chunk + sa::kScRows - 1) / sa::kScRows) * sa::kScRows;
-    if (chunk < sa::kScRows) chunk = sa::kScRows;
-    a.chunk = (int)chunk;
-    const int nchunks = Ncap > 0 ? cdiv(Ncap, chunk) : 1;
-
-    SA_CUDA(cudaMemsetAsync(base + w.zero_off, 0, w.zero_bytes, st));
+    a.chunk = score_chunk(B, Ncap);
+    a.nchunks = Ncap > 0 ? cdiv(Ncap, a.chunk) : 1;
+    if (a.nchunks > w.maxchunks || a.nchunks > sa::kSelMaxChunks)
+        return fail(SA_ERR_WORKSPACE, "internal: chunk count above the workspace bound");
+    static bool init = false;
+    const size_t smem = sa::kScStages * sa::kScTileBytes + sa::kScStages * 8 + 1024;
+    if (!init) {
+        SA_CUDA(cudaFuncSetAttribute(sa::score_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        SA_CUDA(cudaFuncSetAttribute(sa::topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     sa::kSelSmem));
+        init = true;
+    }
     if (Ncap > 0) {
         CUtensorMap map;
         sa_status r = make_ic_map(&map, c->kidx, B, Ncap);
         if (r != SA_OK) return r;
-        const size_t smem = sa::kScStages * sa::kScTileBytes + sa::kBins * 4 + sa::kScStages * 8 + 1024;
-        static bool init = false;
-        if (!init) {
-            SA_CUDA(cudaFuncSetAttribute(sa::score_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem));
-            init = true;
-        }
         stage_mark(SA_STAGE_INDEX_SCORE, 0, st);
-        sa::score_decode_kernel<<<dim3(nchunks, B), sa::kScThreads, smem, st>>>(map, a);
+        SA_CUDA(cudaMemsetAsync(a.hist1, 0, w.done - w.hist + (size_t)B * 4, st));
+        sa::score_decode_kernel<<<dim3(a.nchunks, B), sa::kScThreads, smem, st>>>(map, a);
         SA_LAUNCHED();
         stage_mark(SA_STAGE_INDEX_SCORE, 1, st);
-        stage_mark(SA_STAGE_TOPK_SELECT, 0, st);
-        sa::topk_filter_kernel<<<dim3(nchunks, B), sa::kFiltThreads, 0, st>>>(a);
-        SA_LAUNCHED();
     }
-    else stage_mark(SA_STAGE_TOPK_SELECT, 0, st);
-    sa::topk_resolve_kernel<<<B, sa::kResThreads, 0, st>>>(a);
+    sa_status r = between();
+    if (r != SA_OK) return r;
+    stage_mark(SA_STAGE_TOPK_SELECT, 0, st);
+    sa::topk_select_kernel<<<dim3(a.nchunks, B), sa::kSelThreads, sa::kSelSmem, st>>>(a);
     SA_LAUNCHED();
     stage_mark(SA_STAGE_TOPK_SELECT, 1, st);
     return SA_OK;
@@ -355,7 +419,7 @@ sa_status run_topk_prefill(const void* q_idx, int Tq, const int32_t* pos, const 
         SA_CUDA(cudaFuncSetAttribute(sa::score_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      sa::kPsSmem));
         SA_CUDA(cudaFuncSetAttribute(sa::select_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     sa::kSelSmemKeys * 4));
+                                     sa::kPselSmemKeys * 4));
         init = true;
     }
     const int etiles = std::max(1, cdiv(c->Ncap, sa::kPsE));
@@ -368,7 +432,7 @@ sa_status run_topk_prefill(const void* q_idx, int Tq, const int32_t* pos, const 
                 sa::score_prefill_kernel<<<dim3(etiles, cdiv(a.qb, sa::kPsQ)), sa::kPsThreads, sa::kPsSmem, st>>>(a);
                 SA_LAUNCHED();
             }
-            sa::select_prefill_kernel<<<a.qb, sa::kSelThreads, sa::kSelSmemKeys * 4, st>>>(a);
+            sa::select_prefill_kernel<<<a.qb, sa::kPselThreads, sa::kPselSmemKeys * 4, st>>>(a);
             SA_LAUNCHED();
         }
     }
@@ -510,7 +574,7 @@ sa_status csa_index_topk(const void* q_idx, int32_t Tq, const int32_t* q_pos, co
         TopkDecodeWs w = topk_decode_layout(csa->B, csa->Ncap, k, false);
         r = check_ws(ws, ws_bytes, w.total);
         if (r != SA_OK) return r;
-        return run_topk_decode(q_idx, csa, k, idx, cnt, ws, w, st);
+        return run_topk_decode(q_idx, csa, k, idx, cnt, ws, w, st, [] { return SA_OK; });
     }
     SA_CHECK(aligned16(q_pos), "csa_index_topk: q_pos must be 16-byte aligned");
     r = check_ws(ws, ws_bytes, prefill_topk_bytes(csa->B, Tq, csa->Ncap, k));
@@ -582,18 +646,31 @@ sa_status hybrid_attn_decode(const void* q, const void* q_idx, int32_t H, const 
     uint8_t* base = static_cast<uint8_t*>(ws);
     int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + w.idx);
     int32_t* cnt = cnt_out ? cnt_out : reinterpret_cast<int32_t*>(base + w.cnt);
-    r = run_topk_decode(q_idx, csa, k, idx, cnt, ws, w, st);
-    if (r != SA_OK) return r;
     const Split sc = attn_split(k, false);
+    // HCA needs neither the indexer nor the top-k: once the indexer stream is
+    // queued, fork it onto the side stream so that it overlaps the selection
+    // and the CSA attention instead of competing with the indexer stream.
+    SideStream* side = nullptr;
+    r = side_stream(&side);
+    if (r != SA_OK) return r;
+    auto fork_hca = [&]() -> sa_status {
+        SA_CUDA(cudaEventRecord(side->fork, st));
+        SA_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
+        stage_mark(SA_STAGE_HCA_ATTN, 0, side->s);
+        sa_status rr = run_attn(q, 1, H, hca, false, nullptr, nullptr, 0, nullptr, scale, out_hca, lse_hca, ws,
+                                w.total + attn_partial_bytes(csa->B, sc.splits, H), side->s);
+        if (rr != SA_OK) return rr;
+        stage_mark(SA_STAGE_HCA_ATTN, 1, side->s);
+        SA_CUDA(cudaEventRecord(side->join, side->s));
+        return SA_OK;
+    };
+    r = run_topk_decode(q_idx, csa, k, idx, cnt, ws, w, st, fork_hca);
+    if (r != SA_OK) return r;
     stage_mark(SA_STAGE_CSA_ATTN, 0, st);
     r = run_attn(q, 1, H, csa, true, idx, cnt, k, nullptr, scale, out_csa, lse_csa, ws, w.total, st);
     if (r != SA_OK) return r;
     stage_mark(SA_STAGE_CSA_ATTN, 1, st);
-    stage_mark(SA_STAGE_HCA_ATTN, 0, st);
-    r = run_attn(q, 1, H, hca, false, nullptr, nullptr, 0, nullptr, scale, out_hca, lse_hca, ws,
-                 w.total + attn_partial_bytes(csa->B, sc.splits, H), st);
-    if (r != SA_OK) return r;
-    stage_mark(SA_STAGE_HCA_ATTN, 1, st);
+    SA_CUDA(cudaStreamWaitEvent(st, side->join, 0));
     return SA_OK;
 }
 

@@ -2,25 +2,36 @@
 // per sequence), "DeepSeek-V4 ... Review", section 3-2 (2) (CSA keeps a sparse
 // top-k of the compressed entries) and 3-2 (4) (the CSA indexer QK path).
 //
-// score_j = fp32( fp64 sum_{i=0..63, ascending} qI[i] * Ic[j][i] ).  Each
-// bf16 x bf16 product is exact in fp64, so the fp64 FMA chain in ascending i
-// reproduces the definition bit for bit.  Selection keeps the k entries with
-// the largest (score, -j) and reports them in ascending j.
+// The selection is defined on s_j = fp32( fp64 sum_{i=0..63, ascending}
+// qI[i] * Ic[j][i] ): keep the k entries with the largest (s_j, -j), report
+// them in ascending j.  The kernels reach exactly that set without computing
+// every s_j in fp64:
 //
-// Three kernels, ordered on one stream:
-//   1. score_decode_kernel   -- streams the indexer keys Ic (the dominant HBM
-//      read of a decode step) through a TMA pipeline (128-byte rows, 128B
-//      swizzle, 4 stages), one row per thread, writes a 32-bit order key per
-//      entry and a histogram of the top 11 key bits (global atomics).
-//   2. topk_filter_kernel    -- finds the 11-bit digit holding the k-th key;
-//      writes a bitmap of entries whose digit is above it (surely selected),
-//      and compacts the entries of that digit into a candidate list with a
-//      histogram of their next 11 bits.
-//   3. topk_resolve_kernel   -- one CTA per sequence: resolves the remaining
-//      bits on the (small) candidate list, breaks ties at the threshold by
-//      lowest index, marks the winners in the bitmap and compacts the bitmap
-//      into ascending indices.
-// No kernel waits on another CTA: every hand-off is a kernel boundary.
+//   screen   s~_j = fp32 FMA chain over the same products (each bf16 x bf16
+//            product is exact in fp32), a~_j = fp32 FMA chain of |q||k|.
+//            Recursive summation bounds |s~_j - s_j| <= e_j with
+//              e_j = 2^-16 a~_j + 2^-22 |s~_j| + 2^-140
+//            (2^-18 would already cover the 64-term fp32 chain, the fp64
+//            chain and the final fp32 rounding; the absolute term covers
+//            products that underflow fp32).  E = max_j e_j per sequence.
+//   order    if t~ is the k-th largest s~, the k-th largest s lies within E
+//            of it, so entries with s~ > t~ + 2E are surely selected, entries
+//            with s~ < t~ - 2E surely not, and only the band |s~ - t~| <= 2E
+//            is rescored exactly (the fp64 definition) and ranked exactly.
+//
+// Two kernels, ordered on one stream:
+//   1. score_decode_kernel -- streams Ic through a 4-stage TMA pipeline
+//      (128-byte rows, 128B swizzle, one row per thread) and writes an order
+//      key of s~ per entry, a histogram of the top 11 key bits (per CTA in
+//      shared memory, then added to the sequence's) and each CTA's max e_j.
+//   2. topk_select_kernel  -- one CTA per score chunk: from the histogram the
+//      bin of t~; entries above that bin widened by 2E become bitmap bits
+//      (surely selected), entries in the widened bin become candidates in the
+//      chunk's own slot.  The last CTA of a sequence to finish (it takes a
+//      ticket after a fence; no CTA ever waits on another) gathers the
+//      candidates, finds t~ among them, rescores the band exactly, ranks it
+//      by (s, -j), marks the winners and compacts the bitmap into ascending
+//      indices.
 #pragma once
 #include "sa_common.cuh"
 
@@ -35,17 +46,22 @@ constexpr int kBinsLow = 1024;    // last 10-bit digit
 
 struct TopkDecodeArgs {
     const uint16_t* q_idx;  // [B][64]
+    const uint16_t* kidx;   // [B][Ncap][64] (exact rescoring)
     const int32_t* n;       // [B]
-    uint32_t* keys;         // [B][Ncap]
-    uint32_t* hist1;        // [B][2048]
-    uint32_t* hist2;        // [B][2048]
-    uint32_t* cand_cnt;     // [B]
-    uint32_t* cand_key;     // [B][Ncap]
+    uint32_t* keys;         // [B][Ncap]     order keys of the screened scores
+    uint32_t* hist1;        // [B][2048]     histogram of the top 11 key bits (zeroed per call)
+    float* emax_part;       // [B][nchunks]  per score CTA: max e_j
+    uint32_t* cand_key;     // [B][Ncap]     candidates, each chunk in its own slot
     int32_t* cand_idx;      // [B][Ncap]
-    uint32_t* bitmap;       // [B][Wcap]
+    uint32_t* cand_cnt;     // [B][nchunks]  candidates per chunk
+    uint32_t* in_cnt;       // [B][nchunks]  surely selected entries per chunk
+    uint32_t* bitmap;       // [B][Wcap]     selection bitmap
+    uint32_t* done;         // [B]           chunks filtered so far (zero between calls)
+    uint32_t* amb_key;      // [B][Ncap]     exact keys of the band, when it is large
+    int32_t* amb_idx;       // [B][Ncap]
     int32_t* idx;           // [B][k]
     int32_t* cnt;           // [B]
-    int Ncap, Wcap, chunk, k;
+    int Ncap, Wcap, chunk, nchunks, k;
 };
 
 __device__ __forceinline__ int clamp_n(const int32_t* n, int b, int Ncap) {
@@ -57,6 +73,30 @@ __device__ __forceinline__ int clamp_n(const int32_t* n, int b, int Ncap) {
     return v;
 }
 
+__device__ __forceinline__ float key_to_float(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+// The exact score of one indexer row (the definition): fp64 FMA chain in
+// ascending i over exact products, rounded once to fp32, -0 -> +0, as a key.
+__device__ __noinline__ uint32_t exact_key(const uint16_t* qI, const uint16_t* row) {
+    const uint4* r4 = reinterpret_cast<const uint4*>(row);
+    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qI);
+    double acc = 0.0;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const uint4 w = __ldg(r4 + c);
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const uint32_t qw = __ldg(q32 + c * 4 + h);
+            acc = fma((double)bf16lo_f32(qw), (double)bf16lo_f32(ws[h]), acc);
+            acc = fma((double)bf16hi_f32(qw), (double)bf16hi_f32(ws[h]), acc);
+        }
+    }
+    return score_key(__double2float_rn(acc));
+}
+
 // ------------------------------------------------------------ 1. scores ----
 __global__ void __launch_bounds__(kScThreads, 3)
     score_decode_kernel(const __grid_constant__ CUtensorMap ic_map, TopkDecodeArgs a) {
@@ -64,28 +104,30 @@ __global__ void __launch_bounds__(kScThreads, 3)
     // TMA with 128B swizzle needs a 1024-byte aligned destination
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* tiles = smem;
-    uint32_t* hist = reinterpret_cast<uint32_t*>(smem + kScStages * kScTileBytes);
-    uint64_t* full = reinterpret_cast<uint64_t*>(hist + kBins);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kScStages * kScTileBytes);
+    __shared__ float s_emax[kScThreads / 32];
+    __shared__ uint32_t hist[kBins];  // top 11 key bits of this CTA's rows
 
     const int b = blockIdx.y;
     const int n = clamp_n(a.n, b, a.Ncap);
     if (n <= a.k) return;  // everything visible is selected; nothing to score
     const int row0 = blockIdx.x * a.chunk;
     const int row1 = min(row0 + a.chunk, n);
-    if (row0 >= row1) return;
-    const int ntiles = (row1 - row0 + kScRows - 1) / kScRows;
     const int tid = threadIdx.x;
+    if (row0 >= row1) {
+        if (tid == 0) a.emax_part[(size_t)b * a.nchunks + blockIdx.x] = 0.f;
+        return;
+    }
+    const int ntiles = (row1 - row0 + kScRows - 1) / kScRows;
 
-    // qI * 2^768 in fp64: with keys held as x * 2^-896, each product is
-    // qI*k * 2^-128 exactly and no partial sum leaves the normal range.
-    double q[64];
+    float q[64];
     {
         const uint32_t* qw = reinterpret_cast<const uint32_t*>(a.q_idx + (size_t)b * 64);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const uint32_t w = __ldg(qw + i);
-            q[2 * i] = (double)bf16lo_f32(w) * 0x1p768;
-            q[2 * i + 1] = (double)bf16hi_f32(w) * 0x1p768;
+            q[2 * i] = bf16lo_f32(w);
+            q[2 * i + 1] = bf16hi_f32(w);
         }
     }
     for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0;
@@ -105,6 +147,7 @@ __global__ void __launch_bounds__(kScThreads, 3)
     }
     int consumed = 0;
     bool timed_out = false;
+    float emax = 0.f;
     for (int i = 0; i < ntiles; ++i) {
         const int s = i % kScStages;
         const bool ok = mbar_wait(&full[s], (i / kScStages) & 1);
@@ -116,22 +159,24 @@ __global__ void __launch_bounds__(kScThreads, 3)
         const int row = row0 + i * kScRows + tid;
         if (row < row1) {
             const uint8_t* rp = tiles + s * kScTileBytes + tid * 128;
-            double acc = 0.0;
+            float acc = 0.f, aab = 0.f;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 const uint4 w = *reinterpret_cast<const uint4*>(rp + ((c ^ (tid & 7)) << 4));
-                acc = fma(q[8 * c + 0], bf16lo_scaled(w.x), acc);
-                acc = fma(q[8 * c + 1], bf16hi_scaled(w.x), acc);
-                acc = fma(q[8 * c + 2], bf16lo_scaled(w.y), acc);
-                acc = fma(q[8 * c + 3], bf16hi_scaled(w.y), acc);
-                acc = fma(q[8 * c + 4], bf16lo_scaled(w.z), acc);
-                acc = fma(q[8 * c + 5], bf16hi_scaled(w.z), acc);
-                acc = fma(q[8 * c + 6], bf16lo_scaled(w.w), acc);
-                acc = fma(q[8 * c + 7], bf16hi_scaled(w.w), acc);
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const float k0 = bf16lo_f32(ws[h]), k1 = bf16hi_f32(ws[h]);
+                    acc = fmaf(q[8 * c + 2 * h], k0, acc);
+                    aab = fmaf(fabsf(q[8 * c + 2 * h]), fabsf(k0), aab);
+                    acc = fmaf(q[8 * c + 2 * h + 1], k1, acc);
+                    aab = fmaf(fabsf(q[8 * c + 2 * h + 1]), fabsf(k1), aab);
+                }
             }
-            const uint32_t key = score_key(__double2float_rn(acc * 0x1p128));
+            const uint32_t key = score_key(acc);
             a.keys[(size_t)b * a.Ncap + row] = key;
             atomicAdd(&hist[key >> 21], 1u);
+            emax = fmaxf(emax, fmaf(aab, 0x1p-16f, fmaf(fabsf(acc), 0x1p-22f, 0x1p-140f)));
         }
         __syncthreads();  // slot s is free again
         if (tid == 0 && issued < ntiles) {
@@ -143,21 +188,33 @@ __global__ void __launch_bounds__(kScThreads, 3)
     }
     if (timed_out) {
         // let copies still in flight land before the CTA's shared memory goes away
-        if (tid == 0)
+        if (tid == 0) {
             for (int i = consumed; i < issued; ++i) mbar_wait(&full[i % kScStages], (i / kScStages) & 1);
+            a.emax_part[(size_t)b * a.nchunks + blockIdx.x] = 0.f;
+        }
         __syncthreads();
         return;
     }
+    // e_j is rounded to nearest in fp32: one more ulp keeps it an upper bound
+    emax = __uint_as_float(__float_as_uint(emax) + 1u);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) emax = fmaxf(emax, __shfl_xor_sync(0xFFFFFFFFu, emax, o));
+    if ((tid & 31) == 0) s_emax[tid >> 5] = emax;
     __syncthreads();
+    if (tid == 0) {
+        float m = s_emax[0];
+        for (int w = 1; w < kScThreads / 32; ++w) m = fmaxf(m, s_emax[w]);
+        a.emax_part[(size_t)b * a.nchunks + blockIdx.x] = m;
+    }
     for (int i = tid; i < kBins; i += blockDim.x)
         if (hist[i]) atomicAdd(&a.hist1[(size_t)b * kBins + i], hist[i]);
 }
 
 // --------------------------------------------------- digit search helpers --
-// Descending: returns the digit d with  above(d) < K <= above(d) + h[d], where
+// Descending: the digit d with  above(d) < K <= above(d) + h[d], where
 // above(d) = sum of h[e] for e > d.  Every thread gets (d, above(d)).
 template <int NB>
-__device__ void find_digit_desc(const uint32_t* h, uint32_t K, uint32_t* sh32, int* out_d, uint32_t* out_above,
+__device__ __forceinline__ void find_digit_desc(const uint32_t* h, uint32_t K, uint32_t* sh32, int* out_d, uint32_t* out_above,
                                 int* res) {
     const int T = blockDim.x;
     const int per = (NB + T - 1) / T;
@@ -187,7 +244,7 @@ __device__ void find_digit_desc(const uint32_t* h, uint32_t K, uint32_t* sh32, i
 
 // Ascending: the digit d with  below(d) < R <= below(d) + h[d].
 template <int NB>
-__device__ void find_digit_asc(const uint32_t* h, uint32_t R, uint32_t* sh32, int* out_d, uint32_t* out_below,
+__device__ __forceinline__ void find_digit_asc(const uint32_t* h, uint32_t R, uint32_t* sh32, int* out_d, uint32_t* out_below,
                                int* res) {
     const int T = blockDim.x;
     const int per = (NB + T - 1) / T;
@@ -214,174 +271,529 @@ __device__ void find_digit_asc(const uint32_t* h, uint32_t R, uint32_t* sh32, in
     __syncthreads();
 }
 
-// ------------------------------------------------------------ 2. filter ----
-constexpr int kFiltThreads = 256;
-
-__global__ void __launch_bounds__(kFiltThreads) topk_filter_kernel(TopkDecodeArgs a) {
-    __shared__ uint32_t hsh[kBins];
-    __shared__ uint32_t sh32[32];
-    __shared__ int res[2];
-    const int b = blockIdx.y;
-    const int n = clamp_n(a.n, b, a.Ncap);
-    if (n <= a.k) return;
-    const int row0 = blockIdx.x * a.chunk;
-    const int row1 = min(row0 + a.chunk, n);
-    if (row0 >= row1) return;
-
-    for (int i = threadIdx.x; i < kBins; i += blockDim.x) hsh[i] = a.hist1[(size_t)b * kBins + i];
-    __syncthreads();
-    int d1;
-    uint32_t above1;
-    find_digit_desc<kBins>(hsh, (uint32_t)a.k, sh32, &d1, &above1, res);
-    for (int i = threadIdx.x; i < kBins; i += blockDim.x) hsh[i] = 0;
-    __syncthreads();
-
-    const int lane = threadIdx.x & 31;
-    const uint32_t* keys = a.keys + (size_t)b * a.Ncap;
-    // chunk and row0 are multiples of 32, so each warp owns whole bitmap words
-    const int rend = row0 + ((row1 - row0 + 31) & ~31);
-    for (int base = row0 + (threadIdx.x & ~31); base < rend; base += blockDim.x) {
-        const int row = base + lane;
-        const bool valid = row < row1;
-        const uint32_t key = valid ? keys[row] : 0u;
-        const int dig = (int)(key >> 21);
-        const bool sel = valid && dig > d1;
-        const bool cand = valid && dig == d1;
-        const uint32_t selm = __ballot_sync(0xFFFFFFFFu, sel);
-        const uint32_t candm = __ballot_sync(0xFFFFFFFFu, cand);
-        if (lane == 0) a.bitmap[(size_t)b * a.Wcap + (row >> 5)] = selm;
-        if (candm) {
-            uint32_t basepos = 0;
-            if (lane == 0) basepos = atomicAdd(&a.cand_cnt[b], (uint32_t)__popc(candm));
-            basepos = __shfl_sync(0xFFFFFFFFu, basepos, 0);
-            if (cand) {
-                const uint32_t pos = basepos + __popc(candm & ((1u << lane) - 1u));
-                if (pos < (uint32_t)a.Ncap) {
-                    a.cand_key[(size_t)b * a.Ncap + pos] = key;
-                    a.cand_idx[(size_t)b * a.Ncap + pos] = row;
-                }
-                atomicAdd(&hsh[(key >> 10) & (kBins - 1)], 1u);
-            }
-        }
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < kBins; i += blockDim.x)
-        if (hsh[i]) atomicAdd(&a.hist2[(size_t)b * kBins + i], hsh[i]);
+// Warp-aggregated shared-memory histogram increment (many equal bins).
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool valid) {
+    const uint32_t b = valid ? bin : 0xFFFFFFFFu;
+    const uint32_t peers = __match_any_sync(0xFFFFFFFFu, b);
+    const int leader = __ffs(peers) - 1;
+    if (valid && (int)(threadIdx.x & 31) == leader) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
 }
 
-// ----------------------------------------------------------- 3. resolve ----
-constexpr int kResThreads = 1024;
+// Among list entries (key[i], idx[i]), i < cnt, find the R-th largest by
+// (key desc, idx asc): returns T and jmax such that exactly R entries satisfy
+// key > T || (key == T && idx <= jmax).  hist: >= 2048 words of shared memory.
+__device__ __forceinline__ void select_rank(const uint32_t* key, const int32_t* idx, uint32_t cnt, uint32_t R, uint32_t* hist,
+                            uint32_t* sh32, int* res, uint32_t* T_out, int32_t* jmax_out) {
+    const int shifts[3] = {21, 10, 0};
+    const int widths[3] = {11, 11, 10};
+    uint32_t prefix = 0, pmask = 0, rem = R;
+    for (int p = 0; p < 3; ++p) {
+        for (int i = threadIdx.x; i < kBins; i += blockDim.x) hist[i] = 0;
+        __syncthreads();
+        for (uint32_t i0 = 0; i0 < cnt; i0 += blockDim.x) {  // warp-uniform trip count
+            const uint32_t i = i0 + threadIdx.x;
+            const uint32_t kk = i < cnt ? key[i] : 0u;
+            hist_add(hist, (kk >> shifts[p]) & ((1u << widths[p]) - 1), i < cnt && (kk & pmask) == prefix);
+        }
+        __syncthreads();
+        int d;
+        uint32_t above;
+        find_digit_desc<kBins>(hist, rem, sh32, &d, &above, res);
+        if (d < 0) {
+            if (threadIdx.x == 0) flag(DEV_LEN);  // inconsistent counts: cannot happen
+            d = 0;
+        }
+        rem -= above;
+        prefix |= (uint32_t)d << shifts[p];
+        pmask |= ((1u << widths[p]) - 1) << shifts[p];
+    }
+    const uint32_t T = prefix;
+    // ties at T: keep the rem with the lowest indices (indices < 2^31)
+    uint32_t nties = 0;
+    for (uint32_t i = threadIdx.x; i < cnt; i += blockDim.x) nties += key[i] == T;
+    uint32_t total;
+    block_exclusive_scan(nties, sh32, &total);
+    int32_t jmax = 0x7FFFFFFF;
+    if (rem < total) {
+        const int ishift[3] = {20, 9, 0};
+        const int iwidth[3] = {11, 11, 9};
+        uint32_t ip = 0, im = 0, r2 = rem;
+        for (int p = 0; p < 3; ++p) {
+            for (int i = threadIdx.x; i < kBins; i += blockDim.x) hist[i] = 0;
+            __syncthreads();
+            for (uint32_t i0 = 0; i0 < cnt; i0 += blockDim.x) {
+                const uint32_t i = i0 + threadIdx.x;
+                const bool tie = i < cnt && key[i] == T;
+                const uint32_t j = tie ? (uint32_t)idx[i] : 0u;
+                hist_add(hist, (j >> ishift[p]) & ((1u << iwidth[p]) - 1), tie && (j & im) == ip);
+            }
+            __syncthreads();
+            int d;
+            uint32_t below;
+            find_digit_asc<kBins>(hist, r2, sh32, &d, &below, res);
+            if (d < 0) d = 0;
+            r2 -= below;
+            ip |= (uint32_t)d << ishift[p];
+            im |= ((1u << iwidth[p]) - 1) << ishift[p];
+        }
+        jmax = (int32_t)ip;
+    }
+    *T_out = T;
+    *jmax_out = jmax;
+}
 
-// Writes the set bits of bm[0..nwords) as ascending indices into out[0..cap).
-__device__ void compact_bitmap(const uint32_t* bm, int nwords, int32_t* out, uint32_t cap, uint32_t* sh32,
-                               uint32_t* total_out) {
+// The R-th largest key among cnt list keys, knowing that all of them except
+// a rare fringe share the top 11 bits d1 (the candidates of a filter bin):
+// keys above the bin are counted, the rest resolved with two digit passes
+// (bits 20..10 and 9..0), whose bins are well spread, with plain shared
+// atomics.  Returns false if the rank falls outside the bin (caller then
+// uses the general select_rank).
+__device__ __forceinline__ bool rank_in_bin(const uint32_t* key, uint32_t cnt, uint32_t R, int d1, uint32_t* hist,
+                                            uint32_t* sh32, int* res, uint32_t* T_out) {
+    uint32_t above = 0, inbin = 0;
+    for (uint32_t i = threadIdx.x; i < cnt; i += blockDim.x) {
+        const int dig = (int)(key[i] >> 21);
+        above += dig > d1;
+        inbin += dig == d1;
+    }
+    uint32_t tot_above, tot_in;
+    block_exclusive_scan(above, sh32, &tot_above);
+    block_exclusive_scan(inbin, sh32, &tot_in);
+    if (R <= tot_above || R > tot_above + tot_in) return false;
+    uint32_t rem = R - tot_above;
+    for (int i = threadIdx.x; i < kBins; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (uint32_t i = threadIdx.x; i < cnt; i += blockDim.x) {
+        const uint32_t kk = key[i];
+        if ((int)(kk >> 21) == d1) atomicAdd(&hist[(kk >> 10) & (kBins - 1)], 1u);
+    }
+    __syncthreads();
+    int d2, d3;
+    uint32_t ab;
+    find_digit_desc<kBins>(hist, rem, sh32, &d2, &ab, res);
+    rem -= ab;
+    const uint32_t pre = ((uint32_t)d1 << 11) | (uint32_t)d2;
+    for (int i = threadIdx.x; i < kBinsLow; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (uint32_t i = threadIdx.x; i < cnt; i += blockDim.x) {
+        const uint32_t kk = key[i];
+        if ((kk >> 10) == pre) atomicAdd(&hist[kk & (kBinsLow - 1)], 1u);
+    }
+    __syncthreads();
+    find_digit_desc<kBinsLow>(hist, rem, sh32, &d3, &ab, res);
+    if (d2 < 0 || d3 < 0) return false;
+    *T_out = (pre << 10) | (uint32_t)d3;
+    return true;
+}
+
+// --------------------------------------------------------- 2. selection ----
+constexpr int kSelThreads = 256;
+constexpr int kSelKPT = 16;                  // keys per thread held in registers per pass
+constexpr int kSelCap = 6144;                // candidates the resolving CTA holds in shared memory
+constexpr int kSelSmem = kSelCap * 8;
+constexpr int kSelMaxChunks = 1024;
+
+struct FilterBounds {
+    float in_above;  // s~ > in_above  : surely selected
+    float c_lo;      // c_lo <= s~ <= in_above : candidate
+};
+
+// The bin of the k-th largest screened key, widened by 2E on both sides.
+__device__ __forceinline__ FilterBounds filter_bounds(int d1, float E) {
+    float lo = key_to_float((uint32_t)d1 << 21);
+    float hi = key_to_float(((uint32_t)d1 << 21) | 0x1FFFFFu);
+    if (isnan(lo)) lo = -INFINITY;  // the outermost bins also hold the NaN key ranges
+    if (isnan(hi)) hi = INFINITY;
+    const float e2 = __fmul_ru(2.f, E);
+    return {__fadd_ru(hi, e2), __fsub_rd(lo, e2)};
+}
+
+// Writes the set bits of (bm | extra)[0..nwords) as ascending indices into
+// out[0..cap); `extra` is an optional bitmap in shared memory.  Per round of
+// 16 * blockDim words, word w0 + i*T + t goes to thread t (coalesced loads,
+// all issued first); prefixes come from one warp scan per i and a single
+// block scan over the (i, warp) totals, taken in word order.  With `ostage`
+// (shared, >= cap words) the indices are staged and leave in coalesced
+// stores; scattered 4-byte global stores from one SM are slow.
+// `wt` is shared scratch of 16 * blockDim / 32 words.
+__device__ __forceinline__ void compact_bitmap(const uint32_t* bm, const uint32_t* extra, int nwords, int32_t* out,
+                                               uint32_t cap, uint32_t* ostage, uint32_t* wt, uint32_t* sh32,
+                                               uint32_t* total_out) {
+    constexpr int P = 16;
+    const int T = blockDim.x, W = T >> 5;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t running = 0;
-    for (int w0 = 0; w0 < nwords; w0 += blockDim.x) {
-        const int w = w0 + threadIdx.x;
-        uint32_t word = w < nwords ? bm[w] : 0u;
+    for (int w0 = 0; w0 < nwords; w0 += T * P) {
+        uint32_t v[P], incl[P];
+#pragma unroll
+        for (int i = 0; i < P; ++i) {
+            const int w = w0 + i * T + threadIdx.x;
+            v[i] = w < nwords ? __ldcg(bm + w) : 0u;
+        }
+        if (extra) {
+#pragma unroll
+            for (int i = 0; i < P; ++i) {
+                const int w = w0 + i * T + threadIdx.x;
+                if (w < nwords) v[i] |= extra[w];
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < P; ++i) {
+            uint32_t x = __popc(v[i]);
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+                if (lane >= o) x += y;
+            }
+            incl[i] = x;
+            if (lane == 31) wt[i * W + warp] = x;
+        }
+        __syncthreads();
         uint32_t tot;
-        uint32_t pos = running + block_exclusive_scan((uint32_t)__popc(word), sh32, &tot);
-        while (word) {
-            const int bit = __ffs(word) - 1;
-            word &= word - 1;
-            if (pos < cap) out[pos] = w * 32 + bit;
-            ++pos;
+        const uint32_t mine = threadIdx.x < P * W ? wt[threadIdx.x] : 0u;  // (i, warp) in word order
+        const uint32_t ex = block_exclusive_scan(mine, sh32, &tot);
+        if (threadIdx.x < P * W) wt[threadIdx.x] = ex;
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < P; ++i) {
+            uint32_t word = v[i];
+            uint32_t pos = running + wt[i * W + warp] + incl[i] - __popc(word);
+            const int wbase = (w0 + i * T + threadIdx.x) * 32;
+            while (word) {
+                const int bit = __ffs(word) - 1;
+                word &= word - 1;
+                if (pos < cap) {
+                    if (ostage) ostage[pos] = (uint32_t)(wbase + bit);
+                    else out[pos] = wbase + bit;
+                }
+                ++pos;
+            }
         }
         running += tot;
+        __syncthreads();  // wt is reused
+    }
+    if (ostage) {
+        const uint32_t nout = running < cap ? running : cap;
+        for (uint32_t i = threadIdx.x; i < nout; i += T) out[i] = (int32_t)ostage[i];
     }
     *total_out = running;
 }
 
-__global__ void __launch_bounds__(kResThreads) topk_resolve_kernel(TopkDecodeArgs a) {
-    __shared__ uint32_t hsh[kBins];
-    __shared__ uint32_t sh32[32];
-    __shared__ int res[2];
-    const int b = blockIdx.x;
+struct SelSmem {
+    uint32_t hist[kBins];
+    uint32_t coff[kSelMaxChunks + 1];
+    uint32_t sh32[32];
+    int res[2];
+    float red[kSelThreads / 32];
+    uint32_t last, amb_cnt, in2, wcnt, T2;
+    int32_t jmax2;
+    uint32_t amb_key[kSelThreads];
+    int32_t amb_idx[kSelThreads];
+};
+
+// The resolve step of topk_select_kernel over the C gathered candidates, with
+// the candidate list in shared memory (SMEM) or in global memory.
+template <bool SMEM>
+__device__ __forceinline__ void resolve_candidates(const TopkDecodeArgs& a, SelSmem& S, uint32_t* csm, int b,
+                                                   uint32_t C, uint32_t R1, int d1, float E) {
+    constexpr bool fits = SMEM;
+    uint32_t* lk = fits ? csm : a.amb_key + (size_t)b * a.Ncap;
+    int32_t* li = fits ? reinterpret_cast<int32_t*>(csm + kSelCap) : a.amb_idx + (size_t)b * a.Ncap;
+    const int tid = threadIdx.x;
+    uint32_t* bm = a.bitmap + (size_t)b * a.Wcap;
+    const int k = a.k;
+    const uint32_t* sk = a.cand_key + (size_t)b * a.Ncap;
+    const int32_t* si = a.cand_idx + (size_t)b * a.Ncap;
+    {
+        // 4 candidates per thread and round: loads first, then the stores
+        constexpr int U = 4;
+        for (uint32_t e0 = 0; e0 < C; e0 += U * kSelThreads) {
+            uint32_t kv[U];
+            int32_t iv[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const uint32_t e_ = e0 + u * kSelThreads + tid;
+                int lo_ = 0, hi_ = a.nchunks;  // the chunk q with coff[q] <= e_ < coff[q+1]
+                while (hi_ - lo_ > 1) {
+                    const int mid = (lo_ + hi_) >> 1;
+                    if (S.coff[mid] <= e_) lo_ = mid;
+                    else hi_ = mid;
+                }
+                const size_t src = (size_t)lo_ * a.chunk + (e_ - S.coff[lo_]);
+                kv[u] = e_ < C ? __ldcg(sk + src) : 0u;
+                iv[u] = e_ < C ? __ldcg(si + src) : 0;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const uint32_t e_ = e0 + u * kSelThreads + tid;
+                if (e_ < C) {
+                    if (fits) {
+                        csm[e_] = kv[u];
+                        csm[kSelCap + e_] = (uint32_t)iv[u];
+                    } else {
+                        lk[e_] = kv[u];
+                        li[e_] = iv[u];
+                    }
+                }
+            }
+        }
+    }
+    __syncthreads();
+
+    uint32_t tkey;
+    if (!rank_in_bin(lk, C, R1, d1, S.hist, S.sh32, S.res, &tkey)) {
+        int32_t jd;
+        select_rank(lk, li, C, R1, S.hist, S.sh32, S.res, &tkey, &jd);
+    }
+    const float t = key_to_float(tkey);
+    const float e2 = __fmul_ru(2.f, E);
+    const float band_hi = __fadd_ru(t, e2), band_lo = __fsub_rd(t, e2);
+    const uint16_t* qI = a.q_idx + (size_t)b * 64;
+    const uint16_t* icx = a.kidx + (size_t)b * a.Ncap * 64;
+    // the band list: global arrays not in use as the candidate list
+    uint32_t* gak = fits ? a.amb_key + (size_t)b * a.Ncap : a.cand_key + (size_t)b * a.Ncap;
+    int32_t* gai = fits ? a.amb_idx + (size_t)b * a.Ncap : a.cand_idx + (size_t)b * a.Ncap;
+    uint32_t my_in2 = 0;
+    for (uint32_t i = tid; i < C; i += kSelThreads) {
+        const float sv = key_to_float(lk[i]);
+        if (sv > band_hi) {
+            ++my_in2;
+        } else if (sv >= band_lo) {
+            const int32_t j = li[i];
+            const uint32_t p = atomicAdd(&S.amb_cnt, 1u);
+            const uint32_t ek = exact_key(qI, icx + (size_t)j * 64);
+            if (p < (uint32_t)kSelThreads) {
+                S.amb_key[p] = ek;
+                S.amb_idx[p] = j;
+            }
+            gak[p] = ek;
+            gai[p] = j;
+        }
+    }
+    uint32_t in2;
+    block_exclusive_scan(my_in2, S.sh32, &in2);
+    const uint32_t na = S.amb_cnt;
+    const uint32_t R2 = R1 - in2;  // winners to take from the band (1 <= R2 <= na)
+    // the exact cut of the band: a member wins iff (key, -j) >= (T2, -jmax2)
+    if (na <= (uint32_t)kSelThreads) {
+        if (tid < na) {
+            const uint32_t mk = S.amb_key[tid];
+            const int32_t mj = S.amb_idx[tid];
+            uint32_t rank = 0;
+            for (uint32_t o = 0; o < na; ++o) {
+                const uint32_t ok = S.amb_key[o];
+                rank += (ok > mk) || (ok == mk && S.amb_idx[o] < mj);
+            }
+            if (rank == R2 - 1) {
+                S.T2 = mk;
+                S.jmax2 = mj;
+            }
+        }
+        __syncthreads();
+    } else {
+        __syncthreads();
+        uint32_t T2;
+        int32_t jmax2;
+        select_rank(gak, gai, na, R2, S.hist, S.sh32, S.res, &T2, &jmax2);
+        if (tid == 0) {
+            S.T2 = T2;
+            S.jmax2 = jmax2;
+        }
+        __syncthreads();
+    }
+    const uint32_t T2 = S.T2;
+    const int32_t jmax2 = S.jmax2;
+    // winners of the candidates -> a list in shared memory (S.hist, R1 <= 2048
+    // of them) when it fits, else straight into the global bitmap
+    const bool wlist = R1 <= (uint32_t)kBins;
+    if (tid == 0) S.wcnt = 0;
+    __syncthreads();
+    for (uint32_t i = tid; i < C; i += kSelThreads) {
+        if (key_to_float(lk[i]) > band_hi) {
+            const int32_t j = li[i];
+            if (wlist) S.hist[atomicAdd(&S.wcnt, 1u)] = (uint32_t)j;
+            else atomicOr(&bm[j >> 5], 1u << (j & 31));
+        }
+    }
+    for (uint32_t i = tid; i < na; i += kSelThreads) {
+        const uint32_t kk = na <= (uint32_t)kSelThreads ? S.amb_key[i] : __ldcg(gak + i);
+        const int32_t j = na <= (uint32_t)kSelThreads ? S.amb_idx[i] : __ldcg(gai + i);
+        if (kk > T2 || (kk == T2 && j <= jmax2)) {
+            if (wlist) S.hist[atomicAdd(&S.wcnt, 1u)] = (uint32_t)j;
+            else atomicOr(&bm[j >> 5], 1u << (j & 31));
+        }
+    }
+    __syncthreads();
+}
+
+// One CTA per score chunk.  Filter: surely-selected entries become bitmap
+// bits, candidates go to the chunk's own slot.  The last CTA of a sequence to
+// finish (a ticket taken after a fence; nobody waits) then resolves it: finds
+// t~ among the gathered candidates, rescores the band exactly, marks the
+// winners and compacts the bitmap into ascending indices.
+__global__ void __launch_bounds__(kSelThreads, 3) topk_select_kernel(TopkDecodeArgs a) {
+    extern __shared__ __align__(16) uint32_t csm[];  // resolver: [kSelCap] keys, [kSelCap] indices
+    __shared__ SelSmem S;
+    const int b = blockIdx.y, c = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int n = clamp_n(a.n, b, a.Ncap);
     const int k = a.k;
-    int32_t* idx = a.idx + (size_t)b * k;
     if (n <= k) {
-        for (int i = threadIdx.x; i < k; i += blockDim.x) idx[i] = i < n ? i : -1;
-        if (threadIdx.x == 0) a.cnt[b] = n;
+        if (c == 0) {
+            int32_t* idx = a.idx + (size_t)b * k;
+            for (int i = tid; i < k; i += blockDim.x) idx[i] = i < n ? i : -1;
+            if (tid == 0) a.cnt[b] = n;
+        }
         return;
     }
-    // digit 1 (bits 31..21)
-    for (int i = threadIdx.x; i < kBins; i += blockDim.x) hsh[i] = a.hist1[(size_t)b * kBins + i];
-    __syncthreads();
-    int d1, d2, d3;
-    uint32_t above;
-    find_digit_desc<kBins>(hsh, (uint32_t)k, sh32, &d1, &above, res);
-    uint32_t K1 = (uint32_t)k - above;
-    // digit 2 (bits 20..10) among the candidates of digit 1
-    for (int i = threadIdx.x; i < kBins; i += blockDim.x) hsh[i] = a.hist2[(size_t)b * kBins + i];
-    __syncthreads();
-    find_digit_desc<kBins>(hsh, K1, sh32, &d2, &above, res);
-    uint32_t K2 = K1 - above;
-    // digit 3 (bits 9..0)
-    uint32_t c1 = a.cand_cnt[b];
-    if (c1 > (uint32_t)a.Ncap) {
-        if (threadIdx.x == 0) flag(DEV_LEN);
-        c1 = a.Ncap;
-    }
-    const uint32_t* ck = a.cand_key + (size_t)b * a.Ncap;
-    const int32_t* ci = a.cand_idx + (size_t)b * a.Ncap;
-    for (int i = threadIdx.x; i < kBinsLow; i += blockDim.x) hsh[i] = 0;
-    __syncthreads();
-    for (uint32_t i = threadIdx.x; i < c1; i += blockDim.x) {
-        const uint32_t key = ck[i];
-        if ((int)((key >> 10) & (kBins - 1)) == d2) atomicAdd(&hsh[key & (kBinsLow - 1)], 1u);
-    }
-    __syncthreads();
-    find_digit_desc<kBinsLow>(hsh, K2, sh32, &d3, &above, res);
-    const uint32_t r = K2 - above;  // ties at the threshold key to keep (>= 1)
-    const uint32_t nties = hsh[d3 < 0 ? 0 : d3];
-    __syncthreads();
-    const uint32_t T = ((uint32_t)d1 << 21) | ((uint32_t)d2 << 10) | (uint32_t)d3;
-    if (d1 < 0 || d2 < 0 || d3 < 0) {
-        if (threadIdx.x == 0) flag(DEV_LEN);  // inconsistent histograms: cannot happen
-    }
+    const int row0 = c * a.chunk;
+    const int row1 = min(row0 + a.chunk, n);
 
-    // lowest-index tie-break: jmax = the r-th smallest index among ties at T
-    int32_t jmax = 0x7FFFFFFF;
-    if (r < nties) {
-        uint32_t prefix = 0, R = r;
-        // indices < 2^31: digits of 11, 11 and 9 bits from the top
-        const int shifts[3] = {20, 9, 0};
-        const int widths[3] = {11, 11, 9};
-        uint32_t pmask = 0;
-        for (int p = 0; p < 3; ++p) {
-            const int nb = 1 << widths[p];
-            for (int i = threadIdx.x; i < kBins; i += blockDim.x) hsh[i] = 0;
-            __syncthreads();
-            for (uint32_t i = threadIdx.x; i < c1; i += blockDim.x) {
-                if (ck[i] != T) continue;
-                const uint32_t j = (uint32_t)ci[i];
-                if ((j & pmask) != prefix) continue;
-                atomicAdd(&hsh[(j >> shifts[p]) & (nb - 1)], 1u);
-            }
-            __syncthreads();
-            int dd;
-            uint32_t below;
-            find_digit_asc<kBins>(hsh, R, sh32, &dd, &below, res);
-            R -= below;
-            prefix |= (uint32_t)dd << shifts[p];
-            pmask |= (uint32_t)(nb - 1) << shifts[p];
-        }
-        jmax = (int32_t)prefix;
-    }
-
-    // mark winners among the candidates, then compact the bitmap in index order
+    // ---- filter: issue every load first (histogram, error bound, keys)
+    uint32_t hv[kBins / kSelThreads];
+#pragma unroll
+    for (int u = 0; u < kBins / kSelThreads; ++u) hv[u] = __ldcg(a.hist1 + (size_t)b * kBins + u * kSelThreads + tid);
+    float e = 0.f;
+    for (int q = tid; q < a.nchunks; q += kSelThreads) e = fmaxf(e, __ldcg(a.emax_part + (size_t)b * a.nchunks + q));
+    const uint32_t* keys = a.keys + (size_t)b * a.Ncap;
+    uint32_t* ck = a.cand_key + (size_t)b * a.Ncap + row0;
+    int32_t* ci = a.cand_idx + (size_t)b * a.Ncap + row0;
     uint32_t* bm = a.bitmap + (size_t)b * a.Wcap;
-    for (uint32_t i = threadIdx.x; i < c1; i += blockDim.x) {
-        const uint32_t key = ck[i];
-        const int32_t j = ci[i];
-        if (key > T || (key == T && j <= jmax)) atomicOr(&bm[j >> 5], 1u << (j & 31));
+#pragma unroll
+    for (int u = 0; u < kBins / kSelThreads; ++u) S.hist[u * kSelThreads + tid] = hv[u];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) e = fmaxf(e, __shfl_xor_sync(0xFFFFFFFFu, e, o));
+    if (lane == 0) S.red[warp] = e;
+    __syncthreads();
+    float E = 0.f;
+#pragma unroll
+    for (int w = 0; w < kSelThreads / 32; ++w) E = fmaxf(E, S.red[w]);
+    int d1;
+    uint32_t above1;
+    find_digit_desc<kBins>(S.hist, (uint32_t)k, S.sh32, &d1, &above1, S.res);
+    if (d1 < 0) d1 = 0;  // cannot happen: the histogram counts all n > k keys
+    const FilterBounds fb = filter_bounds(d1, E);
+
+    uint32_t ncand = 0, nin = 0;
+    for (int p0 = row0; p0 < row1; p0 += kSelKPT * kSelThreads) {  // passes of up to 8192 rows
+        uint32_t kr[kSelKPT];
+#pragma unroll
+        for (int i = 0; i < kSelKPT; ++i) {
+            const int row = p0 + i * kSelThreads + tid;
+            kr[i] = row < row1 ? __ldcg(keys + row) : 0u;
+        }
+        uint32_t cmask = 0, mycnt = 0;
+#pragma unroll
+        for (int i = 0; i < kSelKPT; ++i) {
+            const int row = p0 + i * kSelThreads + tid;
+            const int wrow = p0 + i * kSelThreads + warp * 32;  // this warp's 32 consecutive rows
+            const float sv = key_to_float(kr[i]);
+            const bool valid = row < row1;
+            const bool sel = valid && sv > fb.in_above;
+            const bool cand = valid && !sel && sv >= fb.c_lo;
+            const uint32_t selm = __ballot_sync(0xFFFFFFFFu, sel);
+            if (lane == 0 && wrow < row1) bm[wrow >> 5] = selm;  // row0 is a multiple of 32
+            nin += __popc(selm);
+            if (cand) {
+                cmask |= 1u << i;
+                ++mycnt;
+            }
+        }
+        uint32_t tot;
+        uint32_t pos = ncand + block_exclusive_scan(mycnt, S.sh32, &tot);
+#pragma unroll
+        for (int i = 0; i < kSelKPT; ++i) {
+            if ((cmask >> i) & 1u) {
+                ck[pos] = kr[i];
+                ci[pos] = p0 + i * kSelThreads + tid;
+                ++pos;
+            }
+        }
+        ncand += tot;
+    }
+    if (lane == 0) S.amb_key[warp] = nin;  // (scratch) per-warp sure-in counts
+    __syncthreads();
+    if (tid == 0) {
+        uint32_t s_in = 0;
+        for (int w = 0; w < kSelThreads / 32; ++w) s_in += S.amb_key[w];
+        a.cand_cnt[(size_t)b * a.nchunks + c] = ncand;
+        a.in_cnt[(size_t)b * a.nchunks + c] = s_in;
+        __threadfence();  // publish this chunk's slot, counts and bitmap words before the ticket
+        const uint32_t prev = atomicAdd(&a.done[b], 1u);
+        S.last = prev == (uint32_t)(a.nchunks - 1);
     }
     __syncthreads();
+    if (!S.last) return;
+
+    // ---- resolve (the last CTA of sequence b); cross-CTA data is read through L2
+    if (tid == 0) {
+        __threadfence();
+        a.done[b] = 0;  // ready for the next call
+        S.amb_cnt = 0;
+        S.in2 = 0;
+    }
+    uint32_t C = 0, A = 0;
+    {
+        // chunk offsets (nchunks <= kSelMaxChunks)
+        constexpr int CPT = kSelMaxChunks / kSelThreads;
+        uint32_t cc[CPT], ic[CPT], sc = 0, si = 0;
+#pragma unroll
+        for (int u = 0; u < CPT; ++u) {
+            const int q = tid * CPT + u;
+            cc[u] = q < a.nchunks ? __ldcg(a.cand_cnt + (size_t)b * a.nchunks + q) : 0u;
+            ic[u] = q < a.nchunks ? __ldcg(a.in_cnt + (size_t)b * a.nchunks + q) : 0u;
+            sc += cc[u];
+            si += ic[u];
+        }
+        uint32_t off = block_exclusive_scan(sc, S.sh32, &C);
+        block_exclusive_scan(si, S.sh32, &A);
+#pragma unroll
+        for (int u = 0; u < CPT; ++u) {
+            S.coff[tid * CPT + u] = off;
+            off += cc[u];
+        }
+        if (tid == 0) S.coff[kSelMaxChunks] = C;
+    }
+    __syncthreads();
+    const uint32_t R1 = (uint32_t)k - A;  // rank of t~ among the candidates (>= 1)
+    if (C <= (uint32_t)kSelCap)
+        resolve_candidates<true>(a, S, csm, b, C, R1, d1, E);
+    else
+        resolve_candidates<false>(a, S, csm, b, C, R1, d1, E);
+    __syncthreads();
+    // candidates are consumed: csm now holds a shared bitmap of the winners
+    // (when it fits next to an output stage of k indices)
+    const int nwords = (n + 31) >> 5;
+    const bool sbm = S.wcnt > 0 && R1 <= (uint32_t)kBins &&
+                     (size_t)nwords + (size_t)k <= (size_t)kSelCap * 2;
+    const bool was_list = R1 <= (uint32_t)kBins;
+    uint32_t* extra = nullptr;
+    if (was_list) {
+        if (sbm) {
+            for (int w = tid; w < nwords; w += kSelThreads) csm[w] = 0u;
+            __syncthreads();
+            for (uint32_t i = tid; i < S.wcnt; i += kSelThreads) {
+                const uint32_t j = S.hist[i];
+                atomicOr(&csm[j >> 5], 1u << (j & 31));
+            }
+            extra = csm;
+        } else {
+            for (uint32_t i = tid; i < S.wcnt; i += kSelThreads) {
+                const uint32_t j = S.hist[i];
+                atomicOr(&bm[j >> 5], 1u << (j & 31));
+            }
+            __threadfence_block();
+        }
+        __syncthreads();
+    }
+    uint32_t* ostage = ((size_t)(extra ? nwords : 0) + (size_t)k <= (size_t)kSelCap * 2) ? csm + (extra ? nwords : 0)
+                                                                                          : nullptr;
     uint32_t total;
-    compact_bitmap(bm, (n + 31) >> 5, idx, (uint32_t)k, sh32, &total);
-    if (total != (uint32_t)k && threadIdx.x == 0) flag(DEV_LEN);  // cannot happen
-    if (threadIdx.x == 0) a.cnt[b] = k;
+    compact_bitmap(bm, extra, nwords, a.idx + (size_t)b * k, (uint32_t)k, ostage, S.coff, S.sh32, &total);
+    if (tid == 0) {
+        if (total != (uint32_t)k) flag(DEV_LEN);  // cannot happen
+        a.cnt[b] = k;
+    }
 }
 
 }  // namespace sa

@@ -23,8 +23,8 @@ constexpr int kPsQ = 64;         // queries per score tile
 constexpr int kPsE = 128;        // entries per score tile
 constexpr int kPsThreads = 256;  // 16 x 16 threads, 4 queries x 8 entries each
 constexpr int kPsSmem = 64 * kPsQ * 8 + 32 * kPsE * 4;  // fp64 queries + packed key pairs
-constexpr int kSelThreads = 1024;
-constexpr int kSelSmemKeys = 48 * 1024;  // keys held in shared memory (192 KB)
+constexpr int kPselThreads = 1024;
+constexpr int kPselSmemKeys = 48 * 1024;  // keys held in shared memory (192 KB)
 
 struct TopkPrefillArgs {
     const uint16_t* q_idx;  // [B][Tq][64]
@@ -139,16 +139,8 @@ __global__ void __launch_bounds__(kPsThreads, 2) score_prefill_kernel(TopkPrefil
     }
 }
 
-// Warp-aggregated shared-memory histogram increment (many equal bins).
-__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool valid) {
-    const uint32_t b = valid ? bin : 0xFFFFFFFFu;
-    const uint32_t peers = __match_any_sync(0xFFFFFFFFu, b);
-    const int leader = __ffs(peers) - 1;
-    if (valid && (int)(threadIdx.x & 31) == leader) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
-}
-
-__global__ void __launch_bounds__(kSelThreads, 1) select_prefill_kernel(TopkPrefillArgs a) {
-    extern __shared__ __align__(16) uint32_t skeys[];  // [kSelSmemKeys]
+__global__ void __launch_bounds__(kPselThreads, 1) select_prefill_kernel(TopkPrefillArgs a) {
+    extern __shared__ __align__(16) uint32_t skeys[];  // [kPselSmemKeys]
     __shared__ uint32_t hist[kBins];
     __shared__ uint32_t sh32[32];
     __shared__ int res[2];
@@ -164,7 +156,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_prefill_kernel(TopkPref
     }
     const uint32_t* grow = a.keys + (size_t)ql * a.KS;
     const uint32_t* kp = grow;
-    if (nv <= kSelSmemKeys) {
+    if (nv <= kPselSmemKeys) {
         const int n4 = (nv + 3) >> 2;  // rows are 16-byte aligned (KS multiple of 128)
         for (int i = threadIdx.x; i < n4; i += blockDim.x)
             reinterpret_cast<uint4*>(skeys)[i] = reinterpret_cast<const uint4*>(grow)[i];

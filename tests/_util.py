@@ -16,7 +16,8 @@ from sparse_attention_pool_b200 import synth
 SCALE = float(np.float32(1.0 / math.sqrt(128.0)))
 TOL_BF16 = 1e-2   # max-abs, bf16 cache, fp32 accumulation
 TOL_FP8 = 3e-2    # max-abs, e4m3 cache
-TOL_REL = 1e-2    # max|err| / rms(oracle output)
+TOL_REL = 1e-2    # rms(err) / rms(oracle output), bf16 cache
+TOL_REL_FP8 = 3e-2
 
 
 def bits_to_torch_bf16(a: np.ndarray) -> torch.Tensor:
@@ -69,8 +70,10 @@ def compress_on_gpu(S, g, B, Lcap, fp8=False, m_csa=4, m_hca=128):
 
 
 def out_errors(gpu_out: torch.Tensor, ref: np.ndarray):
+    """(max |err|, rms(err) / rms(ref))."""
     got = gpu_out.detach().float().cpu().numpy().astype(np.float64)
     err = np.abs(got - ref)
     rms = float(np.sqrt(np.mean(ref ** 2))) if ref.size else 0.0
     mx = float(err.max()) if err.size else 0.0
-    return mx, (mx / rms if rms > 0 else mx)
+    rerr = float(np.sqrt(np.mean(err ** 2))) if err.size else 0.0
+    return mx, (rerr / rms if rms > 0 else rerr)

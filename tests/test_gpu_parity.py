@@ -2,7 +2,7 @@
 
 Compressed caches and fp8 codes/scales: bit-exact.  Top-k indices and counts:
 bit-exact.  Attention outputs: max-abs error <= 1e-2 (bf16 cache) or 3e-2
-(fp8 cache), and max-abs error / rms(oracle) <= 1e-2 on top.  Sizes span
+(fp8 cache), and rms(err) / rms(oracle) <= 1e-2 (bf16) or 3e-2 (fp8) on top.  Sizes span
 several tiles and ragged tails; full-size workloads are checked on samples in
 test_gpu_fullsize.py.
 """
@@ -13,7 +13,7 @@ import pytest
 import torch
 
 from oracle import oracle as O
-from tests._util import (SCALE, TOL_BF16, TOL_FP8, TOL_REL, Inputs, bf16_to_f64, compress_on_gpu, out_errors,
+from tests._util import (SCALE, TOL_BF16, TOL_FP8, TOL_REL, TOL_REL_FP8, Inputs, bf16_to_f64, compress_on_gpu, out_errors,
                          torch_bf16_to_bits)
 
 pytestmark = pytest.mark.gpu
@@ -110,6 +110,34 @@ def test_decode_topk_ties_lowest_index(S):
     assert np.array_equal(idx[0], ridx) and cnt[0] == rcnt
 
 
+def test_decode_topk_near_ties_need_exact_rescoring(S):
+    # clusters of entries whose scores differ by far less than the fp32 screen
+    # can resolve (and often tie exactly after the final fp32 rounding)
+    B, Lcap, k = 1, 16384, 100
+    inp = Inputs(304, B, Lcap, 8)
+    q = bf16_to_f64(inp.qI[0])
+    sign = np.where(q >= 0, 1.0, -1.0)
+    rows = []
+    for base, count in ((1.0, 80), (0.984375, 70)):   # two clusters at the top
+        for v in range(count):
+            r = sign * base
+            r[63] = 0.0
+            if v % 3:
+                r[63] = sign[63] * 2.0 ** -(18 + v % 7)    # exact bf16, below the screen's resolution
+            rows.append(r)
+    rows = np.array(rows, dtype=np.float32)
+    rb = torch.tensor(rows).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    ents = np.random.default_rng(5).choice(Lcap // 4, size=len(rows), replace=False)
+    for e, r in zip(ents, rb):
+        inp.KI[0, 4 * e:4 * e + 4] = r                   # constant block -> the entry is exactly r
+    _, _, _, idx, cnt = _topk_case(S, inp, k)
+    cs = inp.oracle_seq(0)
+    s = O.index_scores(inp.qI[0], cs.cidx)
+    ridx, rcnt = O.topk(s, k)
+    assert len(set(s[ents].tolist())) < len(ents)       # exact ties exist among the clusters
+    assert np.array_equal(idx[0], ridx) and cnt[0] == rcnt
+
+
 def test_decode_topk_all_equal_scores(S):
     B, Lcap, k = 2, 4000, 77
     inp = Inputs(302, B, Lcap, 8)
@@ -132,7 +160,7 @@ def test_decode_topk_short_and_empty(S):
 def _check_outputs(got, ref, tol):
     mx, rel = out_errors(got, ref)
     assert mx <= tol, (mx, rel)
-    assert rel <= TOL_REL, (mx, rel)
+    assert rel <= (TOL_REL if tol == TOL_BF16 else TOL_REL_FP8), (mx, rel)
 
 
 @pytest.mark.parametrize("fp8", [False, True])
@@ -193,14 +221,12 @@ def test_decode_deterministic_and_batch_invariant(S):
         assert torch.equal(x.view(torch.int16), y.view(torch.int16))
     # sequence 2 alone, with the same cache capacity
     b = 2
-    solo = Inputs(502, B, Lcap, H, lengths=[16000, 15001, 9000, 16000])
-    g1 = {kk: (v[b:b + 1].contiguous()) for kk, v in g.items()}
+    g1 = {kk: v[b:b + 1].clone() for kk, v in g.items()}
     csa1, hca1 = compress_on_gpu(S, g1, 1, Lcap)
     ws1 = S.alloc_workspace(S.workspace_size(S.SA_OP_HYBRID_DECODE, 1, 1, H, csa1.Ncap, hca1.Ncap, k))
     s1 = S.hybrid_attn_decode(g1["q"], g1["qI"], csa1, hca1, k, ws1, scale=SCALE)
     assert torch.equal(s1[0][0].view(torch.int16), a1[0][b].view(torch.int16))
     assert torch.equal(s1[1][0].view(torch.int16), a1[1][b].view(torch.int16))
-    del solo
 
 
 def test_csa_with_k_covering_all_equals_dense(S):
