@@ -16,6 +16,8 @@
 // its lse, merged by attn_combine_kernel in a fixed order (deterministic and
 // independent of the batch: the split size depends only on the entry count).
 #pragma once
+#include <cooperative_groups.h>
+
 #include "sa_common.cuh"
 
 namespace sa {
@@ -75,13 +77,20 @@ struct AttnSmem {
     static constexpr int kTotal = kMeta + ST * kTileN * 4 * 3;
 };
 
+constexpr int kAttnCluster = 8;  // splits of one query merged in shared memory (CLUSTER variant)
+
 // ST = pipeline stages: ST - 1 tiles are in flight while one is computed.
-template <int NW, bool GATHER, bool FP8, int ST>
+// CLUSTER: the grid's x dimension is one cluster of kAttnCluster CTAs (the
+// splits of one query); they merge their partials through distributed shared
+// memory instead of a separate combine pass.
+template <int NW, bool GATHER, bool FP8, int ST, bool CLUSTER>
 __global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
     using L = AttnSmem<NW, GATHER, FP8, ST>;
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int split = blockIdx.x, bq = blockIdx.y;
+    // grid: (splits, queries) in a cluster launch, else (queries, splits)
+    const int split = CLUSTER ? blockIdx.x : blockIdx.y;
+    const int bq = CLUSTER ? blockIdx.y : blockIdx.x;
     const int b = bq / a.Tq;
     int nb = a.n[b];
     if (nb < 0 || nb > a.Ncap) {
@@ -334,6 +343,57 @@ __global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
         lse_r[h] = empty ? -INFINITY : (mrow[h] + __log2f(lrow[h])) * kLn2;
     }
     const int hr[2] = {warp * 16 + (lane >> 2), warp * 16 + (lane >> 2) + 8};
+    if (CLUSTER) {
+        // partials into this CTA's shared memory (Q and the K/V buffers are free now)
+        static_assert(L::kMeta >= NW * 16 * 129 * 4, "partial buffer");
+        namespace cg = cooperative_groups;
+        cg::cluster_group cluster = cg::this_cluster();
+        __syncthreads();
+        float* po = reinterpret_cast<float*>(smem);  // [NW*16][128]
+        float* pl = po + NW * 16 * 128;                          // [NW*16]
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int d = i * 8 + (lane & 3) * 2;
+                *reinterpret_cast<float2*>(po + hr[h] * 128 + d) = make_float2(o[i][2 * h] * inv[h], o[i][2 * h + 1] * inv[h]);
+            }
+            if ((lane & 3) == 0) pl[hr[h]] = lse_r[h];
+        }
+        cluster.sync();
+        // CTA r merges heads r, r + 8, ...: one warp per head, 4 dims per lane
+        const int r = (int)cluster.block_rank();
+        for (int h = r + kAttnCluster * warp; h < a.H; h += kAttnCluster * NW) {
+            float ls[kAttnCluster];
+            float M = -INFINITY;
+#pragma unroll
+            for (int q = 0; q < kAttnCluster; ++q) {
+                ls[q] = cluster.map_shared_rank(pl, q)[h];
+                M = fmaxf(M, ls[q]);
+            }
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            float ws = 0.f;
+            if (M != -INFINITY) {
+#pragma unroll
+                for (int q = 0; q < kAttnCluster; ++q) {
+                    const float w = ls[q] == -INFINITY ? 0.f : __expf(ls[q] - M);
+                    const float4 v = *reinterpret_cast<const float4*>(cluster.map_shared_rank(po, q) + h * 128 + lane * 4);
+                    acc.x += w * v.x;
+                    acc.y += w * v.y;
+                    acc.z += w * v.z;
+                    acc.w += w * v.w;
+                    ws += w;
+                }
+            }
+            const float iw = ws > 0.f ? 1.f / ws : 0.f;
+            uint16_t* op = a.out + ((size_t)bq * a.H + h) * 128 + lane * 4;
+            *reinterpret_cast<uint2*>(op) =
+                make_uint2(pack_bf16x2(acc.x * iw, acc.y * iw), pack_bf16x2(acc.z * iw, acc.w * iw));
+            if (a.lse && lane == 0) a.lse[(size_t)bq * a.H + h] = ws > 0.f ? M + __logf(ws) : -INFINITY;
+        }
+        cluster.sync();  // no CTA leaves while others read its shared memory
+        return;
+    }
     if (a.splits == 1) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {

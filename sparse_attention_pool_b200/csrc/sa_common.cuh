@@ -170,6 +170,20 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// Shared-memory atomics through explicit shared-space addresses (a generic
+// pointer into shared memory would otherwise compile to a generic atomic).
+__device__ __forceinline__ uint32_t atom_add_shared(uint32_t* p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.shared.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(smem_u32(p)), "r"(v) : "memory");
+    return old;
+}
+__device__ __forceinline__ void red_add_shared(uint32_t* p, uint32_t v) {
+    asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_or_shared(uint32_t* p, uint32_t v) {
+    asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+
 // ------------------------------------------------------------ block scans --
 // Exclusive prefix sum over the block (blockDim.x multiple of 32, <= 1024).
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* sh32, uint32_t* total) {

@@ -140,7 +140,7 @@ sa_status make_ic_map(CUtensorMap* map, const void* kidx, int B, int Ncap) {
 
 // ------------------------------------------------------- workspace layout --
 struct TopkDecodeWs {
-    size_t hist, done, keys, emax, cand_key, cand_idx, amb_key, amb_idx, cand_cnt, in_cnt, bitmap, idx, cnt, total;
+    size_t hist, totals, keys, emax, cand_key, cand_idx, amb_key, amb_idx, bitmap, idx, cnt, total;
     int maxchunks, Wcap;
 };
 
@@ -152,17 +152,17 @@ int score_chunk(int B, int Ncap) {
     return (int)std::max<long long>(chunk, sa::kScRows);
 }
 
-// [reserved 256 B][histograms][keys][per-chunk max error][candidate slots key/idx]
-// [band key/idx][per-chunk counts][bitmap][idx][cnt]
+// [reserved 256 B][histograms][totals][keys][per-chunk max error][candidates key/idx]
+// [band key/idx][bitmap][idx][cnt]
 TopkDecodeWs topk_decode_layout(int B, int Ncap, int k, bool own_idx) {
     TopkDecodeWs w{};
     w.maxchunks = std::max(1, cdiv(Ncap, sa::kScRows));
     w.Wcap = ((Ncap + 31) / 32 + 1) & ~1;
     size_t o = 256;
-    w.hist = o;  // histograms and tickets are zeroed together before every call
+    w.hist = o;  // histograms and totals are zeroed together before every call
     o += (size_t)B * sa::kBins * 4;
-    w.done = o;
-    o += up256((size_t)B * 4);
+    w.totals = o;
+    o += up256((size_t)B * 16);
     const size_t col = up256((size_t)B * Ncap * 4);
     w.keys = o;
     o += col;
@@ -176,10 +176,6 @@ TopkDecodeWs topk_decode_layout(int B, int Ncap, int k, bool own_idx) {
     o += col;
     w.amb_idx = o;
     o += col;
-    w.cand_cnt = o;
-    o += up256((size_t)B * w.maxchunks * 4);
-    w.in_cnt = o;
-    o += up256((size_t)B * w.maxchunks * 4);
     w.bitmap = o;
     o += up256((size_t)B * w.Wcap * 4);
     w.idx = o;
@@ -195,9 +191,10 @@ TopkDecodeWs topk_decode_layout(int B, int Ncap, int k, bool own_idx) {
 struct Split {
     int tps, splits;
 };
-Split attn_split(int rows_cap, bool prefill) {
+Split attn_split(int rows_cap, bool prefill, bool gather = false) {
     const int tiles = cdiv(rows_cap > 0 ? rows_cap : 1, sa::kTileN);
     if (prefill) return {tiles, 1};
+    (void)gather;  // both lists split the same way: at most 32 splits
     const int tps = cdiv(tiles, 32);
     return {tps, cdiv(tiles, tps)};
 }
@@ -208,34 +205,57 @@ size_t attn_partial_bytes(long long BQ, int splits, int H) {
 }
 
 // ------------------------------------------------------------ launchers ----
-template <int NW, bool G, bool F, int ST>
+template <int NW, bool G, bool F, int ST, bool CL>
 sa_status launch_attn_t(const sa::AttnArgs& a, dim3 grid, cudaStream_t st) {
     using L = sa::AttnSmem<NW, G, F, ST>;
     static bool init = false;
     if (!init) {
-        SA_CUDA(cudaFuncSetAttribute(sa::attn_split_kernel<NW, G, F, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     L::kTotal));
+        SA_CUDA(cudaFuncSetAttribute(sa::attn_split_kernel<NW, G, F, ST, CL>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal));
         init = true;
     }
-    sa::attn_split_kernel<NW, G, F, ST><<<grid, NW * 32, L::kTotal, st>>>(a);
+    if (CL) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = grid;
+        cfg.blockDim = dim3(NW * 32);
+        cfg.dynamicSmemBytes = L::kTotal;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = sa::kAttnCluster;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        SA_CUDA(cudaLaunchKernelEx(&cfg, sa::attn_split_kernel<NW, G, F, ST, CL>, a));
+    } else {
+        sa::attn_split_kernel<NW, G, F, ST, CL><<<grid, NW * 32, L::kTotal, st>>>(a);
+    }
     SA_LAUNCHED();
     return SA_OK;
 }
 
-template <int NW, int ST>
+template <int NW, int ST, bool CL>
 sa_status launch_attn_nw(const sa::AttnArgs& a, bool gather, bool fp8, dim3 grid, cudaStream_t st) {
-    if (gather) return fp8 ? launch_attn_t<NW, true, true, ST>(a, grid, st) : launch_attn_t<NW, true, false, ST>(a, grid, st);
-    return fp8 ? launch_attn_t<NW, false, true, ST>(a, grid, st) : launch_attn_t<NW, false, false, ST>(a, grid, st);
+    if (gather)
+        return fp8 ? launch_attn_t<NW, true, true, ST, CL>(a, grid, st) : launch_attn_t<NW, true, false, ST, CL>(a, grid, st);
+    return fp8 ? launch_attn_t<NW, false, true, ST, CL>(a, grid, st) : launch_attn_t<NW, false, false, ST, CL>(a, grid, st);
 }
 
 // Splits of up to 4 tiles keep all of them in flight (4 stages); longer
-// lists (prefill) stream through a 2-stage pipeline.
+// lists (prefill) stream through a 2-stage pipeline.  A query split exactly
+// kAttnCluster ways merges inside a cluster.
 sa_status launch_attn(const sa::AttnArgs& a, bool gather, bool fp8, long long BQ, cudaStream_t st) {
-    if (BQ > 2147483647LL) return fail(SA_ERR_INVALID_ARG, "too many queries");
-    dim3 grid(a.splits, (unsigned)BQ);
+    const bool cl = a.splits == sa::kAttnCluster && BQ <= 65535;
+    if (BQ > 2147483647LL || a.splits > 65535) return fail(SA_ERR_INVALID_ARG, "too many queries or splits");
+    const dim3 grid = cl ? dim3(a.splits, (unsigned)BQ) : dim3((unsigned)BQ, a.splits);
     const bool deep = a.tiles_per_split >= 2 && a.tiles_per_split <= 4;
-    if (a.H <= 64) return deep ? launch_attn_nw<4, 4>(a, gather, fp8, grid, st) : launch_attn_nw<4, 2>(a, gather, fp8, grid, st);
-    return deep ? launch_attn_nw<8, 4>(a, gather, fp8, grid, st) : launch_attn_nw<8, 2>(a, gather, fp8, grid, st);
+    if (a.H <= 64) {
+        if (cl) return deep ? launch_attn_nw<4, 4, true>(a, gather, fp8, grid, st) : launch_attn_nw<4, 2, true>(a, gather, fp8, grid, st);
+        return deep ? launch_attn_nw<4, 4, false>(a, gather, fp8, grid, st) : launch_attn_nw<4, 2, false>(a, gather, fp8, grid, st);
+    }
+    if (cl) return deep ? launch_attn_nw<8, 4, true>(a, gather, fp8, grid, st) : launch_attn_nw<8, 2, true>(a, gather, fp8, grid, st);
+    return deep ? launch_attn_nw<8, 4, false>(a, gather, fp8, grid, st) : launch_attn_nw<8, 2, false>(a, gather, fp8, grid, st);
 }
 
 sa_status launch_combine(const float* po, const float* pl, int splits, int H, long long BQ, uint16_t* out, float* lse,
@@ -275,7 +295,7 @@ sa_status run_attn(const void* q, int Tq, int H, const sa_cache* c, bool gather,
                    size_t ws_off, cudaStream_t st) {
     const long long BQ = (long long)c->B * Tq;
     const bool prefill = (Tq > 1) || (pos != nullptr);
-    const Split sp = attn_split(gather ? kmax : c->Ncap, prefill);
+    const Split sp = attn_split(gather ? kmax : c->Ncap, prefill, gather);
     sa::AttnArgs a{};
     a.q = static_cast<const uint16_t*>(q);
     a.K = c->k;
@@ -305,7 +325,9 @@ sa_status run_attn(const void* q, int Tq, int H, const sa_cache* c, bool gather,
     }
     sa_status r = launch_attn(a, gather, c->dtype == SA_FP8_E4M3, BQ, st);
     if (r != SA_OK) return r;
-    if (sp.splits > 1) return launch_combine(a.part_o, a.part_lse, sp.splits, H, BQ, a.out, lse, st);
+    // a query split kAttnCluster ways was merged inside its cluster
+    if (sp.splits > 1 && !(sp.splits == sa::kAttnCluster && BQ <= 65535))
+        return launch_combine(a.part_o, a.part_lse, sp.splits, H, BQ, a.out, lse, st);
     return SA_OK;
 }
 
@@ -328,10 +350,8 @@ sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* 
     a.cand_idx = reinterpret_cast<int32_t*>(base + w.cand_idx);
     a.amb_key = reinterpret_cast<uint32_t*>(base + w.amb_key);
     a.amb_idx = reinterpret_cast<int32_t*>(base + w.amb_idx);
-    a.cand_cnt = reinterpret_cast<uint32_t*>(base + w.cand_cnt);
-    a.in_cnt = reinterpret_cast<uint32_t*>(base + w.in_cnt);
+    a.totals = reinterpret_cast<uint32_t*>(base + w.totals);
     a.bitmap = reinterpret_cast<uint32_t*>(base + w.bitmap);
-    a.done = reinterpret_cast<uint32_t*>(base + w.done);
     a.idx = idx;
     a.cnt = cnt;
     a.Ncap = Ncap;
@@ -345,7 +365,7 @@ sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* 
     const size_t smem = sa::kScStages * sa::kScTileBytes + sa::kScStages * 8 + 1024;
     if (!init) {
         SA_CUDA(cudaFuncSetAttribute(sa::score_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-        SA_CUDA(cudaFuncSetAttribute(sa::topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        SA_CUDA(cudaFuncSetAttribute(sa::topk_resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      sa::kSelSmem));
         init = true;
     }
@@ -354,7 +374,7 @@ sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* 
         sa_status r = make_ic_map(&map, c->kidx, B, Ncap);
         if (r != SA_OK) return r;
         stage_mark(SA_STAGE_INDEX_SCORE, 0, st);
-        SA_CUDA(cudaMemsetAsync(a.hist1, 0, w.done - w.hist + (size_t)B * 4, st));
+        SA_CUDA(cudaMemsetAsync(a.hist1, 0, w.totals - w.hist + (size_t)B * 16, st));
         sa::score_decode_kernel<<<dim3(a.nchunks, B), sa::kScThreads, smem, st>>>(map, a);
         SA_LAUNCHED();
         stage_mark(SA_STAGE_INDEX_SCORE, 1, st);
@@ -362,7 +382,11 @@ sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* 
     sa_status r = between();
     if (r != SA_OK) return r;
     stage_mark(SA_STAGE_TOPK_SELECT, 0, st);
-    sa::topk_select_kernel<<<dim3(a.nchunks, B), sa::kSelThreads, sa::kSelSmem, st>>>(a);
+    if (Ncap > 0) {
+        sa::topk_filter_kernel<<<dim3(a.nchunks, B), sa::kSelThreads, 0, st>>>(a);
+        SA_LAUNCHED();
+    }
+    sa::topk_resolve_kernel<<<B, sa::kResThreads, sa::kSelSmem, st>>>(a);
     SA_LAUNCHED();
     stage_mark(SA_STAGE_TOPK_SELECT, 1, st);
     return SA_OK;
@@ -522,7 +546,7 @@ size_t sa_workspace_size(int32_t op, int32_t B, int32_t Tq, int32_t H, int32_t N
             return topk_decode_layout(B, Ncap_csa, k, false).total;
         case SA_OP_SPARSE_ATTN: {
             if (k < 1) return 0;
-            Split s = attn_split(k, prefill);
+            Split s = attn_split(k, prefill, true);
             return 256 + attn_partial_bytes(BQ, s.splits, H);
         }
         case SA_OP_DENSE_ATTN: {
@@ -532,7 +556,7 @@ size_t sa_workspace_size(int32_t op, int32_t B, int32_t Tq, int32_t H, int32_t N
         case SA_OP_HYBRID_DECODE: {
             if (k < 1 || Tq != 1) return 0;
             TopkDecodeWs w = topk_decode_layout(B, Ncap_csa, k, true);
-            Split sc = attn_split(k, false), sh = attn_split(Ncap_hca, false);
+            Split sc = attn_split(k, false, true), sh = attn_split(Ncap_hca, false);
             return w.total + attn_partial_bytes(BQ, sc.splits, H) + attn_partial_bytes(BQ, sh.splits, H);
         }
         case SA_OP_HYBRID_PREFILL:
@@ -646,7 +670,7 @@ sa_status hybrid_attn_decode(const void* q, const void* q_idx, int32_t H, const 
     uint8_t* base = static_cast<uint8_t*>(ws);
     int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + w.idx);
     int32_t* cnt = cnt_out ? cnt_out : reinterpret_cast<int32_t*>(base + w.cnt);
-    const Split sc = attn_split(k, false);
+    const Split sc = attn_split(k, false, true);
     // HCA needs neither the indexer nor the top-k: once the indexer stream is
     // queued, fork it onto the side stream so that it overlaps the selection
     // and the CSA attention instead of competing with the indexer stream.

@@ -19,16 +19,17 @@
 //            with s~ < t~ - 2E surely not, and only the band |s~ - t~| <= 2E
 //            is rescored exactly (the fp64 definition) and ranked exactly.
 //
-// Two kernels, ordered on one stream:
+// Three kernels, ordered on one stream (every hand-off is a kernel boundary;
+// no CTA waits on another):
 //   1. score_decode_kernel -- streams Ic through a 4-stage TMA pipeline
 //      (128-byte rows, 128B swizzle, one row per thread) and writes an order
 //      key of s~ per entry, a histogram of the top 11 key bits (per CTA in
 //      shared memory, then added to the sequence's) and each CTA's max e_j.
-//   2. topk_select_kernel  -- one CTA per score chunk: from the histogram the
+//   2. topk_filter_kernel  -- one CTA per score chunk: from the histogram the
 //      bin of t~; entries above that bin widened by 2E become bitmap bits
 //      (surely selected), entries in the widened bin become candidates in the
-//      chunk's own slot.  The last CTA of a sequence to finish (it takes a
-//      ticket after a fence; no CTA ever waits on another) gathers the
+//      chunk's own slot.  Plain stores.
+//   3. topk_resolve_kernel -- one 1024-thread CTA per sequence: gathers the
 //      candidates, finds t~ among them, rescores the band exactly, ranks it
 //      by (s, -j), marks the winners and compacts the bitmap into ascending
 //      indices.
@@ -51,12 +52,10 @@ struct TopkDecodeArgs {
     uint32_t* keys;         // [B][Ncap]     order keys of the screened scores
     uint32_t* hist1;        // [B][2048]     histogram of the top 11 key bits (zeroed per call)
     float* emax_part;       // [B][nchunks]  per score CTA: max e_j
-    uint32_t* cand_key;     // [B][Ncap]     candidates, each chunk in its own slot
+    uint32_t* cand_key;     // [B][Ncap]     candidates of the sequence (filter order)
     int32_t* cand_idx;      // [B][Ncap]
-    uint32_t* cand_cnt;     // [B][nchunks]  candidates per chunk
-    uint32_t* in_cnt;       // [B][nchunks]  surely selected entries per chunk
+    uint32_t* totals;       // [B][4]        candidates, sure-ins, bin d1, E bits (zeroed per call)
     uint32_t* bitmap;       // [B][Wcap]     selection bitmap
-    uint32_t* done;         // [B]           chunks filtered so far (zero between calls)
     uint32_t* amb_key;      // [B][Ncap]     exact keys of the band, when it is large
     int32_t* amb_idx;       // [B][Ncap]
     int32_t* idx;           // [B][k]
@@ -79,22 +78,34 @@ __device__ __forceinline__ float key_to_float(uint32_t key) {
 
 // The exact score of one indexer row (the definition): fp64 FMA chain in
 // ascending i over exact products, rounded once to fp32, -0 -> +0, as a key.
-__device__ __noinline__ uint32_t exact_key(const uint16_t* qI, const uint16_t* row) {
+// q2 holds qI[i] * 2^768 in fp64 (see below); the row's bf16 values enter as
+// x * 2^-896 through bit placement, so each product is qI*k * 2^-128 exactly
+// and no conversion instruction is needed per element.
+__device__ __noinline__ uint32_t exact_key(const double* q2, const uint16_t* row) {
     const uint4* r4 = reinterpret_cast<const uint4*>(row);
-    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qI);
     double acc = 0.0;
-#pragma unroll
+#pragma unroll 2
     for (int c = 0; c < 8; ++c) {
         const uint4 w = __ldg(r4 + c);
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            const uint32_t qw = __ldg(q32 + c * 4 + h);
-            acc = fma((double)bf16lo_f32(qw), (double)bf16lo_f32(ws[h]), acc);
-            acc = fma((double)bf16hi_f32(qw), (double)bf16hi_f32(ws[h]), acc);
-        }
+        acc = fma(q2[8 * c + 0], bf16lo_scaled(w.x), acc);
+        acc = fma(q2[8 * c + 1], bf16hi_scaled(w.x), acc);
+        acc = fma(q2[8 * c + 2], bf16lo_scaled(w.y), acc);
+        acc = fma(q2[8 * c + 3], bf16hi_scaled(w.y), acc);
+        acc = fma(q2[8 * c + 4], bf16lo_scaled(w.z), acc);
+        acc = fma(q2[8 * c + 5], bf16hi_scaled(w.z), acc);
+        acc = fma(q2[8 * c + 6], bf16lo_scaled(w.w), acc);
+        acc = fma(q2[8 * c + 7], bf16hi_scaled(w.w), acc);
     }
-    return score_key(__double2float_rn(acc));
+    return score_key(__double2float_rn(acc * 0x1p128));
+}
+
+// qI * 2^768 in fp64 into shared memory (64 values), for exact_key.
+__device__ __forceinline__ void load_q2(double* q2, const uint16_t* qI) {
+    if (threadIdx.x < 32) {
+        const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(qI) + threadIdx.x);
+        q2[2 * threadIdx.x] = (double)bf16lo_f32(w) * 0x1p768;
+        q2[2 * threadIdx.x + 1] = (double)bf16hi_f32(w) * 0x1p768;
+    }
 }
 
 // ------------------------------------------------------------ 1. scores ----
@@ -221,6 +232,7 @@ __device__ __forceinline__ void find_digit_desc(const uint32_t* h, uint32_t K, u
     const int u = T - 1 - threadIdx.x;  // thread t handles the bins of thread u, so the scan runs high -> low
     const int lo = u * per, hi = min(NB, lo + per);
     uint32_t local = 0;
+#pragma unroll 1
     for (int e = lo; e < hi; ++e) local += h[e];
     uint32_t above = block_exclusive_scan(local, sh32, nullptr);
     if (threadIdx.x == 0) {
@@ -228,6 +240,7 @@ __device__ __forceinline__ void find_digit_desc(const uint32_t* h, uint32_t K, u
         res[1] = 0;
     }
     __syncthreads();
+#pragma unroll 1
     for (int e = hi - 1; e >= lo; --e) {
         const uint32_t c = h[e];
         if (above < K && K <= above + c) {
@@ -276,7 +289,7 @@ __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool vali
     const uint32_t b = valid ? bin : 0xFFFFFFFFu;
     const uint32_t peers = __match_any_sync(0xFFFFFFFFu, b);
     const int leader = __ffs(peers) - 1;
-    if (valid && (int)(threadIdx.x & 31) == leader) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+    if (valid && (int)(threadIdx.x & 31) == leader) red_add_shared(&hist[bin], (uint32_t)__popc(peers));
 }
 
 // Among list entries (key[i], idx[i]), i < cnt, find the R-th largest by
@@ -348,9 +361,10 @@ __device__ __forceinline__ void select_rank(const uint32_t* key, const int32_t* 
 // (bits 20..10 and 9..0), whose bins are well spread, with plain shared
 // atomics.  Returns false if the rank falls outside the bin (caller then
 // uses the general select_rank).
-__device__ __forceinline__ bool rank_in_bin(const uint32_t* key, uint32_t cnt, uint32_t R, int d1, uint32_t* hist,
-                                            uint32_t* sh32, int* res, uint32_t* T_out) {
+__device__ __noinline__ bool rank_in_bin(const uint32_t* key, uint32_t cnt, uint32_t R, int d1, uint32_t* hist,
+                                         uint32_t* sh32, int* res, uint32_t* T_out) {
     uint32_t above = 0, inbin = 0;
+#pragma unroll 1
     for (uint32_t i = threadIdx.x; i < cnt; i += blockDim.x) {
         const int dig = (int)(key[i] >> 21);
         above += dig > d1;
@@ -363,9 +377,10 @@ __device__ __forceinline__ bool rank_in_bin(const uint32_t* key, uint32_t cnt, u
     uint32_t rem = R - tot_above;
     for (int i = threadIdx.x; i < kBins; i += blockDim.x) hist[i] = 0;
     __syncthreads();
+#pragma unroll 1
     for (uint32_t i = threadIdx.x; i < cnt; i += blockDim.x) {
         const uint32_t kk = key[i];
-        if ((int)(kk >> 21) == d1) atomicAdd(&hist[(kk >> 10) & (kBins - 1)], 1u);
+        if ((int)(kk >> 21) == d1) red_add_shared(&hist[(kk >> 10) & (kBins - 1)], 1u);
     }
     __syncthreads();
     int d2, d3;
@@ -375,9 +390,10 @@ __device__ __forceinline__ bool rank_in_bin(const uint32_t* key, uint32_t cnt, u
     const uint32_t pre = ((uint32_t)d1 << 11) | (uint32_t)d2;
     for (int i = threadIdx.x; i < kBinsLow; i += blockDim.x) hist[i] = 0;
     __syncthreads();
+#pragma unroll 1
     for (uint32_t i = threadIdx.x; i < cnt; i += blockDim.x) {
         const uint32_t kk = key[i];
-        if ((kk >> 10) == pre) atomicAdd(&hist[kk & (kBinsLow - 1)], 1u);
+        if ((kk >> 10) == pre) red_add_shared(&hist[kk & (kBinsLow - 1)], 1u);
     }
     __syncthreads();
     find_digit_desc<kBinsLow>(hist, rem, sh32, &d3, &ab, res);
@@ -387,9 +403,10 @@ __device__ __forceinline__ bool rank_in_bin(const uint32_t* key, uint32_t cnt, u
 }
 
 // --------------------------------------------------------- 2. selection ----
-constexpr int kSelThreads = 256;
+constexpr int kSelThreads = 256;             // filter CTAs
+constexpr int kResThreads = 1024;            // resolve CTA (one per sequence)
 constexpr int kSelKPT = 16;                  // keys per thread held in registers per pass
-constexpr int kSelCap = 6144;                // candidates the resolving CTA holds in shared memory
+constexpr int kSelCap = 8192;                // candidates the resolving CTA holds in shared memory
 constexpr int kSelSmem = kSelCap * 8;
 constexpr int kSelMaxChunks = 1024;
 
@@ -409,131 +426,102 @@ __device__ __forceinline__ FilterBounds filter_bounds(int d1, float E) {
 }
 
 // Writes the set bits of (bm | extra)[0..nwords) as ascending indices into
-// out[0..cap); `extra` is an optional bitmap in shared memory.  Per round of
-// 16 * blockDim words, word w0 + i*T + t goes to thread t (coalesced loads,
-// all issued first); prefixes come from one warp scan per i and a single
-// block scan over the (i, warp) totals, taken in word order.  With `ostage`
-// (shared, >= cap words) the indices are staged and leave in coalesced
-// stores; scattered 4-byte global stores from one SM are slow.
-// `wt` is shared scratch of 16 * blockDim / 32 words.
-__device__ __forceinline__ void compact_bitmap(const uint32_t* bm, const uint32_t* extra, int nwords, int32_t* out,
-                                               uint32_t cap, uint32_t* ostage, uint32_t* wt, uint32_t* sh32,
-                                               uint32_t* total_out) {
-    constexpr int P = 16;
-    const int T = blockDim.x, W = T >> 5;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+// out[0..cap); `extra` is an optional bitmap in shared memory.  Written for a
+// CTA that runs this code once: rolled loops keep the code small (a cold
+// instruction cache costs more here than loop overhead).  Words are staged in
+// shared memory (`stage`, blockDim*(PER+1) words) so that global reads are
+// coalesced and each thread then owns PER consecutive words; with `ostage`
+// (shared, >= cap words) the indices leave in coalesced stores too.
+constexpr int kCompPer = 4;  // words per thread per round; staging = blockDim * (kCompPer + 1) words
+__device__ __noinline__ void compact_bitmap(const uint32_t* bm, const uint32_t* extra, int nwords, int32_t* out,
+                                            uint32_t cap, uint32_t* ostage, uint32_t* stage, uint32_t* sh32,
+                                            uint32_t* total_out) {
+    const int T = blockDim.x;
+    const int span = T * kCompPer;
     uint32_t running = 0;
-    for (int w0 = 0; w0 < nwords; w0 += T * P) {
-        uint32_t v[P], incl[P];
-#pragma unroll
-        for (int i = 0; i < P; ++i) {
-            const int w = w0 + i * T + threadIdx.x;
-            v[i] = w < nwords ? __ldcg(bm + w) : 0u;
-        }
-        if (extra) {
-#pragma unroll
-            for (int i = 0; i < P; ++i) {
-                const int w = w0 + i * T + threadIdx.x;
-                if (w < nwords) v[i] |= extra[w];
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < P; ++i) {
-            uint32_t x = __popc(v[i]);
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
-                if (lane >= o) x += y;
-            }
-            incl[i] = x;
-            if (lane == 31) wt[i * W + warp] = x;
+#pragma unroll 1
+    for (int w0 = 0; w0 < nwords; w0 += span) {
+        __syncthreads();  // stage is reused
+#pragma unroll 4
+        for (int i = threadIdx.x; i < span; i += T) {
+            const int w = w0 + i;
+            uint32_t v = w < nwords ? __ldcg(bm + w) : 0u;
+            if (extra && w < nwords) v |= extra[w];
+            stage[(i / kCompPer) * (kCompPer + 1) + (i % kCompPer)] = v;
         }
         __syncthreads();
+        const uint32_t* mine = stage + threadIdx.x * (kCompPer + 1);
+        uint32_t c = 0;
+#pragma unroll 1
+        for (int u = 0; u < kCompPer; ++u) c += __popc(mine[u]);
         uint32_t tot;
-        const uint32_t mine = threadIdx.x < P * W ? wt[threadIdx.x] : 0u;  // (i, warp) in word order
-        const uint32_t ex = block_exclusive_scan(mine, sh32, &tot);
-        if (threadIdx.x < P * W) wt[threadIdx.x] = ex;
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < P; ++i) {
-            uint32_t word = v[i];
-            uint32_t pos = running + wt[i * W + warp] + incl[i] - __popc(word);
-            const int wbase = (w0 + i * T + threadIdx.x) * 32;
+        uint32_t pos = running + block_exclusive_scan(c, sh32, &tot);
+        const int wb = w0 + threadIdx.x * kCompPer;
+#pragma unroll 1
+        for (int u = 0; u < kCompPer; ++u) {
+            uint32_t word = mine[u];
             while (word) {
                 const int bit = __ffs(word) - 1;
                 word &= word - 1;
                 if (pos < cap) {
-                    if (ostage) ostage[pos] = (uint32_t)(wbase + bit);
-                    else out[pos] = wbase + bit;
+                    if (ostage) ostage[pos] = (uint32_t)((wb + u) * 32 + bit);
+                    else out[pos] = (wb + u) * 32 + bit;
                 }
                 ++pos;
             }
         }
         running += tot;
-        __syncthreads();  // wt is reused
     }
+    __syncthreads();
     if (ostage) {
         const uint32_t nout = running < cap ? running : cap;
+#pragma unroll 1
         for (uint32_t i = threadIdx.x; i < nout; i += T) out[i] = (int32_t)ostage[i];
     }
     *total_out = running;
 }
 
 struct SelSmem {
+    double q2[64];            // qI * 2^768 for the exact rescoring
     uint32_t hist[kBins];
-    uint32_t coff[kSelMaxChunks + 1];
     uint32_t sh32[32];
     int res[2];
     float red[kSelThreads / 32];
     uint32_t last, amb_cnt, in2, wcnt, T2;
     int32_t jmax2;
-    uint32_t amb_key[kSelThreads];
-    int32_t amb_idx[kSelThreads];
+    uint32_t amb_key[kResThreads];
+    int32_t amb_idx[kResThreads];
 };
 
 // The resolve step of topk_select_kernel over the C gathered candidates, with
 // the candidate list in shared memory (SMEM) or in global memory.
-template <bool SMEM>
-__device__ __forceinline__ void resolve_candidates(const TopkDecodeArgs& a, SelSmem& S, uint32_t* csm, int b,
-                                                   uint32_t C, uint32_t R1, int d1, float E) {
-    constexpr bool fits = SMEM;
-    uint32_t* lk = fits ? csm : a.amb_key + (size_t)b * a.Ncap;
-    int32_t* li = fits ? reinterpret_cast<int32_t*>(csm + kSelCap) : a.amb_idx + (size_t)b * a.Ncap;
+__device__ __noinline__ void resolve_candidates(const TopkDecodeArgs& a, SelSmem& S, uint32_t* csm, int b,
+                                                uint32_t C, uint32_t R1, int d1, float E) {
+    const bool fits = C <= (uint32_t)kSelCap;
+    const uint32_t* gk = a.cand_key + (size_t)b * a.Ncap;
+    const int32_t* gi = a.cand_idx + (size_t)b * a.Ncap;
+    // the candidate list: copied to shared memory when it fits, else read in place
+    uint32_t* lk = fits ? csm : const_cast<uint32_t*>(gk);
+    int32_t* li = fits ? reinterpret_cast<int32_t*>(csm + kSelCap) : const_cast<int32_t*>(gi);
     const int tid = threadIdx.x;
     uint32_t* bm = a.bitmap + (size_t)b * a.Wcap;
-    const int k = a.k;
-    const uint32_t* sk = a.cand_key + (size_t)b * a.Ncap;
-    const int32_t* si = a.cand_idx + (size_t)b * a.Ncap;
-    {
-        // 4 candidates per thread and round: loads first, then the stores
-        constexpr int U = 4;
-        for (uint32_t e0 = 0; e0 < C; e0 += U * kSelThreads) {
+    if (fits) {
+        constexpr int U = 4;  // loads first, then the stores
+        for (uint32_t e0 = 0; e0 < C; e0 += U * kResThreads) {
             uint32_t kv[U];
             int32_t iv[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                const uint32_t e_ = e0 + u * kSelThreads + tid;
-                int lo_ = 0, hi_ = a.nchunks;  // the chunk q with coff[q] <= e_ < coff[q+1]
-                while (hi_ - lo_ > 1) {
-                    const int mid = (lo_ + hi_) >> 1;
-                    if (S.coff[mid] <= e_) lo_ = mid;
-                    else hi_ = mid;
-                }
-                const size_t src = (size_t)lo_ * a.chunk + (e_ - S.coff[lo_]);
-                kv[u] = e_ < C ? __ldcg(sk + src) : 0u;
-                iv[u] = e_ < C ? __ldcg(si + src) : 0;
+                const uint32_t e_ = e0 + u * kResThreads + tid;
+                kv[u] = e_ < C ? __ldcg(gk + e_) : 0u;
+                iv[u] = e_ < C ? __ldcg(gi + e_) : 0;
             }
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                const uint32_t e_ = e0 + u * kSelThreads + tid;
+                const uint32_t e_ = e0 + u * kResThreads + tid;
                 if (e_ < C) {
-                    if (fits) {
-                        csm[e_] = kv[u];
-                        csm[kSelCap + e_] = (uint32_t)iv[u];
-                    } else {
-                        lk[e_] = kv[u];
-                        li[e_] = iv[u];
-                    }
+                    csm[e_] = kv[u];
+                    csm[kSelCap + e_] = (uint32_t)iv[u];
                 }
             }
         }
@@ -548,21 +536,20 @@ __device__ __forceinline__ void resolve_candidates(const TopkDecodeArgs& a, SelS
     const float t = key_to_float(tkey);
     const float e2 = __fmul_ru(2.f, E);
     const float band_hi = __fadd_ru(t, e2), band_lo = __fsub_rd(t, e2);
-    const uint16_t* qI = a.q_idx + (size_t)b * 64;
     const uint16_t* icx = a.kidx + (size_t)b * a.Ncap * 64;
-    // the band list: global arrays not in use as the candidate list
-    uint32_t* gak = fits ? a.amb_key + (size_t)b * a.Ncap : a.cand_key + (size_t)b * a.Ncap;
-    int32_t* gai = fits ? a.amb_idx + (size_t)b * a.Ncap : a.cand_idx + (size_t)b * a.Ncap;
+    // the band list (global, used when the band is large)
+    uint32_t* gak = a.amb_key + (size_t)b * a.Ncap;
+    int32_t* gai = a.amb_idx + (size_t)b * a.Ncap;
     uint32_t my_in2 = 0;
-    for (uint32_t i = tid; i < C; i += kSelThreads) {
+    for (uint32_t i = tid; i < C; i += kResThreads) {
         const float sv = key_to_float(lk[i]);
         if (sv > band_hi) {
             ++my_in2;
         } else if (sv >= band_lo) {
             const int32_t j = li[i];
-            const uint32_t p = atomicAdd(&S.amb_cnt, 1u);
-            const uint32_t ek = exact_key(qI, icx + (size_t)j * 64);
-            if (p < (uint32_t)kSelThreads) {
+            const uint32_t p = atom_add_shared(&S.amb_cnt, 1u);
+            const uint32_t ek = exact_key(S.q2, icx + (size_t)j * 64);
+            if (p < (uint32_t)kResThreads) {
                 S.amb_key[p] = ek;
                 S.amb_idx[p] = j;
             }
@@ -575,7 +562,7 @@ __device__ __forceinline__ void resolve_candidates(const TopkDecodeArgs& a, SelS
     const uint32_t na = S.amb_cnt;
     const uint32_t R2 = R1 - in2;  // winners to take from the band (1 <= R2 <= na)
     // the exact cut of the band: a member wins iff (key, -j) >= (T2, -jmax2)
-    if (na <= (uint32_t)kSelThreads) {
+    if (na <= (uint32_t)kResThreads) {
         if (tid < na) {
             const uint32_t mk = S.amb_key[tid];
             const int32_t mj = S.amb_idx[tid];
@@ -608,31 +595,35 @@ __device__ __forceinline__ void resolve_candidates(const TopkDecodeArgs& a, SelS
     const bool wlist = R1 <= (uint32_t)kBins;
     if (tid == 0) S.wcnt = 0;
     __syncthreads();
-    for (uint32_t i = tid; i < C; i += kSelThreads) {
+    for (uint32_t i = tid; i < C; i += kResThreads) {
         if (key_to_float(lk[i]) > band_hi) {
             const int32_t j = li[i];
-            if (wlist) S.hist[atomicAdd(&S.wcnt, 1u)] = (uint32_t)j;
-            else atomicOr(&bm[j >> 5], 1u << (j & 31));
+            if (wlist) {
+                const uint32_t p = atom_add_shared(&S.wcnt, 1u);
+                if (p < (uint32_t)kBins) S.hist[p] = (uint32_t)j;
+            } else {
+                atomicOr(&bm[j >> 5], 1u << (j & 31));
+            }
         }
     }
-    for (uint32_t i = tid; i < na; i += kSelThreads) {
-        const uint32_t kk = na <= (uint32_t)kSelThreads ? S.amb_key[i] : __ldcg(gak + i);
-        const int32_t j = na <= (uint32_t)kSelThreads ? S.amb_idx[i] : __ldcg(gai + i);
+    for (uint32_t i = tid; i < na; i += kResThreads) {
+        const uint32_t kk = na <= (uint32_t)kResThreads ? S.amb_key[i] : __ldcg(gak + i);
+        const int32_t j = na <= (uint32_t)kResThreads ? S.amb_idx[i] : __ldcg(gai + i);
         if (kk > T2 || (kk == T2 && j <= jmax2)) {
-            if (wlist) S.hist[atomicAdd(&S.wcnt, 1u)] = (uint32_t)j;
-            else atomicOr(&bm[j >> 5], 1u << (j & 31));
+            if (wlist) {
+                const uint32_t p = atom_add_shared(&S.wcnt, 1u);
+                if (p < (uint32_t)kBins) S.hist[p] = (uint32_t)j;
+            } else {
+                atomicOr(&bm[j >> 5], 1u << (j & 31));
+            }
         }
     }
     __syncthreads();
 }
 
-// One CTA per score chunk.  Filter: surely-selected entries become bitmap
-// bits, candidates go to the chunk's own slot.  The last CTA of a sequence to
-// finish (a ticket taken after a fence; nobody waits) then resolves it: finds
-// t~ among the gathered candidates, rescores the band exactly, marks the
-// winners and compacts the bitmap into ascending indices.
-__global__ void __launch_bounds__(kSelThreads, 3) topk_select_kernel(TopkDecodeArgs a) {
-    extern __shared__ __align__(16) uint32_t csm[];  // resolver: [kSelCap] keys, [kSelCap] indices
+// Filter: one CTA per score chunk; surely-selected entries become bitmap
+// bits, candidates go to the chunk's own slot.
+__global__ void __launch_bounds__(kSelThreads, 3) topk_filter_kernel(TopkDecodeArgs a) {
     __shared__ SelSmem S;
     const int b = blockIdx.y, c = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -656,8 +647,9 @@ __global__ void __launch_bounds__(kSelThreads, 3) topk_select_kernel(TopkDecodeA
     float e = 0.f;
     for (int q = tid; q < a.nchunks; q += kSelThreads) e = fmaxf(e, __ldcg(a.emax_part + (size_t)b * a.nchunks + q));
     const uint32_t* keys = a.keys + (size_t)b * a.Ncap;
-    uint32_t* ck = a.cand_key + (size_t)b * a.Ncap + row0;
-    int32_t* ci = a.cand_idx + (size_t)b * a.Ncap + row0;
+    uint32_t* ck = a.cand_key + (size_t)b * a.Ncap;
+    int32_t* ci = a.cand_idx + (size_t)b * a.Ncap;
+    uint32_t* tot4 = a.totals + (size_t)b * 4;
     uint32_t* bm = a.bitmap + (size_t)b * a.Wcap;
 #pragma unroll
     for (int u = 0; u < kBins / kSelThreads; ++u) S.hist[u * kSelThreads + tid] = hv[u];
@@ -673,9 +665,13 @@ __global__ void __launch_bounds__(kSelThreads, 3) topk_select_kernel(TopkDecodeA
     find_digit_desc<kBins>(S.hist, (uint32_t)k, S.sh32, &d1, &above1, S.res);
     if (d1 < 0) d1 = 0;  // cannot happen: the histogram counts all n > k keys
     const FilterBounds fb = filter_bounds(d1, E);
+    if (c == 0 && tid == 0) {  // the resolve reads the bin and the bound from here
+        tot4[2] = (uint32_t)d1;
+        tot4[3] = __float_as_uint(E);
+    }
 
-    uint32_t ncand = 0, nin = 0;
-    for (int p0 = row0; p0 < row1; p0 += kSelKPT * kSelThreads) {  // passes of up to 8192 rows
+    uint32_t nin = 0;
+    for (int p0 = row0; p0 < row1; p0 += kSelKPT * kSelThreads) {  // passes of up to 4096 rows
         uint32_t kr[kSelKPT];
 #pragma unroll
         for (int i = 0; i < kSelKPT; ++i) {
@@ -700,85 +696,89 @@ __global__ void __launch_bounds__(kSelThreads, 3) topk_select_kernel(TopkDecodeA
             }
         }
         uint32_t tot;
-        uint32_t pos = ncand + block_exclusive_scan(mycnt, S.sh32, &tot);
-#pragma unroll
-        for (int i = 0; i < kSelKPT; ++i) {
-            if ((cmask >> i) & 1u) {
-                ck[pos] = kr[i];
-                ci[pos] = p0 + i * kSelThreads + tid;
-                ++pos;
+        uint32_t pos = block_exclusive_scan(mycnt, S.sh32, &tot);
+        if (tot) {  // one append per pass to the sequence's candidate list
+            if (tid == 0) S.last = atomicAdd(&tot4[0], tot);
+            __syncthreads();
+            pos += S.last;
+            if (pos + mycnt > (uint32_t)a.Ncap) {  // cannot happen: at most n candidates
+                flag(DEV_LEN);
+                mycnt = 0;
             }
+#pragma unroll
+            for (int i = 0; i < kSelKPT; ++i) {
+                if ((cmask >> i) & 1u) {
+                    ck[pos] = kr[i];
+                    ci[pos] = p0 + i * kSelThreads + tid;
+                    ++pos;
+                }
+            }
+            __syncthreads();  // S.last is reused
         }
-        ncand += tot;
     }
     if (lane == 0) S.amb_key[warp] = nin;  // (scratch) per-warp sure-in counts
     __syncthreads();
     if (tid == 0) {
         uint32_t s_in = 0;
         for (int w = 0; w < kSelThreads / 32; ++w) s_in += S.amb_key[w];
-        a.cand_cnt[(size_t)b * a.nchunks + c] = ncand;
-        a.in_cnt[(size_t)b * a.nchunks + c] = s_in;
-        __threadfence();  // publish this chunk's slot, counts and bitmap words before the ticket
-        const uint32_t prev = atomicAdd(&a.done[b], 1u);
-        S.last = prev == (uint32_t)(a.nchunks - 1);
+        if (s_in) atomicAdd(&tot4[1], s_in);
     }
-    __syncthreads();
-    if (!S.last) return;
+}
 
-    // ---- resolve (the last CTA of sequence b); cross-CTA data is read through L2
+// One CTA of 1024 threads per sequence: gathers the filter's candidates,
+// finds t~ among them, rescores the band exactly, ranks it by (s, -j), marks
+// the winners and compacts the selection bitmap into ascending indices.
+__global__ void __launch_bounds__(kResThreads, 1) topk_resolve_kernel(TopkDecodeArgs a) {
+    extern __shared__ __align__(16) uint32_t csm[];  // [kSelCap] keys, [kSelCap] indices
+    __shared__ SelSmem S;
+    const int b = blockIdx.x;
+    const int tid = threadIdx.x;
+    const int n = clamp_n(a.n, b, a.Ncap);
+    const int k = a.k;
+    if (n <= k) {
+        int32_t* idx = a.idx + (size_t)b * k;
+        for (int i = tid; i < k; i += blockDim.x) idx[i] = i < n ? i : -1;
+        if (tid == 0) a.cnt[b] = n;
+        return;
+    }
+    uint32_t* bm = a.bitmap + (size_t)b * a.Wcap;
+    load_q2(S.q2, a.q_idx + (size_t)b * 64);
     if (tid == 0) {
-        __threadfence();
-        a.done[b] = 0;  // ready for the next call
         S.amb_cnt = 0;
         S.in2 = 0;
     }
-    uint32_t C = 0, A = 0;
-    {
-        // chunk offsets (nchunks <= kSelMaxChunks)
-        constexpr int CPT = kSelMaxChunks / kSelThreads;
-        uint32_t cc[CPT], ic[CPT], sc = 0, si = 0;
-#pragma unroll
-        for (int u = 0; u < CPT; ++u) {
-            const int q = tid * CPT + u;
-            cc[u] = q < a.nchunks ? __ldcg(a.cand_cnt + (size_t)b * a.nchunks + q) : 0u;
-            ic[u] = q < a.nchunks ? __ldcg(a.in_cnt + (size_t)b * a.nchunks + q) : 0u;
-            sc += cc[u];
-            si += ic[u];
-        }
-        uint32_t off = block_exclusive_scan(sc, S.sh32, &C);
-        block_exclusive_scan(si, S.sh32, &A);
-#pragma unroll
-        for (int u = 0; u < CPT; ++u) {
-            S.coff[tid * CPT + u] = off;
-            off += cc[u];
-        }
-        if (tid == 0) S.coff[kSelMaxChunks] = C;
+    const uint32_t* tot4 = a.totals + (size_t)b * 4;
+    uint32_t C = __ldcg(tot4 + 0);
+    const uint32_t A = __ldcg(tot4 + 1);
+    const int d1 = (int)__ldcg(tot4 + 2);
+    const float E = __uint_as_float(__ldcg(tot4 + 3));
+    if (C > (uint32_t)a.Ncap) {
+        if (tid == 0) flag(DEV_LEN);
+        C = a.Ncap;
     }
     __syncthreads();
     const uint32_t R1 = (uint32_t)k - A;  // rank of t~ among the candidates (>= 1)
-    if (C <= (uint32_t)kSelCap)
-        resolve_candidates<true>(a, S, csm, b, C, R1, d1, E);
-    else
-        resolve_candidates<false>(a, S, csm, b, C, R1, d1, E);
+    resolve_candidates(a, S, csm, b, C, R1, d1, E);
     __syncthreads();
     // candidates are consumed: csm now holds a shared bitmap of the winners
     // (when it fits next to an output stage of k indices)
     const int nwords = (n + 31) >> 5;
-    const bool sbm = S.wcnt > 0 && R1 <= (uint32_t)kBins &&
-                     (size_t)nwords + (size_t)k <= (size_t)kSelCap * 2;
+    const bool sbm = S.wcnt > 0 && R1 <= (uint32_t)kBins && (size_t)nwords <= (size_t)kSelCap * 2;
     const bool was_list = R1 <= (uint32_t)kBins;
     uint32_t* extra = nullptr;
     if (was_list) {
         if (sbm) {
-            for (int w = tid; w < nwords; w += kSelThreads) csm[w] = 0u;
+            for (int w = tid; w < nwords; w += kResThreads) csm[w] = 0u;
             __syncthreads();
-            for (uint32_t i = tid; i < S.wcnt; i += kSelThreads) {
+            const uint32_t nw_ = S.wcnt < (uint32_t)kBins ? S.wcnt : (uint32_t)kBins;
+            for (uint32_t i = tid; i < nw_; i += kResThreads) {
                 const uint32_t j = S.hist[i];
-                atomicOr(&csm[j >> 5], 1u << (j & 31));
+                red_or_shared(&csm[j >> 5], 1u << (j & 31));
             }
             extra = csm;
         } else {
-            for (uint32_t i = tid; i < S.wcnt; i += kSelThreads) {
+            const uint32_t nw_ = S.wcnt < (uint32_t)kBins ? S.wcnt : (uint32_t)kBins;
+            for (uint32_t i = tid; i < nw_; i += kResThreads) {
                 const uint32_t j = S.hist[i];
                 atomicOr(&bm[j >> 5], 1u << (j & 31));
             }
@@ -786,10 +786,24 @@ __global__ void __launch_bounds__(kSelThreads, 3) topk_select_kernel(TopkDecodeA
         }
         __syncthreads();
     }
-    uint32_t* ostage = ((size_t)(extra ? nwords : 0) + (size_t)k <= (size_t)kSelCap * 2) ? csm + (extra ? nwords : 0)
-                                                                                          : nullptr;
+    // shared layout for the compaction: [winner bitmap][staging][output stage of k]
+    const size_t base = extra ? (size_t)nwords : 0;
+    constexpr size_t stg = (size_t)kResThreads * (kCompPer + 1);
+    static_assert(stg <= (size_t)kSelCap * 2, "compaction staging must fit the shared area");
     uint32_t total;
-    compact_bitmap(bm, extra, nwords, a.idx + (size_t)b * k, (uint32_t)k, ostage, S.coff, S.sh32, &total);
+    if (base + stg <= (size_t)kSelCap * 2) {
+        uint32_t* ostage = base + stg + (size_t)k <= (size_t)kSelCap * 2 ? csm + base + stg : nullptr;
+        compact_bitmap(bm, extra, nwords, a.idx + (size_t)b * k, (uint32_t)k, ostage, csm + base, S.sh32, &total);
+    } else {
+        // no room next to the winner bitmap: fold it into the global one first
+        // (extra is set here: without it base is 0 and the staging fits)
+        if (extra)
+            for (int w = tid; w < nwords; w += kResThreads)
+                if (extra[w]) atomicOr(&bm[w], extra[w]);
+        __threadfence_block();
+        __syncthreads();
+        compact_bitmap(bm, nullptr, nwords, a.idx + (size_t)b * k, (uint32_t)k, nullptr, csm, S.sh32, &total);
+    }
     if (tid == 0) {
         if (total != (uint32_t)k) flag(DEV_LEN);  // cannot happen
         a.cnt[b] = k;
