@@ -159,6 +159,22 @@ def decode_bytes(w, lengths):
     return step, score
 
 
+def max_over_ranks(ms, world, device):
+    """The job's time is the slowest rank's: every rank calls this at the same point."""
+    if world == 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank, world, max_ms):
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank * world / (max_ms / 1e3)
+
+
 def make_inputs(w, rank):
     seed = synth.BASE_SEED + w.index + 7919 * rank
     B, L = w.B, w.L
@@ -274,11 +290,7 @@ def run_ours(args, w, rank, world, dev):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     S.read_device_status()
 
     # end to end through the public API: pinned host q / q_idx in, outputs back out
@@ -311,16 +323,11 @@ def run_ours(args, w, rank, world, dev):
         ev1[i].record(stream)
         ev1[i].synchronize()
         e2e_ms.append(ev0[i].elapsed_time(ev1[i]))
-    e2e_total = sum(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
+    e2e_total = max_over_ranks(sum(e2e_ms), world, dev)
     S.read_device_status()
     del graph
 
-    tokens = B * world * args.steps
-    value = tokens / (total_ms / 1e3)
+    value = job_throughput(B * args.steps, world, total_ms)
     step_bytes, score_bytes = decode_bytes(w, lengths)
     peak, peak_kind = measured_peaks()
     score_avg = statistics.mean(score_ms)
@@ -351,7 +358,7 @@ def run_ours(args, w, rank, world, dev):
                      "traffic": recorded_traffic("score_decode_kernel", w.name)},
         "stages_ms": {n: statistics.mean(v) for n, v in zip(stage_names, stage_ms)},
         "gpu_launches": launches_per_step * args.steps,
-        "e2e": {"value": tokens / (e2e_total / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": job_throughput(B * args.steps, world, e2e_total), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "api": "hybrid_attn_decode (eager) + pinned-host copies"},
         "clocks": clk.summary(),
         "setup_s": round(time.time() - t_gen, 1),
