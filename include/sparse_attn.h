@@ -201,6 +201,30 @@ typedef enum {
  * stage off.  The events are the caller's; the library only records them.   */
 sa_status sa_set_stage_events(int32_t stage, void* before, void* after);
 
+/* Maximum scratch of csa_index_topk_noalloc, per device.                    */
+#define SA_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* csa_index_topk for callers that cannot allocate device memory.  (The paper
+ * has no counterpart: this is a deployment convenience.)  Some callers cannot
+ * give the library a workspace: a C caller that only holds its input and
+ * output buffers, or a serving loop whose device memory is entirely owned by
+ * another allocator and which may not call cudaMalloc (that call can also
+ * synchronise the device, which such a loop cannot afford).  This entry point
+ * computes the same decode top-k as csa_index_topk with q_pos == NULL and
+ * Tq == 1, bit for bit, but takes its scratch from a static device array of
+ * SA_NOALLOC_SCRATCH_BYTES that the library owns: every GPU that loads the
+ * library holds that array until the process exits.  It allocates and frees
+ * nothing.  The first call on a device looks the array's address up
+ * (cudaGetSymbolAddress) and should therefore come before any stream capture.
+ * All calls on a device share the one array, which keeps the last call's
+ * contents (each call clears what it needs): calls whose work overlaps on the
+ * GPU, on different streams or host threads, race and must not be issued.
+ * Returns SA_ERR_UNSUPPORTED when B, Ncap and k need more scratch than the
+ * array holds (for example B = 4, Ncap = 262144, k = 2048 needs about 21 MB).
+ *   q_idx [B][d_idx] bf16; idx [B][k] and cnt [B] int32 out, as csa_index_topk. */
+sa_status csa_index_topk_noalloc(const void* q_idx, const sa_cache* csa, int32_t k, int32_t* idx, int32_t* cnt,
+                                 void* stream);
+
 /* Number of kernels this library has launched from the calling host thread
  * since the process started (a diagnostic counter; memsets are not kernels). */
 uint64_t sa_launch_count(void);

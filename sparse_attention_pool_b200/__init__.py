@@ -3,7 +3,8 @@
 The compute path is the CUDA library; ``api`` only marshals torch tensors
 into its C ABI and ``synth`` only generates seeded inputs.
 """
-from .api import (Cache, alloc_cache, alloc_workspace, csa_compress, csa_index_topk, csa_sparse_attn,  # noqa: F401
+from .api import (Cache, alloc_cache, alloc_workspace, csa_compress, csa_index_topk, csa_index_topk_noalloc,  # noqa: F401
+                  csa_sparse_attn,
                   hca_compress, hca_dense_attn, hybrid_attn_decode, hybrid_attn_prefill, read_device_status,
                   workspace_size)
 from ._lib import (SA_OP_DENSE_ATTN, SA_OP_HYBRID_DECODE, SA_OP_HYBRID_PREFILL, SA_OP_INDEX_TOPK,  # noqa: F401

@@ -126,6 +126,21 @@ def csa_index_topk(q_idx, csa: Cache, k: int, ws, *, q_pos=None, idx=None, cnt=N
     return idx, cnt
 
 
+def csa_index_topk_noalloc(q_idx, csa: Cache, k: int, *, idx=None, cnt=None, stream=None):
+    """Decode top-k without a workspace: the library's static device scratch is
+    used instead (for callers that cannot allocate; see the C header)."""
+    _need(q_idx, torch.bfloat16, "q_idx")
+    B = csa.B
+    if idx is None:
+        idx = torch.empty(B, 1, k, dtype=torch.int32, device=q_idx.device)
+    if cnt is None:
+        cnt = torch.empty(B, 1, dtype=torch.int32, device=q_idx.device)
+    cs = csa.struct()
+    check("csa_index_topk_noalloc", lib().csa_index_topk_noalloc(_ptr(q_idx), ctypes.byref(cs), k, _ptr(idx),
+                                                                 _ptr(cnt), _stream(stream)))
+    return idx, cnt
+
+
 def csa_sparse_attn(q, csa: Cache, idx, cnt, k: int, ws, *, scale=0.0, out=None, lse=None, stream=None):
     _need(q, torch.bfloat16, "q")
     B, Tq, H = q.shape[0], (q.shape[1] if q.dim() == 4 else 1), q.shape[-2]

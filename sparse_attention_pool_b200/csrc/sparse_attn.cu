@@ -463,6 +463,32 @@ sa_status run_topk_prefill(const void* q_idx, int Tq, const int32_t* pos, const 
     return SA_OK;
 }
 
+// ------------------------------------------------------- static scratch --
+// The scratch of csa_index_topk_noalloc: a device array owned by the library,
+// resident on every GPU that loads it.  In host code the name is only a
+// stand-in for the symbol; kernels get its device address, looked up once per
+// device with that device current.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[SA_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+sa_status noalloc_scratch(void** out) {
+    int dev = 0;
+    SA_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) return fail(SA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p)
+            return fail(SA_ERR_CUDA, "cudaGetSymbolAddress(static scratch): %s", cudaGetErrorString(e));
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return SA_OK;
+}
+
 }  // namespace
 
 // =========================================================== public ABI ====
@@ -604,6 +630,27 @@ sa_status csa_index_topk(const void* q_idx, int32_t Tq, const int32_t* q_pos, co
     r = check_ws(ws, ws_bytes, prefill_topk_bytes(csa->B, Tq, csa->Ncap, k));
     if (r != SA_OK) return r;
     return run_topk_prefill(q_idx, Tq, q_pos, csa, k, idx, cnt, ws, st);
+}
+
+sa_status csa_index_topk_noalloc(const void* q_idx, const sa_cache* csa, int32_t k, int32_t* idx, int32_t* cnt,
+                                 void* stream) {
+    sa_status r = check_cache(csa, true, "csa_index_topk_noalloc");
+    if (r != SA_OK) return r;
+    SA_CHECK(q_idx && aligned16(q_idx), "csa_index_topk_noalloc: q_idx must be non-NULL and 16-byte aligned");
+    SA_CHECK(idx && cnt && aligned16(idx) && aligned16(cnt),
+             "csa_index_topk_noalloc: idx/cnt must be non-NULL and aligned");
+    SA_CHECK(k >= 1 && k <= 65536, "csa_index_topk_noalloc: k=%d outside 1..65536", k);
+    const TopkDecodeWs w = topk_decode_layout(csa->B, csa->Ncap, k, false);
+    if (w.total > (size_t)SA_NOALLOC_SCRATCH_BYTES)
+        return fail(SA_ERR_UNSUPPORTED,
+                    "csa_index_topk_noalloc: B=%d, Ncap=%d, k=%d need %zu bytes of scratch; the static scratch "
+                    "holds %u (use csa_index_topk with a workspace)",
+                    csa->B, csa->Ncap, k, w.total, (unsigned)SA_NOALLOC_SCRATCH_BYTES);
+    void* scratch = nullptr;
+    r = noalloc_scratch(&scratch);
+    if (r != SA_OK) return r;
+    return run_topk_decode(q_idx, csa, k, idx, cnt, scratch, w, static_cast<cudaStream_t>(stream),
+                           [] { return SA_OK; });
 }
 
 sa_status csa_sparse_attn(const void* q, int32_t Tq, int32_t H, const sa_cache* csa, const int32_t* idx,
