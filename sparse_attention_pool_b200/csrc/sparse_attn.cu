@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -67,6 +68,21 @@ sa_status fail(sa_status s, const char* fmt, ...) {
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 inline int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+// Kernel attributes are set once per device: `done` holds one bit per device.
+inline int cur_device() {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    return dev;
+}
+inline bool attr_done(const std::atomic<uint64_t>& done) {
+    const int dev = cur_device();
+    return dev >= 0 && dev < 64 && (done.load() >> dev & 1u);
+}
+inline void attr_set(std::atomic<uint64_t>& done) {
+    const int dev = cur_device();
+    if (dev >= 0 && dev < 64) done.fetch_or(uint64_t(1) << dev);
+}
 
 int num_sms() {
     static int sms[64] = {0};
@@ -140,7 +156,8 @@ sa_status make_ic_map(CUtensorMap* map, const void* kidx, int B, int Ncap) {
 
 // ------------------------------------------------------- workspace layout --
 struct TopkDecodeWs {
-    size_t hist, totals, keys, emax, cand_key, cand_idx, amb_key, amb_idx, bitmap, idx, cnt, total;
+    size_t hist, hist2, totals, zero_end, keys, emax, chunk_in, chunk_pos, cand_key, cand_idx, amb_key, amb_idx,
+        bitmap, idx, cnt, total;
     int maxchunks, Wcap;
 };
 
@@ -152,8 +169,9 @@ int score_chunk(int B, int Ncap) {
     return (int)std::max<long long>(chunk, sa::kScRows);
 }
 
-// [reserved 256 B][histograms][totals][keys][per-chunk max error][candidates key/idx]
-// [band key/idx][bitmap][idx][cnt]
+// [reserved 256 B][histograms][second histograms][totals][keys][per-chunk max error]
+// [per-chunk sure-in counts][per-chunk output positions][candidates key/idx][band key/idx]
+// [bitmap][idx][cnt]
 TopkDecodeWs topk_decode_layout(int B, int Ncap, int k, bool own_idx) {
     TopkDecodeWs w{};
     w.maxchunks = std::max(1, cdiv(Ncap, sa::kScRows));
@@ -161,13 +179,22 @@ TopkDecodeWs topk_decode_layout(int B, int Ncap, int k, bool own_idx) {
     size_t o = 256;
     w.hist = o;  // histograms and totals are zeroed together before every call
     o += (size_t)B * sa::kBins * 4;
+    w.hist2 = o;
+    o += (size_t)B * sa::kBins * 4;
     w.totals = o;
-    o += up256((size_t)B * 16);
+    o += (size_t)B * sa::kTotals * 4;
+    w.zero_end = o;
+    o = up256(o);
     const size_t col = up256((size_t)B * Ncap * 4);
+    const size_t per_chunk = up256((size_t)B * w.maxchunks * 4);
     w.keys = o;
     o += col;
     w.emax = o;
-    o += up256((size_t)B * w.maxchunks * 4);
+    o += per_chunk;
+    w.chunk_in = o;
+    o += per_chunk;
+    w.chunk_pos = o;
+    o += per_chunk;
     w.cand_key = o;
     o += col;
     w.cand_idx = o;
@@ -208,11 +235,11 @@ size_t attn_partial_bytes(long long BQ, int splits, int H) {
 template <int NW, bool G, bool F, int ST, bool CL>
 sa_status launch_attn_t(const sa::AttnArgs& a, dim3 grid, cudaStream_t st) {
     using L = sa::AttnSmem<NW, G, F, ST>;
-    static bool init = false;
-    if (!init) {
+    static std::atomic<uint64_t> init{0};
+    if (!attr_done(init)) {
         SA_CUDA(cudaFuncSetAttribute(sa::attn_split_kernel<NW, G, F, ST, CL>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal));
-        init = true;
+        attr_set(init);
     }
     if (CL) {
         cudaLaunchConfig_t cfg = {};
@@ -345,7 +372,10 @@ sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* 
     a.n = c->n;
     a.keys = reinterpret_cast<uint32_t*>(base + w.keys);
     a.hist1 = reinterpret_cast<uint32_t*>(base + w.hist);
+    a.hist2 = reinterpret_cast<uint32_t*>(base + w.hist2);
     a.emax_part = reinterpret_cast<float*>(base + w.emax);
+    a.chunk_in = reinterpret_cast<uint32_t*>(base + w.chunk_in);
+    a.chunk_pos = reinterpret_cast<uint32_t*>(base + w.chunk_pos);
     a.cand_key = reinterpret_cast<uint32_t*>(base + w.cand_key);
     a.cand_idx = reinterpret_cast<int32_t*>(base + w.cand_idx);
     a.amb_key = reinterpret_cast<uint32_t*>(base + w.amb_key);
@@ -361,20 +391,20 @@ sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* 
     a.nchunks = Ncap > 0 ? cdiv(Ncap, a.chunk) : 1;
     if (a.nchunks > w.maxchunks || a.nchunks > sa::kSelMaxChunks)
         return fail(SA_ERR_WORKSPACE, "internal: chunk count above the workspace bound");
-    static bool init = false;
+    static std::atomic<uint64_t> init{0};
     const size_t smem = sa::kScStages * sa::kScTileBytes + sa::kScStages * 8 + 1024;
-    if (!init) {
+    if (!attr_done(init)) {
         SA_CUDA(cudaFuncSetAttribute(sa::score_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
         SA_CUDA(cudaFuncSetAttribute(sa::topk_resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      sa::kSelSmem));
-        init = true;
+        attr_set(init);
     }
     if (Ncap > 0) {
         CUtensorMap map;
         sa_status r = make_ic_map(&map, c->kidx, B, Ncap);
         if (r != SA_OK) return r;
         stage_mark(SA_STAGE_INDEX_SCORE, 0, st);
-        SA_CUDA(cudaMemsetAsync(a.hist1, 0, w.totals - w.hist + (size_t)B * 16, st));
+        SA_CUDA(cudaMemsetAsync(a.hist1, 0, w.zero_end - w.hist, st));
         sa::score_decode_kernel<<<dim3(a.nchunks, B), sa::kScThreads, smem, st>>>(map, a);
         SA_LAUNCHED();
         stage_mark(SA_STAGE_INDEX_SCORE, 1, st);
@@ -382,11 +412,13 @@ sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* 
     sa_status r = between();
     if (r != SA_OK) return r;
     stage_mark(SA_STAGE_TOPK_SELECT, 0, st);
-    if (Ncap > 0) {
-        sa::topk_filter_kernel<<<dim3(a.nchunks, B), sa::kSelThreads, 0, st>>>(a);
-        SA_LAUNCHED();
-    }
+    // a sequence with n <= k visible entries (every one, when Ncap is 0) is
+    // answered by the filter's first CTA; the other kernels skip it
+    sa::topk_filter_kernel<<<dim3(a.nchunks, B), sa::kSelThreads, 0, st>>>(a);
+    SA_LAUNCHED();
     sa::topk_resolve_kernel<<<B, sa::kResThreads, sa::kSelSmem, st>>>(a);
+    SA_LAUNCHED();
+    sa::topk_emit_kernel<<<dim3(a.nchunks, B), sa::kEmitThreads, 0, st>>>(a);
     SA_LAUNCHED();
     stage_mark(SA_STAGE_TOPK_SELECT, 1, st);
     return SA_OK;
@@ -438,13 +470,13 @@ sa_status run_topk_prefill(const void* q_idx, int Tq, const int32_t* pos, const 
     a.KS = keys_stride(c->Ncap);
     a.k = k;
     a.log2m = ilog2(c->m);
-    static bool init = false;
-    if (!init) {
+    static std::atomic<uint64_t> init{0};
+    if (!attr_done(init)) {
         SA_CUDA(cudaFuncSetAttribute(sa::score_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      sa::kPsSmem));
         SA_CUDA(cudaFuncSetAttribute(sa::select_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      sa::kPselSmemKeys * 4));
-        init = true;
+        attr_set(init);
     }
     const int etiles = std::max(1, cdiv(c->Ncap, sa::kPsE));
     for (int b = 0; b < c->B; ++b) {

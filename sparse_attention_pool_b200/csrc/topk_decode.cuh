@@ -19,20 +19,23 @@
 //            with s~ < t~ - 2E surely not, and only the band |s~ - t~| <= 2E
 //            is rescored exactly (the fp64 definition) and ranked exactly.
 //
-// Three kernels, ordered on one stream (every hand-off is a kernel boundary;
+// Four kernels, ordered on one stream (every hand-off is a kernel boundary;
 // no CTA waits on another):
 //   1. score_decode_kernel -- streams Ic through a 4-stage TMA pipeline
 //      (128-byte rows, 128B swizzle, one row per thread) and writes an order
 //      key of s~ per entry, a histogram of the top 11 key bits (per CTA in
 //      shared memory, then added to the sequence's) and each CTA's max e_j.
 //   2. topk_filter_kernel  -- one CTA per score chunk: from the histogram the
-//      bin of t~; entries above that bin widened by 2E become bitmap bits
-//      (surely selected), entries in the widened bin become candidates in the
-//      chunk's own slot.  Plain stores.
-//   3. topk_resolve_kernel -- one 1024-thread CTA per sequence: gathers the
-//      candidates, finds t~ among them, rescores the band exactly, ranks it
-//      by (s, -j), marks the winners and compacts the bitmap into ascending
-//      indices.
+//      bin d1 of t~; entries above that bin widened by 2E become bitmap bits
+//      (surely selected, counted per chunk), entries in the widened bin
+//      become candidates, and those inside bin d1 feed a histogram of key
+//      bits 20..10.
+//   3. topk_resolve_kernel -- one 1024-thread CTA per sequence: the second
+//      histogram gives the fine bin of t~, whose few keys are ranked; the band
+//      is rescored exactly and ranked by (s, -j); the winners join the bitmap
+//      and every chunk gets the output position of its first selected entry.
+//   4. topk_emit_kernel    -- one CTA per chunk writes its selected indices,
+//      ascending, from that position on.
 #pragma once
 #include "sa_common.cuh"
 
@@ -45,16 +48,24 @@ constexpr int kScTileBytes = kScRows * 128;
 constexpr int kBins = 2048;       // 11-bit digits
 constexpr int kBinsLow = 1024;    // last 10-bit digit
 
+// totals[B][kTotals] (zeroed per call): candidate count, and from the first
+// filter CTA the bin d1 of t~, the bound E and the count of keys above bin d1
+constexpr int kTotals = 4;
+constexpr int kTotCand = 0, kTotBin = 1, kTotE = 2, kTotAbove = 3;
+
 struct TopkDecodeArgs {
     const uint16_t* q_idx;  // [B][64]
     const uint16_t* kidx;   // [B][Ncap][64] (exact rescoring)
     const int32_t* n;       // [B]
     uint32_t* keys;         // [B][Ncap]     order keys of the screened scores
-    uint32_t* hist1;        // [B][2048]     histogram of the top 11 key bits (zeroed per call)
+    uint32_t* hist1;        // [B][2048]     histogram of key bits 31..21 (zeroed per call)
+    uint32_t* hist2;        // [B][2048]     bits 20..10 of the keys in bin d1 (zeroed per call)
     float* emax_part;       // [B][nchunks]  per score CTA: max e_j
+    uint32_t* chunk_in;     // [B][nchunks]  per filter CTA: surely selected entries
+    uint32_t* chunk_pos;    // [B][nchunks]  output position of each chunk's first selected entry
     uint32_t* cand_key;     // [B][Ncap]     candidates of the sequence (filter order)
     int32_t* cand_idx;      // [B][Ncap]
-    uint32_t* totals;       // [B][4]        candidates, sure-ins, bin d1, E bits (zeroed per call)
+    uint32_t* totals;       // [B][kTotals]
     uint32_t* bitmap;       // [B][Wcap]     selection bitmap
     uint32_t* amb_key;      // [B][Ncap]     exact keys of the band, when it is large
     int32_t* amb_idx;       // [B][Ncap]
@@ -409,6 +420,8 @@ constexpr int kSelKPT = 16;                  // keys per thread held in register
 constexpr int kSelCap = 8192;                // candidates the resolving CTA holds in shared memory
 constexpr int kSelSmem = kSelCap * 8;
 constexpr int kSelMaxChunks = 1024;
+static_assert(kSelMaxChunks <= kResThreads, "the resolve gives one thread to every chunk");
+static_assert(kBins == 2 * kResThreads, "the resolve loads the second histogram two bins per thread");
 
 struct FilterBounds {
     float in_above;  // s~ > in_above  : surely selected
@@ -425,86 +438,222 @@ __device__ __forceinline__ FilterBounds filter_bounds(int d1, float E) {
     return {__fadd_ru(hi, e2), __fsub_rd(lo, e2)};
 }
 
-// Writes the set bits of (bm | extra)[0..nwords) as ascending indices into
-// out[0..cap); `extra` is an optional bitmap in shared memory.  Written for a
-// CTA that runs this code once: rolled loops keep the code small (a cold
-// instruction cache costs more here than loop overhead).  Words are staged in
-// shared memory (`stage`, blockDim*(PER+1) words) so that global reads are
-// coalesced and each thread then owns PER consecutive words; with `ostage`
-// (shared, >= cap words) the indices leave in coalesced stores too.
-constexpr int kCompPer = 4;  // words per thread per round; staging = blockDim * (kCompPer + 1) words
-__device__ __noinline__ void compact_bitmap(const uint32_t* bm, const uint32_t* extra, int nwords, int32_t* out,
-                                            uint32_t cap, uint32_t* ostage, uint32_t* stage, uint32_t* sh32,
-                                            uint32_t* total_out) {
-    const int T = blockDim.x;
-    const int span = T * kCompPer;
-    uint32_t running = 0;
-#pragma unroll 1
-    for (int w0 = 0; w0 < nwords; w0 += span) {
-        __syncthreads();  // stage is reused
-#pragma unroll 4
-        for (int i = threadIdx.x; i < span; i += T) {
-            const int w = w0 + i;
-            uint32_t v = w < nwords ? __ldcg(bm + w) : 0u;
-            if (extra && w < nwords) v |= extra[w];
-            stage[(i / kCompPer) * (kCompPer + 1) + (i % kCompPer)] = v;
-        }
-        __syncthreads();
-        const uint32_t* mine = stage + threadIdx.x * (kCompPer + 1);
-        uint32_t c = 0;
-#pragma unroll 1
-        for (int u = 0; u < kCompPer; ++u) c += __popc(mine[u]);
-        uint32_t tot;
-        uint32_t pos = running + block_exclusive_scan(c, sh32, &tot);
-        const int wb = w0 + threadIdx.x * kCompPer;
-#pragma unroll 1
-        for (int u = 0; u < kCompPer; ++u) {
-            uint32_t word = mine[u];
-            while (word) {
-                const int bit = __ffs(word) - 1;
-                word &= word - 1;
-                if (pos < cap) {
-                    if (ostage) ostage[pos] = (uint32_t)((wb + u) * 32 + bit);
-                    else out[pos] = (wb + u) * 32 + bit;
-                }
-                ++pos;
-            }
-        }
-        running += tot;
-    }
-    __syncthreads();
-    if (ostage) {
-        const uint32_t nout = running < cap ? running : cap;
-#pragma unroll 1
-        for (uint32_t i = threadIdx.x; i < nout; i += T) out[i] = (int32_t)ostage[i];
-    }
-    *total_out = running;
-}
-
 struct SelSmem {
     double q2[64];            // qI * 2^768 for the exact rescoring
-    uint32_t hist[kBins];
+    uint32_t hist[kBins];     // digit histograms; later the per-chunk winner counts
     uint32_t sh32[32];
     int res[2];
     float red[kSelThreads / 32];
-    uint32_t last, amb_cnt, in2, wcnt, T2;
+    uint32_t last, amb_cnt, f_cnt, tkey, T2;
     int32_t jmax2;
-    uint32_t amb_key[kResThreads];
+    uint32_t amb_key[kResThreads];  // the fine bin's keys, then the band's exact keys
     int32_t amb_idx[kResThreads];
 };
 
-// The resolve step of topk_select_kernel over the C gathered candidates, with
-// the candidate list in shared memory (SMEM) or in global memory.
-__device__ __noinline__ void resolve_candidates(const TopkDecodeArgs& a, SelSmem& S, uint32_t* csm, int b,
-                                                uint32_t C, uint32_t R1, int d1, float E) {
+// The R1-th largest screened key t~ among the C candidates.  Fast path: the
+// filter's histogram of bits 20..10 over bin d1 gives the fine bin of t~
+// directly (rank K2 = k - above1 inside bin d1), whose few keys are ranked
+// pairwise.  Otherwise (a crowded fine bin, or counts that do not add up)
+// the digit passes over the whole list.
+__device__ __noinline__ uint32_t find_threshold(const uint32_t* lk, const int32_t* li, uint32_t C, uint32_t R1,
+                                                int d1, uint32_t K2, SelSmem& S) {
+    const int tid = threadIdx.x;
+    int d2;
+    uint32_t above2;
+    find_digit_desc<kBins>(S.hist, K2, S.sh32, &d2, &above2, S.res);
+    if (d2 >= 0) {
+        const uint32_t R3 = K2 - above2;  // rank of t~ inside the fine bin
+        const uint32_t pre = ((uint32_t)d1 << 11) | (uint32_t)d2;
+        if (tid == 0) {
+            S.f_cnt = 0;
+            S.tkey = 0;
+            S.last = 0;
+        }
+        __syncthreads();
+#pragma unroll 1
+        for (uint32_t i = tid; i < C; i += kResThreads) {
+            const uint32_t kk = lk[i];
+            if ((kk >> 10) == pre) {
+                const uint32_t p = atom_add_shared(&S.f_cnt, 1u);
+                if (p < (uint32_t)kResThreads) S.amb_key[p] = kk;
+            }
+        }
+        __syncthreads();
+        const uint32_t nf = S.f_cnt;
+        if (nf <= (uint32_t)kResThreads && R3 <= nf) {
+            if ((uint32_t)tid < nf) {
+                const uint32_t mk = S.amb_key[tid];
+                uint32_t gt = 0, ge = 0;
+                for (uint32_t o = 0; o < nf; ++o) {
+                    const uint32_t ok = S.amb_key[o];
+                    gt += ok > mk;
+                    ge += ok >= mk;
+                }
+                if (gt < R3 && R3 <= ge) {  // every thread holding t~ writes the same value
+                    S.tkey = mk;
+                    S.last = 1;
+                }
+            }
+            __syncthreads();
+            if (S.last) return S.tkey;
+        }
+    }
+    uint32_t tkey;
+    if (!rank_in_bin(lk, C, R1, d1, S.hist, S.sh32, S.res, &tkey)) {
+        int32_t jd;
+        select_rank(lk, li, C, R1, S.hist, S.sh32, S.res, &tkey, &jd);
+    }
+    return tkey;
+}
+
+// Filter: one CTA per score chunk; surely-selected entries become bitmap
+// bits, the rest of the widened bin d1 is appended to the sequence's
+// candidate list, and the keys inside bin d1 feed a histogram of bits 20..10.
+__global__ void __launch_bounds__(kSelThreads, 3) topk_filter_kernel(TopkDecodeArgs a) {
+    __shared__ SelSmem S;
+    const int b = blockIdx.y, c = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n = clamp_n(a.n, b, a.Ncap);
+    const int k = a.k;
+    if (n <= k) {
+        if (c == 0) {
+            int32_t* idx = a.idx + (size_t)b * k;
+            for (int i = tid; i < k; i += blockDim.x) idx[i] = i < n ? i : -1;
+            if (tid == 0) a.cnt[b] = n;
+        }
+        return;
+    }
+    const int row0 = c * a.chunk;
+    const int row1 = min(row0 + a.chunk, n);
+    const uint32_t* keys = a.keys + (size_t)b * a.Ncap;
+
+    // issue every load first: the first pass's keys, the histogram, the error bounds
+    uint32_t kr[kSelKPT];
+#pragma unroll
+    for (int i = 0; i < kSelKPT; ++i) {
+        const int row = row0 + i * kSelThreads + tid;
+        kr[i] = row < row1 ? __ldcg(keys + row) : 0u;
+    }
+    uint32_t hv[kBins / kSelThreads];
+#pragma unroll
+    for (int u = 0; u < kBins / kSelThreads; ++u) hv[u] = __ldcg(a.hist1 + (size_t)b * kBins + u * kSelThreads + tid);
+    float e = 0.f;
+    for (int q = tid; q < a.nchunks; q += kSelThreads) e = fmaxf(e, __ldcg(a.emax_part + (size_t)b * a.nchunks + q));
+    uint32_t* ck = a.cand_key + (size_t)b * a.Ncap;
+    int32_t* ci = a.cand_idx + (size_t)b * a.Ncap;
+    uint32_t* tot = a.totals + (size_t)b * kTotals;
+    uint32_t* bm = a.bitmap + (size_t)b * a.Wcap;
+    uint32_t* h2 = a.hist2 + (size_t)b * kBins;
+#pragma unroll
+    for (int u = 0; u < kBins / kSelThreads; ++u) S.hist[u * kSelThreads + tid] = hv[u];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) e = fmaxf(e, __shfl_xor_sync(0xFFFFFFFFu, e, o));
+    if (lane == 0) S.red[warp] = e;
+    __syncthreads();
+    float E = 0.f;
+#pragma unroll
+    for (int w = 0; w < kSelThreads / 32; ++w) E = fmaxf(E, S.red[w]);
+    int d1;
+    uint32_t above1;
+    find_digit_desc<kBins>(S.hist, (uint32_t)k, S.sh32, &d1, &above1, S.res);
+    if (d1 < 0) d1 = 0;  // cannot happen: the histogram counts all n > k keys
+    const FilterBounds fb = filter_bounds(d1, E);
+    if (c == 0 && tid == 0) {  // the resolve reads these from here
+        tot[kTotBin] = (uint32_t)d1;
+        tot[kTotE] = __float_as_uint(E);
+        tot[kTotAbove] = above1;
+    }
+
+    uint32_t nin = 0;
+    for (int p0 = row0; p0 < row1; p0 += kSelKPT * kSelThreads) {  // passes of up to 4096 rows
+        if (p0 != row0) {
+#pragma unroll
+            for (int i = 0; i < kSelKPT; ++i) {
+                const int row = p0 + i * kSelThreads + tid;
+                kr[i] = row < row1 ? __ldcg(keys + row) : 0u;
+            }
+        }
+        uint32_t cmask = 0, mycnt = 0;
+#pragma unroll
+        for (int i = 0; i < kSelKPT; ++i) {
+            const int row = p0 + i * kSelThreads + tid;
+            const int wrow = p0 + i * kSelThreads + warp * 32;  // this warp's 32 consecutive rows
+            const float sv = key_to_float(kr[i]);
+            const bool valid = row < row1;
+            const bool sel = valid && sv > fb.in_above;
+            const bool cand = valid && !sel && sv >= fb.c_lo;
+            const uint32_t selm = __ballot_sync(0xFFFFFFFFu, sel);
+            if (lane == 0 && wrow < row1) bm[wrow >> 5] = selm;  // row0 is a multiple of 32
+            nin += __popc(selm);
+            if (cand) {
+                cmask |= 1u << i;
+                ++mycnt;
+                if ((int)(kr[i] >> 21) == d1) atomicAdd(h2 + ((kr[i] >> 10) & (kBins - 1)), 1u);
+            }
+        }
+        uint32_t total;
+        uint32_t pos = block_exclusive_scan(mycnt, S.sh32, &total);
+        if (total) {  // one append per pass to the sequence's candidate list
+            if (tid == 0) S.last = atomicAdd(&tot[kTotCand], total);
+            __syncthreads();
+            pos += S.last;
+            if (pos + mycnt > (uint32_t)a.Ncap) {  // cannot happen: at most n candidates
+                flag(DEV_LEN);
+                mycnt = 0;
+                cmask = 0;
+            }
+#pragma unroll
+            for (int i = 0; i < kSelKPT; ++i) {
+                if ((cmask >> i) & 1u) {
+                    ck[pos] = kr[i];
+                    ci[pos] = p0 + i * kSelThreads + tid;
+                    ++pos;
+                }
+            }
+            __syncthreads();  // S.last is reused
+        }
+    }
+    if (lane == 0) S.amb_key[warp] = nin;  // (scratch) the warp's sure-ins: every lane counted the ballots
+    __syncthreads();
+    if (tid == 0) {  // every chunk writes its count, empty chunks too
+        uint32_t s_in = 0;
+        for (int w = 0; w < kSelThreads / 32; ++w) s_in += S.amb_key[w];
+        a.chunk_in[(size_t)b * a.nchunks + c] = s_in;
+    }
+}
+
+// One CTA of 1024 threads per sequence: finds t~ among the filter's
+// candidates, rescores the band exactly, ranks it by (s, -j), adds the
+// winners to the selection bitmap and gives every chunk the output position
+// of its first selected entry.
+__global__ void __launch_bounds__(kResThreads, 1) topk_resolve_kernel(TopkDecodeArgs a) {
+    extern __shared__ __align__(16) uint32_t csm[];  // [kSelCap] keys, [kSelCap] indices
+    __shared__ SelSmem S;
+    const int b = blockIdx.x;
+    const int tid = threadIdx.x;
+    const int n = clamp_n(a.n, b, a.Ncap);
+    const int k = a.k;
+    if (n <= k) return;  // the filter wrote the whole answer
+    // issue every load first
+    const uint32_t* tot = a.totals + (size_t)b * kTotals;
+    uint32_t C = __ldcg(tot + kTotCand);
+    const int d1 = (int)__ldcg(tot + kTotBin);
+    const float E = __uint_as_float(__ldcg(tot + kTotE));
+    const uint32_t above1 = __ldcg(tot + kTotAbove);
+    const uint32_t cin = tid < a.nchunks ? __ldcg(a.chunk_in + (size_t)b * a.nchunks + tid) : 0u;
+    const uint32_t h2a = __ldcg(a.hist2 + (size_t)b * kBins + tid);
+    const uint32_t h2b = __ldcg(a.hist2 + (size_t)b * kBins + kResThreads + tid);
+    load_q2(S.q2, a.q_idx + (size_t)b * 64);
+    if (C > (uint32_t)a.Ncap) {
+        if (tid == 0) flag(DEV_LEN);
+        C = a.Ncap;
+    }
     const bool fits = C <= (uint32_t)kSelCap;
     const uint32_t* gk = a.cand_key + (size_t)b * a.Ncap;
     const int32_t* gi = a.cand_idx + (size_t)b * a.Ncap;
     // the candidate list: copied to shared memory when it fits, else read in place
-    uint32_t* lk = fits ? csm : const_cast<uint32_t*>(gk);
-    int32_t* li = fits ? reinterpret_cast<int32_t*>(csm + kSelCap) : const_cast<int32_t*>(gi);
-    const int tid = threadIdx.x;
-    uint32_t* bm = a.bitmap + (size_t)b * a.Wcap;
+    const uint32_t* lk = fits ? csm : gk;
+    const int32_t* li = fits ? reinterpret_cast<const int32_t*>(csm + kSelCap) : gi;
     if (fits) {
         constexpr int U = 4;  // loads first, then the stores
         for (uint32_t e0 = 0; e0 < C; e0 += U * kResThreads) {
@@ -526,13 +675,15 @@ __device__ __noinline__ void resolve_candidates(const TopkDecodeArgs& a, SelSmem
             }
         }
     }
-    __syncthreads();
+    S.hist[tid] = h2a;
+    S.hist[kResThreads + tid] = h2b;
+    if (tid == 0) S.amb_cnt = 0;
+    uint32_t A;
+    block_exclusive_scan(cin, S.sh32, &A);  // surely selected entries of the sequence
+    const uint32_t R1 = (uint32_t)k - A;    // rank of t~ among the candidates (>= 1)
+    const uint32_t K2 = (uint32_t)k - above1;
 
-    uint32_t tkey;
-    if (!rank_in_bin(lk, C, R1, d1, S.hist, S.sh32, S.res, &tkey)) {
-        int32_t jd;
-        select_rank(lk, li, C, R1, S.hist, S.sh32, S.res, &tkey, &jd);
-    }
+    const uint32_t tkey = find_threshold(lk, li, C, R1, d1, K2, S);
     const float t = key_to_float(tkey);
     const float e2 = __fmul_ru(2.f, E);
     const float band_hi = __fadd_ru(t, e2), band_lo = __fsub_rd(t, e2);
@@ -540,7 +691,9 @@ __device__ __noinline__ void resolve_candidates(const TopkDecodeArgs& a, SelSmem
     // the band list (global, used when the band is large)
     uint32_t* gak = a.amb_key + (size_t)b * a.Ncap;
     int32_t* gai = a.amb_idx + (size_t)b * a.Ncap;
+    __syncthreads();  // S.amb_key held the fine bin
     uint32_t my_in2 = 0;
+#pragma unroll 1
     for (uint32_t i = tid; i < C; i += kResThreads) {
         const float sv = key_to_float(lk[i]);
         if (sv > band_hi) {
@@ -563,7 +716,7 @@ __device__ __noinline__ void resolve_candidates(const TopkDecodeArgs& a, SelSmem
     const uint32_t R2 = R1 - in2;  // winners to take from the band (1 <= R2 <= na)
     // the exact cut of the band: a member wins iff (key, -j) >= (T2, -jmax2)
     if (na <= (uint32_t)kResThreads) {
-        if (tid < na) {
+        if ((uint32_t)tid < na) {
             const uint32_t mk = S.amb_key[tid];
             const int32_t mj = S.amb_idx[tid];
             uint32_t rank = 0;
@@ -590,223 +743,69 @@ __device__ __noinline__ void resolve_candidates(const TopkDecodeArgs& a, SelSmem
     }
     const uint32_t T2 = S.T2;
     const int32_t jmax2 = S.jmax2;
-    // winners of the candidates -> a list in shared memory (S.hist, R1 <= 2048
-    // of them) when it fits, else straight into the global bitmap
-    const bool wlist = R1 <= (uint32_t)kBins;
-    if (tid == 0) S.wcnt = 0;
+    // winners of the candidates: into the bitmap, and counted per chunk (S.hist)
+    uint32_t* bm = a.bitmap + (size_t)b * a.Wcap;
+    uint32_t* wc = S.hist;
+    for (int i = tid; i < kBins; i += kResThreads) wc[i] = 0;
     __syncthreads();
+#pragma unroll 1
     for (uint32_t i = tid; i < C; i += kResThreads) {
         if (key_to_float(lk[i]) > band_hi) {
             const int32_t j = li[i];
-            if (wlist) {
-                const uint32_t p = atom_add_shared(&S.wcnt, 1u);
-                if (p < (uint32_t)kBins) S.hist[p] = (uint32_t)j;
-            } else {
-                atomicOr(&bm[j >> 5], 1u << (j & 31));
-            }
+            atomicOr(&bm[j >> 5], 1u << (j & 31));
+            red_add_shared(&wc[j / a.chunk], 1u);
         }
     }
+#pragma unroll 1
     for (uint32_t i = tid; i < na; i += kResThreads) {
         const uint32_t kk = na <= (uint32_t)kResThreads ? S.amb_key[i] : __ldcg(gak + i);
         const int32_t j = na <= (uint32_t)kResThreads ? S.amb_idx[i] : __ldcg(gai + i);
         if (kk > T2 || (kk == T2 && j <= jmax2)) {
-            if (wlist) {
-                const uint32_t p = atom_add_shared(&S.wcnt, 1u);
-                if (p < (uint32_t)kBins) S.hist[p] = (uint32_t)j;
-            } else {
-                atomicOr(&bm[j >> 5], 1u << (j & 31));
-            }
+            atomicOr(&bm[j >> 5], 1u << (j & 31));
+            red_add_shared(&wc[j / a.chunk], 1u);
         }
     }
     __syncthreads();
-}
-
-// Filter: one CTA per score chunk; surely-selected entries become bitmap
-// bits, candidates go to the chunk's own slot.
-__global__ void __launch_bounds__(kSelThreads, 3) topk_filter_kernel(TopkDecodeArgs a) {
-    __shared__ SelSmem S;
-    const int b = blockIdx.y, c = blockIdx.x;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int n = clamp_n(a.n, b, a.Ncap);
-    const int k = a.k;
-    if (n <= k) {
-        if (c == 0) {
-            int32_t* idx = a.idx + (size_t)b * k;
-            for (int i = tid; i < k; i += blockDim.x) idx[i] = i < n ? i : -1;
-            if (tid == 0) a.cnt[b] = n;
-        }
-        return;
-    }
-    const int row0 = c * a.chunk;
-    const int row1 = min(row0 + a.chunk, n);
-
-    // ---- filter: issue every load first (histogram, error bound, keys)
-    uint32_t hv[kBins / kSelThreads];
-#pragma unroll
-    for (int u = 0; u < kBins / kSelThreads; ++u) hv[u] = __ldcg(a.hist1 + (size_t)b * kBins + u * kSelThreads + tid);
-    float e = 0.f;
-    for (int q = tid; q < a.nchunks; q += kSelThreads) e = fmaxf(e, __ldcg(a.emax_part + (size_t)b * a.nchunks + q));
-    const uint32_t* keys = a.keys + (size_t)b * a.Ncap;
-    uint32_t* ck = a.cand_key + (size_t)b * a.Ncap;
-    int32_t* ci = a.cand_idx + (size_t)b * a.Ncap;
-    uint32_t* tot4 = a.totals + (size_t)b * 4;
-    uint32_t* bm = a.bitmap + (size_t)b * a.Wcap;
-#pragma unroll
-    for (int u = 0; u < kBins / kSelThreads; ++u) S.hist[u * kSelThreads + tid] = hv[u];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) e = fmaxf(e, __shfl_xor_sync(0xFFFFFFFFu, e, o));
-    if (lane == 0) S.red[warp] = e;
-    __syncthreads();
-    float E = 0.f;
-#pragma unroll
-    for (int w = 0; w < kSelThreads / 32; ++w) E = fmaxf(E, S.red[w]);
-    int d1;
-    uint32_t above1;
-    find_digit_desc<kBins>(S.hist, (uint32_t)k, S.sh32, &d1, &above1, S.res);
-    if (d1 < 0) d1 = 0;  // cannot happen: the histogram counts all n > k keys
-    const FilterBounds fb = filter_bounds(d1, E);
-    if (c == 0 && tid == 0) {  // the resolve reads the bin and the bound from here
-        tot4[2] = (uint32_t)d1;
-        tot4[3] = __float_as_uint(E);
-    }
-
-    uint32_t nin = 0;
-    for (int p0 = row0; p0 < row1; p0 += kSelKPT * kSelThreads) {  // passes of up to 4096 rows
-        uint32_t kr[kSelKPT];
-#pragma unroll
-        for (int i = 0; i < kSelKPT; ++i) {
-            const int row = p0 + i * kSelThreads + tid;
-            kr[i] = row < row1 ? __ldcg(keys + row) : 0u;
-        }
-        uint32_t cmask = 0, mycnt = 0;
-#pragma unroll
-        for (int i = 0; i < kSelKPT; ++i) {
-            const int row = p0 + i * kSelThreads + tid;
-            const int wrow = p0 + i * kSelThreads + warp * 32;  // this warp's 32 consecutive rows
-            const float sv = key_to_float(kr[i]);
-            const bool valid = row < row1;
-            const bool sel = valid && sv > fb.in_above;
-            const bool cand = valid && !sel && sv >= fb.c_lo;
-            const uint32_t selm = __ballot_sync(0xFFFFFFFFu, sel);
-            if (lane == 0 && wrow < row1) bm[wrow >> 5] = selm;  // row0 is a multiple of 32
-            nin += __popc(selm);
-            if (cand) {
-                cmask |= 1u << i;
-                ++mycnt;
-            }
-        }
-        uint32_t tot;
-        uint32_t pos = block_exclusive_scan(mycnt, S.sh32, &tot);
-        if (tot) {  // one append per pass to the sequence's candidate list
-            if (tid == 0) S.last = atomicAdd(&tot4[0], tot);
-            __syncthreads();
-            pos += S.last;
-            if (pos + mycnt > (uint32_t)a.Ncap) {  // cannot happen: at most n candidates
-                flag(DEV_LEN);
-                mycnt = 0;
-            }
-#pragma unroll
-            for (int i = 0; i < kSelKPT; ++i) {
-                if ((cmask >> i) & 1u) {
-                    ck[pos] = kr[i];
-                    ci[pos] = p0 + i * kSelThreads + tid;
-                    ++pos;
-                }
-            }
-            __syncthreads();  // S.last is reused
-        }
-    }
-    if (lane == 0) S.amb_key[warp] = nin;  // (scratch) per-warp sure-in counts
-    __syncthreads();
-    if (tid == 0) {
-        uint32_t s_in = 0;
-        for (int w = 0; w < kSelThreads / 32; ++w) s_in += S.amb_key[w];
-        if (s_in) atomicAdd(&tot4[1], s_in);
-    }
-}
-
-// One CTA of 1024 threads per sequence: gathers the filter's candidates,
-// finds t~ among them, rescores the band exactly, ranks it by (s, -j), marks
-// the winners and compacts the selection bitmap into ascending indices.
-__global__ void __launch_bounds__(kResThreads, 1) topk_resolve_kernel(TopkDecodeArgs a) {
-    extern __shared__ __align__(16) uint32_t csm[];  // [kSelCap] keys, [kSelCap] indices
-    __shared__ SelSmem S;
-    const int b = blockIdx.x;
-    const int tid = threadIdx.x;
-    const int n = clamp_n(a.n, b, a.Ncap);
-    const int k = a.k;
-    if (n <= k) {
-        int32_t* idx = a.idx + (size_t)b * k;
-        for (int i = tid; i < k; i += blockDim.x) idx[i] = i < n ? i : -1;
-        if (tid == 0) a.cnt[b] = n;
-        return;
-    }
-    uint32_t* bm = a.bitmap + (size_t)b * a.Wcap;
-    load_q2(S.q2, a.q_idx + (size_t)b * 64);
-    if (tid == 0) {
-        S.amb_cnt = 0;
-        S.in2 = 0;
-    }
-    const uint32_t* tot4 = a.totals + (size_t)b * 4;
-    uint32_t C = __ldcg(tot4 + 0);
-    const uint32_t A = __ldcg(tot4 + 1);
-    const int d1 = (int)__ldcg(tot4 + 2);
-    const float E = __uint_as_float(__ldcg(tot4 + 3));
-    if (C > (uint32_t)a.Ncap) {
-        if (tid == 0) flag(DEV_LEN);
-        C = a.Ncap;
-    }
-    __syncthreads();
-    const uint32_t R1 = (uint32_t)k - A;  // rank of t~ among the candidates (>= 1)
-    resolve_candidates(a, S, csm, b, C, R1, d1, E);
-    __syncthreads();
-    // candidates are consumed: csm now holds a shared bitmap of the winners
-    // (when it fits next to an output stage of k indices)
-    const int nwords = (n + 31) >> 5;
-    const bool sbm = S.wcnt > 0 && R1 <= (uint32_t)kBins && (size_t)nwords <= (size_t)kSelCap * 2;
-    const bool was_list = R1 <= (uint32_t)kBins;
-    uint32_t* extra = nullptr;
-    if (was_list) {
-        if (sbm) {
-            for (int w = tid; w < nwords; w += kResThreads) csm[w] = 0u;
-            __syncthreads();
-            const uint32_t nw_ = S.wcnt < (uint32_t)kBins ? S.wcnt : (uint32_t)kBins;
-            for (uint32_t i = tid; i < nw_; i += kResThreads) {
-                const uint32_t j = S.hist[i];
-                red_or_shared(&csm[j >> 5], 1u << (j & 31));
-            }
-            extra = csm;
-        } else {
-            const uint32_t nw_ = S.wcnt < (uint32_t)kBins ? S.wcnt : (uint32_t)kBins;
-            for (uint32_t i = tid; i < nw_; i += kResThreads) {
-                const uint32_t j = S.hist[i];
-                atomicOr(&bm[j >> 5], 1u << (j & 31));
-            }
-            __threadfence_block();
-        }
-        __syncthreads();
-    }
-    // shared layout for the compaction: [winner bitmap][staging][output stage of k]
-    const size_t base = extra ? (size_t)nwords : 0;
-    constexpr size_t stg = (size_t)kResThreads * (kCompPer + 1);
-    static_assert(stg <= (size_t)kSelCap * 2, "compaction staging must fit the shared area");
+    // output position of every chunk's first selected entry
+    const uint32_t v = tid < a.nchunks ? cin + wc[tid] : 0u;
     uint32_t total;
-    if (base + stg <= (size_t)kSelCap * 2) {
-        uint32_t* ostage = base + stg + (size_t)k <= (size_t)kSelCap * 2 ? csm + base + stg : nullptr;
-        compact_bitmap(bm, extra, nwords, a.idx + (size_t)b * k, (uint32_t)k, ostage, csm + base, S.sh32, &total);
-    } else {
-        // no room next to the winner bitmap: fold it into the global one first
-        // (extra is set here: without it base is 0 and the staging fits)
-        if (extra)
-            for (int w = tid; w < nwords; w += kResThreads)
-                if (extra[w]) atomicOr(&bm[w], extra[w]);
-        __threadfence_block();
-        __syncthreads();
-        compact_bitmap(bm, nullptr, nwords, a.idx + (size_t)b * k, (uint32_t)k, nullptr, csm, S.sh32, &total);
-    }
+    const uint32_t pos = block_exclusive_scan(v, S.sh32, &total);
+    if (tid < a.nchunks) a.chunk_pos[(size_t)b * a.nchunks + tid] = pos;
     if (tid == 0) {
         if (total != (uint32_t)k) flag(DEV_LEN);  // cannot happen
         a.cnt[b] = k;
+    }
+}
+
+// Emit: one CTA per (chunk, sequence) writes its chunk's selected indices,
+// ascending, from its output position on.
+constexpr int kEmitThreads = 256;
+__global__ void __launch_bounds__(kEmitThreads) topk_emit_kernel(TopkDecodeArgs a) {
+    __shared__ uint32_t sh32[32];
+    const int b = blockIdx.y, c = blockIdx.x;
+    const int n = clamp_n(a.n, b, a.Ncap);
+    if (n <= a.k) return;
+    const int row0 = c * a.chunk;
+    const int row1 = min(row0 + a.chunk, n);
+    if (row0 >= row1) return;
+    const uint32_t* bm = a.bitmap + (size_t)b * a.Wcap;
+    int32_t* out = a.idx + (size_t)b * a.k;
+    const int w0 = row0 >> 5, w1 = (row1 + 31) >> 5;
+    uint32_t pos = __ldcg(a.chunk_pos + (size_t)b * a.nchunks + c);
+#pragma unroll 1
+    for (int wb = w0; wb < w1; wb += kEmitThreads) {  // block-uniform trip count
+        const int w = wb + threadIdx.x;
+        uint32_t word = w < w1 ? __ldcg(bm + w) : 0u;
+        uint32_t total;
+        uint32_t p = pos + block_exclusive_scan(__popc(word), sh32, &total);
+        while (word) {
+            const int bit = __ffs(word) - 1;
+            word &= word - 1;
+            if (p < (uint32_t)a.k) out[p] = w * 32 + bit;
+            else flag(DEV_LEN);  // cannot happen: exactly k bits are set
+            ++p;
+        }
+        pos += total;
     }
 }
 
