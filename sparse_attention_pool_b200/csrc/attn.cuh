@@ -87,6 +87,8 @@ template <int NW, bool GATHER, bool FP8, int ST, bool CLUSTER>
 __global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
     using L = AttnSmem<NW, GATHER, FP8, ST>;
     extern __shared__ __align__(128) uint8_t smem[];
+    pdl_wait();
+    pdl_release();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     // grid: (splits, queries) in a cluster launch, else (queries, splits)
     const int split = CLUSTER ? blockIdx.x : blockIdx.y;
@@ -430,6 +432,8 @@ __global__ void __launch_bounds__(kCombThreads) attn_combine_kernel(const float*
                                                                     int splits, int H, uint16_t* out, float* lse) {
     __shared__ float4 red[kCombThreads / 32][32];
     __shared__ float wred[kCombThreads / 32];
+    pdl_wait();
+    pdl_release();
     const int bh = blockIdx.x;  // bq * H + h
     const int bq = bh / H, h = bh - bq * H;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;

@@ -184,6 +184,16 @@ __device__ __forceinline__ void red_or_shared(uint32_t* p, uint32_t v) {
     asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while its predecessor on the stream is still
+// running; pdl_wait() returns once that predecessor has completed and its
+// writes are visible (for an ordinary launch it returns at once).  Every
+// kernel calls it before it touches global memory another kernel may write
+// or read, and before any early return, so completion stays transitive along
+// a chain.  pdl_release() lets the next kernel on the stream begin launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------ block scans --
 // Exclusive prefix sum over the block (blockDim.x multiple of 32, <= 1024).
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* sh32, uint32_t* total) {

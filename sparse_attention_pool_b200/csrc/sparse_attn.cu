@@ -12,6 +12,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "../../include/sparse_attn.h"
 #include "attn.cuh"
@@ -37,6 +38,45 @@ inline void stage_mark(int stage, int which, cudaStream_t st) {
         cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal);
     else
         cudaEventRecord(ev, st);
+}
+
+// Programmatic dependent launch joins the library's own consecutive kernels
+// of one call (never a call's first kernel, whose predecessor may be any
+// stream work), and is off while stage events are set: their record nodes
+// sit between the kernels.
+bool pdl_on() {
+    for (const auto& e : g_stage_ev)
+        if (e[0] || e[1]) return false;
+    return true;
+}
+
+// cudaLaunchKernelEx with optional programmatic stream serialization and an
+// optional cluster shape.
+template <typename... P, typename... A>
+cudaError_t launch_k(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                     unsigned cluster_x, A&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    unsigned na = 0;
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    if (cluster_x > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = cluster_x;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
 }
 
 sa_status fail(sa_status s, const char* fmt, ...) {
@@ -233,7 +273,7 @@ size_t attn_partial_bytes(long long BQ, int splits, int H) {
 
 // ------------------------------------------------------------ launchers ----
 template <int NW, bool G, bool F, int ST, bool CL>
-sa_status launch_attn_t(const sa::AttnArgs& a, dim3 grid, cudaStream_t st) {
+sa_status launch_attn_t(const sa::AttnArgs& a, dim3 grid, cudaStream_t st, bool pdl) {
     using L = sa::AttnSmem<NW, G, F, ST>;
     static std::atomic<uint64_t> init{0};
     if (!attr_done(init)) {
@@ -241,54 +281,49 @@ sa_status launch_attn_t(const sa::AttnArgs& a, dim3 grid, cudaStream_t st) {
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal));
         attr_set(init);
     }
-    if (CL) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = grid;
-        cfg.blockDim = dim3(NW * 32);
-        cfg.dynamicSmemBytes = L::kTotal;
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = sa::kAttnCluster;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        SA_CUDA(cudaLaunchKernelEx(&cfg, sa::attn_split_kernel<NW, G, F, ST, CL>, a));
-    } else {
-        sa::attn_split_kernel<NW, G, F, ST, CL><<<grid, NW * 32, L::kTotal, st>>>(a);
-    }
+    SA_CUDA(launch_k(sa::attn_split_kernel<NW, G, F, ST, CL>, grid, dim3(NW * 32), L::kTotal, st, pdl,
+                     CL ? (unsigned)sa::kAttnCluster : 1u, a));
     SA_LAUNCHED();
     return SA_OK;
 }
 
 template <int NW, int ST, bool CL>
-sa_status launch_attn_nw(const sa::AttnArgs& a, bool gather, bool fp8, dim3 grid, cudaStream_t st) {
+sa_status launch_attn_nw(const sa::AttnArgs& a, bool gather, bool fp8, dim3 grid, cudaStream_t st, bool pdl) {
     if (gather)
-        return fp8 ? launch_attn_t<NW, true, true, ST, CL>(a, grid, st) : launch_attn_t<NW, true, false, ST, CL>(a, grid, st);
-    return fp8 ? launch_attn_t<NW, false, true, ST, CL>(a, grid, st) : launch_attn_t<NW, false, false, ST, CL>(a, grid, st);
+        return fp8 ? launch_attn_t<NW, true, true, ST, CL>(a, grid, st, pdl)
+                   : launch_attn_t<NW, true, false, ST, CL>(a, grid, st, pdl);
+    return fp8 ? launch_attn_t<NW, false, true, ST, CL>(a, grid, st, pdl)
+               : launch_attn_t<NW, false, false, ST, CL>(a, grid, st, pdl);
 }
 
 // Splits of up to 4 tiles keep all of them in flight (4 stages); longer
 // lists (prefill) stream through a 2-stage pipeline.  A query split exactly
 // kAttnCluster ways merges inside a cluster.
-sa_status launch_attn(const sa::AttnArgs& a, bool gather, bool fp8, long long BQ, cudaStream_t st) {
+sa_status launch_attn(const sa::AttnArgs& a, bool gather, bool fp8, long long BQ, cudaStream_t st, bool pdl) {
     const bool cl = a.splits == sa::kAttnCluster && BQ <= 65535;
     if (BQ > 2147483647LL || a.splits > 65535) return fail(SA_ERR_INVALID_ARG, "too many queries or splits");
     const dim3 grid = cl ? dim3(a.splits, (unsigned)BQ) : dim3((unsigned)BQ, a.splits);
     const bool deep = a.tiles_per_split >= 2 && a.tiles_per_split <= 4;
     if (a.H <= 64) {
-        if (cl) return deep ? launch_attn_nw<4, 4, true>(a, gather, fp8, grid, st) : launch_attn_nw<4, 2, true>(a, gather, fp8, grid, st);
-        return deep ? launch_attn_nw<4, 4, false>(a, gather, fp8, grid, st) : launch_attn_nw<4, 2, false>(a, gather, fp8, grid, st);
+        if (cl)
+            return deep ? launch_attn_nw<4, 4, true>(a, gather, fp8, grid, st, pdl)
+                        : launch_attn_nw<4, 2, true>(a, gather, fp8, grid, st, pdl);
+        return deep ? launch_attn_nw<4, 4, false>(a, gather, fp8, grid, st, pdl)
+                    : launch_attn_nw<4, 2, false>(a, gather, fp8, grid, st, pdl);
     }
-    if (cl) return deep ? launch_attn_nw<8, 4, true>(a, gather, fp8, grid, st) : launch_attn_nw<8, 2, true>(a, gather, fp8, grid, st);
-    return deep ? launch_attn_nw<8, 4, false>(a, gather, fp8, grid, st) : launch_attn_nw<8, 2, false>(a, gather, fp8, grid, st);
+    if (cl)
+        return deep ? launch_attn_nw<8, 4, true>(a, gather, fp8, grid, st, pdl)
+                    : launch_attn_nw<8, 2, true>(a, gather, fp8, grid, st, pdl);
+    return deep ? launch_attn_nw<8, 4, false>(a, gather, fp8, grid, st, pdl)
+                : launch_attn_nw<8, 2, false>(a, gather, fp8, grid, st, pdl);
 }
 
+// The merge follows its split kernel on the same stream: always chained.
 sa_status launch_combine(const float* po, const float* pl, int splits, int H, long long BQ, uint16_t* out, float* lse,
                          cudaStream_t st) {
     if (BQ * H > 2147483647LL) return fail(SA_ERR_INVALID_ARG, "too many queries");
-    sa::attn_combine_kernel<<<(unsigned)(BQ * H), sa::kCombThreads, 0, st>>>(po, pl, splits, H, out, lse);
+    SA_CUDA(launch_k(sa::attn_combine_kernel, dim3((unsigned)(BQ * H)), dim3(sa::kCombThreads), 0, st, pdl_on(), 1u,
+                     po, pl, splits, H, out, lse));
     SA_LAUNCHED();
     return SA_OK;
 }
@@ -319,7 +354,7 @@ sa_status side_stream(SideStream** out) {
 // Shared body of csa_sparse_attn / hca_dense_attn / the hybrid calls.
 sa_status run_attn(const void* q, int Tq, int H, const sa_cache* c, bool gather, const int32_t* idx,
                    const int32_t* cnt, int kmax, const int32_t* pos, float scale, void* out, float* lse, void* ws,
-                   size_t ws_off, cudaStream_t st) {
+                   size_t ws_off, cudaStream_t st, bool chained = false) {
     const long long BQ = (long long)c->B * Tq;
     const bool prefill = (Tq > 1) || (pos != nullptr);
     const Split sp = attn_split(gather ? kmax : c->Ncap, prefill, gather);
@@ -350,7 +385,7 @@ sa_status run_attn(const void* q, int Tq, int H, const sa_cache* c, bool gather,
         a.part_o = reinterpret_cast<float*>(base);
         a.part_lse = reinterpret_cast<float*>(base + up256((size_t)BQ * sp.splits * H * 128 * 4));
     }
-    sa_status r = launch_attn(a, gather, c->dtype == SA_FP8_E4M3, BQ, st);
+    sa_status r = launch_attn(a, gather, c->dtype == SA_FP8_E4M3, BQ, st, chained && pdl_on());
     if (r != SA_OK) return r;
     // a query split kAttnCluster ways was merged inside its cluster
     if (sp.splits > 1 && !(sp.splits == sa::kAttnCluster && BQ <= 65535))
@@ -414,11 +449,12 @@ sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* 
     stage_mark(SA_STAGE_TOPK_SELECT, 0, st);
     // a sequence with n <= k visible entries (every one, when Ncap is 0) is
     // answered by the filter's first CTA; the other kernels skip it
-    sa::topk_filter_kernel<<<dim3(a.nchunks, B), sa::kSelThreads, 0, st>>>(a);
+    const bool pdl = pdl_on();
+    SA_CUDA(launch_k(sa::topk_filter_kernel, dim3(a.nchunks, B), dim3(sa::kSelThreads), 0, st, pdl && Ncap > 0, 1u, a));
     SA_LAUNCHED();
-    sa::topk_resolve_kernel<<<B, sa::kResThreads, sa::kSelSmem, st>>>(a);
+    SA_CUDA(launch_k(sa::topk_resolve_kernel, dim3(B), dim3(sa::kResThreads), sa::kSelSmem, st, pdl, 1u, a));
     SA_LAUNCHED();
-    sa::topk_emit_kernel<<<dim3(a.nchunks, B), sa::kEmitThreads, 0, st>>>(a);
+    SA_CUDA(launch_k(sa::topk_emit_kernel, dim3(a.nchunks, B), dim3(sa::kEmitThreads), 0, st, pdl, 1u, a));
     SA_LAUNCHED();
     stage_mark(SA_STAGE_TOPK_SELECT, 1, st);
     return SA_OK;
@@ -770,7 +806,7 @@ sa_status hybrid_attn_decode(const void* q, const void* q_idx, int32_t H, const 
     r = run_topk_decode(q_idx, csa, k, idx, cnt, ws, w, st, fork_hca);
     if (r != SA_OK) return r;
     stage_mark(SA_STAGE_CSA_ATTN, 0, st);
-    r = run_attn(q, 1, H, csa, true, idx, cnt, k, nullptr, scale, out_csa, lse_csa, ws, w.total, st);
+    r = run_attn(q, 1, H, csa, true, idx, cnt, k, nullptr, scale, out_csa, lse_csa, ws, w.total, st, true);
     if (r != SA_OK) return r;
     stage_mark(SA_STAGE_CSA_ATTN, 1, st);
     SA_CUDA(cudaStreamWaitEvent(st, side->join, 0));

@@ -130,6 +130,8 @@ __global__ void __launch_bounds__(kScThreads, 3)
     __shared__ float s_emax[kScThreads / 32];
     __shared__ uint32_t hist[kBins];  // top 11 key bits of this CTA's rows
 
+    pdl_wait();
+    pdl_release();
     const int b = blockIdx.y;
     const int n = clamp_n(a.n, b, a.Ncap);
     if (n <= a.k) return;  // everything visible is selected; nothing to score
@@ -511,6 +513,8 @@ __device__ __noinline__ uint32_t find_threshold(const uint32_t* lk, const int32_
 // candidate list, and the keys inside bin d1 feed a histogram of bits 20..10.
 __global__ void __launch_bounds__(kSelThreads, 3) topk_filter_kernel(TopkDecodeArgs a) {
     __shared__ SelSmem S;
+    pdl_wait();
+    pdl_release();
     const int b = blockIdx.y, c = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int n = clamp_n(a.n, b, a.Ncap);
@@ -629,6 +633,8 @@ __global__ void __launch_bounds__(kSelThreads, 3) topk_filter_kernel(TopkDecodeA
 __global__ void __launch_bounds__(kResThreads, 1) topk_resolve_kernel(TopkDecodeArgs a) {
     extern __shared__ __align__(16) uint32_t csm[];  // [kSelCap] keys, [kSelCap] indices
     __shared__ SelSmem S;
+    pdl_wait();
+    pdl_release();
     const int b = blockIdx.x;
     const int tid = threadIdx.x;
     const int n = clamp_n(a.n, b, a.Ncap);
@@ -782,6 +788,8 @@ __global__ void __launch_bounds__(kResThreads, 1) topk_resolve_kernel(TopkDecode
 constexpr int kEmitThreads = 256;
 __global__ void __launch_bounds__(kEmitThreads) topk_emit_kernel(TopkDecodeArgs a) {
     __shared__ uint32_t sh32[32];
+    pdl_wait();
+    pdl_release();
     const int b = blockIdx.y, c = blockIdx.x;
     const int n = clamp_n(a.n, b, a.Ncap);
     if (n <= a.k) return;

@@ -60,6 +60,18 @@ def normal_bf16(seed: int, name: str, shape, scale: float = 1.0) -> np.ndarray:
     return out.reshape(shape)
 
 
+def normal_bf16_span(seed: int, name: str, b: int, lo: int, hi: int) -> np.ndarray:
+    """Values [lo, hi) of leading index b's stream of `name`: the same bits that
+    normal_bf16 puts there, drawn from the chunks that cover the span only."""
+    tid = TENSOR_ID[name]
+    c0, c1 = lo // CHUNK, (hi + CHUNK - 1) // CHUNK
+    buf = np.empty(((c1 - c0) * CHUNK,), dtype=np.uint16)
+    for c in range(c0, c1):
+        g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, tid, b, c])))
+        buf[(c - c0) * CHUNK:(c - c0 + 1) * CHUNK] = _round_bf16(g.standard_normal(CHUNK, dtype=np.float32))
+    return buf[lo - c0 * CHUNK:hi - c0 * CHUNK].copy()
+
+
 def ragged_lengths(seed: int, B: int, lo: int, hi: int) -> np.ndarray:
     """B integers uniform in the inclusive range [lo, hi]."""
     g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, TENSOR_ID["len"]])))
