@@ -83,13 +83,18 @@ constexpr int kAttnCluster = 8;  // splits of one query merged in shared memory 
 // CLUSTER: the grid's x dimension is one cluster of kAttnCluster CTAs (the
 // splits of one query); they merge their partials through distributed shared
 // memory instead of a separate combine pass.
-template <int NW, bool GATHER, bool FP8, int ST, bool CLUSTER>
-__global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
+template <int NW, bool GATHER, bool FP8, int ST, bool CLUSTER, int EG>
+__global__ void __launch_bounds__(NW * EG * 32) attn_split_kernel(AttnArgs a) {
     using L = AttnSmem<NW, GATHER, FP8, ST>;
+    constexpr int NT = NW * EG * 32;  // threads
+    constexpr int EPW = kTileN / EG;  // entries of a tile per warp
+    constexpr int NJ = EPW / 8;       // 8-entry n-tiles per warp
+    static_assert(EPW % 16 == 0, "an entry group is whole 16-entry k-steps");
     extern __shared__ __align__(128) uint8_t smem[];
     pdl_wait();
     pdl_release();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int hg = warp % NW, eg = warp / NW;  // head group (16 heads), entry group of each tile
     // grid: (splits, queries) in a cluster launch, else (queries, splits)
     const int split = CLUSTER ? blockIdx.x : blockIdx.y;
     const int bq = CLUSTER ? blockIdx.y : blockIdx.x;
@@ -132,7 +137,7 @@ __global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
 
     const uint16_t* qp = a.q + (size_t)bq * a.H * 128;
     // Q tile: rows >= H are zero
-    for (int c = tid; c < NW * 16 * 16; c += NW * 32) {
+    for (int c = tid; c < NW * 16 * 16; c += NT) {
         const int r = c >> 4, ch = c & 15;
         cp_async16_zfill(sQ + swz(r, ch), qp + (size_t)min(r, a.H - 1) * 128 + ch * 8, r < a.H);
     }
@@ -145,7 +150,7 @@ __global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
 
     // each thread copies CPT 16-byte chunks of one row; a gathered row costs one index load
     constexpr int cpr = FP8 ? 8 : 16;            // 16-byte chunks per row
-    constexpr int TPR = (NW * 32) / kTileN;      // threads per row
+    constexpr int TPR = NT / kTileN;             // threads per row
     constexpr int CPT = cpr / TPR;               // chunks per thread
     static_assert(TPR >= 1 && CPT >= 1 && CPT * TPR == cpr, "tile mapping");
     auto load_tile = [&](int tile, int stage) {
@@ -204,7 +209,7 @@ __global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
             const uint32_t qbase = smem_u32(sQ);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                const int r = warp * 16 + (lane & 15);
+                const int r = hg * 16 + (lane & 15);
                 const int ch = kk * 2 + (lane >> 4);
                 ldsm_x4(qbase + swz(r, ch), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
             }
@@ -218,7 +223,7 @@ __global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
             const uint8_t* rv = sRaw + (stage * 2 + 1) * L::kStageRaw;
             uint8_t* ck = sConv;
             uint8_t* cv = sConv + L::kKVBytes;
-            for (int c = tid; c < kTileN * 16; c += NW * 32) {  // 8 codes -> one 16-byte bf16 chunk
+            for (int c = tid; c < kTileN * 16; c += NT) {  // 8 codes -> one 16-byte bf16 chunk
                 const int r = c >> 4, ch = c & 15;
                 const uint2 wk = *reinterpret_cast<const uint2*>(rk + r * 128 + ch * 8);
                 const uint2 wv = *reinterpret_cast<const uint2*>(rv + r * 128 + ch * 8);
@@ -246,16 +251,16 @@ __global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
             tv = sRaw + (stage * 2 + 1) * L::kStageRaw;
         }
 
-        // S = Q K^T : 16 rows x 64 entries per warp
-        float s[8][4];
+        // S = Q K^T : 16 heads x EPW entries per warp
+        float s[NJ][4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+        for (int j = 0; j < NJ; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
         const uint32_t kbase = smem_u32(tk);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
 #pragma unroll
-            for (int np = 0; np < 4; ++np) {  // pairs of 8-entry n-tiles
-                const int r = np * 16 + (lane & 7) + ((lane >> 4) << 3);
+            for (int np = 0; np < NJ / 2; ++np) {  // pairs of 8-entry n-tiles
+                const int r = eg * EPW + np * 16 + (lane & 7) + ((lane >> 4) << 3);
                 const int ch = kk * 2 + ((lane >> 3) & 1);
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4(kbase + swz(r, ch), b0, b1, b2, b3);
@@ -267,10 +272,10 @@ __global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
         const int* valid = sValid + stage * kTileN;
         float tmax[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int j = 0; j < NJ; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const int col = j * 8 + (lane & 3) * 2 + (e & 1);
+                const int col = eg * EPW + j * 8 + (lane & 3) * 2 + (e & 1);
                 float v = s[j][e];
                 if (FP8) v *= sKs[stage * kTileN + col];
                 v = valid[col] ? v * a.scale_log2 : -INFINITY;
@@ -287,16 +292,16 @@ __global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
             mrow[h] = mnew[h];
         }
         float lsum[2] = {0.f, 0.f};
-        uint32_t pf[4][4];  // P as bf16 A fragments, 4 k-steps of 16 entries
+        uint32_t pf[NJ / 2][4];  // P as bf16 A fragments, k-steps of 16 entries
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < NJ; ++j) {
             float p[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float mm = mnew[e >> 1];
                 p[e] = (mm == -INFINITY) ? 0.f : exp2f(s[j][e] - mm);
                 lsum[e >> 1] += p[e];
-                if (FP8) p[e] *= sVs[stage * kTileN + j * 8 + (lane & 3) * 2 + (e & 1)];
+                if (FP8) p[e] *= sVs[stage * kTileN + eg * EPW + j * 8 + (lane & 3) * 2 + (e & 1)];
             }
             pf[j >> 1][(j & 1) * 2 + 0] = pack_bf16x2(p[0], p[1]);
             pf[j >> 1][(j & 1) * 2 + 1] = pack_bf16x2(p[2], p[3]);
@@ -313,12 +318,12 @@ __global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
         // O += P V
         const uint32_t vbase = smem_u32(tv);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
+        for (int kk = 0; kk < NJ / 2; ++kk) {
             // pf[kk] = {a0, a1, a2, a3} in mma order: rows r0/r1 x entries 16kk + {0..7, 8..15}
             const uint32_t af[4] = {pf[kk][0], pf[kk][1], pf[kk][2], pf[kk][3]};
 #pragma unroll
             for (int dp = 0; dp < 8; ++dp) {  // pairs of 8-dim n-tiles
-                const int r = kk * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+                const int r = eg * EPW + kk * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
                 const int ch = dp * 2 + (lane >> 4);
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4_t(vbase + swz(r, ch), b0, b1, b2, b3);
@@ -336,6 +341,45 @@ __global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
         lrow[h] += __shfl_xor_sync(0xFFFFFFFFu, lrow[h], 1);
         lrow[h] += __shfl_xor_sync(0xFFFFFFFFu, lrow[h], 2);
     }
+    if (EG > 1) {
+        // merge the entry groups' softmax states into the group-0 warps (the
+        // K/V buffers are free now); equal fragment layouts: lane-wise merge
+        static_assert(L::kMeta - L::kRaw >= (EG - 1) * NW * 17 * 32 * 16, "entry-group merge buffer");
+        float4* mb = reinterpret_cast<float4*>(smem + L::kRaw);
+        __syncthreads();
+        if (eg > 0) {
+            float4* my = mb + (size_t)((eg - 1) * NW + hg) * 17 * 32 + lane;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) my[i * 32] = make_float4(o[i][0], o[i][1], o[i][2], o[i][3]);
+            my[16 * 32] = make_float4(mrow[0], mrow[1], lrow[0], lrow[1]);
+        }
+        __syncthreads();
+        if (eg == 0) {
+#pragma unroll 1
+            for (int g = 1; g < EG; ++g) {
+                const float4* ot = mb + (size_t)((g - 1) * NW + hg) * 17 * 32 + lane;
+                const float4 ml = ot[16 * 32];
+                const float m2[2] = {ml.x, ml.y}, l2[2] = {ml.z, ml.w};
+                float al[2], be[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float M = fmaxf(mrow[h], m2[h]);
+                    al[h] = mrow[h] == -INFINITY ? 0.f : exp2f(mrow[h] - M);
+                    be[h] = m2[h] == -INFINITY ? 0.f : exp2f(m2[h] - M);
+                    mrow[h] = M;
+                    lrow[h] = lrow[h] * al[h] + l2[h] * be[h];
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float4 v = ot[i * 32];
+                    o[i][0] = o[i][0] * al[0] + v.x * be[0];
+                    o[i][1] = o[i][1] * al[0] + v.y * be[0];
+                    o[i][2] = o[i][2] * al[1] + v.z * be[1];
+                    o[i][3] = o[i][3] * al[1] + v.w * be[1];
+                }
+            }
+        }
+    }
     const float kLn2 = 0.6931471805599453f;
     float inv[2], lse_r[2];
 #pragma unroll
@@ -344,7 +388,7 @@ __global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
         inv[h] = empty ? 0.f : 1.f / lrow[h];
         lse_r[h] = empty ? -INFINITY : (mrow[h] + __log2f(lrow[h])) * kLn2;
     }
-    const int hr[2] = {warp * 16 + (lane >> 2), warp * 16 + (lane >> 2) + 8};
+    const int hr[2] = {hg * 16 + (lane >> 2), hg * 16 + (lane >> 2) + 8};
     if (CLUSTER) {
         // partials into this CTA's shared memory (Q and the K/V buffers are free now)
         static_assert(L::kMeta >= NW * 16 * 129 * 4, "partial buffer");
@@ -354,7 +398,7 @@ __global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
         float* po = reinterpret_cast<float*>(smem);  // [NW*16][128]
         float* pl = po + NW * 16 * 128;                          // [NW*16]
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < 2 && eg == 0; ++h) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const int d = i * 8 + (lane & 3) * 2;
@@ -365,7 +409,7 @@ __global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
         cluster.sync();
         // CTA r merges heads r, r + 8, ...: one warp per head, 4 dims per lane
         const int r = (int)cluster.block_rank();
-        for (int h = r + kAttnCluster * warp; h < a.H; h += kAttnCluster * NW) {
+        for (int h = r + kAttnCluster * warp; h < a.H; h += kAttnCluster * NW * EG) {
             float ls[kAttnCluster];
             float M = -INFINITY;
 #pragma unroll
@@ -396,6 +440,7 @@ __global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
         cluster.sync();  // no CTA leaves while others read its shared memory
         return;
     }
+    if (eg != 0) return;  // group 0 holds the merged state
     if (a.splits == 1) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -424,57 +469,93 @@ __global__ void __launch_bounds__(NW * 32) attn_split_kernel(AttnArgs a) {
 }
 
 // Merge the split partials of one (query, head): one CTA of 8 warps, warp w
-// owns splits w, w+8, ...; every load is issued up front, the sums are then
-// reduced across warps in a fixed order (deterministic).
+// owns splits w, w+8, ...  The first four splits of every warp are loaded
+// up front (one round trip for up to 32 splits) and merged against their
+// max; further splits keep a running max.  The warps' states are then merged
+// in a fixed order (deterministic).
 constexpr int kCombThreads = 256;
+constexpr int kCombWarps = kCombThreads / 32;
+constexpr int kCombPre = 4;
 
 __global__ void __launch_bounds__(kCombThreads) attn_combine_kernel(const float* part_o, const float* part_lse,
                                                                     int splits, int H, uint16_t* out, float* lse) {
-    __shared__ float4 red[kCombThreads / 32][32];
-    __shared__ float wred[kCombThreads / 32];
+    __shared__ float4 red[kCombWarps][32];
+    __shared__ float wred[kCombWarps], mred[kCombWarps];
     pdl_wait();
     pdl_release();
     const int bh = blockIdx.x;  // bq * H + h
     const int bq = bh / H, h = bh - bq * H;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const float* pl = part_lse + (size_t)bq * splits * H + h;
-    float M = -INFINITY;
-    for (int s = lane; s < splits; s += 32) M = fmaxf(M, pl[(size_t)s * H]);
+    const float* po = part_o + ((size_t)bq * splits * H + h) * 128 + lane * 4;
+    const size_t so = (size_t)H * 128;  // split stride of part_o
+    float ls[kCombPre];
+    float4 v[kCombPre];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
+    for (int u = 0; u < kCombPre; ++u) {
+        const int sp = warp + u * kCombWarps;
+        ls[u] = sp < splits ? pl[(size_t)sp * H] : -INFINITY;
+        v[u] = sp < splits ? *reinterpret_cast<const float4*>(po + sp * so) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < kCombPre; ++u) M = fmaxf(M, ls[u]);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float wsum = 0.f;
-    if (M != -INFINITY) {
-        for (int s = warp; s < splits; s += kCombThreads / 32) {
-            const float ls = pl[(size_t)s * H];
-            const float w = ls == -INFINITY ? 0.f : __expf(ls - M);
-            const float4 v =
-                *reinterpret_cast<const float4*>(part_o + (((size_t)bq * splits + s) * H + h) * 128 + lane * 4);
-            acc.x += w * v.x;
-            acc.y += w * v.y;
-            acc.z += w * v.z;
-            acc.w += w * v.w;
-            wsum += w;
+#pragma unroll
+    for (int u = 0; u < kCombPre; ++u) {
+        const float w = ls[u] == -INFINITY ? 0.f : __expf(ls[u] - M);
+        acc.x += w * v[u].x;
+        acc.y += w * v[u].y;
+        acc.z += w * v[u].z;
+        acc.w += w * v[u].w;
+        wsum += w;
+    }
+#pragma unroll 1
+    for (int sp = warp + kCombPre * kCombWarps; sp < splits; sp += kCombWarps) {
+        const float l2 = pl[(size_t)sp * H];
+        const float4 v2 = *reinterpret_cast<const float4*>(po + sp * so);
+        if (l2 > M) {
+            const float sc = M == -INFINITY ? 0.f : __expf(M - l2);
+            acc.x *= sc;
+            acc.y *= sc;
+            acc.z *= sc;
+            acc.w *= sc;
+            wsum *= sc;
+            M = l2;
         }
+        const float w = l2 == -INFINITY ? 0.f : __expf(l2 - M);
+        acc.x += w * v2.x;
+        acc.y += w * v2.y;
+        acc.z += w * v2.z;
+        acc.w += w * v2.w;
+        wsum += w;
     }
     red[warp][lane] = acc;
-    if (lane == 0) wred[warp] = wsum;
+    if (lane == 0) {
+        wred[warp] = wsum;
+        mred[warp] = M;
+    }
     __syncthreads();
     if (warp == 0) {
-        float4 t = red[0][lane];
-        float ws = wred[0];
+        float Mt = -INFINITY;
 #pragma unroll
-        for (int w = 1; w < kCombThreads / 32; ++w) {
-            t.x += red[w][lane].x;
-            t.y += red[w][lane].y;
-            t.z += red[w][lane].z;
-            t.w += red[w][lane].w;
-            ws += wred[w];
+        for (int w = 0; w < kCombWarps; ++w) Mt = fmaxf(Mt, mred[w]);
+        float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+        float ws = 0.f;
+#pragma unroll
+        for (int w = 0; w < kCombWarps; ++w) {
+            const float sc = mred[w] == -INFINITY ? 0.f : __expf(mred[w] - Mt);
+            t.x += sc * red[w][lane].x;
+            t.y += sc * red[w][lane].y;
+            t.z += sc * red[w][lane].z;
+            t.w += sc * red[w][lane].w;
+            ws += sc * wred[w];
         }
         const float inv = ws > 0.f ? 1.f / ws : 0.f;
         uint16_t* op = out + ((size_t)bq * H + h) * 128 + lane * 4;
         *reinterpret_cast<uint2*>(op) = make_uint2(pack_bf16x2(t.x * inv, t.y * inv), pack_bf16x2(t.z * inv, t.w * inv));
-        if (lse && lane == 0) lse[(size_t)bq * H + h] = ws > 0.f ? M + __logf(ws) : -INFINITY;
+        if (lse && lane == 0) lse[(size_t)bq * H + h] = ws > 0.f ? Mt + __logf(ws) : -INFINITY;
     }
 }
 

@@ -196,10 +196,18 @@ sa_status make_ic_map(CUtensorMap* map, const void* kidx, int B, int Ncap) {
 
 // ------------------------------------------------------- workspace layout --
 struct TopkDecodeWs {
-    size_t hist, hist2, totals, zero_end, keys, emax, chunk_in, chunk_pos, cand_key, cand_idx, amb_key, amb_idx,
-        bitmap, idx, cnt, total;
-    int maxchunks, Wcap;
+    size_t hist, hist2, totals, zero_end, keys, emax, chunk_in, chunk_cnt, chunk_pos, cand_key, cand_idx, cmp_key,
+        cmp_idx, amb_key, amb_idx, bitmap, idx, cnt, total;
+    int maxchunks, fchunk, nfch, Wcap;
 };
+
+// Rows per filter / emit CTA: 1024, or a multiple of it once a sequence
+// would need more than kSelMaxChunks filter chunks.
+int filter_chunk(int Ncap) {
+    const long long per = (long long)sa::kFiltRows * sa::kSelMaxChunks;
+    const long long m = std::max<long long>(1, (Ncap + per - 1) / per);
+    return (int)(m * sa::kFiltRows);
+}
 
 // Rows per score CTA: about three CTAs per SM over the whole batch, whole tiles.
 int score_chunk(int B, int Ncap) {
@@ -209,15 +217,17 @@ int score_chunk(int B, int Ncap) {
     return (int)std::max<long long>(chunk, sa::kScRows);
 }
 
-// [reserved 256 B][histograms][second histograms][totals][keys][per-chunk max error]
-// [per-chunk sure-in counts][per-chunk output positions][candidates key/idx][band key/idx]
-// [bitmap][idx][cnt]
+// [reserved 256 B][histograms][second histograms][totals]  (zeroed per call)
+// [keys][per-score-chunk max error][per-filter-chunk sure-ins, candidates, output positions]
+// [candidates key/idx][compact candidates key/idx][band key/idx][bitmap][idx][cnt]
 TopkDecodeWs topk_decode_layout(int B, int Ncap, int k, bool own_idx) {
     TopkDecodeWs w{};
     w.maxchunks = std::max(1, cdiv(Ncap, sa::kScRows));
+    w.fchunk = filter_chunk(Ncap);
+    w.nfch = std::max(1, cdiv(Ncap, w.fchunk));
     w.Wcap = ((Ncap + 31) / 32 + 1) & ~1;
     size_t o = 256;
-    w.hist = o;  // histograms and totals are zeroed together before every call
+    w.hist = o;
     o += (size_t)B * sa::kBins * 4;
     w.hist2 = o;
     o += (size_t)B * sa::kBins * 4;
@@ -226,18 +236,24 @@ TopkDecodeWs topk_decode_layout(int B, int Ncap, int k, bool own_idx) {
     w.zero_end = o;
     o = up256(o);
     const size_t col = up256((size_t)B * Ncap * 4);
-    const size_t per_chunk = up256((size_t)B * w.maxchunks * 4);
+    const size_t per_fch = up256((size_t)B * w.nfch * 4);
     w.keys = o;
     o += col;
     w.emax = o;
-    o += per_chunk;
+    o += up256((size_t)B * w.maxchunks * 4);
     w.chunk_in = o;
-    o += per_chunk;
+    o += per_fch;
+    w.chunk_cnt = o;
+    o += per_fch;
     w.chunk_pos = o;
-    o += per_chunk;
+    o += per_fch;
     w.cand_key = o;
     o += col;
     w.cand_idx = o;
+    o += col;
+    w.cmp_key = o;
+    o += col;
+    w.cmp_idx = o;
     o += col;
     w.amb_key = o;
     o += col;
@@ -272,50 +288,60 @@ size_t attn_partial_bytes(long long BQ, int splits, int H) {
 }
 
 // ------------------------------------------------------------ launchers ----
-template <int NW, bool G, bool F, int ST, bool CL>
+template <int NW, bool G, bool F, int ST, bool CL, int EG>
 sa_status launch_attn_t(const sa::AttnArgs& a, dim3 grid, cudaStream_t st, bool pdl) {
     using L = sa::AttnSmem<NW, G, F, ST>;
     static std::atomic<uint64_t> init{0};
     if (!attr_done(init)) {
-        SA_CUDA(cudaFuncSetAttribute(sa::attn_split_kernel<NW, G, F, ST, CL>,
+        SA_CUDA(cudaFuncSetAttribute(sa::attn_split_kernel<NW, G, F, ST, CL, EG>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal));
         attr_set(init);
     }
-    SA_CUDA(launch_k(sa::attn_split_kernel<NW, G, F, ST, CL>, grid, dim3(NW * 32), L::kTotal, st, pdl,
+    SA_CUDA(launch_k(sa::attn_split_kernel<NW, G, F, ST, CL, EG>, grid, dim3(NW * EG * 32), L::kTotal, st, pdl,
                      CL ? (unsigned)sa::kAttnCluster : 1u, a));
     SA_LAUNCHED();
     return SA_OK;
 }
 
-template <int NW, int ST, bool CL>
+template <int NW, int ST, bool CL, int EG>
 sa_status launch_attn_nw(const sa::AttnArgs& a, bool gather, bool fp8, dim3 grid, cudaStream_t st, bool pdl) {
     if (gather)
-        return fp8 ? launch_attn_t<NW, true, true, ST, CL>(a, grid, st, pdl)
-                   : launch_attn_t<NW, true, false, ST, CL>(a, grid, st, pdl);
-    return fp8 ? launch_attn_t<NW, false, true, ST, CL>(a, grid, st, pdl)
-               : launch_attn_t<NW, false, false, ST, CL>(a, grid, st, pdl);
+        return fp8 ? launch_attn_t<NW, true, true, ST, CL, EG>(a, grid, st, pdl)
+                   : launch_attn_t<NW, true, false, ST, CL, EG>(a, grid, st, pdl);
+    return fp8 ? launch_attn_t<NW, false, true, ST, CL, EG>(a, grid, st, pdl)
+               : launch_attn_t<NW, false, false, ST, CL, EG>(a, grid, st, pdl);
 }
 
 // Splits of up to 4 tiles keep all of them in flight (4 stages); longer
 // lists (prefill) stream through a 2-stage pipeline.  A query split exactly
-// kAttnCluster ways merges inside a cluster.
-sa_status launch_attn(const sa::AttnArgs& a, bool gather, bool fp8, long long BQ, cudaStream_t st, bool pdl) {
+// kAttnCluster ways merges inside a cluster.  Decode with up to 64 heads
+// splits every tile between two warp groups (8 warps), which halves the
+// serial work per warp; prefill keeps one group.
+sa_status launch_attn(const sa::AttnArgs& a, bool gather, bool fp8, long long BQ, cudaStream_t st, bool pdl,
+                      bool decode) {
     const bool cl = a.splits == sa::kAttnCluster && BQ <= 65535;
     if (BQ > 2147483647LL || a.splits > 65535) return fail(SA_ERR_INVALID_ARG, "too many queries or splits");
     const dim3 grid = cl ? dim3(a.splits, (unsigned)BQ) : dim3((unsigned)BQ, a.splits);
     const bool deep = a.tiles_per_split >= 2 && a.tiles_per_split <= 4;
     if (a.H <= 64) {
+        if (decode) {
+            if (cl)
+                return deep ? launch_attn_nw<4, 4, true, 2>(a, gather, fp8, grid, st, pdl)
+                            : launch_attn_nw<4, 2, true, 2>(a, gather, fp8, grid, st, pdl);
+            return deep ? launch_attn_nw<4, 4, false, 2>(a, gather, fp8, grid, st, pdl)
+                        : launch_attn_nw<4, 2, false, 2>(a, gather, fp8, grid, st, pdl);
+        }
         if (cl)
-            return deep ? launch_attn_nw<4, 4, true>(a, gather, fp8, grid, st, pdl)
-                        : launch_attn_nw<4, 2, true>(a, gather, fp8, grid, st, pdl);
-        return deep ? launch_attn_nw<4, 4, false>(a, gather, fp8, grid, st, pdl)
-                    : launch_attn_nw<4, 2, false>(a, gather, fp8, grid, st, pdl);
+            return deep ? launch_attn_nw<4, 4, true, 1>(a, gather, fp8, grid, st, pdl)
+                        : launch_attn_nw<4, 2, true, 1>(a, gather, fp8, grid, st, pdl);
+        return deep ? launch_attn_nw<4, 4, false, 1>(a, gather, fp8, grid, st, pdl)
+                    : launch_attn_nw<4, 2, false, 1>(a, gather, fp8, grid, st, pdl);
     }
     if (cl)
-        return deep ? launch_attn_nw<8, 4, true>(a, gather, fp8, grid, st, pdl)
-                    : launch_attn_nw<8, 2, true>(a, gather, fp8, grid, st, pdl);
-    return deep ? launch_attn_nw<8, 4, false>(a, gather, fp8, grid, st, pdl)
-                : launch_attn_nw<8, 2, false>(a, gather, fp8, grid, st, pdl);
+        return deep ? launch_attn_nw<8, 4, true, 1>(a, gather, fp8, grid, st, pdl)
+                    : launch_attn_nw<8, 2, true, 1>(a, gather, fp8, grid, st, pdl);
+    return deep ? launch_attn_nw<8, 4, false, 1>(a, gather, fp8, grid, st, pdl)
+                : launch_attn_nw<8, 2, false, 1>(a, gather, fp8, grid, st, pdl);
 }
 
 // The merge follows its split kernel on the same stream: always chained.
@@ -385,7 +411,7 @@ sa_status run_attn(const void* q, int Tq, int H, const sa_cache* c, bool gather,
         a.part_o = reinterpret_cast<float*>(base);
         a.part_lse = reinterpret_cast<float*>(base + up256((size_t)BQ * sp.splits * H * 128 * 4));
     }
-    sa_status r = launch_attn(a, gather, c->dtype == SA_FP8_E4M3, BQ, st, chained && pdl_on());
+    sa_status r = launch_attn(a, gather, c->dtype == SA_FP8_E4M3, BQ, st, chained && pdl_on(), !prefill);
     if (r != SA_OK) return r;
     // a query split kAttnCluster ways was merged inside its cluster
     if (sp.splits > 1 && !(sp.splits == sa::kAttnCluster && BQ <= 65535))
@@ -410,9 +436,12 @@ sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* 
     a.hist2 = reinterpret_cast<uint32_t*>(base + w.hist2);
     a.emax_part = reinterpret_cast<float*>(base + w.emax);
     a.chunk_in = reinterpret_cast<uint32_t*>(base + w.chunk_in);
+    a.chunk_cnt = reinterpret_cast<uint32_t*>(base + w.chunk_cnt);
     a.chunk_pos = reinterpret_cast<uint32_t*>(base + w.chunk_pos);
     a.cand_key = reinterpret_cast<uint32_t*>(base + w.cand_key);
     a.cand_idx = reinterpret_cast<int32_t*>(base + w.cand_idx);
+    a.cmp_key = reinterpret_cast<uint32_t*>(base + w.cmp_key);
+    a.cmp_idx = reinterpret_cast<int32_t*>(base + w.cmp_idx);
     a.amb_key = reinterpret_cast<uint32_t*>(base + w.amb_key);
     a.amb_idx = reinterpret_cast<int32_t*>(base + w.amb_idx);
     a.totals = reinterpret_cast<uint32_t*>(base + w.totals);
@@ -424,7 +453,9 @@ sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* 
     a.k = k;
     a.chunk = score_chunk(B, Ncap);
     a.nchunks = Ncap > 0 ? cdiv(Ncap, a.chunk) : 1;
-    if (a.nchunks > w.maxchunks || a.nchunks > sa::kSelMaxChunks)
+    a.fchunk = w.fchunk;
+    a.nfch = w.nfch;
+    if (a.nchunks > w.maxchunks || a.nfch > sa::kSelMaxChunks)
         return fail(SA_ERR_WORKSPACE, "internal: chunk count above the workspace bound");
     static std::atomic<uint64_t> init{0};
     const size_t smem = sa::kScStages * sa::kScTileBytes + sa::kScStages * 8 + 1024;
@@ -438,8 +469,8 @@ sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* 
         CUtensorMap map;
         sa_status r = make_ic_map(&map, c->kidx, B, Ncap);
         if (r != SA_OK) return r;
-        stage_mark(SA_STAGE_INDEX_SCORE, 0, st);
         SA_CUDA(cudaMemsetAsync(a.hist1, 0, w.zero_end - w.hist, st));
+        stage_mark(SA_STAGE_INDEX_SCORE, 0, st);
         sa::score_decode_kernel<<<dim3(a.nchunks, B), sa::kScThreads, smem, st>>>(map, a);
         SA_LAUNCHED();
         stage_mark(SA_STAGE_INDEX_SCORE, 1, st);
@@ -450,11 +481,11 @@ sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* 
     // a sequence with n <= k visible entries (every one, when Ncap is 0) is
     // answered by the filter's first CTA; the other kernels skip it
     const bool pdl = pdl_on();
-    SA_CUDA(launch_k(sa::topk_filter_kernel, dim3(a.nchunks, B), dim3(sa::kSelThreads), 0, st, pdl && Ncap > 0, 1u, a));
+    SA_CUDA(launch_k(sa::topk_filter_kernel, dim3(a.nfch, B), dim3(sa::kSelThreads), 0, st, pdl && Ncap > 0, 1u, a));
     SA_LAUNCHED();
     SA_CUDA(launch_k(sa::topk_resolve_kernel, dim3(B), dim3(sa::kResThreads), sa::kSelSmem, st, pdl, 1u, a));
     SA_LAUNCHED();
-    SA_CUDA(launch_k(sa::topk_emit_kernel, dim3(a.nchunks, B), dim3(sa::kEmitThreads), 0, st, pdl, 1u, a));
+    SA_CUDA(launch_k(sa::topk_emit_kernel, dim3(a.nfch, B), dim3(sa::kEmitThreads), 0, st, pdl, 1u, a));
     SA_LAUNCHED();
     stage_mark(SA_STAGE_TOPK_SELECT, 1, st);
     return SA_OK;

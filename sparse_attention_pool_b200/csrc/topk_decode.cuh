@@ -48,10 +48,12 @@ constexpr int kScTileBytes = kScRows * 128;
 constexpr int kBins = 2048;       // 11-bit digits
 constexpr int kBinsLow = 1024;    // last 10-bit digit
 
-// totals[B][kTotals] (zeroed per call): candidate count, and from the first
-// filter CTA the bin d1 of t~, the bound E and the count of keys above bin d1
+// totals[B][kTotals] (zeroed per call): the score CTAs' finish ticket, and
+// from the last of them the bin d1 of t~, the bound E and the count of keys
+// above bin d1
 constexpr int kTotals = 4;
-constexpr int kTotCand = 0, kTotBin = 1, kTotE = 2, kTotAbove = 3;
+constexpr int kTotTicket = 0, kTotBin = 1, kTotE = 2, kTotAbove = 3;
+constexpr int kFiltRows = 1024;  // rows per filter / emit CTA (one pass of 256 threads x 4 keys)
 
 struct TopkDecodeArgs {
     const uint16_t* q_idx;  // [B][64]
@@ -61,17 +63,20 @@ struct TopkDecodeArgs {
     uint32_t* hist1;        // [B][2048]     histogram of key bits 31..21 (zeroed per call)
     uint32_t* hist2;        // [B][2048]     bits 20..10 of the keys in bin d1 (zeroed per call)
     float* emax_part;       // [B][nchunks]  per score CTA: max e_j
-    uint32_t* chunk_in;     // [B][nchunks]  per filter CTA: surely selected entries
-    uint32_t* chunk_pos;    // [B][nchunks]  output position of each chunk's first selected entry
-    uint32_t* cand_key;     // [B][Ncap]     candidates of the sequence (filter order)
+    uint32_t* chunk_in;     // [B][nfch]     per filter chunk: surely selected entries
+    uint32_t* chunk_cnt;    // [B][nfch]     per filter chunk: candidates
+    uint32_t* chunk_pos;    // [B][nfch]     output position of each filter chunk's first selected entry
+    uint32_t* cand_key;     // [B][Ncap]     candidates, each filter chunk in its own rows
     int32_t* cand_idx;      // [B][Ncap]
+    uint32_t* cmp_key;      // [B][Ncap]     all candidates in one list, when they overflow shared memory
+    int32_t* cmp_idx;       // [B][Ncap]
     uint32_t* totals;       // [B][kTotals]
     uint32_t* bitmap;       // [B][Wcap]     selection bitmap
     uint32_t* amb_key;      // [B][Ncap]     exact keys of the band, when it is large
     int32_t* amb_idx;       // [B][Ncap]
     int32_t* idx;           // [B][k]
     int32_t* cnt;           // [B]
-    int Ncap, Wcap, chunk, nchunks, k;
+    int Ncap, Wcap, chunk, nchunks, fchunk, nfch, k;
 };
 
 __device__ __forceinline__ int clamp_n(const int32_t* n, int b, int Ncap) {
@@ -117,121 +122,6 @@ __device__ __forceinline__ void load_q2(double* q2, const uint16_t* qI) {
         q2[2 * threadIdx.x] = (double)bf16lo_f32(w) * 0x1p768;
         q2[2 * threadIdx.x + 1] = (double)bf16hi_f32(w) * 0x1p768;
     }
-}
-
-// ------------------------------------------------------------ 1. scores ----
-__global__ void __launch_bounds__(kScThreads, 3)
-    score_decode_kernel(const __grid_constant__ CUtensorMap ic_map, TopkDecodeArgs a) {
-    extern __shared__ uint8_t smem_raw[];
-    // TMA with 128B swizzle needs a 1024-byte aligned destination
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* tiles = smem;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kScStages * kScTileBytes);
-    __shared__ float s_emax[kScThreads / 32];
-    __shared__ uint32_t hist[kBins];  // top 11 key bits of this CTA's rows
-
-    pdl_wait();
-    pdl_release();
-    const int b = blockIdx.y;
-    const int n = clamp_n(a.n, b, a.Ncap);
-    if (n <= a.k) return;  // everything visible is selected; nothing to score
-    const int row0 = blockIdx.x * a.chunk;
-    const int row1 = min(row0 + a.chunk, n);
-    const int tid = threadIdx.x;
-    if (row0 >= row1) {
-        if (tid == 0) a.emax_part[(size_t)b * a.nchunks + blockIdx.x] = 0.f;
-        return;
-    }
-    const int ntiles = (row1 - row0 + kScRows - 1) / kScRows;
-
-    float q[64];
-    {
-        const uint32_t* qw = reinterpret_cast<const uint32_t*>(a.q_idx + (size_t)b * 64);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const uint32_t w = __ldg(qw + i);
-            q[2 * i] = bf16lo_f32(w);
-            q[2 * i + 1] = bf16hi_f32(w);
-        }
-    }
-    for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0;
-    if (tid == 0) {
-        for (int s = 0; s < kScStages; ++s) mbar_init(&full[s], 1);
-        fence_barrier_init();
-    }
-    __syncthreads();
-
-    // the map views Ic as [B][Ncap][64]: coordinates (dim, row, sequence)
-    int issued = 0;
-    if (tid == 0) {
-        for (; issued < kScStages && issued < ntiles; ++issued) {
-            mbar_expect_tx(&full[issued], kScTileBytes);
-            tma_load_3d(tiles + issued * kScTileBytes, &ic_map, 0, row0 + issued * kScRows, b, &full[issued]);
-        }
-    }
-    int consumed = 0;
-    bool timed_out = false;
-    float emax = 0.f;
-    for (int i = 0; i < ntiles; ++i) {
-        const int s = i % kScStages;
-        const bool ok = mbar_wait(&full[s], (i / kScStages) & 1);
-        if (__syncthreads_or(!ok)) {
-            timed_out = true;
-            break;
-        }
-        consumed = i + 1;
-        const int row = row0 + i * kScRows + tid;
-        if (row < row1) {
-            const uint8_t* rp = tiles + s * kScTileBytes + tid * 128;
-            float acc = 0.f, aab = 0.f;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 w = *reinterpret_cast<const uint4*>(rp + ((c ^ (tid & 7)) << 4));
-                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const float k0 = bf16lo_f32(ws[h]), k1 = bf16hi_f32(ws[h]);
-                    acc = fmaf(q[8 * c + 2 * h], k0, acc);
-                    aab = fmaf(fabsf(q[8 * c + 2 * h]), fabsf(k0), aab);
-                    acc = fmaf(q[8 * c + 2 * h + 1], k1, acc);
-                    aab = fmaf(fabsf(q[8 * c + 2 * h + 1]), fabsf(k1), aab);
-                }
-            }
-            const uint32_t key = score_key(acc);
-            a.keys[(size_t)b * a.Ncap + row] = key;
-            atomicAdd(&hist[key >> 21], 1u);
-            emax = fmaxf(emax, fmaf(aab, 0x1p-16f, fmaf(fabsf(acc), 0x1p-22f, 0x1p-140f)));
-        }
-        __syncthreads();  // slot s is free again
-        if (tid == 0 && issued < ntiles) {
-            fence_proxy_async();
-            mbar_expect_tx(&full[s], kScTileBytes);
-            tma_load_3d(tiles + s * kScTileBytes, &ic_map, 0, row0 + issued * kScRows, b, &full[s]);
-            ++issued;
-        }
-    }
-    if (timed_out) {
-        // let copies still in flight land before the CTA's shared memory goes away
-        if (tid == 0) {
-            for (int i = consumed; i < issued; ++i) mbar_wait(&full[i % kScStages], (i / kScStages) & 1);
-            a.emax_part[(size_t)b * a.nchunks + blockIdx.x] = 0.f;
-        }
-        __syncthreads();
-        return;
-    }
-    // e_j is rounded to nearest in fp32: one more ulp keeps it an upper bound
-    emax = __uint_as_float(__float_as_uint(emax) + 1u);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) emax = fmaxf(emax, __shfl_xor_sync(0xFFFFFFFFu, emax, o));
-    if ((tid & 31) == 0) s_emax[tid >> 5] = emax;
-    __syncthreads();
-    if (tid == 0) {
-        float m = s_emax[0];
-        for (int w = 1; w < kScThreads / 32; ++w) m = fmaxf(m, s_emax[w]);
-        a.emax_part[(size_t)b * a.nchunks + blockIdx.x] = m;
-    }
-    for (int i = tid; i < kBins; i += blockDim.x)
-        if (hist[i]) atomicAdd(&a.hist1[(size_t)b * kBins + i], hist[i]);
 }
 
 // --------------------------------------------------- digit search helpers --
@@ -294,6 +184,73 @@ __device__ __forceinline__ void find_digit_asc(const uint32_t* h, uint32_t R, ui
     __syncthreads();
     *out_d = res[0];
     *out_below = (uint32_t)res[1];
+    __syncthreads();
+}
+
+// Descending digit search over T * NPT bins held in registers: thread t
+// holds bins [T*NPT - (t+1)*NPT, T*NPT - t*NPT) as h[0..NPT) in ascending
+// order (thread 0 holds the top bins).  Loaded straight from global memory,
+// the bins need no shared-memory staging (no bank conflicts).
+template <int NPT>
+__device__ __forceinline__ void find_digit_desc_regs(const uint32_t (&h)[NPT], uint32_t K, uint32_t* sh32, int* res,
+                                                     int* out_d, uint32_t* out_above) {
+    const int t = threadIdx.x;
+    uint32_t local = 0;
+#pragma unroll
+    for (int j = 0; j < NPT; ++j) local += h[j];
+    if (t == 0) res[0] = -1;  // ordered before every write below by the scan's barriers
+    uint32_t above = block_exclusive_scan(local, sh32, nullptr);  // keys in the bins above this range
+    const int lo = ((int)blockDim.x - 1 - t) * NPT;
+#pragma unroll
+    for (int j = NPT - 1; j >= 0; --j) {
+        if (above < K && K <= above + h[j]) {
+            res[0] = lo + j;
+            res[1] = (int)above;
+        }
+        above += h[j];
+    }
+    __syncthreads();
+    *out_d = res[0];
+    *out_above = (uint32_t)res[1];
+    __syncthreads();
+}
+
+// Exclusive scans of two values at once (one set of barriers).
+__device__ __forceinline__ void block_exclusive_scan2(uint32_t v0, uint32_t v1, uint32_t* sh64, uint32_t* e0,
+                                                      uint32_t* e1, uint32_t* t0, uint32_t* t1) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    uint32_t x0 = v0, x1 = v1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y0 = __shfl_up_sync(0xFFFFFFFFu, x0, o), y1 = __shfl_up_sync(0xFFFFFFFFu, x1, o);
+        if (lane >= o) {
+            x0 += y0;
+            x1 += y1;
+        }
+    }
+    if (lane == 31) {
+        sh64[warp] = x0;
+        sh64[32 + warp] = x1;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t w0 = lane < nw ? sh64[lane] : 0u, w1 = lane < nw ? sh64[32 + lane] : 0u;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y0 = __shfl_up_sync(0xFFFFFFFFu, w0, o), y1 = __shfl_up_sync(0xFFFFFFFFu, w1, o);
+            if (lane >= o) {
+                w0 += y0;
+                w1 += y1;
+            }
+        }
+        sh64[lane] = w0;
+        sh64[32 + lane] = w1;
+    }
+    __syncthreads();
+    *e0 = (warp ? sh64[warp - 1] : 0u) + x0 - v0;
+    *e1 = (warp ? sh64[32 + warp - 1] : 0u) + x1 - v1;
+    *t0 = sh64[nw - 1];
+    *t1 = sh64[32 + nw - 1];
     __syncthreads();
 }
 
@@ -415,15 +372,177 @@ __device__ __noinline__ bool rank_in_bin(const uint32_t* key, uint32_t cnt, uint
     return true;
 }
 
+// ------------------------------------------------------------ 1. scores ----
+__global__ void __launch_bounds__(kScThreads, 3)
+    score_decode_kernel(const __grid_constant__ CUtensorMap ic_map, TopkDecodeArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    // TMA with 128B swizzle needs a 1024-byte aligned destination
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* tiles = smem;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kScStages * kScTileBytes);
+    __shared__ float s_emax[kScThreads / 32];
+    __shared__ uint32_t hist[kBins];  // top 11 key bits of this CTA's rows
+    __shared__ uint32_t s_sh32[32];
+    __shared__ int s_res[2];
+    __shared__ uint32_t s_last;
+
+    pdl_wait();
+    pdl_release();
+    const int b = blockIdx.y;
+    const int n = clamp_n(a.n, b, a.Ncap);
+    if (n <= a.k) return;  // everything visible is selected; nothing to score
+    const int row0 = blockIdx.x * a.chunk;
+    const int row1 = min(row0 + a.chunk, n);
+    const int tid = threadIdx.x;
+    // an empty chunk scans nothing but still takes part in the finish below
+    const int ntiles = row1 > row0 ? (row1 - row0 + kScRows - 1) / kScRows : 0;
+
+    float q[64];
+    {
+        const uint32_t* qw = reinterpret_cast<const uint32_t*>(a.q_idx + (size_t)b * 64);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const uint32_t w = __ldg(qw + i);
+            q[2 * i] = bf16lo_f32(w);
+            q[2 * i + 1] = bf16hi_f32(w);
+        }
+    }
+    for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0;
+    if (tid == 0) {
+        for (int s = 0; s < kScStages; ++s) mbar_init(&full[s], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    // the map views Ic as [B][Ncap][64]: coordinates (dim, row, sequence)
+    int issued = 0;
+    if (tid == 0) {
+        for (; issued < kScStages && issued < ntiles; ++issued) {
+            mbar_expect_tx(&full[issued], kScTileBytes);
+            tma_load_3d(tiles + issued * kScTileBytes, &ic_map, 0, row0 + issued * kScRows, b, &full[issued]);
+        }
+    }
+    int consumed = 0;
+    bool timed_out = false;
+    float emax = 0.f;
+    for (int i = 0; i < ntiles; ++i) {
+        const int s = i % kScStages;
+        const bool ok = mbar_wait(&full[s], (i / kScStages) & 1);
+        if (__syncthreads_or(!ok)) {
+            timed_out = true;
+            break;
+        }
+        consumed = i + 1;
+        const int row = row0 + i * kScRows + tid;
+        if (row < row1) {
+            const uint8_t* rp = tiles + s * kScTileBytes + tid * 128;
+            float acc = 0.f, aab = 0.f;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint4 w = *reinterpret_cast<const uint4*>(rp + ((c ^ (tid & 7)) << 4));
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const float k0 = bf16lo_f32(ws[h]), k1 = bf16hi_f32(ws[h]);
+                    acc = fmaf(q[8 * c + 2 * h], k0, acc);
+                    aab = fmaf(fabsf(q[8 * c + 2 * h]), fabsf(k0), aab);
+                    acc = fmaf(q[8 * c + 2 * h + 1], k1, acc);
+                    aab = fmaf(fabsf(q[8 * c + 2 * h + 1]), fabsf(k1), aab);
+                }
+            }
+            const uint32_t key = score_key(acc);
+            a.keys[(size_t)b * a.Ncap + row] = key;
+            atomicAdd(&hist[key >> 21], 1u);
+            emax = fmaxf(emax, fmaf(aab, 0x1p-16f, fmaf(fabsf(acc), 0x1p-22f, 0x1p-140f)));
+        }
+        __syncthreads();  // slot s is free again
+        if (tid == 0 && issued < ntiles) {
+            fence_proxy_async();
+            mbar_expect_tx(&full[s], kScTileBytes);
+            tma_load_3d(tiles + s * kScTileBytes, &ic_map, 0, row0 + issued * kScRows, b, &full[s]);
+            ++issued;
+        }
+    }
+    if (timed_out) {
+        // let copies still in flight land before the CTA's shared memory goes away
+        // (the device status records the timeout; the results are not used)
+        if (tid == 0)
+            for (int i = consumed; i < issued; ++i) mbar_wait(&full[i % kScStages], (i / kScStages) & 1);
+        __syncthreads();
+    }
+    // e_j is rounded to nearest in fp32: one more ulp keeps it an upper bound
+    emax = __uint_as_float(__float_as_uint(emax) + 1u);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) emax = fmaxf(emax, __shfl_xor_sync(0xFFFFFFFFu, emax, o));
+    if ((tid & 31) == 0) s_emax[tid >> 5] = emax;
+    __syncthreads();
+    if (tid == 0) {
+        float m = s_emax[0];
+        for (int w = 1; w < kScThreads / 32; ++w) m = fmaxf(m, s_emax[w]);
+        a.emax_part[(size_t)b * a.nchunks + blockIdx.x] = m;
+    }
+    for (int i = tid; i < kBins; i += blockDim.x)
+        if (hist[i]) atomicAdd(&a.hist1[(size_t)b * kBins + i], hist[i]);
+
+    // The last CTA of the sequence to finish finds, once for every filter
+    // CTA, the bin d1 of the k-th largest key, the count of keys above it
+    // and the sequence's bound E.  (Ticket pattern: no CTA waits.)
+    uint32_t* tot = a.totals + (size_t)b * kTotals;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(tot + kTotTicket, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    constexpr int NPT = kBins / kScThreads;  // 16 bins per thread
+    uint32_t hb[NPT];
+    {
+        const uint32_t* src = a.hist1 + (size_t)b * kBins + (kScThreads - 1 - tid) * NPT;
+#pragma unroll
+        for (int v = 0; v < NPT / 4; ++v) {
+            const uint4 x = ld_cg_u32x4(src + 4 * v);
+            hb[4 * v] = x.x;
+            hb[4 * v + 1] = x.y;
+            hb[4 * v + 2] = x.z;
+            hb[4 * v + 3] = x.w;
+        }
+    }
+    float e = 0.f;
+    for (int q = tid; q < a.nchunks; q += blockDim.x) e = fmaxf(e, __ldcg(a.emax_part + (size_t)b * a.nchunks + q));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) e = fmaxf(e, __shfl_xor_sync(0xFFFFFFFFu, e, o));
+    __syncthreads();  // every s_emax read above is done
+    if ((tid & 31) == 0) s_emax[tid >> 5] = e;
+    __syncthreads();
+    float E = s_emax[0];
+#pragma unroll
+    for (int w = 1; w < kScThreads / 32; ++w) E = fmaxf(E, s_emax[w]);
+    int d1;
+    uint32_t above1;
+    find_digit_desc_regs<NPT>(hb, (uint32_t)a.k, s_sh32, s_res, &d1, &above1);
+    if (tid == 0) {
+        if (d1 < 0) {  // cannot happen: the histogram counts all n > k keys
+            flag(DEV_LEN);
+            d1 = 0;
+            above1 = 0;
+        }
+        tot[kTotBin] = (uint32_t)d1;
+        tot[kTotE] = __float_as_uint(E);
+        tot[kTotAbove] = above1;
+    }
+}
+
 // --------------------------------------------------------- 2. selection ----
 constexpr int kSelThreads = 256;             // filter CTAs
+constexpr int kFiltKPT = kFiltRows / kSelThreads;
 constexpr int kResThreads = 1024;            // resolve CTA (one per sequence)
-constexpr int kSelKPT = 16;                  // keys per thread held in registers per pass
 constexpr int kSelCap = 8192;                // candidates the resolving CTA holds in shared memory
 constexpr int kSelSmem = kSelCap * 8;
-constexpr int kSelMaxChunks = 1024;
+constexpr int kSelMaxChunks = 1024;          // filter chunks per sequence
+constexpr int kGatherJ = 8;                  // filter chunks per warp loaded ahead by the resolve
 static_assert(kSelMaxChunks <= kResThreads, "the resolve gives one thread to every chunk");
 static_assert(kBins == 2 * kResThreads, "the resolve loads the second histogram two bins per thread");
+static_assert(kFiltKPT * kSelThreads == kFiltRows, "one filter pass covers a chunk");
 
 struct FilterBounds {
     float in_above;  // s~ > in_above  : surely selected
@@ -441,78 +560,24 @@ __device__ __forceinline__ FilterBounds filter_bounds(int d1, float E) {
 }
 
 struct SelSmem {
-    double q2[64];            // qI * 2^768 for the exact rescoring
-    uint32_t hist[kBins];     // digit histograms; later the per-chunk winner counts
-    uint32_t sh32[32];
+    double q2[64];                  // qI * 2^768 for the exact rescoring
+    uint32_t hist[kBins];           // digit histograms of the fallback; then the per-chunk winner counts
+    uint32_t base[kSelMaxChunks];   // compact position of each filter chunk's candidates
+    uint32_t ccnt[kSelMaxChunks];   // candidates per filter chunk
+    uint32_t sh64[64];
     int res[2];
-    float red[kSelThreads / 32];
-    uint32_t last, amb_cnt, f_cnt, tkey, T2;
+    uint32_t f_cnt, found, tkey, amb_cnt, T2;
     int32_t jmax2;
     uint32_t amb_key[kResThreads];  // the fine bin's keys, then the band's exact keys
     int32_t amb_idx[kResThreads];
 };
 
-// The R1-th largest screened key t~ among the C candidates.  Fast path: the
-// filter's histogram of bits 20..10 over bin d1 gives the fine bin of t~
-// directly (rank K2 = k - above1 inside bin d1), whose few keys are ranked
-// pairwise.  Otherwise (a crowded fine bin, or counts that do not add up)
-// the digit passes over the whole list.
-__device__ __noinline__ uint32_t find_threshold(const uint32_t* lk, const int32_t* li, uint32_t C, uint32_t R1,
-                                                int d1, uint32_t K2, SelSmem& S) {
-    const int tid = threadIdx.x;
-    int d2;
-    uint32_t above2;
-    find_digit_desc<kBins>(S.hist, K2, S.sh32, &d2, &above2, S.res);
-    if (d2 >= 0) {
-        const uint32_t R3 = K2 - above2;  // rank of t~ inside the fine bin
-        const uint32_t pre = ((uint32_t)d1 << 11) | (uint32_t)d2;
-        if (tid == 0) {
-            S.f_cnt = 0;
-            S.tkey = 0;
-            S.last = 0;
-        }
-        __syncthreads();
-#pragma unroll 1
-        for (uint32_t i = tid; i < C; i += kResThreads) {
-            const uint32_t kk = lk[i];
-            if ((kk >> 10) == pre) {
-                const uint32_t p = atom_add_shared(&S.f_cnt, 1u);
-                if (p < (uint32_t)kResThreads) S.amb_key[p] = kk;
-            }
-        }
-        __syncthreads();
-        const uint32_t nf = S.f_cnt;
-        if (nf <= (uint32_t)kResThreads && R3 <= nf) {
-            if ((uint32_t)tid < nf) {
-                const uint32_t mk = S.amb_key[tid];
-                uint32_t gt = 0, ge = 0;
-                for (uint32_t o = 0; o < nf; ++o) {
-                    const uint32_t ok = S.amb_key[o];
-                    gt += ok > mk;
-                    ge += ok >= mk;
-                }
-                if (gt < R3 && R3 <= ge) {  // every thread holding t~ writes the same value
-                    S.tkey = mk;
-                    S.last = 1;
-                }
-            }
-            __syncthreads();
-            if (S.last) return S.tkey;
-        }
-    }
-    uint32_t tkey;
-    if (!rank_in_bin(lk, C, R1, d1, S.hist, S.sh32, S.res, &tkey)) {
-        int32_t jd;
-        select_rank(lk, li, C, R1, S.hist, S.sh32, S.res, &tkey, &jd);
-    }
-    return tkey;
-}
-
-// Filter: one CTA per score chunk; surely-selected entries become bitmap
-// bits, the rest of the widened bin d1 is appended to the sequence's
-// candidate list, and the keys inside bin d1 feed a histogram of bits 20..10.
-__global__ void __launch_bounds__(kSelThreads, 3) topk_filter_kernel(TopkDecodeArgs a) {
-    __shared__ SelSmem S;
+// Filter: one CTA per 1024 rows.  Entries above the widened bin of t~ become
+// bitmap bits (surely selected, counted), the rest of the widened bin become
+// candidates in the chunk's own rows of the candidate arrays, and keys
+// inside bin d1 feed the second histogram.  Integer compares on order keys.
+__global__ void __launch_bounds__(kSelThreads) topk_filter_kernel(TopkDecodeArgs a) {
+    __shared__ uint32_t s_cnt, s_in;
     pdl_wait();
     pdl_release();
     const int b = blockIdx.y, c = blockIdx.x;
@@ -527,173 +592,146 @@ __global__ void __launch_bounds__(kSelThreads, 3) topk_filter_kernel(TopkDecodeA
         }
         return;
     }
-    const int row0 = c * a.chunk;
-    const int row1 = min(row0 + a.chunk, n);
+    const int row0 = c * a.fchunk;
+    const int row1 = min(row0 + a.fchunk, n);
     const uint32_t* keys = a.keys + (size_t)b * a.Ncap;
-
-    // issue every load first: the first pass's keys, the histogram, the error bounds
-    uint32_t kr[kSelKPT];
+    const uint32_t* tot = a.totals + (size_t)b * kTotals;
+    // the first pass's keys go out with the thresholds: one round trip
+    uint32_t kr[kFiltKPT];
 #pragma unroll
-    for (int i = 0; i < kSelKPT; ++i) {
+    for (int i = 0; i < kFiltKPT; ++i) {
         const int row = row0 + i * kSelThreads + tid;
-        kr[i] = row < row1 ? __ldcg(keys + row) : 0u;
+        kr[i] = row < row1 ? ld_cg_u32(keys + row) : 0u;
     }
-    uint32_t hv[kBins / kSelThreads];
-#pragma unroll
-    for (int u = 0; u < kBins / kSelThreads; ++u) hv[u] = __ldcg(a.hist1 + (size_t)b * kBins + u * kSelThreads + tid);
-    float e = 0.f;
-    for (int q = tid; q < a.nchunks; q += kSelThreads) e = fmaxf(e, __ldcg(a.emax_part + (size_t)b * a.nchunks + q));
-    uint32_t* ck = a.cand_key + (size_t)b * a.Ncap;
-    int32_t* ci = a.cand_idx + (size_t)b * a.Ncap;
-    uint32_t* tot = a.totals + (size_t)b * kTotals;
+    const int d1 = (int)ld_cg_u32(tot + kTotBin);
+    const float E = __uint_as_float(ld_cg_u32(tot + kTotE));
+    if (tid == 0) {
+        s_cnt = 0;
+        s_in = 0;
+    }
+    const FilterBounds fb = filter_bounds(d1, E);
+    const uint32_t in_key = score_key(fb.in_above), lo_key = score_key(fb.c_lo);  // order-preserving
+    uint32_t* ck = a.cand_key + (size_t)b * a.Ncap + row0;
+    int32_t* ci = a.cand_idx + (size_t)b * a.Ncap + row0;
     uint32_t* bm = a.bitmap + (size_t)b * a.Wcap;
     uint32_t* h2 = a.hist2 + (size_t)b * kBins;
-#pragma unroll
-    for (int u = 0; u < kBins / kSelThreads; ++u) S.hist[u * kSelThreads + tid] = hv[u];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) e = fmaxf(e, __shfl_xor_sync(0xFFFFFFFFu, e, o));
-    if (lane == 0) S.red[warp] = e;
     __syncthreads();
-    float E = 0.f;
-#pragma unroll
-    for (int w = 0; w < kSelThreads / 32; ++w) E = fmaxf(E, S.red[w]);
-    int d1;
-    uint32_t above1;
-    find_digit_desc<kBins>(S.hist, (uint32_t)k, S.sh32, &d1, &above1, S.res);
-    if (d1 < 0) d1 = 0;  // cannot happen: the histogram counts all n > k keys
-    const FilterBounds fb = filter_bounds(d1, E);
-    if (c == 0 && tid == 0) {  // the resolve reads these from here
-        tot[kTotBin] = (uint32_t)d1;
-        tot[kTotE] = __float_as_uint(E);
-        tot[kTotAbove] = above1;
-    }
-
     uint32_t nin = 0;
-    for (int p0 = row0; p0 < row1; p0 += kSelKPT * kSelThreads) {  // passes of up to 4096 rows
+#pragma unroll 1
+    for (int p0 = row0; p0 < row1; p0 += kFiltRows) {  // one pass unless the chunk is larger
         if (p0 != row0) {
 #pragma unroll
-            for (int i = 0; i < kSelKPT; ++i) {
+            for (int i = 0; i < kFiltKPT; ++i) {
                 const int row = p0 + i * kSelThreads + tid;
                 kr[i] = row < row1 ? __ldcg(keys + row) : 0u;
             }
         }
-        uint32_t cmask = 0, mycnt = 0;
 #pragma unroll
-        for (int i = 0; i < kSelKPT; ++i) {
+        for (int i = 0; i < kFiltKPT; ++i) {
             const int row = p0 + i * kSelThreads + tid;
             const int wrow = p0 + i * kSelThreads + warp * 32;  // this warp's 32 consecutive rows
-            const float sv = key_to_float(kr[i]);
             const bool valid = row < row1;
-            const bool sel = valid && sv > fb.in_above;
-            const bool cand = valid && !sel && sv >= fb.c_lo;
+            const bool sel = valid && kr[i] > in_key;
             const uint32_t selm = __ballot_sync(0xFFFFFFFFu, sel);
             if (lane == 0 && wrow < row1) bm[wrow >> 5] = selm;  // row0 is a multiple of 32
             nin += __popc(selm);
-            if (cand) {
-                cmask |= 1u << i;
-                ++mycnt;
+            if (valid && !sel && kr[i] >= lo_key) {
+                const uint32_t p = atom_add_shared(&s_cnt, 1u);
+                ck[p] = kr[i];
+                ci[p] = row;
                 if ((int)(kr[i] >> 21) == d1) atomicAdd(h2 + ((kr[i] >> 10) & (kBins - 1)), 1u);
             }
         }
-        uint32_t total;
-        uint32_t pos = block_exclusive_scan(mycnt, S.sh32, &total);
-        if (total) {  // one append per pass to the sequence's candidate list
-            if (tid == 0) S.last = atomicAdd(&tot[kTotCand], total);
-            __syncthreads();
-            pos += S.last;
-            if (pos + mycnt > (uint32_t)a.Ncap) {  // cannot happen: at most n candidates
-                flag(DEV_LEN);
-                mycnt = 0;
-                cmask = 0;
-            }
-#pragma unroll
-            for (int i = 0; i < kSelKPT; ++i) {
-                if ((cmask >> i) & 1u) {
-                    ck[pos] = kr[i];
-                    ci[pos] = p0 + i * kSelThreads + tid;
-                    ++pos;
-                }
-            }
-            __syncthreads();  // S.last is reused
-        }
     }
-    if (lane == 0) S.amb_key[warp] = nin;  // (scratch) the warp's sure-ins: every lane counted the ballots
+    if (lane == 0 && nin) red_add_shared(&s_in, nin);  // every lane counted the same ballots
     __syncthreads();
-    if (tid == 0) {  // every chunk writes its count, empty chunks too
-        uint32_t s_in = 0;
-        for (int w = 0; w < kSelThreads / 32; ++w) s_in += S.amb_key[w];
-        a.chunk_in[(size_t)b * a.nchunks + c] = s_in;
+    if (tid == 0) {
+        a.chunk_in[(size_t)b * a.nfch + c] = s_in;
+        a.chunk_cnt[(size_t)b * a.nfch + c] = s_cnt;
     }
 }
 
-// One CTA of 1024 threads per sequence: finds t~ among the filter's
-// candidates, rescores the band exactly, ranks it by (s, -j), adds the
-// winners to the selection bitmap and gives every chunk the output position
-// of its first selected entry.
-__global__ void __launch_bounds__(kResThreads, 1) topk_resolve_kernel(TopkDecodeArgs a) {
-    extern __shared__ __align__(16) uint32_t csm[];  // [kSelCap] keys, [kSelCap] indices
-    __shared__ SelSmem S;
-    pdl_wait();
-    pdl_release();
-    const int b = blockIdx.x;
-    const int tid = threadIdx.x;
-    const int n = clamp_n(a.n, b, a.Ncap);
-    const int k = a.k;
-    if (n <= k) return;  // the filter wrote the whole answer
-    // issue every load first
-    const uint32_t* tot = a.totals + (size_t)b * kTotals;
-    uint32_t C = __ldcg(tot + kTotCand);
-    const int d1 = (int)__ldcg(tot + kTotBin);
-    const float E = __uint_as_float(__ldcg(tot + kTotE));
-    const uint32_t above1 = __ldcg(tot + kTotAbove);
-    const uint32_t cin = tid < a.nchunks ? __ldcg(a.chunk_in + (size_t)b * a.nchunks + tid) : 0u;
-    const uint32_t h2a = __ldcg(a.hist2 + (size_t)b * kBins + tid);
-    const uint32_t h2b = __ldcg(a.hist2 + (size_t)b * kBins + kResThreads + tid);
-    load_q2(S.q2, a.q_idx + (size_t)b * 64);
-    if (C > (uint32_t)a.Ncap) {
-        if (tid == 0) flag(DEV_LEN);
-        C = a.Ncap;
-    }
-    const bool fits = C <= (uint32_t)kSelCap;
+// The resolve once the counts are scanned, over the candidate list held in
+// shared memory (SMEM, the usual case) or in global memory (overflow).
+// Gathers the chunks' candidates into one list (collecting the keys of the
+// fine bin of t~ and prefetching into L2 the index rows around it, which
+// the exact rescoring of the band will read), finds t~, rescores the band
+// exactly, cuts it by (s, -j), adds the winners to the bitmap and gives
+// every chunk its output position.
+template <bool SMEM>
+__device__ __forceinline__ void resolve_body(const TopkDecodeArgs& a, SelSmem& S, uint32_t* csm, int b, uint32_t C,
+                                             uint32_t A, int d1, float E, int d2, uint32_t above2, uint32_t K2,
+                                             const uint32_t (&pk)[kGatherJ], const int32_t (&pi)[kGatherJ],
+                                             uint32_t cin) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int k = a.k, nfch = a.nfch;
+    uint32_t* lk = SMEM ? csm : a.cmp_key + (size_t)b * a.Ncap;
+    int32_t* li = SMEM ? reinterpret_cast<int32_t*>(csm + kSelCap) : a.cmp_idx + (size_t)b * a.Ncap;
     const uint32_t* gk = a.cand_key + (size_t)b * a.Ncap;
     const int32_t* gi = a.cand_idx + (size_t)b * a.Ncap;
-    // the candidate list: copied to shared memory when it fits, else read in place
-    const uint32_t* lk = fits ? csm : gk;
-    const int32_t* li = fits ? reinterpret_cast<const int32_t*>(csm + kSelCap) : gi;
-    if (fits) {
-        constexpr int U = 4;  // loads first, then the stores
-        for (uint32_t e0 = 0; e0 < C; e0 += U * kResThreads) {
-            uint32_t kv[U];
-            int32_t iv[U];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const uint32_t e_ = e0 + u * kResThreads + tid;
-                kv[u] = e_ < C ? __ldcg(gk + e_) : 0u;
-                iv[u] = e_ < C ? __ldcg(gi + e_) : 0;
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const uint32_t e_ = e0 + u * kResThreads + tid;
-                if (e_ < C) {
-                    csm[e_] = kv[u];
-                    csm[kSelCap + e_] = (uint32_t)iv[u];
-                }
+    const uint16_t* icx = a.kidx + (size_t)b * a.Ncap * 64;
+    const uint32_t pre = ((uint32_t)d1 << 11) | (uint32_t)(d2 < 0 ? 0 : d2);
+    auto put = [&](uint32_t pos, uint32_t kk, int32_t j) {
+        lk[pos] = kk;
+        li[pos] = j;
+        const uint32_t f = kk >> 10;
+        if (d2 >= 0 && f + 2 >= pre && f <= pre + 2) {
+            prefetch_l2(icx + (size_t)j * 64);
+            if (f == pre) {
+                const uint32_t p = atom_add_shared(&S.f_cnt, 1u);
+                if (p < (uint32_t)kResThreads) S.amb_key[p] = kk;
             }
         }
+    };
+#pragma unroll
+    for (int j = 0; j < kGatherJ; ++j) {
+        const int c = warp + 32 * j;
+        if (c < nfch && (uint32_t)lane < S.ccnt[c]) put(S.base[c] + lane, pk[j], pi[j]);
     }
-    S.hist[tid] = h2a;
-    S.hist[kResThreads + tid] = h2b;
-    if (tid == 0) S.amb_cnt = 0;
-    uint32_t A;
-    block_exclusive_scan(cin, S.sh32, &A);  // surely selected entries of the sequence
-    const uint32_t R1 = (uint32_t)k - A;    // rank of t~ among the candidates (>= 1)
-    const uint32_t K2 = (uint32_t)k - above1;
+#pragma unroll 1
+    for (int c = warp; c < nfch; c += 32) {  // slots beyond 32, chunks beyond the first kGatherJ per warp
+        const uint32_t cn = S.ccnt[c], cb = S.base[c];
+        const uint32_t from = c < 32 * kGatherJ ? 32u : 0u;
+        for (uint32_t i = from + lane; i < cn; i += 32)
+            put(cb + i, __ldcg(gk + (size_t)c * a.fchunk + i), __ldcg(gi + (size_t)c * a.fchunk + i));
+    }
+    if (!SMEM) __threadfence_block();
+    __syncthreads();
 
-    const uint32_t tkey = find_threshold(lk, li, C, R1, d1, K2, S);
+    // t~: the R3-th largest key of the fine bin (few keys: ranked pairwise)
+    const uint32_t R1 = (uint32_t)k - A;  // rank of t~ among the candidates (>= 1)
+    bool fast = false;
+    if (d2 >= 0) {
+        const uint32_t nf = S.f_cnt;
+        const uint32_t R3 = K2 - above2;
+        if (nf <= (uint32_t)kResThreads && R3 >= 1 && R3 <= nf) {
+            if ((uint32_t)tid < nf) {
+                const uint32_t mk = S.amb_key[tid];
+                uint32_t gt = 0, ge = 0;
+                for (uint32_t o = 0; o < nf; ++o) {
+                    const uint32_t ok = S.amb_key[o];
+                    gt += ok > mk;
+                    ge += ok >= mk;
+                }
+                if (gt < R3 && R3 <= ge) {  // every thread holding t~ writes the same value
+                    S.tkey = mk;
+                    S.found = 1;
+                }
+            }
+            __syncthreads();
+            fast = S.found != 0;
+        }
+    }
+    uint32_t tkey;
+    if (fast) {
+        tkey = S.tkey;
+    } else if (!rank_in_bin(lk, C, R1, d1, S.hist, S.sh64, S.res, &tkey)) {
+        int32_t jd;
+        select_rank(lk, li, C, R1, S.hist, S.sh64, S.res, &tkey, &jd);
+    }
     const float t = key_to_float(tkey);
     const float e2 = __fmul_ru(2.f, E);
-    const float band_hi = __fadd_ru(t, e2), band_lo = __fsub_rd(t, e2);
-    const uint16_t* icx = a.kidx + (size_t)b * a.Ncap * 64;
+    const uint32_t bhi_key = score_key(__fadd_ru(t, e2)), blo_key = score_key(__fsub_rd(t, e2));
     // the band list (global, used when the band is large)
     uint32_t* gak = a.amb_key + (size_t)b * a.Ncap;
     int32_t* gai = a.amb_idx + (size_t)b * a.Ncap;
@@ -701,10 +739,10 @@ __global__ void __launch_bounds__(kResThreads, 1) topk_resolve_kernel(TopkDecode
     uint32_t my_in2 = 0;
 #pragma unroll 1
     for (uint32_t i = tid; i < C; i += kResThreads) {
-        const float sv = key_to_float(lk[i]);
-        if (sv > band_hi) {
+        const uint32_t kk = lk[i];
+        if (kk > bhi_key) {
             ++my_in2;
-        } else if (sv >= band_lo) {
+        } else if (kk >= blo_key) {
             const int32_t j = li[i];
             const uint32_t p = atom_add_shared(&S.amb_cnt, 1u);
             const uint32_t ek = exact_key(S.q2, icx + (size_t)j * 64);
@@ -717,7 +755,7 @@ __global__ void __launch_bounds__(kResThreads, 1) topk_resolve_kernel(TopkDecode
         }
     }
     uint32_t in2;
-    block_exclusive_scan(my_in2, S.sh32, &in2);
+    block_exclusive_scan(my_in2, S.sh64, &in2);
     const uint32_t na = S.amb_cnt;
     const uint32_t R2 = R1 - in2;  // winners to take from the band (1 <= R2 <= na)
     // the exact cut of the band: a member wins iff (key, -j) >= (T2, -jmax2)
@@ -737,10 +775,11 @@ __global__ void __launch_bounds__(kResThreads, 1) topk_resolve_kernel(TopkDecode
         }
         __syncthreads();
     } else {
+        __threadfence_block();
         __syncthreads();
         uint32_t T2;
         int32_t jmax2;
-        select_rank(gak, gai, na, R2, S.hist, S.sh32, S.res, &T2, &jmax2);
+        select_rank(gak, gai, na, R2, S.hist, S.sh64, S.res, &T2, &jmax2);
         if (tid == 0) {
             S.T2 = T2;
             S.jmax2 = jmax2;
@@ -756,10 +795,10 @@ __global__ void __launch_bounds__(kResThreads, 1) topk_resolve_kernel(TopkDecode
     __syncthreads();
 #pragma unroll 1
     for (uint32_t i = tid; i < C; i += kResThreads) {
-        if (key_to_float(lk[i]) > band_hi) {
+        if (lk[i] > bhi_key) {
             const int32_t j = li[i];
             atomicOr(&bm[j >> 5], 1u << (j & 31));
-            red_add_shared(&wc[j / a.chunk], 1u);
+            red_add_shared(&wc[j / a.fchunk], 1u);
         }
     }
 #pragma unroll 1
@@ -768,23 +807,92 @@ __global__ void __launch_bounds__(kResThreads, 1) topk_resolve_kernel(TopkDecode
         const int32_t j = na <= (uint32_t)kResThreads ? S.amb_idx[i] : __ldcg(gai + i);
         if (kk > T2 || (kk == T2 && j <= jmax2)) {
             atomicOr(&bm[j >> 5], 1u << (j & 31));
-            red_add_shared(&wc[j / a.chunk], 1u);
+            red_add_shared(&wc[j / a.fchunk], 1u);
         }
     }
     __syncthreads();
     // output position of every chunk's first selected entry
-    const uint32_t v = tid < a.nchunks ? cin + wc[tid] : 0u;
+    const uint32_t v = tid < nfch ? cin + wc[tid] : 0u;
     uint32_t total;
-    const uint32_t pos = block_exclusive_scan(v, S.sh32, &total);
-    if (tid < a.nchunks) a.chunk_pos[(size_t)b * a.nchunks + tid] = pos;
+    const uint32_t pos = block_exclusive_scan(v, S.sh64, &total);
+    if (tid < nfch) a.chunk_pos[(size_t)b * nfch + tid] = pos;
     if (tid == 0) {
         if (total != (uint32_t)k) flag(DEV_LEN);  // cannot happen
         a.cnt[b] = k;
     }
 }
 
-// Emit: one CTA per (chunk, sequence) writes its chunk's selected indices,
-// ascending, from its output position on.
+// One CTA of 1024 threads per sequence.  One round trip brings the totals,
+// every chunk's counts, the second histogram (two bins per thread, kept in
+// registers) and, ahead of their counts, the first 32 candidate slots of
+// each warp's first kGatherJ chunks; the fine bin of t~ then follows from
+// the registers.
+__global__ void __launch_bounds__(kResThreads, 1) topk_resolve_kernel(TopkDecodeArgs a) {
+    extern __shared__ __align__(16) uint32_t csm[];  // [kSelCap] keys, [kSelCap] indices
+    __shared__ SelSmem S;
+    pdl_wait();
+    pdl_release();
+    const int b = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n = clamp_n(a.n, b, a.Ncap);
+    const int k = a.k;
+    if (n <= k) return;  // the filter wrote the whole answer
+    const int nfch = a.nfch;
+    const uint32_t* tot = a.totals + (size_t)b * kTotals;
+    const int d1 = (int)ld_cg_u32(tot + kTotBin);
+    const float E = __uint_as_float(ld_cg_u32(tot + kTotE));
+    const uint32_t above1 = ld_cg_u32(tot + kTotAbove);
+    const uint32_t cin = tid < nfch ? ld_cg_u32(a.chunk_in + (size_t)b * nfch + tid) : 0u;
+    const uint32_t ccn = tid < nfch ? ld_cg_u32(a.chunk_cnt + (size_t)b * nfch + tid) : 0u;
+    uint32_t h2[2];
+    {
+        const uint2 x = ld_cg_u32x2(a.hist2 + (size_t)b * kBins + (kResThreads - 1 - tid) * 2);
+        h2[0] = x.x;
+        h2[1] = x.y;
+    }
+    const uint32_t* gk = a.cand_key + (size_t)b * a.Ncap;
+    const int32_t* gi = a.cand_idx + (size_t)b * a.Ncap;
+    uint32_t pk[kGatherJ];
+    int32_t pi[kGatherJ];
+#pragma unroll
+    for (int j = 0; j < kGatherJ; ++j) {
+        const int c = warp + 32 * j;
+        const int r = c * a.fchunk + lane;
+        const bool ok = c < nfch && r < n;
+        pk[j] = ok ? ld_cg_u32(gk + r) : 0u;
+        pi[j] = ok ? (int32_t)ld_cg_u32(gi + r) : 0;
+    }
+    load_q2(S.q2, a.q_idx + (size_t)b * 64);
+    if (tid == 0) {
+        S.amb_cnt = 0;
+        S.f_cnt = 0;
+        S.found = 0;
+    }
+    // the fine bin d2 of t~ inside bin d1 (rank K2 there)
+    const uint32_t K2 = (uint32_t)k - above1;
+    int d2;
+    uint32_t above2;
+    find_digit_desc_regs<2>(h2, K2, S.sh64, S.res, &d2, &above2);
+    uint32_t base, ain, C, A;
+    block_exclusive_scan2(ccn, cin, S.sh64, &base, &ain, &C, &A);
+    if (tid < nfch) {
+        S.base[tid] = base;
+        S.ccnt[tid] = ccn;
+    }
+    __syncthreads();
+    if (C > (uint32_t)a.Ncap) {  // cannot happen: at most n candidates
+        if (tid == 0) flag(DEV_LEN);
+        C = a.Ncap;
+    }
+    if (C <= (uint32_t)kSelCap)
+        resolve_body<true>(a, S, csm, b, C, A, d1, E, d2, above2, K2, pk, pi, cin);
+    else
+        resolve_body<false>(a, S, csm, b, C, A, d1, E, d2, above2, K2, pk, pi, cin);
+    (void)ain;
+}
+
+// Emit: one CTA per filter chunk writes its selected indices, ascending,
+// from its output position on.
 constexpr int kEmitThreads = 256;
 __global__ void __launch_bounds__(kEmitThreads) topk_emit_kernel(TopkDecodeArgs a) {
     __shared__ uint32_t sh32[32];
@@ -793,13 +901,13 @@ __global__ void __launch_bounds__(kEmitThreads) topk_emit_kernel(TopkDecodeArgs 
     const int b = blockIdx.y, c = blockIdx.x;
     const int n = clamp_n(a.n, b, a.Ncap);
     if (n <= a.k) return;
-    const int row0 = c * a.chunk;
-    const int row1 = min(row0 + a.chunk, n);
+    const int row0 = c * a.fchunk;
+    const int row1 = min(row0 + a.fchunk, n);
     if (row0 >= row1) return;
     const uint32_t* bm = a.bitmap + (size_t)b * a.Wcap;
     int32_t* out = a.idx + (size_t)b * a.k;
     const int w0 = row0 >> 5, w1 = (row1 + 31) >> 5;
-    uint32_t pos = __ldcg(a.chunk_pos + (size_t)b * a.nchunks + c);
+    uint32_t pos = __ldcg(a.chunk_pos + (size_t)b * a.nfch + c);
 #pragma unroll 1
     for (int wb = w0; wb < w1; wb += kEmitThreads) {  // block-uniform trip count
         const int w = wb + threadIdx.x;
