@@ -99,6 +99,15 @@ __global__ void __launch_bounds__(NW * EG * 32) attn_split_kernel(AttnArgs a) {
     const int split = CLUSTER ? blockIdx.x : blockIdx.y;
     const int bq = CLUSTER ? blockIdx.y : blockIdx.x;
     const int b = bq / a.Tq;
+    constexpr int TPR = NT / kTileN;  // threads per row of a tile
+    const int p_begin = split * a.tiles_per_split * kTileN;
+    // the list entries of the first tiles go out before the counts are known
+    int jpre[ST - 1];
+#pragma unroll
+    for (int s = 0; s < ST - 1; ++s) {
+        const int p = p_begin + s * kTileN + tid / TPR;
+        jpre[s] = GATHER && p < a.kmax ? (int)ld_cg_u32(a.idx + (size_t)bq * a.kmax + p) : 0;
+    }
     int nb = a.n[b];
     if (nb < 0 || nb > a.Ncap) {
         if (tid == 0 && split == 0) flag(DEV_LEN);
@@ -124,7 +133,6 @@ __global__ void __launch_bounds__(NW * EG * 32) attn_split_kernel(AttnArgs a) {
             }
         }
     }
-    const int p_begin = split * a.tiles_per_split * kTileN;
     const int p_end = min(R, p_begin + a.tiles_per_split * kTileN);
     const int ntiles = p_end > p_begin ? (p_end - p_begin + kTileN - 1) / kTileN : 0;
 
@@ -150,10 +158,9 @@ __global__ void __launch_bounds__(NW * EG * 32) attn_split_kernel(AttnArgs a) {
 
     // each thread copies CPT 16-byte chunks of one row; a gathered row costs one index load
     constexpr int cpr = FP8 ? 8 : 16;            // 16-byte chunks per row
-    constexpr int TPR = NT / kTileN;             // threads per row
     constexpr int CPT = cpr / TPR;               // chunks per thread
     static_assert(TPR >= 1 && CPT >= 1 && CPT * TPR == cpr, "tile mapping");
-    auto load_tile = [&](int tile, int stage) {
+    auto load_tile = [&](int tile, int stage, int jv, bool have_j) {
         const int p0 = p_begin + tile * kTileN;
         uint8_t* rk = sRaw + (stage * 2 + 0) * L::kStageRaw;
         uint8_t* rv = sRaw + (stage * 2 + 1) * L::kStageRaw;
@@ -162,7 +169,7 @@ __global__ void __launch_bounds__(NW * EG * 32) attn_split_kernel(AttnArgs a) {
         int j = p;
         bool ok = p < p_end;
         if (GATHER && ok) {
-            j = a.idx[(size_t)bq * a.kmax + p];
+            j = have_j ? jv : a.idx[(size_t)bq * a.kmax + p];
             if (j < 0 || j >= nb) {
                 ok = false;
                 if (c0 == 0) flag(DEV_INDEX);
@@ -188,7 +195,7 @@ __global__ void __launch_bounds__(NW * EG * 32) attn_split_kernel(AttnArgs a) {
 
 #pragma unroll
     for (int s = 0; s < ST - 1; ++s) {
-        if (s < ntiles) load_tile(s, s);
+        if (s < ntiles) load_tile(s, s, jpre[s], true);
         cp_async_commit();
     }
 
@@ -201,7 +208,7 @@ __global__ void __launch_bounds__(NW * EG * 32) attn_split_kernel(AttnArgs a) {
 
     for (int t = 0; t < ntiles; ++t) {
         const int stage = t % ST;
-        if (t + ST - 1 < ntiles) load_tile(t + ST - 1, (t + ST - 1) % ST);
+        if (t + ST - 1 < ntiles) load_tile(t + ST - 1, (t + ST - 1) % ST, 0, false);
         cp_async_commit();
         cp_async_wait<ST - 1>();  // Q (first group) and tile t have landed
         __syncthreads();

@@ -196,7 +196,7 @@ sa_status make_ic_map(CUtensorMap* map, const void* kidx, int B, int Ncap) {
 
 // ------------------------------------------------------- workspace layout --
 struct TopkDecodeWs {
-    size_t hist, hist2, totals, zero_end, keys, emax, chunk_in, chunk_cnt, chunk_pos, cand_key, cand_idx, cmp_key,
+    size_t hist, hist2, totals, zero_end, keys, emax, chunk_in, chunk_cnt, chunk_pos, cslot, cand_key, cand_idx, cmp_key,
         cmp_idx, amb_key, amb_idx, bitmap, idx, cnt, total;
     int maxchunks, fchunk, nfch, Wcap;
 };
@@ -217,9 +217,12 @@ int score_chunk(int B, int Ncap) {
     return (int)std::max<long long>(chunk, sa::kScRows);
 }
 
-// [reserved 256 B][histograms][second histograms][totals]  (zeroed per call)
-// [keys][per-score-chunk max error][per-filter-chunk sure-ins, candidates, output positions]
-// [candidates key/idx][compact candidates key/idx][band key/idx][bitmap][idx][cnt]
+// Small per-call arrays first, so that the latency-bound selection kernels
+// touch few pages: [reserved 256 B][histograms][second histograms][totals]
+// (zeroed per call) [per-score-chunk max error][per-filter-chunk sure-ins,
+// candidates, output positions][compact candidate slots][bitmap], then the
+// large ones: [keys][further candidates key/idx][compact list key/idx]
+// [band key/idx][idx][cnt].
 TopkDecodeWs topk_decode_layout(int B, int Ncap, int k, bool own_idx) {
     TopkDecodeWs w{};
     w.maxchunks = std::max(1, cdiv(Ncap, sa::kScRows));
@@ -237,8 +240,6 @@ TopkDecodeWs topk_decode_layout(int B, int Ncap, int k, bool own_idx) {
     o = up256(o);
     const size_t col = up256((size_t)B * Ncap * 4);
     const size_t per_fch = up256((size_t)B * w.nfch * 4);
-    w.keys = o;
-    o += col;
     w.emax = o;
     o += up256((size_t)B * w.maxchunks * 4);
     w.chunk_in = o;
@@ -247,6 +248,12 @@ TopkDecodeWs topk_decode_layout(int B, int Ncap, int k, bool own_idx) {
     o += per_fch;
     w.chunk_pos = o;
     o += per_fch;
+    w.cslot = o;
+    o += up256((size_t)B * w.nfch * sa::kSlots * 8);
+    w.bitmap = o;
+    o += up256((size_t)B * w.Wcap * 4);
+    w.keys = o;
+    o += col;
     w.cand_key = o;
     o += col;
     w.cand_idx = o;
@@ -259,8 +266,6 @@ TopkDecodeWs topk_decode_layout(int B, int Ncap, int k, bool own_idx) {
     o += col;
     w.amb_idx = o;
     o += col;
-    w.bitmap = o;
-    o += up256((size_t)B * w.Wcap * 4);
     w.idx = o;
     if (own_idx) o += up256((size_t)B * k * 4);
     w.cnt = o;
@@ -438,6 +443,7 @@ sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* 
     a.chunk_in = reinterpret_cast<uint32_t*>(base + w.chunk_in);
     a.chunk_cnt = reinterpret_cast<uint32_t*>(base + w.chunk_cnt);
     a.chunk_pos = reinterpret_cast<uint32_t*>(base + w.chunk_pos);
+    a.cslot = reinterpret_cast<uint2*>(base + w.cslot);
     a.cand_key = reinterpret_cast<uint32_t*>(base + w.cand_key);
     a.cand_idx = reinterpret_cast<int32_t*>(base + w.cand_idx);
     a.cmp_key = reinterpret_cast<uint32_t*>(base + w.cmp_key);

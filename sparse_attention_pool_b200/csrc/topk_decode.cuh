@@ -54,6 +54,7 @@ constexpr int kBinsLow = 1024;    // last 10-bit digit
 constexpr int kTotals = 4;
 constexpr int kTotTicket = 0, kTotBin = 1, kTotE = 2, kTotAbove = 3;
 constexpr int kFiltRows = 1024;  // rows per filter / emit CTA (one pass of 256 threads x 4 keys)
+constexpr int kSlots = 64;       // compact candidate slots per filter chunk
 
 struct TopkDecodeArgs {
     const uint16_t* q_idx;  // [B][64]
@@ -66,7 +67,8 @@ struct TopkDecodeArgs {
     uint32_t* chunk_in;     // [B][nfch]     per filter chunk: surely selected entries
     uint32_t* chunk_cnt;    // [B][nfch]     per filter chunk: candidates
     uint32_t* chunk_pos;    // [B][nfch]     output position of each filter chunk's first selected entry
-    uint32_t* cand_key;     // [B][Ncap]     candidates, each filter chunk in its own rows
+    uint2* cslot;           // [B][nfch][kSlots] the first kSlots candidates of each filter chunk (key, index)
+    uint32_t* cand_key;     // [B][Ncap]     further candidates of a chunk, in the chunk's own rows
     int32_t* cand_idx;      // [B][Ncap]
     uint32_t* cmp_key;      // [B][Ncap]     all candidates in one list, when they overflow shared memory
     int32_t* cmp_idx;       // [B][Ncap]
@@ -97,12 +99,15 @@ __device__ __forceinline__ float key_to_float(uint32_t key) {
 // q2 holds qI[i] * 2^768 in fp64 (see below); the row's bf16 values enter as
 // x * 2^-896 through bit placement, so each product is qI*k * 2^-128 exactly
 // and no conversion instruction is needed per element.
+// SMEM: the row is staged in shared memory (read with ordinary loads);
+// otherwise it is read from global memory through the read-only path.
+template <bool SMEM = false>
 __device__ __noinline__ uint32_t exact_key(const double* q2, const uint16_t* row) {
     const uint4* r4 = reinterpret_cast<const uint4*>(row);
     double acc = 0.0;
 #pragma unroll 2
     for (int c = 0; c < 8; ++c) {
-        const uint4 w = __ldg(r4 + c);
+        const uint4 w = SMEM ? r4[c] : __ldg(r4 + c);
         acc = fma(q2[8 * c + 0], bf16lo_scaled(w.x), acc);
         acc = fma(q2[8 * c + 1], bf16hi_scaled(w.x), acc);
         acc = fma(q2[8 * c + 2], bf16lo_scaled(w.y), acc);
@@ -389,11 +394,31 @@ __global__ void __launch_bounds__(kScThreads, 3)
     pdl_wait();
     pdl_release();
     const int b = blockIdx.y;
-    const int n = clamp_n(a.n, b, a.Ncap);
-    if (n <= a.k) return;  // everything visible is selected; nothing to score
-    const int row0 = blockIdx.x * a.chunk;
-    const int row1 = min(row0 + a.chunk, n);
     const int tid = threadIdx.x;
+    const int row0 = blockIdx.x * a.chunk;
+    // The first tiles go out before the length is known: rows below Ncap
+    // exist in the cache whatever n is (rows at or past n are read, not used).
+    // The map views Ic as [B][Ncap][64]: coordinates (dim, row, sequence).
+    const int srows = max(0, min(row0 + a.chunk, a.Ncap) - row0);
+    const int stiles = (srows + kScRows - 1) / kScRows;
+    int issued = 0;
+    if (tid == 0) {
+        for (int s = 0; s < kScStages; ++s) mbar_init(&full[s], 1);
+        fence_barrier_init();
+        for (; issued < kScStages && issued < stiles; ++issued) {
+            mbar_expect_tx(&full[issued], kScTileBytes);
+            tma_load_3d(tiles + issued * kScTileBytes, &ic_map, 0, row0 + issued * kScRows, b, &full[issued]);
+        }
+    }
+    const int n = clamp_n(a.n, b, a.Ncap);
+    if (n <= a.k) {
+        // everything visible is selected, nothing to score; the early copies
+        // land before the CTA's shared memory goes away
+        if (tid == 0)
+            for (int i = 0; i < issued; ++i) mbar_wait(&full[i % kScStages], (i / kScStages) & 1);
+        return;
+    }
+    const int row1 = min(row0 + a.chunk, n);
     // an empty chunk scans nothing but still takes part in the finish below
     const int ntiles = row1 > row0 ? (row1 - row0 + kScRows - 1) / kScRows : 0;
 
@@ -408,20 +433,8 @@ __global__ void __launch_bounds__(kScThreads, 3)
         }
     }
     for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0;
-    if (tid == 0) {
-        for (int s = 0; s < kScStages; ++s) mbar_init(&full[s], 1);
-        fence_barrier_init();
-    }
     __syncthreads();
 
-    // the map views Ic as [B][Ncap][64]: coordinates (dim, row, sequence)
-    int issued = 0;
-    if (tid == 0) {
-        for (; issued < kScStages && issued < ntiles; ++issued) {
-            mbar_expect_tx(&full[issued], kScTileBytes);
-            tma_load_3d(tiles + issued * kScTileBytes, &ic_map, 0, row0 + issued * kScRows, b, &full[issued]);
-        }
-    }
     int consumed = 0;
     bool timed_out = false;
     float emax = 0.f;
@@ -463,13 +476,12 @@ __global__ void __launch_bounds__(kScThreads, 3)
             ++issued;
         }
     }
-    if (timed_out) {
-        // let copies still in flight land before the CTA's shared memory goes away
-        // (the device status records the timeout; the results are not used)
-        if (tid == 0)
-            for (int i = consumed; i < issued; ++i) mbar_wait(&full[i % kScStages], (i / kScStages) & 1);
-        __syncthreads();
-    }
+    // copies not consumed (tiles issued past the chunk's end, or after a
+    // timeout, which the device status records) land before the CTA's shared
+    // memory goes away
+    if (tid == 0)
+        for (int i = consumed; i < issued; ++i) mbar_wait(&full[i % kScStages], (i / kScStages) & 1);
+    if (timed_out) __syncthreads();
     // e_j is rounded to nearest in fp32: one more ulp keeps it an upper bound
     emax = __uint_as_float(__float_as_uint(emax) + 1u);
 #pragma unroll
@@ -540,6 +552,7 @@ constexpr int kSelCap = 8192;                // candidates the resolving CTA hol
 constexpr int kSelSmem = kSelCap * 8;
 constexpr int kSelMaxChunks = 1024;          // filter chunks per sequence
 constexpr int kGatherJ = 8;                  // filter chunks per warp loaded ahead by the resolve
+constexpr int kPf = 64;                      // index rows staged for the band
 static_assert(kSelMaxChunks <= kResThreads, "the resolve gives one thread to every chunk");
 static_assert(kBins == 2 * kResThreads, "the resolve loads the second histogram two bins per thread");
 static_assert(kFiltKPT * kSelThreads == kFiltRows, "one filter pass covers a chunk");
@@ -566,10 +579,15 @@ struct SelSmem {
     uint32_t ccnt[kSelMaxChunks];   // candidates per filter chunk
     uint32_t sh64[64];
     int res[2];
-    uint32_t f_cnt, found, tkey, amb_cnt, T2;
+    uint32_t f_cnt, found, tkey, amb_cnt, T2, pf_cnt;
     int32_t jmax2;
     uint32_t amb_key[kResThreads];  // the fine bin's keys, then the band's exact keys
     int32_t amb_idx[kResThreads];
+    // index rows of the candidates within two fine bins of t~'s, staged for
+    // the exact rescoring of the band
+    uint32_t pf_key[kPf];
+    int32_t pf_j[kPf];
+    __align__(16) uint16_t pf_row[kPf][64];
 };
 
 // Filter: one CTA per 1024 rows.  Entries above the widened bin of t~ become
@@ -582,8 +600,22 @@ __global__ void __launch_bounds__(kSelThreads) topk_filter_kernel(TopkDecodeArgs
     pdl_release();
     const int b = blockIdx.y, c = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int n = clamp_n(a.n, b, a.Ncap);
     const int k = a.k;
+    const int row0 = c * a.fchunk;
+    const int rcap = min(row0 + a.fchunk, a.Ncap);  // rows present in the arrays
+    const uint32_t* keys = a.keys + (size_t)b * a.Ncap;
+    const uint32_t* tot = a.totals + (size_t)b * kTotals;
+    // every load goes out before the length is known: the first pass's keys
+    // and the thresholds (one round trip; none of them depends on n)
+    uint32_t kr[kFiltKPT];
+#pragma unroll
+    for (int i = 0; i < kFiltKPT; ++i) {
+        const int row = row0 + i * kSelThreads + tid;
+        kr[i] = row < rcap ? ld_cg_u32(keys + row) : 0u;
+    }
+    const int d1 = (int)ld_cg_u32(tot + kTotBin);
+    const float E = __uint_as_float(ld_cg_u32(tot + kTotE));
+    const int n = clamp_n(a.n, b, a.Ncap);
     if (n <= k) {
         if (c == 0) {
             int32_t* idx = a.idx + (size_t)b * k;
@@ -592,25 +624,14 @@ __global__ void __launch_bounds__(kSelThreads) topk_filter_kernel(TopkDecodeArgs
         }
         return;
     }
-    const int row0 = c * a.fchunk;
     const int row1 = min(row0 + a.fchunk, n);
-    const uint32_t* keys = a.keys + (size_t)b * a.Ncap;
-    const uint32_t* tot = a.totals + (size_t)b * kTotals;
-    // the first pass's keys go out with the thresholds: one round trip
-    uint32_t kr[kFiltKPT];
-#pragma unroll
-    for (int i = 0; i < kFiltKPT; ++i) {
-        const int row = row0 + i * kSelThreads + tid;
-        kr[i] = row < row1 ? ld_cg_u32(keys + row) : 0u;
-    }
-    const int d1 = (int)ld_cg_u32(tot + kTotBin);
-    const float E = __uint_as_float(ld_cg_u32(tot + kTotE));
     if (tid == 0) {
         s_cnt = 0;
         s_in = 0;
     }
     const FilterBounds fb = filter_bounds(d1, E);
     const uint32_t in_key = score_key(fb.in_above), lo_key = score_key(fb.c_lo);  // order-preserving
+    uint2* cs = a.cslot + ((size_t)b * a.nfch + c) * kSlots;
     uint32_t* ck = a.cand_key + (size_t)b * a.Ncap + row0;
     int32_t* ci = a.cand_idx + (size_t)b * a.Ncap + row0;
     uint32_t* bm = a.bitmap + (size_t)b * a.Wcap;
@@ -637,8 +658,12 @@ __global__ void __launch_bounds__(kSelThreads) topk_filter_kernel(TopkDecodeArgs
             nin += __popc(selm);
             if (valid && !sel && kr[i] >= lo_key) {
                 const uint32_t p = atom_add_shared(&s_cnt, 1u);
-                ck[p] = kr[i];
-                ci[p] = row;
+                if (p < (uint32_t)kSlots) {
+                    cs[p] = make_uint2(kr[i], (uint32_t)row);
+                } else {
+                    ck[p] = kr[i];
+                    ci[p] = row;
+                }
                 if ((int)(kr[i] >> 21) == d1) atomicAdd(h2 + ((kr[i] >> 10) & (kBins - 1)), 1u);
             }
         }
@@ -667,6 +692,7 @@ __device__ __forceinline__ void resolve_body(const TopkDecodeArgs& a, SelSmem& S
     const int k = a.k, nfch = a.nfch;
     uint32_t* lk = SMEM ? csm : a.cmp_key + (size_t)b * a.Ncap;
     int32_t* li = SMEM ? reinterpret_cast<int32_t*>(csm + kSelCap) : a.cmp_idx + (size_t)b * a.Ncap;
+    const uint2* cs = a.cslot + (size_t)b * nfch * kSlots;
     const uint32_t* gk = a.cand_key + (size_t)b * a.Ncap;
     const int32_t* gi = a.cand_idx + (size_t)b * a.Ncap;
     const uint16_t* icx = a.kidx + (size_t)b * a.Ncap * 64;
@@ -675,8 +701,15 @@ __device__ __forceinline__ void resolve_body(const TopkDecodeArgs& a, SelSmem& S
         lk[pos] = kk;
         li[pos] = j;
         const uint32_t f = kk >> 10;
-        if (d2 >= 0 && f + 2 >= pre && f <= pre + 2) {
-            prefetch_l2(icx + (size_t)j * 64);
+        if (d2 >= 0 && f + 2 >= pre && f <= pre + 2) {  // within two fine bins of t~'s
+            const uint32_t q = atom_add_shared(&S.pf_cnt, 1u);
+            if (q < (uint32_t)kPf) {
+                S.pf_key[q] = kk;
+                S.pf_j[q] = j;
+                const uint16_t* row = icx + (size_t)j * 64;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) cp_async16(&S.pf_row[q][u * 8], row + u * 8);
+            }
             if (f == pre) {
                 const uint32_t p = atom_add_shared(&S.f_cnt, 1u);
                 if (p < (uint32_t)kResThreads) S.amb_key[p] = kk;
@@ -692,9 +725,17 @@ __device__ __forceinline__ void resolve_body(const TopkDecodeArgs& a, SelSmem& S
     for (int c = warp; c < nfch; c += 32) {  // slots beyond 32, chunks beyond the first kGatherJ per warp
         const uint32_t cn = S.ccnt[c], cb = S.base[c];
         const uint32_t from = c < 32 * kGatherJ ? 32u : 0u;
-        for (uint32_t i = from + lane; i < cn; i += 32)
-            put(cb + i, __ldcg(gk + (size_t)c * a.fchunk + i), __ldcg(gi + (size_t)c * a.fchunk + i));
+        for (uint32_t i = from + lane; i < cn; i += 32) {
+            if (i < (uint32_t)kSlots) {
+                const uint2 e = cs[(size_t)c * kSlots + i];
+                put(cb + i, e.x, (int32_t)e.y);
+            } else {
+                put(cb + i, __ldcg(gk + (size_t)c * a.fchunk + i), __ldcg(gi + (size_t)c * a.fchunk + i));
+            }
+        }
     }
+    cp_async_commit();
+    cp_async_wait<0>();
     if (!SMEM) __threadfence_block();
     __syncthreads();
 
@@ -736,22 +777,38 @@ __device__ __forceinline__ void resolve_body(const TopkDecodeArgs& a, SelSmem& S
     uint32_t* gak = a.amb_key + (size_t)b * a.Ncap;
     int32_t* gai = a.amb_idx + (size_t)b * a.Ncap;
     __syncthreads();  // S.amb_key held the fine bin
+    // when the band lies inside the staged window, its members are all staged
+    const uint32_t lo_w = pre >= 2u ? (pre - 2u) << 10 : 0u;
+    const bool win = fast && S.pf_cnt <= (uint32_t)kPf && blo_key >= lo_w && (bhi_key >> 10) <= pre + 2u;
     uint32_t my_in2 = 0;
+    if (win) {
 #pragma unroll 1
-    for (uint32_t i = tid; i < C; i += kResThreads) {
-        const uint32_t kk = lk[i];
-        if (kk > bhi_key) {
-            ++my_in2;
-        } else if (kk >= blo_key) {
-            const int32_t j = li[i];
-            const uint32_t p = atom_add_shared(&S.amb_cnt, 1u);
-            const uint32_t ek = exact_key(S.q2, icx + (size_t)j * 64);
-            if (p < (uint32_t)kResThreads) {
-                S.amb_key[p] = ek;
-                S.amb_idx[p] = j;
+        for (uint32_t i = tid; i < C; i += kResThreads) my_in2 += lk[i] > bhi_key;
+        if ((uint32_t)tid < S.pf_cnt) {
+            const uint32_t kk = S.pf_key[tid];
+            if (kk >= blo_key && kk <= bhi_key) {
+                const uint32_t p = atom_add_shared(&S.amb_cnt, 1u);
+                S.amb_key[p] = exact_key<true>(S.q2, S.pf_row[tid]);
+                S.amb_idx[p] = S.pf_j[tid];
             }
-            gak[p] = ek;
-            gai[p] = j;
+        }
+    } else {
+#pragma unroll 1
+        for (uint32_t i = tid; i < C; i += kResThreads) {
+            const uint32_t kk = lk[i];
+            if (kk > bhi_key) {
+                ++my_in2;
+            } else if (kk >= blo_key) {
+                const int32_t j = li[i];
+                const uint32_t p = atom_add_shared(&S.amb_cnt, 1u);
+                const uint32_t ek = exact_key(S.q2, icx + (size_t)j * 64);
+                if (p < (uint32_t)kResThreads) {
+                    S.amb_key[p] = ek;
+                    S.amb_idx[p] = j;
+                }
+                gak[p] = ek;
+                gai[p] = j;
+            }
         }
     }
     uint32_t in2;
@@ -834,10 +891,9 @@ __global__ void __launch_bounds__(kResThreads, 1) topk_resolve_kernel(TopkDecode
     pdl_release();
     const int b = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int n = clamp_n(a.n, b, a.Ncap);
     const int k = a.k;
-    if (n <= k) return;  // the filter wrote the whole answer
     const int nfch = a.nfch;
+    // every load goes out before the length is known (none depends on it)
     const uint32_t* tot = a.totals + (size_t)b * kTotals;
     const int d1 = (int)ld_cg_u32(tot + kTotBin);
     const float E = __uint_as_float(ld_cg_u32(tot + kTotE));
@@ -850,23 +906,24 @@ __global__ void __launch_bounds__(kResThreads, 1) topk_resolve_kernel(TopkDecode
         h2[0] = x.x;
         h2[1] = x.y;
     }
-    const uint32_t* gk = a.cand_key + (size_t)b * a.Ncap;
-    const int32_t* gi = a.cand_idx + (size_t)b * a.Ncap;
+    const uint2* cs = a.cslot + (size_t)b * nfch * kSlots;
     uint32_t pk[kGatherJ];
     int32_t pi[kGatherJ];
 #pragma unroll
     for (int j = 0; j < kGatherJ; ++j) {
         const int c = warp + 32 * j;
-        const int r = c * a.fchunk + lane;
-        const bool ok = c < nfch && r < n;
-        pk[j] = ok ? ld_cg_u32(gk + r) : 0u;
-        pi[j] = ok ? (int32_t)ld_cg_u32(gi + r) : 0;
+        const uint2 e = c < nfch ? ld_cg_u32x2(cs + (size_t)c * kSlots + lane) : make_uint2(0u, 0u);
+        pk[j] = e.x;
+        pi[j] = (int32_t)e.y;
     }
+    const int n = clamp_n(a.n, b, a.Ncap);
+    if (n <= k) return;  // the filter wrote the whole answer
     load_q2(S.q2, a.q_idx + (size_t)b * 64);
     if (tid == 0) {
         S.amb_cnt = 0;
         S.f_cnt = 0;
         S.found = 0;
+        S.pf_cnt = 0;
     }
     // the fine bin d2 of t~ inside bin d1 (rank K2 there)
     const uint32_t K2 = (uint32_t)k - above1;
@@ -899,19 +956,23 @@ __global__ void __launch_bounds__(kEmitThreads) topk_emit_kernel(TopkDecodeArgs 
     pdl_wait();
     pdl_release();
     const int b = blockIdx.y, c = blockIdx.x;
+    const int row0 = c * a.fchunk;
+    const uint32_t* bm = a.bitmap + (size_t)b * a.Wcap;
+    // the first words and the position go out before the length is known
+    const int wcap = (min(row0 + a.fchunk, a.Ncap) + 31) >> 5;
+    const int wf = (row0 >> 5) + (int)threadIdx.x;
+    const uint32_t word0 = wf < wcap ? ld_cg_u32(bm + wf) : 0u;
+    uint32_t pos = ld_cg_u32(a.chunk_pos + (size_t)b * a.nfch + c);
     const int n = clamp_n(a.n, b, a.Ncap);
     if (n <= a.k) return;
-    const int row0 = c * a.fchunk;
     const int row1 = min(row0 + a.fchunk, n);
     if (row0 >= row1) return;
-    const uint32_t* bm = a.bitmap + (size_t)b * a.Wcap;
     int32_t* out = a.idx + (size_t)b * a.k;
     const int w0 = row0 >> 5, w1 = (row1 + 31) >> 5;
-    uint32_t pos = __ldcg(a.chunk_pos + (size_t)b * a.nfch + c);
 #pragma unroll 1
     for (int wb = w0; wb < w1; wb += kEmitThreads) {  // block-uniform trip count
         const int w = wb + threadIdx.x;
-        uint32_t word = w < w1 ? __ldcg(bm + w) : 0u;
+        uint32_t word = w < w1 ? (wb == w0 ? word0 : __ldcg(bm + w)) : 0u;
         uint32_t total;
         uint32_t p = pos + block_exclusive_scan(__popc(word), sh32, &total);
         while (word) {
