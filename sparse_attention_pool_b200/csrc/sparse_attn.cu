@@ -16,6 +16,7 @@
 
 #include "../../include/sparse_attn.h"
 #include "attn.cuh"
+#include "attn_prefill_tc.cuh"
 #include "compress.cuh"
 #include "sa_common.cuh"
 #include "topk_decode.cuh"
@@ -282,8 +283,9 @@ struct Split {
 Split attn_split(int rows_cap, bool prefill, bool gather = false) {
     const int tiles = cdiv(rows_cap > 0 ? rows_cap : 1, sa::kTileN);
     if (prefill) return {tiles, 1};
-    (void)gather;  // both lists split the same way: at most 32 splits
-    const int tps = cdiv(tiles, 32);
+    (void)gather;  // both lists split the same way (measured: 32 one-tile splits and a merge kernel beat
+                   // 8 four-tile splits merged in a cluster for a 2048-entry list)
+    const int tps = cdiv(tiles, 32);  // at most 32 splits, merged by the combine kernel
     return {tps, cdiv(tiles, tps)};
 }
 
@@ -317,25 +319,29 @@ sa_status launch_attn_nw(const sa::AttnArgs& a, bool gather, bool fp8, dim3 grid
                : launch_attn_t<NW, false, false, ST, CL, EG>(a, grid, st, pdl);
 }
 
-// Splits of up to 4 tiles keep all of them in flight (4 stages); longer
-// lists (prefill) stream through a 2-stage pipeline.  A query split exactly
-// kAttnCluster ways merges inside a cluster.  Decode with up to 64 heads
-// splits every tile between two warp groups (8 warps), which halves the
-// serial work per warp; prefill keeps one group.
+// Splits of up to 4 tiles keep all of them in flight (4 or 5 stages);
+// longer lists (prefill) stream through a 2-stage pipeline.  A query split
+// exactly kAttnCluster ways merges inside a cluster.  Decode with up to 64
+// heads splits every tile between two warp groups (8 warps), which halves
+// the serial work per warp; prefill and more heads keep one group.
 sa_status launch_attn(const sa::AttnArgs& a, bool gather, bool fp8, long long BQ, cudaStream_t st, bool pdl,
                       bool decode) {
     const bool cl = a.splits == sa::kAttnCluster && BQ <= 65535;
     if (BQ > 2147483647LL || a.splits > 65535) return fail(SA_ERR_INVALID_ARG, "too many queries or splits");
     const dim3 grid = cl ? dim3(a.splits, (unsigned)BQ) : dim3((unsigned)BQ, a.splits);
     const bool deep = a.tiles_per_split >= 2 && a.tiles_per_split <= 4;
-    if (a.H <= 64) {
-        if (decode) {
-            if (cl)
-                return deep ? launch_attn_nw<4, 4, true, 2>(a, gather, fp8, grid, st, pdl)
-                            : launch_attn_nw<4, 2, true, 2>(a, gather, fp8, grid, st, pdl);
-            return deep ? launch_attn_nw<4, 4, false, 2>(a, gather, fp8, grid, st, pdl)
-                        : launch_attn_nw<4, 2, false, 2>(a, gather, fp8, grid, st, pdl);
-        }
+    if (a.H <= 64 && decode) {
+        // splits of 4 tiles keep all four in flight (5 stages)
+        const bool d5 = a.tiles_per_split == 4;
+        if (cl)
+            return d5 ? launch_attn_nw<4, 5, true, 2>(a, gather, fp8, grid, st, pdl)
+                      : deep ? launch_attn_nw<4, 4, true, 2>(a, gather, fp8, grid, st, pdl)
+                             : launch_attn_nw<4, 2, true, 2>(a, gather, fp8, grid, st, pdl);
+        return d5 ? launch_attn_nw<4, 5, false, 2>(a, gather, fp8, grid, st, pdl)
+                  : deep ? launch_attn_nw<4, 4, false, 2>(a, gather, fp8, grid, st, pdl)
+                         : launch_attn_nw<4, 2, false, 2>(a, gather, fp8, grid, st, pdl);
+    }
+    if (a.H <= 64) {  // prefill: long lists, one warp group measured faster
         if (cl)
             return deep ? launch_attn_nw<4, 4, true, 1>(a, gather, fp8, grid, st, pdl)
                         : launch_attn_nw<4, 2, true, 1>(a, gather, fp8, grid, st, pdl);
@@ -347,6 +353,42 @@ sa_status launch_attn(const sa::AttnArgs& a, bool gather, bool fp8, long long BQ
                     : launch_attn_nw<8, 2, true, 1>(a, gather, fp8, grid, st, pdl);
     return deep ? launch_attn_nw<8, 4, false, 1>(a, gather, fp8, grid, st, pdl)
                 : launch_attn_nw<8, 2, false, 1>(a, gather, fp8, grid, st, pdl);
+}
+
+// Causal prefill with 64 heads over a bf16 cache: the tensor-memory kernel
+// (two query positions per CTA, 128-row MMAs).
+sa_status launch_prefill_tc(const sa::AttnArgs& aa, const sa_cache* c, bool gather, cudaStream_t st) {
+    sa::TcArgs a{};
+    a.q = aa.q;
+    a.K = static_cast<const uint16_t*>(c->k);
+    a.V = static_cast<const uint16_t*>(c->v);
+    a.n = c->n;
+    a.pos = aa.pos;
+    a.idx = aa.idx;
+    a.cnt = aa.cnt;
+    a.T = aa.Tq;
+    a.Ncap = c->Ncap;
+    a.kmax = aa.kmax;
+    a.m = c->m;
+    a.scale_log2 = aa.scale_log2;
+    a.out = aa.out;
+    a.lse = aa.lse;
+    static std::atomic<uint64_t> init{0};
+    if (!attr_done(init)) {
+        SA_CUDA(cudaFuncSetAttribute(sa::attn_prefill_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     sa::kTcSmem));
+        SA_CUDA(cudaFuncSetAttribute(sa::attn_prefill_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     sa::kTcSmem));
+        attr_set(init);
+    }
+    const dim3 grid((unsigned)((a.T + 1) / 2), (unsigned)c->B);
+    if (grid.y > 65535) return fail(SA_ERR_INVALID_ARG, "too many sequences");
+    if (gather)
+        sa::attn_prefill_tc_kernel<true><<<grid, sa::kTcThreads, sa::kTcSmem, st>>>(a);
+    else
+        sa::attn_prefill_tc_kernel<false><<<grid, sa::kTcThreads, sa::kTcSmem, st>>>(a);
+    SA_LAUNCHED();
+    return SA_OK;
 }
 
 // The merge follows its split kernel on the same stream: always chained.
@@ -416,6 +458,9 @@ sa_status run_attn(const void* q, int Tq, int H, const sa_cache* c, bool gather,
         a.part_o = reinterpret_cast<float*>(base);
         a.part_lse = reinterpret_cast<float*>(base + up256((size_t)BQ * sp.splits * H * 128 * 4));
     }
+    // dense causal prefill (HCA) on the tensor-memory kernel; the gathered one
+    // (CSA) stays on the mma.sync kernel, which measured faster (see DESIGN)
+    if (prefill && !gather && H == 64 && c->dtype == SA_BF16 && pos) return launch_prefill_tc(a, c, false, st);
     sa_status r = launch_attn(a, gather, c->dtype == SA_FP8_E4M3, BQ, st, chained && pdl_on(), !prefill);
     if (r != SA_OK) return r;
     // a query split kAttnCluster ways was merged inside its cluster
@@ -424,8 +469,8 @@ sa_status run_attn(const void* q, int Tq, int H, const sa_cache* c, bool gather,
     return SA_OK;
 }
 
-// The indexer + top-k of a decode step: the score kernel (the HBM stream) and
-// the cluster selection kernel.  `between` runs after the score kernel is
+// The indexer + top-k of a decode step: the score kernel (the HBM stream),
+// the filter, the resolve and the emit.  `between` runs after the filter is
 // queued (the hybrid step forks its HCA branch there).
 template <typename F>
 sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* idx, int32_t* cnt, void* ws,
@@ -481,14 +526,16 @@ sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* 
         SA_LAUNCHED();
         stage_mark(SA_STAGE_INDEX_SCORE, 1, st);
     }
-    sa_status r = between();
-    if (r != SA_OK) return r;
     stage_mark(SA_STAGE_TOPK_SELECT, 0, st);
     // a sequence with n <= k visible entries (every one, when Ncap is 0) is
     // answered by the filter's first CTA; the other kernels skip it
     const bool pdl = pdl_on();
     SA_CUDA(launch_k(sa::topk_filter_kernel, dim3(a.nfch, B), dim3(sa::kSelThreads), 0, st, pdl && Ncap > 0, 1u, a));
     SA_LAUNCHED();
+    // `between` runs here: the many small filter CTAs have the SMs to
+    // themselves, and what it queues overlaps the latency-bound rest
+    sa_status r = between();
+    if (r != SA_OK) return r;
     SA_CUDA(launch_k(sa::topk_resolve_kernel, dim3(B), dim3(sa::kResThreads), sa::kSelSmem, st, pdl, 1u, a));
     SA_LAUNCHED();
     SA_CUDA(launch_k(sa::topk_emit_kernel, dim3(a.nfch, B), dim3(sa::kEmitThreads), 0, st, pdl, 1u, a));
@@ -823,9 +870,10 @@ sa_status hybrid_attn_decode(const void* q, const void* q_idx, int32_t H, const 
     int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + w.idx);
     int32_t* cnt = cnt_out ? cnt_out : reinterpret_cast<int32_t*>(base + w.cnt);
     const Split sc = attn_split(k, false, true);
-    // HCA needs neither the indexer nor the top-k: once the indexer stream is
-    // queued, fork it onto the side stream so that it overlaps the selection
-    // and the CSA attention instead of competing with the indexer stream.
+    // HCA needs neither the indexer nor the top-k: once the indexer stream and
+    // the filter are queued, fork it onto the side stream so that it overlaps
+    // the latency-bound resolve, emit and CSA attention instead of competing
+    // with the indexer stream or the filter's many CTAs.
     SideStream* side = nullptr;
     r = side_stream(&side);
     if (r != SA_OK) return r;

@@ -53,7 +53,7 @@ constexpr int kBinsLow = 1024;    // last 10-bit digit
 // above bin d1
 constexpr int kTotals = 4;
 constexpr int kTotTicket = 0, kTotBin = 1, kTotE = 2, kTotAbove = 3;
-constexpr int kFiltRows = 1024;  // rows per filter / emit CTA (one pass of 256 threads x 4 keys)
+constexpr int kFiltRows = 2048;  // rows per filter / emit CTA (one pass of 256 threads x 8 keys)
 constexpr int kSlots = 64;       // compact candidate slots per filter chunk
 
 struct TopkDecodeArgs {
@@ -551,11 +551,13 @@ constexpr int kResThreads = 1024;            // resolve CTA (one per sequence)
 constexpr int kSelCap = 8192;                // candidates the resolving CTA holds in shared memory
 constexpr int kSelSmem = kSelCap * 8;
 constexpr int kSelMaxChunks = 1024;          // filter chunks per sequence
-constexpr int kGatherJ = 8;                  // filter chunks per warp loaded ahead by the resolve
+constexpr int kGatherJ = 4;                  // filter chunks per warp loaded ahead by the resolve
+constexpr int kGatherS = 2;                  // ... and compact slots per lane of each
 constexpr int kPf = 64;                      // index rows staged for the band
 static_assert(kSelMaxChunks <= kResThreads, "the resolve gives one thread to every chunk");
 static_assert(kBins == 2 * kResThreads, "the resolve loads the second histogram two bins per thread");
 static_assert(kFiltKPT * kSelThreads == kFiltRows, "one filter pass covers a chunk");
+static_assert(32 * kGatherS <= kSlots, "preloaded slots are compact slots");
 
 struct FilterBounds {
     float in_above;  // s~ > in_above  : surely selected
@@ -686,7 +688,8 @@ __global__ void __launch_bounds__(kSelThreads) topk_filter_kernel(TopkDecodeArgs
 template <bool SMEM>
 __device__ __forceinline__ void resolve_body(const TopkDecodeArgs& a, SelSmem& S, uint32_t* csm, int b, uint32_t C,
                                              uint32_t A, int d1, float E, int d2, uint32_t above2, uint32_t K2,
-                                             const uint32_t (&pk)[kGatherJ], const int32_t (&pi)[kGatherJ],
+                                             const uint32_t (&pk)[kGatherJ * kGatherS],
+                                             const int32_t (&pi)[kGatherJ * kGatherS],
                                              uint32_t cin) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int k = a.k, nfch = a.nfch;
@@ -719,12 +722,16 @@ __device__ __forceinline__ void resolve_body(const TopkDecodeArgs& a, SelSmem& S
 #pragma unroll
     for (int j = 0; j < kGatherJ; ++j) {
         const int c = warp + 32 * j;
-        if (c < nfch && (uint32_t)lane < S.ccnt[c]) put(S.base[c] + lane, pk[j], pi[j]);
+#pragma unroll
+        for (int u = 0; u < kGatherS; ++u) {
+            const uint32_t sl = (uint32_t)(lane + 32 * u);
+            if (c < nfch && sl < S.ccnt[c]) put(S.base[c] + sl, pk[j * kGatherS + u], pi[j * kGatherS + u]);
+        }
     }
 #pragma unroll 1
-    for (int c = warp; c < nfch; c += 32) {  // slots beyond 32, chunks beyond the first kGatherJ per warp
+    for (int c = warp; c < nfch; c += 32) {  // further slots, chunks beyond the first kGatherJ per warp
         const uint32_t cn = S.ccnt[c], cb = S.base[c];
-        const uint32_t from = c < 32 * kGatherJ ? 32u : 0u;
+        const uint32_t from = c < 32 * kGatherJ ? 32u * kGatherS : 0u;
         for (uint32_t i = from + lane; i < cn; i += 32) {
             if (i < (uint32_t)kSlots) {
                 const uint2 e = cs[(size_t)c * kSlots + i];
@@ -734,8 +741,7 @@ __device__ __forceinline__ void resolve_body(const TopkDecodeArgs& a, SelSmem& S
             }
         }
     }
-    cp_async_commit();
-    cp_async_wait<0>();
+    cp_async_commit();  // the staged rows are awaited just before the band
     if (!SMEM) __threadfence_block();
     __syncthreads();
 
@@ -776,7 +782,8 @@ __device__ __forceinline__ void resolve_body(const TopkDecodeArgs& a, SelSmem& S
     // the band list (global, used when the band is large)
     uint32_t* gak = a.amb_key + (size_t)b * a.Ncap;
     int32_t* gai = a.amb_idx + (size_t)b * a.Ncap;
-    __syncthreads();  // S.amb_key held the fine bin
+    cp_async_wait<0>();
+    __syncthreads();  // S.amb_key held the fine bin; the staged rows have landed
     // when the band lies inside the staged window, its members are all staged
     const uint32_t lo_w = pre >= 2u ? (pre - 2u) << 10 : 0u;
     const bool win = fast && S.pf_cnt <= (uint32_t)kPf && blo_key >= lo_w && (bhi_key >> 10) <= pre + 2u;
@@ -907,18 +914,25 @@ __global__ void __launch_bounds__(kResThreads, 1) topk_resolve_kernel(TopkDecode
         h2[1] = x.y;
     }
     const uint2* cs = a.cslot + (size_t)b * nfch * kSlots;
-    uint32_t pk[kGatherJ];
-    int32_t pi[kGatherJ];
+    uint32_t pk[kGatherJ * kGatherS];
+    int32_t pi[kGatherJ * kGatherS];
 #pragma unroll
     for (int j = 0; j < kGatherJ; ++j) {
         const int c = warp + 32 * j;
-        const uint2 e = c < nfch ? ld_cg_u32x2(cs + (size_t)c * kSlots + lane) : make_uint2(0u, 0u);
-        pk[j] = e.x;
-        pi[j] = (int32_t)e.y;
+#pragma unroll
+        for (int u = 0; u < kGatherS; ++u) {
+            const uint2 e = c < nfch ? ld_cg_u32x2(cs + (size_t)c * kSlots + lane + 32 * u) : make_uint2(0u, 0u);
+            pk[j * kGatherS + u] = e.x;
+            pi[j * kGatherS + u] = (int32_t)e.y;
+        }
     }
+    const uint32_t qw = tid < 32 ? ld_cg_u32(reinterpret_cast<const uint32_t*>(a.q_idx + (size_t)b * 64) + tid) : 0u;
     const int n = clamp_n(a.n, b, a.Ncap);
     if (n <= k) return;  // the filter wrote the whole answer
-    load_q2(S.q2, a.q_idx + (size_t)b * 64);
+    if (tid < 32) {  // qI * 2^768 in fp64 for the exact rescoring (see load_q2)
+        S.q2[2 * tid] = (double)bf16lo_f32(qw) * 0x1p768;
+        S.q2[2 * tid + 1] = (double)bf16hi_f32(qw) * 0x1p768;
+    }
     if (tid == 0) {
         S.amb_cnt = 0;
         S.f_cnt = 0;

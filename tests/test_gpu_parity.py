@@ -280,6 +280,39 @@ def test_prefill_vs_oracle_every_row(S, fp8):
     assert worst_c <= tol and worst_h <= tol, (worst_c, worst_h)
 
 
+@pytest.mark.parametrize("T,k", [(1001, 96), (640, 256)])
+def test_prefill_tensor_core_path_vs_oracle_every_row(S, T, k):
+    """64 heads over a bf16 cache: the HCA branch runs on the tcgen05 prefill
+    kernel (two query positions per CTA; an odd T leaves one alone), the CSA
+    branch on the mma.sync kernel (k not a multiple of its 64-entry tile)."""
+    B, H = 2, 64
+    inp = Inputs(611 + T, B, T, H, Tq=T)
+    g = inp.to_device()
+    csa, hca = compress_on_gpu(S, g, B, T)
+    ws = S.alloc_workspace(S.workspace_size(S.SA_OP_HYBRID_PREFILL, B, T, H, csa.Ncap, hca.Ncap, k))
+    idx = torch.empty(B, T, k, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(B, T, dtype=torch.int32, device="cuda")
+    lc = torch.empty(B, T, H, dtype=torch.float32, device="cuda")
+    lh = torch.empty(B, T, H, dtype=torch.float32, device="cuda")
+    oc, oh = S.hybrid_attn_prefill(g["q"], g["qI"], csa, hca, k, ws, idx, cnt, scale=SCALE, lse_csa=lc, lse_hca=lh)
+    S.read_device_status()
+    for b in range(B):
+        cs = inp.oracle_seq(b)
+        ocf, ohf = oc[b].float().cpu().numpy(), oh[b].float().cpu().numpy()
+        lcf, lhf = lc[b].cpu().numpy(), lh[b].cpu().numpy()
+        worst = 0.0
+        for t in range(T):
+            r = O.hybrid_query(cs, inp.q[b, t], inp.qI[b, t], t=t, k=k, scale=SCALE)
+            worst = max(worst, float(np.abs(ocf[t] - r["out_csa"]).max()), float(np.abs(ohf[t] - r["out_hca"]).max()))
+            if r["cnt"] == 0:
+                assert not ocf[t].any() and np.isneginf(lcf[t]).all(), t
+            else:
+                assert np.abs(lcf[t] - r["lse_csa"]).max() < 1e-3, t
+            if t >= 128:
+                assert np.abs(lhf[t] - r["lse_hca"]).max() < 1e-3, t
+        assert worst <= TOL_BF16, (b, worst)
+
+
 def test_prefill_row_equals_decode(S):
     B, T, H, k = 1, 3000, 64, 128
     inp = Inputs(602, B, T, H, Tq=T)
