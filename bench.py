@@ -17,6 +17,7 @@ scaling, no collective on the data path); time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -287,8 +288,14 @@ def run_ours(args, w, rank, world, dev):
     with torch.cuda.graph(graph_staged):
         step()
     torch.cuda.synchronize()
-    for si in range(len(stage_names)):
+    # the roofline kernel alone between two events (the score kernel's stage)
+    for si in range(1, len(stage_names)):
         L.sa_set_stage_events(si, None, None)
+    graph_score = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_score):
+        step()
+    torch.cuda.synchronize()
+    L.sa_set_stage_events(0, None, None)
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         step()
@@ -298,6 +305,8 @@ def run_ours(args, w, rank, world, dev):
         graph.replay()
         flush_l2()
         graph_staged.replay()
+        flush_l2()
+        graph_score.replay()
     torch.cuda.synchronize()
 
     ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -331,8 +340,13 @@ def run_ours(args, w, rank, world, dev):
             staged_ms.append(ev0[i].elapsed_time(ev1[i]))
             for si, (e0, e1) in enumerate(stage_ev):
                 stage_ms[si].append(e0.elapsed_time(e1))
+        score_ms = []
+        for i in range(args.steps):
+            flush_l2()
+            graph_score.replay()
+            stage_ev[0][1].synchronize()
+            score_ms.append(stage_ev[0][0].elapsed_time(stage_ev[0][1]))
         clk.keep_busy(lambda: (flush_l2(), graph.replay()), min_samples=2)
-    score_ms = stage_ms[0]
     torch.cuda.synchronize()
     S.read_device_status()
 
@@ -366,7 +380,7 @@ def run_ours(args, w, rank, world, dev):
         e2e_ms.append(ev0[i].elapsed_time(ev1[i]))
     e2e_total = max_over_ranks(sum(e2e_ms), world, dev)
     S.read_device_status()
-    del graph, graph_staged
+    del graph, graph_staged, graph_score
 
     value = job_throughput(B * args.steps, world, total_ms)
     step_bytes, score_bytes = decode_bytes(w, lengths)
@@ -632,10 +646,16 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=[x.name for x in configs.WORKLOADS])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="prefill only: a shorter sequence than the workload's (small cases for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = configs.BY_NAME[args.workload]
+    if args.tokens:
+        if w.mode != "prefill":
+            ap.error("--tokens applies to prefill workloads")
+        w = dataclasses.replace(w, L=args.tokens)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
