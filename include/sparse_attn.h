@@ -100,7 +100,8 @@ typedef enum {
     SA_OP_SPARSE_ATTN = 2,
     SA_OP_DENSE_ATTN = 3,
     SA_OP_HYBRID_DECODE = 4,
-    SA_OP_HYBRID_PREFILL = 5
+    SA_OP_HYBRID_PREFILL = 5,
+    SA_OP_WINDOW_ATTN = 6   /* k = the window */
 } sa_op;
 
 /* Compression, section 3-2 (2) component table, CSA row ("every 4 tokens ->
@@ -114,6 +115,44 @@ sa_status csa_compress(const sa_raw* raw, const sa_cache* out, void* stream);
 /* Compression, HCA row ("every 128 tokens -> 1 compressed entry"): as
  * csa_compress for k and v only (kidx ignored); out->m is normally 128.      */
 sa_status hca_compress(const sa_raw* raw, const sa_cache* out, void* stream);
+
+/* Compress-when-ready, section 3-2 (4) (the state cache holds the tail until
+ * a block is complete): the raw sequences have grown since the cache was last
+ * brought up to date (cache->n[b] entries).  Computes the entries
+ * cache->n[b] .. floor(len[b] / m) - 1, recomputes the partly filled group of
+ * 64 entries they join (an fp8 group's scale covers every entry present) and
+ * sets cache->n[b] = floor(len[b] / m).  The result is bit-identical to
+ * csa_compress / hca_compress of the new lengths.
+ *   max_new_tokens: an upper bound, per sequence, on the raw tokens added
+ *   since cache->n[b] was set (the launch is sized from it).  A sequence that
+ *   grew by more is completed only as far as the launch reaches (cache->n[b]
+ *   says how far) and flagged in the device status (SA_ERR_DEVICE from
+ *   sa_read_device_status).
+ * Other arguments and requirements as for csa_compress / hca_compress.        */
+sa_status csa_append(const sa_raw* raw, const sa_cache* cache, int32_t max_new_tokens, void* stream);
+sa_status hca_append(const sa_raw* raw, const sa_cache* cache, int32_t max_new_tokens, void* stream);
+
+/* Sliding-window branch, section 3-2 (2) (a small window of the latest
+ * uncompressed tokens beside the compressed branches).  Softmax attention of
+ * the H query heads over the last `window` raw tokens visible to the query:
+ * tokens max(0, T - window) .. T - 1 with T = len[b] (decode, q_pos NULL,
+ * Tq 1) or T = min(len[b], t) for a query at position t (q_pos [B][Tq]).
+ *   q [B][Tq][H][128] bf16; raw->k, raw->v [B][Lcap][128] bf16, raw->len [B].
+ *   out [B][Tq][H][128] bf16; lse [B][Tq][H] fp32 (natural log) or NULL.
+ * ws / ws_bytes: at least sa_workspace_size(SA_OP_WINDOW_ATTN, B, Tq, H, 0, 0,
+ * window).  No visible token: out 0, lse -inf.                               */
+sa_status swa_attn(const void* q, int32_t Tq, int32_t H, const int32_t* q_pos, const sa_raw* raw,
+                   int32_t window, float scale, void* out, float* lse, void* ws, size_t ws_bytes,
+                   void* stream);
+
+/* Merges two attentions over disjoint key sets (for instance a compressed
+ * branch and the window branch) into the attention over their union:
+ * lse = log(e^lse_a + e^lse_b), out = (e^lse_a out_a + e^lse_b out_b) / e^lse.
+ * rows = B * Tq * H; out_* [rows][128] bf16, lse_* [rows] fp32; out may alias
+ * out_a or out_b (each row is read before it is written); lse may be NULL.
+ * A row whose lse_a and lse_b are both -inf gets out 0, lse -inf.            */
+sa_status attn_lse_merge(const void* out_a, const float* lse_a, const void* out_b, const float* lse_b,
+                         int64_t rows, void* out, float* lse, void* stream);
 
 /* CSA indexer + top-k, section 3-2 (2) (CSA "sparse top-k selection") and
  * 3-2 (4) ("CSA indexer QK path").

@@ -219,3 +219,29 @@ def hybrid_query(cs: CompressedSeq, q: np.ndarray, qI: np.ndarray, t: int, k: in
                       cs.n_hca, int(cs.fp8), int(k), float(scale),
                       _p(idx), _p(cnt), _p(oc), _p(lc), _p(oh), _p(lh))
     return {"idx": idx, "cnt": int(cnt[0]), "out_csa": oc, "lse_csa": lc, "out_hca": oh, "lse_hca": lh}
+
+
+def window_rows(t: int, n_raw: int, window: int):
+    """Raw tokens a query at position t sees in the sliding-window branch:
+    the last `window` of the tokens before t (reading in the design notes)."""
+    T = min(int(n_raw), int(t))
+    return np.arange(max(0, T - int(window)), T, dtype=np.int32)
+
+
+def union_attention(q: np.ndarray, parts, scale: float):
+    """Softmax attention over the union of several key sets, each given as
+    (K [N][d] uint16 bf16, V [N][d] uint16 bf16, rows); one softmax over all
+    of them (the sliding-window branch joined with a compressed branch,
+    "DeepSeek-V4 ... Review" section 3-2 (2)).  Returns (out [H][d], lse [H])."""
+    Ks, Vs = [], []
+    for K, V, rows in parts:
+        rows = np.asarray(rows, dtype=np.int64)
+        Ks.append(np.asarray(K, dtype=np.uint16)[rows])
+        Vs.append(np.asarray(V, dtype=np.uint16)[rows])
+    d = np.asarray(q).shape[1]
+    Ku = np.concatenate(Ks, axis=0) if Ks else np.zeros((0, d), np.uint16)
+    Vu = np.concatenate(Vs, axis=0) if Vs else np.zeros((0, d), np.uint16)
+    if Ku.shape[0] == 0:
+        H = np.asarray(q).shape[0]
+        return np.zeros((H, d)), np.full((H,), -np.inf)
+    return attention(q, Ku, Vu, np.arange(Ku.shape[0], dtype=np.int32), scale)

@@ -12,6 +12,7 @@ LIB_PATH = os.path.join(HERE, "libsparse_attn.so")
 SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_CUDA, SA_ERR_TIMEOUT, SA_ERR_DEVICE = range(7)
 SA_BF16, SA_FP8_E4M3 = 0, 1
 SA_OP_INDEX_TOPK, SA_OP_SPARSE_ATTN, SA_OP_DENSE_ATTN, SA_OP_HYBRID_DECODE, SA_OP_HYBRID_PREFILL = 1, 2, 3, 4, 5
+SA_OP_WINDOW_ATTN = 6
 
 STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3: "SA_ERR_WORKSPACE",
                 4: "SA_ERR_CUDA", 5: "SA_ERR_TIMEOUT", 6: "SA_ERR_DEVICE"}
@@ -20,7 +21,7 @@ STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3:
 EXPORTS = ["csa_compress", "hca_compress", "csa_index_topk", "csa_sparse_attn", "hca_dense_attn",
            "hybrid_attn_decode", "hybrid_attn_prefill", "sa_workspace_size", "sa_read_device_status",
            "sa_last_error", "sa_abi_version", "sa_set_stage_events", "sa_launch_count",
-           "csa_index_topk_noalloc"]
+           "csa_index_topk_noalloc", "csa_append", "hca_append", "swa_attn", "attn_lse_merge"]
 SA_NOALLOC_SCRATCH_BYTES = 32 << 20
 SA_STAGE_INDEX_SCORE, SA_STAGE_TOPK_SELECT, SA_STAGE_CSA_ATTN, SA_STAGE_HCA_ATTN = 0, 1, 2, 3
 
@@ -60,6 +61,10 @@ def lib():
         RP, CP = ctypes.POINTER(SaRaw), ctypes.POINTER(SaCache)
         L.csa_compress.argtypes = [RP, CP, P]
         L.hca_compress.argtypes = [RP, CP, P]
+        L.csa_append.argtypes = [RP, CP, I32, P]
+        L.swa_attn.argtypes = [P, I32, I32, P, RP, I32, F32, P, P, P, SZ, P]
+        L.attn_lse_merge.argtypes = [P, P, P, P, ctypes.c_int64, P, P, P]
+        L.hca_append.argtypes = [RP, CP, I32, P]
         L.csa_index_topk.argtypes = [P, I32, P, CP, I32, P, P, P, SZ, P]
         L.csa_index_topk_noalloc.argtypes = [P, CP, I32, P, P, P]
         L.csa_sparse_attn.argtypes = [P, I32, I32, CP, P, P, I32, F32, P, P, P, SZ, P]

@@ -103,6 +103,49 @@ def hca_compress(k, v, lengths, cache: Cache, stream=None):
     check("hca_compress", lib().hca_compress(ctypes.byref(raw), ctypes.byref(cs), _stream(stream)))
 
 
+def csa_append(k, v, kidx, lengths, cache: Cache, max_new_tokens: int, stream=None):
+    """Brings a CSA cache up to date with raw sequences that have grown by at most
+    max_new_tokens tokens each since cache.n was set (bit-identical to a full
+    csa_compress of the new lengths)."""
+    raw = _raw(k, v, kidx, lengths)
+    cs = cache.struct()
+    check("csa_append", lib().csa_append(ctypes.byref(raw), ctypes.byref(cs), int(max_new_tokens), _stream(stream)))
+
+
+def hca_append(k, v, lengths, cache: Cache, max_new_tokens: int, stream=None):
+    """As csa_append, for an HCA cache (k and v only)."""
+    raw = _raw(k, v, None, lengths)
+    cs = cache.struct()
+    check("hca_append", lib().hca_append(ctypes.byref(raw), ctypes.byref(cs), int(max_new_tokens), _stream(stream)))
+
+
+def swa_attn(q, k_raw, v_raw, lengths, window: int, ws, *, q_pos=None, scale=0.0, out=None, lse=None, stream=None):
+    """Sliding-window branch: attention over the last `window` raw tokens visible
+    to each query (q [B][H][128] for decode, or [B][Tq][H][128] with q_pos)."""
+    _need(q, torch.bfloat16, "q")
+    Tq, H = (q.shape[1] if q.dim() == 4 else 1), q.shape[-2]
+    if out is None:
+        out = torch.empty_like(q)
+    raw = _raw(k_raw, v_raw, None, lengths)
+    check("swa_attn", lib().swa_attn(_ptr(q), Tq, H, _ptr(q_pos), ctypes.byref(raw), int(window), float(scale),
+                                     _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def attn_lse_merge(out_a, lse_a, out_b, lse_b, *, out=None, lse=None, stream=None):
+    """Attention over the union of two disjoint key sets from the two partial
+    attentions (outputs [..., 128] bf16 and their natural-log lse [...])."""
+    _need(out_a, torch.bfloat16, "out_a")
+    _need(out_b, torch.bfloat16, "out_b")
+    _need(lse_a, torch.float32, "lse_a")
+    _need(lse_b, torch.float32, "lse_b")
+    if out is None:
+        out = torch.empty_like(out_a)
+    check("attn_lse_merge", lib().attn_lse_merge(_ptr(out_a), _ptr(lse_a), _ptr(out_b), _ptr(lse_b),
+                                                 lse_a.numel(), _ptr(out), _ptr(lse), _stream(stream)))
+    return out
+
+
 def workspace_size(op: int, B: int, Tq: int, H: int, Ncap_csa: int, Ncap_hca: int, k: int) -> int:
     return int(lib().sa_workspace_size(op, B, Tq, H, Ncap_csa, Ncap_hca, k))
 

@@ -35,6 +35,7 @@ struct AttnArgs {
     const int32_t* cnt;  // gather: [BQ]
     const int32_t* pos;  // dense: [BQ] token positions, or NULL (all n[b] visible)
     int Tq, H, Ncap, nG, kmax, m;
+    int win;             // dense: keep only the last `win` visible rows (0: all)
     float scale_log2;    // softmax scale * log2(e)
     int tiles_per_split, splits;
     float* part_o;       // [BQ][splits][H][128]
@@ -133,6 +134,12 @@ __global__ void __launch_bounds__(NW * EG * 32) attn_split_kernel(AttnArgs a) {
             }
         }
     }
+    // a sliding window keeps the last `win` visible rows: rbase .. rbase + R
+    int rbase = 0;
+    if (!GATHER && a.win > 0 && R > a.win) {
+        rbase = R - a.win;
+        R = a.win;
+    }
     const int p_end = min(R, p_begin + a.tiles_per_split * kTileN);
     const int ntiles = p_end > p_begin ? (p_end - p_begin + kTileN - 1) / kTileN : 0;
 
@@ -166,7 +173,7 @@ __global__ void __launch_bounds__(NW * EG * 32) attn_split_kernel(AttnArgs a) {
         uint8_t* rv = sRaw + (stage * 2 + 1) * L::kStageRaw;
         const int r = tid / TPR, c0 = (tid % TPR) * CPT;
         const int p = p0 + r;
-        int j = p;
+        int j = rbase + p;
         bool ok = p < p_end;
         if (GATHER && ok) {
             j = have_j ? jv : a.idx[(size_t)bq * a.kmax + p];
@@ -564,6 +571,30 @@ __global__ void __launch_bounds__(kCombThreads) attn_combine_kernel(const float*
         *reinterpret_cast<uint2*>(op) = make_uint2(pack_bf16x2(t.x * inv, t.y * inv), pack_bf16x2(t.z * inv, t.w * inv));
         if (lse && lane == 0) lse[(size_t)bq * H + h] = ws > 0.f ? Mt + __logf(ws) : -INFINITY;
     }
+}
+
+// Log-sum-exp merge of two attentions over disjoint key sets into the
+// attention over their union: one warp per (query, head) row, 4 dims a lane.
+__global__ void __launch_bounds__(256) attn_lse_merge_kernel(const uint16_t* oa, const float* la, const uint16_t* ob,
+                                                             const float* lb, uint16_t* out, float* lse, long long rows) {
+    pdl_wait();
+    pdl_release();
+    const long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (r >= rows) return;
+    const float x = la[r], y = lb[r];
+    const float M = fmaxf(x, y);
+    const float wa = x == -INFINITY ? 0.f : __expf(x - M), wb = y == -INFINITY ? 0.f : __expf(y - M);
+    const float ws = wa + wb;
+    const float inv = ws > 0.f ? 1.f / ws : 0.f;
+    const uint2 va = *reinterpret_cast<const uint2*>(oa + r * 128 + lane * 4);
+    const uint2 vb = *reinterpret_cast<const uint2*>(ob + r * 128 + lane * 4);
+    const float a0 = bf16lo_f32(va.x), a1 = bf16hi_f32(va.x), a2 = bf16lo_f32(va.y), a3 = bf16hi_f32(va.y);
+    const float b0 = bf16lo_f32(vb.x), b1 = bf16hi_f32(vb.x), b2 = bf16lo_f32(vb.y), b3 = bf16hi_f32(vb.y);
+    *reinterpret_cast<uint2*>(out + r * 128 + lane * 4) =
+        make_uint2(pack_bf16x2((wa * a0 + wb * b0) * inv, (wa * a1 + wb * b1) * inv),
+                   pack_bf16x2((wa * a2 + wb * b2) * inv, (wa * a3 + wb * b3) * inv));
+    if (lse && lane == 0) lse[r] = ws > 0.f ? M + __logf(ws) : -INFINITY;
 }
 
 }  // namespace sa

@@ -7,6 +7,10 @@
 // caches ("Mixed KV storage" row) then get one fp32 scale per 64 consecutive
 // entries, scale = fp32(amax / 448), and codes e4m3_rne_satfinite(x / scale).
 //
+// Append (compress-when-ready): once more raw tokens are present, only the
+// group holding the first new entry and the groups after it are computed;
+// the result is bit-identical to compressing the whole sequence again.
+//
 // One CTA compresses one group of 64 entries of one sequence for every tensor
 // (k, v and optionally the indexer keys).  Each thread owns one 16-byte chunk
 // (8 dims) of one entry and streams the m tokens of its block; the sums run in
@@ -24,7 +28,8 @@ struct CompressArgs {
     int dims[3];             // D of each tensor
     int ntensors;            // 2 (HCA) or 3 (CSA)
     const int32_t* len;      // [B]
-    int32_t* n_out;          // [B]
+    int32_t* n_out;          // [B] (full compression only)
+    const int32_t* n_from;   // [B] entries already in the cache (append), or NULL
     int Lcap, Ncap, nG, m, log2m, fp8;
 };
 
@@ -45,14 +50,25 @@ __global__ void __launch_bounds__(kCompThreads) compress_kernel(CompressArgs a) 
     __shared__ __align__(16) uint16_t stage[64 * 128];  // bf16 entries of one fp8 group
     __shared__ float red[kCompThreads / 32];
 
-    const int g = blockIdx.x, b = blockIdx.y;
+    const int b = blockIdx.y;
     int len = a.len[b];
     if (len < 0 || len > a.Lcap) {
-        if (g == 0 && threadIdx.x == 0) flag(DEV_LEN);
+        if (blockIdx.x == 0 && threadIdx.x == 0) flag(DEV_LEN);
         len = len < 0 ? 0 : a.Lcap;
     }
     const int n = len >> a.log2m;
-    if (g == 0 && threadIdx.x == 0) a.n_out[b] = n;
+    int g = blockIdx.x;
+    if (a.n_from) {
+        // append: start at the group holding the first new entry; that group is
+        // recomputed whole (an fp8 group's scale covers all its present entries;
+        // bf16 entries recompute to the same bits)
+        int n0 = a.n_from[b];
+        n0 = n0 < 0 ? 0 : min(n0, n);
+        g += n0 >> 6;
+        if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0 && (g + 1) * 64 < n) flag(DEV_LEN);  // bound exceeded
+    } else if (g == 0 && threadIdx.x == 0) {
+        a.n_out[b] = n;
+    }
     const int e0 = g * 64;
     if (e0 >= n) return;
     const int ne = min(64, n - e0);
@@ -128,6 +144,19 @@ __global__ void __launch_bounds__(kCompThreads) compress_kernel(CompressArgs a) 
             __syncthreads();  // `stage` and `red` are reused by the next tensor
         }
     }
+}
+
+// After an append: the entry counts follow the raw lengths, up to the groups
+// the append computed (`groups` from the one holding the old count).
+__global__ void set_counts_kernel(const int32_t* len, int32_t* n, int B, int Lcap, int log2m, int groups) {
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= B) return;
+    int l = len[b];
+    l = l < 0 ? 0 : min(l, Lcap);
+    const int full = l >> log2m;
+    int n0 = n[b];
+    n0 = n0 < 0 ? 0 : min(n0, full);
+    n[b] = min(full, ((n0 >> 6) + groups) * 64);
 }
 
 }  // namespace sa

@@ -427,10 +427,10 @@ sa_status side_stream(SideStream** out) {
 // Shared body of csa_sparse_attn / hca_dense_attn / the hybrid calls.
 sa_status run_attn(const void* q, int Tq, int H, const sa_cache* c, bool gather, const int32_t* idx,
                    const int32_t* cnt, int kmax, const int32_t* pos, float scale, void* out, float* lse, void* ws,
-                   size_t ws_off, cudaStream_t st, bool chained = false) {
+                   size_t ws_off, cudaStream_t st, bool chained = false, int win = 0) {
     const long long BQ = (long long)c->B * Tq;
     const bool prefill = (Tq > 1) || (pos != nullptr);
-    const Split sp = attn_split(gather ? kmax : c->Ncap, prefill, gather);
+    const Split sp = attn_split(gather ? kmax : (win > 0 ? std::min(win, c->Ncap) : c->Ncap), prefill, gather);
     sa::AttnArgs a{};
     a.q = static_cast<const uint16_t*>(q);
     a.K = c->k;
@@ -447,6 +447,7 @@ sa_status run_attn(const void* q, int Tq, int H, const sa_cache* c, bool gather,
     a.nG = (c->Ncap + 63) / 64;
     a.kmax = kmax;
     a.m = c->m;
+    a.win = win;
     const float s = scale == 0.f ? 1.0f / sqrtf(128.0f) : scale;
     a.scale_log2 = s * 1.4426950408889634f;
     a.tiles_per_split = sp.tps;
@@ -460,7 +461,7 @@ sa_status run_attn(const void* q, int Tq, int H, const sa_cache* c, bool gather,
     }
     // dense causal prefill (HCA) on the tensor-memory kernel; the gathered one
     // (CSA) stays on the mma.sync kernel, which measured faster (see DESIGN)
-    if (prefill && !gather && H == 64 && c->dtype == SA_BF16 && pos) return launch_prefill_tc(a, c, false, st);
+    if (prefill && !gather && win == 0 && H == 64 && c->dtype == SA_BF16 && pos) return launch_prefill_tc(a, c, false, st);
     sa_status r = launch_attn(a, gather, c->dtype == SA_FP8_E4M3, BQ, st, chained && pdl_on(), !prefill);
     if (r != SA_OK) return r;
     // a query split kAttnCluster ways was merged inside its cluster
@@ -660,8 +661,12 @@ sa_status sa_set_stage_events(int32_t stage, void* before, void* after) {
 
 const char* sa_last_error(void) { return g_err; }
 
-static sa_status compress_common(const sa_raw* raw, const sa_cache* out, void* stream, bool csa) {
-    const char* what = csa ? "csa_compress" : "hca_compress";
+static sa_status check_common_q(const void* q, int H, const char* what);
+
+static sa_status compress_common(const sa_raw* raw, const sa_cache* out, void* stream, bool csa,
+                                 int32_t max_new_tokens = -1) {
+    const bool append = max_new_tokens >= 0;
+    const char* what = append ? (csa ? "csa_append" : "hca_append") : (csa ? "csa_compress" : "hca_compress");
     SA_CHECK(raw != nullptr, "%s: raw descriptor is NULL", what);
     sa_status r = check_cache(out, csa, what);
     if (r != SA_OK) return r;
@@ -698,8 +703,22 @@ static sa_status compress_common(const sa_raw* raw, const sa_cache* out, void* s
     a.m = out->m;
     a.log2m = ilog2(out->m);
     a.fp8 = out->dtype == SA_FP8_E4M3;
-    const int groups = std::max(1, cdiv(raw->Lcap / out->m, 64));
-    sa::compress_kernel<<<dim3(groups, raw->B), sa::kCompThreads, 0, static_cast<cudaStream_t>(stream)>>>(a);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (!append) {
+        const int groups = std::max(1, cdiv(raw->Lcap / out->m, 64));
+        sa::compress_kernel<<<dim3(groups, raw->B), sa::kCompThreads, 0, st>>>(a);
+        SA_LAUNCHED();
+        return SA_OK;
+    }
+    // new entries: at most (max_new_tokens + m - 1) / m (a partial block may
+    // complete); groups: those, plus the partly filled group they join
+    a.n_from = out->n;
+    const long long new_entries = ((long long)max_new_tokens + out->m - 1) / out->m;
+    const long long groups = std::min<long long>((new_entries + 63) / 64 + 1, cdiv(out->Ncap, 64) + 1LL);
+    sa::compress_kernel<<<dim3((unsigned)groups, raw->B), sa::kCompThreads, 0, st>>>(a);
+    SA_LAUNCHED();
+    sa::set_counts_kernel<<<cdiv(raw->B, 128), 128, 0, st>>>(raw->len, out->n, raw->B, raw->Lcap, a.log2m,
+                                                               (int)groups);
     SA_LAUNCHED();
     return SA_OK;
 }
@@ -710,6 +729,66 @@ sa_status csa_compress(const sa_raw* raw, const sa_cache* out, void* stream) {
 
 sa_status hca_compress(const sa_raw* raw, const sa_cache* out, void* stream) {
     return compress_common(raw, out, stream, false);
+}
+
+sa_status csa_append(const sa_raw* raw, const sa_cache* cache, int32_t max_new_tokens, void* stream) {
+    SA_CHECK(max_new_tokens >= 0, "csa_append: max_new_tokens=%d", max_new_tokens);
+    return compress_common(raw, cache, stream, true, max_new_tokens);
+}
+
+sa_status hca_append(const sa_raw* raw, const sa_cache* cache, int32_t max_new_tokens, void* stream) {
+    SA_CHECK(max_new_tokens >= 0, "hca_append: max_new_tokens=%d", max_new_tokens);
+    return compress_common(raw, cache, stream, false, max_new_tokens);
+}
+
+sa_status swa_attn(const void* q, int32_t Tq, int32_t H, const int32_t* q_pos, const sa_raw* raw, int32_t window,
+                   float scale, void* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+    SA_CHECK(raw != nullptr, "swa_attn: raw descriptor is NULL");
+    sa_status r = check_common_q(q, H, "swa_attn");
+    if (r != SA_OK) return r;
+    SA_CHECK(raw->B >= 1 && raw->Lcap >= 0 && raw->d == 128, "swa_attn: raw B=%d Lcap=%d d=%d", raw->B, raw->Lcap,
+             raw->d);
+    SA_CHECK(raw->k && raw->v && raw->len && aligned16(raw->k) && aligned16(raw->v) && aligned16(raw->len),
+             "swa_attn: raw k, v, len must be non-NULL and 16-byte aligned");
+    SA_CHECK(window >= 1, "swa_attn: window=%d", window);
+    SA_CHECK(Tq >= 1, "swa_attn: Tq=%d", Tq);
+    SA_CHECK(q_pos != nullptr || Tq == 1, "swa_attn: decode (q_pos == NULL) needs Tq == 1");
+    SA_CHECK(!q_pos || aligned16(q_pos), "swa_attn: q_pos must be 16-byte aligned");
+    SA_CHECK(out && aligned16(out), "swa_attn: out must be non-NULL and 16-byte aligned");
+    SA_CHECK(!lse || aligned16(lse), "swa_attn: lse must be 16-byte aligned");
+    SA_CHECK(std::isfinite(scale) && scale >= 0.f, "swa_attn: scale must be finite and >= 0");
+    r = check_ws(ws, ws_bytes, sa_workspace_size(SA_OP_WINDOW_ATTN, raw->B, Tq, H, 0, 0, window));
+    if (r != SA_OK) return r;
+    // the raw tokens as a cache of single-token entries (m = 1): entry t is token t
+    sa_cache view{};
+    view.k = const_cast<void*>(raw->k);
+    view.v = const_cast<void*>(raw->v);
+    view.n = const_cast<int32_t*>(raw->len);
+    view.B = raw->B;
+    view.Ncap = raw->Lcap;
+    view.d = 128;
+    view.d_idx = 64;
+    view.m = 1;
+    view.dtype = SA_BF16;
+    return run_attn(q, Tq, H, &view, false, nullptr, nullptr, 0, q_pos, scale, out, lse, ws, 256,
+                    static_cast<cudaStream_t>(stream), false, window);
+}
+
+sa_status attn_lse_merge(const void* out_a, const float* lse_a, const void* out_b, const float* lse_b, int64_t rows,
+                         void* out, float* lse, void* stream) {
+    SA_CHECK(rows >= 0, "attn_lse_merge: rows=%lld", (long long)rows);
+    SA_CHECK(out_a && out_b && lse_a && lse_b && out, "attn_lse_merge: inputs and out must be non-NULL");
+    SA_CHECK(aligned16(out_a) && aligned16(out_b) && aligned16(out) && aligned16(lse_a) && aligned16(lse_b) &&
+                 (!lse || aligned16(lse)),
+             "attn_lse_merge: pointers must be 16-byte aligned");
+    if (rows == 0) return SA_OK;
+    const long long blocks = (rows + 7) / 8;
+    SA_CHECK(blocks <= 2147483647LL, "attn_lse_merge: too many rows");
+    sa::attn_lse_merge_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint16_t*>(out_a), lse_a, static_cast<const uint16_t*>(out_b), lse_b,
+        static_cast<uint16_t*>(out), lse, rows);
+    SA_LAUNCHED();
+    return SA_OK;
 }
 
 size_t sa_workspace_size(int32_t op, int32_t B, int32_t Tq, int32_t H, int32_t Ncap_csa, int32_t Ncap_hca,
@@ -740,6 +819,11 @@ size_t sa_workspace_size(int32_t op, int32_t B, int32_t Tq, int32_t H, int32_t N
         case SA_OP_HYBRID_PREFILL:
             if (k < 1) return 0;
             return prefill_topk_bytes(B, Tq, Ncap_csa, k);
+        case SA_OP_WINDOW_ATTN: {  // k = the window
+            if (k < 1) return 0;
+            Split s = attn_split(k, prefill);
+            return 256 + attn_partial_bytes(BQ, s.splits, H);
+        }
         default:
             return 0;
     }

@@ -86,6 +86,40 @@ def test_compress_rejects_bad_arguments(L, raw_kw, cache_kw, frag):
     assert frag in L.sa_last_error().decode()
 
 
+@pytest.mark.parametrize("raw_kw,cache_kw,frag", [
+    ({}, {"m": 3}, "power of two"),
+    ({"Lcap": 8192}, {}, "Ncap"),
+    ({"kidx": None}, {}, "kidx"),
+])
+def test_append_rejects_bad_arguments(L, raw_kw, cache_kw, frag):
+    r, c = _raw(**raw_kw), _cache(**cache_kw)
+    assert L.csa_append(ctypes.byref(r), ctypes.byref(c), 1, None) == _lib.SA_ERR_INVALID_ARG
+    assert frag in L.sa_last_error().decode()
+    r, c = _raw(), _cache()
+    assert L.csa_append(ctypes.byref(r), ctypes.byref(c), -1, None) == _lib.SA_ERR_INVALID_ARG
+    assert "max_new_tokens" in L.sa_last_error().decode()
+    h = _cache(m=128, kidx=None)
+    assert L.hca_append(ctypes.byref(r), ctypes.byref(h), -5, None) == _lib.SA_ERR_INVALID_ARG
+    assert "hca_append" in L.sa_last_error().decode()
+
+
+def test_window_and_merge_reject_bad_arguments(L):
+    P = ctypes.c_void_p
+    r = _raw()
+    assert L.swa_attn(P(FAKE), 1, 8, None, ctypes.byref(r), 0, 0.0, P(FAKE), None, P(FAKE), 1 << 30, None) == 1
+    assert "window" in L.sa_last_error().decode()
+    assert L.swa_attn(P(FAKE), 4, 8, None, ctypes.byref(r), 64, 0.0, P(FAKE), None, P(FAKE), 1 << 30, None) == 1
+    assert "q_pos" in L.sa_last_error().decode()
+    assert L.swa_attn(P(FAKE), 1, 8, None, None, 64, 0.0, P(FAKE), None, P(FAKE), 1 << 30, None) == 1
+    assert L.swa_attn(P(FAKE), 1, 8, None, ctypes.byref(r), 64, 0.0, P(FAKE), None, P(FAKE), 16, None) == 3
+    assert L.attn_lse_merge(P(FAKE), P(FAKE), P(FAKE), P(FAKE), -1, P(FAKE), None, None) == 1
+    assert L.attn_lse_merge(P(FAKE), P(FAKE), P(FAKE + 4), P(FAKE), 8, P(FAKE), None, None) == 1
+    assert "aligned" in L.sa_last_error().decode()
+    assert L.attn_lse_merge(P(FAKE), P(FAKE), P(FAKE), P(FAKE), 0, P(FAKE), None, None) == 0  # nothing to do
+    assert L.sa_workspace_size(6, 2, 1, 64, 0, 0, 128) > 256
+    assert L.sa_workspace_size(6, 2, 1, 64, 0, 0, 0) == 0
+
+
 def test_null_descriptors(L):
     assert L.csa_compress(None, None, None) == _lib.SA_ERR_INVALID_ARG
     c = _cache()

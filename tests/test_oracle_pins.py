@@ -53,7 +53,7 @@ def test_bf16_decode_exhaustive_vs_numpy_view():
     codes = np.arange(65536, dtype=np.uint32).astype(np.uint16)
     with np.errstate(invalid="ignore"):
         ref = synth.bf16_bits_to_f32(codes).astype(np.float64)
-    got = O.bf16_array_to_f64(codes)
+    got = synth.bf16_bits_to_f32(codes).astype(np.float64)
     nan = np.isnan(ref)
     assert np.array_equal(np.isnan(got), nan)
     assert np.array_equal(got[~nan], ref[~nan])
@@ -430,3 +430,44 @@ def test_prefill_row_equals_decode_at_that_length():
         assert causal["cnt"] == min(k, t // 4)
         if t < 4:
             assert not causal["out_csa"].any() and np.isneginf(causal["lse_csa"]).all()
+
+
+# ------------------------------------------------- sliding-window branch ----
+
+def test_window_rows_are_the_last_tokens_before_the_query():
+    assert O.window_rows(10, 100, 4).tolist() == [6, 7, 8, 9]
+    assert O.window_rows(3, 100, 8).tolist() == [0, 1, 2]
+    assert O.window_rows(50, 20, 8).tolist() == list(range(12, 20))   # only tokens that exist
+    assert O.window_rows(0, 100, 8).tolist() == []
+
+
+def test_union_attention_is_one_softmax_and_the_lse_merge_of_its_parts():
+    H, d = 4, 128
+    q = synth.normal_bf16(31, "q", (1, H * d)).reshape(H, d)
+    Ka, Va = synth.normal_bf16(31, "k", (1, 40 * d)).reshape(40, d), synth.normal_bf16(31, "v", (1, 40 * d)).reshape(40, d)
+    Kb, Vb = synth.normal_bf16(32, "k", (1, 25 * d)).reshape(25, d), synth.normal_bf16(32, "v", (1, 25 * d)).reshape(25, d)
+    ra, rb = [3, 17, 5, 39], list(range(10, 25))
+    scale = 1 / np.sqrt(128.0)
+    out, lse = O.union_attention(q, [(Ka, Va, ra), (Kb, Vb, rb)], scale)
+    # one softmax over the stacked keys, in numpy fp64
+    qf = synth.bf16_bits_to_f32(q).astype(np.float64)
+    Kf = np.concatenate([synth.bf16_bits_to_f32(Ka).astype(np.float64)[ra], synth.bf16_bits_to_f32(Kb).astype(np.float64)[rb]])
+    Vf = np.concatenate([synth.bf16_bits_to_f32(Va).astype(np.float64)[ra], synth.bf16_bits_to_f32(Vb).astype(np.float64)[rb]])
+    z = qf @ Kf.T * scale
+    ref_lse = np.log(np.exp(z - z.max(1, keepdims=True)).sum(1)) + z.max(1)
+    p = np.exp(z - ref_lse[:, None])
+    np.testing.assert_allclose(out, p @ Vf, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=1e-12)
+    # the exact merge of the two separate attentions gives the same
+    oa, la = O.attention(q, Ka, Va, ra, scale)
+    ob, lb = O.attention(q, Kb, Vb, rb, scale)
+    m = np.logaddexp(la, lb)
+    merged = oa * np.exp(la - m)[:, None] + ob * np.exp(lb - m)[:, None]
+    np.testing.assert_allclose(out, merged, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, m, rtol=0, atol=1e-12)
+
+
+def test_union_attention_of_nothing_is_empty():
+    q = np.full((2, 128), 0x3F80, dtype=np.uint16)  # bf16 1.0
+    out, lse = O.union_attention(q, [(np.zeros((4, 128), np.uint16), np.zeros((4, 128), np.uint16), [])], 0.1)
+    assert not out.any() and np.isneginf(lse).all()
