@@ -159,11 +159,6 @@ __device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, boo
                  "r"(valid ? 16 : 0)
                  : "memory");
 }
-__device__ __forceinline__ void cp_async8_zfill(void* dst, const void* src, bool valid) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_u32(dst)), "l"(src),
-                 "r"(valid ? 8 : 0)
-                 : "memory");
-}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
@@ -179,9 +174,6 @@ __device__ __forceinline__ uint32_t atom_add_shared(uint32_t* p, uint32_t v) {
 }
 __device__ __forceinline__ void red_add_shared(uint32_t* p, uint32_t v) {
     asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
-}
-__device__ __forceinline__ void red_or_shared(uint32_t* p, uint32_t v) {
-    asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
 }
 
 // L2 loads kept where they are written: issued early, consumed later (the
@@ -201,7 +193,6 @@ __device__ __forceinline__ uint4 ld_cg_u32x4(const void* p) {
     asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
     return v;
 }
-__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 
 // Programmatic dependent launch.  A kernel launched with programmatic stream
 // serialization may start while its predecessor on the stream is still

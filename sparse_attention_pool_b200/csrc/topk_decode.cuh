@@ -120,15 +120,6 @@ __device__ __noinline__ uint32_t exact_key(const double* q2, const uint16_t* row
     return score_key(__double2float_rn(acc * 0x1p128));
 }
 
-// qI * 2^768 in fp64 into shared memory (64 values), for exact_key.
-__device__ __forceinline__ void load_q2(double* q2, const uint16_t* qI) {
-    if (threadIdx.x < 32) {
-        const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(qI) + threadIdx.x);
-        q2[2 * threadIdx.x] = (double)bf16lo_f32(w) * 0x1p768;
-        q2[2 * threadIdx.x + 1] = (double)bf16hi_f32(w) * 0x1p768;
-    }
-}
-
 // --------------------------------------------------- digit search helpers --
 // Descending: the digit d with  above(d) < K <= above(d) + h[d], where
 // above(d) = sum of h[e] for e > d.  Every thread gets (d, above(d)).
@@ -929,7 +920,7 @@ __global__ void __launch_bounds__(kResThreads, 1) topk_resolve_kernel(TopkDecode
     const uint32_t qw = tid < 32 ? ld_cg_u32(reinterpret_cast<const uint32_t*>(a.q_idx + (size_t)b * 64) + tid) : 0u;
     const int n = clamp_n(a.n, b, a.Ncap);
     if (n <= k) return;  // the filter wrote the whole answer
-    if (tid < 32) {  // qI * 2^768 in fp64 for the exact rescoring (see load_q2)
+    if (tid < 32) {  // qI * 2^768 in fp64 for the exact rescoring (see exact_key)
         S.q2[2 * tid] = (double)bf16lo_f32(qw) * 0x1p768;
         S.q2[2 * tid + 1] = (double)bf16hi_f32(qw) * 0x1p768;
     }
