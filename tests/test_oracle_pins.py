@@ -53,7 +53,7 @@ def test_bf16_decode_exhaustive_vs_numpy_view():
     codes = np.arange(65536, dtype=np.uint32).astype(np.uint16)
     with np.errstate(invalid="ignore"):
         ref = synth.bf16_bits_to_f32(codes).astype(np.float64)
-    got = synth.bf16_bits_to_f32(codes).astype(np.float64)
+    got = O.bf16_array_to_f64(codes)
     nan = np.isnan(ref)
     assert np.array_equal(np.isnan(got), nan)
     assert np.array_equal(got[~nan], ref[~nan])
