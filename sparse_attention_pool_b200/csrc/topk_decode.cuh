@@ -545,7 +545,7 @@ constexpr int kSelMaxChunks = 1024;          // filter chunks per sequence
 constexpr int kGatherJ = 4;                  // filter chunks per warp loaded ahead by the resolve
 constexpr int kGatherS = 2;                  // ... and compact slots per lane of each
 constexpr int kPf = 64;                      // index rows staged for the band
-static_assert(kSelMaxChunks <= kResThreads, "the resolve gives one thread to every chunk");
+static_assert(kSelMaxChunks == kResThreads, "the resolve gives one thread to every chunk");
 static_assert(kBins == 2 * kResThreads, "the resolve loads the second histogram two bins per thread");
 static_assert(kFiltKPT * kSelThreads == kFiltRows, "one filter pass covers a chunk");
 static_assert(32 * kGatherS <= kSlots, "preloaded slots are compact slots");
@@ -567,9 +567,10 @@ __device__ __forceinline__ FilterBounds filter_bounds(int d1, float E) {
 
 struct SelSmem {
     double q2[64];                  // qI * 2^768 for the exact rescoring
-    uint32_t hist[kBins];           // digit histograms of the fallback; then the per-chunk winner counts
+    uint32_t hist[kBins];           // digit histograms of the fallback searches
     uint32_t base[kSelMaxChunks];   // compact position of each filter chunk's candidates
     uint32_t ccnt[kSelMaxChunks];   // candidates per filter chunk
+    uint32_t wcnt[kSelMaxChunks];   // winners among each chunk's candidates
     uint32_t sh64[64];
     int res[2];
     uint32_t f_cnt, found, tkey, amb_cnt, T2, pf_cnt;
@@ -779,9 +780,20 @@ __device__ __forceinline__ void resolve_body(const TopkDecodeArgs& a, SelSmem& S
     const uint32_t lo_w = pre >= 2u ? (pre - 2u) << 10 : 0u;
     const bool win = fast && S.pf_cnt <= (uint32_t)kPf && blo_key >= lo_w && (bhi_key >> 10) <= pre + 2u;
     uint32_t my_in2 = 0;
+    // candidates above the band are winners whatever the cut: marked here
+    uint32_t* bm = a.bitmap + (size_t)b * a.Wcap;
+    auto mark = [&](int32_t j) {
+        atomicOr(&bm[j >> 5], 1u << (j & 31));
+        red_add_shared(&S.wcnt[j / a.fchunk], 1u);
+    };
     if (win) {
 #pragma unroll 1
-        for (uint32_t i = tid; i < C; i += kResThreads) my_in2 += lk[i] > bhi_key;
+        for (uint32_t i = tid; i < C; i += kResThreads) {
+            if (lk[i] > bhi_key) {
+                ++my_in2;
+                mark(li[i]);
+            }
+        }
         if ((uint32_t)tid < S.pf_cnt) {
             const uint32_t kk = S.pf_key[tid];
             if (kk >= blo_key && kk <= bhi_key) {
@@ -796,6 +808,7 @@ __device__ __forceinline__ void resolve_body(const TopkDecodeArgs& a, SelSmem& S
             const uint32_t kk = lk[i];
             if (kk > bhi_key) {
                 ++my_in2;
+                mark(li[i]);
             } else if (kk >= blo_key) {
                 const int32_t j = li[i];
                 const uint32_t p = atom_add_shared(&S.amb_cnt, 1u);
@@ -843,31 +856,16 @@ __device__ __forceinline__ void resolve_body(const TopkDecodeArgs& a, SelSmem& S
     }
     const uint32_t T2 = S.T2;
     const int32_t jmax2 = S.jmax2;
-    // winners of the candidates: into the bitmap, and counted per chunk (S.hist)
-    uint32_t* bm = a.bitmap + (size_t)b * a.Wcap;
-    uint32_t* wc = S.hist;
-    for (int i = tid; i < kBins; i += kResThreads) wc[i] = 0;
-    __syncthreads();
-#pragma unroll 1
-    for (uint32_t i = tid; i < C; i += kResThreads) {
-        if (lk[i] > bhi_key) {
-            const int32_t j = li[i];
-            atomicOr(&bm[j >> 5], 1u << (j & 31));
-            red_add_shared(&wc[j / a.fchunk], 1u);
-        }
-    }
+    // the band's winners
 #pragma unroll 1
     for (uint32_t i = tid; i < na; i += kResThreads) {
         const uint32_t kk = na <= (uint32_t)kResThreads ? S.amb_key[i] : __ldcg(gak + i);
         const int32_t j = na <= (uint32_t)kResThreads ? S.amb_idx[i] : __ldcg(gai + i);
-        if (kk > T2 || (kk == T2 && j <= jmax2)) {
-            atomicOr(&bm[j >> 5], 1u << (j & 31));
-            red_add_shared(&wc[j / a.fchunk], 1u);
-        }
+        if (kk > T2 || (kk == T2 && j <= jmax2)) mark(j);
     }
     __syncthreads();
     // output position of every chunk's first selected entry
-    const uint32_t v = tid < nfch ? cin + wc[tid] : 0u;
+    const uint32_t v = tid < nfch ? cin + S.wcnt[tid] : 0u;
     uint32_t total;
     const uint32_t pos = block_exclusive_scan(v, S.sh64, &total);
     if (tid < nfch) a.chunk_pos[(size_t)b * nfch + tid] = pos;
@@ -930,6 +928,7 @@ __global__ void __launch_bounds__(kResThreads, 1) topk_resolve_kernel(TopkDecode
         S.found = 0;
         S.pf_cnt = 0;
     }
+    S.wcnt[tid] = 0;  // kResThreads == kSelMaxChunks
     // the fine bin d2 of t~ inside bin d1 (rank K2 there)
     const uint32_t K2 = (uint32_t)k - above1;
     int d2;
