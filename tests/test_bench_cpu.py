@@ -1,0 +1,49 @@
+"""The bench's roofline arithmetic: algorithmic bytes of a decode step.
+
+Per sequence: N^C * 128 (indexer keys) + min(k, N^C) * 2 * 128 * b_kv
+(gathered K and V) + N^H * 2 * 128 * b_kv (HCA K and V) + H * 256 (q) + 128
+(q_I) + 2 * H * 256 (two outputs), with 8 more bytes per gathered entry and
+per 64 HCA entries for fp8 scales.  The totals are checked against the
+figures worked out by hand for the three uniform decode workloads, and the
+fp8 terms against a sum written out term by term.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+import bench
+from sparse_attention_pool_b200 import configs
+
+
+def test_decode_step_bytes_match_the_worked_figures():
+    expect = {  # bytes per step (all sequences)
+        "decode_b1_t4k_h8_k64": 186_496,
+        "decode_b16_t64k_h64_k512": 42_731_520,
+        "decode_b4_t1m_h64_k2048": 155_386_368,
+    }
+    for name, total in expect.items():
+        w = configs.BY_NAME[name]
+        step, score = bench.decode_bytes(w, np.full((w.B,), w.L))
+        assert step == total, name
+        nc = w.L // 4
+        assert score == w.B * nc * (128 + 4), name  # keys read + one 32-bit order key written
+
+
+def test_fp8_step_bytes_term_by_term():
+    w = configs.BY_NAME["ragged_fp8_b32_t64k-256k_h64_k1024"]
+    lengths = np.array([65536, 262144, 100003], dtype=np.int32)
+    step, _ = bench.decode_bytes(w, lengths)
+    ref = 0
+    for L in lengths:
+        nc, nh = int(L) // 4, int(L) // 128
+        sel = min(w.topk, nc)
+        ref += nc * 128                            # indexer keys (bf16)
+        ref += sel * 2 * 128 + sel * 8             # gathered e4m3 K, V + their two scales
+        ref += nh * 2 * 128 + ((nh + 63) // 64) * 8  # HCA e4m3 K, V + scales per 64 entries
+        ref += w.H * 256 + 128 + 2 * w.H * 256     # q, q_I, two outputs
+    assert step == ref
+
+
+def test_job_throughput_counts_every_rank():
+    assert bench.job_throughput(units_per_rank=40, world=1, max_ms=10.0) == 4000.0
+    assert bench.job_throughput(units_per_rank=40, world=8, max_ms=10.0) == 32000.0
