@@ -146,6 +146,18 @@ def test_decode_topk_all_equal_scores(S):
     assert (idx == np.arange(k)[None, :]).all() and (cnt == k).all()
 
 
+@pytest.mark.parametrize("k", [77, 2000])
+def test_decode_topk_all_equal_scores_overflow_paths(S, k):
+    # 10,000 identical entries: more candidates than the resolve holds in shared
+    # memory (the list goes to global memory), a crowded fine bin (the digit
+    # passes) and a band wider than 1024 (the global band cut)
+    B, Lcap = 1, 40000
+    inp = Inputs(305, B, Lcap, 8)
+    inp.KI[:] = inp.KI[:, :1, :]
+    _, _, _, idx, cnt = _topk_case(S, inp, k)
+    assert (idx == np.arange(k)[None, :]).all() and (cnt == k).all()
+
+
 def test_decode_topk_short_and_empty(S):
     B, Lcap, k = 3, 512, 200
     inp = Inputs(303, B, Lcap, 8, lengths=[512, 3, 0])         # 128, 0, 0 entries
