@@ -19,17 +19,18 @@
 //            with s~ < t~ - 2E surely not, and only the band |s~ - t~| <= 2E
 //            is rescored exactly (the fp64 definition) and ranked exactly.
 //
-// Four kernels, ordered on one stream (every hand-off is a kernel boundary;
-// no CTA waits on another):
+// Four kernels, ordered on one stream (every hand-off is a kernel boundary,
+// chained by programmatic dependent launch; no CTA waits on another):
 //   1. score_decode_kernel -- streams Ic through a 4-stage TMA pipeline
 //      (128-byte rows, 128B swizzle, one row per thread) and writes an order
 //      key of s~ per entry, a histogram of the top 11 key bits (per CTA in
-//      shared memory, then added to the sequence's) and each CTA's max e_j.
-//   2. topk_filter_kernel  -- one CTA per score chunk: from the histogram the
-//      bin d1 of t~; entries above that bin widened by 2E become bitmap bits
-//      (surely selected, counted per chunk), entries in the widened bin
-//      become candidates, and those inside bin d1 feed a histogram of key
-//      bits 20..10.
+//      shared memory, then added to the sequence's) and each CTA's max e_j;
+//      the sequence's last CTA to finish then finds the bin d1 of t~, the
+//      keys above it and E, once.
+//   2. topk_filter_kernel  -- one CTA per 2048 rows: entries above bin d1
+//      widened by 2E become bitmap bits (surely selected, counted per chunk),
+//      entries in the widened bin become candidates (compact slots of the
+//      chunk), and those inside bin d1 feed a histogram of key bits 20..10.
 //   3. topk_resolve_kernel -- one 1024-thread CTA per sequence: the second
 //      histogram gives the fine bin of t~, whose few keys are ranked; the band
 //      is rescored exactly and ranked by (s, -j); the winners join the bitmap
@@ -584,7 +585,7 @@ struct SelSmem {
     __align__(16) uint16_t pf_row[kPf][64];
 };
 
-// Filter: one CTA per 1024 rows.  Entries above the widened bin of t~ become
+// Filter: one CTA per kFiltRows (2048) rows.  Entries above the widened bin of t~ become
 // bitmap bits (surely selected, counted), the rest of the widened bin become
 // candidates in the chunk's own rows of the candidate arrays, and keys
 // inside bin d1 feed the second histogram.  Integer compares on order keys.
