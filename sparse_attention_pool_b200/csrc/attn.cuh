@@ -6,10 +6,14 @@
 // out_h = sum_j softmax_j(scale * q_h . K_j) V_j,  lse_h = log sum_j exp(.)
 //
 // One CTA handles one query (all H heads: M = 16 rows per warp) and one split
-// of its entry list, 64 entries per tile, double-buffered with cp.async into
-// XOR-swizzled shared memory.  QK^T and PV run on bf16 tensor-core MMAs with
-// fp32 accumulation (flash-decoding: online softmax in registers, P re-used
-// from the S accumulators).  An fp8 cache is widened to bf16 in shared memory
+// of its entry list, 64 entries per tile, pipelined with cp.async into
+// XOR-swizzled shared memory (all tiles of a short split in flight).  In
+// decode each tile is shared by two warp groups, 32 entries each, whose
+// softmax states merge at the end.  QK^T and PV run on bf16 tensor-core MMAs
+// (mma.sync) with fp32 accumulation (flash-decoding: online softmax in
+// registers, P re-used from the S accumulators).  The dense path can keep
+// only the last `win` visible rows: the sliding-window branch over raw
+// tokens.  An fp8 cache is widened to bf16 in shared memory
 // (every e4m3 value is exact in bf16); its per-64-entry scales multiply the S
 // columns (K) and the P columns (V) in fp32.  With one split the CTA writes
 // the bf16 output directly; otherwise it writes a normalised fp32 partial and

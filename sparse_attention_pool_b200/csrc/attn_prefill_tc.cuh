@@ -10,7 +10,9 @@
 //     visible count floor(t / m).
 //   * CSA (gathered): a tile holds 64 entries of each query's top-k list
 //     (rows 0-63 of the tile from query 0's list, 64-127 from query 1's);
-//     a row sees only its own query's half (block-diagonal mask).
+//     a row sees only its own query's half (block-diagonal mask).  This
+//     variant wastes half of every MMA and is not dispatched: the mma.sync
+//     kernel is faster for the gathered lists; the dense one is used.
 // Per tile: S = Q K^T (tcgen05.mma, M=128 N=128, fp32 in tensor memory),
 // the softmax reads S with tcgen05.ld (one thread per row), writes P in
 // bf16 to shared memory, then PV = P V (tcgen05.mma, V as an MN-major
