@@ -66,6 +66,22 @@ def lib():
                                       ctypes.c_int, P, P, P, P, i64, ctypes.c_int, i32, dbl,
                                       P, P, P, P, P, P]
         L.or_hybrid_query.restype = None
+        L.or_e2m1_to_double.argtypes = [ctypes.c_uint8]
+        L.or_e2m1_to_double.restype = dbl
+        L.or_e2m1_from_double_satfinite.argtypes = [dbl]
+        L.or_e2m1_from_double_satfinite.restype = ctypes.c_uint8
+        L.or_e8m0_to_double.argtypes = [ctypes.c_uint8]
+        L.or_e8m0_to_double.restype = dbl
+        L.or_mxfp4_quantize.argtypes = [P, i64, ctypes.c_int, P, P]
+        L.or_mxfp4_quantize.restype = None
+        L.or_mxfp4_index_scores.argtypes = [P, P, P, P, i64, ctypes.c_int, P]
+        L.or_mxfp4_index_scores.restype = None
+        L.or_mixed_quantize.argtypes = [P, i64, ctypes.c_int, ctypes.c_int, P, P, P]
+        L.or_mixed_quantize.restype = None
+        L.or_attention_kv.argtypes = [P, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_int, P, P, P, ctypes.c_int, P, P, P, ctypes.c_int,
+                                      P, i64, dbl, P, P]
+        L.or_attention_kv.restype = None
         _lib = L
     return _lib
 
@@ -245,3 +261,117 @@ def union_attention(q: np.ndarray, parts, scale: float):
         H = np.asarray(q).shape[0]
         return np.zeros((H, d)), np.full((H,), -np.inf)
     return attention(q, Ku, Vu, np.arange(Ku.shape[0], dtype=np.int32), scale)
+
+
+# -- low-precision storage on the CSA path ------------------------------------
+# "DeepSeek-V4 ... Review", section 3-2 (2) ("Mixed KV storage": rotary dims in
+# BF16, the rest in FP8) and section 3-2 (4) (FP4 on the CSA indexer QK path).
+# The readings (MXFP4 for the indexer, the last d_rope dims of K as the rotary
+# dims, V all e4m3) are stated in the header of sa_oracle.c.
+
+def e2m1_to_double(code: int) -> float:
+    return lib().or_e2m1_to_double(int(code))
+
+
+def e2m1_from_double(x: float) -> int:
+    return int(lib().or_e2m1_from_double_satfinite(float(x)))
+
+
+def e8m0_to_double(code: int) -> float:
+    return lib().or_e8m0_to_double(int(code))
+
+
+def mxfp4_quantize(x: np.ndarray):
+    """x [n][d] uint16 (bf16), d a multiple of 32 -> (codes [n][d/2] uint8,
+    element 2i in the low nibble; scales [n][d/32] uint8 E8M0 codes)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    n, d = x.shape
+    assert d % 32 == 0
+    codes = np.zeros((n, d // 2), dtype=np.uint8)
+    scales = np.zeros((n, d // 32), dtype=np.uint8)
+    lib().or_mxfp4_quantize(_p(x), n, d, _p(codes), _p(scales))
+    return codes, scales
+
+
+def mxfp4_to_f64(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """Dequantize MXFP4 rows: [n][d/2] codes, [n][d/32] scales -> [n][d] f64."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    n, half = codes.shape
+    table = np.array([lib().or_e2m1_to_double(c) for c in range(16)], dtype=np.float64)
+    el = np.empty((n, 2 * half), dtype=np.float64)
+    el[:, 0::2] = table[codes & 0xF]
+    el[:, 1::2] = table[codes >> 4]
+    sc = np.array([lib().or_e8m0_to_double(c) for c in range(256)], dtype=np.float64)[np.asarray(scales, np.uint8)]
+    return el * np.repeat(sc, 32, axis=1)
+
+
+def mxfp4_index_scores(q_codes, q_scales, k_codes, k_scales) -> np.ndarray:
+    """FP4 index scores of one MXFP4 query against n MXFP4 key rows (fp32)."""
+    qc = np.ascontiguousarray(np.asarray(q_codes, np.uint8).reshape(-1))
+    qs = np.ascontiguousarray(np.asarray(q_scales, np.uint8).reshape(-1))
+    kc = np.ascontiguousarray(k_codes, dtype=np.uint8)
+    ks = np.ascontiguousarray(k_scales, dtype=np.uint8)
+    n = kc.shape[0]
+    d = 2 * qc.shape[0]
+    assert kc.shape[1] * 2 == d and ks.shape == (n, d // 32) and qs.shape[0] == d // 32
+    s = np.zeros((n,), dtype=np.float32)
+    lib().or_mxfp4_index_scores(_p(qc), _p(qs), _p(kc), _p(ks), n, d, _p(s))
+    return s
+
+
+def mixed_quantize(xc: np.ndarray, d_rope: int = 64):
+    """Mixed storage of a compressed K: (codes [n][d - d_rope] e4m3 for the
+    leading dims, scales [ceil(n/64)] fp32 over those dims, rope [n][d_rope]
+    bf16 bits = the trailing dims unchanged)."""
+    xc = np.ascontiguousarray(xc, dtype=np.uint16)
+    n, d = xc.shape
+    codes = np.zeros((n, d - d_rope), dtype=np.uint8)
+    scales = np.zeros(((n + 63) // 64,), dtype=np.float32)
+    rope = np.zeros((n, d_rope), dtype=np.uint16)
+    lib().or_mixed_quantize(_p(xc), n, d, d_rope, _p(codes), _p(scales), _p(rope))
+    return codes, scales, rope
+
+
+_KV_MODES = {"bf16": 0, "fp8": 1, "mixed": 2}
+
+
+def attention_kv(q: np.ndarray, k: dict, v: dict, rows, scale: float, d_rope: int = 64):
+    """O5 with K and V in any storage: each of k, v is a dict with "mode"
+    ("bf16", "fp8" or "mixed"), "data" (bf16 bits / e4m3 codes), "scales"
+    (fp8 and mixed) and "rope" (mixed).  Returns (out [H][d], lse [H])."""
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    H, d = q.shape
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+    out = np.zeros((H, d), dtype=np.float64)
+    lse = np.zeros((H,), dtype=np.float64)
+
+    def parts(t):
+        data = np.ascontiguousarray(t["data"])
+        sc = t.get("scales")
+        sc = None if sc is None else np.ascontiguousarray(sc, dtype=np.float32)
+        ro = t.get("rope")
+        ro = None if ro is None else np.ascontiguousarray(ro, dtype=np.uint16)
+        return _KV_MODES[t["mode"]], data, sc, ro
+    km, kd, ksc, kro = parts(k)
+    vm, vd, vsc, vro = parts(v)
+    lib().or_attention_kv(_p(q), H, d, km, _p(kd), _p(ksc), _p(kro), vm, _p(vd), _p(vsc), _p(vro),
+                          int(d_rope), _p(rows), rows.shape[0], float(scale), _p(out), _p(lse))
+    return out, lse
+
+
+def lowp_query(K, V, KI, q, qI, t: int, k: int, scale: float, d_rope: int = 64, m: int = 4):
+    """One CSA query with the low-precision storage: compress (O1), MXFP4
+    indexer keys and query, FP4 scores, top-k (O4), then attention over the
+    selected entries with mixed-storage K and e4m3 V.  Returns a dict."""
+    ck, cv, ci = compress(K, m), compress(V, m), compress(KI, m)
+    kc, ks = mxfp4_quantize(ci)
+    qc, qs = mxfp4_quantize(np.asarray(qI, np.uint16).reshape(1, -1))
+    n_vis = min(int(t) // m, ci.shape[0])
+    s = mxfp4_index_scores(qc[0], qs[0], kc[:n_vis], ks[:n_vis])
+    idx, cnt = topk(s, k)
+    codes, sc, rope = mixed_quantize(ck, d_rope)
+    vcodes, vsc = fp8_quantize(cv)
+    out, lse = attention_kv(q, {"mode": "mixed", "data": codes, "scales": sc, "rope": rope},
+                            {"mode": "fp8", "data": vcodes, "scales": vsc}, idx[:cnt], scale, d_rope)
+    return {"scores": s, "idx": idx, "cnt": cnt, "out": out, "lse": lse,
+            "idx_codes": kc, "idx_scales": ks, "q_codes": qc[0], "q_scales": qs[0]}

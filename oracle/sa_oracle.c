@@ -293,3 +293,186 @@ void or_hybrid_query(const uint16_t* q, const uint16_t* qI, int H, int d, int dI
     or_attention(q, H, d, hk, hks, hv, hvs, kv_fp8, rows, vis_h, scale, out_hca, lse_hca, NULL);
     free(rows);
 }
+
+/* ====================================================================== */
+/* Low-precision storage on the CSA path ("DeepSeek-V4 ... Review",        */
+/* section 3-2 (2), the "Mixed KV storage" row of the component table,     */
+/* and section 3-2 (4): FP4 on the CSA indexer QK path).  The pages name   */
+/* the formats only; the readings implemented below are:                   */
+/*   - indexer FP4 = OCP Microscaling MXFP4: e2m1 elements in blocks of 32 */
+/*     consecutive indexer dims, one E8M0 (power of two) scale per block,  */
+/*     X = 2^(floor(log2 amax) - 2) with the exponent clamped to           */
+/*     [-127, 127] (E8M0 code 0 when amax == 0), element =                 */
+/*     e2m1_rne_satfinite(x / X); both the query and the compressed keys   */
+/*     are quantized this way;                                             */
+/*   - FP4 index score = fp32_rne of the exact real sum over the two       */
+/*     blocks of X_q * X_k * sum_i e2m1(q_i) * e2m1(k_i);                   */
+/*   - mixed KV storage = the last d_rope dims of each K entry kept in     */
+/*     bf16 (the rotary dims), the other K dims and all of V in e4m3 with  */
+/*     the per-64-entry scale of O2 taken over the stored-e4m3 dims only.  */
+/* ====================================================================== */
+
+/* e2m1: 1 sign bit, 2 exponent bits (bias 1), 1 fraction bit; no inf or   */
+/* NaN.  Magnitudes: 0, 0.5 (the subnormal), 1, 1.5, 2, 3, 4, 6.            */
+double or_e2m1_to_double(uint8_t c) {
+    int sign = (c >> 3) & 1;
+    int e = (c >> 1) & 0x3;
+    int f = c & 0x1;
+    double v = (e == 0) ? 0.5 * (double)f : ldexp(1.0 + 0.5 * (double)f, e - 1);
+    return sign ? -v : v;
+}
+
+/* Nearest e2m1 value, ties to an even fraction bit, clamped to +-6. */
+uint8_t or_e2m1_from_double_satfinite(double x) {
+    uint8_t sign = signbit(x) ? 0x8 : 0;
+    if (isnan(x)) return sign | 0x7;  /* no NaN in e2m1: saturate */
+    double a = fabs(x);
+    if (isinf(a)) return sign | 0x7;
+    int e2;
+    (void)frexp(a, &e2);
+    int ex = (a == 0.0) ? 0 : e2 - 1;  /* floor(log2 a) */
+    if (ex < 0) ex = 0;                /* spacing 0.5 below 2 (subnormal + first binade) */
+    if (ex > 2) ex = 2;
+    double quantum = ldexp(1.0, ex - 1);
+    double y = nearbyint(a / quantum) * quantum;
+    if (y > 6.0) y = 6.0;
+    if (y < 1.0) return sign | (uint8_t)(y * 2.0);  /* 0 or the subnormal 0.5 */
+    (void)frexp(y, &e2);
+    int ey = e2 - 1;                                  /* 0, 1 or 2 */
+    int frac = (int)((y / ldexp(1.0, ey) - 1.0) * 2.0);
+    return sign | (uint8_t)((ey + 1) << 1) | (uint8_t)frac;
+}
+
+/* E8M0: an unsigned biased exponent, value 2^(c - 127); 0xFF is NaN. */
+double or_e8m0_to_double(uint8_t c) {
+    if (c == 0xFF) return NAN;
+    return ldexp(1.0, (int)c - 127);
+}
+
+/* MXFP4 quantization of rows of bf16 values.  x: [n][d] bf16 bits, d a     */
+/* multiple of 32.  codes: [n][d/2], element 2i in the low nibble of byte i */
+/* and element 2i+1 in the high nibble; scales: [n][d/32] E8M0 codes.       */
+void or_mxfp4_quantize(const uint16_t* x, int64_t n, int d, uint8_t* codes, uint8_t* scales) {
+    for (int64_t j = 0; j < n; ++j) {
+        for (int b = 0; b < d / 32; ++b) {
+            const uint16_t* xb = x + j * d + b * 32;
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i) {
+                double v = fabs(or_bf16_to_double(xb[i]));
+                if (v > amax) amax = v;
+            }
+            int se;
+            if (amax == 0.0) {
+                se = -127;
+            } else {
+                int e2;
+                (void)frexp(amax, &e2);
+                se = (e2 - 1) - 2;  /* floor(log2 amax) - (largest e2m1 exponent) */
+                if (se < -127) se = -127;
+                if (se > 127) se = 127;
+            }
+            scales[j * (d / 32) + b] = (uint8_t)(se + 127);
+            double X = ldexp(1.0, se);
+            for (int i = 0; i < 32; ++i) {
+                uint8_t c = or_e2m1_from_double_satfinite(or_bf16_to_double(xb[i]) / X);
+                int64_t byte = j * (d / 2) + b * 16 + i / 2;
+                if (i % 2 == 0) codes[byte] = c;
+                else codes[byte] |= (uint8_t)(c << 4);
+            }
+        }
+    }
+}
+
+static double or_mxfp4_elem(const uint8_t* codes, int64_t row, int d, int i) {
+    uint8_t byte = codes[row * (d / 2) + i / 2];
+    return or_e2m1_to_double((i % 2 == 0) ? (byte & 0xF) : (byte >> 4));
+}
+
+/* FP4 index scores.  qc/qs: one MXFP4 query ([d/2] codes, [d/32] scales);  */
+/* kc/ks: n MXFP4 key rows.  Each block's dot product is a multiple of 1/4  */
+/* below 2^11 in magnitude and is exact in fp64, as is its product with the */
+/* two power-of-two scales; the sum of the two block terms is exact in fp64 */
+/* whenever their exponents lie within 40 of each other.  Otherwise the     */
+/* smaller term is below 2^-27 of the larger, which has at most 13          */
+/* significant bits, and rounding the fp64 sum to fp32 gives the larger     */
+/* term -- the correctly rounded result -- in the normal fp32 range.        */
+void or_mxfp4_index_scores(const uint8_t* qc, const uint8_t* qs, const uint8_t* kc, const uint8_t* ks,
+                           int64_t n, int d, float* s) {
+    for (int64_t j = 0; j < n; ++j) {
+        double acc = 0.0;
+        for (int b = 0; b < d / 32; ++b) {
+            double blk = 0.0;
+            for (int i = b * 32; i < b * 32 + 32; ++i)
+                blk += or_mxfp4_elem(qc, 0, d, i) * or_mxfp4_elem(kc, j, d, i);
+            acc += blk * or_e8m0_to_double(qs[b]) * or_e8m0_to_double(ks[j * (d / 32) + b]);
+        }
+        float r = (float)acc;
+        if (r == 0.0f) r = 0.0f; /* -0 -> +0 */
+        s[j] = r;
+    }
+}
+
+/* Mixed KV storage of one compressed K tensor.  xc: [n][d] bf16 bits.      */
+/* codes: [n][d - d_rope] e4m3 for dims [0, d - d_rope); scales:            */
+/* [ceil(n/64)] fp32 over those dims (the O2 rule); rope: [n][d_rope] bf16  */
+/* bits, dims [d - d_rope, d) unchanged.                                    */
+void or_mixed_quantize(const uint16_t* xc, int64_t n, int d, int d_rope,
+                       uint8_t* codes, float* scales, uint16_t* rope) {
+    int dn = d - d_rope;
+    uint16_t* nope = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(n > 0 ? n : 1) * (size_t)(dn > 0 ? dn : 1));
+    for (int64_t j = 0; j < n; ++j) {
+        for (int i = 0; i < dn; ++i) nope[j * dn + i] = xc[j * d + i];
+        for (int i = 0; i < d_rope; ++i) rope[j * d_rope + i] = xc[j * d + dn + i];
+    }
+    if (dn > 0) or_fp8_quantize(nope, n, dn, codes, scales);
+    free(nope);
+}
+
+/* One stored K or V tensor for or_attention_kv.  mode 0: bf16 [N][d];      */
+/* mode 1: e4m3 [N][d] + scales; mode 2: mixed (e4m3 [N][d - d_rope] +      */
+/* scales, then bf16 rope [N][d_rope]).                                     */
+static double or_kv_elem(int mode, const void* base, const float* scales, const uint16_t* rope, int d_rope,
+                         int64_t j, int d, int i) {
+    if (mode == 0) return or_bf16_to_double(((const uint16_t*)base)[j * d + i]);
+    if (mode == 1) return or_e4m3_to_double(((const uint8_t*)base)[j * d + i]) * (double)scales[j / 64];
+    int dn = d - d_rope;
+    if (i >= dn) return or_bf16_to_double(rope[j * d_rope + (i - dn)]);
+    return or_e4m3_to_double(((const uint8_t*)base)[j * dn + i]) * (double)scales[j / 64];
+}
+
+/* O5 with K and V each in any of the storage modes above. */
+void or_attention_kv(const uint16_t* q, int H, int d,
+                     int k_mode, const void* K, const float* ks, const uint16_t* k_rope,
+                     int v_mode, const void* V, const float* vs, const uint16_t* v_rope, int d_rope,
+                     const int32_t* rows, int64_t nrows, double scale,
+                     double* out, double* lse) {
+    double* z = (double*)malloc(sizeof(double) * (size_t)(nrows > 0 ? nrows : 1));
+    for (int h = 0; h < H; ++h) {
+        double* o = out + (int64_t)h * d;
+        for (int i = 0; i < d; ++i) o[i] = 0.0;
+        if (nrows == 0) {
+            lse[h] = -INFINITY;
+            continue;
+        }
+        double zmax = -INFINITY;
+        for (int64_t r = 0; r < nrows; ++r) {
+            double acc = 0.0;
+            for (int i = 0; i < d; ++i)
+                acc += or_bf16_to_double(q[(int64_t)h * d + i]) *
+                       or_kv_elem(k_mode, K, ks, k_rope, d_rope, rows[r], d, i);
+            z[r] = acc * scale;
+            if (z[r] > zmax) zmax = z[r];
+        }
+        double l = 0.0;
+        for (int64_t r = 0; r < nrows; ++r) {
+            z[r] = exp(z[r] - zmax);
+            l += z[r];
+        }
+        for (int64_t r = 0; r < nrows; ++r) {
+            double w = z[r] / l;
+            for (int i = 0; i < d; ++i) o[i] += w * or_kv_elem(v_mode, V, vs, v_rope, d_rope, rows[r], d, i);
+        }
+        lse[h] = zmax + log(l);
+    }
+    free(z);
+}
