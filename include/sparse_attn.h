@@ -167,6 +167,34 @@ sa_status csa_index_topk(const void* q_idx, int32_t Tq, const int32_t* q_pos,
                          const sa_cache* csa, int32_t k, int32_t* idx, int32_t* cnt,
                          void* ws, size_t ws_bytes, void* stream);
 
+/* FP4 indexer keys, section 3-2 (4) ("FP4 quantization-aware training ... in
+ * the CSA indexer QK path"; the page names the precision only).  Format read
+ * here: MXFP4 of the OCP Microscaling specification.  Each compressed
+ * indexer key (64 bf16 dims, as csa_compress writes them) becomes two blocks
+ * of 32 e2m1 elements with one E8M0 scale per block:
+ *   X = 2^(floor(log2 amax) - 2), exponent clamped to [-127, 127], E8M0 code
+ *       0 when amax == 0;  element = e2m1 round-to-nearest-even of x / X,
+ *       saturating at +-6, sign kept.
+ *   codes  [B][Ncap][32] uint8 out: element 2i in the low nibble of byte i,
+ *          element 2i+1 in the high nibble.
+ *   scales [B][Ncap][2] uint8 out: E8M0 codes of blocks 0 (dims 0..31) and 1.
+ * Entries row_from .. n[b]-1 of every sequence are (re)written; the others
+ * are left alone (after an append, pass the smallest old n to refresh the new
+ * entries only).  Both buffers are the caller's, 16-byte aligned.            */
+sa_status csa_index_quantize_mxfp4(const sa_cache* csa, int32_t row_from, uint8_t* codes, uint8_t* scales,
+                                   void* stream);
+
+/* Decode top-k on FP4 indexer scores (same section).  The query q_idx
+ * [B][d_idx] bf16 is quantized in the kernel by the rule above; the score of
+ * entry j is the fp32 value, rounded to nearest even once, of the exact sum
+ * over the two blocks of X_q * X_k * sum_i e2m1(q_i) * e2m1(k_ji) (-0 -> +0).
+ * Selection, order, padding and count are those of csa_index_topk with
+ * q_pos == NULL.  codes / scales as written by csa_index_quantize_mxfp4 for
+ * the entries 0..n[b]-1; the bf16 indexer keys of the cache are not read.
+ * ws / ws_bytes: at least sa_workspace_size(SA_OP_INDEX_TOPK, B, 1, ...).     */
+sa_status csa_index_topk_mxfp4(const void* q_idx, const sa_cache* csa, const uint8_t* codes, const uint8_t* scales,
+                               int32_t k, int32_t* idx, int32_t* cnt, void* ws, size_t ws_bytes, void* stream);
+
 /* CSA attention over the chosen entries, section 3-2 (2) (CSA attends over
  * the selected entries only).
  *   q   [B][Tq][H][d] bf16; idx / cnt as produced by csa_index_topk (an index

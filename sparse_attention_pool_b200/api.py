@@ -184,6 +184,40 @@ def csa_index_topk_noalloc(q_idx, csa: Cache, k: int, *, idx=None, cnt=None, str
     return idx, cnt
 
 
+def csa_index_quantize_mxfp4(csa: Cache, *, codes=None, scales=None, row_from: int = 0, stream=None):
+    """MXFP4 copy of the cache's bf16 indexer keys (entries row_from .. n-1):
+    codes [B][Ncap][32] uint8 (two e2m1 per byte, even element low), scales
+    [B][Ncap][2] uint8 (E8M0).  Returns (codes, scales)."""
+    dev = csa.k.device
+    if codes is None:
+        codes = torch.zeros(csa.B, csa.Ncap, 32, dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.zeros(csa.B, csa.Ncap, 2, dtype=torch.uint8, device=dev)
+    _need(codes, torch.uint8, "codes")
+    _need(scales, torch.uint8, "scales")
+    cs = csa.struct()
+    check("csa_index_quantize_mxfp4", lib().csa_index_quantize_mxfp4(ctypes.byref(cs), int(row_from), _ptr(codes),
+                                                                     _ptr(scales), _stream(stream)))
+    return codes, scales
+
+
+def csa_index_topk_mxfp4(q_idx, csa: Cache, codes, scales, k: int, ws, *, idx=None, cnt=None, stream=None):
+    """Decode top-k on FP4 (MXFP4) indexer scores; idx [B][1][k], cnt [B][1]."""
+    _need(q_idx, torch.bfloat16, "q_idx")
+    _need(codes, torch.uint8, "codes")
+    _need(scales, torch.uint8, "scales")
+    B = csa.B
+    if idx is None:
+        idx = torch.empty(B, 1, k, dtype=torch.int32, device=q_idx.device)
+    if cnt is None:
+        cnt = torch.empty(B, 1, dtype=torch.int32, device=q_idx.device)
+    cs = csa.struct()
+    check("csa_index_topk_mxfp4", lib().csa_index_topk_mxfp4(_ptr(q_idx), ctypes.byref(cs), _ptr(codes), _ptr(scales),
+                                                             k, _ptr(idx), _ptr(cnt), _ptr(ws), ws.numel(),
+                                                             _stream(stream)))
+    return idx, cnt
+
+
 def csa_sparse_attn(q, csa: Cache, idx, cnt, k: int, ws, *, scale=0.0, out=None, lse=None, stream=None):
     _need(q, torch.bfloat16, "q")
     B, Tq, H = q.shape[0], (q.shape[1] if q.dim() == 4 else 1), q.shape[-2]

@@ -18,6 +18,7 @@
 #include "attn.cuh"
 #include "attn_prefill_tc.cuh"
 #include "compress.cuh"
+#include "lowp_index.cuh"
 #include "sa_common.cuh"
 #include "topk_decode.cuh"
 #include "topk_prefill.cuh"
@@ -470,12 +471,25 @@ sa_status run_attn(const void* q, int Tq, int H, const sa_cache* c, bool gather,
     return SA_OK;
 }
 
+// Rows per FP4 score CTA: about four CTAs per SM over the whole batch, whole
+// passes of the CTA.
+int fp4_score_chunk(int B, int Ncap) {
+    const long long target = (long long)num_sms() * 4;
+    long long chunk = ((long long)B * Ncap + target - 1) / target;
+    chunk = ((chunk + sa::kF4Rows - 1) / sa::kF4Rows) * sa::kF4Rows;
+    return (int)std::max<long long>(chunk, sa::kF4Rows);
+}
+
 // The indexer + top-k of a decode step: the score kernel (the HBM stream),
 // the filter, the resolve and the emit.  `between` runs after the filter is
-// queued (the hybrid step forks its HCA branch there).
+// queued (the hybrid step forks its HCA branch there).  With MXFP4 keys
+// (codes4 / scales4 non-NULL) the FP4 score kernel writes exact keys and the
+// resolve runs its EXACT variant; the bf16 keys are then not read.
 template <typename F>
 sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* idx, int32_t* cnt, void* ws,
-                          const TopkDecodeWs& w, cudaStream_t st, F&& between) {
+                          const TopkDecodeWs& w, cudaStream_t st, F&& between, const uint8_t* codes4 = nullptr,
+                          const uint8_t* scales4 = nullptr) {
+    const bool fp4 = codes4 != nullptr;
     const int B = c->B, Ncap = c->Ncap;
     uint8_t* base = static_cast<uint8_t*>(ws);
     sa::TopkDecodeArgs a{};
@@ -503,7 +517,7 @@ sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* 
     a.Ncap = Ncap;
     a.Wcap = w.Wcap;
     a.k = k;
-    a.chunk = score_chunk(B, Ncap);
+    a.chunk = fp4 ? fp4_score_chunk(B, Ncap) : score_chunk(B, Ncap);
     a.nchunks = Ncap > 0 ? cdiv(Ncap, a.chunk) : 1;
     a.fchunk = w.fchunk;
     a.nfch = w.nfch;
@@ -513,11 +527,19 @@ sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* 
     const size_t smem = sa::kScStages * sa::kScTileBytes + sa::kScStages * 8 + 1024;
     if (!attr_done(init)) {
         SA_CUDA(cudaFuncSetAttribute(sa::score_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-        SA_CUDA(cudaFuncSetAttribute(sa::topk_resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        SA_CUDA(cudaFuncSetAttribute(sa::topk_resolve_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     sa::kSelSmem));
+        SA_CUDA(cudaFuncSetAttribute(sa::topk_resolve_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      sa::kSelSmem));
         attr_set(init);
     }
-    if (Ncap > 0) {
+    if (Ncap > 0 && fp4) {
+        SA_CUDA(cudaMemsetAsync(a.hist1, 0, w.zero_end - w.hist, st));
+        stage_mark(SA_STAGE_INDEX_SCORE, 0, st);
+        sa::score_decode_mxfp4_kernel<<<dim3(a.nchunks, B), sa::kF4Threads, 0, st>>>(a, codes4, scales4);
+        SA_LAUNCHED();
+        stage_mark(SA_STAGE_INDEX_SCORE, 1, st);
+    } else if (Ncap > 0) {
         CUtensorMap map;
         sa_status r = make_ic_map(&map, c->kidx, B, Ncap);
         if (r != SA_OK) return r;
@@ -537,7 +559,8 @@ sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* 
     // themselves, and what it queues overlaps the latency-bound rest
     sa_status r = between();
     if (r != SA_OK) return r;
-    SA_CUDA(launch_k(sa::topk_resolve_kernel, dim3(B), dim3(sa::kResThreads), sa::kSelSmem, st, pdl, 1u, a));
+    SA_CUDA(launch_k(fp4 ? sa::topk_resolve_kernel<true> : sa::topk_resolve_kernel<false>, dim3(B),
+                     dim3(sa::kResThreads), sa::kSelSmem, st, pdl, 1u, a));
     SA_LAUNCHED();
     SA_CUDA(launch_k(sa::topk_emit_kernel, dim3(a.nfch, B), dim3(sa::kEmitThreads), 0, st, pdl, 1u, a));
     SA_LAUNCHED();
@@ -887,6 +910,45 @@ sa_status csa_index_topk_noalloc(const void* q_idx, const sa_cache* csa, int32_t
     if (r != SA_OK) return r;
     return run_topk_decode(q_idx, csa, k, idx, cnt, scratch, w, static_cast<cudaStream_t>(stream),
                            [] { return SA_OK; });
+}
+
+sa_status csa_index_quantize_mxfp4(const sa_cache* csa, int32_t row_from, uint8_t* codes, uint8_t* scales,
+                                   void* stream) {
+    sa_status r = check_cache(csa, true, "csa_index_quantize_mxfp4");
+    if (r != SA_OK) return r;
+    SA_CHECK(row_from >= 0, "csa_index_quantize_mxfp4: row_from=%d", row_from);
+    SA_CHECK(codes && scales && aligned16(codes) && aligned16(scales),
+             "csa_index_quantize_mxfp4: codes and scales must be non-NULL and 16-byte aligned");
+    if (row_from >= csa->Ncap) return SA_OK;
+    sa::Mxfp4QuantArgs a{};
+    a.kidx = static_cast<const uint16_t*>(csa->kidx);
+    a.n = csa->n;
+    a.codes = codes;
+    a.scales = scales;
+    a.Ncap = csa->Ncap;
+    a.row_from = row_from;
+    const long long threads = 2LL * (csa->Ncap - row_from);
+    sa::mxfp4_quantize_kernel<<<dim3((unsigned)cdiv(threads, sa::kQuantThreads), csa->B), sa::kQuantThreads, 0,
+                                 static_cast<cudaStream_t>(stream)>>>(a);
+    SA_LAUNCHED();
+    return SA_OK;
+}
+
+sa_status csa_index_topk_mxfp4(const void* q_idx, const sa_cache* csa, const uint8_t* codes, const uint8_t* scales,
+                               int32_t k, int32_t* idx, int32_t* cnt, void* ws, size_t ws_bytes, void* stream) {
+    sa_status r = check_cache(csa, false, "csa_index_topk_mxfp4");
+    if (r != SA_OK) return r;
+    SA_CHECK(q_idx && aligned16(q_idx), "csa_index_topk_mxfp4: q_idx must be non-NULL and 16-byte aligned");
+    SA_CHECK(codes && scales && aligned16(codes) && aligned16(scales),
+             "csa_index_topk_mxfp4: codes and scales must be non-NULL and 16-byte aligned");
+    SA_CHECK(idx && cnt && aligned16(idx) && aligned16(cnt),
+             "csa_index_topk_mxfp4: idx/cnt must be non-NULL and aligned");
+    SA_CHECK(k >= 1 && k <= 65536, "csa_index_topk_mxfp4: k=%d outside 1..65536", k);
+    const TopkDecodeWs w = topk_decode_layout(csa->B, csa->Ncap, k, false);
+    r = check_ws(ws, ws_bytes, w.total);
+    if (r != SA_OK) return r;
+    return run_topk_decode(q_idx, csa, k, idx, cnt, ws, w, static_cast<cudaStream_t>(stream),
+                           [] { return SA_OK; }, codes, scales);
 }
 
 sa_status csa_sparse_attn(const void* q, int32_t Tq, int32_t H, const sa_cache* csa, const int32_t* idx,

@@ -677,8 +677,10 @@ __global__ void __launch_bounds__(kSelThreads) topk_filter_kernel(TopkDecodeArgs
 // fine bin of t~ and prefetching into L2 the index rows around it, which
 // the exact rescoring of the band will read), finds t~, rescores the band
 // exactly, cuts it by (s, -j), adds the winners to the bitmap and gives
-// every chunk its output position.
-template <bool SMEM>
+// every chunk its output position.  EXACT: the keys are the exact scores
+// already (E = 0, the band is the keys equal to t~'s), so nothing is staged
+// or rescored.
+template <bool SMEM, bool EXACT>
 __device__ __forceinline__ void resolve_body(const TopkDecodeArgs& a, SelSmem& S, uint32_t* csm, int b, uint32_t C,
                                              uint32_t A, int d1, float E, int d2, uint32_t above2, uint32_t K2,
                                              const uint32_t (&pk)[kGatherJ * kGatherS],
@@ -702,9 +704,11 @@ __device__ __forceinline__ void resolve_body(const TopkDecodeArgs& a, SelSmem& S
             if (q < (uint32_t)kPf) {
                 S.pf_key[q] = kk;
                 S.pf_j[q] = j;
-                const uint16_t* row = icx + (size_t)j * 64;
+                if (!EXACT) {
+                    const uint16_t* row = icx + (size_t)j * 64;
 #pragma unroll
-                for (int u = 0; u < 8; ++u) cp_async16(&S.pf_row[q][u * 8], row + u * 8);
+                    for (int u = 0; u < 8; ++u) cp_async16(&S.pf_row[q][u * 8], row + u * 8);
+                }
             }
             if (f == pre) {
                 const uint32_t p = atom_add_shared(&S.f_cnt, 1u);
@@ -799,7 +803,7 @@ __device__ __forceinline__ void resolve_body(const TopkDecodeArgs& a, SelSmem& S
             const uint32_t kk = S.pf_key[tid];
             if (kk >= blo_key && kk <= bhi_key) {
                 const uint32_t p = atom_add_shared(&S.amb_cnt, 1u);
-                S.amb_key[p] = exact_key<true>(S.q2, S.pf_row[tid]);
+                S.amb_key[p] = EXACT ? kk : exact_key<true>(S.q2, S.pf_row[tid]);
                 S.amb_idx[p] = S.pf_j[tid];
             }
         }
@@ -813,7 +817,7 @@ __device__ __forceinline__ void resolve_body(const TopkDecodeArgs& a, SelSmem& S
             } else if (kk >= blo_key) {
                 const int32_t j = li[i];
                 const uint32_t p = atom_add_shared(&S.amb_cnt, 1u);
-                const uint32_t ek = exact_key(S.q2, icx + (size_t)j * 64);
+                const uint32_t ek = EXACT ? kk : exact_key(S.q2, icx + (size_t)j * 64);
                 if (p < (uint32_t)kResThreads) {
                     S.amb_key[p] = ek;
                     S.amb_idx[p] = j;
@@ -881,6 +885,7 @@ __device__ __forceinline__ void resolve_body(const TopkDecodeArgs& a, SelSmem& S
 // registers) and, ahead of their counts, the first 32 candidate slots of
 // each warp's first kGatherJ chunks; the fine bin of t~ then follows from
 // the registers.
+template <bool EXACT>
 __global__ void __launch_bounds__(kResThreads, 1) topk_resolve_kernel(TopkDecodeArgs a) {
     extern __shared__ __align__(16) uint32_t csm[];  // [kSelCap] keys, [kSelCap] indices
     __shared__ SelSmem S;
@@ -947,9 +952,9 @@ __global__ void __launch_bounds__(kResThreads, 1) topk_resolve_kernel(TopkDecode
         C = a.Ncap;
     }
     if (C <= (uint32_t)kSelCap)
-        resolve_body<true>(a, S, csm, b, C, A, d1, E, d2, above2, K2, pk, pi, cin);
+        resolve_body<true, EXACT>(a, S, csm, b, C, A, d1, E, d2, above2, K2, pk, pi, cin);
     else
-        resolve_body<false>(a, S, csm, b, C, A, d1, E, d2, above2, K2, pk, pi, cin);
+        resolve_body<false, EXACT>(a, S, csm, b, C, A, d1, E, d2, above2, K2, pk, pi, cin);
     (void)ain;
 }
 

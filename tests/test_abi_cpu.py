@@ -157,3 +157,22 @@ def test_topk_and_attention_reject_bad_arguments(L):
     assert L.hybrid_attn_decode(P(FAKE), P(FAKE), 8, ctypes.byref(c), ctypes.byref(h2), 8, 0.0, P(FAKE), P(FAKE),
                                 None, None, None, None, P(FAKE), 1 << 30, None) == 1
     assert "B=" in L.sa_last_error().decode()
+
+
+def test_mxfp4_entry_points_reject_bad_arguments(L):
+    c = _cache()
+    P = ctypes.c_void_p
+    q = L.csa_index_quantize_mxfp4
+    assert q(ctypes.byref(c), 0, None, P(FAKE), None) == 1
+    assert q(ctypes.byref(c), 0, P(FAKE), P(FAKE + 2), None) == 1
+    assert "aligned" in L.sa_last_error().decode()
+    assert q(ctypes.byref(c), -1, P(FAKE), P(FAKE), None) == 1
+    assert "row_from" in L.sa_last_error().decode()
+    assert q(ctypes.byref(_cache(kidx=None)), 0, P(FAKE), P(FAKE), None) == 1
+    assert q(ctypes.byref(c), c.Ncap, P(FAKE), P(FAKE), None) == 0  # no entry to write: nothing launched
+    t = L.csa_index_topk_mxfp4
+    assert t(P(FAKE), ctypes.byref(c), P(FAKE), P(FAKE), 0, P(FAKE), P(FAKE), P(FAKE), 1 << 30, None) == 1
+    assert t(P(FAKE), ctypes.byref(c), P(FAKE + 8), P(FAKE), 8, P(FAKE), P(FAKE), P(FAKE), 1 << 30, None) == 1
+    assert t(P(FAKE), ctypes.byref(c), None, P(FAKE), 8, P(FAKE), P(FAKE), P(FAKE), 1 << 30, None) == 1
+    st = t(P(FAKE), ctypes.byref(c), P(FAKE), P(FAKE), 8, P(FAKE), P(FAKE), P(FAKE), 16, None)
+    assert st == _lib.SA_ERR_WORKSPACE

@@ -1,0 +1,137 @@
+"""The FP4 (MXFP4) CSA indexer against the oracle: csa_index_quantize_mxfp4
+must give the oracle's codes and scales bit for bit, and csa_index_topk_mxfp4
+the oracle's top-k of its FP4 scores ("DeepSeek-V4 ... Review", section 3-2
+(4), FP4 on the CSA indexer QK path; section 3-2 (2) top-k).
+
+These kernels have not yet run on a B200: the module runs only with
+SA_MXFP4_GPU_TESTS=1, so that their first run is a deliberate one.
+"""
+from __future__ import annotations
+
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from sparse_attention_pool_b200 import synth
+from tests._util import bits_to_torch_bf16
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(os.environ.get("SA_MXFP4_GPU_TESTS") != "1",
+                                 reason="MXFP4 kernels not yet run on a B200 (set SA_MXFP4_GPU_TESTS=1)")]
+
+
+@pytest.fixture(scope="module")
+def S():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import sparse_attention_pool_b200 as S
+    return S
+
+
+def _cache_with_keys(S, kidx_bits: np.ndarray, n):
+    """A CSA cache whose indexer keys are the given bf16 bits [B][Ncap][64]."""
+    B, Ncap, _ = kidx_bits.shape
+    c = S.alloc_cache(B, Ncap, 4, with_kidx=True)
+    c.kidx.copy_(bits_to_torch_bf16(kidx_bits).cuda())
+    c.n.copy_(torch.tensor(n, dtype=torch.int32))
+    return c
+
+
+def _edge_rows(x: np.ndarray):
+    """Plant rows that exercise the format: zero blocks, tiny and huge
+    magnitudes, -0, exact e2m1 midpoints and saturation."""
+    x[0, :32] = 0.0
+    x[1] *= 1e-30
+    x[2] *= 1e30
+    x[3, 5] = -0.0
+    x[4, :8] = [4.0, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, -0.25]
+    x[5, :4] = [6.0, 5.0, -5.0, 7.0]
+    x[6] = 0.0
+    return x
+
+
+def test_quantize_matches_oracle(S):
+    B, Ncap = 3, 3000
+    n = [3000, 1234, 7]
+    xf = synth.bf16_bits_to_f32(synth.normal_bf16(71, "kidx", (B, Ncap, 64))).copy()
+    xf[0] = _edge_rows(xf[0])
+    bits = (xf.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    c = _cache_with_keys(S, bits, n)
+    codes = torch.full((B, Ncap, 32), 0xAB, dtype=torch.uint8, device="cuda")
+    scales = torch.full((B, Ncap, 2), 0xCD, dtype=torch.uint8, device="cuda")
+    S.csa_index_quantize_mxfp4(c, codes=codes, scales=scales)
+    S.read_device_status()
+    gc, gs = codes.cpu().numpy(), scales.cpu().numpy()
+    for b in range(B):
+        oc, osc = O.mxfp4_quantize(bits[b, :n[b]])
+        assert np.array_equal(gc[b, :n[b]], oc), b
+        assert np.array_equal(gs[b, :n[b]], osc), b
+        assert (gc[b, n[b]:] == 0xAB).all() and (gs[b, n[b]:] == 0xCD).all(), b  # past n: untouched
+    # row_from: earlier rows are left alone
+    codes.fill_(0x11)
+    scales.fill_(0x22)
+    S.csa_index_quantize_mxfp4(c, codes=codes, scales=scales, row_from=1000)
+    S.read_device_status()
+    gc, gs = codes.cpu().numpy(), scales.cpu().numpy()
+    assert (gc[:, :1000] == 0x11).all() and (gs[:, :1000] == 0x22).all()
+    oc, osc = O.mxfp4_quantize(bits[0, :3000])
+    assert np.array_equal(gc[0, 1000:3000], oc[1000:]) and np.array_equal(gs[0, 1000:3000], osc[1000:])
+
+
+def _oracle_topk(qI_bits, kidx_bits, n, k):
+    qc, qs = O.mxfp4_quantize(qI_bits.reshape(1, -1))
+    kc, ks = O.mxfp4_quantize(kidx_bits[:n])
+    s = O.mxfp4_index_scores(qc[0], qs[0], kc, ks)
+    return O.topk(s, k)
+
+
+@pytest.mark.parametrize("k", [64, 512])
+def test_topk_matches_oracle(S, k):
+    B, Ncap = 5, 20000
+    n = [20000, 9000, k + 1, k, 3]  # large, ragged, one above k, exactly k, fewer than k
+    bits = synth.normal_bf16(72, "kidx", (B, Ncap, 64))
+    qI = synth.normal_bf16(72, "qidx", (B, 64))
+    c = _cache_with_keys(S, bits, n)
+    codes, scales = S.csa_index_quantize_mxfp4(c)
+    ws = S.alloc_workspace(S.workspace_size(S.SA_OP_INDEX_TOPK, B, 1, 8, Ncap, 0, k))
+    idx, cnt = S.csa_index_topk_mxfp4(bits_to_torch_bf16(qI).cuda(), c, codes, scales, k, ws)
+    S.read_device_status()
+    gi, gn = idx[:, 0].cpu().numpy(), cnt[:, 0].cpu().numpy()
+    for b in range(B):
+        ref, rc = _oracle_topk(qI[b], bits[b], n[b], k)
+        assert gn[b] == rc, b
+        assert np.array_equal(gi[b], ref), b
+
+
+def test_topk_all_equal_scores_take_the_lowest_indices(S):
+    B, Ncap, k = 2, 8192, 300
+    row = synth.normal_bf16(73, "kidx", (1, 64))[0]
+    bits = np.broadcast_to(row, (B, Ncap, 64)).copy()
+    qI = synth.normal_bf16(73, "qidx", (B, 64))
+    c = _cache_with_keys(S, bits, [Ncap, 5000])
+    codes, scales = S.csa_index_quantize_mxfp4(c)
+    ws = S.alloc_workspace(S.workspace_size(S.SA_OP_INDEX_TOPK, B, 1, 8, Ncap, 0, k))
+    idx, cnt = S.csa_index_topk_mxfp4(bits_to_torch_bf16(qI).cuda(), c, codes, scales, k, ws)
+    S.read_device_status()
+    assert (cnt[:, 0].cpu() == k).all()
+    assert (idx[:, 0].cpu().numpy() == np.arange(k)).all()
+
+
+def test_topk_full_size_decode(S):
+    """Four sequences of 262,144 entries (1M tokens each), k = 2048: every
+    index against the oracle."""
+    B, Ncap, k = 4, 262144, 2048
+    bits = synth.normal_bf16(74, "kidx", (B, Ncap, 64), scale=0.5)
+    qI = synth.normal_bf16(74, "qidx", (B, 64))
+    c = _cache_with_keys(S, bits, [Ncap] * B)
+    codes, scales = S.csa_index_quantize_mxfp4(c)
+    ws = S.alloc_workspace(S.workspace_size(S.SA_OP_INDEX_TOPK, B, 1, 64, Ncap, 0, k))
+    idx, cnt = S.csa_index_topk_mxfp4(bits_to_torch_bf16(qI).cuda(), c, codes, scales, k, ws)
+    S.read_device_status()
+    gi = idx[:, 0].cpu().numpy()
+    for b in range(B):
+        ref, rc = _oracle_topk(qI[b], bits[b], Ncap, k)
+        assert rc == k and np.array_equal(gi[b], ref), b
