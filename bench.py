@@ -167,18 +167,20 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def decode_bytes(w, lengths):
-    """Algorithmic HBM bytes of one decode step and of its indexer score kernel."""
+def decode_bytes(w, lengths, indexer="bf16"):
+    """Algorithmic HBM bytes of one decode step and of its indexer score kernel
+    (an indexer key is 128 bytes in bf16, 32 + 2 in MXFP4)."""
     bkv = 1 if w.fp8 else 2
+    ib = 128 if indexer == "bf16" else 34
     step = 0
     score = 0
     for L in lengths:
         nc, nh = int(L) // w.m_csa, int(L) // w.m_hca
         sel = min(w.topk, nc)
-        step += nc * 128 + sel * 2 * 128 * bkv + nh * 2 * 128 * bkv + w.H * 256 + 128 + 2 * w.H * 256
+        step += nc * ib + sel * 2 * 128 * bkv + nh * 2 * 128 * bkv + w.H * 256 + 128 + 2 * w.H * 256
         if w.fp8:
             step += sel * 8 + ((nh + 63) // 64) * 8
-        score += nc * 128 + nc * 4  # read the indexer keys, write one 32-bit key per entry
+        score += nc * ib + nc * 4  # read the indexer keys, write one 32-bit key per entry
     return step, score
 
 
@@ -235,6 +237,8 @@ def run_ours(args, w, rank, world, dev):
     hca = S.alloc_cache(w.B, w.L // w.m_hca, w.m_hca, fp8=w.fp8, device=dev)
     S.csa_compress(Kd, Vd, KId, lens, csa)
     S.hca_compress(Kd, Vd, lens, hca)
+    fp4 = args.indexer == "mxfp4"
+    codes4, scales4 = S.csa_index_quantize_mxfp4(csa) if fp4 else (None, None)  # like compression: untimed
     torch.cuda.synchronize()
     del Kd, Vd, KId
     torch.cuda.empty_cache()
@@ -260,9 +264,16 @@ def run_ours(args, w, rank, world, dev):
         flush_sink.copy_(flush.view(torch.int64).sum())
     L = _lib.lib()
 
+    def decode(qq, qqI):
+        if fp4:
+            S.hybrid_attn_decode_mxfp4(qq, qqI, csa, hca, codes4, scales4, k, ws, scale=SCALE, out_csa=out_c,
+                                       out_hca=out_h, lse_csa=lse_c, lse_hca=lse_h, idx_out=idx, cnt_out=cnt)
+        else:
+            S.hybrid_attn_decode(qq, qqI, csa, hca, k, ws, scale=SCALE, out_csa=out_c, out_hca=out_h,
+                                 lse_csa=lse_c, lse_hca=lse_h, idx_out=idx, cnt_out=cnt)
+
     def step():
-        S.hybrid_attn_decode(q, qI, csa, hca, k, ws, scale=SCALE, out_csa=out_c, out_hca=out_h, lse_csa=lse_c,
-                             lse_hca=lse_h, idx_out=idx, cnt_out=cnt)
+        decode(q, qI)
 
     # events around every stage of the step (captured into the graph as record nodes)
     stage_names = ["index_score", "topk_select", "csa_attn", "hca_attn"]
@@ -369,8 +380,7 @@ def run_ours(args, w, rank, world, dev):
         ev0[i].record(stream)
         q_dev.copy_(q_pin, non_blocking=True)
         qi_dev.copy_(qi_pin, non_blocking=True)
-        S.hybrid_attn_decode(q_dev.view(torch.bfloat16), qi_dev.view(torch.bfloat16), csa, hca, k, ws, scale=SCALE,
-                             out_csa=out_c, out_hca=out_h, lse_csa=lse_c, lse_hca=lse_h, idx_out=idx, cnt_out=cnt)
+        decode(q_dev.view(torch.bfloat16), qi_dev.view(torch.bfloat16))
         oc_pin.copy_(out_c.view(torch.int16), non_blocking=True)
         oh_pin.copy_(out_h.view(torch.int16), non_blocking=True)
         lc_pin.copy_(lse_c, non_blocking=True)
@@ -383,7 +393,7 @@ def run_ours(args, w, rank, world, dev):
     del graph, graph_staged, graph_score
 
     value = job_throughput(B * args.steps, world, total_ms)
-    step_bytes, score_bytes = decode_bytes(w, lengths)
+    step_bytes, score_bytes = decode_bytes(w, lengths, args.indexer)
     peak, peak_kind = measured_peaks()
     score_avg = statistics.mean(score_ms)
     achieved = score_bytes / (score_avg / 1e3) / 1e9
@@ -399,30 +409,34 @@ def run_ours(args, w, rank, world, dev):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16" if not w.fp8 else "fp8e4m3-kv/bf16",
+        "dtype": ("bf16" if not w.fp8 else "fp8e4m3-kv/bf16") + ("+mxfp4-indexer" if fp4 else ""),
         "data": "synthetic",
         "config": {"workload": w.name, "B_per_gpu": B, "context": int(w.L), "heads": H, "head_dim": 128,
                    "csa_m": w.m_csa, "topk": k, "hca_m": w.m_hca, "kv_dtype": "e4m3" if w.fp8 else "bf16",
+                   "indexer": args.indexer,
                    "parallelism": f"replicas x{world} (independent sequences)",
                    "l2": "flushed between timed steps: 512 MB written then read back (clean L2)", "launch": "CUDA graph replay"},
         "hbm": {"step_bytes": step_bytes, "step_gbs": step_gbs, "step_frac": step_gbs / peak,
                 "step_frac_of_8tbs": step_gbs / 8000.0},
-        "roofline": {"kernel": "score_decode_kernel", "bound": "hbm", "achieved": achieved, "peak": peak,
+        "roofline": {"kernel": "score_decode_mxfp4_kernel" if fp4 else "score_decode_kernel", "bound": "hbm",
+                     "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                      "bytes_per_launch": score_bytes, "avg_launch_ms": score_avg,
-                     "traffic": recorded_traffic("score_decode_kernel", w.name)},
+                     "traffic": None if fp4 else recorded_traffic("score_decode_kernel", w.name)},
         "stages_ms": {n: statistics.mean(v) for n, v in zip(stage_names, stage_ms)},
         "staged_step_ms": statistics.mean(staged_ms),
         "gpu_launches": launches_per_step * args.steps,
         "e2e": {"value": job_throughput(B * args.steps, world, e2e_total), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "api": "hybrid_attn_decode (eager) + pinned-host copies"},
+                "d2h_bytes_per_step": d2h,
+                "api": ("hybrid_attn_decode_mxfp4" if fp4 else "hybrid_attn_decode") + " (eager) + pinned-host copies"},
         "clocks": clk.summary(),
         "setup_s": round(time.time() - t_gen, 1),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"], cs = cpu_baseline(w, lengths, K, V, KI, q_h, qI_h, budget_s=args.cpu_budget)
+        result["cpu_baseline"], cs = cpu_baseline(w, lengths, K, V, KI, q_h, qI_h, budget_s=args.cpu_budget,
+                                                  indexer=args.indexer)
         result["cpu_baseline_all_cores"] = cpu_baseline_all_cores(w, lengths, K, V, KI, q_h, qI_h, cs=cs,
-                                                                  budget_s=args.cpu_budget / 2)
+                                                                  budget_s=args.cpu_budget / 2, indexer=args.indexer)
     return result
 
 
@@ -548,33 +562,45 @@ def run_prefill(args, w, rank, world, dev):
 
 # ----------------------------------------------------------- oracle (CPU) ---
 
-def oracle_decode_one(w, lengths, K, V, KI, q_h, qI_h, b):
+def oracle_query(w, cs, q, qI, t, indexer="bf16"):
+    """One decode query on the fp64 oracle: bf16 indexer scores, or FP4 ones
+    (the MXFP4 keys are built once per sequence, outside any timing)."""
+    from oracle import oracle as O
+    if indexer == "bf16":
+        return O.hybrid_query(cs, q, qI, t=t, k=w.topk, scale=SCALE)
+    if not hasattr(cs, "mx"):
+        cs.mx = O.mxfp4_quantize(cs.cidx)
+    return O.hybrid_query_mxfp4(cs, q, qI, t=t, k=w.topk, scale=SCALE, idx_codes=cs.mx[0], idx_scales=cs.mx[1])
+
+
+def oracle_decode_one(w, lengths, K, V, KI, q_h, qI_h, b, indexer="bf16"):
     """One decode token of sequence b on the fp64 oracle; returns (seconds, setup seconds)."""
     from oracle import oracle as O
     t0 = time.time()
     Lb = int(lengths[b])
     cs = O.CompressedSeq(K[b, :Lb], V[b, :Lb], KI[b, :Lb], m_csa=w.m_csa, m_hca=w.m_hca, fp8=w.fp8)
+    if indexer != "bf16":
+        cs.mx = O.mxfp4_quantize(cs.cidx)
     setup = time.time() - t0
     t1 = time.perf_counter()
-    O.hybrid_query(cs, q_h[b], qI_h[b], t=Lb, k=w.topk, scale=SCALE)
+    oracle_query(w, cs, q_h[b], qI_h[b], Lb, indexer)
     return time.perf_counter() - t1, setup, cs
 
 
-def cpu_baseline(w, lengths, K, V, KI, q_h, qI_h, budget_s=20.0):
-    from oracle import oracle as O
-    el, setup, cs = oracle_decode_one(w, lengths, K, V, KI, q_h, qI_h, 0)
+def cpu_baseline(w, lengths, K, V, KI, q_h, qI_h, budget_s=20.0, indexer="bf16"):
+    el, setup, cs = oracle_decode_one(w, lengths, K, V, KI, q_h, qI_h, 0, indexer)
     times = [el]
     t_end = time.time() + max(0.0, budget_s - el)
     while time.time() < t_end and len(times) < 8:
         t1 = time.perf_counter()
-        O.hybrid_query(cs, q_h[0], qI_h[0], t=int(lengths[0]), k=w.topk, scale=SCALE)
+        oracle_query(w, cs, q_h[0], qI_h[0], int(lengths[0]), indexer)
         times.append(time.perf_counter() - t1)
     return {"value": len(times) / sum(times), "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"{len(times)} decode token(s) of sequence 0 ({int(lengths[0])} tokens of context) on the "
                       f"single-threaded fp64 C oracle, caches pre-built by the oracle ({setup:.1f} s, untimed)"}, cs
 
 
-def cpu_baseline_all_cores(w, lengths, K, V, KI, q_h, qI_h, cs=None, budget_s=10.0):
+def cpu_baseline_all_cores(w, lengths, K, V, KI, q_h, qI_h, cs=None, budget_s=10.0, indexer="bf16"):
     """The same oracle on every host core: independent decode tokens of
     sequence 0 in parallel threads (the C oracle releases the GIL and keeps no
     shared state), tokens over wall time."""
@@ -586,8 +612,11 @@ def cpu_baseline_all_cores(w, lengths, K, V, KI, q_h, qI_h, cs=None, budget_s=10
         cs = O.CompressedSeq(K[0, :Lb], V[0, :Lb], KI[0, :Lb], m_csa=w.m_csa, m_hca=w.m_hca, fp8=w.fp8)
     cores = max(1, len(os.sched_getaffinity(0)))
 
+    if indexer != "bf16" and not hasattr(cs, "mx"):
+        cs.mx = O.mxfp4_quantize(cs.cidx)
+
     def one(_):
-        O.hybrid_query(cs, q_h[0], qI_h[0], t=int(lengths[0]), k=w.topk, scale=SCALE)
+        oracle_query(w, cs, q_h[0], qI_h[0], int(lengths[0]), indexer)
 
     with cf.ThreadPoolExecutor(cores) as ex:
         list(ex.map(one, range(cores)))  # warm-up round
@@ -651,8 +680,10 @@ def run_reference(args, w, rank, world):
         if b not in cs:
             Lb = int(lengths[b])
             cs[b] = O.CompressedSeq(K[b, :Lb], V[b, :Lb], KI[b, :Lb], m_csa=w.m_csa, m_hca=w.m_hca, fp8=w.fp8)
+            if args.indexer != "bf16":
+                cs[b].mx = O.mxfp4_quantize(cs[b].cidx)
         t1 = time.perf_counter()
-        O.hybrid_query(cs[b], q_h[b], qI_h[b], t=int(lengths[b]), k=w.topk, scale=SCALE)
+        oracle_query(w, cs[b], q_h[b], qI_h[b], int(lengths[b]), args.indexer)
         el = time.perf_counter() - t1
         if i >= args.warmup:
             times.append(el)
@@ -663,7 +694,8 @@ def run_reference(args, w, rank, world):
     return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total / len(times) * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": w.name, "B_per_gpu": w.B, "context": int(w.L), "heads": w.H, "topk": w.topk},
+            "config": {"workload": w.name, "B_per_gpu": w.B, "context": int(w.L), "heads": w.H, "topk": w.topk,
+                       "indexer": args.indexer},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -677,12 +709,16 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=[x.name for x in configs.WORKLOADS])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--indexer", default="bf16", choices=["bf16", "mxfp4"],
+                    help="decode only: the CSA indexer keys in bf16 (the workload) or FP4 (MXFP4)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="prefill only: a shorter sequence than the workload's (small cases for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = configs.BY_NAME[args.workload]
+    if args.indexer != "bf16" and w.mode != "decode":
+        ap.error("--indexer applies to decode workloads")
     if args.tokens:
         if w.mode != "prefill":
             ap.error("--tokens applies to prefill workloads")

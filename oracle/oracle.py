@@ -375,3 +375,22 @@ def lowp_query(K, V, KI, q, qI, t: int, k: int, scale: float, d_rope: int = 64, 
                             {"mode": "fp8", "data": vcodes, "scales": vsc}, idx[:cnt], scale, d_rope)
     return {"scores": s, "idx": idx, "cnt": cnt, "out": out, "lse": lse,
             "idx_codes": kc, "idx_scales": ks, "q_codes": qc[0], "q_scales": qs[0]}
+
+
+def hybrid_query_mxfp4(cs: CompressedSeq, q: np.ndarray, qI: np.ndarray, t: int, k: int, scale: float,
+                       idx_codes=None, idx_scales=None):
+    """O6 with the CSA selection on FP4 scores: the query and the compressed
+    indexer keys in MXFP4 (reading in the header of sa_oracle.c), top-k (O4),
+    then both attentions as in O6.  idx_codes / idx_scales: the keys' MXFP4
+    form when already built (mxfp4_quantize(cs.cidx)).  Returns a dict like
+    hybrid_query."""
+    if idx_codes is None:
+        idx_codes, idx_scales = mxfp4_quantize(cs.cidx)
+    qc, qs = mxfp4_quantize(np.asarray(qI, np.uint16).reshape(1, -1))
+    n_vis = min(int(t) // cs.m_csa, cs.n_csa)
+    s = mxfp4_index_scores(qc[0], qs[0], idx_codes[:n_vis], idx_scales[:n_vis])
+    idx, cnt = topk(s, k)
+    oc, lc = attention(q, cs.ck, cs.cv, idx[:cnt], scale, k_scales=cs.cks, v_scales=cs.cvs)
+    n_h = min(int(t) // cs.m_hca, cs.n_hca)
+    oh, lh = attention(q, cs.hk, cs.hv, np.arange(n_h, dtype=np.int32), scale, k_scales=cs.hks, v_scales=cs.hvs)
+    return {"idx": idx, "cnt": cnt, "out_csa": oc, "lse_csa": lc, "out_hca": oh, "lse_hca": lh}

@@ -22,7 +22,7 @@ EXPORTS = ["csa_compress", "hca_compress", "csa_index_topk", "csa_sparse_attn", 
            "hybrid_attn_decode", "hybrid_attn_prefill", "sa_workspace_size", "sa_read_device_status",
            "sa_last_error", "sa_abi_version", "sa_set_stage_events", "sa_launch_count",
            "csa_index_topk_noalloc", "csa_append", "hca_append", "swa_attn", "attn_lse_merge",
-           "csa_index_quantize_mxfp4", "csa_index_topk_mxfp4"]
+           "csa_index_quantize_mxfp4", "csa_index_topk_mxfp4", "hybrid_attn_decode_mxfp4"]
 SA_NOALLOC_SCRATCH_BYTES = 32 << 20
 SA_STAGE_INDEX_SCORE, SA_STAGE_TOPK_SELECT, SA_STAGE_CSA_ATTN, SA_STAGE_HCA_ATTN = 0, 1, 2, 3
 
@@ -73,6 +73,7 @@ def lib():
         L.csa_sparse_attn.argtypes = [P, I32, I32, CP, P, P, I32, F32, P, P, P, SZ, P]
         L.hca_dense_attn.argtypes = [P, I32, I32, P, CP, F32, P, P, P, SZ, P]
         L.hybrid_attn_decode.argtypes = [P, P, I32, CP, CP, I32, F32, P, P, P, P, P, P, P, SZ, P]
+        L.hybrid_attn_decode_mxfp4.argtypes = [P, P, I32, CP, CP, P, P, I32, F32, P, P, P, P, P, P, P, SZ, P]
         L.hybrid_attn_prefill.argtypes = [P, P, I32, I32, CP, CP, I32, F32, P, P, P, P, P, P, P, SZ, P]
         L.sa_workspace_size.argtypes = [I32, I32, I32, I32, I32, I32, I32]
         L.sa_workspace_size.restype = SZ

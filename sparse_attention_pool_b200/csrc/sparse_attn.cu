@@ -990,23 +990,31 @@ sa_status hca_dense_attn(const void* q, int32_t Tq, int32_t H, const int32_t* q_
                     static_cast<cudaStream_t>(stream));
 }
 
-sa_status hybrid_attn_decode(const void* q, const void* q_idx, int32_t H, const sa_cache* csa, const sa_cache* hca,
-                             int32_t k, float scale, void* out_csa, void* out_hca, float* lse_csa, float* lse_hca,
-                             int32_t* idx_out, int32_t* cnt_out, void* ws, size_t ws_bytes, void* stream) {
-    sa_status r = check_cache(csa, true, "hybrid_attn_decode(csa)");
+// One decode step of both branches; with MXFP4 indexer keys (codes4 /
+// scales4 non-NULL) the CSA selection runs on FP4 scores.
+static sa_status hybrid_decode_impl(const char* what, const void* q, const void* q_idx, int32_t H,
+                                    const sa_cache* csa, const sa_cache* hca, const uint8_t* codes4,
+                                    const uint8_t* scales4, int32_t k, float scale, void* out_csa, void* out_hca,
+                                    float* lse_csa, float* lse_hca, int32_t* idx_out, int32_t* cnt_out, void* ws,
+                                    size_t ws_bytes, void* stream) {
+    const bool fp4 = codes4 != nullptr || scales4 != nullptr;
+    sa_status r = check_cache(csa, !fp4, fp4 ? "hybrid_attn_decode_mxfp4(csa)" : "hybrid_attn_decode(csa)");
     if (r != SA_OK) return r;
-    r = check_cache(hca, false, "hybrid_attn_decode(hca)");
+    r = check_cache(hca, false, fp4 ? "hybrid_attn_decode_mxfp4(hca)" : "hybrid_attn_decode(hca)");
     if (r != SA_OK) return r;
-    r = check_common_q(q, H, "hybrid_attn_decode");
+    r = check_common_q(q, H, what);
     if (r != SA_OK) return r;
-    SA_CHECK(csa->B == hca->B, "hybrid_attn_decode: csa B=%d != hca B=%d", csa->B, hca->B);
-    SA_CHECK(q_idx && aligned16(q_idx), "hybrid_attn_decode: q_idx must be non-NULL and aligned");
-    SA_CHECK(k >= 1 && k <= 65536, "hybrid_attn_decode: k=%d outside 1..65536", k);
-    SA_CHECK(out_csa && out_hca && aligned16(out_csa) && aligned16(out_hca), "hybrid_attn_decode: outputs must be aligned");
-    SA_CHECK((!lse_csa || aligned16(lse_csa)) && (!lse_hca || aligned16(lse_hca)), "hybrid_attn_decode: lse alignment");
-    SA_CHECK((idx_out == nullptr) == (cnt_out == nullptr), "hybrid_attn_decode: give both idx_out and cnt_out or neither");
-    SA_CHECK((!idx_out || aligned16(idx_out)) && (!cnt_out || aligned16(cnt_out)), "hybrid_attn_decode: idx/cnt alignment");
-    SA_CHECK(std::isfinite(scale) && scale >= 0.f, "hybrid_attn_decode: scale must be finite and >= 0");
+    if (fp4)
+        SA_CHECK(codes4 && scales4 && aligned16(codes4) && aligned16(scales4),
+                 "%s: codes and scales must be non-NULL and 16-byte aligned", what);
+    SA_CHECK(csa->B == hca->B, "%s: csa B=%d != hca B=%d", what, csa->B, hca->B);
+    SA_CHECK(q_idx && aligned16(q_idx), "%s: q_idx must be non-NULL and aligned", what);
+    SA_CHECK(k >= 1 && k <= 65536, "%s: k=%d outside 1..65536", what, k);
+    SA_CHECK(out_csa && out_hca && aligned16(out_csa) && aligned16(out_hca), "%s: outputs must be aligned", what);
+    SA_CHECK((!lse_csa || aligned16(lse_csa)) && (!lse_hca || aligned16(lse_hca)), "%s: lse alignment", what);
+    SA_CHECK((idx_out == nullptr) == (cnt_out == nullptr), "%s: give both idx_out and cnt_out or neither", what);
+    SA_CHECK((!idx_out || aligned16(idx_out)) && (!cnt_out || aligned16(cnt_out)), "%s: idx/cnt alignment", what);
+    SA_CHECK(std::isfinite(scale) && scale >= 0.f, "%s: scale must be finite and >= 0", what);
     const size_t need = sa_workspace_size(SA_OP_HYBRID_DECODE, csa->B, 1, H, csa->Ncap, hca->Ncap, k);
     r = check_ws(ws, ws_bytes, need);
     if (r != SA_OK) return r;
@@ -1034,7 +1042,7 @@ sa_status hybrid_attn_decode(const void* q, const void* q_idx, int32_t H, const 
         SA_CUDA(cudaEventRecord(side->join, side->s));
         return SA_OK;
     };
-    r = run_topk_decode(q_idx, csa, k, idx, cnt, ws, w, st, fork_hca);
+    r = run_topk_decode(q_idx, csa, k, idx, cnt, ws, w, st, fork_hca, codes4, scales4);
     if (r != SA_OK) return r;
     stage_mark(SA_STAGE_CSA_ATTN, 0, st);
     r = run_attn(q, 1, H, csa, true, idx, cnt, k, nullptr, scale, out_csa, lse_csa, ws, w.total, st, true);
@@ -1042,6 +1050,22 @@ sa_status hybrid_attn_decode(const void* q, const void* q_idx, int32_t H, const 
     stage_mark(SA_STAGE_CSA_ATTN, 1, st);
     SA_CUDA(cudaStreamWaitEvent(st, side->join, 0));
     return SA_OK;
+}
+
+sa_status hybrid_attn_decode(const void* q, const void* q_idx, int32_t H, const sa_cache* csa, const sa_cache* hca,
+                             int32_t k, float scale, void* out_csa, void* out_hca, float* lse_csa, float* lse_hca,
+                             int32_t* idx_out, int32_t* cnt_out, void* ws, size_t ws_bytes, void* stream) {
+    return hybrid_decode_impl("hybrid_attn_decode", q, q_idx, H, csa, hca, nullptr, nullptr, k, scale, out_csa,
+                              out_hca, lse_csa, lse_hca, idx_out, cnt_out, ws, ws_bytes, stream);
+}
+
+sa_status hybrid_attn_decode_mxfp4(const void* q, const void* q_idx, int32_t H, const sa_cache* csa,
+                                   const sa_cache* hca, const uint8_t* codes, const uint8_t* scales, int32_t k,
+                                   float scale, void* out_csa, void* out_hca, float* lse_csa, float* lse_hca,
+                                   int32_t* idx_out, int32_t* cnt_out, void* ws, size_t ws_bytes, void* stream) {
+    SA_CHECK(codes && scales, "hybrid_attn_decode_mxfp4: codes and scales must be non-NULL");
+    return hybrid_decode_impl("hybrid_attn_decode_mxfp4", q, q_idx, H, csa, hca, codes, scales, k, scale, out_csa,
+                              out_hca, lse_csa, lse_hca, idx_out, cnt_out, ws, ws_bytes, stream);
 }
 
 sa_status hybrid_attn_prefill(const void* q, const void* q_idx, int32_t T, int32_t H, const sa_cache* csa,

@@ -176,3 +176,23 @@ def test_mxfp4_entry_points_reject_bad_arguments(L):
     assert t(P(FAKE), ctypes.byref(c), None, P(FAKE), 8, P(FAKE), P(FAKE), P(FAKE), 1 << 30, None) == 1
     st = t(P(FAKE), ctypes.byref(c), P(FAKE), P(FAKE), 8, P(FAKE), P(FAKE), P(FAKE), 16, None)
     assert st == _lib.SA_ERR_WORKSPACE
+
+
+def test_hybrid_decode_mxfp4_rejects_bad_arguments(L):
+    c, h = _cache(kidx=None), _cache(m=128, kidx=None)
+    P = ctypes.c_void_p
+    f = L.hybrid_attn_decode_mxfp4
+    args = [P(FAKE), P(FAKE), 8, ctypes.byref(c), ctypes.byref(h)]
+    rest = [8, 0.0, P(FAKE), P(FAKE), None, None, None, None, P(FAKE), 1 << 30, None]
+    assert f(*args, None, P(FAKE), *rest) == 1
+    assert "codes" in L.sa_last_error().decode()
+    assert f(*args, P(FAKE + 4), P(FAKE), *rest) == 1
+    assert "aligned" in L.sa_last_error().decode()
+    h2 = _cache(m=128, kidx=None, B=2)
+    assert f(P(FAKE), P(FAKE), 8, ctypes.byref(c), ctypes.byref(h2), P(FAKE), P(FAKE), *rest) == 1
+    assert "B=" in L.sa_last_error().decode()
+    small = [8, 0.0, P(FAKE), P(FAKE), None, None, None, None, P(FAKE), 16, None]
+    assert f(*args, P(FAKE), P(FAKE), *small) == _lib.SA_ERR_WORKSPACE
+    # the bf16 entry point still needs the bf16 indexer keys
+    assert L.hybrid_attn_decode(P(FAKE), P(FAKE), 8, ctypes.byref(c), ctypes.byref(h), *rest) == 1
+    assert "kidx" in L.sa_last_error().decode()

@@ -47,3 +47,16 @@ def test_fp8_step_bytes_term_by_term():
 def test_job_throughput_counts_every_rank():
     assert bench.job_throughput(units_per_rank=40, world=1, max_ms=10.0) == 4000.0
     assert bench.job_throughput(units_per_rank=40, world=8, max_ms=10.0) == 32000.0
+
+
+def test_mxfp4_indexer_bytes():
+    """With MXFP4 indexer keys an entry's key is 32 bytes of e2m1 codes plus 2
+    E8M0 scale bytes instead of 128 bytes of bf16; nothing else changes."""
+    w = configs.BY_NAME["decode_b4_t1m_h64_k2048"]
+    lengths = np.full((w.B,), w.L)
+    step16, score16 = bench.decode_bytes(w, lengths)
+    step4, score4 = bench.decode_bytes(w, lengths, "mxfp4")
+    nc = w.L // 4
+    assert score4 == w.B * nc * (34 + 4) == 39_845_888
+    assert step16 - step4 == w.B * nc * (128 - 34)
+    assert step4 == 56_820_224

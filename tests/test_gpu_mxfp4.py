@@ -135,3 +135,26 @@ def test_topk_full_size_decode(S):
     for b in range(B):
         ref, rc = _oracle_topk(qI[b], bits[b], Ncap, k)
         assert rc == k and np.array_equal(gi[b], ref), b
+
+
+def test_hybrid_decode_mxfp4_matches_oracle(S):
+    """One decode step of both branches with the CSA selection on FP4 scores:
+    indices bit for bit, outputs within the bf16 tolerance."""
+    from tests._util import SCALE, TOL_BF16, Inputs, compress_on_gpu
+    B, Lcap, H, k = 3, 6000, 64, 256
+    inp = Inputs(75, B, Lcap, H, lengths=[6000, 3001, 700])
+    g = inp.to_device()
+    csa, hca = compress_on_gpu(S, g, B, Lcap)
+    codes, scales = S.csa_index_quantize_mxfp4(csa)
+    ws = S.alloc_workspace(S.workspace_size(S.SA_OP_HYBRID_DECODE, B, 1, H, csa.Ncap, hca.Ncap, k))
+    idx = torch.empty(B, k, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(B, dtype=torch.int32, device="cuda")
+    oc, oh = S.hybrid_attn_decode_mxfp4(g["q"], g["qI"], csa, hca, codes, scales, k, ws, scale=SCALE,
+                                        idx_out=idx, cnt_out=cnt)
+    S.read_device_status()
+    for b in range(B):
+        L = int(inp.lengths[b])
+        r = O.hybrid_query_mxfp4(inp.oracle_seq(b), inp.q[b], inp.qI[b], t=L, k=k, scale=SCALE)
+        assert int(cnt[b]) == r["cnt"] and np.array_equal(idx[b].cpu().numpy(), r["idx"]), b
+        assert np.abs(oc[b].float().cpu().numpy() - r["out_csa"]).max() <= TOL_BF16, b
+        assert np.abs(oh[b].float().cpu().numpy() - r["out_hca"]).max() <= TOL_BF16, b

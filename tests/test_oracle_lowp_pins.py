@@ -321,3 +321,28 @@ def test_planted_mistakes_are_caught(mistake):
             c = (codes[j, e // 2] >> (4 * (e % 2))) & 0xF
             bad += c != _brute_e2m1(xd[j, e] / X)
     assert bad > 0
+
+
+def test_hybrid_query_mxfp4_composition():
+    """The FP4 hybrid query is the pinned pieces composed: its HCA half is the
+    bf16 hybrid query's (HCA has no indexer), its CSA half the attention over
+    the top-k of the FP4 scores."""
+    rng = np.random.default_rng(51)
+    L, k, H = 3000, 64, 4
+
+    def bits(shape):
+        return (rng.standard_normal(shape).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    K, V, KI, q, qI = bits((L, 128)), bits((L, 128)), bits((L, 64)), bits((H, 128)), bits(64)
+    cs = O.CompressedSeq(K, V, KI)
+    sc = 128 ** -0.5
+    r4 = O.hybrid_query_mxfp4(cs, q, qI, t=L - 1, k=k, scale=sc)
+    r16 = O.hybrid_query(cs, q, qI, t=L - 1, k=k, scale=sc)
+    assert np.array_equal(r4["out_hca"], r16["out_hca"]) and np.array_equal(r4["lse_hca"], r16["lse_hca"])
+    kc, ks = O.mxfp4_quantize(cs.cidx)
+    qc, qs = O.mxfp4_quantize(qI.reshape(1, -1))
+    n_vis = (L - 1) // 4
+    idx, cnt = O.topk(O.mxfp4_index_scores(qc[0], qs[0], kc[:n_vis], ks[:n_vis]), k)
+    assert cnt == r4["cnt"] == k and np.array_equal(idx, r4["idx"])
+    o, lse = O.attention(q, cs.ck, cs.cv, idx, sc)
+    assert np.array_equal(o, r4["out_csa"]) and np.array_equal(lse, r4["lse_csa"])
+    assert len(set(idx.tolist()) & set(r16["idx"].tolist())) > k // 2  # FP4 keeps most of the bf16 selection
