@@ -70,7 +70,18 @@ typedef enum {
     SA_ERR_DEVICE = 6        /* device status: a length exceeded its capacity, ... */
 } sa_status;
 
-typedef enum { SA_BF16 = 0, SA_FP8_E4M3 = 1 } sa_kv_dtype;
+/* Storage of the compressed K and V ("Mixed KV storage" row of the review's
+ * section 3-2 (2) table: rotary dims in BF16, the rest in FP8).
+ *   SA_BF16:     K, V [B][Ncap][d] bf16.
+ *   SA_FP8_E4M3: K, V [B][Ncap][d] e4m3 codes; k_scale / v_scale
+ *                [B][ceil(Ncap/64)] fp32, one per 64 consecutive entries,
+ *                scale = fp32(amax / 448) (1 when amax == 0).
+ *   SA_KV_MIXED: K [B][Ncap][192] bytes per entry: dims 0..63 as e4m3 codes
+ *                (bytes 0..63) then the rotary dims 64..127 as bf16 (bytes
+ *                64..191); k_scale over dims 0..63 only.  V as SA_FP8_E4M3.
+ *                The page gives no rotary width; the last 64 of the 128 dims
+ *                is the reading taken here.                                   */
+typedef enum { SA_BF16 = 0, SA_FP8_E4M3 = 1, SA_KV_MIXED = 2 } sa_kv_dtype;
 
 /* Raw (uncompressed) tokens of B sequences, padded to Lcap tokens each. */
 typedef struct {
@@ -83,9 +94,9 @@ typedef struct {
 
 /* A compressed cache (CSA: m = 4 with indexer keys; HCA: m = 128 without). */
 typedef struct {
-    void* k;               /* [B][Ncap][d] bf16, or e4m3 codes                     */
+    void* k;               /* [B][Ncap][d] bf16 or e4m3, or [B][Ncap][192] mixed    */
     void* v;               /* [B][Ncap][d] bf16, or e4m3 codes                     */
-    float* k_scale;        /* [B][ceil(Ncap/64)] fp32 when dtype == SA_FP8_E4M3     */
+    float* k_scale;        /* [B][ceil(Ncap/64)] fp32 unless dtype == SA_BF16       */
     float* v_scale;        /* same for v; both NULL for bf16                        */
     void* kidx;            /* [B][Ncap][d_idx] bf16 (needed by the CSA indexer)     */
     int32_t* n;            /* device [B]: complete entries per sequence             */

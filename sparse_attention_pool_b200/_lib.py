@@ -10,7 +10,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libsparse_attn.so")
 
 SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_CUDA, SA_ERR_TIMEOUT, SA_ERR_DEVICE = range(7)
-SA_BF16, SA_FP8_E4M3 = 0, 1
+SA_BF16, SA_FP8_E4M3, SA_KV_MIXED = 0, 1, 2
 SA_OP_INDEX_TOPK, SA_OP_SPARSE_ATTN, SA_OP_DENSE_ATTN, SA_OP_HYBRID_DECODE, SA_OP_HYBRID_PREFILL = 1, 2, 3, 4, 5
 SA_OP_WINDOW_ATTN = 6
 

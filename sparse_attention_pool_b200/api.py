@@ -16,6 +16,7 @@ from . import _lib
 from ._lib import SaCache, SaRaw, check, lib
 
 D, D_IDX = 128, 64
+MIXED_K_ROW = 192  # bytes of a mixed-storage K row
 
 
 def _ptr(t):
@@ -58,20 +59,29 @@ class Cache:
 
     @property
     def fp8(self):
+        """e4m3 storage (with per-64-entry scales), plain or mixed."""
         return self.k.dtype == torch.uint8
 
+    @property
+    def mixed(self):
+        """Mixed storage: K rows of 192 bytes (64 e4m3 codes, then the 64 rotary
+        dims in bf16), V in e4m3."""
+        return self.k.dtype == torch.uint8 and self.k.shape[2] == MIXED_K_ROW
+
     def struct(self) -> SaCache:
+        dtype = _lib.SA_KV_MIXED if self.mixed else _lib.SA_FP8_E4M3 if self.fp8 else _lib.SA_BF16
         return SaCache(_ptr(self.k), _ptr(self.v), _ptr(self.k_scale), _ptr(self.v_scale), _ptr(self.kidx),
-                       _ptr(self.n), self.B, self.Ncap, D, D_IDX, self.m,
-                       _lib.SA_FP8_E4M3 if self.fp8 else _lib.SA_BF16)
+                       _ptr(self.n), self.B, self.Ncap, D, D_IDX, self.m, dtype)
 
 
-def alloc_cache(B: int, Ncap: int, m: int, *, fp8: bool = False, with_kidx: bool = False,
+def alloc_cache(B: int, Ncap: int, m: int, *, fp8: bool = False, with_kidx: bool = False, mixed: bool = False,
                 device="cuda") -> Cache:
+    """A zeroed cache: bf16, e4m3 (fp8=True) or mixed storage (mixed=True)."""
+    fp8 = fp8 or mixed
     kv_dtype = torch.uint8 if fp8 else torch.bfloat16
     nG = (Ncap + 63) // 64
     return Cache(
-        k=torch.zeros(B, Ncap, D, dtype=kv_dtype, device=device),
+        k=torch.zeros(B, Ncap, MIXED_K_ROW if mixed else D, dtype=kv_dtype, device=device),
         v=torch.zeros(B, Ncap, D, dtype=kv_dtype, device=device),
         n=torch.zeros(B, dtype=torch.int32, device=device),
         m=m,

@@ -15,7 +15,10 @@
 // only the last `win` visible rows: the sliding-window branch over raw
 // tokens.  An fp8 cache is widened to bf16 in shared memory
 // (every e4m3 value is exact in bf16); its per-64-entry scales multiply the S
-// columns (K) and the P columns (V) in fp32.  With one split the CTA writes
+// columns (K) and the P columns (V) in fp32.  A mixed cache (MIXED) keeps K's
+// rotary dims 64..127 in bf16 after its 64 e4m3 codes (192-byte rows): the
+// QK^T product runs over the widened e4m3 dims first, their S columns are
+// scaled, and the bf16 dims then accumulate on top; V is e4m3.  With one split the CTA writes
 // the bf16 output directly; otherwise it writes a normalised fp32 partial and
 // its lse, merged by attn_combine_kernel in a fixed order (deterministic and
 // independent of the batch: the split size depends only on the entry count).
@@ -70,14 +73,18 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-template <int NW, bool GATHER, bool FP8, int ST>
+constexpr int kMixedKRow = 192;  // mixed K row: 64 e4m3 codes, then 64 bf16 rotary dims
+
+template <int NW, bool GATHER, bool FP8, int ST, bool MIXED = false>
 struct AttnSmem {
     static constexpr int kQBytes = NW * 16 * 256;
     static constexpr int kKVBytes = kTileN * 256;                 // one bf16 tile
-    static constexpr int kStageRaw = FP8 ? kTileN * 128 : kKVBytes;  // one raw tile (K or V)
+    static constexpr int kStageRaw = FP8 ? kTileN * 128 : kKVBytes;  // one raw tile (V, and K unless mixed)
+    static constexpr int kStageRawK = MIXED ? kTileN * kMixedKRow : kStageRaw;  // one raw K tile
+    static constexpr int kStagePair = kStageRawK + kStageRaw;
     static constexpr int kQ = 0;
     static constexpr int kRaw = kQ + kQBytes;                      // [ST stages][K, V] raw tiles
-    static constexpr int kConv = kRaw + ST * 2 * kStageRaw;        // fp8: widened K, V tiles
+    static constexpr int kConv = kRaw + ST * kStagePair;           // fp8: widened K, V tiles
     static constexpr int kMeta = kConv + (FP8 ? 2 * kKVBytes : 0);  // [ST][64] valid + (fp8) scales
     static constexpr int kTotal = kMeta + ST * kTileN * 4 * 3;
 };
@@ -88,9 +95,10 @@ constexpr int kAttnCluster = 8;  // splits of one query merged in shared memory 
 // CLUSTER: the grid's x dimension is one cluster of kAttnCluster CTAs (the
 // splits of one query); they merge their partials through distributed shared
 // memory instead of a separate combine pass.
-template <int NW, bool GATHER, bool FP8, int ST, bool CLUSTER, int EG>
+template <int NW, bool GATHER, bool FP8, int ST, bool CLUSTER, int EG, bool MIXED = false>
 __global__ void __launch_bounds__(NW * EG * 32) attn_split_kernel(AttnArgs a) {
-    using L = AttnSmem<NW, GATHER, FP8, ST>;
+    using L = AttnSmem<NW, GATHER, FP8, ST, MIXED>;
+    static_assert(!MIXED || FP8, "a mixed cache is widened like an e4m3 one");
     constexpr int NT = NW * EG * 32;  // threads
     constexpr int EPW = kTileN / EG;  // entries of a tile per warp
     constexpr int NJ = EPW / 8;       // 8-entry n-tiles per warp
@@ -173,8 +181,8 @@ __global__ void __launch_bounds__(NW * EG * 32) attn_split_kernel(AttnArgs a) {
     static_assert(TPR >= 1 && CPT >= 1 && CPT * TPR == cpr, "tile mapping");
     auto load_tile = [&](int tile, int stage, int jv, bool have_j) {
         const int p0 = p_begin + tile * kTileN;
-        uint8_t* rk = sRaw + (stage * 2 + 0) * L::kStageRaw;
-        uint8_t* rv = sRaw + (stage * 2 + 1) * L::kStageRaw;
+        uint8_t* rk = sRaw + stage * L::kStagePair;
+        uint8_t* rv = rk + L::kStageRawK;
         const int r = tid / TPR, c0 = (tid % TPR) * CPT;
         const int p = p0 + r;
         int j = rbase + p;
@@ -191,8 +199,13 @@ __global__ void __launch_bounds__(NW * EG * 32) attn_split_kernel(AttnArgs a) {
         for (int c = 0; c < CPT; ++c) {
             const int ch = c0 + c;
             const uint32_t doff = FP8 ? (uint32_t)(r * 128 + ch * 16) : swz(r, ch);
-            cp_async16_zfill(rk + doff, Kb + rowOff + ch * 16, ok);
+            if (!MIXED) cp_async16_zfill(rk + doff, Kb + rowOff + ch * 16, ok);
             cp_async16_zfill(rv + doff, Vb + rowOff + ch * 16, ok);
+        }
+        if (MIXED) {  // 12 chunks of a 192-byte K row, TPR threads per row
+            const size_t rowOffK = ((size_t)b * a.Ncap + (size_t)(ok ? j : 0)) * kMixedKRow;
+            for (int ch = tid % TPR; ch < kMixedKRow / 16; ch += TPR)
+                cp_async16_zfill(rk + r * kMixedKRow + ch * 16, Kb + rowOffK + ch * 16, ok);
         }
         if (c0 == 0) {
             sValid[stage * kTileN + r] = ok;
@@ -237,13 +250,15 @@ __global__ void __launch_bounds__(NW * EG * 32) attn_split_kernel(AttnArgs a) {
         const uint8_t* tv;
         if (FP8) {
             // widen e4m3 codes to bf16 (exact), into swizzled tiles
-            const uint8_t* rk = sRaw + (stage * 2 + 0) * L::kStageRaw;
-            const uint8_t* rv = sRaw + (stage * 2 + 1) * L::kStageRaw;
+            const uint8_t* rk = sRaw + stage * L::kStagePair;
+            const uint8_t* rv = rk + L::kStageRawK;
             uint8_t* ck = sConv;
             uint8_t* cv = sConv + L::kKVBytes;
             for (int c = tid; c < kTileN * 16; c += NT) {  // 8 codes -> one 16-byte bf16 chunk
                 const int r = c >> 4, ch = c & 15;
-                const uint2 wk = *reinterpret_cast<const uint2*>(rk + r * 128 + ch * 8);
+                const uint2 wk = MIXED ? (ch < 8 ? *reinterpret_cast<const uint2*>(rk + r * kMixedKRow + ch * 8)
+                                                 : make_uint2(0u, 0u))
+                                       : *reinterpret_cast<const uint2*>(rk + r * 128 + ch * 8);
                 const uint2 wv = *reinterpret_cast<const uint2*>(rv + r * 128 + ch * 8);
                 uint4 ok4, ov4;
                 uint32_t* okp = &ok4.x;
@@ -258,6 +273,8 @@ __global__ void __launch_bounds__(NW * EG * 32) attn_split_kernel(AttnArgs a) {
                         ovp[h * 2 + e] = pack_bf16x2(e4m3_to_f32((vw[h] >> (16 * e)) & 0xFF),
                                                      e4m3_to_f32((vw[h] >> (16 * e + 8)) & 0xFF));
                     }
+                if (MIXED && ch >= 8)  // rotary dims: already bf16
+                    ok4 = *reinterpret_cast<const uint4*>(rk + r * kMixedKRow + 64 + (ch - 8) * 16);
                 *reinterpret_cast<uint4*>(ck + swz(r, ch)) = ok4;
                 *reinterpret_cast<uint4*>(cv + swz(r, ch)) = ov4;
             }
@@ -265,8 +282,8 @@ __global__ void __launch_bounds__(NW * EG * 32) attn_split_kernel(AttnArgs a) {
             tk = ck;
             tv = cv;
         } else {
-            tk = sRaw + (stage * 2 + 0) * L::kStageRaw;
-            tv = sRaw + (stage * 2 + 1) * L::kStageRaw;
+            tk = sRaw + stage * L::kStagePair;
+            tv = tk + L::kStageRawK;
         }
 
         // S = Q K^T : 16 heads x EPW entries per warp
@@ -276,6 +293,13 @@ __global__ void __launch_bounds__(NW * EG * 32) attn_split_kernel(AttnArgs a) {
         const uint32_t kbase = smem_u32(tk);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
+            if (MIXED && kk == 4) {  // dims 0..63 (e4m3) done: scale them before the bf16 dims add in
+#pragma unroll
+                for (int j = 0; j < NJ; ++j)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        s[j][e] *= sKs[stage * kTileN + eg * EPW + j * 8 + (lane & 3) * 2 + (e & 1)];
+            }
 #pragma unroll
             for (int np = 0; np < NJ / 2; ++np) {  // pairs of 8-entry n-tiles
                 const int r = eg * EPW + np * 16 + (lane & 7) + ((lane >> 4) << 3);
@@ -295,7 +319,7 @@ __global__ void __launch_bounds__(NW * EG * 32) attn_split_kernel(AttnArgs a) {
             for (int e = 0; e < 4; ++e) {
                 const int col = eg * EPW + j * 8 + (lane & 3) * 2 + (e & 1);
                 float v = s[j][e];
-                if (FP8) v *= sKs[stage * kTileN + col];
+                if (FP8 && !MIXED) v *= sKs[stage * kTileN + col];
                 v = valid[col] ? v * a.scale_log2 : -INFINITY;
                 s[j][e] = v;
                 tmax[e >> 1] = fmaxf(tmax[e >> 1], v);

@@ -11,6 +11,10 @@
 // group holding the first new entry and the groups after it are computed;
 // the result is bit-identical to compressing the whole sequence again.
 //
+// Mixed storage (MIXED): K keeps its rotary dims 64..127 in bf16 and stores
+// dims 0..63 as e4m3, in one 192-byte row per entry (codes, then the bf16
+// dims); the group scale of K covers dims 0..63 only.  V is stored as e4m3.
+//
 // One CTA compresses one group of 64 entries of one sequence for every tensor
 // (k, v and optionally the indexer keys).  Each thread owns one 16-byte chunk
 // (8 dims) of one entry and streams the m tokens of its block; the sums run in
@@ -46,6 +50,10 @@ __device__ __forceinline__ void acc8(double (&a)[8], const uint4 w) {
     a[7] += bf16hi_scaled(w.w);
 }
 
+constexpr int kMixedRowBytes = 192;  // mixed K row: 64 e4m3 codes + 64 bf16 rotary dims
+constexpr int kMixedFp8Chunks = 8;   // 16-byte bf16 chunks of K (8 dims each) stored as e4m3
+
+template <bool MIXED>
 __global__ void __launch_bounds__(kCompThreads) compress_kernel(CompressArgs a) {
     __shared__ __align__(16) uint16_t stage[64 * 128];  // bf16 entries of one fp8 group
     __shared__ float red[kCompThreads / 32];
@@ -78,6 +86,7 @@ __global__ void __launch_bounds__(kCompThreads) compress_kernel(CompressArgs a) 
         const int D = a.dims[t];
         const int cpe = D / 8;  // 16-byte chunks per entry
         const bool to_fp8 = a.fp8 && t < 2;
+        const bool mixed_k = MIXED && t == 0;  // rotary chunks c >= 8 stay bf16
         const uint4* src = reinterpret_cast<const uint4*>(a.src[t]) + (size_t)b * a.Lcap * cpe;
         float amax = 0.f;
         for (int task = threadIdx.x; task < ne * cpe; task += blockDim.x) {
@@ -107,6 +116,9 @@ __global__ void __launch_bounds__(kCompThreads) compress_kernel(CompressArgs a) 
             if (!to_fp8) {
                 uint4* dst = reinterpret_cast<uint4*>(a.dst[t]) + ((size_t)b * a.Ncap + e) * cpe + c;
                 *dst = make_uint4(r[0], r[1], r[2], r[3]);
+            } else if (mixed_k && c >= kMixedFp8Chunks) {
+                uint8_t* row = reinterpret_cast<uint8_t*>(a.dst[t]) + ((size_t)b * a.Ncap + e) * kMixedRowBytes;
+                *reinterpret_cast<uint4*>(row + 64 + (c - kMixedFp8Chunks) * 16) = make_uint4(r[0], r[1], r[2], r[3]);
             } else {
                 *reinterpret_cast<uint4*>(&stage[el * 128 + c * 8]) = make_uint4(r[0], r[1], r[2], r[3]);
 #pragma unroll
@@ -124,8 +136,9 @@ __global__ void __launch_bounds__(kCompThreads) compress_kernel(CompressArgs a) 
             for (int w = 0; w < (int)(blockDim.x >> 5); ++w) gmax = fmaxf(gmax, red[w]);
             const float s = (gmax == 0.f) ? 1.0f : __fdiv_rn(gmax, 448.0f);
             if (threadIdx.x == 0) a.scale[t][(size_t)b * a.nG + g] = s;
-            for (int task = threadIdx.x; task < ne * cpe; task += blockDim.x) {
-                const int el = task / cpe, c = task - el * cpe;
+            const int qcpe = mixed_k ? kMixedFp8Chunks : cpe;  // chunks stored as e4m3
+            for (int task = threadIdx.x; task < ne * qcpe; task += blockDim.x) {
+                const int el = task / qcpe, c = task - el * qcpe;
                 const uint4 w = *reinterpret_cast<const uint4*>(&stage[el * 128 + c * 8]);
                 const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
                 uint32_t codes[2];
@@ -137,8 +150,9 @@ __global__ void __launch_bounds__(kCompThreads) compress_kernel(CompressArgs a) 
                                                          __fdiv_rn(bf16hi_f32(ws[2 * h + 1]), s));
                     codes[h] = c01 | (c23 << 16);
                 }
+                const int rowBytes = mixed_k ? kMixedRowBytes : D;
                 uint2* dst = reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(a.dst[t]) +
-                                                      ((size_t)b * a.Ncap + e0 + el) * D + c * 8);
+                                                      ((size_t)b * a.Ncap + e0 + el) * rowBytes + c * 8);
                 *dst = make_uint2(codes[0], codes[1]);
             }
             __syncthreads();  // `stage` and `red` are reused by the next tensor

@@ -146,10 +146,11 @@ sa_status check_cache(const sa_cache* c, bool need_kidx, const char* what) {
     SA_CHECK(c->d == 128, "%s: head dim d=%d (only 128 is supported)", what, c->d);
     SA_CHECK(c->m >= 1 && c->m <= 1024 && (c->m & (c->m - 1)) == 0, "%s: m=%d is not a power of two in 1..1024",
              what, c->m);
-    SA_CHECK(c->dtype == SA_BF16 || c->dtype == SA_FP8_E4M3, "%s: dtype=%d", what, c->dtype);
+    SA_CHECK(c->dtype == SA_BF16 || c->dtype == SA_FP8_E4M3 || c->dtype == SA_KV_MIXED, "%s: dtype=%d", what,
+             c->dtype);
     SA_CHECK(c->k && c->v && c->n, "%s: k, v and n must be non-NULL", what);
     SA_CHECK(aligned16(c->k) && aligned16(c->v) && aligned16(c->n), "%s: k, v, n must be 16-byte aligned", what);
-    if (c->dtype == SA_FP8_E4M3) {
+    if (c->dtype != SA_BF16) {
         SA_CHECK(c->k_scale && c->v_scale, "%s: fp8 cache needs k_scale and v_scale", what);
         SA_CHECK(aligned16(c->k_scale) && aligned16(c->v_scale), "%s: scales must be 16-byte aligned", what);
     }
@@ -296,28 +297,32 @@ size_t attn_partial_bytes(long long BQ, int splits, int H) {
 }
 
 // ------------------------------------------------------------ launchers ----
-template <int NW, bool G, bool F, int ST, bool CL, int EG>
+template <int NW, bool G, bool F, int ST, bool CL, int EG, bool MX = false>
 sa_status launch_attn_t(const sa::AttnArgs& a, dim3 grid, cudaStream_t st, bool pdl) {
-    using L = sa::AttnSmem<NW, G, F, ST>;
+    using L = sa::AttnSmem<NW, G, F, ST, MX>;
     static std::atomic<uint64_t> init{0};
     if (!attr_done(init)) {
-        SA_CUDA(cudaFuncSetAttribute(sa::attn_split_kernel<NW, G, F, ST, CL, EG>,
+        SA_CUDA(cudaFuncSetAttribute(sa::attn_split_kernel<NW, G, F, ST, CL, EG, MX>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal));
         attr_set(init);
     }
-    SA_CUDA(launch_k(sa::attn_split_kernel<NW, G, F, ST, CL, EG>, grid, dim3(NW * EG * 32), L::kTotal, st, pdl,
+    SA_CUDA(launch_k(sa::attn_split_kernel<NW, G, F, ST, CL, EG, MX>, grid, dim3(NW * EG * 32), L::kTotal, st, pdl,
                      CL ? (unsigned)sa::kAttnCluster : 1u, a));
     SA_LAUNCHED();
     return SA_OK;
 }
 
+// kv: 0 = bf16 cache, 1 = e4m3 K and V, 2 = mixed K (e4m3 + bf16 rotary dims) and e4m3 V.
 template <int NW, int ST, bool CL, int EG>
-sa_status launch_attn_nw(const sa::AttnArgs& a, bool gather, bool fp8, dim3 grid, cudaStream_t st, bool pdl) {
-    if (gather)
-        return fp8 ? launch_attn_t<NW, true, true, ST, CL, EG>(a, grid, st, pdl)
-                   : launch_attn_t<NW, true, false, ST, CL, EG>(a, grid, st, pdl);
-    return fp8 ? launch_attn_t<NW, false, true, ST, CL, EG>(a, grid, st, pdl)
-               : launch_attn_t<NW, false, false, ST, CL, EG>(a, grid, st, pdl);
+sa_status launch_attn_nw(const sa::AttnArgs& a, bool gather, int kv, dim3 grid, cudaStream_t st, bool pdl) {
+    if (gather) {
+        if (kv == 2) return launch_attn_t<NW, true, true, ST, CL, EG, true>(a, grid, st, pdl);
+        return kv == 1 ? launch_attn_t<NW, true, true, ST, CL, EG>(a, grid, st, pdl)
+                       : launch_attn_t<NW, true, false, ST, CL, EG>(a, grid, st, pdl);
+    }
+    if (kv == 2) return launch_attn_t<NW, false, true, ST, CL, EG, true>(a, grid, st, pdl);
+    return kv == 1 ? launch_attn_t<NW, false, true, ST, CL, EG>(a, grid, st, pdl)
+                   : launch_attn_t<NW, false, false, ST, CL, EG>(a, grid, st, pdl);
 }
 
 // Splits of up to 4 tiles keep all of them in flight (4 or 5 stages);
@@ -325,7 +330,7 @@ sa_status launch_attn_nw(const sa::AttnArgs& a, bool gather, bool fp8, dim3 grid
 // exactly kAttnCluster ways merges inside a cluster.  Decode with up to 64
 // heads splits every tile between two warp groups (8 warps), which halves
 // the serial work per warp; prefill and more heads keep one group.
-sa_status launch_attn(const sa::AttnArgs& a, bool gather, bool fp8, long long BQ, cudaStream_t st, bool pdl,
+sa_status launch_attn(const sa::AttnArgs& a, bool gather, int kv, long long BQ, cudaStream_t st, bool pdl,
                       bool decode) {
     const bool cl = a.splits == sa::kAttnCluster && BQ <= 65535;
     if (BQ > 2147483647LL || a.splits > 65535) return fail(SA_ERR_INVALID_ARG, "too many queries or splits");
@@ -335,25 +340,25 @@ sa_status launch_attn(const sa::AttnArgs& a, bool gather, bool fp8, long long BQ
         // splits of 4 tiles keep all four in flight (5 stages)
         const bool d5 = a.tiles_per_split == 4;
         if (cl)
-            return d5 ? launch_attn_nw<4, 5, true, 2>(a, gather, fp8, grid, st, pdl)
-                      : deep ? launch_attn_nw<4, 4, true, 2>(a, gather, fp8, grid, st, pdl)
-                             : launch_attn_nw<4, 2, true, 2>(a, gather, fp8, grid, st, pdl);
-        return d5 ? launch_attn_nw<4, 5, false, 2>(a, gather, fp8, grid, st, pdl)
-                  : deep ? launch_attn_nw<4, 4, false, 2>(a, gather, fp8, grid, st, pdl)
-                         : launch_attn_nw<4, 2, false, 2>(a, gather, fp8, grid, st, pdl);
+            return d5 ? launch_attn_nw<4, 5, true, 2>(a, gather, kv, grid, st, pdl)
+                      : deep ? launch_attn_nw<4, 4, true, 2>(a, gather, kv, grid, st, pdl)
+                             : launch_attn_nw<4, 2, true, 2>(a, gather, kv, grid, st, pdl);
+        return d5 ? launch_attn_nw<4, 5, false, 2>(a, gather, kv, grid, st, pdl)
+                  : deep ? launch_attn_nw<4, 4, false, 2>(a, gather, kv, grid, st, pdl)
+                         : launch_attn_nw<4, 2, false, 2>(a, gather, kv, grid, st, pdl);
     }
     if (a.H <= 64) {  // prefill: long lists, one warp group measured faster
         if (cl)
-            return deep ? launch_attn_nw<4, 4, true, 1>(a, gather, fp8, grid, st, pdl)
-                        : launch_attn_nw<4, 2, true, 1>(a, gather, fp8, grid, st, pdl);
-        return deep ? launch_attn_nw<4, 4, false, 1>(a, gather, fp8, grid, st, pdl)
-                    : launch_attn_nw<4, 2, false, 1>(a, gather, fp8, grid, st, pdl);
+            return deep ? launch_attn_nw<4, 4, true, 1>(a, gather, kv, grid, st, pdl)
+                        : launch_attn_nw<4, 2, true, 1>(a, gather, kv, grid, st, pdl);
+        return deep ? launch_attn_nw<4, 4, false, 1>(a, gather, kv, grid, st, pdl)
+                    : launch_attn_nw<4, 2, false, 1>(a, gather, kv, grid, st, pdl);
     }
     if (cl)
-        return deep ? launch_attn_nw<8, 4, true, 1>(a, gather, fp8, grid, st, pdl)
-                    : launch_attn_nw<8, 2, true, 1>(a, gather, fp8, grid, st, pdl);
-    return deep ? launch_attn_nw<8, 4, false, 1>(a, gather, fp8, grid, st, pdl)
-                : launch_attn_nw<8, 2, false, 1>(a, gather, fp8, grid, st, pdl);
+        return deep ? launch_attn_nw<8, 4, true, 1>(a, gather, kv, grid, st, pdl)
+                    : launch_attn_nw<8, 2, true, 1>(a, gather, kv, grid, st, pdl);
+    return deep ? launch_attn_nw<8, 4, false, 1>(a, gather, kv, grid, st, pdl)
+                : launch_attn_nw<8, 2, false, 1>(a, gather, kv, grid, st, pdl);
 }
 
 // Causal prefill with 64 heads over a bf16 cache: the tensor-memory kernel
@@ -463,7 +468,8 @@ sa_status run_attn(const void* q, int Tq, int H, const sa_cache* c, bool gather,
     // dense causal prefill (HCA) on the tensor-memory kernel; the gathered one
     // (CSA) stays on the mma.sync kernel, which measured faster (see DESIGN)
     if (prefill && !gather && win == 0 && H == 64 && c->dtype == SA_BF16 && pos) return launch_prefill_tc(a, c, false, st);
-    sa_status r = launch_attn(a, gather, c->dtype == SA_FP8_E4M3, BQ, st, chained && pdl_on(), !prefill);
+    const int kv = c->dtype == SA_KV_MIXED ? 2 : c->dtype == SA_FP8_E4M3 ? 1 : 0;
+    sa_status r = launch_attn(a, gather, kv, BQ, st, chained && pdl_on(), !prefill);
     if (r != SA_OK) return r;
     // a query split kAttnCluster ways was merged inside its cluster
     if (sp.splits > 1 && !(sp.splits == sa::kAttnCluster && BQ <= 65535))
@@ -725,11 +731,15 @@ static sa_status compress_common(const sa_raw* raw, const sa_cache* out, void* s
     a.nG = (out->Ncap + 63) / 64;
     a.m = out->m;
     a.log2m = ilog2(out->m);
-    a.fp8 = out->dtype == SA_FP8_E4M3;
+    a.fp8 = out->dtype != SA_BF16;  // e4m3 K and V, or mixed K + e4m3 V
+    const bool mixed = out->dtype == SA_KV_MIXED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (!append) {
         const int groups = std::max(1, cdiv(raw->Lcap / out->m, 64));
-        sa::compress_kernel<<<dim3(groups, raw->B), sa::kCompThreads, 0, st>>>(a);
+        if (mixed)
+            sa::compress_kernel<true><<<dim3(groups, raw->B), sa::kCompThreads, 0, st>>>(a);
+        else
+            sa::compress_kernel<false><<<dim3(groups, raw->B), sa::kCompThreads, 0, st>>>(a);
         SA_LAUNCHED();
         return SA_OK;
     }
@@ -738,7 +748,10 @@ static sa_status compress_common(const sa_raw* raw, const sa_cache* out, void* s
     a.n_from = out->n;
     const long long new_entries = ((long long)max_new_tokens + out->m - 1) / out->m;
     const long long groups = std::min<long long>((new_entries + 63) / 64 + 1, cdiv(out->Ncap, 64) + 1LL);
-    sa::compress_kernel<<<dim3((unsigned)groups, raw->B), sa::kCompThreads, 0, st>>>(a);
+    if (mixed)
+        sa::compress_kernel<true><<<dim3((unsigned)groups, raw->B), sa::kCompThreads, 0, st>>>(a);
+    else
+        sa::compress_kernel<false><<<dim3((unsigned)groups, raw->B), sa::kCompThreads, 0, st>>>(a);
     SA_LAUNCHED();
     sa::set_counts_kernel<<<cdiv(raw->B, 128), 128, 0, st>>>(raw->len, out->n, raw->B, raw->Lcap, a.log2m,
                                                                (int)groups);

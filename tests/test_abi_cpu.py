@@ -75,6 +75,8 @@ def _raw(**kw):
     ({}, {"kidx": None}, "kidx"),
     ({}, {"k": FAKE + 4}, "aligned"),
     ({}, {"dtype": _lib.SA_FP8_E4M3}, "k_scale"),
+    ({}, {"dtype": _lib.SA_KV_MIXED}, "k_scale"),
+    ({}, {"dtype": 3}, "dtype"),
     ({"kidx": None}, {}, "kidx"),
     ({"B": 2}, {}, "B=2"),
     ({"Lcap": 8192}, {}, "Ncap"),
