@@ -112,7 +112,8 @@ typedef enum {
     SA_OP_DENSE_ATTN = 3,
     SA_OP_HYBRID_DECODE = 4,
     SA_OP_HYBRID_PREFILL = 5,
-    SA_OP_WINDOW_ATTN = 6   /* k = the window */
+    SA_OP_WINDOW_ATTN = 6,  /* k = the window */
+    SA_OP_CP_CANDIDATES = 7 /* cp_decode_candidates (Tq = 1) */
 } sa_op;
 
 /* Compression, section 3-2 (2) component table, CSA row ("every 4 tokens ->
@@ -313,6 +314,58 @@ sa_status sa_set_stage_events(int32_t stage, void* before, void* after);
  *   q_idx [B][d_idx] bf16; idx [B][k] and cnt [B] int32 out, as csa_index_topk. */
 sa_status csa_index_topk_noalloc(const void* q_idx, const sa_cache* csa, int32_t k, int32_t* idx, int32_t* cnt,
                                  void* stream);
+
+/* ---- Context-parallel decode -------------------------------------------
+ * The review's section 3-2 (4) lists contextual parallelism among the
+ * inference infrastructure without describing it; the exchange here is this
+ * library's own.  One sequence's compressed entries are split over W ranks in
+ * contiguous shards, rank w holding global entries base[b] .. base[b] +
+ * n[b] - 1 of sequence b (shards in rank order, shard boundaries on whole
+ * HCA blocks).  Because every entry of the global top-k is in the top-k of
+ * its own shard, a step is exact:
+ *   1. cp_decode_candidates on every rank;
+ *   2. all-gather of (keys, gidx, gcnt) in rank order (W x the arrays);
+ *   3. cp_decode_merge_select on every rank: its share of the global top-k;
+ *   4. csa_sparse_attn over that share and hca_dense_attn over the HCA
+ *      shard, each with its lse;
+ *   5. all-gather of the partial (out, lse) and attn_lse_merge_n.
+ * The collectives are the caller's (NCCL through torch.distributed in the
+ * Python binding); these calls are the per-rank compute.                   */
+
+/* Exact local top-k of this rank's CSA shard for B decode queries, then the
+ * exact order key and global index of each winner.
+ *   base  [B] int32: global index of the shard's entry 0.
+ *   keys  [B][k] uint32 out: order key of the winner's fp32 score s: the
+ *         bits of s with the sign bit set for s >= 0, all bits flipped for
+ *         s < 0 (-0 counts as +0); 0 past the count.
+ *   gidx  [B][k] int32 out: global indices, ascending, -1 past the count.
+ *   gcnt  [B] int32 out: min(k, n[b]).
+ * ws / ws_bytes: at least sa_workspace_size(SA_OP_CP_CANDIDATES, B, 1, H,
+ * Ncap, 0, k).                                                              */
+sa_status cp_decode_candidates(const void* q_idx, const sa_cache* csa, int32_t k, const int32_t* base,
+                               uint32_t* keys, int32_t* gidx, int32_t* gcnt, void* ws, size_t ws_bytes,
+                               void* stream);
+
+/* The global top-k from the gathered candidates of all W ranks and this
+ * rank's share of it.
+ *   keys, gidx [W][B][k], gcnt [W][B]: the candidate arrays of ranks 0..W-1
+ *              stacked in rank order.
+ *   base [B]: this rank's shard start (as given to cp_decode_candidates).
+ *   local_idx [B][k] int32 out: this rank's winners as shard-local indices,
+ *              ascending, -1 padded; local_cnt [B] out: their count.
+ *   sel_idx [B][k] / sel_cnt [B] out, or both NULL: the global selection,
+ *              ascending, -1 padded, and min(k, total candidates).
+ * W * k must be at most 16384 (SA_ERR_UNSUPPORTED otherwise).              */
+sa_status cp_decode_merge_select(const uint32_t* keys, const int32_t* gidx, const int32_t* gcnt, int32_t W,
+                                 int32_t B, int32_t k, int32_t rank, const int32_t* base, int32_t* local_idx,
+                                 int32_t* local_cnt, int32_t* sel_idx, int32_t* sel_cnt, void* stream);
+
+/* W-way log-sum-exp merge of attentions over disjoint key sets:
+ * lse = log sum_w e^lse_w, out = sum_w e^lse_w out_w / e^lse.
+ *   outs [W][rows][128] bf16, lses [W][rows] fp32; out [rows][128] bf16,
+ *   lse [rows] fp32 or NULL.  A row whose lses are all -inf gets 0, -inf.   */
+sa_status attn_lse_merge_n(const void* outs, const float* lses, int32_t W, int64_t rows, void* out, float* lse,
+                           void* stream);
 
 /* Number of kernels this library has launched from the calling host thread
  * since the process started (a diagnostic counter; memsets are not kernels). */

@@ -228,6 +228,56 @@ def csa_index_topk_mxfp4(q_idx, csa: Cache, codes, scales, k: int, ws, *, idx=No
     return idx, cnt
 
 
+def cp_decode_candidates(q_idx, csa: Cache, k: int, base, ws, *, keys=None, gidx=None, gcnt=None, stream=None):
+    """This rank's exact local top-k with the order keys and global indices of
+    its winners: (keys [B][k] int32 holding the uint32 order keys, gidx [B][k],
+    gcnt [B])."""
+    _need(q_idx, torch.bfloat16, "q_idx")
+    _need(base, torch.int32, "base")
+    B, dev = csa.B, q_idx.device
+    keys = torch.empty(B, k, dtype=torch.int32, device=dev) if keys is None else keys
+    gidx = torch.empty(B, k, dtype=torch.int32, device=dev) if gidx is None else gidx
+    gcnt = torch.empty(B, dtype=torch.int32, device=dev) if gcnt is None else gcnt
+    cs = csa.struct()
+    check("cp_decode_candidates", lib().cp_decode_candidates(_ptr(q_idx), ctypes.byref(cs), k, _ptr(base), _ptr(keys),
+                                                             _ptr(gidx), _ptr(gcnt), _ptr(ws), ws.numel(),
+                                                             _stream(stream)))
+    return keys, gidx, gcnt
+
+
+def cp_decode_merge_select(keys, gidx, gcnt, rank: int, base, *, local_idx=None, local_cnt=None, sel_idx=None,
+                           sel_cnt=None, stream=None):
+    """From the candidates of all ranks stacked in rank order (keys, gidx
+    [W][B][k], gcnt [W][B]): (local_idx [B][k], local_cnt [B], sel_idx [B][k],
+    sel_cnt [B]), this rank's share of the global top-k and the selection."""
+    for t, name in ((keys, "keys"), (gidx, "gidx"), (gcnt, "gcnt"), (base, "base")):
+        _need(t, torch.int32, name)
+    W, B, k = gidx.shape
+    dev = gidx.device
+    local_idx = torch.empty(B, k, dtype=torch.int32, device=dev) if local_idx is None else local_idx
+    local_cnt = torch.empty(B, dtype=torch.int32, device=dev) if local_cnt is None else local_cnt
+    sel_idx = torch.empty(B, k, dtype=torch.int32, device=dev) if sel_idx is None else sel_idx
+    sel_cnt = torch.empty(B, dtype=torch.int32, device=dev) if sel_cnt is None else sel_cnt
+    check("cp_decode_merge_select",
+          lib().cp_decode_merge_select(_ptr(keys), _ptr(gidx), _ptr(gcnt), W, B, k, rank, _ptr(base), _ptr(local_idx),
+                                       _ptr(local_cnt), _ptr(sel_idx), _ptr(sel_cnt), _stream(stream)))
+    return local_idx, local_cnt, sel_idx, sel_cnt
+
+
+def attn_lse_merge_n(outs, lses, *, out=None, lse=None, stream=None):
+    """W-way log-sum-exp merge: outs [W][..][128] bf16, lses [W][..] fp32 ->
+    (out [..][128], lse [..])."""
+    _need(outs, torch.bfloat16, "outs")
+    _need(lses, torch.float32, "lses")
+    W = outs.shape[0]
+    rows = lses[0].numel()
+    out = torch.empty(outs.shape[1:], dtype=torch.bfloat16, device=outs.device) if out is None else out
+    lse = torch.empty(lses.shape[1:], dtype=torch.float32, device=outs.device) if lse is None else lse
+    check("attn_lse_merge_n", lib().attn_lse_merge_n(_ptr(outs), _ptr(lses), W, rows, _ptr(out), _ptr(lse),
+                                                     _stream(stream)))
+    return out, lse
+
+
 def csa_sparse_attn(q, csa: Cache, idx, cnt, k: int, ws, *, scale=0.0, out=None, lse=None, stream=None):
     _need(q, torch.bfloat16, "q")
     B, Tq, H = q.shape[0], (q.shape[1] if q.dim() == 4 else 1), q.shape[-2]

@@ -1,0 +1,100 @@
+"""Context-parallel decode over torch.distributed.
+
+One long sequence's compressed entries are split over the W ranks of a
+process group in contiguous shards, one per rank; each rank compresses and
+holds only its shard (the review's section 3-2 (4) lists contextual
+parallelism among the inference infrastructure; this exchange is the
+library's own).  Every entry of the global top-k is in the top-k of its own
+shard, so one decode step is exact:
+
+  1. ``cp_decode_candidates``: this rank's exact local top-k, with the order
+     key and global index of each winner;
+  2. all-gather of the candidates (k per rank and sequence);
+  3. ``cp_decode_merge_select``: the global top-k, and this rank's share;
+  4. CSA attention over the share and HCA attention over the HCA shard, each
+     with its log-sum-exp;
+  5. all-gather of the partials and one W-way log-sum-exp merge of both
+     branches (``attn_lse_merge_n``).
+
+Every rank ends with the same outputs and the same selection.  The compute
+runs in the library's kernels; this module holds the host logic: the shard
+boundaries and the collectives (NCCL over NVLink on B200s; any backend whose
+``all_gather`` takes tensors on the data's device).
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+from . import api as S
+from ._lib import SA_OP_CP_CANDIDATES, SA_OP_DENSE_ATTN, SA_OP_SPARSE_ATTN
+
+HCA_BLOCK = 128  # shard boundaries fall on whole HCA blocks (hence whole CSA blocks)
+
+
+def shard_bounds(length: int, world: int, align: int = HCA_BLOCK) -> list[tuple[int, int]]:
+    """Token ranges [t0, t1) of the W shards of a sequence of `length` tokens:
+    contiguous, in rank order, covering [0, length), every inner boundary a
+    multiple of `align`, with the aligned blocks spread as evenly as that
+    allows (the tail of an incomplete block goes to the shard holding the
+    last block).  A shard may be empty."""
+    if length < 0 or world < 1 or align < 1:
+        raise ValueError(f"length={length}, world={world}, align={align}")
+    blocks = -(-length // align)
+    per, extra = divmod(blocks, world)
+    out, b0 = [], 0
+    for w in range(world):
+        b1 = b0 + per + (1 if w < extra else 0)
+        out.append((min(length, b0 * align), min(length, b1 * align)))
+        b0 = b1
+    return out
+
+
+def entry_base(bounds: list[tuple[int, int]], rank: int, m: int) -> int:
+    """Global index of the first compressed entry of `rank`'s shard (an empty
+    shard, which holds no entry, may start anywhere)."""
+    t0, t1 = bounds[rank]
+    if t0 % m and t1 > t0:
+        raise ValueError(f"shard start {t0} is not a multiple of m={m}")
+    return t0 // m
+
+
+def workspace_size(B: int, H: int, Ncap_csa: int, Ncap_hca: int, k: int) -> int:
+    """Scratch bytes of one cp_decode_step (its calls run in order on one stream)."""
+    return max(S.workspace_size(SA_OP_CP_CANDIDATES, B, 1, H, Ncap_csa, 0, k),
+               S.workspace_size(SA_OP_SPARSE_ATTN, B, 1, H, Ncap_csa, 0, k),
+               S.workspace_size(SA_OP_DENSE_ATTN, B, 1, H, 0, Ncap_hca, 0))
+
+
+def gather_ranks(t: torch.Tensor, group=None) -> torch.Tensor:
+    """All-gather `t` from every rank of the group into one [W, *t.shape]
+    tensor, in rank order (each rank's slice written in place)."""
+    W = dist.get_world_size(group)
+    buf = torch.empty((W,) + tuple(t.shape), dtype=t.dtype, device=t.device)
+    dist.all_gather(list(buf.unbind(0)), t.contiguous(), group=group)
+    return buf
+
+
+def cp_decode_step(q, q_idx, csa: S.Cache, hca: S.Cache, base_csa, k: int, ws, *, group=None, scale=0.0,
+                   stream=None):
+    """One decode step of both branches for B sequences sharded over the group.
+
+    q [B][H][128] and q_idx [B][64] bf16 (the same on every rank); csa / hca:
+    this rank's shards (m = 4 / 128); base_csa [B] int32: the global index of
+    the CSA shard's entry 0 (entry_base).  Returns (out_csa, out_hca, lse_csa,
+    lse_hca, sel_idx, sel_cnt): the outputs of the whole sequence and the
+    global selection (ascending global indices, -1 padded), equal on every
+    rank."""
+    rank = dist.get_rank(group)
+    B, H = q.shape[0], q.shape[1]
+    keys, gidx, gcnt = S.cp_decode_candidates(q_idx, csa, k, base_csa, ws, stream=stream)
+    all_keys, all_gidx, all_gcnt = gather_ranks(keys, group), gather_ranks(gidx, group), gather_ranks(gcnt, group)
+    local_idx, local_cnt, sel_idx, sel_cnt = S.cp_decode_merge_select(all_keys, all_gidx, all_gcnt, rank, base_csa,
+                                                                      stream=stream)
+    part_o = torch.empty(2, B, H, 128, dtype=torch.bfloat16, device=q.device)
+    part_l = torch.empty(2, B, H, dtype=torch.float32, device=q.device)
+    S.csa_sparse_attn(q, csa, local_idx, local_cnt, k, ws, scale=scale, out=part_o[0], lse=part_l[0], stream=stream)
+    S.hca_dense_attn(q, hca, ws, scale=scale, out=part_o[1], lse=part_l[1], stream=stream)
+    # both branches merge row by row in one launch
+    out, lse = S.attn_lse_merge_n(gather_ranks(part_o, group), gather_ranks(part_l, group), stream=stream)
+    return out[0], out[1], lse[0], lse[1], sel_idx, sel_cnt

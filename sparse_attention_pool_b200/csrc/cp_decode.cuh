@@ -1,0 +1,201 @@
+// cp_decode.cuh -- context-parallel decode: the compressed entries of one
+// sequence split over W ranks in contiguous shards (the review's section 3-2
+// (4) names contextual parallelism among its infrastructure; the exchange
+// below is this library's own).
+//
+// Exactness of the split selection: every entry of the global top-k (by
+// score desc, index asc) is in the top-k of its own shard, so the global
+// top-k is the top-k of the union of the W local top-k lists.  A step is
+//   1. each rank: exact local top-k of its shard (the decode kernels), then
+//      cp_candidates_kernel: the exact order key and the global index of each
+//      local winner;
+//   2. all-gather of the W candidate lists (k pairs per rank and sequence);
+//   3. each rank: cp_merge_select_kernel cuts the union at the k-th largest
+//      (key, -index) and keeps its own share of the winners;
+//   4. each rank: attention over its share (CSA) and over its HCA shard, with
+//      the log-sum-exp of each;
+//   5. all-gather of the W partial (out, lse) and attn_lse_merge_n_kernel: the
+//      attention over the union is the log-sum-exp merge of the partials.
+// Gathered rank-major, the candidates are in ascending global index order
+// (the shards are contiguous and each local list is ascending), which the
+// merge uses for both its tie-break and its ordered outputs.
+#pragma once
+#include "sa_common.cuh"
+#include "topk_decode.cuh"
+
+namespace sa {
+
+// ---------------------------------------------- 1. candidate keys ----------
+struct CandArgs {
+    const uint16_t* q_idx;  // [B][64] bf16
+    const uint16_t* kidx;   // [B][Ncap][64] bf16: this rank's shard
+    const int32_t* idx;     // [B][k] local winners (ascending, -1 padded)
+    const int32_t* cnt;     // [B]
+    const int32_t* base;    // [B] global index of the shard's entry 0
+    uint32_t* keys;         // [B][k] out: exact order keys (0 past the count)
+    int32_t* gidx;          // [B][k] out: global indices (-1 past the count)
+    int32_t* gcnt;          // [B] out: the count
+    int Ncap, k;
+};
+
+constexpr int kCandThreads = 256;
+
+// grid (ceil(k / 256), B): one thread per list position.
+__global__ void __launch_bounds__(kCandThreads) cp_candidates_kernel(CandArgs a) {
+    __shared__ double q2[64];  // qI * 2^768 in fp64 (the layout exact_key reads)
+    pdl_wait();
+    pdl_release();
+    const int b = blockIdx.y;
+    const int tid = threadIdx.x;
+    if (tid < 32) {
+        const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(a.q_idx + (size_t)b * 64) + tid);
+        q2[2 * tid] = (double)bf16lo_f32(w) * 0x1p768;
+        q2[2 * tid + 1] = (double)bf16hi_f32(w) * 0x1p768;
+    }
+    __syncthreads();
+    int c = a.cnt[b];
+    if (c < 0 || c > a.k) {
+        if (blockIdx.x == 0 && tid == 0) flag(DEV_LEN);
+        c = c < 0 ? 0 : a.k;
+    }
+    const int i = blockIdx.x * kCandThreads + tid;
+    if (i >= a.k) return;
+    if (i == 0) a.gcnt[b] = c;
+    uint32_t key = 0u;
+    int32_t g = -1;
+    if (i < c) {
+        const int j = a.idx[(size_t)b * a.k + i];
+        if (j < 0 || j >= a.Ncap) {
+            flag(DEV_INDEX);
+        } else {
+            key = exact_key(q2, a.kidx + ((size_t)b * a.Ncap + j) * 64);
+            g = a.base[b] + j;
+        }
+    }
+    a.keys[(size_t)b * a.k + i] = key;
+    a.gidx[(size_t)b * a.k + i] = g;
+}
+
+// ------------------------------------------- 3. merge and select -----------
+constexpr int kMergeThreads = 1024;
+constexpr int kMergeCap = 16384;  // candidates of one sequence held in shared memory (W * k)
+constexpr int kMergeMaxRanks = 64;
+constexpr size_t kMergeSmem = (size_t)kMergeCap * 8;
+
+struct MergeArgs {
+    const uint32_t* keys;  // [W][B][k] gathered candidate keys
+    const int32_t* gidx;   // [W][B][k]
+    const int32_t* gcnt;   // [W][B]
+    const int32_t* base;   // [B] this rank's shard start
+    int32_t* local_idx;    // [B][k] out: this rank's winners, shard-local, ascending, -1 padded
+    int32_t* local_cnt;    // [B] out
+    int32_t* sel_idx;      // [B][k] out (or NULL): the global selection, ascending, -1 padded
+    int32_t* sel_cnt;      // [B] out (or NULL)
+    int W, B, k, rank;
+};
+
+// One CTA per sequence: the W candidate lists, rank-major, into shared
+// memory; the exact cut at rank min(k, C) by (key desc, index asc); then
+// the winners in list order (= ascending global index), globally and for
+// this rank.
+__global__ void __launch_bounds__(kMergeThreads, 1) cp_merge_select_kernel(MergeArgs a) {
+    extern __shared__ __align__(16) uint32_t csm[];  // [kMergeCap] keys, [kMergeCap] global indices
+    __shared__ uint32_t hist[kBins];
+    __shared__ uint32_t sh64[64];
+    __shared__ int res[2];
+    __shared__ int s_off[kMergeMaxRanks + 1];
+    pdl_wait();
+    pdl_release();
+    const int b = blockIdx.x;
+    const int tid = threadIdx.x;
+    uint32_t* lk = csm;
+    int32_t* li = reinterpret_cast<int32_t*>(csm + kMergeCap);
+    if (tid == 0) {
+        int o = 0;
+        for (int w = 0; w < a.W; ++w) {
+            int c = a.gcnt[(size_t)w * a.B + b];
+            if (c < 0 || c > a.k) {
+                flag(DEV_LEN);
+                c = c < 0 ? 0 : a.k;
+            }
+            s_off[w] = o;
+            o += c;
+        }
+        s_off[a.W] = o;
+    }
+    __syncthreads();
+    const uint32_t C = (uint32_t)s_off[a.W];  // <= W * k <= kMergeCap (checked on the host)
+    for (uint32_t p = tid; p < C; p += kMergeThreads) {
+        int w = 0;
+        while (s_off[w + 1] <= (int)p) ++w;  // W is small
+        const size_t src = ((size_t)w * a.B + b) * a.k + (p - (uint32_t)s_off[w]);
+        lk[p] = __ldg(a.keys + src);
+        li[p] = __ldg(a.gidx + src);
+    }
+    __syncthreads();
+    const uint32_t R = min(C, (uint32_t)a.k);
+    uint32_t T = 0u;
+    int32_t jmax = 0x7FFFFFFF;
+    const bool all = C <= (uint32_t)a.k;
+    if (!all) select_rank(lk, li, C, R, hist, sh64, res, &T, &jmax);
+    // winners in list order: globally, and this rank's rows
+    const uint32_t lo = (uint32_t)s_off[a.rank], hi = (uint32_t)s_off[a.rank + 1];
+    const int32_t base = a.base[b];
+    uint32_t gpos = 0, lpos = 0;
+    for (uint32_t p0 = 0; p0 < C; p0 += kMergeThreads) {  // block-uniform trip count
+        const uint32_t p = p0 + tid;
+        bool win = false;
+        if (p < C) {
+            const uint32_t kk = lk[p];
+            win = all || kk > T || (kk == T && li[p] <= jmax);
+        }
+        const bool mine = win && p >= lo && p < hi;
+        uint32_t gt, lt;
+        const uint32_t ge = block_exclusive_scan(win ? 1u : 0u, sh64, &gt);
+        const uint32_t le = block_exclusive_scan(mine ? 1u : 0u, sh64, &lt);
+        if (win && a.sel_idx) a.sel_idx[(size_t)b * a.k + gpos + ge] = li[p];
+        if (mine) a.local_idx[(size_t)b * a.k + lpos + le] = li[p] - base;
+        gpos += gt;
+        lpos += lt;
+    }
+    for (uint32_t i = gpos + tid; a.sel_idx && i < (uint32_t)a.k; i += kMergeThreads) a.sel_idx[(size_t)b * a.k + i] = -1;
+    for (uint32_t i = lpos + tid; i < (uint32_t)a.k; i += kMergeThreads) a.local_idx[(size_t)b * a.k + i] = -1;
+    if (tid == 0) {
+        if (gpos != R) flag(DEV_LEN);  // cannot happen
+        a.local_cnt[b] = (int32_t)lpos;
+        if (a.sel_cnt) a.sel_cnt[b] = (int32_t)R;
+    }
+}
+
+// ------------------------------------------------- 5. W-way merge ----------
+// Log-sum-exp merge of W attentions over disjoint key sets into the
+// attention over their union: one warp per row, 4 dims a lane, fp32
+// accumulation, one rounding to bf16.
+__global__ void __launch_bounds__(256) attn_lse_merge_n_kernel(const uint16_t* outs, const float* lses, int W,
+                                                               long long rows, uint16_t* out, float* lse) {
+    pdl_wait();
+    pdl_release();
+    const long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (r >= rows) return;
+    float M = -INFINITY;
+    for (int w = 0; w < W; ++w) M = fmaxf(M, lses[(size_t)w * rows + r]);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float ws = 0.f;
+    for (int w = 0; w < W; ++w) {
+        const float l = lses[(size_t)w * rows + r];
+        const float wt = l == -INFINITY ? 0.f : __expf(l - M);
+        const uint2 v = *reinterpret_cast<const uint2*>(outs + ((size_t)w * rows + r) * 128 + lane * 4);
+        acc[0] += wt * bf16lo_f32(v.x);
+        acc[1] += wt * bf16hi_f32(v.x);
+        acc[2] += wt * bf16lo_f32(v.y);
+        acc[3] += wt * bf16hi_f32(v.y);
+        ws += wt;
+    }
+    const float inv = ws > 0.f ? 1.f / ws : 0.f;
+    *reinterpret_cast<uint2*>(out + r * 128 + lane * 4) =
+        make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
+    if (lse && lane == 0) lse[r] = ws > 0.f ? M + __logf(ws) : -INFINITY;
+}
+
+}  // namespace sa

@@ -18,6 +18,7 @@
 #include "attn.cuh"
 #include "attn_prefill_tc.cuh"
 #include "compress.cuh"
+#include "cp_decode.cuh"
 #include "lowp_index.cuh"
 #include "sa_common.cuh"
 #include "topk_decode.cuh"
@@ -860,6 +861,9 @@ size_t sa_workspace_size(int32_t op, int32_t B, int32_t Tq, int32_t H, int32_t N
             Split s = attn_split(k, prefill);
             return 256 + attn_partial_bytes(BQ, s.splits, H);
         }
+        case SA_OP_CP_CANDIDATES:
+            if (k < 1 || Tq != 1) return 0;
+            return topk_decode_layout(B, Ncap_csa, k, true).total;
         default:
             return 0;
     }
@@ -962,6 +966,98 @@ sa_status csa_index_topk_mxfp4(const void* q_idx, const sa_cache* csa, const uin
     if (r != SA_OK) return r;
     return run_topk_decode(q_idx, csa, k, idx, cnt, ws, w, static_cast<cudaStream_t>(stream),
                            [] { return SA_OK; }, codes, scales);
+}
+
+sa_status cp_decode_candidates(const void* q_idx, const sa_cache* csa, int32_t k, const int32_t* base,
+                               uint32_t* keys, int32_t* gidx, int32_t* gcnt, void* ws, size_t ws_bytes,
+                               void* stream) {
+    sa_status r = check_cache(csa, true, "cp_decode_candidates");
+    if (r != SA_OK) return r;
+    SA_CHECK(q_idx && aligned16(q_idx), "cp_decode_candidates: q_idx must be non-NULL and 16-byte aligned");
+    SA_CHECK(base && keys && gidx && gcnt && aligned16(base) && aligned16(keys) && aligned16(gidx) &&
+                 aligned16(gcnt),
+             "cp_decode_candidates: base, keys, gidx, gcnt must be non-NULL and 16-byte aligned");
+    SA_CHECK(k >= 1 && k <= 65536, "cp_decode_candidates: k=%d outside 1..65536", k);
+    const TopkDecodeWs w = topk_decode_layout(csa->B, csa->Ncap, k, true);
+    r = check_ws(ws, ws_bytes, w.total);
+    if (r != SA_OK) return r;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    int32_t* idx = reinterpret_cast<int32_t*>(wsb + w.idx);
+    int32_t* cnt = reinterpret_cast<int32_t*>(wsb + w.cnt);
+    r = run_topk_decode(q_idx, csa, k, idx, cnt, ws, w, st, [] { return SA_OK; });
+    if (r != SA_OK) return r;
+    sa::CandArgs a{};
+    a.q_idx = static_cast<const uint16_t*>(q_idx);
+    a.kidx = static_cast<const uint16_t*>(csa->kidx);
+    a.idx = idx;
+    a.cnt = cnt;
+    a.base = base;
+    a.keys = keys;
+    a.gidx = gidx;
+    a.gcnt = gcnt;
+    a.Ncap = csa->Ncap;
+    a.k = k;
+    SA_CUDA(launch_k(sa::cp_candidates_kernel, dim3((unsigned)cdiv(k, sa::kCandThreads), csa->B),
+                     dim3(sa::kCandThreads), 0, st, pdl_on(), 1u, a));
+    SA_LAUNCHED();
+    return SA_OK;
+}
+
+sa_status cp_decode_merge_select(const uint32_t* keys, const int32_t* gidx, const int32_t* gcnt, int32_t W,
+                                 int32_t B, int32_t k, int32_t rank, const int32_t* base, int32_t* local_idx,
+                                 int32_t* local_cnt, int32_t* sel_idx, int32_t* sel_cnt, void* stream) {
+    SA_CHECK(W >= 1 && W <= sa::kMergeMaxRanks, "cp_decode_merge_select: W=%d outside 1..%d", W, sa::kMergeMaxRanks);
+    SA_CHECK(rank >= 0 && rank < W, "cp_decode_merge_select: rank=%d outside 0..W-1", rank);
+    SA_CHECK(B >= 1 && B <= 65535, "cp_decode_merge_select: B=%d outside 1..65535", B);
+    SA_CHECK(k >= 1 && k <= 65536, "cp_decode_merge_select: k=%d outside 1..65536", k);
+    if ((long long)W * k > sa::kMergeCap)
+        return fail(SA_ERR_UNSUPPORTED, "cp_decode_merge_select: W*k=%lld candidates exceed %d", (long long)W * k,
+                    sa::kMergeCap);
+    SA_CHECK(keys && gidx && gcnt && base && local_idx && local_cnt,
+             "cp_decode_merge_select: keys, gidx, gcnt, base, local_idx, local_cnt must be non-NULL");
+    SA_CHECK((sel_idx == nullptr) == (sel_cnt == nullptr), "cp_decode_merge_select: give sel_idx and sel_cnt or neither");
+    SA_CHECK(aligned16(keys) && aligned16(gidx) && aligned16(gcnt) && aligned16(base) && aligned16(local_idx) &&
+                 aligned16(local_cnt) && (!sel_idx || (aligned16(sel_idx) && aligned16(sel_cnt))),
+             "cp_decode_merge_select: pointers must be 16-byte aligned");
+    static std::atomic<uint64_t> init{0};
+    if (!attr_done(init)) {
+        SA_CUDA(cudaFuncSetAttribute(sa::cp_merge_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)sa::kMergeSmem));
+        attr_set(init);
+    }
+    sa::MergeArgs a{};
+    a.keys = keys;
+    a.gidx = gidx;
+    a.gcnt = gcnt;
+    a.base = base;
+    a.local_idx = local_idx;
+    a.local_cnt = local_cnt;
+    a.sel_idx = sel_idx;
+    a.sel_cnt = sel_cnt;
+    a.W = W;
+    a.B = B;
+    a.k = k;
+    a.rank = rank;
+    sa::cp_merge_select_kernel<<<B, sa::kMergeThreads, sa::kMergeSmem, static_cast<cudaStream_t>(stream)>>>(a);
+    SA_LAUNCHED();
+    return SA_OK;
+}
+
+sa_status attn_lse_merge_n(const void* outs, const float* lses, int32_t W, int64_t rows, void* out, float* lse,
+                           void* stream) {
+    SA_CHECK(W >= 1 && W <= 1024, "attn_lse_merge_n: W=%d outside 1..1024", W);
+    SA_CHECK(rows >= 0, "attn_lse_merge_n: rows=%lld", (long long)rows);
+    SA_CHECK(outs && lses && out, "attn_lse_merge_n: outs, lses and out must be non-NULL");
+    SA_CHECK(aligned16(outs) && aligned16(lses) && aligned16(out) && (!lse || aligned16(lse)),
+             "attn_lse_merge_n: pointers must be 16-byte aligned");
+    if (rows == 0) return SA_OK;
+    const long long blocks = (rows + 7) / 8;
+    SA_CHECK(blocks <= 2147483647LL, "attn_lse_merge_n: too many rows");
+    sa::attn_lse_merge_n_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint16_t*>(outs), lses, W, rows, static_cast<uint16_t*>(out), lse);
+    SA_LAUNCHED();
+    return SA_OK;
 }
 
 sa_status csa_sparse_attn(const void* q, int32_t Tq, int32_t H, const sa_cache* csa, const int32_t* idx,
