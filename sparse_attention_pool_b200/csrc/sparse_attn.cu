@@ -205,7 +205,7 @@ struct TopkDecodeWs {
     int maxchunks, fchunk, nfch, Wcap;
 };
 
-// Rows per filter / emit CTA: 1024, or a multiple of it once a sequence
+// Rows per filter / emit CTA: kFiltRows (2048), or a multiple of it once a sequence
 // would need more than kSelMaxChunks filter chunks.
 int filter_chunk(int Ncap) {
     const long long per = (long long)sa::kFiltRows * sa::kSelMaxChunks;
