@@ -357,3 +357,60 @@ def hybrid_attn_prefill(q, q_idx, csa: Cache, hca: Cache, k: int, ws, idx_out, c
 def read_device_status(stream=None):
     """Synchronises the stream and raises if a kernel recorded a device-side anomaly."""
     check("sa_read_device_status", lib().sa_read_device_status(_stream(stream)))
+
+
+class CapturedDecode:
+    """A hybrid decode step captured once into a CUDA graph, for serving loops
+    that decode the same batch step after step.
+
+    The graph reads the caches in place (appends between steps are seen) and
+    its own static buffers: ``q`` [B][H][128] and ``q_idx`` [B][64] bf16 in,
+    ``out_csa`` / ``out_hca`` [B][H][128] bf16, ``lse_csa`` / ``lse_hca`` [B][H]
+    fp32, ``idx`` [B][k] / ``cnt`` [B] int32 out.  ``step`` copies new queries
+    in (from host or device tensors, asynchronously on the current stream),
+    replays the graph and, if given host tensors, copies the outputs out.
+    With MXFP4 ``codes`` / ``scales`` the CSA selection runs on FP4 scores.
+    """
+
+    def __init__(self, csa: Cache, hca: Cache, k: int, H: int, *, scale: float = 0.0, codes=None, scales=None):
+        dev = csa.k.device
+        B = csa.B
+        self.csa, self.hca, self.k, self.scale = csa, hca, k, scale
+        self.codes, self.scales = codes, scales
+        self.q = torch.zeros(B, H, D, dtype=torch.bfloat16, device=dev)
+        self.q_idx = torch.zeros(B, D_IDX, dtype=torch.bfloat16, device=dev)
+        self.out_csa = torch.empty(B, H, D, dtype=torch.bfloat16, device=dev)
+        self.out_hca = torch.empty_like(self.out_csa)
+        self.lse_csa = torch.empty(B, H, dtype=torch.float32, device=dev)
+        self.lse_hca = torch.empty_like(self.lse_csa)
+        self.idx = torch.empty(B, k, dtype=torch.int32, device=dev)
+        self.cnt = torch.empty(B, dtype=torch.int32, device=dev)
+        self.ws = alloc_workspace(workspace_size(_lib.SA_OP_HYBRID_DECODE, B, 1, H, csa.Ncap, hca.Ncap, k), device=dev)
+        self._call()  # first call outside the capture: one-time kernel attributes and the side stream
+        torch.cuda.synchronize(dev)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self._call()
+        torch.cuda.synchronize(dev)
+
+    def _call(self):
+        kw = dict(scale=self.scale, out_csa=self.out_csa, out_hca=self.out_hca, lse_csa=self.lse_csa,
+                  lse_hca=self.lse_hca, idx_out=self.idx, cnt_out=self.cnt)
+        if self.codes is not None:
+            hybrid_attn_decode_mxfp4(self.q, self.q_idx, self.csa, self.hca, self.codes, self.scales, self.k, self.ws,
+                                     **kw)
+        else:
+            hybrid_attn_decode(self.q, self.q_idx, self.csa, self.hca, self.k, self.ws, **kw)
+
+    def step(self, q=None, q_idx=None, out_csa=None, out_hca=None, lse_csa=None, lse_hca=None):
+        """Copy q / q_idx in (when given), replay, copy outputs to the given
+        tensors (when given).  Asynchronous on the current stream."""
+        if q is not None:
+            self.q.copy_(q.view(torch.bfloat16) if q.dtype == torch.int16 else q, non_blocking=True)
+        if q_idx is not None:
+            self.q_idx.copy_(q_idx.view(torch.bfloat16) if q_idx.dtype == torch.int16 else q_idx, non_blocking=True)
+        self.graph.replay()
+        for dst, src in ((out_csa, self.out_csa), (out_hca, self.out_hca), (lse_csa, self.lse_csa),
+                         (lse_hca, self.lse_hca)):
+            if dst is not None:
+                dst.copy_(src.view(dst.dtype) if dst.dtype != src.dtype else src, non_blocking=True)
