@@ -153,8 +153,16 @@ __global__ void __launch_bounds__(kMergeThreads, 1) cp_merge_select_kernel(Merge
         uint32_t gt, lt;
         const uint32_t ge = block_exclusive_scan(win ? 1u : 0u, sh64, &gt);
         const uint32_t le = block_exclusive_scan(mine ? 1u : 0u, sh64, &lt);
-        if (win && a.sel_idx) a.sel_idx[(size_t)b * a.k + gpos + ge] = li[p];
-        if (mine) a.local_idx[(size_t)b * a.k + lpos + le] = li[p] - base;
+        // exactly R <= k winners (the cut's contract); a position past k is
+        // flagged, never written
+        if (win && a.sel_idx) {
+            if (gpos + ge < (uint32_t)a.k) a.sel_idx[(size_t)b * a.k + gpos + ge] = li[p];
+            else flag(DEV_LEN);
+        }
+        if (mine) {
+            if (lpos + le < (uint32_t)a.k) a.local_idx[(size_t)b * a.k + lpos + le] = li[p] - base;
+            else flag(DEV_LEN);
+        }
         gpos += gt;
         lpos += lt;
     }
@@ -162,7 +170,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) cp_merge_select_kernel(Merge
     for (uint32_t i = lpos + tid; i < (uint32_t)a.k; i += kMergeThreads) a.local_idx[(size_t)b * a.k + i] = -1;
     if (tid == 0) {
         if (gpos != R) flag(DEV_LEN);  // cannot happen
-        a.local_cnt[b] = (int32_t)lpos;
+        a.local_cnt[b] = (int32_t)min(lpos, (uint32_t)a.k);
         if (a.sel_cnt) a.sel_cnt[b] = (int32_t)R;
     }
 }
