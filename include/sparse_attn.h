@@ -63,7 +63,7 @@ extern "C" {
 typedef enum {
     SA_OK = 0,
     SA_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, bad size or shape      */
-    SA_ERR_UNSUPPORTED = 2,  /* a valid request this build does not implement      */
+    SA_ERR_UNSUPPORTED = 2,  /* a valid request the library does not implement     */
     SA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than sa_workspace_size */
     SA_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch, memset, ...)   */
     SA_ERR_TIMEOUT = 5,      /* device status: a bounded wait ran out              */
