@@ -167,18 +167,21 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def decode_bytes(w, lengths, indexer="bf16"):
+def decode_bytes(w, lengths, indexer="bf16", kv="workload"):
     """Algorithmic HBM bytes of one decode step and of its indexer score kernel
-    (an indexer key is 128 bytes in bf16, 32 + 2 in MXFP4)."""
-    bkv = 1 if w.fp8 else 2
+    (an indexer key is 128 bytes in bf16, 32 + 2 in MXFP4; a K + V entry is
+    512 bytes in bf16, 256 in e4m3 and 192 + 128 in mixed storage, the last
+    two with a scale each per gathered entry and per 64 HCA entries)."""
+    fp8 = w.fp8 or kv == "mixed"
+    kvb = 320 if kv == "mixed" else 2 * 128 * (1 if w.fp8 else 2)
     ib = 128 if indexer == "bf16" else 34
     step = 0
     score = 0
     for L in lengths:
         nc, nh = int(L) // w.m_csa, int(L) // w.m_hca
         sel = min(w.topk, nc)
-        step += nc * ib + sel * 2 * 128 * bkv + nh * 2 * 128 * bkv + w.H * 256 + 128 + 2 * w.H * 256
-        if w.fp8:
+        step += nc * ib + sel * kvb + nh * kvb + w.H * 256 + 128 + 2 * w.H * 256
+        if fp8:
             step += sel * 8 + ((nh + 63) // 64) * 8
         score += nc * ib + nc * 4  # read the indexer keys, write one 32-bit key per entry
     return step, score
@@ -233,8 +236,9 @@ def run_ours(args, w, rank, world, dev):
     t_gen = time.time()
     Kd, Vd, KId = to_bf16_tensor(K, dev), to_bf16_tensor(V, dev), to_bf16_tensor(KI, dev)
     lens = torch.from_numpy(lengths).to(dev)
-    csa = S.alloc_cache(w.B, w.L // w.m_csa, w.m_csa, fp8=w.fp8, with_kidx=True, device=dev)
-    hca = S.alloc_cache(w.B, w.L // w.m_hca, w.m_hca, fp8=w.fp8, device=dev)
+    mixed = args.kv == "mixed"
+    csa = S.alloc_cache(w.B, w.L // w.m_csa, w.m_csa, fp8=w.fp8, mixed=mixed, with_kidx=True, device=dev)
+    hca = S.alloc_cache(w.B, w.L // w.m_hca, w.m_hca, fp8=w.fp8, mixed=mixed, device=dev)
     S.csa_compress(Kd, Vd, KId, lens, csa)
     S.hca_compress(Kd, Vd, lens, hca)
     fp4 = args.indexer == "mxfp4"
@@ -414,7 +418,7 @@ def run_ours(args, w, rank, world, dev):
     del graph, graph_staged, graph_score, cap
 
     value = job_throughput(B * args.steps, world, total_ms)
-    step_bytes, score_bytes = decode_bytes(w, lengths, args.indexer)
+    step_bytes, score_bytes = decode_bytes(w, lengths, args.indexer, args.kv)
     peak, peak_kind = measured_peaks()
     score_avg = statistics.mean(score_ms)
     achieved = score_bytes / (score_avg / 1e3) / 1e9
@@ -430,10 +434,12 @@ def run_ours(args, w, rank, world, dev):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": ("bf16" if not w.fp8 else "fp8e4m3-kv/bf16") + ("+mxfp4-indexer" if fp4 else ""),
+        "dtype": ("mixed-kv(e4m3+bf16-rope)/bf16" if mixed else "bf16" if not w.fp8 else "fp8e4m3-kv/bf16")
+        + ("+mxfp4-indexer" if fp4 else ""),
         "data": "synthetic",
         "config": {"workload": w.name, "B_per_gpu": B, "context": int(w.L), "heads": H, "head_dim": 128,
-                   "csa_m": w.m_csa, "topk": k, "hca_m": w.m_hca, "kv_dtype": "e4m3" if w.fp8 else "bf16",
+                   "csa_m": w.m_csa, "topk": k, "hca_m": w.m_hca,
+                   "kv_dtype": "mixed" if mixed else "e4m3" if w.fp8 else "bf16",
                    "indexer": args.indexer,
                    "parallelism": f"replicas x{world} (independent sequences)",
                    "l2": "flushed between timed steps: 512 MB written then read back (clean L2)", "launch": "CUDA graph replay"},
@@ -454,9 +460,10 @@ def run_ours(args, w, rank, world, dev):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"], cs = cpu_baseline(w, lengths, K, V, KI, q_h, qI_h, budget_s=args.cpu_budget,
-                                                  indexer=args.indexer)
+                                                  indexer=args.indexer, kv=args.kv)
         result["cpu_baseline_all_cores"] = cpu_baseline_all_cores(w, lengths, K, V, KI, q_h, qI_h, cs=cs,
-                                                                  budget_s=args.cpu_budget / 2, indexer=args.indexer)
+                                                                  budget_s=args.cpu_budget / 2, indexer=args.indexer,
+                                                                  kv=args.kv)
     return result
 
 
@@ -582,10 +589,32 @@ def run_prefill(args, w, rank, world, dev):
 
 # ----------------------------------------------------------- oracle (CPU) ---
 
-def oracle_query(w, cs, q, qI, t, indexer="bf16"):
+def oracle_query(w, cs, q, qI, t, indexer="bf16", kv="workload"):
     """One decode query on the fp64 oracle: bf16 indexer scores, or FP4 ones
-    (the MXFP4 keys are built once per sequence, outside any timing)."""
+    (the MXFP4 keys are built once per sequence, outside any timing); the
+    workload's KV storage, or mixed storage (built once the same way)."""
     from oracle import oracle as O
+    if kv == "mixed":
+        if indexer != "bf16" and not hasattr(cs, "mx"):
+            cs.mx = O.mxfp4_quantize(cs.cidx)
+        if not hasattr(cs, "mixed"):
+            cs.mixed = {}
+            for name, (kb, vb) in (("c", (cs.ck_bf16, cs.cv_bf16)), ("h", (cs.hk_bf16, cs.hv_bf16))):
+                codes, ks, rope = O.mixed_quantize(kb, 64)
+                vc, vs = O.fp8_quantize(vb)
+                cs.mixed[name] = ({"mode": "mixed", "data": codes, "scales": ks, "rope": rope},
+                                  {"mode": "fp8", "data": vc, "scales": vs})
+        n_vis = min(int(t) // cs.m_csa, cs.n_csa)
+        if indexer == "bf16":
+            s = O.index_scores(qI, cs.cidx[:n_vis])
+        else:
+            qc, qs = O.mxfp4_quantize(np.asarray(qI, np.uint16).reshape(1, -1))
+            s = O.mxfp4_index_scores(qc[0], qs[0], cs.mx[0][:n_vis], cs.mx[1][:n_vis])
+        idx, cnt = O.topk(s, w.topk)
+        oc = O.attention_kv(q, *cs.mixed["c"], idx[:cnt], SCALE)
+        n_h = min(int(t) // cs.m_hca, cs.n_hca)
+        oh = O.attention_kv(q, *cs.mixed["h"], np.arange(n_h, dtype=np.int32), SCALE)
+        return {"idx": idx, "cnt": cnt, "out_csa": oc[0], "out_hca": oh[0]}
     if indexer == "bf16":
         return O.hybrid_query(cs, q, qI, t=t, k=w.topk, scale=SCALE)
     if not hasattr(cs, "mx"):
@@ -593,7 +622,7 @@ def oracle_query(w, cs, q, qI, t, indexer="bf16"):
     return O.hybrid_query_mxfp4(cs, q, qI, t=t, k=w.topk, scale=SCALE, idx_codes=cs.mx[0], idx_scales=cs.mx[1])
 
 
-def oracle_decode_one(w, lengths, K, V, KI, q_h, qI_h, b, indexer="bf16"):
+def oracle_decode_one(w, lengths, K, V, KI, q_h, qI_h, b, indexer="bf16", kv="workload"):
     """One decode token of sequence b on the fp64 oracle; returns (seconds, setup seconds)."""
     from oracle import oracle as O
     t0 = time.time()
@@ -601,26 +630,28 @@ def oracle_decode_one(w, lengths, K, V, KI, q_h, qI_h, b, indexer="bf16"):
     cs = O.CompressedSeq(K[b, :Lb], V[b, :Lb], KI[b, :Lb], m_csa=w.m_csa, m_hca=w.m_hca, fp8=w.fp8)
     if indexer != "bf16":
         cs.mx = O.mxfp4_quantize(cs.cidx)
+    if kv == "mixed":  # the mixed copies are built here, untimed
+        oracle_query(w, cs, q_h[b], qI_h[b], 0, indexer, kv)
     setup = time.time() - t0
     t1 = time.perf_counter()
-    oracle_query(w, cs, q_h[b], qI_h[b], Lb, indexer)
+    oracle_query(w, cs, q_h[b], qI_h[b], Lb, indexer, kv)
     return time.perf_counter() - t1, setup, cs
 
 
-def cpu_baseline(w, lengths, K, V, KI, q_h, qI_h, budget_s=20.0, indexer="bf16"):
-    el, setup, cs = oracle_decode_one(w, lengths, K, V, KI, q_h, qI_h, 0, indexer)
+def cpu_baseline(w, lengths, K, V, KI, q_h, qI_h, budget_s=20.0, indexer="bf16", kv="workload"):
+    el, setup, cs = oracle_decode_one(w, lengths, K, V, KI, q_h, qI_h, 0, indexer, kv)
     times = [el]
     t_end = time.time() + max(0.0, budget_s - el)
     while time.time() < t_end and len(times) < 8:
         t1 = time.perf_counter()
-        oracle_query(w, cs, q_h[0], qI_h[0], int(lengths[0]), indexer)
+        oracle_query(w, cs, q_h[0], qI_h[0], int(lengths[0]), indexer, kv)
         times.append(time.perf_counter() - t1)
     return {"value": len(times) / sum(times), "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"{len(times)} decode token(s) of sequence 0 ({int(lengths[0])} tokens of context) on the "
                       f"single-threaded fp64 C oracle, caches pre-built by the oracle ({setup:.1f} s, untimed)"}, cs
 
 
-def cpu_baseline_all_cores(w, lengths, K, V, KI, q_h, qI_h, cs=None, budget_s=10.0, indexer="bf16"):
+def cpu_baseline_all_cores(w, lengths, K, V, KI, q_h, qI_h, cs=None, budget_s=10.0, indexer="bf16", kv="workload"):
     """The same oracle on every host core: independent decode tokens of
     sequence 0 in parallel threads (the C oracle releases the GIL and keeps no
     shared state), tokens over wall time."""
@@ -635,8 +666,11 @@ def cpu_baseline_all_cores(w, lengths, K, V, KI, q_h, qI_h, cs=None, budget_s=10
     if indexer != "bf16" and not hasattr(cs, "mx"):
         cs.mx = O.mxfp4_quantize(cs.cidx)
 
+    if kv == "mixed" and not hasattr(cs, "mixed"):
+        oracle_query(w, cs, q_h[0], qI_h[0], 0, indexer, kv)
+
     def one(_):
-        oracle_query(w, cs, q_h[0], qI_h[0], int(lengths[0]), indexer)
+        oracle_query(w, cs, q_h[0], qI_h[0], int(lengths[0]), indexer, kv)
 
     with cf.ThreadPoolExecutor(cores) as ex:
         list(ex.map(one, range(cores)))  # warm-up round
@@ -702,8 +736,10 @@ def run_reference(args, w, rank, world):
             cs[b] = O.CompressedSeq(K[b, :Lb], V[b, :Lb], KI[b, :Lb], m_csa=w.m_csa, m_hca=w.m_hca, fp8=w.fp8)
             if args.indexer != "bf16":
                 cs[b].mx = O.mxfp4_quantize(cs[b].cidx)
+            if args.kv == "mixed":
+                oracle_query(w, cs[b], q_h[b], qI_h[b], 0, args.indexer, args.kv)
         t1 = time.perf_counter()
-        oracle_query(w, cs[b], q_h[b], qI_h[b], int(lengths[b]), args.indexer)
+        oracle_query(w, cs[b], q_h[b], qI_h[b], int(lengths[b]), args.indexer, args.kv)
         el = time.perf_counter() - t1
         if i >= args.warmup:
             times.append(el)
@@ -715,7 +751,7 @@ def run_reference(args, w, rank, world):
             "warmup": args.warmup, "ms_per_step": total / len(times) * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": w.name, "B_per_gpu": w.B, "context": int(w.L), "heads": w.H, "topk": w.topk,
-                       "indexer": args.indexer},
+                       "indexer": args.indexer, "kv": args.kv},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -731,14 +767,16 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--indexer", default="bf16", choices=["bf16", "mxfp4"],
                     help="decode only: the CSA indexer keys in bf16 (the workload) or FP4 (MXFP4)")
+    ap.add_argument("--kv", default="workload", choices=["workload", "mixed"],
+                    help="decode only: the workload's KV storage, or mixed storage (rotary dims bf16, the rest e4m3)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="prefill only: a shorter sequence than the workload's (small cases for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = configs.BY_NAME[args.workload]
-    if args.indexer != "bf16" and w.mode != "decode":
-        ap.error("--indexer applies to decode workloads")
+    if (args.indexer != "bf16" or args.kv != "workload") and w.mode != "decode":
+        ap.error("--indexer and --kv apply to decode workloads")
     if args.tokens:
         if w.mode != "prefill":
             ap.error("--tokens applies to prefill workloads")

@@ -60,3 +60,17 @@ def test_mxfp4_indexer_bytes():
     assert score4 == w.B * nc * (34 + 4) == 39_845_888
     assert step16 - step4 == w.B * nc * (128 - 34)
     assert step4 == 56_820_224
+
+
+def test_mixed_kv_bytes_term_by_term():
+    """Mixed storage: a K + V entry is 192 + 128 bytes, with a K and a V scale
+    (4 bytes each) per gathered entry and per 64 HCA entries."""
+    w = configs.BY_NAME["decode_b1_t4k_h8_k64"]
+    lengths = np.array([4096])
+    step, score = bench.decode_bytes(w, lengths, kv="mixed")
+    nc, nh, sel = 1024, 32, 64
+    ref = nc * 128 + sel * (192 + 128) + sel * 8 + nh * (192 + 128) + 8 + w.H * 256 + 128 + 2 * w.H * 256
+    assert step == ref == 168_584
+    assert score == nc * (128 + 4)  # the indexer is unchanged
+    step4, score4 = bench.decode_bytes(w, lengths, "mxfp4", "mixed")
+    assert step4 == ref - nc * (128 - 34) and score4 == nc * 38
