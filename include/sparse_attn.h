@@ -113,7 +113,8 @@ typedef enum {
     SA_OP_HYBRID_DECODE = 4,
     SA_OP_HYBRID_PREFILL = 5,
     SA_OP_WINDOW_ATTN = 6,  /* k = the window */
-    SA_OP_CP_CANDIDATES = 7 /* cp_decode_candidates (Tq = 1) */
+    SA_OP_CP_CANDIDATES = 7, /* cp_decode_candidates (Tq = 1) */
+    SA_OP_HYBRID_DECODE_SWA = 8 /* hybrid_attn_decode_swa (Tq = 1; any window) */
 } sa_op;
 
 /* Compression, section 3-2 (2) component table, CSA row ("every 4 tokens ->
@@ -233,6 +234,23 @@ sa_status hybrid_attn_decode(const void* q, const void* q_idx, int32_t H,
                              void* out_csa, void* out_hca, float* lse_csa, float* lse_hca,
                              int32_t* idx_out, int32_t* cnt_out,
                              void* ws, size_t ws_bytes, void* stream);
+
+/* hybrid_attn_decode with the sliding-window branch of both layers: the
+ * review (section 3-2 (2)) adds a window of recent uncompressed tokens to CSA
+ * and to HCA alike.  out_csa is the attention over the CSA selection joined
+ * with the last `window` raw tokens, out_hca over the HCA entries joined with
+ * the same window (one softmax over each union: the log-sum-exp merge of the
+ * branch and the window, as attn_lse_merge computes it).
+ *   raw: the raw tokens (k, v [B][Lcap][d] bf16, len [B]) as for swa_attn;
+ *        its B must equal the caches'.
+ *   lse_csa / lse_hca: the lse of each union, or NULL.
+ * ws / ws_bytes: at least sa_workspace_size(SA_OP_HYBRID_DECODE_SWA, B, 1, H,
+ * Ncap_csa, Ncap_hca, k) (independent of the window).                      */
+sa_status hybrid_attn_decode_swa(const void* q, const void* q_idx, int32_t H,
+                                 const sa_cache* csa, const sa_cache* hca, const sa_raw* raw, int32_t window,
+                                 int32_t k, float scale, void* out_csa, void* out_hca, float* lse_csa,
+                                 float* lse_hca, int32_t* idx_out, int32_t* cnt_out,
+                                 void* ws, size_t ws_bytes, void* stream);
 
 /* hybrid_attn_decode with the CSA selection on FP4 indexer scores (the
  * selection of csa_index_topk_mxfp4; codes / scales as written by

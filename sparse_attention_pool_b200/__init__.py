@@ -5,10 +5,11 @@ into its C ABI and ``synth`` only generates seeded inputs.
 """
 from .api import (Cache, CapturedDecode, alloc_cache, alloc_workspace, attn_lse_merge, csa_append, csa_compress,  # noqa: F401
                   csa_index_topk, csa_index_topk_noalloc, hca_append, swa_attn,
-                  csa_index_quantize_mxfp4, csa_index_topk_mxfp4, hybrid_attn_decode_mxfp4,
+                  csa_index_quantize_mxfp4, csa_index_topk_mxfp4, hybrid_attn_decode_mxfp4, hybrid_attn_decode_swa,
                   cp_decode_candidates, cp_decode_merge_select, attn_lse_merge_n,
                   csa_sparse_attn,
                   hca_compress, hca_dense_attn, hybrid_attn_decode, hybrid_attn_prefill, read_device_status,
                   workspace_size)
 from ._lib import (SA_OP_DENSE_ATTN, SA_OP_HYBRID_DECODE, SA_OP_HYBRID_PREFILL, SA_OP_INDEX_TOPK,  # noqa: F401
-                   SA_OP_SPARSE_ATTN, SA_OP_WINDOW_ATTN, SA_OP_CP_CANDIDATES, SparseAttnError)
+                   SA_OP_SPARSE_ATTN, SA_OP_WINDOW_ATTN, SA_OP_CP_CANDIDATES,
+                   SA_OP_HYBRID_DECODE_SWA, SparseAttnError)

@@ -14,6 +14,7 @@ SA_BF16, SA_FP8_E4M3, SA_KV_MIXED = 0, 1, 2
 SA_OP_INDEX_TOPK, SA_OP_SPARSE_ATTN, SA_OP_DENSE_ATTN, SA_OP_HYBRID_DECODE, SA_OP_HYBRID_PREFILL = 1, 2, 3, 4, 5
 SA_OP_WINDOW_ATTN = 6
 SA_OP_CP_CANDIDATES = 7
+SA_OP_HYBRID_DECODE_SWA = 8
 
 STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3: "SA_ERR_WORKSPACE",
                 4: "SA_ERR_CUDA", 5: "SA_ERR_TIMEOUT", 6: "SA_ERR_DEVICE"}
@@ -24,7 +25,7 @@ EXPORTS = ["csa_compress", "hca_compress", "csa_index_topk", "csa_sparse_attn", 
            "sa_last_error", "sa_abi_version", "sa_set_stage_events", "sa_launch_count",
            "csa_index_topk_noalloc", "csa_append", "hca_append", "swa_attn", "attn_lse_merge",
            "csa_index_quantize_mxfp4", "csa_index_topk_mxfp4", "hybrid_attn_decode_mxfp4",
-           "cp_decode_candidates", "cp_decode_merge_select", "attn_lse_merge_n"]
+           "cp_decode_candidates", "cp_decode_merge_select", "attn_lse_merge_n", "hybrid_attn_decode_swa"]
 SA_NOALLOC_SCRATCH_BYTES = 32 << 20
 SA_STAGE_INDEX_SCORE, SA_STAGE_TOPK_SELECT, SA_STAGE_CSA_ATTN, SA_STAGE_HCA_ATTN = 0, 1, 2, 3
 
@@ -78,6 +79,7 @@ def lib():
         L.cp_decode_candidates.argtypes = [P, CP, I32, P, P, P, P, P, SZ, P]
         L.cp_decode_merge_select.argtypes = [P, P, P, I32, I32, I32, I32, P, P, P, P, P, P]
         L.attn_lse_merge_n.argtypes = [P, P, I32, ctypes.c_int64, P, P, P]
+        L.hybrid_attn_decode_swa.argtypes = [P, P, I32, CP, CP, RP, I32, I32, F32, P, P, P, P, P, P, P, SZ, P]
         L.hybrid_attn_decode_mxfp4.argtypes = [P, P, I32, CP, CP, P, P, I32, F32, P, P, P, P, P, P, P, SZ, P]
         L.hybrid_attn_prefill.argtypes = [P, P, I32, I32, CP, CP, I32, F32, P, P, P, P, P, P, P, SZ, P]
         L.sa_workspace_size.argtypes = [I32, I32, I32, I32, I32, I32, I32]

@@ -317,6 +317,27 @@ def hybrid_attn_decode(q, q_idx, csa: Cache, hca: Cache, k: int, ws, *, scale=0.
     return out_csa, out_hca
 
 
+def hybrid_attn_decode_swa(q, q_idx, csa: Cache, hca: Cache, k_raw, v_raw, lengths, window: int, k: int, ws, *,
+                           scale=0.0, out_csa=None, out_hca=None, lse_csa=None, lse_hca=None, idx_out=None,
+                           cnt_out=None, stream=None):
+    """hybrid_attn_decode with the sliding-window branch of both layers: each
+    output is the attention over its branch joined with the last `window` raw
+    tokens (k_raw, v_raw [B][Lcap][128] bf16, lengths [B] int32)."""
+    _need(q, torch.bfloat16, "q")
+    _need(q_idx, torch.bfloat16, "q_idx")
+    H = q.shape[1]
+    out_csa = torch.empty_like(q) if out_csa is None else out_csa
+    out_hca = torch.empty_like(q) if out_hca is None else out_hca
+    raw = _raw(k_raw, v_raw, None, lengths)
+    c, h = csa.struct(), hca.struct()
+    check("hybrid_attn_decode_swa",
+          lib().hybrid_attn_decode_swa(_ptr(q), _ptr(q_idx), H, ctypes.byref(c), ctypes.byref(h), ctypes.byref(raw),
+                                       int(window), k, float(scale), _ptr(out_csa), _ptr(out_hca), _ptr(lse_csa),
+                                       _ptr(lse_hca), _ptr(idx_out), _ptr(cnt_out), _ptr(ws), ws.numel(),
+                                       _stream(stream)))
+    return out_csa, out_hca
+
+
 def hybrid_attn_decode_mxfp4(q, q_idx, csa: Cache, hca: Cache, codes, scales, k: int, ws, *, scale=0.0,
                              out_csa=None, out_hca=None, lse_csa=None, lse_hca=None, idx_out=None, cnt_out=None,
                              stream=None):

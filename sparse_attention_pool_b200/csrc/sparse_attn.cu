@@ -278,6 +278,15 @@ TopkDecodeWs topk_decode_layout(int B, int Ncap, int k, bool own_idx) {
     return w;
 }
 
+// Workspace of hybrid_attn_decode_swa: the hybrid step's, then the window
+// attention's (partials for the most splits a decode list takes, so the size
+// does not depend on the window), the window's output and lse, and the two
+// branches' lse when the caller keeps none.
+struct SwaDecodeWs {
+    size_t hybrid, win_ws, win_out, win_lse, lse_c, lse_h, total;
+};
+SwaDecodeWs swa_decode_layout(int B, int H, int Ncap_csa, int Ncap_hca, int k);
+
 // Split rule of the attention kernels: depends only on the list capacity, never
 // on the batch, so a sequence's result does not depend on its batch-mates.
 struct Split {
@@ -295,6 +304,31 @@ Split attn_split(int rows_cap, bool prefill, bool gather = false) {
 size_t attn_partial_bytes(long long BQ, int splits, int H) {
     if (splits <= 1) return 0;
     return up256((size_t)BQ * splits * H * 128 * 4) + up256((size_t)BQ * splits * H * 4);
+}
+
+size_t hybrid_decode_bytes(int B, int H, int Ncap_csa, int Ncap_hca, int k) {
+    TopkDecodeWs w = topk_decode_layout(B, Ncap_csa, k, true);
+    Split sc = attn_split(k, false, true), sh = attn_split(Ncap_hca, false);
+    return w.total + attn_partial_bytes(B, sc.splits, H) + attn_partial_bytes(B, sh.splits, H);
+}
+
+SwaDecodeWs swa_decode_layout(int B, int H, int Ncap_csa, int Ncap_hca, int k) {
+    SwaDecodeWs w{};
+    size_t o = up256(hybrid_decode_bytes(B, H, Ncap_csa, Ncap_hca, k));
+    w.hybrid = o;
+    w.win_ws = o;
+    o += 256 + attn_partial_bytes(B, 32, H);  // decode lists take at most 32 splits
+    o = up256(o);
+    w.win_out = o;
+    o += up256((size_t)B * H * 128 * 2);
+    w.win_lse = o;
+    o += up256((size_t)B * H * 4);
+    w.lse_c = o;
+    o += up256((size_t)B * H * 4);
+    w.lse_h = o;
+    o += up256((size_t)B * H * 4);
+    w.total = o;
+    return w;
 }
 
 // ------------------------------------------------------------ launchers ----
@@ -849,9 +883,7 @@ size_t sa_workspace_size(int32_t op, int32_t B, int32_t Tq, int32_t H, int32_t N
         }
         case SA_OP_HYBRID_DECODE: {
             if (k < 1 || Tq != 1) return 0;
-            TopkDecodeWs w = topk_decode_layout(B, Ncap_csa, k, true);
-            Split sc = attn_split(k, false, true), sh = attn_split(Ncap_hca, false);
-            return w.total + attn_partial_bytes(BQ, sc.splits, H) + attn_partial_bytes(BQ, sh.splits, H);
+            return hybrid_decode_bytes(B, H, Ncap_csa, Ncap_hca, k);
         }
         case SA_OP_HYBRID_PREFILL:
             if (k < 1) return 0;
@@ -864,6 +896,9 @@ size_t sa_workspace_size(int32_t op, int32_t B, int32_t Tq, int32_t H, int32_t N
         case SA_OP_CP_CANDIDATES:
             if (k < 1 || Tq != 1) return 0;
             return topk_decode_layout(B, Ncap_csa, k, true).total;
+        case SA_OP_HYBRID_DECODE_SWA:
+            if (k < 1 || Tq != 1) return 0;
+            return swa_decode_layout(B, H, Ncap_csa, Ncap_hca, k).total;
         default:
             return 0;
     }
@@ -1166,6 +1201,36 @@ sa_status hybrid_attn_decode(const void* q, const void* q_idx, int32_t H, const 
                              int32_t* idx_out, int32_t* cnt_out, void* ws, size_t ws_bytes, void* stream) {
     return hybrid_decode_impl("hybrid_attn_decode", q, q_idx, H, csa, hca, nullptr, nullptr, k, scale, out_csa,
                               out_hca, lse_csa, lse_hca, idx_out, cnt_out, ws, ws_bytes, stream);
+}
+
+sa_status hybrid_attn_decode_swa(const void* q, const void* q_idx, int32_t H, const sa_cache* csa,
+                                 const sa_cache* hca, const sa_raw* raw, int32_t window, int32_t k, float scale,
+                                 void* out_csa, void* out_hca, float* lse_csa, float* lse_hca, int32_t* idx_out,
+                                 int32_t* cnt_out, void* ws, size_t ws_bytes, void* stream) {
+    SA_CHECK(csa != nullptr && hca != nullptr, "hybrid_attn_decode_swa: cache descriptors must be non-NULL");
+    SA_CHECK(raw != nullptr, "hybrid_attn_decode_swa: raw descriptor is NULL");
+    SA_CHECK(raw->B == csa->B, "hybrid_attn_decode_swa: raw B=%d != csa B=%d", raw->B, csa->B);
+    SA_CHECK(window >= 1, "hybrid_attn_decode_swa: window=%d", window);
+    SA_CHECK(H >= 1 && H <= 128, "hybrid_attn_decode_swa: H=%d outside 1..128", H);
+    SA_CHECK(k >= 1 && k <= 65536, "hybrid_attn_decode_swa: k=%d outside 1..65536", k);
+    const SwaDecodeWs w = swa_decode_layout(csa->B, H, csa->Ncap, hca->Ncap, k);
+    sa_status r = check_ws(ws, ws_bytes, w.total);
+    if (r != SA_OK) return r;
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    float* lc = lse_csa ? lse_csa : reinterpret_cast<float*>(base + w.lse_c);
+    float* lh = lse_hca ? lse_hca : reinterpret_cast<float*>(base + w.lse_h);
+    r = hybrid_decode_impl("hybrid_attn_decode_swa", q, q_idx, H, csa, hca, nullptr, nullptr, k, scale, out_csa,
+                           out_hca, lc, lh, idx_out, cnt_out, ws, w.win_ws, stream);
+    if (r != SA_OK) return r;
+    // the window over the raw tokens, once for both layers, then one merge each
+    void* wo = base + w.win_out;
+    float* wl = reinterpret_cast<float*>(base + w.win_lse);
+    r = swa_attn(q, 1, H, nullptr, raw, window, scale, wo, wl, base + w.win_ws, w.win_out - w.win_ws, stream);
+    if (r != SA_OK) return r;
+    const int64_t rows = (int64_t)csa->B * H;
+    r = attn_lse_merge(out_csa, lc, wo, wl, rows, out_csa, lc, stream);
+    if (r != SA_OK) return r;
+    return attn_lse_merge(out_hca, lh, wo, wl, rows, out_hca, lh, stream);
 }
 
 sa_status hybrid_attn_decode_mxfp4(const void* q, const void* q_idx, int32_t H, const sa_cache* csa,

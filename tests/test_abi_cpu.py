@@ -228,3 +228,24 @@ def test_context_parallel_entry_points_reject_bad_arguments(L):
     assert mn(P(FAKE), P(FAKE), 2, 0, P(FAKE), None, None) == 0  # nothing to do
     assert L.sa_workspace_size(7, 2, 1, 64, 262144, 0, 2048) > 0
     assert L.sa_workspace_size(7, 2, 2, 64, 262144, 0, 2048) == 0  # decode only
+
+
+def test_hybrid_decode_swa_rejects_bad_arguments(L):
+    c, h, r = _cache(), _cache(m=128, kidx=None), _raw()
+    P = ctypes.c_void_p
+    f = L.hybrid_attn_decode_swa
+    tail = [P(FAKE), P(FAKE), None, None, None, None, P(FAKE), 1 << 30, None]
+    assert f(P(FAKE), P(FAKE), 8, ctypes.byref(c), ctypes.byref(h), None, 64, 8, 0.0, *tail) == 1
+    assert "raw" in L.sa_last_error().decode()
+    assert f(P(FAKE), P(FAKE), 8, ctypes.byref(c), ctypes.byref(h), ctypes.byref(r), 0, 8, 0.0, *tail) == 1
+    assert "window" in L.sa_last_error().decode()
+    r2 = _raw(B=2)
+    assert f(P(FAKE), P(FAKE), 8, ctypes.byref(c), ctypes.byref(h), ctypes.byref(r2), 64, 8, 0.0, *tail) == 1
+    assert "B=" in L.sa_last_error().decode()
+    small = [P(FAKE), P(FAKE), None, None, None, None, P(FAKE), 16, None]
+    assert f(P(FAKE), P(FAKE), 8, ctypes.byref(c), ctypes.byref(h), ctypes.byref(r), 64, 8, 0.0, *small) == \
+        _lib.SA_ERR_WORKSPACE
+    ws = L.sa_workspace_size
+    # the window-inclusive step needs more than the plain one, whatever the window
+    assert ws(8, 4, 1, 64, 262144, 8192, 2048) > ws(4, 4, 1, 64, 262144, 8192, 2048) > 0
+    assert ws(8, 4, 2, 64, 262144, 8192, 2048) == 0
