@@ -288,6 +288,15 @@ size_t sa_workspace_size(int32_t op, int32_t B, int32_t Tq, int32_t H,
  * SA_ERR_TIMEOUT or SA_ERR_DEVICE.                                           */
 sa_status sa_read_device_status(void* stream);
 
+/* Failure-detection self-test.  Every cross-CTA wait in the library is
+ * bounded: a wait that runs out records a timeout in the device status word
+ * and its kernel returns instead of hanging or trapping.  This launches one
+ * small kernel whose wait on a barrier that nothing completes gives up after
+ * wait_tries polls (1..4194304; 65536 takes well under a second); the next
+ * sa_read_device_status then returns SA_ERR_TIMEOUT, and the context stays
+ * usable.  A diagnostic only: the method has no counterpart.               */
+sa_status sa_selftest_wait_timeout(uint32_t wait_tries, void* stream);
+
 /* Text for the last non-OK status returned on the calling host thread.      */
 const char* sa_last_error(void);
 

@@ -25,7 +25,8 @@ EXPORTS = ["csa_compress", "hca_compress", "csa_index_topk", "csa_sparse_attn", 
            "sa_last_error", "sa_abi_version", "sa_set_stage_events", "sa_launch_count",
            "csa_index_topk_noalloc", "csa_append", "hca_append", "swa_attn", "attn_lse_merge",
            "csa_index_quantize_mxfp4", "csa_index_topk_mxfp4", "hybrid_attn_decode_mxfp4",
-           "cp_decode_candidates", "cp_decode_merge_select", "attn_lse_merge_n", "hybrid_attn_decode_swa"]
+           "cp_decode_candidates", "cp_decode_merge_select", "attn_lse_merge_n", "hybrid_attn_decode_swa",
+           "sa_selftest_wait_timeout"]
 SA_NOALLOC_SCRATCH_BYTES = 32 << 20
 SA_STAGE_INDEX_SCORE, SA_STAGE_TOPK_SELECT, SA_STAGE_CSA_ATTN, SA_STAGE_HCA_ATTN = 0, 1, 2, 3
 
@@ -90,6 +91,7 @@ def lib():
         L.sa_abi_version.argtypes = []
         L.sa_abi_version.restype = I32
         L.sa_set_stage_events.argtypes = [I32, P, P]
+        L.sa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, P]
         L.sa_launch_count.argtypes = []
         L.sa_launch_count.restype = ctypes.c_uint64
         for name in EXPORTS:

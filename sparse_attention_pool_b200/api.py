@@ -380,6 +380,12 @@ def read_device_status(stream=None):
     check("sa_read_device_status", lib().sa_read_device_status(_stream(stream)))
 
 
+def selftest_wait_timeout(wait_tries: int = 65536, stream=None):
+    """Launch the failure-detection self-test (a bounded wait that cannot
+    complete); the next read_device_status raises SA_ERR_TIMEOUT."""
+    check("sa_selftest_wait_timeout", lib().sa_selftest_wait_timeout(int(wait_tries), _stream(stream)))
+
+
 class CapturedDecode:
     """A hybrid decode step captured once into a CUDA graph, for serving loops
     that decode the same batch step after step.

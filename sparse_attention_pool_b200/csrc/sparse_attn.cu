@@ -708,6 +708,22 @@ sa_status noalloc_scratch(void** out) {
 
 }  // namespace
 
+namespace sa {
+// Failure-detection self-test: one CTA waits on an mbarrier that nothing
+// arrives at.  The bounded wait gives up after `limit` tries, records
+// DEV_TIMEOUT in the status word and returns; no copy is in flight, so the
+// CTA exits cleanly and the context stays usable.
+__global__ void selftest_wait_kernel(uint32_t limit) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, limit);
+}
+}  // namespace sa
+
 // =========================================================== public ABI ====
 extern "C" {
 
@@ -724,6 +740,14 @@ sa_status sa_set_stage_events(int32_t stage, void* before, void* after) {
 }
 
 const char* sa_last_error(void) { return g_err; }
+
+sa_status sa_selftest_wait_timeout(uint32_t wait_tries, void* stream) {
+    SA_CHECK(wait_tries >= 1 && wait_tries <= sa::kWaitLimit, "sa_selftest_wait_timeout: wait_tries=%u outside 1..%u",
+             wait_tries, sa::kWaitLimit);
+    sa::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(wait_tries);
+    SA_LAUNCHED();
+    return SA_OK;
+}
 
 static sa_status check_common_q(const void* q, int H, const char* what);
 

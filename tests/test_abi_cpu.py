@@ -249,3 +249,9 @@ def test_hybrid_decode_swa_rejects_bad_arguments(L):
     # the window-inclusive step needs more than the plain one, whatever the window
     assert ws(8, 4, 1, 64, 262144, 8192, 2048) > ws(4, 4, 1, 64, 262144, 8192, 2048) > 0
     assert ws(8, 4, 2, 64, 262144, 8192, 2048) == 0
+
+
+def test_selftest_rejects_bad_arguments(L):
+    assert L.sa_selftest_wait_timeout(0, None) == _lib.SA_ERR_INVALID_ARG
+    assert L.sa_selftest_wait_timeout((1 << 22) + 1, None) == _lib.SA_ERR_INVALID_ARG
+    assert "wait_tries" in L.sa_last_error().decode()
