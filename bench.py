@@ -187,6 +187,51 @@ def decode_bytes(w, lengths, indexer="bf16", kv="workload"):
     return step, score
 
 
+def compress_bytes(w, lengths, kv="workload"):
+    """Algorithmic HBM bytes of compressing the raw tokens once: (CSA, HCA),
+    each the complete blocks' raw K, V (+ indexer keys for CSA) read once and
+    the entries (+ fp8 scales per 64 entries) written once."""
+    fp8 = w.fp8 or kv == "mixed"
+    kv_entry = 320 if kv == "mixed" else 2 * 128 * (1 if w.fp8 else 2)
+    csa = hca = 0
+    for L in lengths:
+        nc, nh = int(L) // w.m_csa, int(L) // w.m_hca
+        csa += nc * w.m_csa * (128 + 128 + 64) * 2 + nc * (kv_entry + 128)
+        hca += nh * w.m_hca * (128 + 128) * 2 + nh * kv_entry
+        if fp8:
+            csa += ((nc + 63) // 64) * 8
+            hca += ((nh + 63) // 64) * 8
+    return csa, hca
+
+
+def time_compress(S, w, lengths, Kd, Vd, KId, lens, csa, hca, kv, reps=5):
+    """CUDA-event time of csa_compress and hca_compress over the bench's raw
+    tokens (inputs far larger than L2), after two warm-up calls each."""
+    import torch
+    stream = torch.cuda.current_stream()
+    out = {}
+    for name, fn in (("csa", lambda: S.csa_compress(Kd, Vd, KId, lens, csa)),
+                     ("hca", lambda: S.hca_compress(Kd, Vd, lens, hca))):
+        fn()
+        fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        e1.synchronize()
+        out[name + "_ms"] = e0.elapsed_time(e1) / reps
+    S.read_device_status()
+    cb, hb = compress_bytes(w, lengths, kv)
+    peak, kind = measured_peaks()
+    out["csa_bytes"], out["hca_bytes"] = cb, hb
+    out["csa_gbs"] = cb / (out["csa_ms"] / 1e3) / 1e9
+    out["hca_gbs"] = hb / (out["hca_ms"] / 1e3) / 1e9
+    out["csa_frac"], out["hca_frac"] = out["csa_gbs"] / peak, out["hca_gbs"] / peak
+    out["peak_gbs"], out["peak_kind"] = peak, kind
+    return out
+
+
 def max_over_ranks(ms, world, device):
     """The job's time is the slowest rank's: every rank calls this at the same point."""
     if world == 1:
@@ -244,6 +289,10 @@ def run_ours(args, w, rank, world, dev):
     fp4 = args.indexer == "mxfp4"
     codes4, scales4 = S.csa_index_quantize_mxfp4(csa) if fp4 else (None, None)  # like compression: untimed
     torch.cuda.synchronize()
+    try:  # compression on its own (recompressing gives the same caches)
+        compress_info = time_compress(S, w, lengths, Kd, Vd, KId, lens, csa, hca, args.kv)
+    except Exception as ex:  # noqa: BLE001 -- recorded in the JSON line
+        compress_info = {"error": str(ex)[:160]}
     del Kd, Vd, KId
     torch.cuda.empty_cache()
     q = to_bf16_tensor(q_h, dev)
@@ -451,6 +500,7 @@ def run_ours(args, w, rank, world, dev):
                      "bytes_per_launch": score_bytes, "avg_launch_ms": score_avg,
                      "traffic": None if fp4 else recorded_traffic("score_decode_kernel", w.name)},
         "stages_ms": {n: statistics.mean(v) for n, v in zip(stage_names, stage_ms)},
+        "compress": compress_info,
         "staged_step_ms": statistics.mean(staged_ms),
         "gpu_launches": launches_per_step * args.steps,
         "e2e": {"value": job_throughput(B * args.steps, world, e2e_total), "unit": "tokens/s", "h2d_bytes_per_step": h2d,

@@ -74,3 +74,18 @@ def test_mixed_kv_bytes_term_by_term():
     assert score == nc * (128 + 4)  # the indexer is unchanged
     step4, score4 = bench.decode_bytes(w, lengths, "mxfp4", "mixed")
     assert step4 == ref - nc * (128 - 34) and score4 == nc * 38
+
+
+def test_compress_bytes_match_the_worked_figures():
+    """1M-token decode workload: CSA reads 4 x 1M x (512 + 128) B of raw K, V and
+    indexer keys and writes 4 x 262,144 x 640 B of entries; HCA reads the raw
+    K and V of 4 x 8192 blocks and writes 4 x 8192 x 512 B."""
+    w = configs.BY_NAME["decode_b4_t1m_h64_k2048"]
+    csa, hca = bench.compress_bytes(w, np.full((w.B,), w.L))
+    assert csa == 4 * (1 << 20) * 640 + 4 * 262144 * 640 == 3_355_443_200
+    assert hca == 4 * 8192 * 128 * 512 + 4 * 8192 * 512 == 2_164_260_864
+    wf = configs.BY_NAME["ragged_fp8_b32_t64k-256k_h64_k1024"]
+    c8, h8 = bench.compress_bytes(wf, np.array([65536 + 5]))
+    nc, nh = 16385, 512
+    assert c8 == nc * 4 * 640 + nc * (256 + 128) + ((nc + 63) // 64) * 8
+    assert h8 == nh * 128 * 512 + nh * 256 + ((nh + 63) // 64) * 8
