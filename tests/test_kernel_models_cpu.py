@@ -1,0 +1,218 @@
+"""Models, on the CPU, of the integer and bit-level schemes two kernels rely
+on, checked against the oracle and against plain sorting:
+
+* the FP4 indexer (mxfp4_quantize_kernel, score_decode_mxfp4_kernel): the
+  e2m1 encoder by threshold compares, the E8M0 exponent from the fp32 bit
+  pattern, the doubled-magnitude byte table picked by a byte permute, the
+  sign applied by selecting +q or -q bytes, dp4a accumulation and the
+  per-block exponent offsets -- the model's codes, scales and scores must
+  equal the oracle's bit for bit;
+* the context-parallel merge (cp_merge_select_kernel): rank-major candidate
+  offsets, the cut "key > T or (key == T and index <= jmax)" at the k-th
+  largest, and ordered compaction by block scans in chunks of the CTA --
+  the model's global selection and per-rank shares must equal sorting.
+
+The models restate the kernels' schemes in Python; the CUDA kernels
+themselves are checked against the oracle by the GPU tests.
+"""
+from __future__ import annotations
+
+import math
+import struct
+
+import numpy as np
+
+from oracle import oracle as O
+
+
+# -- FP4 indexer ----------------------------------------------------------------
+
+def _f2u(x) -> int:
+    return struct.unpack("<I", struct.pack("<f", float(np.float32(x))))[0]
+
+
+def _u2f(u: int):
+    return np.float32(struct.unpack("<f", struct.pack("<I", u & 0xFFFFFFFF))[0])
+
+
+def _byte_perm(x: int, y: int, s: int) -> int:
+    """CUDA __byte_perm: bytes 0-3 from x, 4-7 from y; selector nibble j's
+    low three bits pick output byte j."""
+    b = [(x >> (8 * i)) & 0xFF for i in range(4)] + [(y >> (8 * i)) & 0xFF for i in range(4)]
+    return sum(b[(s >> (4 * j)) & 7] << (8 * j) for j in range(4))
+
+
+def _dp4a(a: int, b: int, c: int) -> int:
+    def s8(v):
+        return v - 256 if v >= 128 else v
+    return c + sum(s8((a >> (8 * i)) & 0xFF) * s8((b >> (8 * i)) & 0xFF) for i in range(4))
+
+
+def _e2m1_code(y) -> int:
+    y = np.float32(y)
+    a = abs(y)
+    c = sum(int(v) for v in (a > 0.25, a >= 0.75, a > 1.25, a >= 1.75, a > 2.5, a >= 3.5, a > 5))
+    if a != a:
+        c = 7
+    return c | ((_f2u(y) >> 28) & 8)
+
+
+def _scale_exp(amax) -> int:
+    if not amax > 0:
+        return -127
+    u = _f2u(amax)
+    e = (u >> 23) & 0xFF
+    fl = e - 127 if e else ((u & 0x7FFFFF).bit_length() - 1) - 149
+    return min(127, max(-127, fl - 2))
+
+
+def _inv_scale(se: int):
+    return _u2f((127 - se) << 23) if 127 - se <= 254 else _u2f(0x00400000)
+
+
+LUT_LO, LUT_HI = 0x03020100, 0x0C080604  # doubled e2m1 magnitudes 0 1 2 3 | 4 6 8 12
+
+
+def _bf16(bits) -> np.float32:
+    return _u2f(int(bits) << 16)
+
+
+def _model_quantize_row(row):
+    codes, scales = bytearray(32), []
+    for blk in range(2):
+        w = row[32 * blk:32 * blk + 32]
+        amax = max((abs(_bf16(v)) for v in w), default=np.float32(0))
+        se = _scale_exp(np.float32(amax))
+        inv = _inv_scale(se)
+        for i in range(16):
+            lo = _e2m1_code(np.float32(_bf16(w[2 * i]) * inv))
+            hi = _e2m1_code(np.float32(_bf16(w[2 * i + 1]) * inv))
+            codes[16 * blk + i] = lo | (hi << 4)
+        scales.append(se + 127)
+    return bytes(codes), scales
+
+
+def _model_query(qbits):
+    qp, qn, qe = [0] * 16, [0] * 16, [0, 0]
+    vals = [_bf16(b) for b in qbits]
+    for blk in range(2):
+        se = _scale_exp(np.float32(max(abs(v) for v in vals[32 * blk:32 * blk + 32])))
+        inv = _inv_scale(se)
+        qe[blk] = se + 127
+        for e in range(32 * blk, 32 * blk + 32):
+            c = _e2m1_code(np.float32(vals[e] * inv))
+            v = (_byte_perm(LUT_LO, LUT_HI, c & 7) & 0xFF) * (-1 if c & 8 else 1)
+            qp[e // 4] |= (v & 0xFF) << (8 * (e % 4))
+            qn[e // 4] |= ((-v) & 0xFF) << (8 * (e % 4))
+    return qp, qn, qe
+
+
+def _model_score(codes: bytes, sc, qp, qn, qe):
+    w = struct.unpack("<8I", codes)
+
+    def dot8(x, a, b, c, d, acc):
+        m0 = _byte_perm(LUT_LO, LUT_HI, x & 0x7777)
+        s0 = _byte_perm(a, b, 0x3210 | ((x >> 1) & 0x4444))
+        m1 = _byte_perm(LUT_LO, LUT_HI, (x >> 16) & 0x7777)
+        s1 = _byte_perm(c, d, 0x3210 | ((x >> 17) & 0x4444))
+        return _dp4a(m1, s1, _dp4a(m0, s0, acc))
+    A = [0, 0]
+    for blk in range(2):
+        for i in range(4):
+            m = 8 * blk + 2 * i
+            A[blk] = dot8(w[4 * blk + i], qp[m], qn[m], qp[m + 1], qn[m + 1], A[blk])
+    t = [np.float32(math.ldexp(A[blk], int(sc[blk]) + int(qe[blk]) - 254 - 2)) for blk in range(2)]
+    s = np.float32(t[0] + t[1])
+    return np.float32(0) if s == 0 else s
+
+
+def test_fp4_kernel_scheme_matches_the_oracle_bit_for_bit():
+    rng = np.random.default_rng(3)
+    n = 300
+    x = rng.standard_normal((n, 64)).astype(np.float32)
+    x[5] *= 1e-30
+    x[6] *= 1e30
+    x[7, :32] = 0
+    x[8, 3] = -0.0
+    x[9, :8] = [4.0, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, -0.25]
+    x[10, :4] = [6.0, 5.0, -5.0, 7.0]
+    xb = (x.view(np.uint32) >> 16).astype(np.uint16)
+    oc, osc = O.mxfp4_quantize(xb)
+    for j in range(n):
+        c, s = _model_quantize_row(xb[j])
+        assert c == bytes(oc[j]) and s == [int(v) for v in osc[j]], j
+    qb = (rng.standard_normal(64).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    qp, qn, qe = _model_query(qb)
+    qc, qs = O.mxfp4_quantize(qb.reshape(1, -1))
+    assert qe == [int(v) for v in qs[0]]
+    ref = O.mxfp4_index_scores(qc[0], qs[0], oc, osc)
+    for j in range(n):
+        got = _model_score(bytes(oc[j]), [int(v) for v in osc[j]], qp, qn, qe)
+        assert _f2u(got) == _f2u(ref[j]), j
+
+
+# -- context-parallel merge -----------------------------------------------------
+
+def _select_rank(keys, idx, R):
+    """The cut's contract: exactly R entries satisfy key > T or (key == T and
+    idx <= jmax)."""
+    order = sorted(range(len(keys)), key=lambda p: (-int(keys[p]), int(idx[p])))
+    T = int(keys[order[R - 1]])
+    ties = sorted(int(idx[q]) for q in range(len(keys)) if keys[q] == T)
+    rem = R - sum(1 for q in range(len(keys)) if keys[q] > T)
+    return T, (0x7FFFFFFF if rem >= len(ties) else ties[rem - 1])
+
+
+def _model_merge(keys, gidx, gcnt, W, k, rank, base, NT=1024):
+    off = [0]
+    for w in range(W):
+        off.append(off[-1] + gcnt[w])
+    C = off[W]
+    lk, li = [], []
+    for p in range(C):
+        w = 0
+        while off[w + 1] <= p:
+            w += 1
+        lk.append(keys[w][p - off[w]])
+        li.append(gidx[w][p - off[w]])
+    R = min(C, k)
+    every = C <= k
+    T, jmax = (0, 0x7FFFFFFF) if every else _select_rank(lk, li, R)
+    sel, loc, gpos, lpos = [-1] * k, [-1] * k, 0, 0
+    for p0 in range(0, C, NT):
+        win = [p0 + t < C and (every or lk[p0 + t] > T or (lk[p0 + t] == T and li[p0 + t] <= jmax))
+               for t in range(NT)]
+        mine = [win[t] and off[rank] <= p0 + t < off[rank + 1] for t in range(NT)]
+        ge, le = np.cumsum([0] + win[:-1]), np.cumsum([0] + mine[:-1])
+        for t in range(NT):
+            if win[t]:
+                sel[gpos + ge[t]] = li[p0 + t]
+            if mine[t]:
+                loc[lpos + le[t]] = li[p0 + t] - base
+        gpos += sum(win)
+        lpos += sum(mine)
+    return sel, R, loc, lpos
+
+
+def test_context_parallel_merge_scheme_matches_sorting():
+    rng = np.random.default_rng(0)
+    for trial in range(150):
+        W, k = int(rng.integers(1, 6)), int(rng.integers(1, 600))
+        sizes = [int(rng.integers(0, 1300)) for _ in range(W)]
+        bases = np.cumsum([0] + sizes[:-1])
+        nvals = int(rng.integers(1, 50))  # few distinct scores: ties at the cut are common
+        scores = [rng.integers(0, nvals, sz).astype(np.int64) + 0x80000000 for sz in sizes]
+        keys, gidx, gcnt = [], [], []
+        for w in range(W):
+            s = scores[w]
+            loc = sorted(sorted(range(len(s)), key=lambda j: (-int(s[j]), j))[:k])
+            keys.append([int(s[j]) for j in loc])
+            gidx.append([int(bases[w] + j) for j in loc])
+            gcnt.append(len(loc))
+        full = np.concatenate(scores) if sum(sizes) else np.zeros(0, np.int64)
+        want = sorted(sorted(range(len(full)), key=lambda j: (-int(full[j]), j))[:k])
+        for rank in range(W):
+            sel, R, loc, lc = _model_merge(keys, gidx, gcnt, W, k, rank, int(bases[rank]))
+            assert R == len(want) and sel[:R] == want and all(v == -1 for v in sel[R:]), trial
+            mine = [j - int(bases[rank]) for j in want if bases[rank] <= j < bases[rank] + sizes[rank]]
+            assert loc[:lc] == mine and all(v == -1 for v in loc[lc:]), trial
