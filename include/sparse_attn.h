@@ -297,6 +297,24 @@ sa_status sa_read_device_status(void* stream);
  * usable.  A diagnostic only: the method has no counterpart.               */
 sa_status sa_selftest_wait_timeout(uint32_t wait_tries, void* stream);
 
+/* Device timelines (a profiling build only).  A library compiled with
+ * -DSA_TRACE (libsparse_attn_trace.so) has per-CTA phase marks in its
+ * decode-path kernels: thread 0 of a CTA appends a 16-byte record
+ *   { uint64 t_ns (%globaltimer); uint16 kernel; uint16 phase; uint16 sm;
+ *     uint16 cta (blockIdx.x + gridDim.x * blockIdx.y, mod 2^16) }
+ * kernel: 1 indexer score, 2 filter, 3 resolve, 4 emit, 5 attention split,
+ * 6 split merge, 7 FP4 indexer score.  Phases: score 0 start, 1 scan done,
+ * 2 threshold found (last CTA); filter 0 start, 1 rows done; resolve 0
+ * start, 1 counts scanned, 2 candidates gathered, 3 t~ known, 4 band done,
+ * 5 cut done, 6 positions written; emit, attention 0 start, 1 end; merge 0.
+ * sa_trace_install(buf, capacity) waits for `stream`, then makes buf (device
+ * memory, 16-byte aligned, capacity records) the destination and resets the
+ * count; capacity 0 switches tracing off.  sa_trace_count waits for `stream`
+ * and returns the records written (marks past capacity are dropped but
+ * counted).  The default library returns SA_ERR_UNSUPPORTED from both.    */
+sa_status sa_trace_install(void* buf, uint32_t capacity, void* stream);
+sa_status sa_trace_count(uint32_t* n, void* stream);
+
 /* Text for the last non-OK status returned on the calling host thread.      */
 const char* sa_last_error(void);
 

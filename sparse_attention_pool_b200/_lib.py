@@ -8,6 +8,7 @@ import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libsparse_attn.so")
+TRACE_LIB_PATH = os.path.join(HERE, "libsparse_attn_trace.so")  # loaded instead when SA_TRACE_LIB=1
 
 SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_CUDA, SA_ERR_TIMEOUT, SA_ERR_DEVICE = range(7)
 SA_BF16, SA_FP8_E4M3, SA_KV_MIXED = 0, 1, 2
@@ -26,7 +27,7 @@ EXPORTS = ["csa_compress", "hca_compress", "csa_index_topk", "csa_sparse_attn", 
            "csa_index_topk_noalloc", "csa_append", "hca_append", "swa_attn", "attn_lse_merge",
            "csa_index_quantize_mxfp4", "csa_index_topk_mxfp4", "hybrid_attn_decode_mxfp4",
            "cp_decode_candidates", "cp_decode_merge_select", "attn_lse_merge_n", "hybrid_attn_decode_swa",
-           "sa_selftest_wait_timeout"]
+           "sa_selftest_wait_timeout", "sa_trace_install", "sa_trace_count"]
 SA_NOALLOC_SCRATCH_BYTES = 32 << 20
 SA_STAGE_INDEX_SCORE, SA_STAGE_TOPK_SELECT, SA_STAGE_CSA_ATTN, SA_STAGE_HCA_ATTN = 0, 1, 2, 3
 
@@ -59,10 +60,11 @@ def lib():
     """The loaded library (raises if it is missing)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise ImportError(f"libsparse_attn.so is not built ({LIB_PATH}); run "
+        path = TRACE_LIB_PATH if os.environ.get("SA_TRACE_LIB") == "1" else LIB_PATH
+        if not os.path.exists(path):
+            raise ImportError(f"{os.path.basename(path)} is not built ({path}); run "
                               f"`python -m sparse_attention_pool_b200.build`")
-        L = ctypes.CDLL(LIB_PATH)
+        L = ctypes.CDLL(path)
         RP, CP = ctypes.POINTER(SaRaw), ctypes.POINTER(SaCache)
         L.csa_compress.argtypes = [RP, CP, P]
         L.hca_compress.argtypes = [RP, CP, P]
@@ -92,6 +94,8 @@ def lib():
         L.sa_abi_version.restype = I32
         L.sa_set_stage_events.argtypes = [I32, P, P]
         L.sa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, P]
+        L.sa_trace_install.argtypes = [P, ctypes.c_uint32, P]
+        L.sa_trace_count.argtypes = [ctypes.POINTER(ctypes.c_uint32), P]
         L.sa_launch_count.argtypes = []
         L.sa_launch_count.restype = ctypes.c_uint64
         for name in EXPORTS:

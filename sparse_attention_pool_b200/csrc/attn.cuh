@@ -106,6 +106,7 @@ __global__ void __launch_bounds__(NW * EG * 32) attn_split_kernel(AttnArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     pdl_wait();
     pdl_release();
+    SA_TRACE_MARK(TR_ATTN, 0);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int hg = warp % NW, eg = warp / NW;  // head group (16 heads), entry group of each tile
     // grid: (splits, queries) in a cluster launch, else (queries, splits)
@@ -508,6 +509,7 @@ __global__ void __launch_bounds__(NW * EG * 32) attn_split_kernel(AttnArgs a) {
             if ((lane & 3) == 0) a.part_lse[((size_t)bq * a.splits + split) * a.H + hr[h]] = lse_r[h];
         }
     }
+    SA_TRACE_MARK(TR_ATTN, 1);
 }
 
 // Merge the split partials of one (query, head): one CTA of 8 warps, warp w
@@ -525,6 +527,7 @@ __global__ void __launch_bounds__(kCombThreads) attn_combine_kernel(const float*
     __shared__ float wred[kCombWarps], mred[kCombWarps];
     pdl_wait();
     pdl_release();
+    SA_TRACE_MARK(TR_COMBINE, 0);
     const int bh = blockIdx.x;  // bq * H + h
     const int bq = bh / H, h = bh - bq * H;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;

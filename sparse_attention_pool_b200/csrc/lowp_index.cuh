@@ -140,6 +140,7 @@ __global__ void __launch_bounds__(kF4Threads) score_decode_mxfp4_kernel(TopkDeco
     __shared__ uint32_t s_last;
     pdl_wait();
     pdl_release();
+    SA_TRACE_MARK(TR_SCORE_FP4, 0);
     const int b = blockIdx.y;
     const int tid = threadIdx.x;
     const int n = clamp_n(a.n, b, a.Ncap);
@@ -226,6 +227,7 @@ __global__ void __launch_bounds__(kF4Threads) score_decode_mxfp4_kernel(TopkDeco
     uint32_t* tot = a.totals + (size_t)b * kTotals;
     __threadfence();
     __syncthreads();
+    SA_TRACE_MARK(TR_SCORE_FP4, 1);
     if (tid == 0) s_last = atomicAdd(tot + kTotTicket, 1u) == gridDim.x - 1;
     __syncthreads();
     if (!s_last) return;
@@ -256,6 +258,7 @@ __global__ void __launch_bounds__(kF4Threads) score_decode_mxfp4_kernel(TopkDeco
         tot[kTotE] = __float_as_uint(0.f);
         tot[kTotAbove] = above1;
     }
+    SA_TRACE_MARK(TR_SCORE_FP4, 2);
 }
 
 }  // namespace sa

@@ -24,6 +24,41 @@ __device__ uint32_t g_status = 0;  // one translation unit holds all device code
 
 __device__ __forceinline__ void flag(uint32_t f) { atomicOr(&g_status, f); }
 
+// --------------------------------------------------------------- tracing --
+// Per-CTA phase marks for device timelines, compiled in only when the library
+// is built with -DSA_TRACE (the default build has none).  Thread 0 of a CTA
+// appends one 16-byte record -- the global nanosecond timer, the kernel, the
+// phase, the SM and the CTA's linear index -- to a device buffer the host
+// installs with sa_trace_install; marks past the buffer's capacity are
+// counted and dropped.  Marks sit after a barrier where they stand for the
+// whole CTA.
+enum : uint32_t {
+    TR_SCORE = 1, TR_FILTER = 2, TR_RESOLVE = 3, TR_EMIT = 4, TR_ATTN = 5, TR_COMBINE = 6, TR_SCORE_FP4 = 7,
+};
+#ifdef SA_TRACE
+struct TraceRec {
+    unsigned long long t;
+    uint16_t kernel, phase, sm, cta;
+};
+__device__ TraceRec* g_trace_buf = nullptr;
+__device__ uint32_t g_trace_cap = 0;
+__device__ uint32_t g_trace_n = 0;
+__device__ __forceinline__ void trace_mark(uint32_t kernel, uint32_t phase) {
+    if (threadIdx.x != 0 || g_trace_buf == nullptr) return;
+    unsigned long long t;
+    uint32_t sm;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+    const uint32_t i = atomicAdd(&g_trace_n, 1u);
+    if (i < g_trace_cap)
+        g_trace_buf[i] = {t, (uint16_t)kernel, (uint16_t)phase, (uint16_t)sm,
+                          (uint16_t)(blockIdx.x + gridDim.x * blockIdx.y)};
+}
+#define SA_TRACE_MARK(kernel, phase) ::sa::trace_mark((kernel), (phase))
+#else
+#define SA_TRACE_MARK(kernel, phase) ((void)0)
+#endif
+
 // Iteration limit of every spin on an mbarrier: each try_wait may itself
 // suspend for a while, so this is far above any legitimate copy latency.
 constexpr uint32_t kWaitLimit = 1u << 22;

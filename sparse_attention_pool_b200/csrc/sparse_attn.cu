@@ -741,6 +741,38 @@ sa_status sa_set_stage_events(int32_t stage, void* before, void* after) {
 
 const char* sa_last_error(void) { return g_err; }
 
+sa_status sa_trace_install(void* buf, uint32_t capacity, void* stream) {
+#ifdef SA_TRACE
+    SA_CHECK(capacity == 0 || (buf != nullptr && aligned16(buf)),
+             "sa_trace_install: buf must be non-NULL and 16-byte aligned when capacity > 0");
+    SA_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+    sa::TraceRec* p = capacity ? static_cast<sa::TraceRec*>(buf) : nullptr;
+    const uint32_t zero = 0;
+    SA_CUDA(cudaMemcpyToSymbol(sa::g_trace_buf, &p, sizeof(p)));
+    SA_CUDA(cudaMemcpyToSymbol(sa::g_trace_cap, &capacity, sizeof(capacity)));
+    SA_CUDA(cudaMemcpyToSymbol(sa::g_trace_n, &zero, sizeof(zero)));
+    return SA_OK;
+#else
+    (void)buf;
+    (void)capacity;
+    (void)stream;
+    return fail(SA_ERR_UNSUPPORTED, "sa_trace_install: this library was built without SA_TRACE");
+#endif
+}
+
+sa_status sa_trace_count(uint32_t* n, void* stream) {
+    SA_CHECK(n != nullptr, "sa_trace_count: n is NULL");
+#ifdef SA_TRACE
+    SA_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+    SA_CUDA(cudaMemcpyFromSymbol(n, sa::g_trace_n, sizeof(*n)));
+    return SA_OK;
+#else
+    (void)stream;
+    *n = 0;
+    return fail(SA_ERR_UNSUPPORTED, "sa_trace_count: this library was built without SA_TRACE");
+#endif
+}
+
 sa_status sa_selftest_wait_timeout(uint32_t wait_tries, void* stream) {
     SA_CHECK(wait_tries >= 1 && wait_tries <= sa::kWaitLimit, "sa_selftest_wait_timeout: wait_tries=%u outside 1..%u",
              wait_tries, sa::kWaitLimit);

@@ -385,6 +385,7 @@ __global__ void __launch_bounds__(kScThreads, 3)
 
     pdl_wait();
     pdl_release();
+    SA_TRACE_MARK(TR_SCORE, 0);
     const int b = blockIdx.y;
     const int tid = threadIdx.x;
     const int row0 = blockIdx.x * a.chunk;
@@ -494,6 +495,7 @@ __global__ void __launch_bounds__(kScThreads, 3)
     uint32_t* tot = a.totals + (size_t)b * kTotals;
     __threadfence();
     __syncthreads();
+    SA_TRACE_MARK(TR_SCORE, 1);
     if (tid == 0) s_last = atomicAdd(tot + kTotTicket, 1u) == gridDim.x - 1;
     __syncthreads();
     if (!s_last) return;
@@ -534,6 +536,7 @@ __global__ void __launch_bounds__(kScThreads, 3)
         tot[kTotE] = __float_as_uint(E);
         tot[kTotAbove] = above1;
     }
+    SA_TRACE_MARK(TR_SCORE, 2);
 }
 
 // --------------------------------------------------------- 2. selection ----
@@ -593,6 +596,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_filter_kernel(TopkDecodeArgs
     __shared__ uint32_t s_cnt, s_in;
     pdl_wait();
     pdl_release();
+    SA_TRACE_MARK(TR_FILTER, 0);
     const int b = blockIdx.y, c = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int k = a.k;
@@ -665,6 +669,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_filter_kernel(TopkDecodeArgs
     }
     if (lane == 0 && nin) red_add_shared(&s_in, nin);  // every lane counted the same ballots
     __syncthreads();
+    SA_TRACE_MARK(TR_FILTER, 1);
     if (tid == 0) {
         a.chunk_in[(size_t)b * a.nfch + c] = s_in;
         a.chunk_cnt[(size_t)b * a.nfch + c] = s_cnt;
@@ -741,6 +746,7 @@ __device__ __forceinline__ void resolve_body(const TopkDecodeArgs& a, SelSmem& S
     cp_async_commit();  // the staged rows are awaited just before the band
     if (!SMEM) __threadfence_block();
     __syncthreads();
+    SA_TRACE_MARK(TR_RESOLVE, 2);
 
     // t~: the R3-th largest key of the fine bin (few keys: ranked pairwise)
     const uint32_t R1 = (uint32_t)k - A;  // rank of t~ among the candidates (>= 1)
@@ -781,6 +787,7 @@ __device__ __forceinline__ void resolve_body(const TopkDecodeArgs& a, SelSmem& S
     int32_t* gai = a.amb_idx + (size_t)b * a.Ncap;
     cp_async_wait<0>();
     __syncthreads();  // S.amb_key held the fine bin; the staged rows have landed
+    SA_TRACE_MARK(TR_RESOLVE, 3);
     // when the band lies inside the staged window, its members are all staged
     const uint32_t lo_w = pre >= 2u ? (pre - 2u) << 10 : 0u;
     const bool win = fast && S.pf_cnt <= (uint32_t)kPf && blo_key >= lo_w && (bhi_key >> 10) <= pre + 2u;
@@ -829,6 +836,7 @@ __device__ __forceinline__ void resolve_body(const TopkDecodeArgs& a, SelSmem& S
     }
     uint32_t in2;
     block_exclusive_scan(my_in2, S.sh64, &in2);
+    SA_TRACE_MARK(TR_RESOLVE, 4);
     const uint32_t na = S.amb_cnt;
     const uint32_t R2 = R1 - in2;  // winners to take from the band (1 <= R2 <= na)
     // the exact cut of the band: a member wins iff (key, -j) >= (T2, -jmax2)
@@ -861,6 +869,7 @@ __device__ __forceinline__ void resolve_body(const TopkDecodeArgs& a, SelSmem& S
     }
     const uint32_t T2 = S.T2;
     const int32_t jmax2 = S.jmax2;
+    SA_TRACE_MARK(TR_RESOLVE, 5);
     // the band's winners
 #pragma unroll 1
     for (uint32_t i = tid; i < na; i += kResThreads) {
@@ -878,6 +887,7 @@ __device__ __forceinline__ void resolve_body(const TopkDecodeArgs& a, SelSmem& S
         if (total != (uint32_t)k) flag(DEV_LEN);  // cannot happen
         a.cnt[b] = k;
     }
+    SA_TRACE_MARK(TR_RESOLVE, 6);
 }
 
 // One CTA of 1024 threads per sequence.  One round trip brings the totals,
@@ -891,6 +901,7 @@ __global__ void __launch_bounds__(kResThreads, 1) topk_resolve_kernel(TopkDecode
     __shared__ SelSmem S;
     pdl_wait();
     pdl_release();
+    SA_TRACE_MARK(TR_RESOLVE, 0);
     const int b = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int k = a.k;
@@ -947,6 +958,7 @@ __global__ void __launch_bounds__(kResThreads, 1) topk_resolve_kernel(TopkDecode
         S.ccnt[tid] = ccn;
     }
     __syncthreads();
+    SA_TRACE_MARK(TR_RESOLVE, 1);
     if (C > (uint32_t)a.Ncap) {  // cannot happen: at most n candidates
         if (tid == 0) flag(DEV_LEN);
         C = a.Ncap;
@@ -965,6 +977,7 @@ __global__ void __launch_bounds__(kEmitThreads) topk_emit_kernel(TopkDecodeArgs 
     __shared__ uint32_t sh32[32];
     pdl_wait();
     pdl_release();
+    SA_TRACE_MARK(TR_EMIT, 0);
     const int b = blockIdx.y, c = blockIdx.x;
     const int row0 = c * a.fchunk;
     const uint32_t* bm = a.bitmap + (size_t)b * a.Wcap;
@@ -994,6 +1007,7 @@ __global__ void __launch_bounds__(kEmitThreads) topk_emit_kernel(TopkDecodeArgs 
         }
         pos += total;
     }
+    SA_TRACE_MARK(TR_EMIT, 1);
 }
 
 }  // namespace sa

@@ -1,0 +1,87 @@
+"""Device timelines from the profiling build of the library.
+
+``libsparse_attn_trace.so`` is the library compiled with -DSA_TRACE: its
+decode-path kernels append one record per CTA and phase (global nanosecond
+timer, kernel, phase, SM, CTA) to a device buffer.  Set SA_TRACE_LIB=1
+before the first library call of the process to load it; the default
+library has no marks (its kernels are unchanged) and refuses these calls.
+
+    os.environ["SA_TRACE_LIB"] = "1"
+    import sparse_attention_pool_b200 as S
+    from sparse_attention_pool_b200 import trace
+    buf = trace.install(1 << 16)
+    S.hybrid_attn_decode(...)
+    print(trace.format_summary(trace.records(buf)))
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+import torch
+
+from ._lib import check, lib
+
+KERNELS = {1: "score", 2: "filter", 3: "resolve", 4: "emit", 5: "attn_split", 6: "attn_merge", 7: "score_fp4"}
+PHASES = {
+    "score": ["start", "scan done", "threshold found"],
+    "score_fp4": ["start", "scan done", "threshold found"],
+    "filter": ["start", "rows done"],
+    "resolve": ["start", "counts scanned", "gathered", "t~ known", "band done", "cut done", "positions written"],
+    "emit": ["start", "end"],
+    "attn_split": ["start", "end"],
+    "attn_merge": ["start"],
+}
+RECORD = np.dtype([("t", "<u8"), ("kernel", "<u2"), ("phase", "<u2"), ("sm", "<u2"), ("cta", "<u2")])
+
+
+def install(capacity: int, device="cuda", stream=None) -> torch.Tensor:
+    """A zeroed device buffer of `capacity` records, installed as the
+    destination of the marks (the count starts at 0)."""
+    buf = torch.zeros(capacity * RECORD.itemsize, dtype=torch.uint8, device=device)
+    s = torch.cuda.current_stream() if stream is None else stream
+    check("sa_trace_install", lib().sa_trace_install(ctypes.c_void_p(buf.data_ptr()), capacity,
+                                                     ctypes.c_void_p(s.cuda_stream)))
+    return buf
+
+
+def uninstall(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    check("sa_trace_install", lib().sa_trace_install(None, 0, ctypes.c_void_p(s.cuda_stream)))
+
+
+def records(buf: torch.Tensor, stream=None) -> np.ndarray:
+    """The records written so far (waits for the stream), in append order."""
+    s = torch.cuda.current_stream() if stream is None else stream
+    n = ctypes.c_uint32(0)
+    check("sa_trace_count", lib().sa_trace_count(ctypes.byref(n), ctypes.c_void_p(s.cuda_stream)))
+    cap = buf.numel() // RECORD.itemsize
+    m = min(int(n.value), cap)
+    return buf[:m * RECORD.itemsize].cpu().numpy().view(RECORD)
+
+
+def summary(rec: np.ndarray) -> list[dict]:
+    """Per (kernel, phase): the CTAs that reached it and the first, median
+    and last time (µs from the earliest mark), in time order."""
+    if rec.size == 0:
+        return []
+    t0 = int(rec["t"].min())
+    rows = []
+    for kid in np.unique(rec["kernel"]):
+        name = KERNELS.get(int(kid), f"kernel{int(kid)}")
+        sel = rec[rec["kernel"] == kid]
+        for ph in np.unique(sel["phase"]):
+            ts = (sel["t"][sel["phase"] == ph].astype(np.int64) - t0) / 1e3
+            labels = PHASES.get(name, [])
+            rows.append({"kernel": name, "phase": labels[ph] if ph < len(labels) else str(int(ph)),
+                         "ctas": int(ts.size), "first_us": float(ts.min()), "median_us": float(np.median(ts)),
+                         "last_us": float(ts.max())})
+    return sorted(rows, key=lambda r: r["first_us"])
+
+
+def format_summary(rec: np.ndarray) -> str:
+    lines = [f"{'kernel':<11} {'phase':<18} {'CTAs':>6} {'first':>9} {'median':>9} {'last':>9}  (µs)"]
+    for r in summary(rec):
+        lines.append(f"{r['kernel']:<11} {r['phase']:<18} {r['ctas']:>6} {r['first_us']:>9.2f} "
+                     f"{r['median_us']:>9.2f} {r['last_us']:>9.2f}")
+    return "\n".join(lines)

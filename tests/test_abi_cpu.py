@@ -255,3 +255,23 @@ def test_selftest_rejects_bad_arguments(L):
     assert L.sa_selftest_wait_timeout(0, None) == _lib.SA_ERR_INVALID_ARG
     assert L.sa_selftest_wait_timeout((1 << 22) + 1, None) == _lib.SA_ERR_INVALID_ARG
     assert "wait_tries" in L.sa_last_error().decode()
+
+
+def test_trace_calls_need_the_profiling_build(L):
+    n = ctypes.c_uint32(7)
+    assert L.sa_trace_install(None, 0, None) == _lib.SA_ERR_UNSUPPORTED
+    assert "SA_TRACE" in L.sa_last_error().decode()
+    assert L.sa_trace_count(ctypes.byref(n), None) == _lib.SA_ERR_UNSUPPORTED and n.value == 0
+    assert L.sa_trace_count(None, None) == _lib.SA_ERR_INVALID_ARG
+
+
+def test_profiling_build_exports_every_header_symbol():
+    build.build(trace=True)
+    T = ctypes.CDLL(_lib.TRACE_LIB_PATH)
+    for n in header_functions():
+        assert hasattr(T, n), n
+    T.sa_trace_install.argtypes = [ctypes.c_void_p, ctypes.c_uint32, ctypes.c_void_p]
+    T.sa_trace_install.restype = ctypes.c_int32
+    T.sa_last_error.restype = ctypes.c_char_p
+    # argument checks run before any CUDA call
+    assert T.sa_trace_install(ctypes.c_void_p(0x10004), 8, None) == _lib.SA_ERR_INVALID_ARG
