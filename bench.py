@@ -517,6 +517,124 @@ def run_ours(args, w, rank, world, dev):
     return result
 
 
+# ------------------------------------------------- context-parallel mode ---
+
+def run_cp(args, w, rank, world, dev):
+    """--cp: one batch sharded by context over the ranks (each rank holds and
+    compresses its shard of every sequence); a step is cp_decode_step, the
+    exchange over NCCL.  Strong scaling: the same B tokens per step at every
+    world size.  With one rank the selection is checked against
+    hybrid_attn_decode on the same caches."""
+    import socket
+
+    import torch
+    import torch.distributed as dist
+
+    import sparse_attention_pool_b200 as S
+    from sparse_attention_pool_b200 import _lib, cp
+
+    own_group = not dist.is_initialized()
+    if own_group:  # a one-rank NCCL group for the exchange calls
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        store = dist.TCPStore("127.0.0.1", port, 1, True)
+        dist.init_process_group("nccl", store=store, rank=0, world_size=1,
+                                timeout=datetime.timedelta(seconds=300), device_id=dev)
+    try:
+        lengths, K, V, KI, q_h, qI_h = make_inputs(w, 0)  # one batch, the same on every rank
+        B, H, k = w.B, w.H, w.topk
+        t_gen = time.time()
+        bounds = [cp.shard_bounds(int(lengths[b]), world) for b in range(B)]
+        span = [bounds[b][rank] for b in range(B)]
+        Lw = max(1, max(t1 - t0 for t0, t1 in span))
+        Lw = -(-Lw // 128) * 128
+        Ks = np.zeros((B, Lw, 128), np.uint16)
+        Vs = np.zeros((B, Lw, 128), np.uint16)
+        KIs = np.zeros((B, Lw, 64), np.uint16)
+        for b, (t0, t1) in enumerate(span):
+            Ks[b, :t1 - t0], Vs[b, :t1 - t0], KIs[b, :t1 - t0] = K[b, t0:t1], V[b, t0:t1], KI[b, t0:t1]
+        del K, V, KI
+        lens = torch.tensor([t1 - t0 for t0, t1 in span], dtype=torch.int32, device=dev)
+        Kd, Vd, KId = to_bf16_tensor(Ks, dev), to_bf16_tensor(Vs, dev), to_bf16_tensor(KIs, dev)
+        csa = S.alloc_cache(B, Lw // w.m_csa, w.m_csa, fp8=w.fp8, with_kidx=True, device=dev)
+        hca = S.alloc_cache(B, Lw // w.m_hca, w.m_hca, fp8=w.fp8, device=dev)
+        S.csa_compress(Kd, Vd, KId, lens, csa)
+        S.hca_compress(Kd, Vd, lens, hca)
+        torch.cuda.synchronize()
+        del Kd, Vd, KId
+        base = torch.tensor([cp.entry_base(bounds[b], rank, w.m_csa) for b in range(B)], dtype=torch.int32,
+                            device=dev)
+        q, qI = to_bf16_tensor(q_h, dev), to_bf16_tensor(qI_h, dev)
+        ws = S.alloc_workspace(cp.workspace_size(B, H, csa.Ncap, hca.Ncap, k), device=dev)
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        flush_sink = torch.empty(1, dtype=torch.int64, device=dev)
+        stream = torch.cuda.current_stream()
+
+        def flush_l2():  # written then read back: L2 ends up clean (as in the main line)
+            flush.fill_(1)
+            flush_sink.copy_(flush.view(torch.int64).sum())
+
+        def step():
+            return cp.cp_decode_step(q, qI, csa, hca, base, k, ws, scale=SCALE)
+
+        oc, oh, lc, lh, sel, scnt = step()
+        torch.cuda.synchronize()
+        S.read_device_status()
+        check = None
+        if world == 1:
+            ws1 = S.alloc_workspace(S.workspace_size(S.SA_OP_HYBRID_DECODE, B, 1, H, csa.Ncap, hca.Ncap, k),
+                                    device=dev)
+            idx = torch.empty(B, k, dtype=torch.int32, device=dev)
+            cnt = torch.empty(B, dtype=torch.int32, device=dev)
+            S.hybrid_attn_decode(q, qI, csa, hca, k, ws1, scale=SCALE, idx_out=idx, cnt_out=cnt)
+            torch.cuda.synchronize()
+            check = "selection equals hybrid_attn_decode" if torch.equal(idx, sel) and torch.equal(cnt, scnt) \
+                else "MISMATCH with hybrid_attn_decode"
+        L = _lib.lib()
+        n0 = L.sa_launch_count()
+        step()
+        torch.cuda.synchronize()
+        launches_per_step = int(L.sa_launch_count() - n0)
+        for _ in range(args.warmup):
+            flush_l2()
+            step()
+        torch.cuda.synchronize()
+        ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        step_ms = []
+        dist.barrier()
+        torch.cuda.synchronize()
+        with ClockSampler(torch.cuda.current_device()) as clk:
+            for i in range(args.steps):
+                flush_l2()  # untimed: evict the shards from L2
+                ev0[i].record(stream)
+                step()
+                ev1[i].record(stream)
+                ev1[i].synchronize()
+                step_ms.append(ev0[i].elapsed_time(ev1[i]))
+        torch.cuda.synchronize()
+        dist.barrier()
+        total_ms = max_over_ranks(sum(step_ms), world, dev)
+        S.read_device_status()
+        return {
+            "metric": METRIC, "value": B * args.steps / (total_ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": "bf16" if not w.fp8 else "fp8e4m3-kv/bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": B, "context": int(w.L), "heads": H, "topk": k,
+                       "parallelism": f"context-parallel x{world} (one batch sharded by context)",
+                       "l2": "flushed between timed steps: 512 MB written then read back (clean L2)",
+                       "launch": "eager, NCCL all-gathers"},
+            "gpu_launches": launches_per_step * args.steps, "check": check,
+            "e2e": {"value": None, "note": "not measured in --cp mode"},
+            "clocks": clk.summary(), "setup_s": round(time.time() - t_gen, 1),
+        }
+    finally:
+        if own_group:
+            dist.destroy_process_group()
+
+
 # ------------------------------------------------------------ prefill arm ---
 
 FP64_FMA_PER_CLK_PER_SM = 64  # B200: 64 fp64 lanes per SM (nominal 37 TFLOP/s at 1965 MHz)
@@ -819,14 +937,18 @@ def main():
                     help="decode only: the CSA indexer keys in bf16 (the workload) or FP4 (MXFP4)")
     ap.add_argument("--kv", default="workload", choices=["workload", "mixed"],
                     help="decode only: the workload's KV storage, or mixed storage (rotary dims bf16, the rest e4m3)")
+    ap.add_argument("--cp", action="store_true",
+                    help="decode only: context-parallel mode, one batch sharded by context over the ranks")
     ap.add_argument("--tokens", type=int, default=0,
                     help="prefill only: a shorter sequence than the workload's (small cases for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = configs.BY_NAME[args.workload]
-    if (args.indexer != "bf16" or args.kv != "workload") and w.mode != "decode":
-        ap.error("--indexer and --kv apply to decode workloads")
+    if (args.indexer != "bf16" or args.kv != "workload" or args.cp) and w.mode != "decode":
+        ap.error("--indexer, --kv and --cp apply to decode workloads")
+    if args.cp and (args.indexer != "bf16" or args.kv != "workload" or args.impl != "ours"):
+        ap.error("--cp runs the workload's own storage and indexer on our arm")
     if args.tokens:
         if w.mode != "prefill":
             ap.error("--tokens applies to prefill workloads")
@@ -846,7 +968,10 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
     try:
-        res = run_ours(args, w, rank, world, dev) if w.mode == "decode" else run_prefill(args, w, rank, world, dev)
+        if args.cp:
+            res = run_cp(args, w, rank, world, dev)
+        else:
+            res = run_ours(args, w, rank, world, dev) if w.mode == "decode" else run_prefill(args, w, rank, world, dev)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:
