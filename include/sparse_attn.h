@@ -197,16 +197,18 @@ sa_status csa_index_topk(const void* q_idx, int32_t Tq, const int32_t* q_pos,
 sa_status csa_index_quantize_mxfp4(const sa_cache* csa, int32_t row_from, uint8_t* codes, uint8_t* scales,
                                    void* stream);
 
-/* Decode top-k on FP4 indexer scores (same section).  The query q_idx
- * [B][d_idx] bf16 is quantized in the kernel by the rule above; the score of
- * entry j is the fp32 value, rounded to nearest even once, of the exact sum
- * over the two blocks of X_q * X_k * sum_i e2m1(q_i) * e2m1(k_ji) (-0 -> +0).
- * Selection, order, padding and count are those of csa_index_topk with
- * q_pos == NULL.  codes / scales as written by csa_index_quantize_mxfp4 for
+/* Top-k on FP4 indexer scores (same section), in decode and in causal
+ * prefill.  The queries q_idx [B][Tq][d_idx] bf16 are quantized in the kernel
+ * by the rule above; the score of entry j is the fp32 value, rounded to
+ * nearest even once, of the exact sum over the two blocks of
+ * X_q * X_k * sum_i e2m1(q_i) * e2m1(k_ji) (-0 -> +0).  Tq, q_pos,
+ * visibility, selection, order, padding and count are those of
+ * csa_index_topk.  codes / scales as written by csa_index_quantize_mxfp4 for
  * the entries 0..n[b]-1; the bf16 indexer keys of the cache are not read.
- * ws / ws_bytes: at least sa_workspace_size(SA_OP_INDEX_TOPK, B, 1, ...).     */
-sa_status csa_index_topk_mxfp4(const void* q_idx, const sa_cache* csa, const uint8_t* codes, const uint8_t* scales,
-                               int32_t k, int32_t* idx, int32_t* cnt, void* ws, size_t ws_bytes, void* stream);
+ * ws / ws_bytes: at least sa_workspace_size(SA_OP_INDEX_TOPK, B, Tq, ...).    */
+sa_status csa_index_topk_mxfp4(const void* q_idx, int32_t Tq, const int32_t* q_pos, const sa_cache* csa,
+                               const uint8_t* codes, const uint8_t* scales, int32_t k, int32_t* idx, int32_t* cnt,
+                               void* ws, size_t ws_bytes, void* stream);
 
 /* CSA attention over the chosen entries, section 3-2 (2) (CSA attends over
  * the selected entries only).

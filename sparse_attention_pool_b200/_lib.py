@@ -75,7 +75,7 @@ def lib():
         L.csa_index_topk.argtypes = [P, I32, P, CP, I32, P, P, P, SZ, P]
         L.csa_index_topk_noalloc.argtypes = [P, CP, I32, P, P, P]
         L.csa_index_quantize_mxfp4.argtypes = [CP, I32, P, P, P]
-        L.csa_index_topk_mxfp4.argtypes = [P, CP, P, P, I32, P, P, P, SZ, P]
+        L.csa_index_topk_mxfp4.argtypes = [P, I32, P, CP, P, P, I32, P, P, P, SZ, P]
         L.csa_sparse_attn.argtypes = [P, I32, I32, CP, P, P, I32, F32, P, P, P, SZ, P]
         L.hca_dense_attn.argtypes = [P, I32, I32, P, CP, F32, P, P, P, SZ, P]
         L.hybrid_attn_decode.argtypes = [P, P, I32, CP, CP, I32, F32, P, P, P, P, P, P, P, SZ, P]

@@ -211,20 +211,24 @@ def csa_index_quantize_mxfp4(csa: Cache, *, codes=None, scales=None, row_from: i
     return codes, scales
 
 
-def csa_index_topk_mxfp4(q_idx, csa: Cache, codes, scales, k: int, ws, *, idx=None, cnt=None, stream=None):
-    """Decode top-k on FP4 (MXFP4) indexer scores; idx [B][1][k], cnt [B][1]."""
+def csa_index_topk_mxfp4(q_idx, csa: Cache, codes, scales, k: int, ws, *, q_pos=None, idx=None, cnt=None,
+                         stream=None):
+    """Top-k on FP4 (MXFP4) indexer scores, decode (q_pos None: q_idx [B][64])
+    or causal prefill (q_idx [B][T][64], q_pos [B][T]); idx [B][Tq][k], cnt
+    [B][Tq]."""
     _need(q_idx, torch.bfloat16, "q_idx")
     _need(codes, torch.uint8, "codes")
     _need(scales, torch.uint8, "scales")
     B = csa.B
+    Tq = 1 if q_pos is None else q_idx.shape[1]
     if idx is None:
-        idx = torch.empty(B, 1, k, dtype=torch.int32, device=q_idx.device)
+        idx = torch.empty(B, Tq, k, dtype=torch.int32, device=q_idx.device)
     if cnt is None:
-        cnt = torch.empty(B, 1, dtype=torch.int32, device=q_idx.device)
+        cnt = torch.empty(B, Tq, dtype=torch.int32, device=q_idx.device)
     cs = csa.struct()
-    check("csa_index_topk_mxfp4", lib().csa_index_topk_mxfp4(_ptr(q_idx), ctypes.byref(cs), _ptr(codes), _ptr(scales),
-                                                             k, _ptr(idx), _ptr(cnt), _ptr(ws), ws.numel(),
-                                                             _stream(stream)))
+    check("csa_index_topk_mxfp4", lib().csa_index_topk_mxfp4(_ptr(q_idx), Tq, _ptr(q_pos), ctypes.byref(cs),
+                                                             _ptr(codes), _ptr(scales), k, _ptr(idx), _ptr(cnt),
+                                                             _ptr(ws), ws.numel(), _stream(stream)))
     return idx, cnt
 
 

@@ -22,6 +22,7 @@
 #pragma once
 #include "sa_common.cuh"
 #include "topk_decode.cuh"
+#include "topk_prefill.cuh"
 
 namespace sa {
 
@@ -259,6 +260,138 @@ __global__ void __launch_bounds__(kF4Threads) score_decode_mxfp4_kernel(TopkDeco
         tot[kTotAbove] = above1;
     }
     SA_TRACE_MARK(TR_SCORE_FP4, 2);
+}
+
+// ------------------------------------------------- FP4 prefill scores ---
+// The causal-prefill counterpart: order keys of the FP4 scores of a block of
+// queries against every entry, in the key block select_prefill_kernel reads.
+// A CTA takes 64 queries x 128 entries (the bf16 kernel's tiling); each
+// thread owns 4 queries x 8 entries and one exact int32 accumulator per
+// 32-dim block.  The queries are quantized here by the rule of the keys;
+// the keys' codes are widened once per tile to doubled signed int8 values
+// (+-{0,1,2,3,4,6,8,12}) in shared memory, four per 32-bit word.
+constexpr int kPf4Smem = kPsQ * 16 * 4 + 16 * kPsE * 4;  // query words [64][16] + key words [16][128]
+
+__device__ __forceinline__ uint32_t e2m1_doubled_s8(uint32_t code) {  // signed doubled value as a byte
+    const int m = (int)(__byte_perm(kE2m1LutLo, kE2m1LutHi, code & 7u) & 0xFFu);
+    return (uint32_t)((code & 8u) ? -m : m) & 0xFFu;
+}
+
+__global__ void __launch_bounds__(kPsThreads, 2) score_prefill_mxfp4_kernel(TopkPrefillArgs a,
+                                                                           const uint8_t* __restrict__ codes,
+                                                                           const uint8_t* __restrict__ scales) {
+    extern __shared__ __align__(16) uint32_t smem_w[];
+    uint32_t* sQ = smem_w;                 // [64 queries][16 words]
+    uint32_t* sK = smem_w + kPsQ * 16;     // [16 words][128 entries]
+    __shared__ int sQe[kPsQ][2];           // E8M0 codes of the queries' blocks
+    __shared__ uint8_t sKe[kPsE][2];       // ... and of the entries'
+    __shared__ int s_maxvis;
+
+    const int tid = threadIdx.x;
+    const int e0 = blockIdx.x * kPsE;
+    const int ql0 = blockIdx.y * kPsQ;
+    if (tid == 0) s_maxvis = 0;
+    __syncthreads();
+    if (tid < kPsQ && ql0 + tid < a.qb) atomicMax(&s_maxvis, visible_entries(a, a.t0 + ql0 + tid));
+    __syncthreads();
+    if (e0 >= s_maxvis) return;  // no query of this tile sees these entries
+
+    if (tid < 2 * kPsQ) {  // one thread per (query, 32-dim block): quantize
+        const int ql = tid >> 1, blk = tid & 1;
+        const bool ok = ql0 + ql < a.qb;
+        uint32_t w[16];
+        const uint4* src = reinterpret_cast<const uint4*>(a.q_idx + ((size_t)a.b * a.Tq + a.t0 + ql0 + ql) * 64 +
+                                                          blk * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint4 v = ok ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+            w[4 * i] = v.x;
+            w[4 * i + 1] = v.y;
+            w[4 * i + 2] = v.z;
+            w[4 * i + 3] = v.w;
+        }
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fmaxf(fabsf(bf16lo_f32(w[i])), fabsf(bf16hi_f32(w[i]))));
+        const int se = mx_scale_exp(amax);
+        const float inv = mx_inv_scale(se);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {  // word i: elements 4i .. 4i+3 of the block
+            const uint32_t b0 = e2m1_doubled_s8(e2m1_code(bf16lo_f32(w[2 * i]) * inv));
+            const uint32_t b1 = e2m1_doubled_s8(e2m1_code(bf16hi_f32(w[2 * i]) * inv));
+            const uint32_t b2 = e2m1_doubled_s8(e2m1_code(bf16lo_f32(w[2 * i + 1]) * inv));
+            const uint32_t b3 = e2m1_doubled_s8(e2m1_code(bf16hi_f32(w[2 * i + 1]) * inv));
+            sQ[ql * 16 + blk * 8 + i] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+        }
+        sQe[ql][blk] = se + 127;
+    }
+    {  // keys: one thread per (entry, 16-byte half of its codes)
+        const int e = tid >> 1, half = tid & 1;
+        const bool ok = e0 + e < a.Ncap;
+        const size_t row = (size_t)a.b * a.Ncap + e0 + e;
+        const uint4 c = ok ? __ldg(reinterpret_cast<const uint4*>(codes + row * 32) + half) : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {  // 8 codes -> two words of 4 doubled int8
+            uint32_t lo = 0u, hi = 0u;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                lo |= e2m1_doubled_s8((cw[i] >> (4 * j)) & 0xFu) << (8 * j);
+                hi |= e2m1_doubled_s8((cw[i] >> (4 * (j + 4))) & 0xFu) << (8 * j);
+            }
+            sK[(half * 8 + 2 * i) * kPsE + e] = lo;
+            sK[(half * 8 + 2 * i + 1) * kPsE + e] = hi;
+        }
+        if (half == 0) {
+            const uint16_t sc = ok ? __ldg(reinterpret_cast<const uint16_t*>(scales + row * 2)) : (uint16_t)0x7F7F;
+            sKe[e][0] = (uint8_t)(sc & 0xFFu);
+            sKe[e][1] = (uint8_t)(sc >> 8);
+        }
+    }
+    __syncthreads();
+
+    const int tq = tid >> 4, te = tid & 15;
+    int acc[2][4][8];
+#pragma unroll
+    for (int g = 0; g < 2; ++g)
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 8; ++v) acc[g][u][v] = 0;
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {  // the two 32-dim blocks
+#pragma unroll 2
+        for (int i = 0; i < 8; ++i) {
+            const int wi = g * 8 + i;
+            const uint4 k0 = *reinterpret_cast<const uint4*>(sK + wi * kPsE + te * 4);
+            const uint4 k1 = *reinterpret_cast<const uint4*>(sK + wi * kPsE + 64 + te * 4);
+            const uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+            uint32_t qw[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) qw[u] = sQ[(tq * 4 + u) * 16 + wi];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int v = 0; v < 8; ++v) acc[g][u][v] = __dp4a((int)qw[u], (int)kw[v], acc[g][u][v]);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int ql = ql0 + tq * 4 + u;
+        if (ql >= a.qb) continue;
+        uint32_t kk[8];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+            const int e = (v < 4 ? te * 4 + v : 64 + te * 4 + v - 4);
+            // block b scores A_b * 2^(cq_b - 127) * 2^(ck_b - 127) / 4
+            const float t0 = ldexpf((float)acc[0][u][v], sQe[tq * 4 + u][0] + (int)sKe[e][0] - 256);
+            const float t1 = ldexpf((float)acc[1][u][v], sQe[tq * 4 + u][1] + (int)sKe[e][1] - 256);
+            kk[v] = score_key(__fadd_rn(t0, t1));
+        }
+        uint32_t* row = a.keys + (size_t)ql * a.KS + e0;
+        *reinterpret_cast<uint4*>(row + te * 4) = make_uint4(kk[0], kk[1], kk[2], kk[3]);
+        *reinterpret_cast<uint4*>(row + 64 + te * 4) = make_uint4(kk[4], kk[5], kk[6], kk[7]);
+    }
 }
 
 }  // namespace sa

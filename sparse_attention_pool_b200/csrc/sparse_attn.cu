@@ -640,8 +640,11 @@ const int32_t* prefill_positions(void* ws, int B, int T, cudaStream_t st) {
     return pos;
 }
 
+// With MXFP4 keys (codes4 / scales4 non-NULL) the FP4 score kernel writes the
+// key block; the selection is the same.
 sa_status run_topk_prefill(const void* q_idx, int Tq, const int32_t* pos, const sa_cache* c, int k, int32_t* idx,
-                           int32_t* cnt, void* ws, cudaStream_t st) {
+                           int32_t* cnt, void* ws, cudaStream_t st, const uint8_t* codes4 = nullptr,
+                           const uint8_t* scales4 = nullptr) {
     sa::TopkPrefillArgs a{};
     a.q_idx = static_cast<const uint16_t*>(q_idx);
     a.kidx = static_cast<const uint16_t*>(c->kidx);
@@ -669,7 +672,11 @@ sa_status run_topk_prefill(const void* q_idx, int Tq, const int32_t* pos, const 
             a.b = b;
             a.t0 = t0;
             a.qb = std::min(kPrefillQB, Tq - t0);
-            if (c->Ncap > 0) {
+            if (c->Ncap > 0 && codes4) {
+                sa::score_prefill_mxfp4_kernel<<<dim3(etiles, cdiv(a.qb, sa::kPsQ)), sa::kPsThreads, sa::kPf4Smem,
+                                                 st>>>(a, codes4, scales4);
+                SA_LAUNCHED();
+            } else if (c->Ncap > 0) {
                 sa::score_prefill_kernel<<<dim3(etiles, cdiv(a.qb, sa::kPsQ)), sa::kPsThreads, sa::kPsSmem, st>>>(a);
                 SA_LAUNCHED();
             }
@@ -1042,8 +1049,9 @@ sa_status csa_index_quantize_mxfp4(const sa_cache* csa, int32_t row_from, uint8_
     return SA_OK;
 }
 
-sa_status csa_index_topk_mxfp4(const void* q_idx, const sa_cache* csa, const uint8_t* codes, const uint8_t* scales,
-                               int32_t k, int32_t* idx, int32_t* cnt, void* ws, size_t ws_bytes, void* stream) {
+sa_status csa_index_topk_mxfp4(const void* q_idx, int32_t Tq, const int32_t* q_pos, const sa_cache* csa,
+                               const uint8_t* codes, const uint8_t* scales, int32_t k, int32_t* idx, int32_t* cnt,
+                               void* ws, size_t ws_bytes, void* stream) {
     sa_status r = check_cache(csa, false, "csa_index_topk_mxfp4");
     if (r != SA_OK) return r;
     SA_CHECK(q_idx && aligned16(q_idx), "csa_index_topk_mxfp4: q_idx must be non-NULL and 16-byte aligned");
@@ -1052,11 +1060,19 @@ sa_status csa_index_topk_mxfp4(const void* q_idx, const sa_cache* csa, const uin
     SA_CHECK(idx && cnt && aligned16(idx) && aligned16(cnt),
              "csa_index_topk_mxfp4: idx/cnt must be non-NULL and aligned");
     SA_CHECK(k >= 1 && k <= 65536, "csa_index_topk_mxfp4: k=%d outside 1..65536", k);
-    const TopkDecodeWs w = topk_decode_layout(csa->B, csa->Ncap, k, false);
-    r = check_ws(ws, ws_bytes, w.total);
+    SA_CHECK(Tq >= 1, "csa_index_topk_mxfp4: Tq=%d", Tq);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (q_pos == nullptr) {
+        SA_CHECK(Tq == 1, "csa_index_topk_mxfp4: decode (q_pos == NULL) needs Tq == 1, got %d", Tq);
+        const TopkDecodeWs w = topk_decode_layout(csa->B, csa->Ncap, k, false);
+        r = check_ws(ws, ws_bytes, w.total);
+        if (r != SA_OK) return r;
+        return run_topk_decode(q_idx, csa, k, idx, cnt, ws, w, st, [] { return SA_OK; }, codes, scales);
+    }
+    SA_CHECK(aligned16(q_pos), "csa_index_topk_mxfp4: q_pos must be 16-byte aligned");
+    r = check_ws(ws, ws_bytes, prefill_topk_bytes(csa->B, Tq, csa->Ncap, k));
     if (r != SA_OK) return r;
-    return run_topk_decode(q_idx, csa, k, idx, cnt, ws, w, static_cast<cudaStream_t>(stream),
-                           [] { return SA_OK; }, codes, scales);
+    return run_topk_prefill(q_idx, Tq, q_pos, csa, k, idx, cnt, ws, st, codes, scales);
 }
 
 sa_status cp_decode_candidates(const void* q_idx, const sa_cache* csa, int32_t k, const int32_t* base,

@@ -173,10 +173,17 @@ def test_mxfp4_entry_points_reject_bad_arguments(L):
     assert q(ctypes.byref(_cache(kidx=None)), 0, P(FAKE), P(FAKE), None) == 1
     assert q(ctypes.byref(c), c.Ncap, P(FAKE), P(FAKE), None) == 0  # no entry to write: nothing launched
     t = L.csa_index_topk_mxfp4
-    assert t(P(FAKE), ctypes.byref(c), P(FAKE), P(FAKE), 0, P(FAKE), P(FAKE), P(FAKE), 1 << 30, None) == 1
-    assert t(P(FAKE), ctypes.byref(c), P(FAKE + 8), P(FAKE), 8, P(FAKE), P(FAKE), P(FAKE), 1 << 30, None) == 1
-    assert t(P(FAKE), ctypes.byref(c), None, P(FAKE), 8, P(FAKE), P(FAKE), P(FAKE), 1 << 30, None) == 1
-    st = t(P(FAKE), ctypes.byref(c), P(FAKE), P(FAKE), 8, P(FAKE), P(FAKE), P(FAKE), 16, None)
+    assert t(P(FAKE), 1, None, ctypes.byref(c), P(FAKE), P(FAKE), 0, P(FAKE), P(FAKE), P(FAKE), 1 << 30, None) == 1
+    assert t(P(FAKE), 1, None, ctypes.byref(c), P(FAKE + 8), P(FAKE), 8, P(FAKE), P(FAKE), P(FAKE), 1 << 30, None) == 1
+    assert t(P(FAKE), 1, None, ctypes.byref(c), None, P(FAKE), 8, P(FAKE), P(FAKE), P(FAKE), 1 << 30, None) == 1
+    st = t(P(FAKE), 1, None, ctypes.byref(c), P(FAKE), P(FAKE), 8, P(FAKE), P(FAKE), P(FAKE), 16, None)
+    assert st == _lib.SA_ERR_WORKSPACE
+    # decode needs Tq == 1; prefill needs an aligned q_pos and the prefill workspace
+    assert t(P(FAKE), 2, None, ctypes.byref(c), P(FAKE), P(FAKE), 8, P(FAKE), P(FAKE), P(FAKE), 1 << 30, None) == 1
+    assert "Tq == 1" in L.sa_last_error().decode()
+    assert t(P(FAKE), 2, P(FAKE + 4), ctypes.byref(c), P(FAKE), P(FAKE), 8, P(FAKE), P(FAKE), P(FAKE), 1 << 30,
+             None) == 1
+    st = t(P(FAKE), 64, P(FAKE), ctypes.byref(c), P(FAKE), P(FAKE), 8, P(FAKE), P(FAKE), P(FAKE), 256, None)
     assert st == _lib.SA_ERR_WORKSPACE
 
 

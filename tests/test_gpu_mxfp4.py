@@ -158,3 +158,27 @@ def test_hybrid_decode_mxfp4_matches_oracle(S):
         assert int(cnt[b]) == r["cnt"] and np.array_equal(idx[b].cpu().numpy(), r["idx"]), b
         assert np.abs(oc[b].float().cpu().numpy() - r["out_csa"]).max() <= TOL_BF16, b
         assert np.abs(oh[b].float().cpu().numpy() - r["out_hca"]).max() <= TOL_BF16, b
+
+
+def test_topk_prefill_every_row(S):
+    """Causal prefill on FP4 scores: row t sees the entries with (c+1)*4 <= t;
+    every row's indices against the oracle."""
+    from tests._util import compress_on_gpu, Inputs
+    B, T, k = 1, 1500, 64
+    inp = Inputs(76, B, T, 8, Tq=T)
+    g = inp.to_device()
+    csa, _ = compress_on_gpu(S, g, B, T)
+    codes, scales = S.csa_index_quantize_mxfp4(csa)
+    pos = torch.arange(T, dtype=torch.int32, device="cuda").view(1, T).contiguous()
+    ws = S.alloc_workspace(S.workspace_size(S.SA_OP_INDEX_TOPK, B, T, 8, csa.Ncap, 0, k))
+    idx, cnt = S.csa_index_topk_mxfp4(g["qI"], csa, codes, scales, k, ws, q_pos=pos)
+    S.read_device_status()
+    ci = O.compress(inp.KI[0], 4)
+    kc, ks = O.mxfp4_quantize(ci)
+    gi, gn = idx[0].cpu().numpy(), cnt[0].cpu().numpy()
+    for t in range(T):
+        qc, qs = O.mxfp4_quantize(inp.qI[0, t].reshape(1, -1))
+        nv = t // 4
+        s = O.mxfp4_index_scores(qc[0], qs[0], kc[:nv], ks[:nv])
+        ref, rc = O.topk(s, k)
+        assert gn[t] == rc and np.array_equal(gi[t], ref), t

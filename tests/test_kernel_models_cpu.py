@@ -1,7 +1,8 @@
 """Models, on the CPU, of the integer and bit-level schemes two kernels rely
 on, checked against the oracle and against plain sorting:
 
-* the FP4 indexer (mxfp4_quantize_kernel, score_decode_mxfp4_kernel): the
+* the FP4 indexer (mxfp4_quantize_kernel, score_decode_mxfp4_kernel and the
+  prefill kernel's int8 words, score_prefill_mxfp4_kernel): the
   e2m1 encoder by threshold compares, the E8M0 exponent from the fp32 bit
   pattern, the doubled-magnitude byte table picked by a byte permute, the
   sign applied by selecting +q or -q bytes, dp4a accumulation and the
@@ -216,3 +217,40 @@ def test_context_parallel_merge_scheme_matches_sorting():
             assert R == len(want) and sel[:R] == want and all(v == -1 for v in sel[R:]), trial
             mine = [j - int(bases[rank]) for j in want if bases[rank] <= j < bases[rank] + sizes[rank]]
             assert loc[:lc] == mine and all(v == -1 for v in loc[lc:]), trial
+
+
+def test_fp4_prefill_word_scheme_matches_the_oracle():
+    """The prefill kernel widens codes to doubled signed int8 (four to a word,
+    word w holding elements 32*(w//8) + 4*(w%8) ..) for queries and keys alike,
+    sums each block with dp4a and combines the blocks with their exponents."""
+    rng = np.random.default_rng(8)
+    keys = (rng.standard_normal((64, 64)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    qbits = (rng.standard_normal((5, 64)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    kc, ks = O.mxfp4_quantize(keys)
+    qc, qs = O.mxfp4_quantize(qbits)
+
+    def s8(code):  # doubled signed value as a byte
+        m = _byte_perm(LUT_LO, LUT_HI, code & 7) & 0xFF
+        return (-m if code & 8 else m) & 0xFF
+
+    def words_from_codes(row_codes):  # 32 code bytes -> 16 words of 4 bytes
+        out = []
+        for half in range(2):
+            cw = struct.unpack("<4I", bytes(row_codes[16 * half:16 * half + 16]))
+            for i in range(4):
+                lo = sum(s8((cw[i] >> (4 * j)) & 0xF) << (8 * j) for j in range(4))
+                hi = sum(s8((cw[i] >> (4 * (j + 4))) & 0xF) << (8 * j) for j in range(4))
+                out += [lo, hi]
+        return out
+    for qi in range(5):
+        qw = words_from_codes(qc[qi])
+        ref = O.mxfp4_index_scores(qc[qi], qs[qi], kc, ks)
+        for e in range(64):
+            kw = words_from_codes(kc[e])
+            A = [0, 0]
+            for w in range(16):
+                A[w // 8] = _dp4a(qw[w], kw[w], A[w // 8])
+            t = [np.float32(math.ldexp(A[b], int(qs[qi][b]) + int(ks[e][b]) - 256)) for b in range(2)]
+            s = np.float32(t[0] + t[1])
+            s = np.float32(0) if s == 0 else s
+            assert _f2u(s) == _f2u(ref[e]), (qi, e)
