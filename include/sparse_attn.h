@@ -237,6 +237,17 @@ sa_status hybrid_attn_decode(const void* q, const void* q_idx, int32_t H,
                              int32_t* idx_out, int32_t* cnt_out,
                              void* ws, size_t ws_bytes, void* stream);
 
+/* hybrid_attn_prefill with the CSA selection on FP4 indexer scores (the
+ * prefill selection of csa_index_topk_mxfp4; codes / scales as written by
+ * csa_index_quantize_mxfp4).  Same workspace, shapes and outputs; the bf16
+ * indexer keys of the CSA cache are not read and may be NULL.               */
+sa_status hybrid_attn_prefill_mxfp4(const void* q, const void* q_idx, int32_t T, int32_t H,
+                                    const sa_cache* csa, const sa_cache* hca,
+                                    const uint8_t* codes, const uint8_t* scales, int32_t k, float scale,
+                                    void* out_csa, void* out_hca, float* lse_csa, float* lse_hca,
+                                    int32_t* idx_out, int32_t* cnt_out,
+                                    void* ws, size_t ws_bytes, void* stream);
+
 /* hybrid_attn_decode with the sliding-window branch of both layers: the
  * review (section 3-2 (2)) adds a window of recent uncompressed tokens to CSA
  * and to HCA alike.  out_csa is the attention over the CSA selection joined

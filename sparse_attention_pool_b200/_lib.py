@@ -27,7 +27,7 @@ EXPORTS = ["csa_compress", "hca_compress", "csa_index_topk", "csa_sparse_attn", 
            "csa_index_topk_noalloc", "csa_append", "hca_append", "swa_attn", "attn_lse_merge",
            "csa_index_quantize_mxfp4", "csa_index_topk_mxfp4", "hybrid_attn_decode_mxfp4",
            "cp_decode_candidates", "cp_decode_merge_select", "attn_lse_merge_n", "hybrid_attn_decode_swa",
-           "sa_selftest_wait_timeout", "sa_trace_install", "sa_trace_count"]
+           "sa_selftest_wait_timeout", "sa_trace_install", "sa_trace_count", "hybrid_attn_prefill_mxfp4"]
 SA_NOALLOC_SCRATCH_BYTES = 32 << 20
 SA_STAGE_INDEX_SCORE, SA_STAGE_TOPK_SELECT, SA_STAGE_CSA_ATTN, SA_STAGE_HCA_ATTN = 0, 1, 2, 3
 
@@ -83,6 +83,7 @@ def lib():
         L.cp_decode_merge_select.argtypes = [P, P, P, I32, I32, I32, I32, P, P, P, P, P, P]
         L.attn_lse_merge_n.argtypes = [P, P, I32, ctypes.c_int64, P, P, P]
         L.hybrid_attn_decode_swa.argtypes = [P, P, I32, CP, CP, RP, I32, I32, F32, P, P, P, P, P, P, P, SZ, P]
+        L.hybrid_attn_prefill_mxfp4.argtypes = [P, P, I32, I32, CP, CP, P, P, I32, F32, P, P, P, P, P, P, P, SZ, P]
         L.hybrid_attn_decode_mxfp4.argtypes = [P, P, I32, CP, CP, P, P, I32, F32, P, P, P, P, P, P, P, SZ, P]
         L.hybrid_attn_prefill.argtypes = [P, P, I32, I32, CP, CP, I32, F32, P, P, P, P, P, P, P, SZ, P]
         L.sa_workspace_size.argtypes = [I32, I32, I32, I32, I32, I32, I32]

@@ -363,6 +363,25 @@ def hybrid_attn_decode_mxfp4(q, q_idx, csa: Cache, hca: Cache, codes, scales, k:
     return out_csa, out_hca
 
 
+def hybrid_attn_prefill_mxfp4(q, q_idx, csa: Cache, hca: Cache, codes, scales, k: int, ws, idx_out, cnt_out, *,
+                              scale=0.0, out_csa=None, out_hca=None, lse_csa=None, lse_hca=None, stream=None):
+    """hybrid_attn_prefill with the CSA selection on FP4 (MXFP4) indexer scores."""
+    _need(q, torch.bfloat16, "q")
+    _need(q_idx, torch.bfloat16, "q_idx")
+    _need(codes, torch.uint8, "codes")
+    _need(scales, torch.uint8, "scales")
+    T, H = q.shape[1], q.shape[2]
+    out_csa = torch.empty_like(q) if out_csa is None else out_csa
+    out_hca = torch.empty_like(q) if out_hca is None else out_hca
+    c, h = csa.struct(), hca.struct()
+    check("hybrid_attn_prefill_mxfp4",
+          lib().hybrid_attn_prefill_mxfp4(_ptr(q), _ptr(q_idx), T, H, ctypes.byref(c), ctypes.byref(h), _ptr(codes),
+                                          _ptr(scales), k, float(scale), _ptr(out_csa), _ptr(out_hca),
+                                          _ptr(lse_csa), _ptr(lse_hca), _ptr(idx_out), _ptr(cnt_out), _ptr(ws),
+                                          ws.numel(), _stream(stream)))
+    return out_csa, out_hca
+
+
 def hybrid_attn_prefill(q, q_idx, csa: Cache, hca: Cache, k: int, ws, idx_out, cnt_out, *, scale=0.0,
                         out_csa=None, out_hca=None, lse_csa=None, lse_hca=None, stream=None):
     """q [B][T][H][128] bf16, q_idx [B][T][64] bf16; idx_out [B][T][k], cnt_out [B][T] int32."""

@@ -1314,36 +1314,60 @@ sa_status hybrid_attn_decode_mxfp4(const void* q, const void* q_idx, int32_t H, 
                               out_hca, lse_csa, lse_hca, idx_out, cnt_out, ws, ws_bytes, stream);
 }
 
-sa_status hybrid_attn_prefill(const void* q, const void* q_idx, int32_t T, int32_t H, const sa_cache* csa,
-                              const sa_cache* hca, int32_t k, float scale, void* out_csa, void* out_hca,
-                              float* lse_csa, float* lse_hca, int32_t* idx_out, int32_t* cnt_out, void* ws,
-                              size_t ws_bytes, void* stream) {
-    sa_status r = check_cache(csa, true, "hybrid_attn_prefill(csa)");
+// Causal prefill of both branches; with MXFP4 indexer keys (codes4 /
+// scales4 non-NULL) the CSA selection runs on FP4 scores.
+static sa_status hybrid_prefill_impl(const char* what, const void* q, const void* q_idx, int32_t T, int32_t H,
+                                     const sa_cache* csa, const sa_cache* hca, const uint8_t* codes4,
+                                     const uint8_t* scales4, int32_t k, float scale, void* out_csa, void* out_hca,
+                                     float* lse_csa, float* lse_hca, int32_t* idx_out, int32_t* cnt_out, void* ws,
+                                     size_t ws_bytes, void* stream) {
+    const bool fp4 = codes4 != nullptr || scales4 != nullptr;
+    sa_status r = check_cache(csa, !fp4, fp4 ? "hybrid_attn_prefill_mxfp4(csa)" : "hybrid_attn_prefill(csa)");
     if (r != SA_OK) return r;
-    r = check_cache(hca, false, "hybrid_attn_prefill(hca)");
+    r = check_cache(hca, false, fp4 ? "hybrid_attn_prefill_mxfp4(hca)" : "hybrid_attn_prefill(hca)");
     if (r != SA_OK) return r;
-    r = check_common_q(q, H, "hybrid_attn_prefill");
+    r = check_common_q(q, H, what);
     if (r != SA_OK) return r;
-    SA_CHECK(csa->B == hca->B, "hybrid_attn_prefill: csa B=%d != hca B=%d", csa->B, hca->B);
-    SA_CHECK(T >= 1, "hybrid_attn_prefill: T=%d", T);
-    SA_CHECK(q_idx && aligned16(q_idx), "hybrid_attn_prefill: q_idx must be non-NULL and aligned");
-    SA_CHECK(k >= 1 && k <= 65536, "hybrid_attn_prefill: k=%d outside 1..65536", k);
-    SA_CHECK(out_csa && out_hca && aligned16(out_csa) && aligned16(out_hca), "hybrid_attn_prefill: outputs must be aligned");
-    SA_CHECK((!lse_csa || aligned16(lse_csa)) && (!lse_hca || aligned16(lse_hca)), "hybrid_attn_prefill: lse alignment");
+    if (fp4)
+        SA_CHECK(codes4 && scales4 && aligned16(codes4) && aligned16(scales4),
+                 "%s: codes and scales must be non-NULL and 16-byte aligned", what);
+    SA_CHECK(csa->B == hca->B, "%s: csa B=%d != hca B=%d", what, csa->B, hca->B);
+    SA_CHECK(T >= 1, "%s: T=%d", what, T);
+    SA_CHECK(q_idx && aligned16(q_idx), "%s: q_idx must be non-NULL and aligned", what);
+    SA_CHECK(k >= 1 && k <= 65536, "%s: k=%d outside 1..65536", what, k);
+    SA_CHECK(out_csa && out_hca && aligned16(out_csa) && aligned16(out_hca), "%s: outputs must be aligned", what);
+    SA_CHECK((!lse_csa || aligned16(lse_csa)) && (!lse_hca || aligned16(lse_hca)), "%s: lse alignment", what);
     SA_CHECK(idx_out && cnt_out && aligned16(idx_out) && aligned16(cnt_out),
-             "hybrid_attn_prefill: idx_out and cnt_out are required and must be aligned");
-    SA_CHECK(std::isfinite(scale) && scale >= 0.f, "hybrid_attn_prefill: scale must be finite and >= 0");
+             "%s: idx_out and cnt_out are required and must be aligned", what);
+    SA_CHECK(std::isfinite(scale) && scale >= 0.f, "%s: scale must be finite and >= 0", what);
     r = check_ws(ws, ws_bytes, sa_workspace_size(SA_OP_HYBRID_PREFILL, csa->B, T, H, csa->Ncap, hca->Ncap, k));
     if (r != SA_OK) return r;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // positions 0..T-1 for every sequence live in the workspace
     const int32_t* pos = prefill_positions(ws, csa->B, T, st);
     if (!pos) return fail(SA_ERR_CUDA, "could not write query positions");
-    r = run_topk_prefill(q_idx, T, pos, csa, k, idx_out, cnt_out, ws, st);
+    r = run_topk_prefill(q_idx, T, pos, csa, k, idx_out, cnt_out, ws, st, codes4, scales4);
     if (r != SA_OK) return r;
     r = run_attn(q, T, H, csa, true, idx_out, cnt_out, k, pos, scale, out_csa, lse_csa, ws, 0, st);
     if (r != SA_OK) return r;
     return run_attn(q, T, H, hca, false, nullptr, nullptr, 0, pos, scale, out_hca, lse_hca, ws, 0, st);
+}
+
+sa_status hybrid_attn_prefill(const void* q, const void* q_idx, int32_t T, int32_t H, const sa_cache* csa,
+                              const sa_cache* hca, int32_t k, float scale, void* out_csa, void* out_hca,
+                              float* lse_csa, float* lse_hca, int32_t* idx_out, int32_t* cnt_out, void* ws,
+                              size_t ws_bytes, void* stream) {
+    return hybrid_prefill_impl("hybrid_attn_prefill", q, q_idx, T, H, csa, hca, nullptr, nullptr, k, scale, out_csa,
+                               out_hca, lse_csa, lse_hca, idx_out, cnt_out, ws, ws_bytes, stream);
+}
+
+sa_status hybrid_attn_prefill_mxfp4(const void* q, const void* q_idx, int32_t T, int32_t H, const sa_cache* csa,
+                                    const sa_cache* hca, const uint8_t* codes, const uint8_t* scales, int32_t k,
+                                    float scale, void* out_csa, void* out_hca, float* lse_csa, float* lse_hca,
+                                    int32_t* idx_out, int32_t* cnt_out, void* ws, size_t ws_bytes, void* stream) {
+    SA_CHECK(codes && scales, "hybrid_attn_prefill_mxfp4: codes and scales must be non-NULL");
+    return hybrid_prefill_impl("hybrid_attn_prefill_mxfp4", q, q_idx, T, H, csa, hca, codes, scales, k, scale,
+                               out_csa, out_hca, lse_csa, lse_hca, idx_out, cnt_out, ws, ws_bytes, stream);
 }
 
 }  // extern "C"

@@ -282,3 +282,18 @@ def test_profiling_build_exports_every_header_symbol():
     T.sa_last_error.restype = ctypes.c_char_p
     # argument checks run before any CUDA call
     assert T.sa_trace_install(ctypes.c_void_p(0x10004), 8, None) == _lib.SA_ERR_INVALID_ARG
+
+
+def test_hybrid_prefill_mxfp4_rejects_bad_arguments(L):
+    c, h = _cache(kidx=None), _cache(m=128, kidx=None)
+    P = ctypes.c_void_p
+    f = L.hybrid_attn_prefill_mxfp4
+    rest = [8, 0.0, P(FAKE), P(FAKE), None, None, P(FAKE), P(FAKE), P(FAKE), 1 << 30, None]
+    assert f(P(FAKE), P(FAKE), 16, 8, ctypes.byref(c), ctypes.byref(h), None, P(FAKE), *rest) == 1
+    assert "codes" in L.sa_last_error().decode()
+    nocnt = [8, 0.0, P(FAKE), P(FAKE), None, None, P(FAKE), None, P(FAKE), 1 << 30, None]
+    assert f(P(FAKE), P(FAKE), 16, 8, ctypes.byref(c), ctypes.byref(h), P(FAKE), P(FAKE), *nocnt) == 1
+    assert "idx_out" in L.sa_last_error().decode()
+    # the bf16 prefill still needs the bf16 indexer keys
+    assert L.hybrid_attn_prefill(P(FAKE), P(FAKE), 16, 8, ctypes.byref(c), ctypes.byref(h), *rest) == 1
+    assert "kidx" in L.sa_last_error().decode()

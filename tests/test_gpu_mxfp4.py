@@ -182,3 +182,26 @@ def test_topk_prefill_every_row(S):
         s = O.mxfp4_index_scores(qc[0], qs[0], kc[:nv], ks[:nv])
         ref, rc = O.topk(s, k)
         assert gn[t] == rc and np.array_equal(gi[t], ref), t
+
+
+def test_hybrid_prefill_mxfp4_matches_oracle(S):
+    """Causal prefill of both branches with the CSA selection on FP4 scores:
+    every row's indices bit for bit, sampled rows' outputs within the bf16
+    tolerance."""
+    from tests._util import SCALE, TOL_BF16, Inputs, compress_on_gpu
+    B, T, H, k = 1, 1100, 64, 64
+    inp = Inputs(77, B, T, H, Tq=T)
+    g = inp.to_device()
+    csa, hca = compress_on_gpu(S, g, B, T)
+    codes, scales = S.csa_index_quantize_mxfp4(csa)
+    ws = S.alloc_workspace(S.workspace_size(S.SA_OP_HYBRID_PREFILL, B, T, H, csa.Ncap, hca.Ncap, k))
+    idx = torch.empty(B, T, k, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(B, T, dtype=torch.int32, device="cuda")
+    oc, oh = S.hybrid_attn_prefill_mxfp4(g["q"], g["qI"], csa, hca, codes, scales, k, ws, idx, cnt, scale=SCALE)
+    S.read_device_status()
+    cs = inp.oracle_seq(0)
+    for t in list(range(0, T, 11)) + [T - 1]:
+        r = O.hybrid_query_mxfp4(cs, inp.q[0, t], inp.qI[0, t], t=t, k=k, scale=SCALE)
+        assert int(cnt[0, t]) == r["cnt"] and np.array_equal(idx[0, t].cpu().numpy(), r["idx"]), t
+        assert np.abs(oc[0, t].float().cpu().numpy() - r["out_csa"]).max() <= TOL_BF16, t
+        assert np.abs(oh[0, t].float().cpu().numpy() - r["out_hca"]).max() <= TOL_BF16, t
