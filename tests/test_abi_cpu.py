@@ -297,3 +297,24 @@ def test_hybrid_prefill_mxfp4_rejects_bad_arguments(L):
     # the bf16 prefill still needs the bf16 indexer keys
     assert L.hybrid_attn_prefill(P(FAKE), P(FAKE), 16, 8, ctypes.byref(c), ctypes.byref(h), *rest) == 1
     assert "kidx" in L.sa_last_error().decode()
+
+
+def test_header_is_plain_c_and_cpp():
+    """The boundary is a C ABI: the header compiles as strict C99 and as C++17,
+    and a C caller links against the library's exports."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no gcc")
+    for std, lang in (("c99", "c"), ("c++17", "c++")):
+        subprocess.check_call([gcc, f"-std={std}", "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only",
+                               "-x", lang, HEADER])
+    caller = ("#include \"sparse_attn.h\"\n"
+              "int main(void) {\n"
+              "    size_t n = sa_workspace_size(SA_OP_HYBRID_DECODE, 4, 1, 64, 262144, 8192, 2048);\n"
+              "    return (sa_abi_version() == SA_ABI_VERSION && n > 0) ? 0 : 1;\n"
+              "}\n")
+    lib_dir = os.path.dirname(_lib.LIB_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), "-x", "c", "-", "-o",
+                    os.devnull, "-L", lib_dir, "-l:libsparse_attn.so"], input=caller.encode(), check=True)
