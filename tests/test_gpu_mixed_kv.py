@@ -156,3 +156,31 @@ def test_prefill_matches_oracle_every_row(S):
         rh, _ = _oracle_attn(inp.q[0, t], refh, np.arange(t // 128))
         worst = max(worst, float(np.abs(ocf[t] - rc).max()), float(np.abs(ohf[t] - rh).max()))
     assert worst <= TOL_FP8, worst
+
+
+def test_fp4_selection_on_mixed_storage(S):
+    """FP4 indexer scores and mixed KV storage together (the low-precision
+    decode step): indices bit for bit against the oracle's FP4 selection,
+    outputs within the fp8 tolerance against attention over the oracle's mixed
+    storage."""
+    B, Lcap, H, k = 2, 20000, 64, 512
+    inp = Inputs(907, B, Lcap, H, lengths=[20000, 7777])
+    g = inp.to_device()
+    csa, hca = _caches(S, B, Lcap)
+    S.csa_compress(g["K"], g["V"], g["KI"], g["len"], csa)
+    S.hca_compress(g["K"], g["V"], g["len"], hca)
+    codes, scales = S.csa_index_quantize_mxfp4(csa)
+    ws = S.alloc_workspace(S.workspace_size(S.SA_OP_HYBRID_DECODE, B, 1, H, csa.Ncap, hca.Ncap, k))
+    idx = torch.empty(B, k, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(B, dtype=torch.int32, device="cuda")
+    oc, oh = S.hybrid_attn_decode_mxfp4(g["q"], g["qI"], csa, hca, codes, scales, k, ws, scale=SCALE,
+                                        idx_out=idx, cnt_out=cnt)
+    S.read_device_status()
+    for b in range(B):
+        L = int(inp.lengths[b])
+        r = O.hybrid_query_mxfp4(inp.oracle_seq(b), inp.q[b], inp.qI[b], t=L, k=k, scale=SCALE)
+        assert int(cnt[b]) == r["cnt"] and np.array_equal(idx[b].cpu().numpy(), r["idx"]), b
+        ref_c = _oracle_attn(inp.q[b], _oracle_mixed(inp.K[b, :L], inp.V[b, :L], 4), r["idx"][:r["cnt"]])
+        ref_h = _oracle_attn(inp.q[b], _oracle_mixed(inp.K[b, :L], inp.V[b, :L], 128), np.arange(L // 128))
+        assert np.abs(oc[b].float().cpu().numpy() - ref_c[0]).max() <= TOL_FP8, b
+        assert np.abs(oh[b].float().cpu().numpy() - ref_h[0]).max() <= TOL_FP8, b
