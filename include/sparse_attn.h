@@ -391,7 +391,8 @@ sa_status csa_index_topk_noalloc(const void* q_idx, const sa_cache* csa, int32_t
  * Python binding); these calls are the per-rank compute.                   */
 
 /* Exact local top-k of this rank's CSA shard for B decode queries, then the
- * exact order key and global index of each winner.
+ * exact order key and global index of each winner (the four int32 arrays
+ * need 4-byte alignment: they may sit packed in one buffer).
  *   base  [B] int32: global index of the shard's entry 0.
  *   keys  [B][k] uint32 out: order key of the winner's fp32 score s: the
  *         bits of s with the sign bit set for s >= 0, all bits flipped for
@@ -406,24 +407,32 @@ sa_status cp_decode_candidates(const void* q_idx, const sa_cache* csa, int32_t k
 
 /* The global top-k from the gathered candidates of all W ranks and this
  * rank's share of it.
- *   keys, gidx [W][B][k], gcnt [W][B]: the candidate arrays of ranks 0..W-1
- *              stacked in rank order.
+ *   keys, gidx, gcnt: rank w's candidate arrays ([B][k], [B][k], [B]) start
+ *              at keys + w * stride_list, gidx + w * stride_list and
+ *              gcnt + w * stride_cnt (elements): arrays stacked in rank order
+ *              (stride_list = B*k, stride_cnt = B), or one packed
+ *              [keys | gidx | gcnt] int32 buffer per rank gathered whole
+ *              (both strides = 2*B*k + B), which needs one all-gather.
  *   base [B]: this rank's shard start (as given to cp_decode_candidates).
  *   local_idx [B][k] int32 out: this rank's winners as shard-local indices,
  *              ascending, -1 padded; local_cnt [B] out: their count.
  *   sel_idx [B][k] / sel_cnt [B] out, or both NULL: the global selection,
  *              ascending, -1 padded, and min(k, total candidates).
  * W * k must be at most 16384 (SA_ERR_UNSUPPORTED otherwise).              */
-sa_status cp_decode_merge_select(const uint32_t* keys, const int32_t* gidx, const int32_t* gcnt, int32_t W,
-                                 int32_t B, int32_t k, int32_t rank, const int32_t* base, int32_t* local_idx,
-                                 int32_t* local_cnt, int32_t* sel_idx, int32_t* sel_cnt, void* stream);
+sa_status cp_decode_merge_select(const uint32_t* keys, const int32_t* gidx, const int32_t* gcnt, int64_t stride_list,
+                                 int64_t stride_cnt, int32_t W, int32_t B, int32_t k, int32_t rank,
+                                 const int32_t* base, int32_t* local_idx, int32_t* local_cnt, int32_t* sel_idx,
+                                 int32_t* sel_cnt, void* stream);
 
 /* W-way log-sum-exp merge of attentions over disjoint key sets:
  * lse = log sum_w e^lse_w, out = sum_w e^lse_w out_w / e^lse.
- *   outs [W][rows][128] bf16, lses [W][rows] fp32; out [rows][128] bf16,
- *   lse [rows] fp32 or NULL.  A row whose lses are all -inf gets 0, -inf.   */
-sa_status attn_lse_merge_n(const void* outs, const float* lses, int32_t W, int64_t rows, void* out, float* lse,
-                           void* stream);
+ *   part w's [rows][128] bf16 outputs start at outs + w * stride_out and its
+ *   [rows] fp32 lse at lses + w * stride_lse (elements; stride_out a multiple
+ *   of 8): stacked arrays, or one gathered byte buffer per part.
+ *   out [rows][128] bf16, lse [rows] fp32 or NULL.  A row whose lses are all
+ *   -inf gets 0, -inf.                                                        */
+sa_status attn_lse_merge_n(const void* outs, const float* lses, int32_t W, int64_t rows, int64_t stride_out,
+                           int64_t stride_lse, void* out, float* lse, void* stream);
 
 /* Number of kernels this library has launched from the calling host thread
  * since the process started (a diagnostic counter; memsets are not kernels). */

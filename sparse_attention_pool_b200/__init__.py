@@ -7,7 +7,8 @@ from .api import (Cache, CapturedDecode, alloc_cache, alloc_workspace, attn_lse_
                   csa_index_topk, csa_index_topk_noalloc, hca_append, swa_attn,
                   csa_index_quantize_mxfp4, csa_index_topk_mxfp4, hybrid_attn_decode_mxfp4, hybrid_attn_decode_swa,
                   hybrid_attn_prefill_mxfp4,
-                  cp_decode_candidates, cp_decode_merge_select, attn_lse_merge_n,
+                  cp_decode_candidates, cp_decode_merge_select, cp_decode_merge_select_packed, attn_lse_merge_n,
+                  attn_lse_merge_n_packed,
                   csa_sparse_attn,
                   hca_compress, hca_dense_attn, hybrid_attn_decode, hybrid_attn_prefill, read_device_status,
                   selftest_wait_timeout,

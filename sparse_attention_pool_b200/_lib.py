@@ -80,8 +80,9 @@ def lib():
         L.hca_dense_attn.argtypes = [P, I32, I32, P, CP, F32, P, P, P, SZ, P]
         L.hybrid_attn_decode.argtypes = [P, P, I32, CP, CP, I32, F32, P, P, P, P, P, P, P, SZ, P]
         L.cp_decode_candidates.argtypes = [P, CP, I32, P, P, P, P, P, SZ, P]
-        L.cp_decode_merge_select.argtypes = [P, P, P, I32, I32, I32, I32, P, P, P, P, P, P]
-        L.attn_lse_merge_n.argtypes = [P, P, I32, ctypes.c_int64, P, P, P]
+        I64 = ctypes.c_int64
+        L.cp_decode_merge_select.argtypes = [P, P, P, I64, I64, I32, I32, I32, I32, P, P, P, P, P, P]
+        L.attn_lse_merge_n.argtypes = [P, P, I32, I64, I64, I64, P, P, P]
         L.hybrid_attn_decode_swa.argtypes = [P, P, I32, CP, CP, RP, I32, I32, F32, P, P, P, P, P, P, P, SZ, P]
         L.hybrid_attn_prefill_mxfp4.argtypes = [P, P, I32, I32, CP, CP, P, P, I32, F32, P, P, P, P, P, P, P, SZ, P]
         L.hybrid_attn_decode_mxfp4.argtypes = [P, P, I32, CP, CP, P, P, I32, F32, P, P, P, P, P, P, P, SZ, P]

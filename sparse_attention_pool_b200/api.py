@@ -257,14 +257,32 @@ def cp_decode_merge_select(keys, gidx, gcnt, rank: int, base, *, local_idx=None,
     for t, name in ((keys, "keys"), (gidx, "gidx"), (gcnt, "gcnt"), (base, "base")):
         _need(t, torch.int32, name)
     W, B, k = gidx.shape
-    dev = gidx.device
+    return _merge_select(keys.data_ptr(), gidx.data_ptr(), gcnt.data_ptr(), B * k, B, W, B, k, rank, base,
+                         gidx.device, local_idx, local_cnt, sel_idx, sel_cnt, stream)
+
+
+def cp_decode_merge_select_packed(gathered, B: int, k: int, rank: int, base, *, stream=None):
+    """The same from one gathered int32 buffer [W][L], rank w's row holding its
+    packed [keys B*k | gidx B*k | gcnt B] (L >= 2*B*k + B)."""
+    _need(gathered, torch.int32, "gathered")
+    _need(base, torch.int32, "base")
+    W, L = gathered.shape
+    p = gathered.data_ptr()
+    return _merge_select(p, p + 4 * B * k, p + 8 * B * k, L, L, W, B, k, rank, base, gathered.device,
+                         None, None, None, None, stream)
+
+
+def _merge_select(pk, pg, pc, stride_list, stride_cnt, W, B, k, rank, base, dev, local_idx, local_cnt, sel_idx,
+                  sel_cnt, stream):
     local_idx = torch.empty(B, k, dtype=torch.int32, device=dev) if local_idx is None else local_idx
     local_cnt = torch.empty(B, dtype=torch.int32, device=dev) if local_cnt is None else local_cnt
     sel_idx = torch.empty(B, k, dtype=torch.int32, device=dev) if sel_idx is None else sel_idx
     sel_cnt = torch.empty(B, dtype=torch.int32, device=dev) if sel_cnt is None else sel_cnt
+    P = ctypes.c_void_p
     check("cp_decode_merge_select",
-          lib().cp_decode_merge_select(_ptr(keys), _ptr(gidx), _ptr(gcnt), W, B, k, rank, _ptr(base), _ptr(local_idx),
-                                       _ptr(local_cnt), _ptr(sel_idx), _ptr(sel_cnt), _stream(stream)))
+          lib().cp_decode_merge_select(P(pk), P(pg), P(pc), stride_list, stride_cnt, W, B, k, rank, _ptr(base),
+                                       _ptr(local_idx), _ptr(local_cnt), _ptr(sel_idx), _ptr(sel_cnt),
+                                       _stream(stream)))
     return local_idx, local_cnt, sel_idx, sel_cnt
 
 
@@ -277,8 +295,25 @@ def attn_lse_merge_n(outs, lses, *, out=None, lse=None, stream=None):
     rows = lses[0].numel()
     out = torch.empty(outs.shape[1:], dtype=torch.bfloat16, device=outs.device) if out is None else out
     lse = torch.empty(lses.shape[1:], dtype=torch.float32, device=outs.device) if lse is None else lse
-    check("attn_lse_merge_n", lib().attn_lse_merge_n(_ptr(outs), _ptr(lses), W, rows, _ptr(out), _ptr(lse),
-                                                     _stream(stream)))
+    check("attn_lse_merge_n", lib().attn_lse_merge_n(_ptr(outs), _ptr(lses), W, rows, rows * 128, rows, _ptr(out),
+                                                     _ptr(lse), _stream(stream)))
+    return out, lse
+
+
+def attn_lse_merge_n_packed(gathered, rows: int, lse_offset: int, *, out=None, lse=None, stream=None):
+    """The same from one gathered byte buffer [W][L]: part w's [rows][128]
+    bf16 outputs at byte 0 of its row and its [rows] fp32 lse at byte
+    lse_offset (L a multiple of 16)."""
+    _need(gathered, torch.uint8, "gathered")
+    W, L = gathered.shape
+    if L % 16 or lse_offset % 4:
+        raise ValueError("packed partials: row bytes must be a multiple of 16, the lse offset of 4")
+    dev = gathered.device
+    out = torch.empty(rows, 128, dtype=torch.bfloat16, device=dev) if out is None else out
+    lse = torch.empty(rows, dtype=torch.float32, device=dev) if lse is None else lse
+    p = gathered.data_ptr()
+    check("attn_lse_merge_n", lib().attn_lse_merge_n(ctypes.c_void_p(p), ctypes.c_void_p(p + lse_offset), W, rows,
+                                                     L // 2, L // 4, _ptr(out), _ptr(lse), _stream(stream)))
     return out, lse
 
 

@@ -9,12 +9,16 @@ shard, so one decode step is exact:
 
   1. ``cp_decode_candidates``: this rank's exact local top-k, with the order
      key and global index of each winner;
-  2. all-gather of the candidates (k per rank and sequence);
+  2. one all-gather of the candidates (k per rank and sequence, packed with
+     their global indices and counts in one int32 buffer);
   3. ``cp_decode_merge_select``: the global top-k, and this rank's share;
   4. CSA attention over the share and HCA attention over the HCA shard, each
      with its log-sum-exp;
-  5. all-gather of the partials and one W-way log-sum-exp merge of both
-     branches (``attn_lse_merge_n``).
+  5. one all-gather of the partials (outputs and lse of both branches packed
+     in one byte buffer) and one W-way log-sum-exp merge (``attn_lse_merge_n``).
+
+Two collectives per step: at decode sizes their latency, not their bytes,
+is what they cost.
 
 Every rank ends with the same outputs and the same selection.  The compute
 runs in the library's kernels; this module holds the host logic: the shard
@@ -66,6 +70,24 @@ def workspace_size(B: int, H: int, Ncap_csa: int, Ncap_hca: int, k: int) -> int:
                S.workspace_size(SA_OP_DENSE_ATTN, B, 1, H, 0, Ncap_hca, 0))
 
 
+def candidate_layout(B: int, k: int) -> tuple[int, int, int, int]:
+    """One rank's packed candidates, in int32 elements: (offset of the keys,
+    of the global indices, of the counts, row length) = [keys B*k | gidx B*k
+    | counts B]."""
+    return 0, B * k, 2 * B * k, 2 * B * k + B
+
+
+def partial_layout(B: int, H: int) -> tuple[int, int, int, int]:
+    """One rank's packed partials, in bytes: (rows, bytes of the outputs,
+    offset of the lse, row length).  rows = 2*B*H (CSA then HCA); the
+    [rows][128] bf16 outputs come first, the [rows] fp32 lse at a 16-byte
+    boundary after them, the row padded to a multiple of 16 bytes."""
+    rows = 2 * B * H
+    o_bytes = rows * 128 * 2
+    l_off = -(-o_bytes // 16) * 16
+    return rows, o_bytes, l_off, -(-(l_off + rows * 4) // 16) * 16
+
+
 def gather_ranks(t: torch.Tensor, group=None) -> torch.Tensor:
     """All-gather `t` from every rank of the group into one [W, *t.shape]
     tensor, in rank order (each rank's slice written in place)."""
@@ -87,14 +109,22 @@ def cp_decode_step(q, q_idx, csa: S.Cache, hca: S.Cache, base_csa, k: int, ws, *
     rank."""
     rank = dist.get_rank(group)
     B, H = q.shape[0], q.shape[1]
-    keys, gidx, gcnt = S.cp_decode_candidates(q_idx, csa, k, base_csa, ws, stream=stream)
-    all_keys, all_gidx, all_gcnt = gather_ranks(keys, group), gather_ranks(gidx, group), gather_ranks(gcnt, group)
-    local_idx, local_cnt, sel_idx, sel_cnt = S.cp_decode_merge_select(all_keys, all_gidx, all_gcnt, rank, base_csa,
-                                                                      stream=stream)
-    part_o = torch.empty(2, B, H, 128, dtype=torch.bfloat16, device=q.device)
-    part_l = torch.empty(2, B, H, dtype=torch.float32, device=q.device)
+    dev = q.device
+    # candidates: [keys | global indices | counts], one int32 row per rank
+    ok, og, oc, ln = candidate_layout(B, k)
+    cand = torch.empty(ln, dtype=torch.int32, device=dev)
+    S.cp_decode_candidates(q_idx, csa, k, base_csa, ws, keys=cand[ok:og].view(B, k), gidx=cand[og:oc].view(B, k),
+                           gcnt=cand[oc:ln], stream=stream)
+    local_idx, local_cnt, sel_idx, sel_cnt = S.cp_decode_merge_select_packed(gather_ranks(cand, group), B, k, rank,
+                                                                             base_csa, stream=stream)
+    # partials: both branches' [2][B][H][128] bf16 outputs, then their [2][B][H] fp32 lse
+    rows, o_bytes, l_off, row_bytes = partial_layout(B, H)
+    part = torch.empty(row_bytes, dtype=torch.uint8, device=dev)
+    part_o = part[:o_bytes].view(torch.bfloat16).view(2, B, H, 128)
+    part_l = part[l_off:l_off + rows * 4].view(torch.float32).view(2, B, H)
     S.csa_sparse_attn(q, csa, local_idx, local_cnt, k, ws, scale=scale, out=part_o[0], lse=part_l[0], stream=stream)
     S.hca_dense_attn(q, hca, ws, scale=scale, out=part_o[1], lse=part_l[1], stream=stream)
     # both branches merge row by row in one launch
-    out, lse = S.attn_lse_merge_n(gather_ranks(part_o, group), gather_ranks(part_l, group), stream=stream)
+    out, lse = S.attn_lse_merge_n_packed(gather_ranks(part, group), rows, l_off, stream=stream)
+    out, lse = out.view(2, B, H, 128), lse.view(2, B, H)
     return out[0], out[1], lse[0], lse[1], sel_idx, sel_cnt

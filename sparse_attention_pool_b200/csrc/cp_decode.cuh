@@ -83,14 +83,15 @@ constexpr int kMergeMaxRanks = 64;
 constexpr size_t kMergeSmem = (size_t)kMergeCap * 8;
 
 struct MergeArgs {
-    const uint32_t* keys;  // [W][B][k] gathered candidate keys
-    const int32_t* gidx;   // [W][B][k]
-    const int32_t* gcnt;   // [W][B]
+    const uint32_t* keys;  // rank w's [B][k] candidate keys at keys + w * stride_list
+    const int32_t* gidx;   // rank w's [B][k] at gidx + w * stride_list
+    const int32_t* gcnt;   // rank w's [B] at gcnt + w * stride_cnt
     const int32_t* base;   // [B] this rank's shard start
     int32_t* local_idx;    // [B][k] out: this rank's winners, shard-local, ascending, -1 padded
     int32_t* local_cnt;    // [B] out
     int32_t* sel_idx;      // [B][k] out (or NULL): the global selection, ascending, -1 padded
     int32_t* sel_cnt;      // [B] out (or NULL)
+    long long stride_list, stride_cnt;  // elements between consecutive ranks' arrays
     int W, B, k, rank;
 };
 
@@ -113,7 +114,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) cp_merge_select_kernel(Merge
     if (tid == 0) {
         int o = 0;
         for (int w = 0; w < a.W; ++w) {
-            int c = a.gcnt[(size_t)w * a.B + b];
+            int c = a.gcnt[(size_t)w * a.stride_cnt + b];
             if (c < 0 || c > a.k) {
                 flag(DEV_LEN);
                 c = c < 0 ? 0 : a.k;
@@ -128,7 +129,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1) cp_merge_select_kernel(Merge
     for (uint32_t p = tid; p < C; p += kMergeThreads) {
         int w = 0;
         while (s_off[w + 1] <= (int)p) ++w;  // W is small
-        const size_t src = ((size_t)w * a.B + b) * a.k + (p - (uint32_t)s_off[w]);
+        const size_t src = (size_t)w * a.stride_list + (size_t)b * a.k + (p - (uint32_t)s_off[w]);
         lk[p] = __ldg(a.keys + src);
         li[p] = __ldg(a.gidx + src);
     }
@@ -180,20 +181,21 @@ __global__ void __launch_bounds__(kMergeThreads, 1) cp_merge_select_kernel(Merge
 // attention over their union: one warp per row, 4 dims a lane, fp32
 // accumulation, one rounding to bf16.
 __global__ void __launch_bounds__(256) attn_lse_merge_n_kernel(const uint16_t* outs, const float* lses, int W,
-                                                               long long rows, uint16_t* out, float* lse) {
+                                                               long long rows, long long stride_out,
+                                                               long long stride_lse, uint16_t* out, float* lse) {
     pdl_wait();
     pdl_release();
     const long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (r >= rows) return;
     float M = -INFINITY;
-    for (int w = 0; w < W; ++w) M = fmaxf(M, lses[(size_t)w * rows + r]);
+    for (int w = 0; w < W; ++w) M = fmaxf(M, lses[(size_t)w * stride_lse + r]);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     float ws = 0.f;
     for (int w = 0; w < W; ++w) {
-        const float l = lses[(size_t)w * rows + r];
+        const float l = lses[(size_t)w * stride_lse + r];
         const float wt = l == -INFINITY ? 0.f : __expf(l - M);
-        const uint2 v = *reinterpret_cast<const uint2*>(outs + ((size_t)w * rows + r) * 128 + lane * 4);
+        const uint2 v = *reinterpret_cast<const uint2*>(outs + (size_t)w * stride_out + (size_t)r * 128 + lane * 4);
         acc[0] += wt * bf16lo_f32(v.x);
         acc[1] += wt * bf16hi_f32(v.x);
         acc[2] += wt * bf16lo_f32(v.y);

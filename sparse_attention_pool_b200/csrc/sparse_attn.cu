@@ -1081,9 +1081,10 @@ sa_status cp_decode_candidates(const void* q_idx, const sa_cache* csa, int32_t k
     sa_status r = check_cache(csa, true, "cp_decode_candidates");
     if (r != SA_OK) return r;
     SA_CHECK(q_idx && aligned16(q_idx), "cp_decode_candidates: q_idx must be non-NULL and 16-byte aligned");
-    SA_CHECK(base && keys && gidx && gcnt && aligned16(base) && aligned16(keys) && aligned16(gidx) &&
-                 aligned16(gcnt),
-             "cp_decode_candidates: base, keys, gidx, gcnt must be non-NULL and 16-byte aligned");
+    SA_CHECK(base && keys && gidx && gcnt, "cp_decode_candidates: base, keys, gidx, gcnt must be non-NULL");
+    SA_CHECK(((reinterpret_cast<uintptr_t>(base) | reinterpret_cast<uintptr_t>(keys) |
+               reinterpret_cast<uintptr_t>(gidx) | reinterpret_cast<uintptr_t>(gcnt)) & 3u) == 0,
+             "cp_decode_candidates: base, keys, gidx, gcnt must be 4-byte aligned");
     SA_CHECK(k >= 1 && k <= 65536, "cp_decode_candidates: k=%d outside 1..65536", k);
     const TopkDecodeWs w = topk_decode_layout(csa->B, csa->Ncap, k, true);
     r = check_ws(ws, ws_bytes, w.total);
@@ -1111,9 +1112,10 @@ sa_status cp_decode_candidates(const void* q_idx, const sa_cache* csa, int32_t k
     return SA_OK;
 }
 
-sa_status cp_decode_merge_select(const uint32_t* keys, const int32_t* gidx, const int32_t* gcnt, int32_t W,
-                                 int32_t B, int32_t k, int32_t rank, const int32_t* base, int32_t* local_idx,
-                                 int32_t* local_cnt, int32_t* sel_idx, int32_t* sel_cnt, void* stream) {
+sa_status cp_decode_merge_select(const uint32_t* keys, const int32_t* gidx, const int32_t* gcnt, int64_t stride_list,
+                                 int64_t stride_cnt, int32_t W, int32_t B, int32_t k, int32_t rank,
+                                 const int32_t* base, int32_t* local_idx, int32_t* local_cnt, int32_t* sel_idx,
+                                 int32_t* sel_cnt, void* stream) {
     SA_CHECK(W >= 1 && W <= sa::kMergeMaxRanks, "cp_decode_merge_select: W=%d outside 1..%d", W, sa::kMergeMaxRanks);
     SA_CHECK(rank >= 0 && rank < W, "cp_decode_merge_select: rank=%d outside 0..W-1", rank);
     SA_CHECK(B >= 1 && B <= 65535, "cp_decode_merge_select: B=%d outside 1..65535", B);
@@ -1123,10 +1125,15 @@ sa_status cp_decode_merge_select(const uint32_t* keys, const int32_t* gidx, cons
                     sa::kMergeCap);
     SA_CHECK(keys && gidx && gcnt && base && local_idx && local_cnt,
              "cp_decode_merge_select: keys, gidx, gcnt, base, local_idx, local_cnt must be non-NULL");
+    SA_CHECK(stride_list >= (int64_t)B * k && stride_cnt >= B,
+             "cp_decode_merge_select: stride_list=%lld must be >= B*k and stride_cnt=%lld >= B",
+             (long long)stride_list, (long long)stride_cnt);
     SA_CHECK((sel_idx == nullptr) == (sel_cnt == nullptr), "cp_decode_merge_select: give sel_idx and sel_cnt or neither");
-    SA_CHECK(aligned16(keys) && aligned16(gidx) && aligned16(gcnt) && aligned16(base) && aligned16(local_idx) &&
-                 aligned16(local_cnt) && (!sel_idx || (aligned16(sel_idx) && aligned16(sel_cnt))),
-             "cp_decode_merge_select: pointers must be 16-byte aligned");
+    SA_CHECK(((reinterpret_cast<uintptr_t>(keys) | reinterpret_cast<uintptr_t>(gidx) |
+               reinterpret_cast<uintptr_t>(gcnt) | reinterpret_cast<uintptr_t>(base) |
+               reinterpret_cast<uintptr_t>(local_idx) | reinterpret_cast<uintptr_t>(local_cnt) |
+               reinterpret_cast<uintptr_t>(sel_idx) | reinterpret_cast<uintptr_t>(sel_cnt)) & 3u) == 0,
+             "cp_decode_merge_select: pointers must be 4-byte aligned");
     static std::atomic<uint64_t> init{0};
     if (!attr_done(init)) {
         SA_CUDA(cudaFuncSetAttribute(sa::cp_merge_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1142,6 +1149,8 @@ sa_status cp_decode_merge_select(const uint32_t* keys, const int32_t* gidx, cons
     a.local_cnt = local_cnt;
     a.sel_idx = sel_idx;
     a.sel_cnt = sel_cnt;
+    a.stride_list = stride_list;
+    a.stride_cnt = stride_cnt;
     a.W = W;
     a.B = B;
     a.k = k;
@@ -1151,18 +1160,22 @@ sa_status cp_decode_merge_select(const uint32_t* keys, const int32_t* gidx, cons
     return SA_OK;
 }
 
-sa_status attn_lse_merge_n(const void* outs, const float* lses, int32_t W, int64_t rows, void* out, float* lse,
-                           void* stream) {
+sa_status attn_lse_merge_n(const void* outs, const float* lses, int32_t W, int64_t rows, int64_t stride_out,
+                           int64_t stride_lse, void* out, float* lse, void* stream) {
     SA_CHECK(W >= 1 && W <= 1024, "attn_lse_merge_n: W=%d outside 1..1024", W);
     SA_CHECK(rows >= 0, "attn_lse_merge_n: rows=%lld", (long long)rows);
     SA_CHECK(outs && lses && out, "attn_lse_merge_n: outs, lses and out must be non-NULL");
-    SA_CHECK(aligned16(outs) && aligned16(lses) && aligned16(out) && (!lse || aligned16(lse)),
-             "attn_lse_merge_n: pointers must be 16-byte aligned");
+    SA_CHECK(stride_out >= rows * 128 && stride_out % 8 == 0 && stride_lse >= rows,
+             "attn_lse_merge_n: stride_out=%lld (>= rows*128, a multiple of 8) / stride_lse=%lld (>= rows)",
+             (long long)stride_out, (long long)stride_lse);
+    SA_CHECK(aligned16(outs) && aligned16(out) && (!lse || (reinterpret_cast<uintptr_t>(lse) & 3u) == 0) &&
+                 (reinterpret_cast<uintptr_t>(lses) & 3u) == 0,
+             "attn_lse_merge_n: outs and out must be 16-byte aligned, lses and lse 4-byte");
     if (rows == 0) return SA_OK;
     const long long blocks = (rows + 7) / 8;
     SA_CHECK(blocks <= 2147483647LL, "attn_lse_merge_n: too many rows");
     sa::attn_lse_merge_n_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const uint16_t*>(outs), lses, W, rows, static_cast<uint16_t*>(out), lse);
+        static_cast<const uint16_t*>(outs), lses, W, rows, stride_out, stride_lse, static_cast<uint16_t*>(out), lse);
     SA_LAUNCHED();
     return SA_OK;
 }

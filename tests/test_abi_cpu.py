@@ -220,19 +220,23 @@ def test_context_parallel_entry_points_reject_bad_arguments(L):
     ms = L.cp_decode_merge_select
     ok = [P(FAKE)] * 3
     outs = [P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), None]
-    assert ms(*ok, 0, 1, 8, 0, *outs) == 1                      # W = 0
-    assert ms(*ok, 2, 1, 8, 2, *outs) == 1                      # rank outside 0..W-1
+    assert ms(*ok, 8, 1, 0, 1, 8, 0, *outs) == 1                        # W = 0
+    assert ms(*ok, 8, 1, 2, 1, 8, 2, *outs) == 1                        # rank outside 0..W-1
     assert "rank" in L.sa_last_error().decode()
-    assert ms(*ok, 8, 1, 4096, 0, *outs) == _lib.SA_ERR_UNSUPPORTED  # 32768 candidates
-    assert ms(*ok, 2, 1, 8, 0, P(FAKE), P(FAKE), P(FAKE), P(FAKE), None, None) == 1  # sel_idx without sel_cnt
+    assert ms(*ok, 4096, 1, 8, 1, 4096, 0, *outs) == _lib.SA_ERR_UNSUPPORTED  # 32768 candidates
+    assert ms(*ok, 8, 1, 2, 1, 8, 0, P(FAKE), P(FAKE), P(FAKE), P(FAKE), None, None) == 1  # sel_idx without sel_cnt
     assert "sel_idx" in L.sa_last_error().decode()
-    assert ms(P(FAKE + 4), P(FAKE), P(FAKE), 2, 1, 8, 0, P(FAKE), P(FAKE), P(FAKE), None, None, None) == 1
+    assert ms(P(FAKE + 2), P(FAKE), P(FAKE), 8, 1, 2, 1, 8, 0, P(FAKE), P(FAKE), P(FAKE), None, None, None) == 1
     assert "aligned" in L.sa_last_error().decode()
+    assert ms(*ok, 7, 1, 2, 1, 8, 0, *outs) == 1                        # stride_list < B*k
+    assert "stride" in L.sa_last_error().decode()
     mn = L.attn_lse_merge_n
-    assert mn(P(FAKE), P(FAKE), 0, 8, P(FAKE), None, None) == 1
-    assert mn(P(FAKE), P(FAKE), 2, -1, P(FAKE), None, None) == 1
-    assert mn(P(FAKE), P(FAKE + 4), 2, 8, P(FAKE), None, None) == 1
-    assert mn(P(FAKE), P(FAKE), 2, 0, P(FAKE), None, None) == 0  # nothing to do
+    assert mn(P(FAKE), P(FAKE), 0, 8, 1024, 8, P(FAKE), None, None) == 1
+    assert mn(P(FAKE), P(FAKE), 2, -1, 1024, 8, P(FAKE), None, None) == 1
+    assert mn(P(FAKE), P(FAKE + 2), 2, 8, 1024, 8, P(FAKE), None, None) == 1
+    assert mn(P(FAKE), P(FAKE), 2, 8, 1020, 8, P(FAKE), None, None) == 1   # stride_out < rows * 128
+    assert mn(P(FAKE), P(FAKE), 2, 8, 1028, 8, P(FAKE), None, None) == 1   # not a multiple of 8
+    assert mn(P(FAKE), P(FAKE), 2, 0, 0, 0, P(FAKE), None, None) == 0      # nothing to do
     assert L.sa_workspace_size(7, 2, 1, 64, 262144, 0, 2048) > 0
     assert L.sa_workspace_size(7, 2, 2, 64, 262144, 0, 2048) == 0  # decode only
 

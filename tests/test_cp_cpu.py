@@ -1,9 +1,11 @@
 """Context-parallel decode on the host: the shard boundaries, the rank-ordered
 all-gather of sparse_attention_pool_b200.cp (gloo ranks on CPU), and the
 exchange protocol itself -- every rank computing its shard with the oracle,
-exchanging through cp.gather_ranks, selecting from the union of the local
-top-k lists and merging the partial attentions by log-sum-exp -- against the
-oracle's single-rank answer (indices exact, outputs to fp64 rounding).
+exchanging packed rows through cp.gather_ranks (cp.candidate_layout,
+cp.partial_layout), selecting from the union of the local top-k lists and
+merging the partial attentions by log-sum-exp -- against the oracle's
+single-rank answer (indices exact; outputs within the bf16 rounding of the
+exchanged partials).
 """
 from __future__ import annotations
 
@@ -92,12 +94,14 @@ def _rank_main(rank, world, port, L, k, out):
         gidx = np.full(k, -1, np.int32)
         keys[:cnt] = _order_key(s[idx[:cnt]])
         gidx[:cnt] = base + idx[:cnt]
-        # 2. exchange (rank order)
-        all_keys = CP.gather_ranks(torch.from_numpy(keys.view(np.int32)))
-        all_gidx = CP.gather_ranks(torch.from_numpy(gidx))
-        all_cnt = CP.gather_ranks(torch.tensor([cnt], dtype=torch.int32))
+        # 2. one exchange of the packed candidates (rank order)
+        ok_, og, oc_, ln = CP.candidate_layout(1, k)
+        row = np.zeros(ln, np.int32)
+        row[ok_:og], row[og:oc_], row[oc_] = keys.view(np.int32), gidx, cnt
+        allc = CP.gather_ranks(torch.from_numpy(row)).numpy()
+        all_keys, all_gidx, all_cnt = allc[:, ok_:og].view(np.uint32), allc[:, og:oc_], allc[:, oc_:oc_ + 1]
         # 3. the global top-k of the union, by plain sorting
-        cand = [(int(all_keys[w, i].numpy().view(np.uint32)), int(all_gidx[w, i]))
+        cand = [(int(all_keys[w, i]), int(all_gidx[w, i]))
                 for w in range(world) for i in range(int(all_cnt[w, 0]))]
         gl = sorted(cand, key=lambda c: (-c[0], c[1]))[:k]
         sel = sorted(g for _, g in gl)
@@ -105,10 +109,18 @@ def _rank_main(rank, world, port, L, k, out):
         # 4. partial attentions over this rank's share and HCA shard
         oc, lc = O.attention(q, ck, cv, np.asarray(mine, np.int32), sc)
         oh, lh = O.attention(q, hk, hv, np.arange(hk.shape[0], dtype=np.int32), sc)
-        # 5. exchange and merge by log-sum-exp
-        po = CP.gather_ranks(torch.from_numpy(np.stack([oc, oh])))
-        pl = CP.gather_ranks(torch.from_numpy(np.stack([lc, lh])))
-        po, pl = po.numpy(), pl.numpy()
+        # 5. one exchange of the packed partials, then the log-sum-exp merge
+        #    (the oracle's fp64 outputs travel as bf16 here, as on the GPU)
+        rows, o_bytes, l_off, row_bytes = CP.partial_layout(1, H)
+        buf = np.zeros(row_bytes, np.uint8)
+        o16 = np.stack([oc, oh]).astype(np.float32).view(np.uint32)
+        o16 = ((o16 + 0x7FFF + ((o16 >> 16) & 1)) >> 16).astype(np.uint16)  # RNE to bf16
+        buf[:o_bytes] = o16.reshape(-1).view(np.uint8)
+        buf[l_off:l_off + rows * 4] = np.stack([lc, lh]).astype(np.float32).reshape(-1).view(np.uint8)
+        allp = CP.gather_ranks(torch.from_numpy(buf)).numpy()
+        po = (allp[:, :o_bytes].copy().view(np.uint16).astype(np.uint32) << 16).view(np.float32)
+        po = po.astype(np.float64).reshape(world, 2, H, 128)
+        pl = allp[:, l_off:l_off + rows * 4].copy().view(np.float32).astype(np.float64).reshape(world, 2, H)
         M = pl.max(axis=0)
         wts = np.where(np.isneginf(pl), 0.0, np.exp(pl - np.where(np.isneginf(M), 0.0, M)))
         merged = (wts[..., None] * po).sum(axis=0) / wts.sum(axis=0)[..., None]
@@ -142,9 +154,20 @@ def test_exchange_protocol_matches_the_single_rank_oracle(world, L, k):
     want = ref["idx"][:ref["cnt"]].tolist()
     for rank, sel, merged, mlse, counts in res:
         assert sel == want, rank                      # the same exact selection on every rank
-        assert np.abs(merged[0] - ref["out_csa"]).max() < 1e-10, rank
-        assert np.abs(merged[1] - ref["out_hca"]).max() < 1e-10, rank
-        assert np.abs(mlse[0] - ref["lse_csa"]).max() < 1e-10, rank
+        # partials travelled as bf16 outputs and fp32 lse: the merge is within their rounding
+        assert np.abs(merged[0] - ref["out_csa"]).max() < 4e-3, rank
+        assert np.abs(merged[1] - ref["out_hca"]).max() < 4e-3, rank
+        assert np.abs(mlse[0] - ref["lse_csa"]).max() < 1e-5, rank
         if L >= 128:
-            assert np.abs(mlse[1] - ref["lse_hca"]).max() < 1e-10, rank
+            assert np.abs(mlse[1] - ref["lse_hca"]).max() < 1e-5, rank
         assert sum(counts) >= min(k, L // 4)          # the union holds at least the global top-k
+
+
+@pytest.mark.parametrize("B,k,H", [(1, 1, 1), (3, 300, 64), (4, 2048, 64), (2, 7, 3)])
+def test_packed_layouts(B, k, H):
+    ok, og, oc, ln = cp.candidate_layout(B, k)
+    assert (ok, og, oc, ln) == (0, B * k, 2 * B * k, 2 * B * k + B)
+    rows, o_bytes, l_off, row_bytes = cp.partial_layout(B, H)
+    assert rows == 2 * B * H and o_bytes == rows * 256
+    assert l_off % 16 == 0 and l_off >= o_bytes and row_bytes % 16 == 0 and row_bytes >= l_off + rows * 4
+    assert (row_bytes // 2) % 8 == 0  # the bf16 stride between ranks suits 8-byte loads
