@@ -27,6 +27,8 @@ boundaries and the collectives (NCCL over NVLink on B200s; any backend whose
 """
 from __future__ import annotations
 
+import contextlib
+
 import torch
 import torch.distributed as dist
 
@@ -106,7 +108,13 @@ def cp_decode_step(q, q_idx, csa: S.Cache, hca: S.Cache, base_csa, k: int, ws, *
     the CSA shard's entry 0 (entry_base).  Returns (out_csa, out_hca, lse_csa,
     lse_hca, sel_idx, sel_cnt): the outputs of the whole sequence and the
     global selection (ascending global indices, -1 padded), equal on every
-    rank."""
+    rank.  Kernels and collectives are ordered on one stream: `stream`, made
+    current for the step, or the current one."""
+    with (torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()):
+        return _step(q, q_idx, csa, hca, base_csa, k, ws, group, scale)
+
+
+def _step(q, q_idx, csa, hca, base_csa, k, ws, group, scale):
     rank = dist.get_rank(group)
     B, H = q.shape[0], q.shape[1]
     dev = q.device
@@ -114,17 +122,17 @@ def cp_decode_step(q, q_idx, csa: S.Cache, hca: S.Cache, base_csa, k: int, ws, *
     ok, og, oc, ln = candidate_layout(B, k)
     cand = torch.empty(ln, dtype=torch.int32, device=dev)
     S.cp_decode_candidates(q_idx, csa, k, base_csa, ws, keys=cand[ok:og].view(B, k), gidx=cand[og:oc].view(B, k),
-                           gcnt=cand[oc:ln], stream=stream)
+                           gcnt=cand[oc:ln])
     local_idx, local_cnt, sel_idx, sel_cnt = S.cp_decode_merge_select_packed(gather_ranks(cand, group), B, k, rank,
-                                                                             base_csa, stream=stream)
+                                                                             base_csa)
     # partials: both branches' [2][B][H][128] bf16 outputs, then their [2][B][H] fp32 lse
     rows, o_bytes, l_off, row_bytes = partial_layout(B, H)
     part = torch.empty(row_bytes, dtype=torch.uint8, device=dev)
     part_o = part[:o_bytes].view(torch.bfloat16).view(2, B, H, 128)
     part_l = part[l_off:l_off + rows * 4].view(torch.float32).view(2, B, H)
-    S.csa_sparse_attn(q, csa, local_idx, local_cnt, k, ws, scale=scale, out=part_o[0], lse=part_l[0], stream=stream)
-    S.hca_dense_attn(q, hca, ws, scale=scale, out=part_o[1], lse=part_l[1], stream=stream)
+    S.csa_sparse_attn(q, csa, local_idx, local_cnt, k, ws, scale=scale, out=part_o[0], lse=part_l[0])
+    S.hca_dense_attn(q, hca, ws, scale=scale, out=part_o[1], lse=part_l[1])
     # both branches merge row by row in one launch
-    out, lse = S.attn_lse_merge_n_packed(gather_ranks(part, group), rows, l_off, stream=stream)
+    out, lse = S.attn_lse_merge_n_packed(gather_ranks(part, group), rows, l_off)
     out, lse = out.view(2, B, H, 128), lse.view(2, B, H)
     return out[0], out[1], lse[0], lse[1], sel_idx, sel_cnt
