@@ -90,8 +90,8 @@ def _oracle_topk(qI_bits, kidx_bits, n, k):
 
 @pytest.mark.parametrize("k", [64, 512])
 def test_topk_matches_oracle(S, k):
-    B, Ncap = 5, 20000
-    n = [20000, 9000, k + 1, k, 3]  # large, ragged, one above k, exactly k, fewer than k
+    B, Ncap = 6, 20000
+    n = [20000, 9000, k + 1, k, 3, 0]  # large, ragged, one above k, exactly k, fewer than k, empty
     bits = synth.normal_bf16(72, "kidx", (B, Ncap, 64))
     qI = synth.normal_bf16(72, "qidx", (B, 64))
     c = _cache_with_keys(S, bits, n)
