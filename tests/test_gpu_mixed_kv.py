@@ -184,3 +184,17 @@ def test_fp4_selection_on_mixed_storage(S):
         ref_h = _oracle_attn(inp.q[b], _oracle_mixed(inp.K[b, :L], inp.V[b, :L], 128), np.arange(L // 128))
         assert np.abs(oc[b].float().cpu().numpy() - ref_c[0]).max() <= TOL_FP8, b
         assert np.abs(oh[b].float().cpu().numpy() - ref_h[0]).max() <= TOL_FP8, b
+
+
+def test_mixed_decode_deterministic(S):
+    B, Lcap, H, k = 2, 16000, 64, 512
+    inp = Inputs(908, B, Lcap, H, lengths=[16000, 5000])
+    g = inp.to_device()
+    csa, hca = _caches(S, B, Lcap)
+    S.csa_compress(g["K"], g["V"], g["KI"], g["len"], csa)
+    S.hca_compress(g["K"], g["V"], g["len"], hca)
+    ws = S.alloc_workspace(S.workspace_size(S.SA_OP_HYBRID_DECODE, B, 1, H, csa.Ncap, hca.Ncap, k))
+    a = S.hybrid_attn_decode(g["q"], g["qI"], csa, hca, k, ws, scale=SCALE)
+    b = S.hybrid_attn_decode(g["q"], g["qI"], csa, hca, k, ws, scale=SCALE)
+    S.read_device_status()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])

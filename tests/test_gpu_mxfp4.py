@@ -205,3 +205,27 @@ def test_hybrid_prefill_mxfp4_matches_oracle(S):
         assert int(cnt[0, t]) == r["cnt"] and np.array_equal(idx[0, t].cpu().numpy(), r["idx"]), t
         assert np.abs(oc[0, t].float().cpu().numpy() - r["out_csa"]).max() <= TOL_BF16, t
         assert np.abs(oh[0, t].float().cpu().numpy() - r["out_hca"]).max() <= TOL_BF16, t
+
+
+def test_fp4_selection_deterministic_and_batch_invariant(S):
+    """Run to run the same bits, and a sequence alone selects what it selects
+    inside a batch."""
+    B, Ncap, k = 3, 30000, 512
+    bits = synth.normal_bf16(78, "kidx", (B, Ncap, 64))
+    qI = synth.normal_bf16(78, "qidx", (B, 64))
+    n = [30000, 17000, 900]
+    c = _cache_with_keys(S, bits, n)
+    codes, scales = S.csa_index_quantize_mxfp4(c)
+    ws = S.alloc_workspace(S.workspace_size(S.SA_OP_INDEX_TOPK, B, 1, 8, Ncap, 0, k))
+    q = bits_to_torch_bf16(qI).cuda()
+    i1, c1 = S.csa_index_topk_mxfp4(q, c, codes, scales, k, ws)
+    i2, c2 = S.csa_index_topk_mxfp4(q, c, codes, scales, k, ws)
+    S.read_device_status()
+    assert torch.equal(i1, i2) and torch.equal(c1, c2)
+    for b in range(B):
+        cb = _cache_with_keys(S, bits[b:b + 1], [n[b]])
+        cdb, scb = S.csa_index_quantize_mxfp4(cb)
+        wsb = S.alloc_workspace(S.workspace_size(S.SA_OP_INDEX_TOPK, 1, 1, 8, Ncap, 0, k))
+        ib, cnb = S.csa_index_topk_mxfp4(q[b:b + 1].contiguous(), cb, cdb, scb, k, wsb)
+        S.read_device_status()
+        assert torch.equal(ib[0], i1[b]) and torch.equal(cnb[0], c1[b]), b
