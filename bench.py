@@ -508,6 +508,9 @@ def run_ours(args, w, rank, world, dev):
         "clocks": clk.summary(),
         "setup_s": round(time.time() - t_gen, 1),
     }
+    if step_bytes < 8_000_000:  # a step this small is bound by launch latency, not by HBM
+        result["roofline"]["note"] = (f"{step_bytes / 1e6:.2f} MB per step: launch-latency bound; "
+                                      "the fraction does not measure the kernel")
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"], cs = cpu_baseline(w, lengths, K, V, KI, q_h, qI_h, budget_s=args.cpu_budget,
                                                   indexer=args.indexer, kv=args.kv)
