@@ -59,10 +59,12 @@ def _shards(S, inp, W):
     return out
 
 
-@pytest.mark.parametrize("W,k", [(2, 512), (4, 2048), (3, 64)])
-def test_emulated_ranks_match_the_single_gpu_step(S, W, k):
-    B, Lcap, H = 3, 40000, 64
-    inp = Inputs(921 + W, B, Lcap, H, lengths=[40000, 23457, 1000])
+@pytest.mark.parametrize("W,k,lengths", [(2, 512, [40000, 23457, 1000]), (4, 2048, [40000, 23457, 1000]),
+                                         (3, 64, [40000, 23457, 1000]),
+                                         (3, 64, [5000, 200, 130])])  # shards of 200 / 130 tokens: some empty
+def test_emulated_ranks_match_the_single_gpu_step(S, W, k, lengths):
+    B, Lcap, H = 3, max(lengths), 64
+    inp = Inputs(921 + W, B, Lcap, H, lengths=lengths)
     g = inp.to_device()
     csa, hca = compress_on_gpu(S, g, B, Lcap)
     ws = S.alloc_workspace(S.workspace_size(S.SA_OP_HYBRID_DECODE, B, 1, H, csa.Ncap, hca.Ncap, k))
