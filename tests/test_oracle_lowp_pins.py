@@ -346,3 +346,21 @@ def test_hybrid_query_mxfp4_composition():
     o, lse = O.attention(q, cs.ck, cs.cv, idx, sc)
     assert np.array_equal(o, r4["out_csa"]) and np.array_equal(lse, r4["lse_csa"])
     assert len(set(idx.tolist()) & set(r16["idx"].tolist())) > k // 2  # FP4 keeps most of the bf16 selection
+
+
+def test_hybrid_query_mxfp4_without_visible_entries():
+    """A query before the first complete block sees nothing: count 0, -1
+    padding, zero outputs and lse -inf in both branches (as the bf16 path)."""
+    rng = np.random.default_rng(52)
+
+    def bits(shape):
+        return (rng.standard_normal(shape).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    cs = O.CompressedSeq(bits((600, 128)), bits((600, 128)), bits((600, 64)))
+    q, qI = bits((4, 128)), bits(64)
+    for t in (0, 1, 3):
+        r = O.hybrid_query_mxfp4(cs, q, qI, t=t, k=16, scale=0.1)
+        assert r["cnt"] == 0 and (r["idx"] == -1).all()
+        assert not r["out_csa"].any() and np.isneginf(r["lse_csa"]).all()
+        assert not r["out_hca"].any() and np.isneginf(r["lse_hca"]).all()
+    r = O.hybrid_query_mxfp4(cs, q, qI, t=4, k=16, scale=0.1)  # the first entry becomes visible
+    assert r["cnt"] == 1 and r["idx"][0] == 0
