@@ -89,3 +89,22 @@ def test_compress_bytes_match_the_worked_figures():
     nc, nh = 16385, 512
     assert c8 == nc * 4 * 640 + nc * (256 + 128) + ((nc + 63) // 64) * 8
     assert h8 == nh * 128 * 512 + nh * 256 + ((nh + 63) // 64) * 8
+
+
+def test_mixed_storage_oracle_leg_is_the_pinned_pieces():
+    """The bench's oracle leg for mixed storage selects what the bf16 oracle
+    selects and attends with attention_kv over the oracle's mixed storage."""
+    from oracle import oracle as O
+    w = configs.BY_NAME["decode_b1_t4k_h8_k64"]
+    lengths, K, V, KI, q, qI = bench.make_inputs(w, 0)
+    L = int(lengths[0])
+    cs = O.CompressedSeq(K[0, :L], V[0, :L], KI[0, :L])
+    r = bench.oracle_query(w, cs, q[0], qI[0], L, "bf16", "mixed")
+    r16 = O.hybrid_query(cs, q[0], qI[0], t=L, k=w.topk, scale=bench.SCALE)
+    assert r["cnt"] == r16["cnt"] and np.array_equal(r["idx"], r16["idx"])
+    codes, ks, rope = O.mixed_quantize(cs.ck_bf16, 64)
+    vc, vs = O.fp8_quantize(cs.cv_bf16)
+    oc, _ = O.attention_kv(q[0], {"mode": "mixed", "data": codes, "scales": ks, "rope": rope},
+                           {"mode": "fp8", "data": vc, "scales": vs}, r16["idx"][:r16["cnt"]], bench.SCALE)
+    assert np.array_equal(r["out_csa"], oc)
+    assert np.abs(r["out_csa"] - r16["out_csa"]).max() < 3e-2  # storage rounding only
