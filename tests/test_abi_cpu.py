@@ -322,3 +322,20 @@ def test_header_is_plain_c_and_cpp():
     lib_dir = os.path.dirname(_lib.LIB_PATH)
     subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), "-x", "c", "-", "-o",
                     os.devnull, "-L", lib_dir, "-l:libsparse_attn.so"], input=caller.encode(), check=True)
+
+
+@pytest.mark.parametrize("op", [1, 2, 3, 4, 5, 6, 7, 8])
+def test_workspace_sizes_are_monotone(L, op):
+    """Every op's scratch never shrinks as the batch, the capacities or k grow."""
+    ws = L.sa_workspace_size
+    Tq = 4096 if op in (5,) else 1
+    base = dict(B=2, Tq=Tq, H=64, Nc=65536, Nh=2048, k=512)
+
+    def size(**kw):
+        a = dict(base, **kw)
+        return ws(op, a["B"], a["Tq"], a["H"], a["Nc"], a["Nh"], a["k"])
+    s0 = size()
+    assert s0 >= 0
+    for key, bigger in (("B", 4), ("Nc", 262144), ("Nh", 8192), ("k", 2048), ("H", 128)):
+        assert size(**{key: bigger}) >= s0, key
+    assert ws(8, 4, 1, 64, 262144, 8192, 2048) >= ws(4, 4, 1, 64, 262144, 8192, 2048)
