@@ -8,6 +8,7 @@
 
 #include <atomic>
 #include <cmath>
+#include <functional>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -1221,11 +1222,14 @@ sa_status hca_dense_attn(const void* q, int32_t Tq, int32_t H, const int32_t* q_
 
 // One decode step of both branches; with MXFP4 indexer keys (codes4 /
 // scales4 non-NULL) the CSA selection runs on FP4 scores.
+// `side_extra`, when given, queues more independent work on the side stream
+// after the HCA branch (it joins the caller's stream with it).
 static sa_status hybrid_decode_impl(const char* what, const void* q, const void* q_idx, int32_t H,
                                     const sa_cache* csa, const sa_cache* hca, const uint8_t* codes4,
                                     const uint8_t* scales4, int32_t k, float scale, void* out_csa, void* out_hca,
                                     float* lse_csa, float* lse_hca, int32_t* idx_out, int32_t* cnt_out, void* ws,
-                                    size_t ws_bytes, void* stream) {
+                                    size_t ws_bytes, void* stream,
+                                    const std::function<sa_status(cudaStream_t)>& side_extra = nullptr) {
     const bool fp4 = codes4 != nullptr || scales4 != nullptr;
     sa_status r = check_cache(csa, !fp4, fp4 ? "hybrid_attn_decode_mxfp4(csa)" : "hybrid_attn_decode(csa)");
     if (r != SA_OK) return r;
@@ -1268,6 +1272,10 @@ static sa_status hybrid_decode_impl(const char* what, const void* q, const void*
                                 w.total + attn_partial_bytes(csa->B, sc.splits, H), side->s);
         if (rr != SA_OK) return rr;
         stage_mark(SA_STAGE_HCA_ATTN, 1, side->s);
+        if (side_extra) {
+            rr = side_extra(side->s);
+            if (rr != SA_OK) return rr;
+        }
         SA_CUDA(cudaEventRecord(side->join, side->s));
         return SA_OK;
     };
@@ -1296,6 +1304,13 @@ sa_status hybrid_attn_decode_swa(const void* q, const void* q_idx, int32_t H, co
     SA_CHECK(raw != nullptr, "hybrid_attn_decode_swa: raw descriptor is NULL");
     SA_CHECK(raw->B == csa->B, "hybrid_attn_decode_swa: raw B=%d != csa B=%d", raw->B, csa->B);
     SA_CHECK(window >= 1, "hybrid_attn_decode_swa: window=%d", window);
+    // every check of the window call, here: it runs on the side stream once the
+    // step is queued, where a refusal would leave that stream unjoined
+    SA_CHECK(raw->Lcap >= 0 && raw->d == 128, "hybrid_attn_decode_swa: raw Lcap=%d d=%d", raw->Lcap, raw->d);
+    SA_CHECK(raw->k && raw->v && raw->len && aligned16(raw->k) && aligned16(raw->v) && aligned16(raw->len),
+             "hybrid_attn_decode_swa: raw k, v, len must be non-NULL and 16-byte aligned");
+    SA_CHECK(std::isfinite(scale) && scale >= 0.f, "hybrid_attn_decode_swa: scale must be finite and >= 0");
+    SA_CHECK(q != nullptr && aligned16(q), "hybrid_attn_decode_swa: q must be non-NULL and 16-byte aligned");
     SA_CHECK(H >= 1 && H <= 128, "hybrid_attn_decode_swa: H=%d outside 1..128", H);
     SA_CHECK(k >= 1 && k <= 65536, "hybrid_attn_decode_swa: k=%d outside 1..65536", k);
     const SwaDecodeWs w = swa_decode_layout(csa->B, H, csa->Ncap, hca->Ncap, k);
@@ -1304,13 +1319,16 @@ sa_status hybrid_attn_decode_swa(const void* q, const void* q_idx, int32_t H, co
     uint8_t* base = static_cast<uint8_t*>(ws);
     float* lc = lse_csa ? lse_csa : reinterpret_cast<float*>(base + w.lse_c);
     float* lh = lse_hca ? lse_hca : reinterpret_cast<float*>(base + w.lse_h);
-    r = hybrid_decode_impl("hybrid_attn_decode_swa", q, q_idx, H, csa, hca, nullptr, nullptr, k, scale, out_csa,
-                           out_hca, lc, lh, idx_out, cnt_out, ws, w.win_ws, stream);
-    if (r != SA_OK) return r;
-    // the window over the raw tokens, once for both layers, then one merge each
+    // the window over the raw tokens, once for both layers: it needs neither
+    // the indexer nor the top-k, so it runs on the side stream after the HCA
+    // branch, beside the CSA chain; then one merge each on the caller's stream
     void* wo = base + w.win_out;
     float* wl = reinterpret_cast<float*>(base + w.win_lse);
-    r = swa_attn(q, 1, H, nullptr, raw, window, scale, wo, wl, base + w.win_ws, w.win_out - w.win_ws, stream);
+    auto window_attn = [&](cudaStream_t s) -> sa_status {
+        return swa_attn(q, 1, H, nullptr, raw, window, scale, wo, wl, base + w.win_ws, w.win_out - w.win_ws, s);
+    };
+    r = hybrid_decode_impl("hybrid_attn_decode_swa", q, q_idx, H, csa, hca, nullptr, nullptr, k, scale, out_csa,
+                           out_hca, lc, lh, idx_out, cnt_out, ws, w.win_ws, stream, window_attn);
     if (r != SA_OK) return r;
     const int64_t rows = (int64_t)csa->B * H;
     r = attn_lse_merge(out_csa, lc, wo, wl, rows, out_csa, lc, stream);
