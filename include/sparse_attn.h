@@ -312,14 +312,20 @@ sa_status sa_selftest_wait_timeout(uint32_t wait_tries, void* stream);
 
 /* Device timelines (a profiling build only).  A library compiled with
  * -DSA_TRACE (libsparse_attn_trace.so) has per-CTA phase marks in its
- * decode-path kernels: thread 0 of a CTA appends a 16-byte record
+ * decode-path kernels and in the prefill indexer's score and selection
+ * kernels: thread 0 of a CTA appends a 16-byte record
  *   { uint64 t_ns (%globaltimer); uint16 kernel; uint16 phase; uint16 sm;
  *     uint16 cta (blockIdx.x + gridDim.x * blockIdx.y, mod 2^16) }
  * kernel: 1 indexer score, 2 filter, 3 resolve, 4 emit, 5 attention split,
- * 6 split merge, 7 FP4 indexer score.  Phases: score 0 start, 1 scan done,
- * 2 threshold found (last CTA); filter 0 start, 1 rows done; resolve 0
+ * 6 split merge, 7 FP4 indexer score, 8 prefill indexer score, 9 prefill
+ * selection, 10 FP4 prefill indexer score.  Phases: score 0 start, 1 scan
+ * done, 2 threshold found (last CTA); filter 0 start, 1 rows done; resolve 0
  * start, 1 counts scanned, 2 candidates gathered, 3 t~ known, 4 band done,
- * 5 cut done, 6 positions written; emit, attention 0 start, 1 end; merge 0.
+ * 5 cut done, 6 positions written; emit, attention 0 start, 1 end; merge 0;
+ * prefill scores (CTAs whose tile some query sees) 0 start, 1 operands
+ * staged, 2 end; prefill selection (one CTA per query) 0 start, then, when
+ * the query sees more than k entries, 1 keys staged, 2..4 digits 1..3
+ * found, 5 ties resolved, 6 end.
  * sa_trace_install(buf, capacity) waits for `stream`, then makes buf (device
  * memory, 16-byte aligned, capacity records) the destination and resets the
  * count; capacity 0 switches tracing off.  sa_trace_count waits for `stream`

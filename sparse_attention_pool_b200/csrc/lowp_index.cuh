@@ -295,6 +295,7 @@ __global__ void __launch_bounds__(kPsThreads, 2) score_prefill_mxfp4_kernel(Topk
     if (tid < kPsQ && ql0 + tid < a.qb) atomicMax(&s_maxvis, visible_entries(a, a.t0 + ql0 + tid));
     __syncthreads();
     if (e0 >= s_maxvis) return;  // no query of this tile sees these entries
+    SA_TRACE_MARK(TR_PSCORE_FP4, 0);
 
     if (tid < 2 * kPsQ) {  // one thread per (query, 32-dim block): quantize
         const int ql = tid >> 1, blk = tid & 1;
@@ -349,6 +350,7 @@ __global__ void __launch_bounds__(kPsThreads, 2) score_prefill_mxfp4_kernel(Topk
         }
     }
     __syncthreads();
+    SA_TRACE_MARK(TR_PSCORE_FP4, 1);
 
     const int tq = tid >> 4, te = tid & 15;
     int acc[2][4][8];
@@ -392,6 +394,7 @@ __global__ void __launch_bounds__(kPsThreads, 2) score_prefill_mxfp4_kernel(Topk
         *reinterpret_cast<uint4*>(row + te * 4) = make_uint4(kk[0], kk[1], kk[2], kk[3]);
         *reinterpret_cast<uint4*>(row + 64 + te * 4) = make_uint4(kk[4], kk[5], kk[6], kk[7]);
     }
+    SA_TRACE_MARK(TR_PSCORE_FP4, 2);
 }
 
 }  // namespace sa

@@ -66,6 +66,7 @@ __global__ void __launch_bounds__(kPsThreads, 2) score_prefill_kernel(TopkPrefil
     if (tid < kPsQ && ql0 + tid < a.qb) atomicMax(&s_maxvis, visible_entries(a, a.t0 + ql0 + tid));
     __syncthreads();
     if (e0 >= s_maxvis) return;  // no query of this tile sees these entries
+    SA_TRACE_MARK(TR_PSCORE, 0);
 
     {  // queries: q * 2^768 as fp64, dim-major
         const int ql = tid & 63;
@@ -94,6 +95,7 @@ __global__ void __launch_bounds__(kPsThreads, 2) score_prefill_kernel(TopkPrefil
         }
     }
     __syncthreads();
+    SA_TRACE_MARK(TR_PSCORE, 1);
 
     const int tq = tid >> 4, te = tid & 15;
     double acc[4][8];
@@ -137,6 +139,7 @@ __global__ void __launch_bounds__(kPsThreads, 2) score_prefill_kernel(TopkPrefil
         *reinterpret_cast<uint4*>(row + te * 4) = lo;       // KS is a multiple of 128: in bounds
         *reinterpret_cast<uint4*>(row + 64 + te * 4) = hi;
     }
+    SA_TRACE_MARK(TR_PSCORE, 2);
 }
 
 __global__ void __launch_bounds__(kPselThreads, 1) select_prefill_kernel(TopkPrefillArgs a) {
@@ -148,6 +151,7 @@ __global__ void __launch_bounds__(kPselThreads, 1) select_prefill_kernel(TopkPre
     const int t = a.t0 + ql;
     const int k = a.k;
     const int nv = visible_entries(a, t);
+    SA_TRACE_MARK(TR_PSELECT, 0);
     int32_t* idx = a.idx + ((size_t)a.b * a.Tq + t) * k;
     if (nv <= k) {
         for (int i = threadIdx.x; i < k; i += blockDim.x) idx[i] = i < nv ? i : -1;
@@ -167,6 +171,7 @@ __global__ void __launch_bounds__(kPselThreads, 1) select_prefill_kernel(TopkPre
     // digit 1
     for (int i = threadIdx.x; i < kBins; i += blockDim.x) hist[i] = 0;
     __syncthreads();
+    SA_TRACE_MARK(TR_PSELECT, 1);
     for (int j = threadIdx.x; j < nround; j += blockDim.x) {
         const bool v = j < nv;
         hist_add(hist, v ? kp[j] >> 21 : 0u, v);
@@ -175,6 +180,7 @@ __global__ void __launch_bounds__(kPselThreads, 1) select_prefill_kernel(TopkPre
     int d1, d2, d3;
     uint32_t above;
     find_digit_desc<kBins>(hist, (uint32_t)k, sh32, &d1, &above, res);
+    SA_TRACE_MARK(TR_PSELECT, 2);
     const uint32_t K1 = (uint32_t)k - above;
     // digit 2
     for (int i = threadIdx.x; i < kBins; i += blockDim.x) hist[i] = 0;
@@ -186,6 +192,7 @@ __global__ void __launch_bounds__(kPselThreads, 1) select_prefill_kernel(TopkPre
     }
     __syncthreads();
     find_digit_desc<kBins>(hist, K1, sh32, &d2, &above, res);
+    SA_TRACE_MARK(TR_PSELECT, 3);
     const uint32_t K2 = K1 - above;
     // digit 3
     const uint32_t pre = ((uint32_t)d1 << 11) | (uint32_t)d2;
@@ -201,6 +208,7 @@ __global__ void __launch_bounds__(kPselThreads, 1) select_prefill_kernel(TopkPre
     const uint32_t r = K2 - above;
     const uint32_t nties = hist[d3 < 0 ? 0 : d3];
     __syncthreads();
+    SA_TRACE_MARK(TR_PSELECT, 4);
     if ((d1 | d2 | d3) < 0 && threadIdx.x == 0) flag(DEV_LEN);  // inconsistent: cannot happen
     const uint32_t T = (pre << 10) | (uint32_t)d3;
 
@@ -221,6 +229,7 @@ __global__ void __launch_bounds__(kPselThreads, 1) select_prefill_kernel(TopkPre
         jmax = res[0];
         __syncthreads();
     }
+    SA_TRACE_MARK(TR_PSELECT, 5);
     // ordered compaction of the selection
     uint32_t running = 0;
     for (int j0 = 0; j0 < nround; j0 += blockDim.x) {
@@ -236,6 +245,7 @@ __global__ void __launch_bounds__(kPselThreads, 1) select_prefill_kernel(TopkPre
         if (running != (uint32_t)k) flag(DEV_LEN);  // cannot happen
         a.cnt[(size_t)a.b * a.Tq + t] = k;
     }
+    SA_TRACE_MARK(TR_PSELECT, 6);
 }
 
 __global__ void fill_positions_kernel(int32_t* pos, int B, int T) {

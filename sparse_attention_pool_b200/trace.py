@@ -1,8 +1,9 @@
 """Device timelines from the profiling build of the library.
 
 ``libsparse_attn_trace.so`` is the library compiled with -DSA_TRACE: its
-decode-path kernels append one record per CTA and phase (global nanosecond
-timer, kernel, phase, SM, CTA) to a device buffer.  Set SA_TRACE_LIB=1
+decode-path kernels and the prefill indexer's score and selection kernels
+append one record per CTA and phase (global nanosecond timer, kernel, phase,
+SM, CTA) to a device buffer.  Set SA_TRACE_LIB=1
 before the first library call of the process to load it; the default
 library has no marks (its kernels are unchanged) and refuses these calls.
 
@@ -12,6 +13,9 @@ library has no marks (its kernels are unchanged) and refuses these calls.
     buf = trace.install(1 << 16)
     S.hybrid_attn_decode(...)
     print(trace.format_summary(trace.records(buf)))
+
+For a prefill, ``cta_phase_durations(records, "prefill_select")`` gives the
+time a selection CTA spends in each phase (median, 90th percentile, max).
 """
 from __future__ import annotations
 
@@ -22,7 +26,8 @@ import torch
 
 from ._lib import check, lib
 
-KERNELS = {1: "score", 2: "filter", 3: "resolve", 4: "emit", 5: "attn_split", 6: "attn_merge", 7: "score_fp4"}
+KERNELS = {1: "score", 2: "filter", 3: "resolve", 4: "emit", 5: "attn_split", 6: "attn_merge", 7: "score_fp4",
+           8: "prefill_score", 9: "prefill_select", 10: "prefill_score_fp4"}
 PHASES = {
     "score": ["start", "scan done", "threshold found"],
     "score_fp4": ["start", "scan done", "threshold found"],
@@ -31,6 +36,11 @@ PHASES = {
     "emit": ["start", "end"],
     "attn_split": ["start", "end"],
     "attn_merge": ["start"],
+    # prefill indexer: only the score CTAs whose tile some query sees mark
+    "prefill_score": ["start", "staged", "end"],
+    "prefill_score_fp4": ["start", "staged", "end"],
+    # one CTA per query; a query that sees at most k entries marks only its start
+    "prefill_select": ["start", "keys staged", "digit 1", "digit 2", "digit 3", "ties", "end"],
 }
 RECORD = np.dtype([("t", "<u8"), ("kernel", "<u2"), ("phase", "<u2"), ("sm", "<u2"), ("cta", "<u2")])
 
@@ -77,6 +87,31 @@ def summary(rec: np.ndarray) -> list[dict]:
                          "ctas": int(ts.size), "first_us": float(ts.min()), "median_us": float(np.median(ts)),
                          "last_us": float(ts.max())})
     return sorted(rows, key=lambda r: r["first_us"])
+
+
+def cta_phase_durations(rec: np.ndarray, kernel: str) -> list[dict]:
+    """Per phase transition of one kernel's CTAs (start -> next mark -> ...):
+    how many CTA runs made it and the median / 90th-percentile / maximum time
+    between the two marks, in µs.  A CTA run is the records of one (CTA
+    index, SM) pair from one start mark to the next in time order, so
+    launches of the kernel must not overlap (true of launches without
+    programmatic dependent launch on one stream)."""
+    kid = next(k for k, v in KERNELS.items() if v == kernel)
+    sel = rec[rec["kernel"] == kid]
+    labels = PHASES.get(kernel, [])
+    steps: dict[tuple[int, int], list[float]] = {}
+    for cta, sm in {(int(c), int(m)) for c, m in zip(sel["cta"], sel["sm"])}:
+        run = sel[(sel["cta"] == cta) & (sel["sm"] == sm)]
+        run = run[np.argsort(run["t"], kind="stable")]
+        for i in range(1, run.size):
+            p0, p1 = int(run["phase"][i - 1]), int(run["phase"][i])
+            if p1 == 0:  # the next run of this CTA index on this SM
+                continue
+            steps.setdefault((p0, p1), []).append((int(run["t"][i]) - int(run["t"][i - 1])) / 1e3)
+    name = lambda p: labels[p] if p < len(labels) else str(p)  # noqa: E731
+    return [{"from": name(p0), "to": name(p1), "runs": len(v), "median_us": float(np.median(v)),
+             "p90_us": float(np.percentile(v, 90)), "max_us": float(np.max(v))}
+            for (p0, p1), v in sorted(steps.items())]
 
 
 def format_summary(rec: np.ndarray) -> str:

@@ -1,7 +1,8 @@
 """The profiling build's device timeline: a traced decode step records, for
 every decode-path kernel, its phases in order, with one filter record per
-filter CTA.  Runs in a child process (the library variant is chosen per
-process by SA_TRACE_LIB).
+filter CTA; a traced prefill top-k records every query's selection CTA and
+its phases, and gives the untraced indices.  Runs in child processes (the
+library variant is chosen per process by SA_TRACE_LIB).
 
 The module runs only with SA_LOWP_GPU_TESTS=1 until its first B200 run.
 """
@@ -59,3 +60,49 @@ def test_traced_decode_step_records_every_kernel_phase():
     r = subprocess.run([sys.executable, "-c", CHILD.replace("ROOT", repr(ROOT))], cwd=ROOT, env=env,
                        capture_output=True, text=True, timeout=600)
     assert r.returncode == 0 and "TRACE_OK" in r.stdout, r.stdout[-3000:] + r.stderr[-3000:]
+
+
+CHILD_PREFILL = r"""
+import os, sys
+sys.path.insert(0, ROOT)
+os.environ["SA_TRACE_LIB"] = "1"
+import numpy as np, torch
+import sparse_attention_pool_b200 as S
+from sparse_attention_pool_b200 import _lib, trace
+from tests._util import Inputs, compress_on_gpu
+assert _lib.lib()._name.endswith("libsparse_attn_trace.so")
+B, T, k = 1, 6000, 256
+inp = Inputs(982, B, T, 8, Tq=T)
+g = inp.to_device()
+csa, _ = compress_on_gpu(S, g, B, T)
+pos = torch.arange(T, dtype=torch.int32, device="cuda").view(1, T).contiguous()
+ws = S.alloc_workspace(S.workspace_size(S.SA_OP_INDEX_TOPK, B, T, 8, csa.Ncap, 0, k))
+i0, c0 = S.csa_index_topk(g["qI"], csa, k, ws, q_pos=pos)   # untraced
+i0, c0 = i0.clone(), c0.clone()
+torch.cuda.synchronize()
+buf = trace.install(1 << 17)
+i1, c1 = S.csa_index_topk(g["qI"], csa, k, ws, q_pos=pos)
+rec = trace.records(buf)
+trace.uninstall()
+S.read_device_status()
+assert torch.equal(i0, i1) and torch.equal(c0, c1)
+sel = rec[rec["kernel"] == 9]
+full = T - 4 * (k + 1)   # queries that see more than k entries: t // 4 > k
+assert int((sel["phase"] == 0).sum()) == T, int((sel["phase"] == 0).sum())
+for ph in range(1, 7):
+    assert int((sel["phase"] == ph).sum()) == full, (ph, int((sel["phase"] == ph).sum()))
+sc = rec[rec["kernel"] == 8]
+assert (sc["phase"] == 0).sum() > 0 and (sc["phase"] == 0).sum() == (sc["phase"] == 2).sum()
+rows = trace.cta_phase_durations(rec, "prefill_select")
+assert len(rows) == 6 and all(r["runs"] == full for r in rows), rows
+for r in rows + trace.cta_phase_durations(rec, "prefill_score"):
+    print(r)
+print("TRACE_PREFILL_OK")
+"""
+
+
+def test_traced_prefill_topk_records_every_selection_phase():
+    env = dict(os.environ, PYTHONPATH=ROOT)
+    r = subprocess.run([sys.executable, "-c", CHILD_PREFILL.replace("ROOT", repr(ROOT))], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0 and "TRACE_PREFILL_OK" in r.stdout, r.stdout[-3000:] + r.stderr[-3000:]

@@ -4,6 +4,7 @@ times from the earliest mark, in time order, with the phase names."""
 from __future__ import annotations
 
 import numpy as np
+import pytest
 
 from sparse_attention_pool_b200 import trace
 
@@ -27,3 +28,27 @@ def test_summary_of_synthetic_records():
     text = trace.format_summary(rec)
     assert "resolve" in text and "counts scanned" in text
     assert trace.summary(np.zeros(0, dtype=trace.RECORD)) == []
+
+
+def test_cta_phase_durations_split_runs_at_start_marks():
+    # two launches of the prefill selection: CTA 0 runs twice on SM 4 (phases
+    # 0..6, then 0 only: a query that sees at most k entries), CTA 1 once on SM 7
+    recs = [(100, 9, 0, 4, 0), (300, 9, 1, 4, 0), (800, 9, 2, 4, 0), (900, 9, 3, 4, 0), (1_000, 9, 4, 4, 0),
+            (1_000, 9, 5, 4, 0), (3_000, 9, 6, 4, 0),
+            (150, 9, 0, 7, 1), (250, 9, 1, 7, 1), (1_250, 9, 2, 7, 1), (1_300, 9, 3, 7, 1), (1_400, 9, 4, 7, 1),
+            (1_400, 9, 5, 7, 1), (5_400, 9, 6, 7, 1),
+            (9_000, 9, 0, 4, 0),
+            (50, 8, 0, 4, 3), (90, 8, 2, 4, 3)]  # another kernel: not counted
+    rec = np.array(recs, dtype=trace.RECORD)
+    rows = trace.cta_phase_durations(rec, "prefill_select")
+    by = {(r["from"], r["to"]): r for r in rows}
+    assert [(r["from"], r["to"]) for r in rows] == [
+        ("start", "keys staged"), ("keys staged", "digit 1"), ("digit 1", "digit 2"), ("digit 2", "digit 3"),
+        ("digit 3", "ties"), ("ties", "end")]
+    assert all(r["runs"] == 2 for r in rows)  # the start-only run adds no transition
+    assert by[("start", "keys staged")]["median_us"] == pytest.approx(0.15)
+    assert by[("keys staged", "digit 1")]["max_us"] == 1.0
+    assert by[("ties", "end")]["median_us"] == 3.0 and by[("ties", "end")]["max_us"] == 4.0
+    score = trace.cta_phase_durations(rec, "prefill_score")
+    assert [(r["from"], r["to"], r["runs"]) for r in score] == [("start", "end", 1)]
+    assert trace.cta_phase_durations(np.zeros(0, dtype=trace.RECORD), "prefill_select") == []
