@@ -232,6 +232,26 @@ def time_compress(S, w, lengths, Kd, Vd, KId, lens, csa, hca, kv, reps=5):
     return out
 
 
+def traced_run(path, fn, capacity=1 << 22):
+    """One untimed run of `fn` with the profiling build's per-CTA marks
+    recorded (the library loaded with SA_TRACE_LIB=1); the timeline report is
+    written to `path`."""
+    import torch
+
+    from sparse_attention_pool_b200 import trace
+
+    torch.cuda.synchronize()
+    buf = trace.install(capacity)
+    fn()
+    rec = trace.records(buf)
+    n = trace.count()
+    trace.uninstall()
+    with open(path, "w") as f:
+        f.write(trace.report(rec) + "\n")
+    return {"path": path, "records": int(rec.size), "dropped": max(0, n - int(rec.size)),
+            "library": "profiling build (marks compiled in): this line's timings are not headline figures"}
+
+
 def max_over_ranks(ms, world, device):
     """The job's time is the slowest rank's: every rank calls this at the same point."""
     if world == 1:
@@ -413,6 +433,7 @@ def run_ours(args, w, rank, world, dev):
         clk.keep_busy(lambda: (flush_l2(), graph.replay()), min_samples=2)
     torch.cuda.synchronize()
     S.read_device_status()
+    trace_info = traced_run(args.trace, lambda: (flush_l2(), graph.replay())) if args.trace else None
 
     # end to end through the public API: pinned host q / q_idx in, outputs back out
     q_pin = torch.from_numpy(np.ascontiguousarray(q_h).view(np.int16)).pin_memory()
@@ -508,6 +529,8 @@ def run_ours(args, w, rank, world, dev):
         "clocks": clk.summary(),
         "setup_s": round(time.time() - t_gen, 1),
     }
+    if trace_info:
+        result["trace"] = trace_info
     if step_bytes < 8_000_000:  # a step this small is bound by launch latency, not by HBM
         result["roofline"]["note"] = (f"{step_bytes / 1e6:.2f} MB per step: launch-latency bound; "
                                       "the fraction does not measure the kernel")
@@ -717,6 +740,7 @@ def run_prefill(args, w, rank, world, dev):
         clk.keep_busy(step, min_samples=2)
     torch.cuda.synchronize()
     S.read_device_status()
+    trace_info = traced_run(args.trace, step) if args.trace else None
     total_ms = max_over_ranks(sum(step_ms), world, dev)
     value = job_throughput(B * T * args.steps, world, total_ms)
     # fp64 indexer: one exact 64-term fp64 dot product per visible (query, entry) pair
@@ -730,7 +754,7 @@ def run_prefill(args, w, rank, world, dev):
     hca_rows = sum(t // w.m_hca for t in range(T)) * B
     csa_tf = 4 * csa_rows * H * 128 / (stages["csa_attn"] / 1e3) / 1e12
     hca_tf = 4 * hca_rows * H * 128 / (stages["hca_attn"] / 1e3) / 1e12
-    return {
+    result = {
         "metric": "hybrid-attn causal prefill tokens/s @128K",
         "value": value,
         "unit": "tokens/s",
@@ -756,6 +780,9 @@ def run_prefill(args, w, rank, world, dev):
         "clocks": clk.summary(),
         "setup_s": round(time.time() - t_gen, 1),
     }
+    if trace_info:
+        result["trace"] = trace_info
+    return result
 
 
 # ----------------------------------------------------------- oracle (CPU) ---
@@ -944,6 +971,10 @@ def main():
                     help="decode only: context-parallel mode, one batch sharded by context over the ranks")
     ap.add_argument("--tokens", type=int, default=0,
                     help="prefill only: a shorter sequence than the workload's (small cases for profiling)")
+    ap.add_argument("--trace", default="",
+                    help="profiling: load the profiling build of the library and write the per-CTA timeline of "
+                         "one extra untimed step to this file (one GPU, our arm; the timings of such a run "
+                         "are not headline figures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -959,6 +990,10 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.trace:
+        if args.impl != "ours" or args.cp or world > 1:
+            ap.error("--trace runs our arm on one GPU, without --cp")
+        os.environ["SA_TRACE_LIB"] = "1"  # before the first library call
     if args.impl == "reference":
         res = run_reference(args, w, rank, world)
         if res is not None:

@@ -98,20 +98,46 @@ def cta_phase_durations(rec: np.ndarray, kernel: str) -> list[dict]:
     programmatic dependent launch on one stream)."""
     kid = next(k for k, v in KERNELS.items() if v == kernel)
     sel = rec[rec["kernel"] == kid]
+    if sel.size < 2:
+        return []
+    # by CTA index, then SM, then time, then append order
+    s = sel[np.lexsort((np.arange(sel.size), sel["t"], sel["sm"], sel["cta"]))]
+    same = (s["cta"][1:] == s["cta"][:-1]) & (s["sm"][1:] == s["sm"][:-1]) & (s["phase"][1:] != 0)
+    p0, p1 = s["phase"][:-1][same].astype(np.int64), s["phase"][1:][same].astype(np.int64)
+    dt = (s["t"][1:].astype(np.int64) - s["t"][:-1].astype(np.int64))[same] / 1e3
     labels = PHASES.get(kernel, [])
-    steps: dict[tuple[int, int], list[float]] = {}
-    for cta, sm in {(int(c), int(m)) for c, m in zip(sel["cta"], sel["sm"])}:
-        run = sel[(sel["cta"] == cta) & (sel["sm"] == sm)]
-        run = run[np.argsort(run["t"], kind="stable")]
-        for i in range(1, run.size):
-            p0, p1 = int(run["phase"][i - 1]), int(run["phase"][i])
-            if p1 == 0:  # the next run of this CTA index on this SM
-                continue
-            steps.setdefault((p0, p1), []).append((int(run["t"][i]) - int(run["t"][i - 1])) / 1e3)
     name = lambda p: labels[p] if p < len(labels) else str(p)  # noqa: E731
-    return [{"from": name(p0), "to": name(p1), "runs": len(v), "median_us": float(np.median(v)),
-             "p90_us": float(np.percentile(v, 90)), "max_us": float(np.max(v))}
-            for (p0, p1), v in sorted(steps.items())]
+    rows = []
+    for a, b in sorted({(int(x), int(y)) for x, y in zip(p0, p1)}):
+        v = dt[(p0 == a) & (p1 == b)]
+        rows.append({"from": name(a), "to": name(b), "runs": int(v.size), "median_us": float(np.median(v)),
+                     "p90_us": float(np.percentile(v, 90)), "max_us": float(np.max(v))})
+    return rows
+
+
+def count(stream=None) -> int:
+    """Marks made since the buffer was installed, dropped ones included."""
+    s = torch.cuda.current_stream() if stream is None else stream
+    n = ctypes.c_uint32(0)
+    check("sa_trace_count", lib().sa_trace_count(ctypes.byref(n), ctypes.c_void_p(s.cuda_stream)))
+    return int(n.value)
+
+
+def report(rec: np.ndarray) -> str:
+    """The per-(kernel, phase) summary, then each kernel's per-CTA phase
+    durations."""
+    out = [format_summary(rec)]
+    for kid in sorted({int(x) for x in np.unique(rec["kernel"])}):
+        name = KERNELS.get(kid)
+        rows = cta_phase_durations(rec, name) if name else []
+        if rows:
+            out.append("")
+            out.append(f"{name}: per-CTA phase durations (µs)")
+            out.append(f"  {'from':<16} {'to':<16} {'runs':>8} {'median':>9} {'p90':>9} {'max':>9}")
+            for r in rows:
+                out.append(f"  {r['from']:<16} {r['to']:<16} {r['runs']:>8} {r['median_us']:>9.2f} "
+                           f"{r['p90_us']:>9.2f} {r['max_us']:>9.2f}")
+    return "\n".join(out)
 
 
 def format_summary(rec: np.ndarray) -> str:

@@ -5,14 +5,22 @@ Per sequence: N^C * 128 (indexer keys) + min(k, N^C) * 2 * 128 * b_kv
 (q_I) + 2 * H * 256 (two outputs), with 8 more bytes per gathered entry and
 per 64 HCA entries for fp8 scales.  The totals are checked against the
 figures worked out by hand for the three uniform decode workloads, and the
-fp8 terms against a sum written out term by term.
+fp8 terms against a sum written out term by term.  Also: the argument
+checks of the profiling option.
 """
 from __future__ import annotations
 
+import os
+import subprocess
+import sys
+
 import numpy as np
+import pytest
 
 import bench
 from sparse_attention_pool_b200 import configs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def test_decode_step_bytes_match_the_worked_figures():
@@ -108,3 +116,12 @@ def test_mixed_storage_oracle_leg_is_the_pinned_pieces():
                            {"mode": "fp8", "data": vc, "scales": vs}, r16["idx"][:r16["cnt"]], bench.SCALE)
     assert np.array_equal(r["out_csa"], oc)
     assert np.abs(r["out_csa"] - r16["out_csa"]).max() < 3e-2  # storage rounding only
+
+
+@pytest.mark.parametrize("extra", [["--cp"], ["--impl", "reference"]])
+def test_trace_option_refuses_other_arms(extra):
+    """--trace loads the profiling build for one GPU on our arm; it is refused
+    (argument error, nothing run) with --cp or the reference arm."""
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--trace", os.devnull, *extra],
+                       capture_output=True, text=True, timeout=120, cwd=ROOT)
+    assert r.returncode == 2 and "--trace runs our arm on one GPU" in r.stderr, r.stderr[-500:]

@@ -52,3 +52,21 @@ def test_cta_phase_durations_split_runs_at_start_marks():
     score = trace.cta_phase_durations(rec, "prefill_score")
     assert [(r["from"], r["to"], r["runs"]) for r in score] == [("start", "end", 1)]
     assert trace.cta_phase_durations(np.zeros(0, dtype=trace.RECORD), "prefill_select") == []
+
+
+def test_report_at_prefill_scale():
+    # 40,000 selection runs of 7 marks on 148 SMs (a long prefill's worth):
+    # the decoding stays vectorised, and every run shows in every transition
+    rng = np.random.default_rng(5)
+    runs, ph = 40_000, 7
+    cta = np.repeat(np.arange(runs) % 1024, ph).astype(np.uint16)
+    sm = np.repeat(rng.integers(0, 148, runs), ph).astype(np.uint16)
+    start = np.repeat(np.arange(runs, dtype=np.uint64) * 50_000, ph)
+    t = start + np.tile(np.arange(ph, dtype=np.uint64) * 1_000, runs)
+    rec = np.zeros(runs * ph, dtype=trace.RECORD)
+    rec["t"], rec["kernel"], rec["phase"], rec["sm"], rec["cta"] = t, 9, np.tile(np.arange(ph), runs), sm, cta
+    rec = rec[rng.permutation(rec.size)]  # append order is not time order across CTAs
+    rows = trace.cta_phase_durations(rec, "prefill_select")
+    assert len(rows) == 6 and all(r["runs"] == runs and r["median_us"] == 1.0 and r["max_us"] == 1.0 for r in rows)
+    text = trace.report(rec)
+    assert "prefill_select: per-CTA phase durations" in text and "digit 3" in text
