@@ -698,6 +698,7 @@ def run_prefill(args, w, rank, world, dev):
     pos = torch.arange(T, dtype=torch.int32, device=dev).repeat(B, 1).contiguous()
     L = _lib.lib()
     stream = torch.cuda.current_stream()
+    S.set_option(S.SA_OPT_PREFILL_SELECT, args.prefill_select)
 
     def step():
         S.hybrid_attn_prefill(q, qI, csa, hca, k, ws, idx, cnt, scale=SCALE, out_csa=out_c, out_hca=out_h)
@@ -769,7 +770,7 @@ def run_prefill(args, w, rank, world, dev):
         "data": "synthetic",
         "config": {"workload": w.name, "B_per_gpu": B, "tokens": T, "heads": H, "head_dim": 128, "topk": k,
                    "l2": "inputs larger than L2 (q alone is %.1f GB)" % (q.numel() * 2 / 1e9),
-                   "launch": "eager (one call per step)"},
+                   "launch": "eager (one call per step)", "prefill_select": args.prefill_select},
         "stages_ms": stages,
         "roofline": {"kernel": "score_prefill_kernel (exact fp64 indexer)", "bound": "alu",
                      "achieved": idx_tflops, "peak": fp64_peak, "unit": "TFLOP/s (fp64)",
@@ -971,6 +972,8 @@ def main():
                     help="decode only: context-parallel mode, one batch sharded by context over the ranks")
     ap.add_argument("--tokens", type=int, default=0,
                     help="prefill only: a shorter sequence than the workload's (small cases for profiling)")
+    ap.add_argument("--prefill-select", type=int, default=1, choices=[1, 2],
+                    help="prefill only: the top-k selection kernel (SA_OPT_PREFILL_SELECT; same indices)")
     ap.add_argument("--trace", default="",
                     help="profiling: load the profiling build of the library and write the per-CTA timeline of "
                          "one extra untimed step to this file (one GPU, our arm; the timings of such a run "
@@ -983,6 +986,8 @@ def main():
         ap.error("--indexer, --kv and --cp apply to decode workloads")
     if args.cp and (args.indexer != "bf16" or args.kv != "workload" or args.impl != "ours"):
         ap.error("--cp runs the workload's own storage and indexer on our arm")
+    if args.prefill_select != 1 and (w.mode != "prefill" or args.impl != "ours"):
+        ap.error("--prefill-select applies to prefill workloads on our arm")
     if args.tokens:
         if w.mode != "prefill":
             ap.error("--tokens applies to prefill workloads")

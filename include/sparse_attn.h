@@ -318,14 +318,15 @@ sa_status sa_selftest_wait_timeout(uint32_t wait_tries, void* stream);
  *     uint16 cta (blockIdx.x + gridDim.x * blockIdx.y, mod 2^16) }
  * kernel: 1 indexer score, 2 filter, 3 resolve, 4 emit, 5 attention split,
  * 6 split merge, 7 FP4 indexer score, 8 prefill indexer score, 9 prefill
- * selection, 10 FP4 prefill indexer score.  Phases: score 0 start, 1 scan
+ * selection, 10 FP4 prefill indexer score, 11 prefill selection (second
+ * form, SA_OPT_PREFILL_SELECT = 2).  Phases: score 0 start, 1 scan
  * done, 2 threshold found (last CTA); filter 0 start, 1 rows done; resolve 0
  * start, 1 counts scanned, 2 candidates gathered, 3 t~ known, 4 band done,
  * 5 cut done, 6 positions written; emit, attention 0 start, 1 end; merge 0;
  * prefill scores (CTAs whose tile some query sees) 0 start, 1 operands
  * staged, 2 end; prefill selection (one CTA per query) 0 start, then, when
  * the query sees more than k entries, 1 keys staged, 2..4 digits 1..3
- * found, 5 ties resolved, 6 end.
+ * found, 5 ties resolved (second form: per-warp counts done), 6 end.
  * sa_trace_install(buf, capacity) waits for `stream`, then makes buf (device
  * memory, 16-byte aligned, capacity records) the destination and resets the
  * count; capacity 0 switches tracing off.  sa_trace_count waits for `stream`
@@ -443,6 +444,26 @@ sa_status attn_lse_merge_n(const void* outs, const float* lses, int32_t W, int64
 /* Number of kernels this library has launched from the calling host thread
  * since the process started (a diagnostic counter; memsets are not kernels). */
 uint64_t sa_launch_count(void);
+
+/* Library options: process-wide, read when a call enqueues its kernels (so a
+ * CUDA graph keeps the choice it was captured with).  Host-only: no device
+ * work, callable without a GPU.
+ *   SA_OPT_PREFILL_SELECT  the selection kernel of the causal prefill top-k
+ *     (csa_index_topk / csa_index_topk_mxfp4 with Tq > 1, and the hybrid
+ *     prefill calls).  Both give the same indices, the exact top-k of
+ *     section 3-2 (4) of the review with the lowest-index tie-break:
+ *       1 (default)  one 1024-thread CTA per query: three radix-digit
+ *                    passes over the query's keys, a tie pass and an
+ *                    ordered block-scan compaction;
+ *       2            the first digit over the keys, the second and third
+ *                    over the threshold bin's keys only (a short list in
+ *                    shared memory), then warp-chunked counting and ordered
+ *                    output with the ties taken in the same pass.
+ * sa_set_option returns SA_ERR_INVALID_ARG for an unknown option or value;
+ * sa_get_option writes the current value to *value.                        */
+typedef enum { SA_OPT_PREFILL_SELECT = 1 } sa_option;
+sa_status sa_set_option(int32_t option, int64_t value);
+sa_status sa_get_option(int32_t option, int64_t* value);
 
 #ifdef __cplusplus
 }

@@ -11,8 +11,8 @@ from .api import (Cache, CapturedDecode, alloc_cache, alloc_workspace, attn_lse_
                   attn_lse_merge_n_packed,
                   csa_sparse_attn,
                   hca_compress, hca_dense_attn, hybrid_attn_decode, hybrid_attn_prefill, read_device_status,
-                  selftest_wait_timeout,
+                  selftest_wait_timeout, set_option, get_option,
                   workspace_size)
 from ._lib import (SA_OP_DENSE_ATTN, SA_OP_HYBRID_DECODE, SA_OP_HYBRID_PREFILL, SA_OP_INDEX_TOPK,  # noqa: F401
                    SA_OP_SPARSE_ATTN, SA_OP_WINDOW_ATTN, SA_OP_CP_CANDIDATES,
-                   SA_OP_HYBRID_DECODE_SWA, SparseAttnError)
+                   SA_OP_HYBRID_DECODE_SWA, SA_OPT_PREFILL_SELECT, SparseAttnError)

@@ -27,9 +27,11 @@ EXPORTS = ["csa_compress", "hca_compress", "csa_index_topk", "csa_sparse_attn", 
            "csa_index_topk_noalloc", "csa_append", "hca_append", "swa_attn", "attn_lse_merge",
            "csa_index_quantize_mxfp4", "csa_index_topk_mxfp4", "hybrid_attn_decode_mxfp4",
            "cp_decode_candidates", "cp_decode_merge_select", "attn_lse_merge_n", "hybrid_attn_decode_swa",
-           "sa_selftest_wait_timeout", "sa_trace_install", "sa_trace_count", "hybrid_attn_prefill_mxfp4"]
+           "sa_selftest_wait_timeout", "sa_trace_install", "sa_trace_count", "hybrid_attn_prefill_mxfp4",
+           "sa_set_option", "sa_get_option"]
 SA_NOALLOC_SCRATCH_BYTES = 32 << 20
 SA_STAGE_INDEX_SCORE, SA_STAGE_TOPK_SELECT, SA_STAGE_CSA_ATTN, SA_STAGE_HCA_ATTN = 0, 1, 2, 3
+SA_OPT_PREFILL_SELECT = 1
 
 P = ctypes.c_void_p
 I32 = ctypes.c_int32
@@ -98,6 +100,8 @@ def lib():
         L.sa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, P]
         L.sa_trace_install.argtypes = [P, ctypes.c_uint32, P]
         L.sa_trace_count.argtypes = [ctypes.POINTER(ctypes.c_uint32), P]
+        L.sa_set_option.argtypes = [I32, ctypes.c_int64]
+        L.sa_get_option.argtypes = [I32, ctypes.POINTER(ctypes.c_int64)]
         L.sa_launch_count.argtypes = []
         L.sa_launch_count.restype = ctypes.c_uint64
         for name in EXPORTS:

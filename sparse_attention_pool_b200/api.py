@@ -433,6 +433,19 @@ def hybrid_attn_prefill(q, q_idx, csa: Cache, hca: Cache, k: int, ws, idx_out, c
     return out_csa, out_hca
 
 
+def set_option(option: int, value: int):
+    """A process-wide library option (host-only; applies to calls made
+    afterwards).  SA_OPT_PREFILL_SELECT: 1 or 2, the prefill top-k's
+    selection kernel (the same indices either way)."""
+    check("sa_set_option", lib().sa_set_option(int(option), int(value)))
+
+
+def get_option(option: int) -> int:
+    v = ctypes.c_int64(0)
+    check("sa_get_option", lib().sa_get_option(int(option), ctypes.byref(v)))
+    return int(v.value)
+
+
 def read_device_status(stream=None):
     """Synchronises the stream and raises if a kernel recorded a device-side anomaly."""
     check("sa_read_device_status", lib().sa_read_device_status(_stream(stream)))

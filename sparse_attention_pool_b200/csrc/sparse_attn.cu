@@ -30,6 +30,7 @@ namespace {
 thread_local char g_err[512] = "";
 thread_local uint64_t g_launches = 0;
 thread_local cudaEvent_t g_stage_ev[SA_NUM_STAGES][2] = {};
+std::atomic<int> g_prefill_select{1};  // SA_OPT_PREFILL_SELECT
 
 // Inside a stream capture the record must become a graph node of its own
 // (an "external" record), so that replays re-record the event.
@@ -665,9 +666,12 @@ sa_status run_topk_prefill(const void* q_idx, int Tq, const int32_t* pos, const 
                                      sa::kPsSmem));
         SA_CUDA(cudaFuncSetAttribute(sa::select_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      sa::kPselSmemKeys * 4));
+        SA_CUDA(cudaFuncSetAttribute(sa::select_prefill_v2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)sa::kPsel2Smem));
         attr_set(init);
     }
     const int etiles = std::max(1, cdiv(c->Ncap, sa::kPsE));
+    const bool select2 = g_prefill_select.load() == 2;
     for (int b = 0; b < c->B; ++b) {
         for (int t0 = 0; t0 < Tq; t0 += kPrefillQB) {
             a.b = b;
@@ -681,7 +685,10 @@ sa_status run_topk_prefill(const void* q_idx, int Tq, const int32_t* pos, const 
                 sa::score_prefill_kernel<<<dim3(etiles, cdiv(a.qb, sa::kPsQ)), sa::kPsThreads, sa::kPsSmem, st>>>(a);
                 SA_LAUNCHED();
             }
-            sa::select_prefill_kernel<<<a.qb, sa::kPselThreads, sa::kPselSmemKeys * 4, st>>>(a);
+            if (select2)
+                sa::select_prefill_v2_kernel<<<a.qb, sa::kPselThreads, sa::kPsel2Smem, st>>>(a);
+            else
+                sa::select_prefill_kernel<<<a.qb, sa::kPselThreads, sa::kPselSmemKeys * 4, st>>>(a);
             SA_LAUNCHED();
         }
     }
@@ -738,6 +745,29 @@ extern "C" {
 int32_t sa_abi_version(void) { return SA_ABI_VERSION; }
 
 uint64_t sa_launch_count(void) { return g_launches; }
+
+sa_status sa_set_option(int32_t option, int64_t value) {
+    switch (option) {
+        case SA_OPT_PREFILL_SELECT:
+            SA_CHECK(value == 1 || value == 2, "sa_set_option: SA_OPT_PREFILL_SELECT=%lld (1 or 2)",
+                     (long long)value);
+            g_prefill_select.store((int)value);
+            return SA_OK;
+        default:
+            return fail(SA_ERR_INVALID_ARG, "sa_set_option: unknown option %d", option);
+    }
+}
+
+sa_status sa_get_option(int32_t option, int64_t* value) {
+    SA_CHECK(value != nullptr, "sa_get_option: value is NULL");
+    switch (option) {
+        case SA_OPT_PREFILL_SELECT:
+            *value = g_prefill_select.load();
+            return SA_OK;
+        default:
+            return fail(SA_ERR_INVALID_ARG, "sa_get_option: unknown option %d", option);
+    }
+}
 
 sa_status sa_set_stage_events(int32_t stage, void* before, void* after) {
     SA_CHECK(stage >= 0 && stage < SA_NUM_STAGES, "sa_set_stage_events: stage=%d", stage);

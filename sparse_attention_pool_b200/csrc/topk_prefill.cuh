@@ -248,6 +248,170 @@ __global__ void __launch_bounds__(kPselThreads, 1) select_prefill_kernel(TopkPre
     SA_TRACE_MARK(TR_PSELECT, 6);
 }
 
+// ---------------------------------------------- selection, second form ----
+// The same exact top-k of one query (ties at the threshold by lowest index,
+// output ascending) in fewer passes and barriers:
+//   pass 1  histogram of digit 1 (bits 31..21) over the query's keys;
+//   pass 2  the keys of digit 1's bin go to a short list in shared memory
+//           (a bin above kPsel2ListCap keys is ranked in place instead), and
+//           digits 2 and 3 are found over that list alone: the threshold
+//           key T and r, the number of keys equal to T that are taken;
+//   pass 3  every warp counts, over its own contiguous run of keys, the keys
+//           above T and those equal to T (ballots, one barrier);
+//   pass 4  every warp writes its selected indices in ascending order at its
+//           exclusive prefix, the ties at T taken in index order while their
+//           running count is below r (ballots, no block scan).
+constexpr int kPsel2SmemKeys = 40 * 1024;  // keys staged in shared memory (160 KB)
+constexpr int kPsel2ListCap = 8192;        // keys of digit 1's bin held in shared memory (32 KB)
+constexpr size_t kPsel2Smem = (size_t)(kPsel2SmemKeys + kPsel2ListCap) * 4;
+
+__global__ void __launch_bounds__(kPselThreads, 1) select_prefill_v2_kernel(TopkPrefillArgs a) {
+    extern __shared__ __align__(16) uint32_t skeys2[];  // [kPsel2SmemKeys] keys, [kPsel2ListCap] bin list
+    __shared__ uint32_t hist[kBins];
+    __shared__ uint32_t sh32[32];
+    __shared__ int res[2];
+    __shared__ uint32_t s_gt[32], s_eq[32];
+    __shared__ uint32_t s_lcnt;
+    static_assert(kPselThreads == 1024, "pass 3 reads one count per warp and lane");
+    const int ql = blockIdx.x;
+    const int t = a.t0 + ql;
+    const int k = a.k;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nv = visible_entries(a, t);
+    SA_TRACE_MARK(TR_PSELECT2, 0);
+    int32_t* idx = a.idx + ((size_t)a.b * a.Tq + t) * k;
+    if (nv <= k) {
+        for (int i = threadIdx.x; i < k; i += blockDim.x) idx[i] = i < nv ? i : -1;
+        if (threadIdx.x == 0) a.cnt[(size_t)a.b * a.Tq + t] = nv;
+        return;
+    }
+    const uint32_t* grow = a.keys + (size_t)ql * a.KS;
+    const uint32_t* kp = grow;
+    uint32_t* list = skeys2 + kPsel2SmemKeys;
+    if (nv <= kPsel2SmemKeys) {
+        const int n4 = (nv + 3) >> 2;  // rows are 16-byte aligned (KS multiple of 128)
+        for (int i = threadIdx.x; i < n4; i += blockDim.x)
+            reinterpret_cast<uint4*>(skeys2)[i] = reinterpret_cast<const uint4*>(grow)[i];
+        kp = skeys2;
+    }
+    const int nround = (nv + blockDim.x - 1) / blockDim.x * blockDim.x;  // whole warps iterate together
+
+    // pass 1: digit 1
+    for (int i = threadIdx.x; i < kBins; i += blockDim.x) hist[i] = 0;
+    if (threadIdx.x == 0) s_lcnt = 0;
+    __syncthreads();
+    SA_TRACE_MARK(TR_PSELECT2, 1);
+    for (int j = threadIdx.x; j < nround; j += blockDim.x) {
+        const bool v = j < nv;
+        hist_add(hist, v ? kp[j] >> 21 : 0u, v);
+    }
+    __syncthreads();
+    int d1, d2, d3;
+    uint32_t above;
+    find_digit_desc<kBins>(hist, (uint32_t)k, sh32, &d1, &above, res);
+    SA_TRACE_MARK(TR_PSELECT2, 2);
+    const uint32_t K1 = (uint32_t)k - above;
+    const uint32_t c1 = d1 < 0 ? 0u : hist[d1];
+    __syncthreads();  // every thread has read c1 before the histogram is cleared
+
+    // pass 2: the keys of bin d1 into the list, then digits 2 and 3 over it
+    const uint32_t* dk = kp;
+    uint32_t dn = (uint32_t)nv;
+    if (c1 <= (uint32_t)kPsel2ListCap) {
+        for (int j0 = 0; j0 < nround; j0 += blockDim.x) {
+            const int j = j0 + threadIdx.x;
+            const uint32_t key = j < nv ? kp[j] : 0u;
+            const bool in = j < nv && (int)(key >> 21) == d1;
+            const uint32_t m = __ballot_sync(0xFFFFFFFFu, in);
+            uint32_t base = 0u;
+            if (lane == 0 && m) base = atom_add_shared(&s_lcnt, (uint32_t)__popc(m));
+            base = __shfl_sync(0xFFFFFFFFu, base, 0);
+            if (in) {
+                const uint32_t p = base + (uint32_t)__popc(m & ((1u << lane) - 1u));
+                if (p < (uint32_t)kPsel2ListCap) list[p] = key;
+            }
+        }
+        __syncthreads();
+        if (threadIdx.x == 0 && s_lcnt != c1) flag(DEV_LEN);  // cannot happen: the bin's own count
+        dk = list;
+        dn = min(s_lcnt, (uint32_t)kPsel2ListCap);
+    }
+    const uint32_t dround = (dn + blockDim.x - 1) / blockDim.x * blockDim.x;
+    for (int i = threadIdx.x; i < kBins; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (uint32_t j = threadIdx.x; j < dround; j += blockDim.x) {
+        const uint32_t key = j < dn ? dk[j] : 0u;
+        const bool v = j < dn && (int)(key >> 21) == d1;
+        hist_add(hist, (key >> 10) & (kBins - 1), v);
+    }
+    __syncthreads();
+    find_digit_desc<kBins>(hist, K1, sh32, &d2, &above, res);
+    SA_TRACE_MARK(TR_PSELECT2, 3);
+    const uint32_t K2 = K1 - above;
+    const uint32_t pre = ((uint32_t)d1 << 11) | (uint32_t)d2;
+    for (int i = threadIdx.x; i < kBinsLow; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (uint32_t j = threadIdx.x; j < dround; j += blockDim.x) {
+        const uint32_t key = j < dn ? dk[j] : 0u;
+        const bool v = j < dn && (key >> 10) == pre;
+        hist_add(hist, key & (kBinsLow - 1), v);
+    }
+    __syncthreads();
+    find_digit_desc<kBinsLow>(hist, K2, sh32, &d3, &above, res);
+    SA_TRACE_MARK(TR_PSELECT2, 4);
+    const uint32_t r = K2 - above;  // keys equal to T that are taken (>= 1)
+    if ((d1 | d2 | d3) < 0 && threadIdx.x == 0) flag(DEV_LEN);  // inconsistent: cannot happen
+    const uint32_t T = (pre << 10) | (uint32_t)d3;
+
+    // pass 3: per warp, over its own run of keys (whole 32-key groups)
+    const uint32_t lt = (1u << lane) - 1u;
+    const int run = ((nv + 31) / 32 + 31) & ~31;
+    const int j_lo = warp * run, j_hi = min(nv, j_lo + run);
+    uint32_t ngt = 0, neq = 0;
+    for (int j0 = j_lo; j0 < j_hi; j0 += 32) {
+        const int j = j0 + lane;
+        const uint32_t key = j < j_hi ? kp[j] : 0u;
+        ngt += (uint32_t)__popc(__ballot_sync(0xFFFFFFFFu, j < j_hi && key > T));
+        neq += (uint32_t)__popc(__ballot_sync(0xFFFFFFFFu, j < j_hi && key == T));
+    }
+    if (lane == 0) {
+        s_gt[warp] = ngt;
+        s_eq[warp] = neq;
+    }
+    __syncthreads();
+    SA_TRACE_MARK(TR_PSELECT2, 5);
+    uint32_t gt_before = lane < warp ? s_gt[lane] : 0u, eq_before = lane < warp ? s_eq[lane] : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        gt_before += __shfl_xor_sync(0xFFFFFFFFu, gt_before, o);
+        eq_before += __shfl_xor_sync(0xFFFFFFFFu, eq_before, o);
+    }
+    // pass 4: this warp's selected entries, ascending, from its prefix on
+    uint32_t pos = gt_before + min(eq_before, r);
+    uint32_t eq_run = eq_before;  // keys equal to T before the current group
+    for (int j0 = j_lo; j0 < j_hi; j0 += 32) {
+        const int j = j0 + lane;
+        const uint32_t key = j < j_hi ? kp[j] : 0u;
+        const bool gt = j < j_hi && key > T;
+        const bool eq = j < j_hi && key == T;
+        const uint32_t em = __ballot_sync(0xFFFFFFFFu, eq);
+        const bool sel = gt || (eq && eq_run + (uint32_t)__popc(em & lt) < r);
+        const uint32_t sm = __ballot_sync(0xFFFFFFFFu, sel);
+        if (sel) {
+            const uint32_t p = pos + (uint32_t)__popc(sm & lt);
+            if (p < (uint32_t)k) idx[p] = j;
+            else flag(DEV_LEN);  // cannot happen: exactly k are selected
+        }
+        pos += (uint32_t)__popc(sm);
+        eq_run += (uint32_t)__popc(em);
+    }
+    if (threadIdx.x == blockDim.x - 1) {  // the last warp ends at the block's total
+        if (pos != (uint32_t)k) flag(DEV_LEN);  // cannot happen
+        a.cnt[(size_t)a.b * a.Tq + t] = k;
+    }
+    SA_TRACE_MARK(TR_PSELECT2, 6);
+}
+
 __global__ void fill_positions_kernel(int32_t* pos, int B, int T) {
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i < (long long)B * T) pos[i] = (int32_t)(i % T);

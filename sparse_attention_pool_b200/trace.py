@@ -27,7 +27,7 @@ import torch
 from ._lib import check, lib
 
 KERNELS = {1: "score", 2: "filter", 3: "resolve", 4: "emit", 5: "attn_split", 6: "attn_merge", 7: "score_fp4",
-           8: "prefill_score", 9: "prefill_select", 10: "prefill_score_fp4"}
+           8: "prefill_score", 9: "prefill_select", 10: "prefill_score_fp4", 11: "prefill_select2"}
 PHASES = {
     "score": ["start", "scan done", "threshold found"],
     "score_fp4": ["start", "scan done", "threshold found"],
@@ -41,6 +41,7 @@ PHASES = {
     "prefill_score_fp4": ["start", "staged", "end"],
     # one CTA per query; a query that sees at most k entries marks only its start
     "prefill_select": ["start", "keys staged", "digit 1", "digit 2", "digit 3", "ties", "end"],
+    "prefill_select2": ["start", "keys staged", "digit 1", "digit 2", "digit 3", "counted", "end"],
 }
 RECORD = np.dtype([("t", "<u8"), ("kernel", "<u2"), ("phase", "<u2"), ("sm", "<u2"), ("cta", "<u2")])
 

@@ -268,6 +268,25 @@ def test_selftest_rejects_bad_arguments(L):
     assert "wait_tries" in L.sa_last_error().decode()
 
 
+def test_options_on_the_host(L):
+    import sparse_attention_pool_b200 as S
+    v = ctypes.c_int64(-1)
+    assert L.sa_get_option(_lib.SA_OPT_PREFILL_SELECT, ctypes.byref(v)) == _lib.SA_OK and v.value == 1  # default
+    try:
+        S.set_option(S.SA_OPT_PREFILL_SELECT, 2)
+        assert S.get_option(S.SA_OPT_PREFILL_SELECT) == 2
+        assert L.sa_set_option(_lib.SA_OPT_PREFILL_SELECT, 3) == _lib.SA_ERR_INVALID_ARG
+        assert "SA_OPT_PREFILL_SELECT" in L.sa_last_error().decode()
+        assert S.get_option(S.SA_OPT_PREFILL_SELECT) == 2  # a refused value changes nothing
+        assert L.sa_set_option(99, 1) == _lib.SA_ERR_INVALID_ARG
+        assert L.sa_get_option(99, ctypes.byref(v)) == _lib.SA_ERR_INVALID_ARG
+        assert L.sa_get_option(_lib.SA_OPT_PREFILL_SELECT, None) == _lib.SA_ERR_INVALID_ARG
+        with pytest.raises(S.SparseAttnError):
+            S.set_option(S.SA_OPT_PREFILL_SELECT, 0)
+    finally:
+        S.set_option(S.SA_OPT_PREFILL_SELECT, 1)
+
+
 def test_trace_calls_need_the_profiling_build(L):
     n = ctypes.c_uint32(7)
     assert L.sa_trace_install(None, 0, None) == _lib.SA_ERR_UNSUPPORTED

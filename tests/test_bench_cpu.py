@@ -125,3 +125,10 @@ def test_trace_option_refuses_other_arms(extra):
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--trace", os.devnull, *extra],
                        capture_output=True, text=True, timeout=120, cwd=ROOT)
     assert r.returncode == 2 and "--trace runs our arm on one GPU" in r.stderr, r.stderr[-500:]
+
+
+@pytest.mark.parametrize("extra", [[], ["--workload", "prefill_b1_t128k_h64_k2048", "--impl", "reference"]])
+def test_prefill_select_option_applies_to_our_prefill_only(extra):
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--prefill-select", "2", *extra],
+                       capture_output=True, text=True, timeout=120, cwd=ROOT)
+    assert r.returncode == 2 and "--prefill-select applies to prefill workloads" in r.stderr, r.stderr[-500:]

@@ -1,0 +1,137 @@
+"""The second form of the prefill selection (SA_OPT_PREFILL_SELECT = 2)
+against the oracle and against the first form: the exact top-k of every
+query row, ties at the threshold by lowest index, ascending output.  Cases:
+every row of a short prefill; equal scores (one crowded bin, larger than
+the in-shared-memory list, and ties at the threshold); rows that see more
+than the 40,960 keys the kernel stages, whose keys are read from the global
+scratch; the FP4 scores; and the hybrid prefill's outputs, identical under
+both forms.
+
+The kernel has not yet run on a B200: the module runs only with
+SA_LOWP_GPU_TESTS=1, so that its first run is a deliberate one.
+"""
+from __future__ import annotations
+
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from tests._util import SCALE, Inputs, compress_on_gpu
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(os.environ.get("SA_LOWP_GPU_TESTS") != "1",
+                                 reason="the second selection form has not yet run on a B200 "
+                                        "(set SA_LOWP_GPU_TESTS=1)")]
+
+STAGED = 40 * 1024  # keys the second form stages in shared memory
+
+
+@pytest.fixture(scope="module")
+def S():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import sparse_attention_pool_b200 as S
+    return S
+
+
+def _topk_both(S, qI, csa, k, pos, fp4=None):
+    """(idx, cnt) under the first and the second selection form."""
+    Tq = qI.shape[1]
+    ws = S.alloc_workspace(S.workspace_size(S.SA_OP_INDEX_TOPK, csa.B, Tq, 8, csa.Ncap, 0, k))
+    out = []
+    for form in (1, 2):
+        S.set_option(S.SA_OPT_PREFILL_SELECT, form)
+        try:
+            if fp4 is None:
+                i, c = S.csa_index_topk(qI, csa, k, ws, q_pos=pos)
+            else:
+                i, c = S.csa_index_topk_mxfp4(qI, csa, fp4[0], fp4[1], k, ws, q_pos=pos)
+            S.read_device_status()
+        finally:
+            S.set_option(S.SA_OPT_PREFILL_SELECT, 1)
+        out.append((i.clone(), c.clone()))
+    return out
+
+
+def _check_rows(inp, csa_keys, pos, got, k):
+    gi, gn = got[0][0].cpu().numpy(), got[0][1].cpu().numpy()
+    for i, t in enumerate(pos):
+        ref, rc = O.topk(O.index_scores(inp.qI[0, i], csa_keys[:t // 4]), k)
+        assert gn[i] == rc and np.array_equal(gi[i], ref), (i, t)
+
+
+def test_every_row_of_a_short_prefill(S):
+    B, T, k = 1, 1500, 64
+    inp = Inputs(1301, B, T, 8, Tq=T)
+    g = inp.to_device()
+    csa, _ = compress_on_gpu(S, g, B, T)
+    pos = list(range(T))
+    (i1, c1), (i2, c2) = _topk_both(S, g["qI"], csa, k, torch.tensor([pos], dtype=torch.int32, device="cuda"))
+    assert torch.equal(i1, i2) and torch.equal(c1, c2)
+    _check_rows(inp, O.compress(inp.KI[0], 4), pos, [(i2, c2)], k)
+
+
+@pytest.mark.parametrize("k", [77, 2048])
+def test_equal_scores_overflow_the_list(S, k):
+    # every indexer key equal: one bin of up to 10,000 keys (above the list's
+    # 8,192), every selection cut inside the ties
+    L = 40000
+    inp = Inputs(1302, 1, L, 8, Tq=12)
+    inp.KI[:] = inp.KI[:, :1, :]
+    g = inp.to_device()
+    csa, _ = compress_on_gpu(S, g, 1, L)
+    pos = [4 * k + 4, 4 * k + 7, 9000, 20000, 32768, 33000, 36000, 36001, 38000, 39000, 39996, L - 1]
+    (i1, c1), (i2, c2) = _topk_both(S, g["qI"], csa, k, torch.tensor([pos], dtype=torch.int32, device="cuda"))
+    assert torch.equal(i1, i2) and torch.equal(c1, c2)
+    want = np.arange(k, dtype=np.int32)
+    assert (i2[0].cpu().numpy() == want[None, :]).all() and (c2 == k).all()
+
+
+def test_rows_past_the_staged_keys(S):
+    L, k = 1 << 18, 2048
+    edge = 4 * STAGED
+    rng = np.random.default_rng(1303)
+    pos = sorted({edge - 4, edge, edge + 3, edge + 4, edge + 7, L - 1,
+                  *(int(x) for x in rng.integers(edge - 3000, L, 30))})
+    inp = Inputs(1303, 1, L, 8, Tq=len(pos))
+    g = inp.to_device()
+    csa, _ = compress_on_gpu(S, g, 1, L)
+    got = _topk_both(S, g["qI"], csa, k, torch.tensor([pos], dtype=torch.int32, device="cuda"))
+    assert torch.equal(got[0][0], got[1][0]) and torch.equal(got[0][1], got[1][1])
+    _check_rows(inp, O.compress(inp.KI[0], 4), pos, [got[1]], k)
+    assert sum(t // 4 > STAGED for t in pos) >= 10 and sum(k < t // 4 <= STAGED for t in pos) >= 2
+
+
+def test_fp4_scores_under_both_forms(S):
+    B, T, k = 1, 3000, 128
+    inp = Inputs(1304, B, T, 8, Tq=T)
+    g = inp.to_device()
+    csa, _ = compress_on_gpu(S, g, B, T)
+    codes, scales = S.csa_index_quantize_mxfp4(csa)
+    pos = torch.arange(T, dtype=torch.int32, device="cuda").view(1, T).contiguous()
+    (i1, c1), (i2, c2) = _topk_both(S, g["qI"], csa, k, pos, fp4=(codes, scales))
+    assert torch.equal(i1, i2) and torch.equal(c1, c2)
+
+
+def test_hybrid_prefill_identical_under_both_forms(S):
+    B, T, H, k = 1, 2100, 64, 128
+    inp = Inputs(1305, B, T, H, Tq=T)
+    g = inp.to_device()
+    csa, hca = compress_on_gpu(S, g, B, T)
+    ws = S.alloc_workspace(S.workspace_size(S.SA_OP_HYBRID_PREFILL, B, T, H, csa.Ncap, hca.Ncap, k))
+    res = []
+    for form in (1, 2):
+        idx = torch.empty(B, T, k, dtype=torch.int32, device="cuda")
+        cnt = torch.empty(B, T, dtype=torch.int32, device="cuda")
+        S.set_option(S.SA_OPT_PREFILL_SELECT, form)
+        try:
+            oc, oh = S.hybrid_attn_prefill(g["q"], g["qI"], csa, hca, k, ws, idx, cnt, scale=SCALE)
+            S.read_device_status()
+        finally:
+            S.set_option(S.SA_OPT_PREFILL_SELECT, 1)
+        res.append((oc, oh, idx, cnt))
+    for a, b in zip(res[0], res[1]):
+        assert torch.equal(a, b)

@@ -13,6 +13,12 @@ on, checked against the oracle and against plain sorting:
   largest, and ordered compaction by block scans in chunks of the CTA --
   the model's global selection and per-rank shares must equal sorting.
 
+* the second form of the prefill selection (select_prefill_v2_kernel): the
+  first radix digit over all keys, the second and third over the threshold
+  bin's keys only (or over all keys when that bin overflows its list), then
+  per-warp runs counted and written with the ties at the threshold taken in
+  index order -- the model's indices must equal the oracle's top-k.
+
 The models restate the kernels' schemes in Python; the CUDA kernels
 themselves are checked against the oracle by the GPU tests.
 """
@@ -254,3 +260,87 @@ def test_fp4_prefill_word_scheme_matches_the_oracle():
             s = np.float32(t[0] + t[1])
             s = np.float32(0) if s == 0 else s
             assert _f2u(s) == _f2u(ref[e]), (qi, e)
+
+
+# -- prefill selection, second form ---------------------------------------------
+
+def _order_key(s: np.ndarray) -> np.ndarray:
+    """The kernels' 32-bit order key of an fp32 score: -0 as +0, then the
+    sign-magnitude bits mapped so that unsigned order is numeric order."""
+    u = np.ascontiguousarray(s, dtype=np.float32).view(np.uint32).copy()
+    u[u == 0x80000000] = 0
+    neg = (u >> 31) == 1
+    return np.where(neg, ~u, u | np.uint32(0x80000000)).astype(np.uint32)
+
+
+def _find_desc(h, K):
+    """The digit d with above(d) < K <= above(d) + h[d], above(d) = the keys in
+    the bins above d."""
+    above = 0
+    for d in range(len(h) - 1, -1, -1):
+        if above < K <= above + int(h[d]):
+            return d, above
+        above += int(h[d])
+    raise AssertionError("inconsistent histogram")
+
+
+def _model_select2(keys, k, list_cap=8192, nw=32):
+    nv = len(keys)
+    if nv <= k:
+        return list(range(nv)) + [-1] * (k - nv), nv
+    h1 = np.bincount(keys >> 21, minlength=2048)
+    d1, above = _find_desc(h1, k)
+    K1 = k - above
+    dk = keys[(keys >> 21) == d1] if h1[d1] <= list_cap else keys  # the list, or every key in place
+    h2 = np.bincount(((dk >> 10) & 2047)[(dk >> 21) == d1], minlength=2048)
+    d2, above = _find_desc(h2, K1)
+    K2 = K1 - above
+    pre = (d1 << 11) | d2
+    h3 = np.bincount((dk & 1023)[(dk >> 10) == pre], minlength=1024)
+    d3, above = _find_desc(h3, K2)
+    r = K2 - above
+    T = np.uint32((pre << 10) | d3)
+    run = ((nv + 31) // 32 + 31) & ~31
+    runs = [(w * run, min(nv, w * run + run)) for w in range(nw)]
+    ngt = [int((keys[lo:hi] > T).sum()) if hi > lo else 0 for lo, hi in runs]
+    neq = [int((keys[lo:hi] == T).sum()) if hi > lo else 0 for lo, hi in runs]
+    out = [-1] * k
+    pos = 0
+    for w, (lo, hi) in enumerate(runs):
+        pos = sum(ngt[:w]) + min(sum(neq[:w]), r)
+        eq_run = sum(neq[:w])
+        for j0 in range(lo, hi, 32):
+            js = np.arange(j0, min(j0 + 32, hi))
+            g, e = keys[js] > T, keys[js] == T
+            erank = eq_run + np.cumsum(e) - e  # ties before each lane
+            sel = g | (e & (erank < r))
+            p = pos + np.cumsum(sel) - sel
+            for j, sl, pp in zip(js, sel, p):
+                if sl:
+                    assert pp < k
+                    out[int(pp)] = int(j)
+            pos += int(sel.sum())
+            eq_run += int(e.sum())
+    assert pos == k  # the last warp ends at the total
+    return out, k
+
+
+def test_prefill_select_v2_scheme_matches_the_oracle():
+    rng = np.random.default_rng(11)
+    cases = []
+    for _ in range(25):  # continuous scores
+        nv = int(rng.integers(1, 60000))
+        cases.append((rng.normal(0, 8, nv).astype(np.float32), int(rng.integers(1, 5000))))
+    for _ in range(15):  # few distinct values: ties at the threshold, overflowing bins
+        nv = int(rng.integers(1000, 60000))
+        vals = rng.normal(0, 8, int(rng.integers(1, 6))).astype(np.float32)
+        cases.append((vals[rng.integers(0, len(vals), nv)], int(rng.integers(1, nv))))
+    z = np.zeros(20000, np.float32)
+    z[::3] = -0.0
+    cases += [(np.full(30000, 1.5, np.float32), 2048),      # all equal: one bin of 30,000 keys
+              (z, 777),                                     # +0 and -0 tie
+              (np.linspace(-4, 4, 45000).astype(np.float32), 40000)]
+    for i, (s, k) in enumerate(cases):
+        got, gc = _model_select2(_order_key(s), k)
+        want, wc = O.topk(s, k)
+        assert gc == wc and got == list(want), i
