@@ -98,13 +98,15 @@ struct MergeArgs {
 // One CTA per sequence: the W candidate lists, rank-major, into shared
 // memory; the exact cut at rank min(k, C) by (key desc, index asc); then
 // the winners in list order (= ascending global index), globally and for
-// this rank.
+// this rank, written by warps over contiguous runs from their prefixes.
 __global__ void __launch_bounds__(kMergeThreads, 1) cp_merge_select_kernel(MergeArgs a) {
     extern __shared__ __align__(16) uint32_t csm[];  // [kMergeCap] keys, [kMergeCap] global indices
     __shared__ uint32_t hist[kBins];
     __shared__ uint32_t sh64[64];
     __shared__ int res[2];
     __shared__ int s_off[kMergeMaxRanks + 1];
+    __shared__ uint32_t s_win[32], s_mine[32], s_tot[2];
+    static_assert(kMergeThreads == 1024, "one count per warp and lane");
     pdl_wait();
     pdl_release();
     const int b = blockIdx.x;
@@ -139,39 +141,69 @@ __global__ void __launch_bounds__(kMergeThreads, 1) cp_merge_select_kernel(Merge
     int32_t jmax = 0x7FFFFFFF;
     const bool all = C <= (uint32_t)a.k;
     if (!all) select_rank(lk, li, C, R, hist, sh64, res, &T, &jmax);
-    // winners in list order: globally, and this rank's rows
+    // winners in list order, globally and this rank's: every warp takes one
+    // contiguous run of the list (whole 32-entry groups), counts its winners
+    // by ballots, and after one barrier writes them from its exclusive prefix
     const uint32_t lo = (uint32_t)s_off[a.rank], hi = (uint32_t)s_off[a.rank + 1];
     const int32_t base = a.base[b];
-    uint32_t gpos = 0, lpos = 0;
-    for (uint32_t p0 = 0; p0 < C; p0 += kMergeThreads) {  // block-uniform trip count
-        const uint32_t p = p0 + tid;
-        bool win = false;
-        if (p < C) {
-            const uint32_t kk = lk[p];
-            win = all || kk > T || (kk == T && li[p] <= jmax);
-        }
+    const int lane = tid & 31, warp = tid >> 5;
+    const uint32_t lt = (1u << lane) - 1u;
+    const uint32_t run = ((C + 31u) / 32u + 31u) & ~31u;
+    const uint32_t p_lo = (uint32_t)warp * run, p_hi = min(C, p_lo + run);
+    auto wins = [&](uint32_t p) {
+        if (p >= p_hi) return false;
+        const uint32_t kk = lk[p];
+        return all || kk > T || (kk == T && li[p] <= jmax);
+    };
+    uint32_t nwin = 0, nmine = 0;
+    for (uint32_t p0 = p_lo; p0 < p_hi; p0 += 32) {  // warp-uniform trip count
+        const uint32_t p = p0 + lane;
+        const bool win = wins(p);
+        nwin += (uint32_t)__popc(__ballot_sync(0xFFFFFFFFu, win));
+        nmine += (uint32_t)__popc(__ballot_sync(0xFFFFFFFFu, win && p >= lo && p < hi));
+    }
+    if (lane == 0) {
+        s_win[warp] = nwin;
+        s_mine[warp] = nmine;
+    }
+    __syncthreads();
+    uint32_t gpos = lane < warp ? s_win[lane] : 0u, lpos = lane < warp ? s_mine[lane] : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        gpos += __shfl_xor_sync(0xFFFFFFFFu, gpos, o);
+        lpos += __shfl_xor_sync(0xFFFFFFFFu, lpos, o);
+    }
+    for (uint32_t p0 = p_lo; p0 < p_hi; p0 += 32) {
+        const uint32_t p = p0 + lane;
+        const bool win = wins(p);
         const bool mine = win && p >= lo && p < hi;
-        uint32_t gt, lt;
-        const uint32_t ge = block_exclusive_scan(win ? 1u : 0u, sh64, &gt);
-        const uint32_t le = block_exclusive_scan(mine ? 1u : 0u, sh64, &lt);
+        const uint32_t wm = __ballot_sync(0xFFFFFFFFu, win), mm = __ballot_sync(0xFFFFFFFFu, mine);
         // exactly R <= k winners (the cut's contract); a position past k is
         // flagged, never written
         if (win && a.sel_idx) {
-            if (gpos + ge < (uint32_t)a.k) a.sel_idx[(size_t)b * a.k + gpos + ge] = li[p];
+            const uint32_t q = gpos + (uint32_t)__popc(wm & lt);
+            if (q < (uint32_t)a.k) a.sel_idx[(size_t)b * a.k + q] = li[p];
             else flag(DEV_LEN);
         }
         if (mine) {
-            if (lpos + le < (uint32_t)a.k) a.local_idx[(size_t)b * a.k + lpos + le] = li[p] - base;
+            const uint32_t q = lpos + (uint32_t)__popc(mm & lt);
+            if (q < (uint32_t)a.k) a.local_idx[(size_t)b * a.k + q] = li[p] - base;
             else flag(DEV_LEN);
         }
-        gpos += gt;
-        lpos += lt;
+        gpos += (uint32_t)__popc(wm);
+        lpos += (uint32_t)__popc(mm);
     }
-    for (uint32_t i = gpos + tid; a.sel_idx && i < (uint32_t)a.k; i += kMergeThreads) a.sel_idx[(size_t)b * a.k + i] = -1;
-    for (uint32_t i = lpos + tid; i < (uint32_t)a.k; i += kMergeThreads) a.local_idx[(size_t)b * a.k + i] = -1;
+    if (tid == kMergeThreads - 1) {  // the last warp ends at the totals
+        s_tot[0] = gpos;
+        s_tot[1] = lpos;
+    }
+    __syncthreads();
+    const uint32_t gtot = s_tot[0], ltot = s_tot[1];
+    for (uint32_t i = gtot + tid; a.sel_idx && i < (uint32_t)a.k; i += kMergeThreads) a.sel_idx[(size_t)b * a.k + i] = -1;
+    for (uint32_t i = ltot + tid; i < (uint32_t)a.k; i += kMergeThreads) a.local_idx[(size_t)b * a.k + i] = -1;
     if (tid == 0) {
-        if (gpos != R) flag(DEV_LEN);  // cannot happen
-        a.local_cnt[b] = (int32_t)min(lpos, (uint32_t)a.k);
+        if (gtot != R) flag(DEV_LEN);  // cannot happen
+        a.local_cnt[b] = (int32_t)min(ltot, (uint32_t)a.k);
         if (a.sel_cnt) a.sel_cnt[b] = (int32_t)R;
     }
 }

@@ -10,8 +10,9 @@ on, checked against the oracle and against plain sorting:
   equal the oracle's bit for bit;
 * the context-parallel merge (cp_merge_select_kernel): rank-major candidate
   offsets, the cut "key > T or (key == T and index <= jmax)" at the k-th
-  largest, and ordered compaction by block scans in chunks of the CTA --
-  the model's global selection and per-rank shares must equal sorting.
+  largest, and ordered output by warps over contiguous runs of the list,
+  each writing from its exclusive prefix -- the model's global selection and
+  per-rank shares must equal sorting.
 
 * the second form of the prefill selection (select_prefill_v2_kernel): the
   first radix digit over all keys, the second and third over the threshold
@@ -170,7 +171,7 @@ def _select_rank(keys, idx, R):
     return T, (0x7FFFFFFF if rem >= len(ties) else ties[rem - 1])
 
 
-def _model_merge(keys, gidx, gcnt, W, k, rank, base, NT=1024):
+def _model_merge(keys, gidx, gcnt, W, k, rank, base, nw=32):
     off = [0]
     for w in range(W):
         off.append(off[-1] + gcnt[w])
@@ -185,19 +186,27 @@ def _model_merge(keys, gidx, gcnt, W, k, rank, base, NT=1024):
     R = min(C, k)
     every = C <= k
     T, jmax = (0, 0x7FFFFFFF) if every else _select_rank(lk, li, R)
-    sel, loc, gpos, lpos = [-1] * k, [-1] * k, 0, 0
-    for p0 in range(0, C, NT):
-        win = [p0 + t < C and (every or lk[p0 + t] > T or (lk[p0 + t] == T and li[p0 + t] <= jmax))
-               for t in range(NT)]
-        mine = [win[t] and off[rank] <= p0 + t < off[rank + 1] for t in range(NT)]
-        ge, le = np.cumsum([0] + win[:-1]), np.cumsum([0] + mine[:-1])
-        for t in range(NT):
-            if win[t]:
-                sel[gpos + ge[t]] = li[p0 + t]
-            if mine[t]:
-                loc[lpos + le[t]] = li[p0 + t] - base
-        gpos += sum(win)
-        lpos += sum(mine)
+    win = [every or lk[p] > T or (lk[p] == T and li[p] <= jmax) for p in range(C)]
+    mine = [win[p] and off[rank] <= p < off[rank + 1] for p in range(C)]
+    # every warp: one contiguous run of whole 32-entry groups, counted, then
+    # written from its exclusive prefix
+    run = ((C + 31) // 32 + 31) & ~31
+    runs = [(w * run, min(C, w * run + run)) for w in range(nw)]
+    nwin = [sum(win[lo:hi]) for lo, hi in runs]
+    nmine = [sum(mine[lo:hi]) for lo, hi in runs]
+    sel, loc = [-1] * k, [-1] * k
+    gpos = lpos = 0
+    for w, (lo, hi) in enumerate(runs):
+        gpos, lpos = sum(nwin[:w]), sum(nmine[:w])
+        for p0 in range(lo, hi, 32):
+            grp = range(p0, min(p0 + 32, hi))
+            for i, p in enumerate(grp):
+                if win[p]:
+                    sel[gpos + sum(win[p0:p0 + i])] = li[p]
+                if mine[p]:
+                    loc[lpos + sum(mine[p0:p0 + i])] = li[p] - base
+            gpos += sum(win[p0:p0 + len(grp)])
+            lpos += sum(mine[p0:p0 + len(grp)])
     return sel, R, loc, lpos
 
 
