@@ -5,14 +5,10 @@ the single-GPU decode step and give its outputs; cp_decode_step itself runs
 in a one-rank NCCL group.  Kernels that wait on other ranks do not exist in
 this path (the exchange is between launches), so the emulation runs the same
 kernels a multi-GPU step runs.
-
-These kernels have not yet run on a B200: the module runs only with
-SA_LOWP_GPU_TESTS=1, so that their first run is a deliberate one.
 """
 from __future__ import annotations
 
 import datetime
-import os
 import socket
 
 import numpy as np
@@ -23,9 +19,7 @@ from oracle import oracle as O
 from sparse_attention_pool_b200 import cp
 from tests._util import SCALE, TOL_BF16, Inputs, bits_to_torch_bf16, compress_on_gpu
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(os.environ.get("SA_LOWP_GPU_TESTS") != "1",
-                                 reason="context-parallel kernels not yet run on a B200 (set SA_LOWP_GPU_TESTS=1)")]
+pytestmark = pytest.mark.gpu
 
 
 @pytest.fixture(scope="module")
