@@ -10,11 +10,14 @@
 //
 // Exactness without a screen: with every e2m1 value doubled (an integer in
 // -12..12), a block's dot product is an integer A with |A| <= 32 * 144 < 2^13
-// (dp4a on int8 operands), and A * 2^e is exact in fp32 while it stays in the
-// normal range; one fp32 addition of the two block terms then rounds the
-// exact sum once.  The keys are therefore exact, the selection needs no
-// rescoring band (bound E = 0), and the filter / resolve / emit kernels of
-// the bf16 path run unchanged (the resolve in its EXACT variant).
+// (dp4a on int8 operands), and its term A * 2^e (e >= -256 from the two
+// E8M0 codes) is exact in fp64.  The two terms are added in fp64 (one
+// rounding) and the sum rounded to fp32: rounding twice, first to 53 and
+// then to 24 bits, gives the correctly rounded sum since 53 >= 2 * 24 + 2.
+// (fp32 terms would round on their own once e < -149, when both blocks are
+// tiny.)  The keys are therefore exact, the selection needs no rescoring
+// band (bound E = 0), and the filter / resolve / emit kernels of the bf16
+// path run unchanged (the resolve in its EXACT variant).
 //
 // Storage: codes [B][Ncap][32] bytes (element 2i in the low nibble of byte
 // i), scales [B][Ncap][2] E8M0 bytes (block 0, block 1).  34 bytes per entry
@@ -31,6 +34,26 @@ namespace sa {
 // between consecutive magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6 are .25, .75,
 // 1.25, 1.75, 2.5, 3.5 and 5; at a midpoint the magnitude with an even
 // fraction bit (0, 1, 1, 2, 2, 4, 4) wins.
+// 2^e as an fp64 bit pattern (exponent field e + 1023), for -1022 <= e <= 1023.
+__device__ __forceinline__ double pow2_f64(int e) { return __longlong_as_double((long long)(e + 1023) << 52); }
+
+// Order key of the score A0 * 2^e0 + A1 * 2^e1 (both terms exact in fp64):
+// one fp64 addition, one rounding to fp32, -0 as +0 (score_key).
+__device__ __noinline__ uint32_t mx_score_key_f64(int A0, int e0, int A1, int e1) {
+    const double t = __dadd_rn((double)A0 * pow2_f64(e0), (double)A1 * pow2_f64(e1));
+    return score_key(__double2float_rn(t));
+}
+
+// While both exponents lie in [-149, 114] the terms are exact and finite in
+// fp32 too (A < 2^13 on the fp32 grid, |A * 2^e| < 2^127) and one fp32
+// addition rounds their sum once; only blocks that small or that large take
+// the fp64 routine (kept out of line: the common path keeps its registers).
+__device__ __forceinline__ uint32_t mx_score_key(int A0, int e0, int A1, int e1) {
+    if (min(e0, e1) >= -149 && max(e0, e1) <= 114)
+        return score_key(__fadd_rn(ldexpf((float)A0, e0), ldexpf((float)A1, e1)));
+    return mx_score_key_f64(A0, e0, A1, e1);
+}
+
 __device__ __forceinline__ uint32_t e2m1_code(float y) {
     const float a = fabsf(y);
     uint32_t c = (uint32_t)(a > 0.25f) + (uint32_t)(a >= 0.75f) + (uint32_t)(a > 1.25f) + (uint32_t)(a >= 1.75f) +
@@ -212,9 +235,7 @@ __global__ void __launch_bounds__(kF4Threads) score_decode_mxfp4_kernel(TopkDeco
             A1 = dot8_e2m1(hi[u].y, qp[10], qn[10], qp[11], qn[11], A1);
             A1 = dot8_e2m1(hi[u].z, qp[12], qn[12], qp[13], qn[13], A1);
             A1 = dot8_e2m1(hi[u].w, qp[14], qn[14], qp[15], qn[15], A1);
-            const float t0 = ldexpf((float)A0, (int)(sc[u] & 0xFFu) + eq0 - 2);
-            const float t1 = ldexpf((float)A1, (int)(sc[u] >> 8) + eq1 - 2);
-            const uint32_t key = score_key(__fadd_rn(t0, t1));
+            const uint32_t key = mx_score_key(A0, (int)(sc[u] & 0xFFu) + eq0 - 2, A1, (int)(sc[u] >> 8) + eq1 - 2);
             keys[row] = key;
             atomicAdd(&hist[key >> 21], 1u);
         }
@@ -386,9 +407,8 @@ __global__ void __launch_bounds__(kPsThreads, 2) score_prefill_mxfp4_kernel(Topk
         for (int v = 0; v < 8; ++v) {
             const int e = (v < 4 ? te * 4 + v : 64 + te * 4 + v - 4);
             // block b scores A_b * 2^(cq_b - 127) * 2^(ck_b - 127) / 4
-            const float t0 = ldexpf((float)acc[0][u][v], sQe[tq * 4 + u][0] + (int)sKe[e][0] - 256);
-            const float t1 = ldexpf((float)acc[1][u][v], sQe[tq * 4 + u][1] + (int)sKe[e][1] - 256);
-            kk[v] = score_key(__fadd_rn(t0, t1));
+            kk[v] = mx_score_key(acc[0][u][v], sQe[tq * 4 + u][0] + (int)sKe[e][0] - 256, acc[1][u][v],
+                                 sQe[tq * 4 + u][1] + (int)sKe[e][1] - 256);
         }
         uint32_t* row = a.keys + (size_t)ql * a.KS + e0;
         *reinterpret_cast<uint4*>(row + te * 4) = make_uint4(kk[0], kk[1], kk[2], kk[3]);

@@ -6,8 +6,10 @@ on, checked against the oracle and against plain sorting:
   e2m1 encoder by threshold compares, the E8M0 exponent from the fp32 bit
   pattern, the doubled-magnitude byte table picked by a byte permute, the
   sign applied by selecting +q or -q bytes, dp4a accumulation and the
-  per-block exponent offsets -- the model's codes, scales and scores must
-  equal the oracle's bit for bit;
+  per-block exponent offsets, each block term exact in fp64 and one
+  rounding of their sum to fp32 -- the model's codes, scales and scores must
+  equal the oracle's bit for bit, also for blocks so small that fp32 terms
+  would round on their own;
 * the context-parallel merge (cp_merge_select_kernel): rank-major candidate
   offsets, the cut "key > T or (key == T and index <= jmax)" at the k-th
   largest, and ordered output by warps over contiguous runs of the list,
@@ -115,7 +117,8 @@ def _model_query(qbits):
     return qp, qn, qe
 
 
-def _model_score(codes: bytes, sc, qp, qn, qe):
+def _block_dots(codes: bytes, qp, qn):
+    """The two exact integer block sums (doubled e2m1 values) of one entry."""
     w = struct.unpack("<8I", codes)
 
     def dot8(x, a, b, c, d, acc):
@@ -129,8 +132,31 @@ def _model_score(codes: bytes, sc, qp, qn, qe):
         for i in range(4):
             m = 8 * blk + 2 * i
             A[blk] = dot8(w[4 * blk + i], qp[m], qn[m], qp[m + 1], qn[m + 1], A[blk])
-    t = [np.float32(math.ldexp(A[blk], int(sc[blk]) + int(qe[blk]) - 254 - 2)) for blk in range(2)]
-    s = np.float32(t[0] + t[1])
+    return A
+
+
+def _model_score(codes: bytes, sc, qp, qn, qe):
+    A = _block_dots(codes, qp, qn)
+    return _mx_sum(A[0], int(sc[0]) + int(qe[0]) - 254 - 2, A[1], int(sc[1]) + int(qe[1]) - 254 - 2)
+
+
+def _mx_sum(A0, e0, A1, e1):
+    """The kernels' score of two exact block terms, -0 as +0: with both
+    exponents in [-149, 114] the terms in fp32 and one fp32 addition;
+    otherwise each term in fp64, one fp64 addition, one rounding to fp32."""
+    with np.errstate(over="ignore"):
+        if min(e0, e1) >= -149 and max(e0, e1) <= 114:
+            s = np.float32(np.float32(math.ldexp(A0, e0)) + np.float32(math.ldexp(A1, e1)))
+        else:
+            s = np.float32(math.ldexp(A0, e0) + math.ldexp(A1, e1))
+    return np.float32(0) if s == 0 else s
+
+
+def _mx_sum_fp32_terms(A0, e0, A1, e1):
+    """A plausible mistake: each term rounded to fp32 first, whatever e (inexact
+    once e < -149)."""
+    with np.errstate(over="ignore"):
+        s = np.float32(np.float32(math.ldexp(A0, e0)) + np.float32(math.ldexp(A1, e1)))
     return np.float32(0) if s == 0 else s
 
 
@@ -265,9 +291,7 @@ def test_fp4_prefill_word_scheme_matches_the_oracle():
             A = [0, 0]
             for w in range(16):
                 A[w // 8] = _dp4a(qw[w], kw[w], A[w // 8])
-            t = [np.float32(math.ldexp(A[b], int(qs[qi][b]) + int(ks[e][b]) - 256)) for b in range(2)]
-            s = np.float32(t[0] + t[1])
-            s = np.float32(0) if s == 0 else s
+            s = _mx_sum(A[0], int(qs[qi][0]) + int(ks[e][0]) - 256, A[1], int(qs[qi][1]) + int(ks[e][1]) - 256)
             assert _f2u(s) == _f2u(ref[e]), (qi, e)
 
 
@@ -353,3 +377,55 @@ def test_prefill_select_v2_scheme_matches_the_oracle():
         got, gc = _model_select2(_order_key(s), k)
         want, wc = O.topk(s, k)
         assert gc == wc and got == list(want), i
+
+
+def test_fp4_scores_of_tiny_blocks_stay_exact():
+    # query and keys both scaled far down: the block terms fall below fp32's
+    # subnormal grid (e < -149) and the sum lands among fp32 subnormals.  The
+    # kernels' fp64 terms give the oracle's single rounding; fp32 terms
+    # (the plausible mistake) round each term first and miss some.
+    rng = np.random.default_rng(7)
+    n = 400
+    x = rng.standard_normal((n, 64)).astype(np.float32) * np.float32(2.0 ** -68)
+    x[:, :32] *= np.float32(2.0 ** -10)  # both blocks' terms below 2^-149 (e about -151 and -155)
+    x[:, 32:] *= np.float32(2.0 ** -14)
+    xb = (x.view(np.uint32) >> 16).astype(np.uint16)
+    kc, ks = O.mxfp4_quantize(xb)
+    q = rng.standard_normal(64).astype(np.float32) * np.float32(2.0 ** -68)
+    qb = (q.view(np.uint32) >> 16).astype(np.uint16)
+    qp, qn, qe = _model_query(qb)
+    qc, qs = O.mxfp4_quantize(qb.reshape(1, -1))
+    ref = O.mxfp4_index_scores(qc[0], qs[0], kc, ks)
+    assert (ref != 0).sum() > n // 2 and (np.abs(ref) < np.finfo(np.float32).tiny).all()  # subnormal scores
+    misses = 0
+    for j in range(n):
+        got = _model_score(bytes(kc[j]), [int(v) for v in ks[j]], qp, qn, qe)
+        assert _f2u(got) == _f2u(ref[j]), j
+        A = _block_dots(bytes(kc[j]), qp, qn)  # the same row through fp32 terms
+        e = [int(ks[j][b]) + int(qe[b]) - 256 for b in range(2)]
+        misses += _f2u(_mx_sum_fp32_terms(A[0], e[0], A[1], e[1])) != _f2u(ref[j])
+    assert misses > n // 10  # the case tells the two schemes apart
+
+
+def test_fp4_scores_of_huge_blocks_match_the_oracle():
+    # large scales: the block terms leave fp32's range (e > 114), the fp64
+    # routine takes over, and scores that overflow fp32 are +-inf as in the
+    # oracle's single rounding
+    rng = np.random.default_rng(8)
+    n = 300
+    x = rng.standard_normal((n, 64)).astype(np.float32) * np.float32(2.0 ** 100)
+    x[: n // 2, 32:] *= np.float32(2.0 ** 14)
+    xb = (x.view(np.uint32) >> 16).astype(np.uint16)
+    kc, ks = O.mxfp4_quantize(xb)
+    q = rng.standard_normal(64).astype(np.float32) * np.float32(2.0 ** 12)
+    qb = (q.view(np.uint32) >> 16).astype(np.uint16)
+    qp, qn, qe = _model_query(qb)
+    qc, qs = O.mxfp4_quantize(qb.reshape(1, -1))
+    ref = O.mxfp4_index_scores(qc[0], qs[0], kc, ks)
+    assert np.isinf(ref).sum() > 0 and np.isfinite(ref).sum() > 0
+    slow = 0
+    for j in range(n):
+        got = _model_score(bytes(kc[j]), [int(v) for v in ks[j]], qp, qn, qe)
+        assert _f2u(got) == _f2u(ref[j]), j
+        slow += max(int(ks[j][b]) + int(qe[b]) - 256 for b in range(2)) > 114
+    assert slow > n // 4  # the fp64 routine's range is exercised
