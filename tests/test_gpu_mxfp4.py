@@ -120,6 +120,47 @@ def test_topk_all_equal_scores_take_the_lowest_indices(S):
     assert (idx[:, 0].cpu().numpy() == np.arange(k)).all()
 
 
+def _scaled_bits(rng, shape, scale0, scale1):
+    """bf16 bits of normals times 2^scale0 (dims 0..31) and 2^scale1 (32..63)."""
+    x = rng.standard_normal(shape).astype(np.float32)
+    x[..., :32] *= np.float32(2.0 ** scale0)
+    x[..., 32:] *= np.float32(2.0 ** scale1)
+    return (x.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def test_topk_of_tiny_and_huge_blocks(S):
+    """Scores whose block terms leave fp32's exact range: subnormal scores
+    (both blocks tiny) and scores that overflow to +-inf (both blocks huge),
+    where the kernels switch to their fp64 routine; decode and every row of a
+    short prefill against the oracle."""
+    rng = np.random.default_rng(76)
+    B, Ncap, k = 2, 5000, 300
+    bits = np.stack([_scaled_bits(rng, (Ncap, 64), -78, -82), _scaled_bits(rng, (Ncap, 64), 100, 114)])
+    qI = np.stack([_scaled_bits(rng, (64,), -68, -68), _scaled_bits(rng, (64,), 12, 12)])
+    c = _cache_with_keys(S, bits, [Ncap, Ncap])
+    codes, scales = S.csa_index_quantize_mxfp4(c)
+    ws = S.alloc_workspace(S.workspace_size(S.SA_OP_INDEX_TOPK, B, 1, 8, Ncap, 0, k))
+    idx, cnt = S.csa_index_topk_mxfp4(bits_to_torch_bf16(qI).cuda(), c, codes, scales, k, ws)
+    S.read_device_status()
+    gi, gn = idx[:, 0].cpu().numpy(), cnt[:, 0].cpu().numpy()
+    for b in range(B):
+        ref, rc = _oracle_topk(qI[b], bits[b], Ncap, k)
+        assert gn[b] == rc and np.array_equal(gi[b], ref), b
+    # prefill: every row of 600 positions over the tiny keys
+    T, kp = 600, 32
+    qP = _scaled_bits(rng, (1, T, 64), -68, -70)
+    c1 = _cache_with_keys(S, bits[:1, : T // 4], [T // 4])
+    codes1, scales1 = S.csa_index_quantize_mxfp4(c1)
+    pos = torch.arange(T, dtype=torch.int32, device="cuda").view(1, T).contiguous()
+    ws1 = S.alloc_workspace(S.workspace_size(S.SA_OP_INDEX_TOPK, 1, T, 8, c1.Ncap, 0, kp))
+    pi, pn = S.csa_index_topk_mxfp4(bits_to_torch_bf16(qP).cuda(), c1, codes1, scales1, kp, ws1, q_pos=pos)
+    S.read_device_status()
+    pi, pn = pi[0].cpu().numpy(), pn[0].cpu().numpy()
+    for t in range(T):
+        ref, rc = _oracle_topk(qP[0, t], bits[0], t // 4, kp)
+        assert pn[t] == rc and np.array_equal(pi[t], ref), t
+
+
 def test_topk_full_size_decode(S):
     """Four sequences of 262,144 entries (1M tokens each), k = 2048: every
     index against the oracle."""
