@@ -90,6 +90,16 @@ def summary(rec: np.ndarray) -> list[dict]:
     return sorted(rows, key=lambda r: r["first_us"])
 
 
+def _runs(sel: np.ndarray):
+    """The records of one kernel sorted by CTA index, SM, time and append
+    order, and a run number per record (a new run at every start mark or
+    change of CTA / SM)."""
+    s = sel[np.lexsort((np.arange(sel.size), sel["t"], sel["sm"], sel["cta"]))]
+    new = np.ones(s.size, dtype=bool)
+    new[1:] = (s["cta"][1:] != s["cta"][:-1]) | (s["sm"][1:] != s["sm"][:-1]) | (s["phase"][1:] == 0)
+    return s, np.cumsum(new) - 1
+
+
 def cta_phase_durations(rec: np.ndarray, kernel: str) -> list[dict]:
     """Per phase transition of one kernel's CTAs (start -> next mark -> ...):
     how many CTA runs made it and the median / 90th-percentile / maximum time
@@ -101,9 +111,8 @@ def cta_phase_durations(rec: np.ndarray, kernel: str) -> list[dict]:
     sel = rec[rec["kernel"] == kid]
     if sel.size < 2:
         return []
-    # by CTA index, then SM, then time, then append order
-    s = sel[np.lexsort((np.arange(sel.size), sel["t"], sel["sm"], sel["cta"]))]
-    same = (s["cta"][1:] == s["cta"][:-1]) & (s["sm"][1:] == s["sm"][:-1]) & (s["phase"][1:] != 0)
+    s, run = _runs(sel)
+    same = run[1:] == run[:-1]
     p0, p1 = s["phase"][:-1][same].astype(np.int64), s["phase"][1:][same].astype(np.int64)
     dt = (s["t"][1:].astype(np.int64) - s["t"][:-1].astype(np.int64))[same] / 1e3
     labels = PHASES.get(kernel, [])
@@ -114,6 +123,25 @@ def cta_phase_durations(rec: np.ndarray, kernel: str) -> list[dict]:
         rows.append({"from": name(a), "to": name(b), "runs": int(v.size), "median_us": float(np.median(v)),
                      "p90_us": float(np.percentile(v, 90)), "max_us": float(np.max(v))})
     return rows
+
+
+def kernel_busy(rec: np.ndarray) -> dict[str, float]:
+    """Per kernel: the time (µs) covered by the union of its CTA runs, each
+    from its first to its last mark -- over several launches, the time the
+    GPU spent in that kernel as far as the marks see it."""
+    out = {}
+    for kid in sorted({int(x) for x in np.unique(rec["kernel"])}):
+        sel = rec[rec["kernel"] == kid]
+        s, run = _runs(sel)
+        starts = np.minimum.reduceat(s["t"].astype(np.int64), np.flatnonzero(np.r_[True, run[1:] != run[:-1]]))
+        ends = np.maximum.reduceat(s["t"].astype(np.int64), np.flatnonzero(np.r_[True, run[1:] != run[:-1]]))
+        order = np.argsort(starts, kind="stable")
+        starts, ends = starts[order], ends[order]
+        reach = np.maximum.accumulate(ends)  # the furthest end among the runs so far
+        prev = np.r_[np.iinfo(np.int64).min, reach[:-1]]
+        covered = np.clip(ends - np.maximum(starts, prev), 0, None)
+        out[KERNELS.get(kid, f"kernel{kid}")] = float(covered.sum()) / 1e3
+    return out
 
 
 def count(stream=None) -> int:
@@ -127,7 +155,8 @@ def count(stream=None) -> int:
 def report(rec: np.ndarray) -> str:
     """The per-(kernel, phase) summary, then each kernel's per-CTA phase
     durations."""
-    out = [format_summary(rec)]
+    out = [format_summary(rec), "", "time covered by each kernel's CTA runs (µs): " +
+           ", ".join(f"{k} {v:.1f}" for k, v in kernel_busy(rec).items())]
     for kid in sorted({int(x) for x in np.unique(rec["kernel"])}):
         name = KERNELS.get(kid)
         rows = cta_phase_durations(rec, name) if name else []

@@ -70,3 +70,16 @@ def test_report_at_prefill_scale():
     assert len(rows) == 6 and all(r["runs"] == runs and r["median_us"] == 1.0 and r["max_us"] == 1.0 for r in rows)
     text = trace.report(rec)
     assert "prefill_select: per-CTA phase durations" in text and "digit 3" in text
+
+
+def test_kernel_busy_is_the_union_of_cta_runs():
+    recs = [  # prefill score CTAs 0 and 1 overlap (100..400 and 300..600), a later launch 1000..1100
+        (100, 8, 0, 1, 0), (400, 8, 2, 1, 0), (300, 8, 0, 2, 1), (600, 8, 2, 2, 1),
+        (1000, 8, 0, 1, 0), (1100, 8, 2, 1, 0),
+        # selection: one run 700..900 and a start-only run (no span)
+        (700, 9, 0, 3, 0), (900, 9, 6, 3, 0), (950, 9, 0, 3, 1)]
+    rec = np.array(recs, dtype=trace.RECORD)
+    busy = trace.kernel_busy(rec[np.random.default_rng(0).permutation(rec.size)])
+    assert busy["prefill_score"] == pytest.approx(0.6)   # (600 - 100) + (1100 - 1000) ns
+    assert busy["prefill_select"] == pytest.approx(0.2)
+    assert "time covered by each kernel's CTA runs" in trace.report(rec)
