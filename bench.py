@@ -972,7 +972,7 @@ def main():
                     help="decode only: context-parallel mode, one batch sharded by context over the ranks")
     ap.add_argument("--tokens", type=int, default=0,
                     help="prefill only: a shorter sequence than the workload's (small cases for profiling)")
-    ap.add_argument("--prefill-select", type=int, default=1, choices=[1, 2],
+    ap.add_argument("--prefill-select", type=int, default=1, choices=[1, 2, 3],
                     help="prefill only: the top-k selection kernel (SA_OPT_PREFILL_SELECT; same indices)")
     ap.add_argument("--trace", default="",
                     help="profiling: load the profiling build of the library and write the per-CTA timeline of "

@@ -458,7 +458,10 @@ uint64_t sa_launch_count(void);
  *       2            the first digit over the keys, the second and third
  *                    over the threshold bin's keys only (a short list in
  *                    shared memory), then warp-chunked counting and ordered
- *                    output with the ties taken in the same pass.
+ *                    output with the ties taken in the same pass;
+ *       3            form 2 in 512-thread CTAs that read the keys from the
+ *                    scratch on every pass instead of staging them, so
+ *                    that three queries share an SM.
  * sa_set_option returns SA_ERR_INVALID_ARG for an unknown option or value;
  * sa_get_option writes the current value to *value.                        */
 typedef enum { SA_OPT_PREFILL_SELECT = 1 } sa_option;

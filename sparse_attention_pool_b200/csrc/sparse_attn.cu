@@ -666,12 +666,12 @@ sa_status run_topk_prefill(const void* q_idx, int Tq, const int32_t* pos, const 
                                      sa::kPsSmem));
         SA_CUDA(cudaFuncSetAttribute(sa::select_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      sa::kPselSmemKeys * 4));
-        SA_CUDA(cudaFuncSetAttribute(sa::select_prefill_v2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)sa::kPsel2Smem));
+        SA_CUDA(cudaFuncSetAttribute(sa::select_prefill_v2_kernel<sa::kPselThreads, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sa::kPsel2Smem));
         attr_set(init);
     }
     const int etiles = std::max(1, cdiv(c->Ncap, sa::kPsE));
-    const bool select2 = g_prefill_select.load() == 2;
+    const int select_form = g_prefill_select.load();
     for (int b = 0; b < c->B; ++b) {
         for (int t0 = 0; t0 < Tq; t0 += kPrefillQB) {
             a.b = b;
@@ -685,8 +685,11 @@ sa_status run_topk_prefill(const void* q_idx, int Tq, const int32_t* pos, const 
                 sa::score_prefill_kernel<<<dim3(etiles, cdiv(a.qb, sa::kPsQ)), sa::kPsThreads, sa::kPsSmem, st>>>(a);
                 SA_LAUNCHED();
             }
-            if (select2)
-                sa::select_prefill_v2_kernel<<<a.qb, sa::kPselThreads, sa::kPsel2Smem, st>>>(a);
+            if (select_form == 2)
+                sa::select_prefill_v2_kernel<sa::kPselThreads, true><<<a.qb, sa::kPselThreads, sa::kPsel2Smem, st>>>(a);
+            else if (select_form == 3)
+                sa::select_prefill_v2_kernel<sa::kPsel3Threads, false>
+                    <<<a.qb, sa::kPsel3Threads, sa::kPsel3Smem, st>>>(a);
             else
                 sa::select_prefill_kernel<<<a.qb, sa::kPselThreads, sa::kPselSmemKeys * 4, st>>>(a);
             SA_LAUNCHED();
@@ -749,7 +752,7 @@ uint64_t sa_launch_count(void) { return g_launches; }
 sa_status sa_set_option(int32_t option, int64_t value) {
     switch (option) {
         case SA_OPT_PREFILL_SELECT:
-            SA_CHECK(value == 1 || value == 2, "sa_set_option: SA_OPT_PREFILL_SELECT=%lld (1 or 2)",
+            SA_CHECK(value >= 1 && value <= 3, "sa_set_option: SA_OPT_PREFILL_SELECT=%lld (1, 2 or 3)",
                      (long long)value);
             g_prefill_select.store((int)value);
             return SA_OK;

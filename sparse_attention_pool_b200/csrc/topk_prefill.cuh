@@ -261,18 +261,26 @@ __global__ void __launch_bounds__(kPselThreads, 1) select_prefill_kernel(TopkPre
 //   pass 4  every warp writes its selected indices in ascending order at its
 //           exclusive prefix, the ties at T taken in index order while their
 //           running count is below r (ballots, no block scan).
+// Two launch forms: NT = 1024 threads staging up to kPsel2SmemKeys keys in
+// shared memory (one CTA per SM), or (STAGE = false) NT = 512 threads that
+// read the keys from the scratch (L2) on every pass, with only the list and
+// the histogram in shared memory, so that three queries share an SM.
 constexpr int kPsel2SmemKeys = 40 * 1024;  // keys staged in shared memory (160 KB)
 constexpr int kPsel2ListCap = 8192;        // keys of digit 1's bin held in shared memory (32 KB)
 constexpr size_t kPsel2Smem = (size_t)(kPsel2SmemKeys + kPsel2ListCap) * 4;
+constexpr size_t kPsel3Smem = (size_t)kPsel2ListCap * 4;
+constexpr int kPsel3Threads = 512;
 
-__global__ void __launch_bounds__(kPselThreads, 1) select_prefill_v2_kernel(TopkPrefillArgs a) {
-    extern __shared__ __align__(16) uint32_t skeys2[];  // [kPsel2SmemKeys] keys, [kPsel2ListCap] bin list
+template <int NT, bool STAGE>
+__global__ void __launch_bounds__(NT, STAGE ? 1 : 3) select_prefill_v2_kernel(TopkPrefillArgs a) {
+    extern __shared__ __align__(16) uint32_t skeys2[];  // [kPsel2SmemKeys] keys (STAGE), [kPsel2ListCap] bin list
     __shared__ uint32_t hist[kBins];
     __shared__ uint32_t sh32[32];
     __shared__ int res[2];
     __shared__ uint32_t s_gt[32], s_eq[32];
     __shared__ uint32_t s_lcnt;
-    static_assert(kPselThreads == 1024, "pass 3 reads one count per warp and lane");
+    static_assert(NT % 32 == 0 && NT <= 1024, "pass 3 reads one count per warp, at most one per lane");
+    constexpr int nw = NT / 32;
     const int ql = blockIdx.x;
     const int t = a.t0 + ql;
     const int k = a.k;
@@ -287,8 +295,8 @@ __global__ void __launch_bounds__(kPselThreads, 1) select_prefill_v2_kernel(Topk
     }
     const uint32_t* grow = a.keys + (size_t)ql * a.KS;
     const uint32_t* kp = grow;
-    uint32_t* list = skeys2 + kPsel2SmemKeys;
-    if (nv <= kPsel2SmemKeys) {
+    uint32_t* list = STAGE ? skeys2 + kPsel2SmemKeys : skeys2;
+    if (STAGE && nv <= kPsel2SmemKeys) {
         const int n4 = (nv + 3) >> 2;  // rows are 16-byte aligned (KS multiple of 128)
         for (int i = threadIdx.x; i < n4; i += blockDim.x)
             reinterpret_cast<uint4*>(skeys2)[i] = reinterpret_cast<const uint4*>(grow)[i];
@@ -365,7 +373,7 @@ __global__ void __launch_bounds__(kPselThreads, 1) select_prefill_v2_kernel(Topk
 
     // pass 3: per warp, over its own run of keys (whole 32-key groups)
     const uint32_t lt = (1u << lane) - 1u;
-    const int run = ((nv + 31) / 32 + 31) & ~31;
+    const int run = ((nv + nw - 1) / nw + 31) & ~31;
     const int j_lo = warp * run, j_hi = min(nv, j_lo + run);
     uint32_t ngt = 0, neq = 0;
     for (int j0 = j_lo; j0 < j_hi; j0 += 32) {

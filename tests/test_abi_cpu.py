@@ -275,7 +275,7 @@ def test_options_on_the_host(L):
     try:
         S.set_option(S.SA_OPT_PREFILL_SELECT, 2)
         assert S.get_option(S.SA_OPT_PREFILL_SELECT) == 2
-        assert L.sa_set_option(_lib.SA_OPT_PREFILL_SELECT, 3) == _lib.SA_ERR_INVALID_ARG
+        assert L.sa_set_option(_lib.SA_OPT_PREFILL_SELECT, 4) == _lib.SA_ERR_INVALID_ARG
         assert "SA_OPT_PREFILL_SELECT" in L.sa_last_error().decode()
         assert S.get_option(S.SA_OPT_PREFILL_SELECT) == 2  # a refused value changes nothing
         assert L.sa_set_option(99, 1) == _lib.SA_ERR_INVALID_ARG

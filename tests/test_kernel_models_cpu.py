@@ -16,7 +16,8 @@ on, checked against the oracle and against plain sorting:
   each writing from its exclusive prefix -- the model's global selection and
   per-rank shares must equal sorting.
 
-* the second form of the prefill selection (select_prefill_v2_kernel): the
+* the second and third forms of the prefill selection
+  (select_prefill_v2_kernel with 32 or 16 warps): the
   first radix digit over all keys, the second and third over the threshold
   bin's keys only (or over all keys when that bin overflows its list), then
   per-warp runs counted and written with the ties at the threshold taken in
@@ -333,7 +334,7 @@ def _model_select2(keys, k, list_cap=8192, nw=32):
     d3, above = _find_desc(h3, K2)
     r = K2 - above
     T = np.uint32((pre << 10) | d3)
-    run = ((nv + 31) // 32 + 31) & ~31
+    run = ((nv + nw - 1) // nw + 31) & ~31  # keys per warp, whole 32-key groups
     runs = [(w * run, min(nv, w * run + run)) for w in range(nw)]
     ngt = [int((keys[lo:hi] > T).sum()) if hi > lo else 0 for lo, hi in runs]
     neq = [int((keys[lo:hi] == T).sum()) if hi > lo else 0 for lo, hi in runs]
@@ -374,9 +375,10 @@ def test_prefill_select_v2_scheme_matches_the_oracle():
               (z, 777),                                     # +0 and -0 tie
               (np.linspace(-4, 4, 45000).astype(np.float32), 40000)]
     for i, (s, k) in enumerate(cases):
-        got, gc = _model_select2(_order_key(s), k)
         want, wc = O.topk(s, k)
-        assert gc == wc and got == list(want), i
+        for nw in (32, 16):  # 1024-thread (second form) and 512-thread (third form) CTAs
+            got, gc = _model_select2(_order_key(s), k, nw=nw)
+            assert gc == wc and got == list(want), (i, nw)
 
 
 def test_fp4_scores_of_tiny_blocks_stay_exact():
