@@ -502,8 +502,11 @@ sa_status run_attn(const void* q, int Tq, int H, const sa_cache* c, bool gather,
         a.part_o = reinterpret_cast<float*>(base);
         a.part_lse = reinterpret_cast<float*>(base + up256((size_t)BQ * sp.splits * H * 128 * 4));
     }
-    // dense causal prefill (HCA) on the tensor-memory kernel; the gathered one
-    // (CSA) stays on the mma.sync kernel, which measured faster (see DESIGN)
+    // dense causal prefill (HCA) on the tensor-memory kernel.  The gathered
+    // (CSA) variant of that kernel is not dispatched: its block-diagonal tiles
+    // (two queries' lists in one 128-row MMA) waste half of every MMA, and on
+    // the 128K-token, 64-head, k = 2048 prefill it took 110-135 ms against
+    // 61 ms for the mma.sync kernel
     if (prefill && !gather && win == 0 && H == 64 && c->dtype == SA_BF16 && pos) return launch_prefill_tc(a, c, false, st);
     const int kv = c->dtype == SA_KV_MIXED ? 2 : c->dtype == SA_FP8_E4M3 ? 1 : 0;
     sa_status r = launch_attn(a, gather, kv, BQ, st, chained && pdl_on(), !prefill);

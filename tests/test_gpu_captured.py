@@ -2,21 +2,16 @@
 Replays with new queries (copied in from pinned host memory) must give the
 eager call's outputs bit for bit, and must see cache appends made between
 steps.
-
-The module runs only with SA_LOWP_GPU_TESTS=1 until its first B200 run.
 """
 from __future__ import annotations
 
-import os
 
 import pytest
 import torch
 
 from tests._util import SCALE, Inputs, compress_on_gpu
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(os.environ.get("SA_LOWP_GPU_TESTS") != "1",
-                                 reason="CapturedDecode not yet run on a B200 (set SA_LOWP_GPU_TESTS=1)")]
+pytestmark = pytest.mark.gpu
 
 
 @pytest.fixture(scope="module")

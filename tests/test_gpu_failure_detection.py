@@ -2,12 +2,9 @@
 complete (a barrier that nothing arrives at) gives up, records a timeout in
 the device status word and returns; the host reads SA_ERR_TIMEOUT, the word
 is cleared, and the context keeps computing correct results.
-
-The module runs only with SA_LOWP_GPU_TESTS=1 until its first B200 run.
 """
 from __future__ import annotations
 
-import os
 
 import numpy as np
 import pytest
@@ -16,9 +13,7 @@ import torch
 from oracle import oracle as O
 from tests._util import SCALE, Inputs, compress_on_gpu
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(os.environ.get("SA_LOWP_GPU_TESTS") != "1",
-                                 reason="the self-test kernel has not yet run on a B200 (set SA_LOWP_GPU_TESTS=1)")]
+pytestmark = pytest.mark.gpu
 
 
 @pytest.fixture(scope="module")

@@ -7,13 +7,9 @@ scratch instead.
 Indices: bit-exact.  Outputs: max-abs <= 1e-2 and rms(err)/rms(oracle) <=
 1e-2 (bf16 cache).  The oracle builds its own caches from the same seeded raw
 tokens.
-
-These sizes have not yet run on a B200: the module runs only with
-SA_LOWP_GPU_TESTS=1, so that their first run is a deliberate one.
 """
 from __future__ import annotations
 
-import os
 
 import numpy as np
 import pytest
@@ -22,9 +18,7 @@ import torch
 from oracle import oracle as O
 from tests._util import SCALE, TOL_BF16, TOL_REL, Inputs, compress_on_gpu, out_errors
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(os.environ.get("SA_LOWP_GPU_TESTS") != "1",
-                                 reason="these sizes not yet run on a B200 (set SA_LOWP_GPU_TESTS=1)")]
+pytestmark = pytest.mark.gpu
 
 K_MAX = 65536
 SELECT_SMEM_KEYS = 49152  # keys the prefill selection stages in shared memory

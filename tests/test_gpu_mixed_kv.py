@@ -5,13 +5,9 @@ FP8).  The cache keeps K's dims 0..63 as e4m3 codes with one fp32 scale per
 Compression and appends must give the oracle's bytes exactly; the attention
 kernels the oracle's output within the fp8 tolerance, in decode and in causal
 prefill.
-
-These kernels have not yet run on a B200: the module runs only with
-SA_LOWP_GPU_TESTS=1, so that their first run is a deliberate one.
 """
 from __future__ import annotations
 
-import os
 
 import numpy as np
 import pytest
@@ -20,9 +16,7 @@ import torch
 from oracle import oracle as O
 from tests._util import SCALE, TOL_FP8, Inputs
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(os.environ.get("SA_LOWP_GPU_TESTS") != "1",
-                                 reason="mixed-storage kernels not yet run on a B200 (set SA_LOWP_GPU_TESTS=1)")]
+pytestmark = pytest.mark.gpu
 
 
 @pytest.fixture(scope="module")

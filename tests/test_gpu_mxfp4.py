@@ -2,13 +2,9 @@
 must give the oracle's codes and scales bit for bit, and csa_index_topk_mxfp4
 the oracle's top-k of its FP4 scores ("DeepSeek-V4 ... Review", section 3-2
 (4), FP4 on the CSA indexer QK path; section 3-2 (2) top-k).
-
-These kernels have not yet run on a B200: the module runs only with
-SA_LOWP_GPU_TESTS=1, so that their first run is a deliberate one.
 """
 from __future__ import annotations
 
-import os
 
 import numpy as np
 import pytest
@@ -18,9 +14,7 @@ from oracle import oracle as O
 from sparse_attention_pool_b200 import synth
 from tests._util import bits_to_torch_bf16
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(os.environ.get("SA_LOWP_GPU_TESTS") != "1",
-                                 reason="MXFP4 kernels not yet run on a B200 (set SA_LOWP_GPU_TESTS=1)")]
+pytestmark = pytest.mark.gpu
 
 
 @pytest.fixture(scope="module")

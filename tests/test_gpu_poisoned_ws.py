@@ -2,21 +2,16 @@
 workspace filled with 0xFF bytes and must give the zeroed workspace's results
 bit for bit (decode with bf16 and e4m3 caches, the FP4 selection, causal
 prefill), also when the poisoned workspace first served a larger call.
-
-The module runs only with SA_LOWP_GPU_TESTS=1 until its first B200 run.
 """
 from __future__ import annotations
 
-import os
 
 import pytest
 import torch
 
 from tests._util import SCALE, Inputs, compress_on_gpu
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(os.environ.get("SA_LOWP_GPU_TESTS") != "1",
-                                 reason="not yet run on a B200 (set SA_LOWP_GPU_TESTS=1)")]
+pytestmark = pytest.mark.gpu
 
 
 @pytest.fixture(scope="module")

@@ -6,16 +6,9 @@ the in-shared-memory list, and ties at the threshold); rows that see more
 than the 40,960 keys the kernel stages, whose keys are read from the global
 scratch; the FP4 scores; and the hybrid prefill's outputs, identical under
 every form.
-
-The module runs only with SA_LOWP_GPU_TESTS=1.  On its first B200 run (the
-first two forms only) every comparison of the two forms held (indices
-identical in all six tests); two oracle comparisons failed in this module's
-own row indexing, since corrected and not yet run again.  The third form has
-not yet run on a B200.
 """
 from __future__ import annotations
 
-import os
 
 import numpy as np
 import pytest
@@ -24,10 +17,7 @@ import torch
 from oracle import oracle as O
 from tests._util import SCALE, Inputs, compress_on_gpu
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(os.environ.get("SA_LOWP_GPU_TESTS") != "1",
-                                 reason="the second selection form has not yet run on a B200 "
-                                        "(set SA_LOWP_GPU_TESTS=1)")]
+pytestmark = pytest.mark.gpu
 
 STAGED = 40 * 1024  # keys the second form stages in shared memory
 

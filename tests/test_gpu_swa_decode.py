@@ -1,12 +1,9 @@
 """hybrid_attn_decode_swa: one decode step whose CSA and HCA outputs each
 include the sliding window over the last raw tokens, against the oracle's
 attention over the union of each branch's entries and the window.
-
-The module runs only with SA_LOWP_GPU_TESTS=1 until its first B200 run.
 """
 from __future__ import annotations
 
-import os
 
 import numpy as np
 import pytest
@@ -15,9 +12,7 @@ import torch
 from oracle import oracle as O
 from tests._util import SCALE, TOL_BF16, Inputs, compress_on_gpu
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(os.environ.get("SA_LOWP_GPU_TESTS") != "1",
-                                 reason="hybrid_attn_decode_swa not yet run on a B200 (set SA_LOWP_GPU_TESTS=1)")]
+pytestmark = pytest.mark.gpu
 
 
 @pytest.fixture(scope="module")

@@ -3,8 +3,6 @@ every decode-path kernel, its phases in order, with one filter record per
 filter CTA; a traced prefill top-k records every query's selection CTA and
 its phases, and gives the untraced indices.  Runs in child processes (the
 library variant is chosen per process by SA_TRACE_LIB).
-
-The module runs only with SA_LOWP_GPU_TESTS=1 until its first B200 run.
 """
 from __future__ import annotations
 
@@ -16,9 +14,7 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(os.environ.get("SA_LOWP_GPU_TESTS") != "1",
-                                 reason="the profiling build has not yet run on a B200 (set SA_LOWP_GPU_TESTS=1)")]
+pytestmark = pytest.mark.gpu
 
 CHILD = r"""
 import os, sys
