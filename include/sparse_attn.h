@@ -462,9 +462,23 @@ uint64_t sa_launch_count(void);
  *       3            form 2 in 512-thread CTAs that read the keys from the
  *                    scratch on every pass instead of staging them, so
  *                    that three queries share an SM.
+ *   SA_OPT_DECODE_FAST  the CSA branch of the hybrid decode calls
+ *     (hybrid_attn_decode, hybrid_attn_decode_swa) for a bf16 cache, at
+ *     most 64 heads and k <= 2048.  Every value gives the same indices (the
+ *     exact top-k) and outputs within the attention tolerance:
+ *       1 (default)  three kernels: a sampled bound on the k-th score, the
+ *                    indexer scan keeping the entries above that bound as
+ *                    candidates, and one 8-CTA cluster per sequence that
+ *                    selects exactly from the candidates (or, when they
+ *                    cannot prove the selection, from every score) and
+ *                    attends over the selection on the tensor cores;
+ *       2            the same kernels, the selection always from every
+ *                    score (the fallback, for testing);
+ *       0            the general kernels (scan, filter, resolve, emit,
+ *                    split attention and merge), as for every other call.
  * sa_set_option returns SA_ERR_INVALID_ARG for an unknown option or value;
  * sa_get_option writes the current value to *value.                        */
-typedef enum { SA_OPT_PREFILL_SELECT = 1 } sa_option;
+typedef enum { SA_OPT_PREFILL_SELECT = 1, SA_OPT_DECODE_FAST = 2 } sa_option;
 sa_status sa_set_option(int32_t option, int64_t value);
 sa_status sa_get_option(int32_t option, int64_t* value);
 

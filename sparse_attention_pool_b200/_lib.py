@@ -32,6 +32,7 @@ EXPORTS = ["csa_compress", "hca_compress", "csa_index_topk", "csa_sparse_attn", 
 SA_NOALLOC_SCRATCH_BYTES = 32 << 20
 SA_STAGE_INDEX_SCORE, SA_STAGE_TOPK_SELECT, SA_STAGE_CSA_ATTN, SA_STAGE_HCA_ATTN = 0, 1, 2, 3
 SA_OPT_PREFILL_SELECT = 1
+SA_OPT_DECODE_FAST = 2
 
 P = ctypes.c_void_p
 I32 = ctypes.c_int32

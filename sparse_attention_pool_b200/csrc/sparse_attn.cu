@@ -20,6 +20,7 @@
 #include "attn_prefill_tc.cuh"
 #include "compress.cuh"
 #include "cp_decode.cuh"
+#include "decode_fast.cuh"
 #include "lowp_index.cuh"
 #include "sa_common.cuh"
 #include "topk_decode.cuh"
@@ -31,6 +32,7 @@ thread_local char g_err[512] = "";
 thread_local uint64_t g_launches = 0;
 thread_local cudaEvent_t g_stage_ev[SA_NUM_STAGES][2] = {};
 std::atomic<int> g_prefill_select{1};  // SA_OPT_PREFILL_SELECT
+std::atomic<int> g_decode_fast{1};      // SA_OPT_DECODE_FAST
 
 // Inside a stream capture the record must become a graph node of its own
 // (an "external" record), so that replays re-record the event.
@@ -204,6 +206,8 @@ sa_status make_ic_map(CUtensorMap* map, const void* kidx, int B, int Ncap) {
 struct TopkDecodeWs {
     size_t hist, hist2, totals, zero_end, keys, emax, chunk_in, chunk_cnt, chunk_pos, cslot, cand_key, cand_idx, cmp_key,
         cmp_idx, amb_key, amb_idx, bitmap, idx, cnt, total;
+    size_t fctrl = 0, fccount = 0, fchist = 0, fcand = 0;  // the fast hybrid path's control words, chunk
+                                                          // counts, candidate histogram, candidates
     int maxchunks, fchunk, nfch, Wcap;
 };
 
@@ -228,8 +232,10 @@ int score_chunk(int B, int Ncap) {
 // (zeroed per call) [per-score-chunk max error][per-filter-chunk sure-ins,
 // candidates, output positions][compact candidate slots][bitmap], then the
 // large ones: [keys][further candidates key/idx][compact list key/idx]
-// [band key/idx][idx][cnt].
-TopkDecodeWs topk_decode_layout(int B, int Ncap, int k, bool own_idx) {
+// [band key/idx][idx][cnt].  `fast` adds the arrays of the fast hybrid
+// decode path: per sequence its control words and per scan chunk its
+// candidate count (small), and a (key, index) candidate row per entry.
+TopkDecodeWs topk_decode_layout(int B, int Ncap, int k, bool own_idx, bool fast = false) {
     TopkDecodeWs w{};
     w.maxchunks = std::max(1, cdiv(Ncap, sa::kScRows));
     w.fchunk = filter_chunk(Ncap);
@@ -244,6 +250,14 @@ TopkDecodeWs topk_decode_layout(int B, int Ncap, int k, bool own_idx) {
     o += (size_t)B * sa::kTotals * 4;
     w.zero_end = o;
     o = up256(o);
+    if (fast) {
+        w.fctrl = o;
+        o += up256((size_t)B * sa::kCtl * 4);
+        w.fccount = o;
+        o += up256((size_t)B * w.maxchunks * 4);
+        w.fchist = o;
+        o += up256((size_t)B * sa::kCH * 4);
+    }
     const size_t col = up256((size_t)B * Ncap * 4);
     const size_t per_fch = up256((size_t)B * w.nfch * 4);
     w.emax = o;
@@ -276,6 +290,10 @@ TopkDecodeWs topk_decode_layout(int B, int Ncap, int k, bool own_idx) {
     if (own_idx) o += up256((size_t)B * k * 4);
     w.cnt = o;
     if (own_idx) o += up256((size_t)B * 4);
+    if (fast) {
+        w.fcand = o;
+        o += up256((size_t)B * Ncap * 8);
+    }
     w.total = o;
     return w;
 }
@@ -309,7 +327,7 @@ size_t attn_partial_bytes(long long BQ, int splits, int H) {
 }
 
 size_t hybrid_decode_bytes(int B, int H, int Ncap_csa, int Ncap_hca, int k) {
-    TopkDecodeWs w = topk_decode_layout(B, Ncap_csa, k, true);
+    TopkDecodeWs w = topk_decode_layout(B, Ncap_csa, k, true, true);
     Split sc = attn_split(k, false, true), sh = attn_split(Ncap_hca, false);
     return w.total + attn_partial_bytes(B, sc.splits, H) + attn_partial_bytes(B, sh.splits, H);
 }
@@ -614,6 +632,102 @@ sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* 
     return SA_OK;
 }
 
+// ---------------------------------------------------- fast hybrid decode --
+// Sample stride of the bound kernel: about 32 expected sample hits above the
+// k-th largest score (k / 32), and at most kFbSamp sample rows.
+int fast_stride(int Ncap, int k) { return std::max(1, std::max(k / 32, cdiv(Ncap, sa::kFbSamp))); }
+
+// The fast path serves a bf16 CSA cache with bf16 indexer keys, up to 64
+// heads and k <= 2048 (eight CTAs of 256 entries); other calls take the
+// general kernels.
+bool fast_decode_ok(const sa_cache* c, int H, int k) {
+    if (g_decode_fast.load() == sa::kFastOff || c->dtype != SA_BF16 || H > 64 || k > sa::kFastMaxK || c->Ncap < 1)
+        return false;
+    const int chunk = score_chunk(c->B, c->Ncap);
+    return cdiv(c->Ncap, chunk) <= sa::kSelMaxChunks;
+}
+
+// The CSA branch of a hybrid decode step on the fast path: the bound
+// kernel, the indexer scan with candidate output, then one cluster kernel
+// per sequence for the exact selection and the attention over it.
+// `between` runs once the scan is queued (the HCA branch forks there).
+template <typename F>
+sa_status run_fast_decode(const void* q, const void* q_idx, int H, const sa_cache* c, int k, float scale, void* out,
+                          float* lse, int32_t* idx, int32_t* cnt, void* ws, const TopkDecodeWs& w, cudaStream_t st,
+                          F&& between) {
+    const int B = c->B, Ncap = c->Ncap;
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    sa::FastArgs a{};
+    a.q = static_cast<const uint16_t*>(q);
+    a.q_idx = static_cast<const uint16_t*>(q_idx);
+    a.kidx = static_cast<const uint16_t*>(c->kidx);
+    a.K = static_cast<const uint16_t*>(c->k);
+    a.V = static_cast<const uint16_t*>(c->v);
+    a.n = c->n;
+    a.ctrl = reinterpret_cast<uint32_t*>(base + w.fctrl);
+    a.ccount = reinterpret_cast<uint32_t*>(base + w.fccount);
+    a.chist = reinterpret_cast<uint32_t*>(base + w.fchist);
+    a.cand = reinterpret_cast<uint2*>(base + w.fcand);
+    a.keys = reinterpret_cast<uint32_t*>(base + w.keys);
+    a.amb_key = reinterpret_cast<uint32_t*>(base + w.amb_key);
+    a.amb_idx = reinterpret_cast<int32_t*>(base + w.amb_idx);
+    a.idx = idx;
+    a.cnt = cnt;
+    a.out = static_cast<uint16_t*>(out);
+    a.lse = lse;
+    a.H = H;
+    a.Ncap = Ncap;
+    a.k = k;
+    a.chunk = score_chunk(B, Ncap);
+    a.nchunks = cdiv(Ncap, a.chunk);
+    a.sstride = fast_stride(Ncap, k);
+    a.mode = g_decode_fast.load();
+    const float sc = scale == 0.f ? 1.0f / sqrtf(128.0f) : scale;
+    a.scale_log2 = sc * 1.4426950408889634f;
+    if (a.nchunks > w.maxchunks || a.nchunks > sa::kSelMaxChunks)
+        return fail(SA_ERR_WORKSPACE, "internal: chunk count above the workspace bound");
+    const size_t smem = sa::kScStages * sa::kScTileBytes + sa::kScStages * 8 + 1024;
+    static std::atomic<uint64_t> init{0};
+    if (!attr_done(init)) {
+        SA_CUDA(cudaFuncSetAttribute(sa::score_fast_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        SA_CUDA(cudaFuncSetAttribute(sa::csa_select_attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     sa::kFaSmem));
+        // the bound kernel's CTAs share SMs with three scan CTAs each: every
+        // kernel of the path asks for the largest shared-memory carveout, so
+        // that no SM is configured too small for the scan while they overlap
+        SA_CUDA(cudaFuncSetAttribute(sa::topk_bound_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     cudaSharedmemCarveoutMaxShared));
+        SA_CUDA(cudaFuncSetAttribute(sa::topk_bound_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+        SA_CUDA(cudaFuncSetAttribute(sa::score_fast_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     cudaSharedmemCarveoutMaxShared));
+        SA_CUDA(cudaFuncSetAttribute(sa::csa_select_attend_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     cudaSharedmemCarveoutMaxShared));
+        attr_set(init);
+    }
+    CUtensorMap map;
+    sa_status r = make_ic_map(&map, c->kidx, B, Ncap);
+    if (r != SA_OK) return r;
+    const bool pdl = pdl_on();
+    stage_mark(SA_STAGE_INDEX_SCORE, 0, st);
+    SA_CUDA(launch_k(sa::topk_bound_kernel, dim3(sa::kFbCluster, B), dim3(sa::kFbThreads), 0, st, false,
+                     (unsigned)sa::kFbCluster, a));
+    SA_LAUNCHED();
+    SA_CUDA(launch_k(sa::score_fast_kernel, dim3(a.nchunks, B), dim3(sa::kScThreads), smem, st, pdl, 1u, map, a));
+    SA_LAUNCHED();
+    stage_mark(SA_STAGE_INDEX_SCORE, 1, st);
+    r = between();
+    if (r != SA_OK) return r;
+    // one kernel selects and attends: the selection stage's events bracket it
+    stage_mark(SA_STAGE_TOPK_SELECT, 0, st);
+    SA_CUDA(launch_k(sa::csa_select_attend_kernel, dim3(sa::kFaCluster, B), dim3(sa::kFaThreads), sa::kFaSmem, st,
+                     pdl, (unsigned)sa::kFaCluster, a));
+    SA_LAUNCHED();
+    stage_mark(SA_STAGE_TOPK_SELECT, 1, st);
+    stage_mark(SA_STAGE_CSA_ATTN, 0, st);
+    stage_mark(SA_STAGE_CSA_ATTN, 1, st);
+    return SA_OK;
+}
+
 sa_status check_ws(void* ws, size_t have, size_t need) {
     if (need == 0) return SA_OK;
     if (!ws) return fail(SA_ERR_WORKSPACE, "workspace is NULL but %zu bytes are needed", need);
@@ -759,6 +873,10 @@ sa_status sa_set_option(int32_t option, int64_t value) {
                      (long long)value);
             g_prefill_select.store((int)value);
             return SA_OK;
+        case SA_OPT_DECODE_FAST:
+            SA_CHECK(value >= 0 && value <= 2, "sa_set_option: SA_OPT_DECODE_FAST=%lld (0, 1 or 2)", (long long)value);
+            g_decode_fast.store((int)value);
+            return SA_OK;
         default:
             return fail(SA_ERR_INVALID_ARG, "sa_set_option: unknown option %d", option);
     }
@@ -769,6 +887,9 @@ sa_status sa_get_option(int32_t option, int64_t* value) {
     switch (option) {
         case SA_OPT_PREFILL_SELECT:
             *value = g_prefill_select.load();
+            return SA_OK;
+        case SA_OPT_DECODE_FAST:
+            *value = g_decode_fast.load();
             return SA_OK;
         default:
             return fail(SA_ERR_INVALID_ARG, "sa_get_option: unknown option %d", option);
@@ -1288,7 +1409,7 @@ static sa_status hybrid_decode_impl(const char* what, const void* q, const void*
     r = check_ws(ws, ws_bytes, need);
     if (r != SA_OK) return r;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    TopkDecodeWs w = topk_decode_layout(csa->B, csa->Ncap, k, true);
+    TopkDecodeWs w = topk_decode_layout(csa->B, csa->Ncap, k, true, true);
     uint8_t* base = static_cast<uint8_t*>(ws);
     int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + w.idx);
     int32_t* cnt = cnt_out ? cnt_out : reinterpret_cast<int32_t*>(base + w.cnt);
@@ -1315,6 +1436,12 @@ static sa_status hybrid_decode_impl(const char* what, const void* q, const void*
         SA_CUDA(cudaEventRecord(side->join, side->s));
         return SA_OK;
     };
+    if (!fp4 && fast_decode_ok(csa, H, k)) {
+        r = run_fast_decode(q, q_idx, H, csa, k, scale, out_csa, lse_csa, idx, cnt, ws, w, st, fork_hca);
+        if (r != SA_OK) return r;
+        SA_CUDA(cudaStreamWaitEvent(st, side->join, 0));
+        return SA_OK;
+    }
     r = run_topk_decode(q_idx, csa, k, idx, cnt, ws, w, st, fork_hca, codes4, scales4);
     if (r != SA_OK) return r;
     stage_mark(SA_STAGE_CSA_ATTN, 0, st);
