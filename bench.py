@@ -336,6 +336,7 @@ def run_ours(args, w, rank, world, dev):
         flush.fill_(1)
         flush_sink.copy_(flush.view(torch.int64).sum())
     L = _lib.lib()
+    S.set_option(S.SA_OPT_DECODE_FAST, args.decode_fast)
 
     def decode(qq, qqI):
         if fp4:
@@ -510,6 +511,7 @@ def run_ours(args, w, rank, world, dev):
         "config": {"workload": w.name, "B_per_gpu": B, "context": int(w.L), "heads": H, "head_dim": 128,
                    "csa_m": w.m_csa, "topk": k, "hca_m": w.m_hca,
                    "kv_dtype": "mixed" if mixed else "e4m3" if w.fp8 else "bf16",
+                   "decode_fast": args.decode_fast,
                    "indexer": args.indexer,
                    "parallelism": f"replicas x{world} (independent sequences)",
                    "l2": "flushed between timed steps: 512 MB written then read back (clean L2)", "launch": "CUDA graph replay"},
@@ -974,6 +976,9 @@ def main():
                     help="decode only: context-parallel mode, one batch sharded by context over the ranks")
     ap.add_argument("--tokens", type=int, default=0,
                     help="prefill only: a shorter sequence than the workload's (small cases for profiling)")
+    ap.add_argument("--decode-fast", type=int, default=0, choices=[0, 1],
+                    help="decode only: the indexer + top-k kernels (SA_OPT_DECODE_FAST: 0 the general ones, "
+                         "1 the sampled-bound fast path; same indices and outputs)")
     ap.add_argument("--prefill-select", type=int, default=1, choices=[1, 2, 3],
                     help="prefill only: the top-k selection kernel (SA_OPT_PREFILL_SELECT; same indices)")
     ap.add_argument("--trace", default="",

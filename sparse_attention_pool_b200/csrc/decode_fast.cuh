@@ -3,53 +3,47 @@
 // "DeepSeek-V4 ... Review", section 3-2 (2) (CSA keeps a sparse top-k of the
 // compressed entries and attends over them) and 3-2 (4) (the indexer QK path).
 //
-// Three kernels, chained by programmatic dependent launch, for a bf16 cache,
-// up to 64 heads and k <= 2048:
+// Three kernels for a bf16 cache, up to 64 heads and k <= 2048, then the
+// split attention of attn.cuh over the selection:
 //
-//   1. topk_bound_kernel  -- one cluster of 16 CTAs per sequence screens a
+//   1. topk_bound_kernel  -- one cluster of 8 CTAs per sequence screens a
 //      strided sample of the indexer rows (at most 4096) and takes a sample
-//      order statistic well below the expected k-th largest score as a
-//      provisional bound t_p.  It only steers how many candidates the scan
-//      keeps; the exactness argument below does not depend on it.
-//   2. score_fast_kernel  -- the indexer stream (the decode_topk scan: TMA
-//      pipeline, fp32 screen s~_j with its certified error bound e_j), which
-//      also writes every row with s~_j >= t_p to its chunk's candidate rows,
-//      in ascending row order (ballots per tile), and the sequence's
-//      E = max e_j.  The bound is awaited only after the first tiles, so the
-//      sample overlaps the stream.  Every key is also written, for the
-//      fallback below.
-//   3. csa_select_attend_kernel -- one cluster of 8 CTAs per sequence.  CTA 0
-//      concatenates the chunks' candidates (ascending entry order), finds the
-//      k-th largest screened key t~, rescores the band |s~ - t~| <= 2E exactly
-//      (the fp64 definition) and cuts it by (s, -j).  This is the exact
-//      selection when at least k candidates were kept and t~ - 2E >= t_p:
-//      every entry outside the list then has s~ < t~ - 2E and is surely not
-//      selected.  Otherwise (or when forced) CTA 0 runs the same selection
-//      over all keys of the sequence in global memory.  The ascending index
-//      list goes to the caller and, through distributed shared memory, to the
-//      cluster: each CTA gathers up to 256 selected K / V rows and computes
-//      its partial softmax attention on the tensor cores (tcgen05, TMEM
-//      accumulators), transposed so that the MMA's 128 rows are entries:
-//          S^T = K_sel Q^T        (M = 128 entries, N = 64 heads, K = 128)
-//          O^T = V_sel^T P^T      (M = 128 dims,    N = 64 heads, K = entries)
-//      The eight partials (o, max, sum per head) merge through distributed
-//      shared memory, each CTA writing eight heads' outputs and lse.
+//      order statistic below the expected k-th largest score as a
+//      provisional bound t_p, and the bin width of a candidate histogram.
+//      The bound only steers how many candidates the scan keeps; the
+//      exactness argument below does not depend on it.
+//   2. score_fast_kernel  -- the indexer stream (TMA pipeline, fp32 screen
+//      s~_j with its certified error bound e_j, as in topk_decode.cuh), which
+//      writes every row with s~_j >= t_p to its chunk's candidate rows, in
+//      ascending row order (ballots per tile), counts it in the sequence's
+//      candidate histogram, and takes E = max e_j.  Every key is also
+//      written, for the fallback below.
+//   3. csa_select_fast_kernel -- one CTA per sequence: the candidate
+//      histogram gives the bin of the k-th largest screened key t~; the
+//      chunks' candidates are concatenated (ascending entry order) and t~ is
+//      ranked inside its bin; the band |s~ - t~| <= 2E is rescored exactly
+//      (the fp64 definition) and cut by (s, -j).  This is the exact selection
+//      when at least k candidates were kept and t~ - 2E >= t_p: every entry
+//      outside the list then has s~ < t~ - 2E and is surely not selected.
+//      Otherwise (or when forced) the same selection runs over every key of
+//      the sequence in global memory.  The ascending index list goes to the
+//      caller's idx / cnt, which the attention reads.
+//
+// The scan waits for the bound kernel before it streams: sharing the SMs
+// with the scan's FMA chains and the memory system with its TMA stream, the
+// sample took longer than the whole prefix of the scan it was to overlap.
 #pragma once
-#include "attn_prefill_tc.cuh"
 #include "topk_decode.cuh"
 
 namespace sa {
 
-constexpr int kFbCluster = 16;   // bound kernel: CTAs per sequence (a non-portable cluster size)
-constexpr int kFbThreads = 128;
-constexpr int kFbRowsPT = 2;     // sample rows per thread, all loads in flight at once
+constexpr int kFbCluster = 8;    // bound kernel: CTAs per sequence
+constexpr int kFbThreads = 512;  // CTA 0's threads also run the order statistic
+constexpr int kFbRowsPT = 1;     // sample rows per thread
 constexpr int kFbSamp = kFbCluster * kFbThreads * kFbRowsPT;  // 4096 sample rows at most
 constexpr int kFastCap = 8192;   // candidates the selecting CTA holds in shared memory
 constexpr int kFastMaxK = 2048;
-constexpr int kFaCluster = 8;    // selection + attention: CTAs per sequence
-constexpr int kFaThreads = 512;  // 16 warps: all select; warps 0-7 run the softmax, 8 heads each merge
-constexpr int kFaEntries = kFastMaxK / kFaCluster;  // 256 selected entries per CTA: two 128-row MMA tiles
-constexpr int kFaEarly = 8;      // scan tiles streamed before the bound is awaited
+constexpr int kFaThreads = 512;  // the selection kernel's CTA (one per sequence)
 constexpr int kFaBand = 1024;    // band members ranked in shared memory
 constexpr int kCtl = 4;          // control words per sequence
 constexpr int kCtlBound = 0, kCtlE = 1, kCtlShift = 2;
@@ -59,11 +53,8 @@ constexpr int kCH = 2048;        // bins of the candidate histogram: key offsets
 constexpr int kFastOff = 0, kFastOn = 1, kFastForceGlobal = 2;
 
 struct FastArgs {
-    const uint16_t* q;      // [B][H][128]
     const uint16_t* q_idx;  // [B][64]
     const uint16_t* kidx;   // [B][Ncap][64]
-    const uint16_t* K;      // [B][Ncap][128] bf16
-    const uint16_t* V;
     const int32_t* n;       // [B]
     uint32_t* ctrl;         // [B][kCtl]: the bound key t_p, E (fp32 bits, max over the scan's CTAs), histogram shift
     uint32_t* chist;        // [B][kCH] histogram of the candidates' keys (zeroed by the bound kernel)
@@ -74,21 +65,30 @@ struct FastArgs {
     int32_t* amb_idx;
     int32_t* idx;           // [B][k] out
     int32_t* cnt;           // [B] out
-    uint16_t* out;          // [B][H][128] out
-    float* lse;             // [B][H] out, or NULL
-    int H, Ncap, k, chunk, nchunks, sstride, mode;
-    float scale_log2;
+    int Ncap, k, chunk, nchunks, sstride, mode;
 };
 
+// The bound kernel's CTAs run beside the scan on SMs of their own (their
+// shared memory leaves no room for a scan CTA) when there are few of them;
+// the scan then awaits the bound only after its last tile.
+constexpr int kFbReserveSmem = 190 * 1024;  // with the static ~33 KB: no 67 KB scan CTA fits beside it
+
 // ------------------------------------------------------------- clusters ----
+// The cluster barrier's ".aligned" forms need every thread of the warp to
+// execute them together: each helper reconverges the warp first.
 __device__ __forceinline__ void cluster_sync() {
+    __syncwarp();
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 // the two halves of a cluster barrier, to overlap its latency with other work
 __device__ __forceinline__ void cluster_arrive_relaxed() {
+    __syncwarp();
     asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() {
+    __syncwarp();
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+}
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -100,21 +100,8 @@ __device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
     return r;
 }
-__device__ __forceinline__ uint32_t ld_dsmem_u32(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr));
-    return v;
-}
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) { return __uint_as_float(ld_dsmem_u32(addr)); }
 __device__ __forceinline__ void st_dsmem_u32(uint32_t addr, uint32_t v) {
     asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t addr) {
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(addr));
-    return v;
 }
 
 // The fp32 screen of one 128-byte indexer row held as eight 16-byte words
@@ -223,9 +210,8 @@ __device__ __forceinline__ float warp_sum(float x) {
 }
 
 // ------------------------------------------------------------ 1. bound ----
-// Grid (kFbCluster, B), clusters of kFbCluster CTAs along x.  Small enough
-// (registers, shared memory) to share an SM with three scan CTAs.
-__global__ void __launch_bounds__(kFbThreads, 5) topk_bound_kernel(FastArgs a) {
+// Grid (kFbCluster, B), clusters of kFbCluster CTAs along x.
+__global__ void __launch_bounds__(kFbThreads, 1) topk_bound_kernel(FastArgs a) {
     __shared__ float sq[64];
     __shared__ uint32_t skey[kFbSamp];  // CTA 0: every sample key of the sequence
     __shared__ uint32_t hist[kDigBins * kFbThreads / 32];
@@ -263,21 +249,20 @@ __global__ void __launch_bounds__(kFbThreads, 5) topk_bound_kernel(FastArgs a) {
     }
     __syncthreads();
     const uint16_t* ic = a.kidx + (size_t)b * a.Ncap * 64;
+    {
+        uint4 w[kFbRowsPT][8];  // every row's loads in flight at once
+        int si[kFbRowsPT];
 #pragma unroll
-    for (int h = 0; h < kFbRowsPT; h += 2) {
-        uint4 w[2][8];
-        int si[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            si[u] = (int)rank * (kFbThreads * kFbRowsPT) + (h + u) * kFbThreads + tid;
+        for (int u = 0; u < kFbRowsPT; ++u) {
+            si[u] = (int)rank * (kFbThreads * kFbRowsPT) + u * kFbThreads + tid;
             const bool ok = si[u] < ns;
             const uint4* rp = reinterpret_cast<const uint4*>(ic + (size_t)(ok ? si[u] * S : 0) * 64);
 #pragma unroll
             for (int c = 0; c < 8; ++c) w[u][c] = ok ? __ldg(rp + c) : make_uint4(0u, 0u, 0u, 0u);
         }
-        if (h == 0) cluster_wait();
+        cluster_wait();
 #pragma unroll
-        for (int u = 0; u < 2; ++u)  // into CTA 0's shared memory (a remote store for the other CTAs)
+        for (int u = 0; u < kFbRowsPT; ++u)  // into CTA 0's shared memory (a remote store for the other CTAs)
             if (si[u] < ns) st_dsmem_u32(dsmem_addr(&skey[si[u]], 0), score_key(screen_row(sq, w[u])));
     }
     SA_TRACE_MARK(TR_BOUND, 1);
@@ -288,11 +273,9 @@ __global__ void __launch_bounds__(kFbThreads, 5) topk_bound_kernel(FastArgs a) {
         const float mu = (float)a.k * (float)ns / (float)n;
         int r = (int)ceilf(mu + 5.f * sqrtf(mu) + 4.f);
         r = max(1, min(r, ns));
-        // the r-th largest of the ns sample keys (three digit passes over the
-        // cluster's shared memory; keys of absent samples are 0 and there are
-        // fewer than ns - r + 1 of them below any real key's rank)
-        // only the samples above mean + 1.5 sd (about 7% of a normal sample)
-        // enter the digit passes, when at least r of them are there
+        // the r-th largest of the ns sample keys; only the samples above
+        // mean + 1.5 sd (about 7% of a normal sample) enter the digit passes,
+        // when at least r of them are there
         const int lane = tid & 31, warp = tid >> 5;
         float s1 = 0.f, s2 = 0.f;
         uint32_t smax = 0u;
@@ -307,11 +290,11 @@ __global__ void __launch_bounds__(kFbThreads, 5) topk_bound_kernel(FastArgs a) {
         s2 = warp_sum(s2);
         smax = __reduce_max_sync(0xFFFFFFFFu, smax);
         __shared__ float sf[2][kFbThreads / 32];
-        __shared__ uint32_t su[2][kFbThreads / 32];
+        __shared__ uint32_t su[kFbThreads / 32];
         if (lane == 0) {
             sf[0][warp] = s1;
             sf[1][warp] = s2;
-            su[0][warp] = smax;
+            su[warp] = smax;
         }
         __syncthreads();
         s1 = s2 = 0.f;
@@ -319,21 +302,50 @@ __global__ void __launch_bounds__(kFbThreads, 5) topk_bound_kernel(FastArgs a) {
         for (int w = 0; w < kFbThreads / 32; ++w) {
             s1 += sf[0][w];
             s2 += sf[1][w];
-            smax = max(smax, su[0][w]);
+            smax = max(smax, su[w]);
         }
         const float mean = s1 / (float)ns, var = fmaxf(0.f, s2 / (float)ns - mean * mean);
         const float cut = mean + 1.5f * sqrtf(var);
         uint32_t floor = isfinite(cut) ? score_key(cut) : 0u;
-        uint32_t above = 0;
-        for (int i = tid; i < ns; i += kFbThreads) above += skey[i] >= floor;
-        above = __reduce_add_sync(0xFFFFFFFFu, above);
-        if (lane == 0) su[1][warp] = above;
+        // the samples at or above the cut, into a short list (hist's words)
+        __shared__ uint32_t s_m, s_bound;
+        if (tid == 0) {
+            s_m = 0;
+            s_bound = 0xFFFFFFFFu;
+        }
         __syncthreads();
-        above = 0;
-        for (int w = 0; w < kFbThreads / 32; ++w) above += su[1][w];
-        if (above < (uint32_t)r) floor = 0u;
-        const uint32_t bound =
-            kth_largest([&](uint32_t i) { return skey[i]; }, (uint32_t)ns, (uint32_t)r, hist, sh32, res, floor);
+        uint32_t* L = hist;
+        constexpr uint32_t kLcap = kDigBins * kFbThreads / 32;
+        for (int i = tid; i < ns; i += kFbThreads) {
+            const uint32_t kk = skey[i];
+            if (kk >= floor) {
+                const uint32_t q = atom_add_shared(&s_m, 1u);
+                if (q < kLcap) L[q] = kk;
+            }
+        }
+        __syncthreads();
+        const uint32_t m = s_m;
+        uint32_t bound;
+        if (m >= (uint32_t)r && m <= kLcap && m <= 1024u) {
+            // the r-th largest of the list by pairwise ranks
+            for (uint32_t i = tid; i < m; i += kFbThreads) {
+                const uint32_t mk = L[i];
+                uint32_t gt = 0, ge = 0;
+                for (uint32_t o = 0; o < m; ++o) {
+                    const uint32_t ok = L[o];
+                    gt += ok > mk;
+                    ge += ok >= mk;
+                }
+                if (gt < (uint32_t)r && (uint32_t)r <= ge) s_bound = mk;  // every holder writes the same value
+            }
+            __syncthreads();
+            bound = s_bound;
+        } else {  // a sample far from normal: digit passes over every sample (or those above the cut)
+            __syncthreads();  // the list's words are the passes' histograms
+            if (m < (uint32_t)r) floor = 0u;
+            bound = kth_largest([&](uint32_t i) { return skey[i]; }, (uint32_t)ns, (uint32_t)r, hist, sh32, res,
+                                floor);
+        }
         // candidate histogram bins: the sample maximum near the middle bin
         const uint32_t spread = (smax - bound) >> 10;
         const uint32_t shift = spread ? 32u - (uint32_t)__clz((int)spread) : 0u;
@@ -349,6 +361,12 @@ __global__ void __launch_bounds__(kFbThreads, 5) topk_bound_kernel(FastArgs a) {
 
 // ------------------------------------------------------------- 2. scan ----
 // The indexer stream with candidate output.  Grid (nchunks, B), 128 threads.
+// LATE: the bound kernel runs beside this one; the candidates are taken
+// after the last tile, from the keys this CTA wrote (read back by the
+// threads that wrote them), eight tiles per barrier.  Otherwise the bound
+// is known before the first tile and every tile's candidates are written as
+// it is scored.
+template <bool LATE>
 __global__ void __launch_bounds__(kScThreads, 4)
     score_fast_kernel(const __grid_constant__ CUtensorMap ic_map, FastArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -356,36 +374,36 @@ __global__ void __launch_bounds__(kScThreads, 4)
     uint8_t* tiles = smem;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kScStages * kScTileBytes);
     __shared__ float s_emax[kScThreads / 32];
-    __shared__ uint32_t s_wc[2][kScThreads / 32];        // per-warp candidate counts of a tile
-    __shared__ uint32_t s_ec[kFaEarly][kScThreads / 32];  // ... of the early tiles
-    // The selection kernel may begin launching: it waits for this grid.  This
-    // kernel reads only the step's inputs and writes only its own rows before
-    // it awaits the bound kernel (pdl_wait below).
+    __shared__ uint32_t s_wc[2][kScThreads / 32];  // per-warp candidate counts of a tile
+    __shared__ uint32_t s_ec[8][kScThreads / 32];  // ... of eight tiles (LATE)
+    if (!LATE) pdl_wait();  // the bound first: nothing is loaded before it is known
     pdl_release();
     SA_TRACE_MARK(TR_SCORE, 0);
     const int b = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int row0 = blockIdx.x * a.chunk;
-    const int srows = max(0, min(row0 + a.chunk, a.Ncap) - row0);
-    const int stiles = (srows + kScRows - 1) / kScRows;
-    int issued = 0;
-    if (tid == 0) {
-        for (int s = 0; s < kScStages; ++s) mbar_init(&full[s], 1);
-        fence_barrier_init();
-        for (; issued < kScStages && issued < stiles; ++issued) {
-            mbar_expect_tx(&full[issued], kScTileBytes);
-            tma_load_3d(tiles + issued * kScTileBytes, &ic_map, 0, row0 + issued * kScRows, b, &full[issued]);
-        }
-    }
     const int n = clamp_n(a.n, b, a.Ncap);
     if (n <= a.k) {
-        if (tid == 0)
-            for (int i = 0; i < issued; ++i) mbar_wait(&full[i % kScStages], (i / kScStages) & 1);
-        pdl_wait();
+        if (LATE) pdl_wait();  // completion stays transitive along the chain
         return;
     }
     const int row1 = min(row0 + a.chunk, n);
     const int ntiles = row1 > row0 ? (row1 - row0 + kScRows - 1) / kScRows : 0;
+    int issued = 0;
+    if (tid == 0) {
+        for (int s = 0; s < kScStages; ++s) mbar_init(&full[s], 1);
+        fence_barrier_init();
+        for (; issued < kScStages && issued < ntiles; ++issued) {
+            mbar_expect_tx(&full[issued], kScTileBytes);
+            tma_load_3d(tiles + issued * kScTileBytes, &ic_map, 0, row0 + issued * kScRows, b, &full[issued]);
+        }
+    }
+    const uint32_t* ctl = a.ctrl + (size_t)b * kCtl;
+    uint32_t tp = 0, hsh = 0;
+    if (!LATE) {
+        tp = ld_cg_u32(ctl + kCtlBound);
+        hsh = ld_cg_u32(ctl + kCtlShift);
+    }
     float q[64];
     {
         const uint32_t* qw = reinterpret_cast<const uint32_t*>(a.q_idx + (size_t)b * 64);
@@ -398,49 +416,9 @@ __global__ void __launch_bounds__(kScThreads, 4)
     }
     uint32_t* kout = a.keys + (size_t)b * a.Ncap;
     uint2* cd = a.cand + (size_t)b * a.Ncap + row0;
-    const uint32_t lt = (1u << lane) - 1u;
-    uint32_t tp = 0, cbase = 0, hsh = 0;
     uint32_t* ch = a.chist + (size_t)b * kCH;
-    auto hist_add_key = [&](uint32_t key) {  // the candidate's histogram bin (a fire-and-forget add)
-        const uint32_t bin = min((key - tp) >> hsh, (uint32_t)(kCH - 1));
-        asm volatile("red.global.add.u32 [%0], 1;" ::"l"(ch + bin) : "memory");
-    };
-    // the early tiles' candidates, once the bound is known: this thread's own
-    // keys of those tiles are read back (its own writes), ballots per tile and
-    // warp, one barrier, then written in (tile, warp, lane) order
-    auto early = [&](int ne) {
-        pdl_wait();
-        tp = ld_cg_u32(a.ctrl + (size_t)b * kCtl + kCtlBound);
-        hsh = ld_cg_u32(a.ctrl + (size_t)b * kCtl + kCtlShift);
-        uint32_t kk[kFaEarly], bal[kFaEarly];
-#pragma unroll
-        for (int j = 0; j < kFaEarly; ++j) {
-            const int r = row0 + j * kScRows + tid;
-            const bool v = j < ne && r < row1;
-            kk[j] = v ? kout[r] : 0u;
-            bal[j] = __ballot_sync(0xFFFFFFFFu, v && kk[j] >= tp);
-            if (lane == 0 && j < ne) s_ec[j][warp] = __popc(bal[j]);
-        }
-        __syncthreads();
-#pragma unroll
-        for (int j = 0; j < kFaEarly; ++j) {
-            if (j < ne) {
-                uint32_t off = cbase, tot = 0;
-#pragma unroll
-                for (int w = 0; w < kScThreads / 32; ++w) {
-                    const uint32_t c = s_ec[j][w];
-                    off += w < warp ? c : 0u;
-                    tot += c;
-                }
-                if ((bal[j] >> lane) & 1u) {
-                    cd[off + __popc(bal[j] & lt)] = make_uint2(kk[j], (uint32_t)(row0 + j * kScRows + tid));
-                    hist_add_key(kk[j]);
-                }
-                cbase += tot;
-            }
-        }
-    };
-
+    const uint32_t lt = (1u << lane) - 1u;
+    uint32_t cbase = 0;
     int consumed = 0;
     bool timed_out = false;
     float emax = 0.f;
@@ -475,12 +453,9 @@ __global__ void __launch_bounds__(kScThreads, 4)
             kout[row] = key;
             emax = fmaxf(emax, fmaf(aab, 0x1p-16f, fmaf(fabsf(acc), 0x1p-22f, 0x1p-140f)));
         }
-        const bool late = i >= kFaEarly;  // block-uniform
-        uint32_t bal = 0;
-        if (late) {
-            bal = __ballot_sync(0xFFFFFFFFu, valid && key >= tp);
-            if (lane == 0) s_wc[i & 1][warp] = __popc(bal);
-        }
+        const bool cand = !LATE && valid && key >= tp;
+        const uint32_t bal = __ballot_sync(0xFFFFFFFFu, cand);
+        if (!LATE && lane == 0) s_wc[i & 1][warp] = __popc(bal);
         __syncthreads();  // slot s is free again; this tile's warp counts are visible
         if (tid == 0 && issued < ntiles) {
             fence_proxy_async();
@@ -488,7 +463,7 @@ __global__ void __launch_bounds__(kScThreads, 4)
             tma_load_3d(tiles + s * kScTileBytes, &ic_map, 0, row0 + issued * kScRows, b, &full[s]);
             ++issued;
         }
-        if (late) {
+        if (!LATE) {
             uint32_t off = cbase, tot = 0;
 #pragma unroll
             for (int w = 0; w < kScThreads / 32; ++w) {
@@ -496,21 +471,51 @@ __global__ void __launch_bounds__(kScThreads, 4)
                 off += w < warp ? c : 0u;
                 tot += c;
             }
-            if ((bal >> lane) & 1u) {
+            if (cand) {  // the candidate row and its histogram bin (a fire-and-forget add)
                 cd[off + __popc(bal & lt)] = make_uint2(key, (uint32_t)row);
-                hist_add_key(key);
+                const uint32_t bin = min((key - tp) >> hsh, (uint32_t)(kCH - 1));
+                asm volatile("red.global.add.u32 [%0], 1;" ::"l"(ch + bin) : "memory");
             }
             cbase += tot;
         }
-        if (i + 1 == kFaEarly) early(kFaEarly);
     }
     if (tid == 0)
         for (int i = consumed; i < issued; ++i) mbar_wait(&full[i % kScStages], (i / kScStages) & 1);
-    if (timed_out) {
-        __syncthreads();
+    if (timed_out) __syncthreads();
+    if (LATE) {
         pdl_wait();
-    } else if (ntiles < kFaEarly) {
-        early(ntiles);
+        tp = ld_cg_u32(ctl + kCtlBound);
+        hsh = ld_cg_u32(ctl + kCtlShift);
+#pragma unroll 1
+        for (int g = 0; g < consumed; g += 8) {
+            uint32_t kk[8], bal[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int row = row0 + (g + j) * kScRows + tid;
+                const bool v = g + j < consumed && row < row1;
+                kk[j] = v ? kout[row] : 0u;
+                bal[j] = __ballot_sync(0xFFFFFFFFu, v && kk[j] >= tp);
+                if (lane == 0) s_ec[j][warp] = __popc(bal[j]);
+            }
+            __syncthreads();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                uint32_t off = cbase, tot = 0;
+#pragma unroll
+                for (int w = 0; w < kScThreads / 32; ++w) {
+                    const uint32_t c = s_ec[j][w];
+                    off += w < warp ? c : 0u;
+                    tot += c;
+                }
+                if ((bal[j] >> lane) & 1u) {
+                    cd[off + __popc(bal[j] & lt)] = make_uint2(kk[j], (uint32_t)(row0 + (g + j) * kScRows + tid));
+                    const uint32_t bin = min((kk[j] - tp) >> hsh, (uint32_t)(kCH - 1));
+                    asm volatile("red.global.add.u32 [%0], 1;" ::"l"(ch + bin) : "memory");
+                }
+                cbase += tot;
+            }
+            __syncthreads();  // s_ec is rewritten by the next group
+        }
     }
     emax = __uint_as_float(__float_as_uint(emax) + 1u);  // e_j rounded to nearest: one ulp up
 #pragma unroll
@@ -526,39 +531,26 @@ __global__ void __launch_bounds__(kScThreads, 4)
     }
 }
 
-// --------------------------------------------------- 3. select + attend ----
-// Shared memory of the selection + attention kernel (offsets from a
-// 1024-aligned base).  The selecting CTA's candidate list and scratch alias
-// the K / V tiles, which are loaded only after the selection.
-constexpr int kFaQ = 0;                          // Q: 64 heads x 128 dims, K-major SW128, halves 8 KB apart
-constexpr int kFaK = kFaQ + 16384;               // K: two 128-row tiles of 32 KB (K-major SW128)
-constexpr int kFaV = kFaK + 65536;               // V: two tiles, read as the MN-major A operand
-constexpr int kFaP = kFaV + 65536;               // P^T: 256 entries x 64 heads, MN-major B operand
-constexpr int kFaSel = kFaP + 32768;             // the selected list (CTA 0)
-constexpr int kFaSmem = kFaSel + kFastMaxK * 4 + 1024;
-// selection scratch, aliased onto K / V / P
-constexpr int kFaLKey = kFaK;                    // candidate keys   [kFastCap]
-constexpr int kFaLIdx = kFaK + kFastCap * 4;     // candidate indices [kFastCap]
-constexpr int kFaHist = kFaV;                    // digit histograms [16 warps][kDigBins] (or [kBins])
-constexpr int kFaBase = kFaV + 16 * kDigBins * 4;  // chunk positions [kSelMaxChunks + 1]
+// --------------------------------------------------------- 3. selection ----
+// Shared memory of the selection kernel (dynamic, byte offsets).
+constexpr int kFaLKey = 0;                          // candidate keys    [kFastCap]
+constexpr int kFaLIdx = kFaLKey + kFastCap * 4;     // candidate indices [kFastCap]
+constexpr int kFaHist = kFaLIdx + kFastCap * 4;     // digit histograms [16 warps][kDigBins] (or [kBins])
+constexpr int kFaBase = kFaHist + 16 * kDigBins * 4;  // chunk positions [kSelMaxChunks + 1]
 constexpr int kFaBKey = kFaBase + (kSelMaxChunks + 1) * 4 + 12;  // band exact keys [kFaBand]
-constexpr int kFaBIdx = kFaBKey + kFaBand * 4;   // band indices    [kFaBand]
-constexpr int kFaBPos = kFaBIdx + kFaBand * 4;   // band list positions [kFaBand]
-constexpr int kFaPart = kFaK;                    // partial O: [64 heads][128 dims] fp32 (after the S MMAs)
-static_assert(kFaBPos + kFaBand * 4 <= kFaP, "selection scratch fits in the V region");
-static_assert(kFaLIdx + kFastCap * 4 <= kFaV, "the candidate list fits in the K region");
+constexpr int kFaBIdx = kFaBKey + kFaBand * 4;      // band indices    [kFaBand]
+constexpr int kFaBPos = kFaBIdx + kFaBand * 4;      // band list positions [kFaBand]
+constexpr int kStage = 256;                          // candidates of the bins around t~'s, staged for the band
+constexpr int kFaSg = kFaBPos + kFaBand * 4;         // staged keys, indices, list positions, exact keys [4][kStage]
+constexpr int kFaSmem = kFaSg + 4 * kStage * 4;
 static_assert(kFaSmem <= 227 * 1024, "shared memory of one CTA");
+static_assert((kFaBase & 15) == 0 && (kFaBKey & 15) == 0, "16-byte aligned scratch");
 
 struct FaStatic {
-    double q2[64];     // qI * 2^768 (exact rescoring)
-    float red[16][32];  // per-warp partial maxima / sums of its 32 heads
-    float m[64];       // this CTA's partial: max of scale*log2e*s per head
-    float l[64];       // ... and the sum of exp2(. - m)
+    double q2[64];  // qI * 2^768 (exact rescoring)
     uint32_t sh64[64];
     int res[2];
-    uint32_t nb, selcnt, nd, a_cnt, tkey;
-    uint32_t tmem;
-    uint64_t bar_s, bar_o;
+    uint32_t nb, nd, a_cnt, tkey, nsg, hnext;
 };
 
 // The exact selection over a list of (screened key, index) pairs in
@@ -566,12 +558,12 @@ struct FaStatic {
 // (index = position), else the candidate list in shared memory.  Returns
 // false (shared-memory list only) when the list cannot prove the selection:
 // fewer than k entries, or the band reaching below the bound t_p, or a band
-// larger than kFaBand.  On success the ascending selection is in sel[0..k)
-// and in the caller's idx / cnt.
+// larger than kFaBand.  On success the ascending selection is in the
+// caller's idx / cnt.
 // T_in: the k-th largest key when the caller found it (0xFFFFFFFF: not yet).
 template <bool GLOBAL>
 __device__ bool select_exact(const FastArgs& a, FaStatic& S, uint8_t* sm, int b, uint32_t C, uint32_t tp, float E,
-                             uint32_t* lkey, int32_t* lidx, int32_t* sel, uint32_t T_in = 0xFFFFFFFFu) {
+                             uint32_t* lkey, int32_t* lidx, uint32_t T_in = 0xFFFFFFFFu) {
     const int tid = threadIdx.x;
     const uint32_t k = (uint32_t)a.k;
     uint32_t* hist = reinterpret_cast<uint32_t*>(sm + kFaHist);
@@ -674,96 +666,24 @@ __device__ bool select_exact(const FastArgs& a, FaStatic& S, uint8_t* sm, int b,
     for (uint32_t p = p0; p < p1; ++p) {
         if (key_at(p) > bhi) {
             const int32_t j = idx_at(p);
-            if (o < k) {
-                sel[o] = j;
-                gout[o] = j;
-            }
+            if (o < k) gout[o] = j;
             ++o;
         }
     }
     if (tid == 0) {
         if (total != k) flag(DEV_LEN);  // cannot happen
         a.cnt[b] = (int32_t)k;
-        S.selcnt = k;
     }
     return true;
 }
 
-// 2^x on the special-function unit (flushes subnormal results to zero: the
-// softmax weights are at least 2^-126 wherever they matter, since the
-// largest is 1)
-__device__ __forceinline__ float fast_exp2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-// Transposed reduction of 32 values per lane over the warp's 32 lanes (max
-// or sum per value index): at each of the five butterfly steps a lane keeps
-// one half of its values and sends the other half to its partner, so that
-// lane l ends with the reduction of value index l.
-template <bool MAX>
-__device__ __forceinline__ float head_reduce32(float (&v)[32], int lane) {
-#pragma unroll
-    for (int step = 0; step < 5; ++step) {
-        const int half = 16 >> step;
-        const int o = 16 >> step;
-        const bool upper = (lane & o) != 0;
-#pragma unroll
-        for (int i = 0; i < half; ++i) {
-            const float keep = upper ? v[half + i] : v[i];
-            const float send = upper ? v[i] : v[half + i];
-            const float got = __shfl_xor_sync(0xFFFFFFFFu, send, o);
-            v[i] = MAX ? fmaxf(keep, got) : keep + got;
-        }
-    }
-    return v[0];
-}
-
-// Byte offset of (row r, 16-byte chunk c) in a K-major SW128 operand whose
-// two 64-element halves lie `half` bytes apart.
-__device__ __forceinline__ uint32_t sw128_off(int r, int c, uint32_t half) {
-    return (uint32_t)(c >> 3) * half + (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + (((c & 7) ^ (r & 7)) << 4));
-}
-
-// Instruction descriptor, kind::f16 with fp32 D and bf16 A / B: M = 128,
-// N = 64; a_mn / b_mn select MN-major operands.
-__device__ __forceinline__ uint32_t fa_idesc(uint32_t a_mn, uint32_t b_mn) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | (a_mn << 15) | (b_mn << 16) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
-}
-
-// Grid (kFaCluster, B), clusters of kFaCluster CTAs along x.
-__global__ void __launch_bounds__(kFaThreads, 1) csa_select_attend_kernel(FastArgs a) {
-    extern __shared__ uint8_t fa_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fa_raw) + 1023) & ~uintptr_t(1023));
+// Grid (B): one CTA per sequence.
+__global__ void __launch_bounds__(kFaThreads, 1) csa_select_fast_kernel(FastArgs a) {
+    extern __shared__ __align__(16) uint8_t sm[];
     __shared__ FaStatic S;
-    const int b = blockIdx.y;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const uint32_t rank = cluster_rank();
-    int32_t* sel = reinterpret_cast<int32_t*>(sm + kFaSel);
-    const uint32_t sQ = smem_u32(sm + kFaQ), sK = smem_u32(sm + kFaK), sV = smem_u32(sm + kFaV),
-                   sP = smem_u32(sm + kFaP);
-
-    // Q (an input) before waiting for the scan: rows h < H, the rest zero
-    {
-        const int h = tid >> 3, c0 = (tid & 7) * 2;  // 64 rows x 16 chunks: 2 chunks per thread
-        const bool ok = h < a.H;
-        const uint16_t* src = a.q + ((size_t)b * a.H + (ok ? h : 0)) * 128;
-#pragma unroll
-        for (int c = c0; c < c0 + 2; ++c) cp_async16_zfill(sm + kFaQ + sw128_off(h, c, 8192), src + c * 8, ok);
-        cp_async_commit();
-    }
-    if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&S.tmem)),
-                     "r"(256));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-    }
-    if (tid == 0) {
-        mbar_init(&S.bar_s, 1);
-        mbar_init(&S.bar_o, 1);
-        fence_barrier_init();
-    }
-    if (rank == 0 && tid < 32) {  // qI * 2^768 in fp64 (exact rescoring)
+    const int b = blockIdx.x;
+    const int tid = threadIdx.x;
+    if (tid < 32) {  // qI * 2^768 in fp64 (exact rescoring); an input, read before the wait
         const uint32_t w = reinterpret_cast<const uint32_t*>(a.q_idx + (size_t)b * 64)[tid];
         S.q2[2 * tid] = (double)bf16lo_f32(w) * 0x1p768;
         S.q2[2 * tid + 1] = (double)bf16hi_f32(w) * 0x1p768;
@@ -772,21 +692,12 @@ __global__ void __launch_bounds__(kFaThreads, 1) csa_select_attend_kernel(FastAr
     pdl_release();
     SA_TRACE_MARK(TR_FAST, 0);
     const int n = clamp_n(a.n, b, a.Ncap);
-
-    // ---- the selection (CTA 0) ----
-    if (rank == 0) {
+    {
         const uint32_t k = (uint32_t)a.k;
         if ((uint32_t)n <= k) {  // every visible entry, ascending
             int32_t* gout = a.idx + (size_t)b * a.k;
-            for (int i = tid; i < a.k; i += kFaThreads) {
-                const int32_t j = i < n ? i : -1;
-                gout[i] = j;
-                if (i < n) sel[i] = j;
-            }
-            if (tid == 0) {
-                a.cnt[b] = n;
-                S.selcnt = (uint32_t)n;
-            }
+            for (int i = tid; i < a.k; i += kFaThreads) gout[i] = i < n ? i : -1;
+            if (tid == 0) a.cnt[b] = n;
         } else {
             const uint32_t* ctl = a.ctrl + (size_t)b * kCtl;
             const uint32_t tp = ld_cg_u32(ctl + kCtlBound);
@@ -809,6 +720,22 @@ __global__ void __launch_bounds__(kFaThreads, 1) csa_select_attend_kernel(FastAr
                     const int c = tid * CPT + j;
                     cv[j] = c < a.nchunks ? ld_cg_u32(cc + c) : 0u;
                     sum += cv[j];
+                }
+                // ahead of the counts: the first kSpecS * 32 candidate slots of each
+                // warp's first kSpecJ chunks (chunk c = warp + 16 j)
+                constexpr int kSpecJ = 8, kSpecS = 2;
+                const int lane = tid & 31, warp = tid >> 5;
+                const uint2* cs = a.cand + (size_t)b * a.Ncap;
+                uint2 spec[kSpecJ][kSpecS];
+#pragma unroll
+                for (int j = 0; j < kSpecJ; ++j) {
+                    const int c = warp + 16 * j;
+                    const int rows = c < a.nchunks ? min(a.chunk, a.Ncap - c * a.chunk) : 0;
+#pragma unroll
+                    for (int u = 0; u < kSpecS; ++u) {
+                        const int slot = lane + 32 * u;
+                        spec[j][u] = slot < rows ? __ldcg(cs + (size_t)c * a.chunk + slot) : make_uint2(0u, 0u);
+                    }
                 }
                 const int htop = kCH - 1 - tid * HPT;  // this thread's highest bin
                 const uint4 hv4 = ld_cg_u32x4(chg + htop - (HPT - 1));
@@ -834,59 +761,76 @@ __global__ void __launch_bounds__(kFaThreads, 1) csa_select_attend_kernel(FastAr
                 if (tid == 0) {
                     base[a.nchunks] = C;
                     S.nd = 0;
+                    S.nsg = 0;
+                    S.hnext = 0;
                 }
                 __syncthreads();
                 const int d = S.res[0];
                 const uint32_t above_d = (uint32_t)S.res[1];
+#pragma unroll
+                for (int j = 0; j < HPT; ++j)  // the count of bin d + 1, for the band's count above it
+                    if (htop - j == d + 1) S.hnext = hv[j];
                 if (C >= k && C <= (uint32_t)kFastCap && htot == C && d >= 0) {
-                    // the list: thread t copies positions [t*per, (t+1)*per), finding its
-                    // first chunk by binary search over the positions; the keys of
-                    // bin d go to a short list as well
+                    // The list: warp w copies chunks w, w + 16, ... (the first slots
+                    // of its first chunks are in registers already).  The keys of
+                    // bin d go to a short list, and the candidates of bins d - 1 ..
+                    // d + 1 (where the band will lie) are staged.
                     uint32_t* lkey = reinterpret_cast<uint32_t*>(sm + kFaLKey);
                     int32_t* lidx = reinterpret_cast<int32_t*>(sm + kFaLIdx);
                     uint32_t* dkey = reinterpret_cast<uint32_t*>(sm + kFaBKey);  // the band's arrays, free until then
-                    constexpr int kPer = kFastCap / kFaThreads;  // positions per thread at most (16)
-                    const uint32_t per = (C + kFaThreads - 1) / kFaThreads;
-                    const uint32_t p0 = min(C, tid * per), p1 = min(C, p0 + per);
-                    if (p0 < p1) {
-                        int lo = 0, hi = a.nchunks - 1;  // the last chunk c with base[c] <= p0
-                        while (lo < hi) {
-                            const int mid = (lo + hi + 1) >> 1;
-                            if (base[mid] <= p0) lo = mid;
-                            else hi = mid - 1;
+                    uint32_t* sg_key = reinterpret_cast<uint32_t*>(sm + kFaSg);
+                    int32_t* sg_idx = reinterpret_cast<int32_t*>(sm + kFaSg + kStage * 4);
+                    uint32_t* sg_pos = reinterpret_cast<uint32_t*>(sm + kFaSg + 2 * kStage * 4);
+                    uint32_t* sg_ek = reinterpret_cast<uint32_t*>(sm + kFaSg + 3 * kStage * 4);
+                    auto put = [&](uint32_t p, uint2 e) {
+                        lkey[p] = e.x;
+                        lidx[p] = (int32_t)e.y;
+                        const int bin = (int)min((e.x - tp) >> hsh, (uint32_t)(kCH - 1));
+                        if (bin == d) {
+                            const uint32_t q = atom_add_shared(&S.nd, 1u);
+                            if (q < (uint32_t)kFaBand) dkey[q] = e.x;
                         }
-                        int c = lo;
-                        const uint2* cs = a.cand + (size_t)b * a.Ncap;
-                        uint2 e[kPer];  // every load in flight before the first store
-#pragma unroll
-                        for (int u = 0; u < kPer; ++u) {
-                            const uint32_t p = p0 + u;
-                            if (p < p1) {
-                                while (p >= base[c + 1]) ++c;  // chunks with no candidates are skipped
-                                e[u] = __ldcg(cs + (size_t)c * a.chunk + (p - base[c]));
+                        if (bin + 1 >= d && bin <= d + 1) {
+                            const uint32_t q = atom_add_shared(&S.nsg, 1u);
+                            if (q < (uint32_t)kStage) {
+                                sg_key[q] = e.x;
+                                sg_idx[q] = (int32_t)e.y;
+                                sg_pos[q] = p;
                             }
                         }
+                    };
 #pragma unroll
-                        for (int u = 0; u < kPer; ++u) {
-                            if (p0 + u < p1) {
-                                lkey[p0 + u] = e[u].x;
-                                lidx[p0 + u] = (int32_t)e[u].y;
-                                if ((int)min((e[u].x - tp) >> hsh, (uint32_t)(kCH - 1)) == d) {
-                                    const uint32_t q = atom_add_shared(&S.nd, 1u);
-                                    if (q < (uint32_t)kFaBand) dkey[q] = e[u].x;
-                                }
-                            }
+                    for (int j = 0; j < kSpecJ; ++j) {
+                        const int c = warp + 16 * j;
+                        if (c < a.nchunks) {
+                            const uint32_t cb = base[c], cn = base[c + 1] - cb;
+#pragma unroll
+                            for (int u = 0; u < kSpecS; ++u)
+                                if ((uint32_t)(lane + 32 * u) < cn) put(cb + lane + 32 * u, spec[j][u]);
                         }
+                    }
+#pragma unroll 1
+                    for (int c = warp; c < a.nchunks; c += 16) {  // slots not loaded ahead
+                        const uint32_t cb = base[c], cn = base[c + 1] - cb;
+                        const uint32_t from = c < 16 * kSpecJ ? 32u * kSpecS : 0u;
+                        for (uint32_t i = from + lane; i < cn; i += 32) put(cb + i, __ldcg(cs + (size_t)c * a.chunk + i));
                     }
                     __syncthreads();
                     SA_TRACE_MARK(TR_FAST, 1);
-                    // the k-th largest key: rank R = k - above_d inside bin d
+                    // the k-th largest key (rank R = k - above_d inside bin d) by
+                    // threads 0-255; the staged candidates' exact keys (the fp64
+                    // definition) meanwhile by threads 256-511
                     uint32_t T = 0xFFFFFFFFu;
-                    const uint32_t nd = S.nd, R = k - above_d;
-                    if (nd <= (uint32_t)kFaBand) {
-                        if (tid == 0) S.tkey = 0xFFFFFFFFu;
-                        __syncthreads();
-                        for (uint32_t i = tid; i < nd; i += kFaThreads) {
+                    const uint32_t nd = S.nd, R = k - above_d, nsg = S.nsg;
+                    if (tid == 0) S.tkey = 0xFFFFFFFFu;
+                    __syncthreads();
+                    const uint16_t* icx = a.kidx + (size_t)b * a.Ncap * 64;
+                    if (tid >= kFaThreads - kStage) {
+                        const int i = tid - (kFaThreads - kStage);
+                        if ((uint32_t)i < nsg && nsg <= (uint32_t)kStage)
+                            sg_ek[i] = exact_key(S.q2, icx + (size_t)sg_idx[i] * 64);
+                    } else if (nd <= (uint32_t)kFaBand) {
+                        for (uint32_t i = tid; i < nd; i += kFaThreads - kStage) {
                             const uint32_t mk = dkey[i];
                             uint32_t gt = 0, ge = 0;
                             for (uint32_t o = 0; o < nd; ++o) {
@@ -896,220 +840,77 @@ __global__ void __launch_bounds__(kFaThreads, 1) csa_select_attend_kernel(FastAr
                             }
                             if (gt < R && R <= ge) S.tkey = mk;  // every holder of the key writes the same value
                         }
-                        __syncthreads();
-                        T = S.tkey;
                     }
-                    done = select_exact<false>(a, S, sm, b, C, tp, E, lkey, lidx, sel, T);
+                    __syncthreads();
+                    T = S.tkey;
+                    SA_TRACE_MARK(TR_FAST, 2);
+                    // the band from the staged candidates when it lies inside their bins
+                    bool staged = false;
+                    uint32_t bhi = 0;
+                    if (T != 0xFFFFFFFFu && nsg <= (uint32_t)kStage) {
+                        const float t = key_to_float(T);
+                        const float e2 = __fmul_ru(2.f, E);
+                        bhi = score_key(__fadd_ru(t, e2));
+                        const uint32_t blo = score_key(__fsub_rd(t, e2));
+                        const unsigned long long lo_edge = (unsigned long long)tp + ((unsigned long long)max(d - 1, 0) << hsh);
+                        const unsigned long long hi_edge =
+                            d + 1 >= kCH - 1 ? 0xFFFFFFFFull
+                                             : (unsigned long long)tp + ((unsigned long long)(d + 2) << hsh) - 1ull;
+                        staged = blo >= tp && (unsigned long long)blo >= lo_edge && (unsigned long long)bhi <= hi_edge;
+                        if (staged) {
+                            // above the band: the bins above d + 1, and staged keys above bhi
+                            const uint32_t hnext = d + 1 <= kCH - 1 ? S.hnext : 0u;
+                            uint32_t A = above_d - hnext;
+                            for (uint32_t o = 0; o < nsg; ++o) A += sg_key[o] > bhi;
+                            const uint32_t R2 = k - A;  // band winners (>= 1)
+                            // the cut among the staged band members by (exact key desc, index asc)
+                            if ((uint32_t)tid < nsg) {
+                                const uint32_t mk = sg_key[tid];
+                                if (mk >= blo && mk <= bhi) {
+                                    const uint32_t me = sg_ek[tid];
+                                    const int32_t mj = sg_idx[tid];
+                                    uint32_t rank = 0;
+                                    for (uint32_t o = 0; o < nsg; ++o) {
+                                        const uint32_t ok = sg_key[o];
+                                        if (ok < blo || ok > bhi) continue;
+                                        const uint32_t oe = sg_ek[o];
+                                        rank += (oe > me) || (oe == me && sg_idx[o] < mj);
+                                    }
+                                    lkey[sg_pos[tid]] = rank < R2 ? 0xFFFFFFFFu : 0u;
+                                }
+                            }
+                            __syncthreads();
+                            SA_TRACE_MARK(TR_FAST, 4);
+                            // ordered compaction: entries with a key above the band, ascending
+                            int32_t* gout = a.idx + (size_t)b * a.k;
+                            const uint32_t per = (C + kFaThreads - 1) / kFaThreads;
+                            const uint32_t p0 = min(C, tid * per), p1 = min(C, p0 + per);
+                            uint32_t mine = 0;
+                            for (uint32_t p = p0; p < p1; ++p) mine += lkey[p] > bhi;
+                            uint32_t total;
+                            uint32_t o = block_exclusive_scan(mine, S.sh64, &total);
+                            for (uint32_t p = p0; p < p1; ++p) {
+                                if (lkey[p] > bhi) {
+                                    if (o < k) gout[o] = lidx[p];
+                                    ++o;
+                                }
+                            }
+                            if (tid == 0) {
+                                if (total != k) flag(DEV_LEN);  // cannot happen
+                                a.cnt[b] = (int32_t)k;
+                            }
+                            done = true;
+                        }
+                    }
+                    if (!done)
+                    done = select_exact<false>(a, S, sm, b, C, tp, E, lkey, lidx, T);
                 }
             }
-            if (!done) select_exact<true>(a, S, sm, b, (uint32_t)n, tp, E, nullptr, nullptr, sel);
+            if (!done) select_exact<true>(a, S, sm, b, (uint32_t)n, tp, E, nullptr, nullptr);
         }
         __syncthreads();
     }
     SA_TRACE_MARK(TR_FAST, 5);
-    cluster_sync();  // the selection is in CTA 0's shared memory
-
-    // ---- this CTA's slice of the selection: gather, S^T, softmax, O^T ----
-    const int p0 = (int)rank * kFaEntries;
-    const int e_g = tid & (kFaEntries - 1);  // the slice entry this thread gathers (K: tid < 256, V: the rest)
-    const uint32_t cnt = ld_dsmem_u32(dsmem_addr(&S.selcnt, 0));
-    const int jl = (int)ld_dsmem_u32(dsmem_addr(&sel[p0 + e_g], 0));  // in the list's capacity; used below len
-    const int len = max(0, min((int)cnt - p0, kFaEntries));
-    {
-        int j = 0;
-        bool ok = e_g < len;
-        if (ok) {
-            j = jl;
-            if (j < 0 || j >= n) {
-                flag(DEV_INDEX);
-                ok = false;
-                j = 0;
-            }
-        }
-        const bool isv = tid >= kFaEntries;
-        const uint16_t* src = (isv ? a.V : a.K) + ((size_t)b * a.Ncap + j) * 128;
-        uint8_t* dst = sm + (isv ? kFaV : kFaK) + (e_g >> 7) * 32768;
-        const int r = e_g & 127;
-#pragma unroll
-        for (int c = 0; c < 16; ++c) cp_async16_zfill(dst + sw128_off(r, c, 16384), src + c * 8, ok);
-        cp_async_commit();
-    }
-    cp_async_wait<0>();
-    fence_async_smem();
-    __syncthreads();
-    SA_TRACE_MARK(TR_FAST, 6);
-    tc_fence_after();
-    const uint32_t tmem = S.tmem;
-    const int ntile = (len + 127) >> 7;  // 0, 1 or 2 (block-uniform)
-    int pend_s = 0, pend_o = 0;
-    if (ntile > 0 && tid == 0) {
-        const uint32_t id = fa_idesc(0, 0);
-        for (int u = 0; u < ntile; ++u) {
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t ka = sK + u * 32768 + (ks >> 2) * 16384 + (ks & 3) * 32;
-                const uint32_t qb = sQ + (ks >> 2) * 8192 + (ks & 3) * 32;
-                tc_mma(tmem + 64 * u, tc_desc(ka, 16, 1024), tc_desc(qb, 16, 1024), id, ks > 0);
-            }
-        }
-        tc_commit(&S.bar_s);
-        pend_s = 1;
-    }
-    if (ntile > 0) {
-        if (mbar_wait(&S.bar_s, 0) && tid == 0) pend_s = 0;  // a timeout is recorded in the status word
-    }
-    tc_fence_after();
-    SA_TRACE_MARK(TR_FAST, 7);
-    // softmax over this slice, per head: thread = (entry, half of the heads);
-    // warp w takes TMEM lane quarter w % 4, tile (w / 4) % 2 and heads
-    // 32 * (w / 8) .. +31, reading its 32 scores from TMEM twice (for the
-    // maxima, then for the weights) rather than holding them across the
-    // reduction
-    const int u = (warp >> 2) & 1, quarter = warp & 3, hh = warp >> 3;
-    const int e = u * 128 + quarter * 32 + lane;
-    const bool valid = e < len;
-    const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + 64 * u + 32 * hh;
-    float v[32];
-    auto load_s = [&]() {
-        uint32_t r[32];
-        tc_ld32_nw(ta, r);
-        tc_wait_ld();
-#pragma unroll
-        for (int h = 0; h < 32; ++h) v[h] = valid ? __uint_as_float(r[h]) * a.scale_log2 : -INFINITY;
-    };
-    if (u < ntile) {
-        load_s();
-    } else {
-#pragma unroll
-        for (int h = 0; h < 32; ++h) v[h] = -INFINITY;
-    }
-    S.red[warp][lane] = head_reduce32<true>(v, lane);  // head 32 * hh + lane
-    __syncthreads();
-    if (tid < 64) {  // head tid: the eight warps of its half
-        const int w0 = (tid >> 5) * 8;
-        float m = S.red[w0][tid & 31];
-#pragma unroll
-        for (int w = 1; w < 8; ++w) m = fmaxf(m, S.red[w0 + w][tid & 31]);
-        S.m[tid] = m;
-    }
-    __syncthreads();
-    if (u < ntile) load_s();
-    // P^T row of this entry (bf16, heads contiguous): p = 2^(s - m), 0 off the slice
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            const int h = c * 8 + w * 2;
-            const float p0v = valid ? fast_exp2(v[h] - S.m[32 * hh + h]) : 0.f;  // valid: m is finite
-            const float p1v = valid ? fast_exp2(v[h + 1] - S.m[32 * hh + h + 1]) : 0.f;
-            v[h] = p0v;
-            v[h + 1] = p1v;
-            pk[w] = pack_bf16x2(p0v, p1v);
-        }
-        const int cc = 4 * hh + c;  // 16-byte chunk of the entry's 128-byte row
-        *reinterpret_cast<uint4*>(sm + kFaP + (e >> 3) * 1024 + (e & 7) * 128 + ((cc ^ (e & 7)) << 4)) =
-            make_uint4(pk[0], pk[1], pk[2], pk[3]);
-    }
-    const float lsum = head_reduce32<false>(v, lane);
-    __syncthreads();  // every read of the maxima in S.red is done
-    S.red[warp][lane] = lsum;
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    SA_TRACE_MARK(TR_FAST, 8);
-    if (tid < 64) {
-        const int w0 = (tid >> 5) * 8;
-        float l = 0.f;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) l += S.red[w0 + w][tid & 31];
-        S.l[tid] = l;
-    }
-    // O^T = V^T P^T over the slice's 16-entry steps
-    const int nks = (len + 15) >> 4;
-    if (nks > 0 && tid == 0) {
-        tc_fence_after();
-        const uint32_t id = fa_idesc(1, 1);
-        for (int ks = 0; ks < nks; ++ks) {
-            const uint32_t va = sV + (ks >> 3) * 32768 + (ks & 7) * 2048;
-            tc_mma(tmem + 128, tc_desc(va, 16384, 1024), tc_desc(sP + ks * 2048, 16384, 1024), id, ks > 0);
-        }
-        tc_commit(&S.bar_o);
-        pend_o = 1;
-    }
-    if (nks > 0) {
-        if (mbar_wait(&S.bar_o, 0) && tid == 0) pend_o = 0;
-    }
-    tc_fence_after();
-    SA_TRACE_MARK(TR_FAST, 9);
-    // the partial O^T (lane = dim, column = head) into shared memory as [head][dim]
-    float* part = reinterpret_cast<float*>(sm + kFaPart);
-    if (warp < 8) {
-        const int d = quarter * 32 + lane, ph = u;  // warps 4-7 take heads 32-63
-        if (nks > 0) {
-            uint32_t r0[32];
-            tc_ld32_nw(tmem + ((uint32_t)(quarter * 32) << 16) + 128 + 32 * ph, r0);
-            tc_wait_ld();
-#pragma unroll
-            for (int h = 0; h < 32; ++h) part[(32 * ph + h) * 128 + d] = __uint_as_float(r0[h]);
-        } else {
-#pragma unroll
-            for (int h = 0; h < 32; ++h) part[(32 * ph + h) * 128 + d] = 0.f;
-        }
-    }
-    if (tid == 0) {  // an MMA still in flight after a timeout is waited for before TMEM is freed
-        if (pend_s) mbar_wait(&S.bar_s, 0);
-        if (pend_o) mbar_wait(&S.bar_o, 0);
-    }
-    tc_fence_before();
-    __syncthreads();
-    SA_TRACE_MARK(TR_FAST, 10);
-    cluster_sync();  // every CTA's partial is in its shared memory
-
-    // ---- merge: CTA r writes heads 8r .. 8r+7 (warps 0-7, one head each) ----
-    {
-        const int h = (int)rank * 8 + (tid >> 5);
-        const int d = (tid & 31) * 4;
-        if (warp < 8 && h < a.H) {
-            // every remote load is issued before the first use
-            float mr[kFaCluster], lr[kFaCluster], M = -INFINITY;
-            float4 xr[kFaCluster];
-#pragma unroll
-            for (int r = 0; r < kFaCluster; ++r) {
-                mr[r] = ld_dsmem_f32(dsmem_addr(&S.m[h], (uint32_t)r));
-                lr[r] = ld_dsmem_f32(dsmem_addr(&S.l[h], (uint32_t)r));
-                xr[r] = ld_dsmem_f32x4(dsmem_addr(part + h * 128 + d, (uint32_t)r));
-            }
-#pragma unroll
-            for (int r = 0; r < kFaCluster; ++r) M = fmaxf(M, mr[r]);
-            float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f, L = 0.f;
-#pragma unroll
-            for (int r = 0; r < kFaCluster; ++r) {
-                if (mr[r] == -INFINITY) continue;  // an empty slice
-                const float w = exp2f(mr[r] - M);
-                const float4 x = xr[r];
-                o0 = fmaf(w, x.x, o0);
-                o1 = fmaf(w, x.y, o1);
-                o2 = fmaf(w, x.z, o2);
-                o3 = fmaf(w, x.w, o3);
-                L = fmaf(w, lr[r], L);
-            }
-            const bool empty = !(L > 0.f);
-            const float inv = empty ? 0.f : 1.f / L;
-            uint2 pk;
-            pk.x = pack_bf16x2(o0 * inv, o1 * inv);
-            pk.y = pack_bf16x2(o2 * inv, o3 * inv);
-            *reinterpret_cast<uint2*>(a.out + ((size_t)b * a.H + h) * 128 + d) = pk;
-            if (a.lse && (tid & 31) == 0)
-                a.lse[(size_t)b * a.H + h] = empty ? -INFINITY : (M + __log2f(L)) * 0.6931471805599453f;
-        }
-    }
-    SA_TRACE_MARK(TR_FAST, 11);
-    cluster_sync();  // no CTA leaves while others read its shared memory
-    if (warp == 0) {
-        tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256));
-    }
 }
 
 }  // namespace sa

@@ -44,16 +44,21 @@ struct TraceRec {
 __device__ TraceRec* g_trace_buf = nullptr;
 __device__ uint32_t g_trace_cap = 0;
 __device__ uint32_t g_trace_n = 0;
+// Marks stand at CTA-uniform points; the warp reconverges after thread 0's
+// record, since a warp-wide ".aligned" instruction (a cluster barrier, a
+// tensor-memory load) may follow.
 __device__ __forceinline__ void trace_mark(uint32_t kernel, uint32_t phase) {
-    if (threadIdx.x != 0 || g_trace_buf == nullptr) return;
-    unsigned long long t;
-    uint32_t sm;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
-    const uint32_t i = atomicAdd(&g_trace_n, 1u);
-    if (i < g_trace_cap)
-        g_trace_buf[i] = {t, (uint16_t)kernel, (uint16_t)phase, (uint16_t)sm,
-                          (uint16_t)(blockIdx.x + gridDim.x * blockIdx.y)};
+    if (threadIdx.x == 0 && g_trace_buf != nullptr) {
+        unsigned long long t;
+        uint32_t sm;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+        const uint32_t i = atomicAdd(&g_trace_n, 1u);
+        if (i < g_trace_cap)
+            g_trace_buf[i] = {t, (uint16_t)kernel, (uint16_t)phase, (uint16_t)sm,
+                              (uint16_t)(blockIdx.x + gridDim.x * blockIdx.y)};
+    }
+    __syncwarp();
 }
 #define SA_TRACE_MARK(kernel, phase) ::sa::trace_mark((kernel), (phase))
 #else

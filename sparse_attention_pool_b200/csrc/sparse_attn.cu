@@ -32,7 +32,7 @@ thread_local char g_err[512] = "";
 thread_local uint64_t g_launches = 0;
 thread_local cudaEvent_t g_stage_ev[SA_NUM_STAGES][2] = {};
 std::atomic<int> g_prefill_select{1};  // SA_OPT_PREFILL_SELECT
-std::atomic<int> g_decode_fast{1};      // SA_OPT_DECODE_FAST
+std::atomic<int> g_decode_fast{0};      // SA_OPT_DECODE_FAST
 
 // Inside a stream capture the record must become a graph node of its own
 // (an "external" record), so that replays re-record the event.
@@ -57,8 +57,24 @@ bool pdl_on() {
     return true;
 }
 
-// cudaLaunchKernelEx with optional programmatic stream serialization and an
-// optional cluster shape.
+// Scheduling priority of the kernels launched through launch_k while set
+// (0: none).  The CSA chain of a hybrid decode step runs at the device's
+// highest priority, so that its latency-bound kernels take SMs ahead of the
+// concurrent HCA branch's CTAs as those drain.
+thread_local int g_launch_priority = 0;
+struct PriorityScope {
+    int old;
+    explicit PriorityScope(int p) : old(g_launch_priority) { g_launch_priority = p; }
+    ~PriorityScope() { g_launch_priority = old; }
+};
+int highest_priority() {
+    int least = 0, greatest = 0;
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return 0;
+    return greatest;
+}
+
+// cudaLaunchKernelEx with optional programmatic stream serialization, an
+// optional cluster shape and the current launch priority.
 template <typename... P, typename... A>
 cudaError_t launch_k(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
                      unsigned cluster_x, A&&... args) {
@@ -67,8 +83,13 @@ cudaError_t launch_k(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, c
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[2];
+    cudaLaunchAttribute attr[3];
     unsigned na = 0;
+    if (g_launch_priority != 0) {
+        attr[na].id = cudaLaunchAttributePriority;
+        attr[na].val.priority = g_launch_priority;
+        ++na;
+    }
     if (pdl) {
         attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[na].val.programmaticStreamSerializationAllowed = 1;
@@ -637,71 +658,69 @@ sa_status run_topk_decode(const void* q_idx, const sa_cache* c, int k, int32_t* 
 // k-th largest score (k / 32), and at most kFbSamp sample rows.
 int fast_stride(int Ncap, int k) { return std::max(1, std::max(k / 32, cdiv(Ncap, sa::kFbSamp))); }
 
-// The fast path serves a bf16 CSA cache with bf16 indexer keys, up to 64
-// heads and k <= 2048 (eight CTAs of 256 entries); other calls take the
-// general kernels.
-bool fast_decode_ok(const sa_cache* c, int H, int k) {
-    if (g_decode_fast.load() == sa::kFastOff || c->dtype != SA_BF16 || H > 64 || k > sa::kFastMaxK || c->Ncap < 1)
-        return false;
-    const int chunk = score_chunk(c->B, c->Ncap);
-    return cdiv(c->Ncap, chunk) <= sa::kSelMaxChunks;
+// With few sequences the bound kernel runs beside the scan on SMs of its own
+// (late candidates); the scan then has three CTAs on every other SM.
+bool fast_late(int B) {
+    (void)B;
+    return false;
+}
+int fast_chunk(int B, int Ncap) {
+    const long long target = 3LL * (fast_late(B) ? num_sms() - B * sa::kFbCluster : num_sms());
+    long long chunk = ((long long)B * Ncap + target - 1) / target;
+    chunk = ((chunk + sa::kScRows - 1) / sa::kScRows) * sa::kScRows;
+    return (int)std::max<long long>(chunk, sa::kScRows);
 }
 
-// The CSA branch of a hybrid decode step on the fast path: the bound
-// kernel, the indexer scan with candidate output, then one cluster kernel
-// per sequence for the exact selection and the attention over it.
+// The fast selection serves bf16 indexer keys with k <= 2048 (twice k fits
+// the selecting CTA's candidate list); other calls take the general kernels.
+bool fast_decode_ok(const sa_cache* c, int H, int k) {
+    (void)H;
+    if (g_decode_fast.load() == sa::kFastOff || k > sa::kFastMaxK || c->Ncap < 1) return false;
+    return cdiv(c->Ncap, fast_chunk(c->B, c->Ncap)) <= sa::kSelMaxChunks;
+}
+
+// The indexer + top-k of a hybrid decode step on the fast path: the bound
+// kernel, the indexer scan with candidate output, and the selection kernel.
 // `between` runs once the scan is queued (the HCA branch forks there).
 template <typename F>
-sa_status run_fast_decode(const void* q, const void* q_idx, int H, const sa_cache* c, int k, float scale, void* out,
-                          float* lse, int32_t* idx, int32_t* cnt, void* ws, const TopkDecodeWs& w, cudaStream_t st,
-                          F&& between) {
+sa_status run_fast_topk(const void* q_idx, const sa_cache* c, int k, int32_t* idx, int32_t* cnt, void* ws,
+                        const TopkDecodeWs& w, cudaStream_t st, F&& between) {
     const int B = c->B, Ncap = c->Ncap;
     uint8_t* base = static_cast<uint8_t*>(ws);
     sa::FastArgs a{};
-    a.q = static_cast<const uint16_t*>(q);
     a.q_idx = static_cast<const uint16_t*>(q_idx);
     a.kidx = static_cast<const uint16_t*>(c->kidx);
-    a.K = static_cast<const uint16_t*>(c->k);
-    a.V = static_cast<const uint16_t*>(c->v);
     a.n = c->n;
     a.ctrl = reinterpret_cast<uint32_t*>(base + w.fctrl);
-    a.ccount = reinterpret_cast<uint32_t*>(base + w.fccount);
     a.chist = reinterpret_cast<uint32_t*>(base + w.fchist);
+    a.ccount = reinterpret_cast<uint32_t*>(base + w.fccount);
     a.cand = reinterpret_cast<uint2*>(base + w.fcand);
     a.keys = reinterpret_cast<uint32_t*>(base + w.keys);
     a.amb_key = reinterpret_cast<uint32_t*>(base + w.amb_key);
     a.amb_idx = reinterpret_cast<int32_t*>(base + w.amb_idx);
     a.idx = idx;
     a.cnt = cnt;
-    a.out = static_cast<uint16_t*>(out);
-    a.lse = lse;
-    a.H = H;
     a.Ncap = Ncap;
     a.k = k;
-    a.chunk = score_chunk(B, Ncap);
+    a.chunk = fast_chunk(B, Ncap);
     a.nchunks = cdiv(Ncap, a.chunk);
     a.sstride = fast_stride(Ncap, k);
+    const bool late = fast_late(B);
     a.mode = g_decode_fast.load();
-    const float sc = scale == 0.f ? 1.0f / sqrtf(128.0f) : scale;
-    a.scale_log2 = sc * 1.4426950408889634f;
     if (a.nchunks > w.maxchunks || a.nchunks > sa::kSelMaxChunks)
         return fail(SA_ERR_WORKSPACE, "internal: chunk count above the workspace bound");
     const size_t smem = sa::kScStages * sa::kScTileBytes + sa::kScStages * 8 + 1024;
     static std::atomic<uint64_t> init{0};
     if (!attr_done(init)) {
-        SA_CUDA(cudaFuncSetAttribute(sa::score_fast_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-        SA_CUDA(cudaFuncSetAttribute(sa::csa_select_attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        SA_CUDA(cudaFuncSetAttribute(sa::score_fast_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)smem));
+        SA_CUDA(cudaFuncSetAttribute(sa::score_fast_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)smem));
+        SA_CUDA(cudaFuncSetAttribute(sa::topk_bound_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     sa::kFbReserveSmem));
+        SA_CUDA(cudaFuncSetAttribute(sa::csa_select_fast_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      sa::kFaSmem));
-        // the bound kernel's CTAs share SMs with three scan CTAs each: every
-        // kernel of the path asks for the largest shared-memory carveout, so
-        // that no SM is configured too small for the scan while they overlap
-        SA_CUDA(cudaFuncSetAttribute(sa::topk_bound_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                     cudaSharedmemCarveoutMaxShared));
         SA_CUDA(cudaFuncSetAttribute(sa::topk_bound_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
-        SA_CUDA(cudaFuncSetAttribute(sa::score_fast_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                     cudaSharedmemCarveoutMaxShared));
-        SA_CUDA(cudaFuncSetAttribute(sa::csa_select_attend_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                     cudaSharedmemCarveoutMaxShared));
         attr_set(init);
     }
     CUtensorMap map;
@@ -709,22 +728,21 @@ sa_status run_fast_decode(const void* q, const void* q_idx, int H, const sa_cach
     if (r != SA_OK) return r;
     const bool pdl = pdl_on();
     stage_mark(SA_STAGE_INDEX_SCORE, 0, st);
-    SA_CUDA(launch_k(sa::topk_bound_kernel, dim3(sa::kFbCluster, B), dim3(sa::kFbThreads), 0, st, false,
-                     (unsigned)sa::kFbCluster, a));
+    // (the reserved shared memory is not used: it keeps the scan's CTAs off
+    // the bound kernel's SMs while both run)
+    SA_CUDA(launch_k(sa::topk_bound_kernel, dim3(sa::kFbCluster, B), dim3(sa::kFbThreads),
+                     late ? (size_t)sa::kFbReserveSmem : 0, st, false, (unsigned)sa::kFbCluster, a));
     SA_LAUNCHED();
-    SA_CUDA(launch_k(sa::score_fast_kernel, dim3(a.nchunks, B), dim3(sa::kScThreads), smem, st, pdl, 1u, map, a));
+    SA_CUDA(launch_k(late ? sa::score_fast_kernel<true> : sa::score_fast_kernel<false>, dim3(a.nchunks, B),
+                     dim3(sa::kScThreads), smem, st, pdl, 1u, map, a));
     SA_LAUNCHED();
     stage_mark(SA_STAGE_INDEX_SCORE, 1, st);
     r = between();
     if (r != SA_OK) return r;
-    // one kernel selects and attends: the selection stage's events bracket it
     stage_mark(SA_STAGE_TOPK_SELECT, 0, st);
-    SA_CUDA(launch_k(sa::csa_select_attend_kernel, dim3(sa::kFaCluster, B), dim3(sa::kFaThreads), sa::kFaSmem, st,
-                     pdl, (unsigned)sa::kFaCluster, a));
+    SA_CUDA(launch_k(sa::csa_select_fast_kernel, dim3(B), dim3(sa::kFaThreads), sa::kFaSmem, st, pdl, 1u, a));
     SA_LAUNCHED();
     stage_mark(SA_STAGE_TOPK_SELECT, 1, st);
-    stage_mark(SA_STAGE_CSA_ATTN, 0, st);
-    stage_mark(SA_STAGE_CSA_ATTN, 1, st);
     return SA_OK;
 }
 
@@ -1422,6 +1440,7 @@ static sa_status hybrid_decode_impl(const char* what, const void* q, const void*
     r = side_stream(&side);
     if (r != SA_OK) return r;
     auto fork_hca = [&]() -> sa_status {
+        PriorityScope normal(0);  // the HCA branch keeps the default priority
         SA_CUDA(cudaEventRecord(side->fork, st));
         SA_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
         stage_mark(SA_STAGE_HCA_ATTN, 0, side->s);
@@ -1436,13 +1455,11 @@ static sa_status hybrid_decode_impl(const char* what, const void* q, const void*
         SA_CUDA(cudaEventRecord(side->join, side->s));
         return SA_OK;
     };
-    if (!fp4 && fast_decode_ok(csa, H, k)) {
-        r = run_fast_decode(q, q_idx, H, csa, k, scale, out_csa, lse_csa, idx, cnt, ws, w, st, fork_hca);
-        if (r != SA_OK) return r;
-        SA_CUDA(cudaStreamWaitEvent(st, side->join, 0));
-        return SA_OK;
-    }
-    r = run_topk_decode(q_idx, csa, k, idx, cnt, ws, w, st, fork_hca, codes4, scales4);
+    PriorityScope high(highest_priority());
+    if (!fp4 && fast_decode_ok(csa, H, k))
+        r = run_fast_topk(q_idx, csa, k, idx, cnt, ws, w, st, fork_hca);
+    else
+        r = run_topk_decode(q_idx, csa, k, idx, cnt, ws, w, st, fork_hca, codes4, scales4);
     if (r != SA_OK) return r;
     stage_mark(SA_STAGE_CSA_ATTN, 0, st);
     r = run_attn(q, 1, H, csa, true, idx, cnt, k, nullptr, scale, out_csa, lse_csa, ws, w.total, st, true);

@@ -28,7 +28,7 @@ from ._lib import check, lib
 
 KERNELS = {1: "score", 2: "filter", 3: "resolve", 4: "emit", 5: "attn_split", 6: "attn_merge", 7: "score_fp4",
            8: "prefill_score", 9: "prefill_select", 10: "prefill_score_fp4", 11: "prefill_select2", 12: "bound",
-           13: "select_attend"}
+           13: "select_fast"}
 PHASES = {
     "score": ["start", "scan done", "threshold found"],
     "score_fp4": ["start", "scan done", "threshold found"],
@@ -44,10 +44,10 @@ PHASES = {
     "prefill_select": ["start", "keys staged", "digit 1", "digit 2", "digit 3", "ties", "end"],
     "prefill_select2": ["start", "keys staged", "digit 1", "digit 2", "digit 3", "counted", "end"],
     # the fast decode path: the sampled bound (CTA 0 of each cluster finds it)
-    # and the selection + attention cluster (CTA 0 selects: phases 1-4)
+    # and the selection (one CTA per sequence; "band rescored" only when the
+    # band is not inside the staged bins)
     "bound": ["start", "sampled", "bound found"],
-    "select_attend": ["start", "list loaded", "t~ known", "band rescored", "cut done", "selected", "gathered",
-                      "S done", "softmax done", "O done", "partial stored", "merged"],
+    "select_fast": ["start", "list loaded", "t~ known", "band rescored", "cut done", "selected"],
 }
 RECORD = np.dtype([("t", "<u8"), ("kernel", "<u2"), ("phase", "<u2"), ("sm", "<u2"), ("cta", "<u2")])
 

@@ -285,17 +285,17 @@ def test_options_on_the_host(L):
             S.set_option(S.SA_OPT_PREFILL_SELECT, 0)
     finally:
         S.set_option(S.SA_OPT_PREFILL_SELECT, 1)
-    assert L.sa_get_option(_lib.SA_OPT_DECODE_FAST, ctypes.byref(v)) == _lib.SA_OK and v.value == 1  # default
+    assert L.sa_get_option(_lib.SA_OPT_DECODE_FAST, ctypes.byref(v)) == _lib.SA_OK and v.value == 0  # default
     try:
-        for val in (0, 2, 1):
+        for val in (1, 2, 0):
             S.set_option(S.SA_OPT_DECODE_FAST, val)
             assert S.get_option(S.SA_OPT_DECODE_FAST) == val
         assert L.sa_set_option(_lib.SA_OPT_DECODE_FAST, 3) == _lib.SA_ERR_INVALID_ARG
         assert "SA_OPT_DECODE_FAST" in L.sa_last_error().decode()
         assert L.sa_set_option(_lib.SA_OPT_DECODE_FAST, -1) == _lib.SA_ERR_INVALID_ARG
-        assert S.get_option(S.SA_OPT_DECODE_FAST) == 1
+        assert S.get_option(S.SA_OPT_DECODE_FAST) == 0
     finally:
-        S.set_option(S.SA_OPT_DECODE_FAST, 1)
+        S.set_option(S.SA_OPT_DECODE_FAST, 0)
 
 
 def test_trace_calls_need_the_profiling_build(L):

@@ -1,12 +1,11 @@
 """The fast hybrid decode path (SA_OPT_DECODE_FAST) against the fp64 oracle.
 
-The CSA branch of hybrid_attn_decode runs three kernels on this path: a
-sampled bound on the k-th score, the indexer scan keeping the entries above
-it as candidates, and one 8-CTA cluster per sequence selecting exactly from
-them and attending over the selection on the tensor cores.  Mode 1 is the
-default; mode 2 forces the selection over every score (the fallback the
-kernel takes when the candidates cannot prove the selection); mode 0 is the
-general path.  Indices and counts: bit-exact against the oracle in every
+The indexer and top-k of hybrid_attn_decode run three kernels on this path:
+a sampled bound on the k-th score, the indexer scan keeping the entries
+above it as candidates, and one CTA per sequence selecting exactly from them.
+Mode 0 (the default) is the general path; mode 1 the fast path; mode 2 the
+fast path with the selection forced over every score (the fallback the kernel
+takes when the candidates cannot prove the selection).  Indices and counts: bit-exact against the oracle in every
 mode.  Outputs: max-abs <= 1e-2 and rms(err)/rms(oracle) <= 1e-2 (bf16
 cache), lse within 1e-3.  Cases cover the sampling regime (more than 8192
 entries), k up to 2048, fewer than k entries, empty and 1-entry sequences,
@@ -21,7 +20,8 @@ import pytest
 import torch
 
 from oracle import oracle as O
-from tests._util import SCALE, TOL_BF16, TOL_REL, Inputs, bf16_to_f64, compress_on_gpu, out_errors
+from tests._util import (SCALE, TOL_BF16, TOL_FP8, TOL_REL, TOL_REL_FP8, Inputs, bf16_to_f64, compress_on_gpu,
+                         out_errors)
 
 pytestmark = pytest.mark.gpu
 
@@ -34,14 +34,14 @@ def S():
         pytest.skip("no CUDA device")
     import sparse_attention_pool_b200 as S
     yield S
-    S.set_option(S.SA_OPT_DECODE_FAST, 1)
+    S.set_option(S.SA_OPT_DECODE_FAST, 0)
 
 
-def _run(S, inp, k, mode, H=None):
+def _run(S, inp, k, mode, H=None, fp8=False):
     B, Lcap = inp.B, inp.Lcap
     H = inp.H if H is None else H
     g = inp.to_device()
-    csa, hca = compress_on_gpu(S, g, B, Lcap)
+    csa, hca = compress_on_gpu(S, g, B, Lcap, fp8=fp8)
     ws = S.alloc_workspace(S.workspace_size(S.SA_OP_HYBRID_DECODE, B, 1, H, csa.Ncap, hca.Ncap, k))
     idx = torch.empty(B, k, dtype=torch.int32, device="cuda")
     cnt = torch.empty(B, dtype=torch.int32, device="cuda")
@@ -53,22 +53,23 @@ def _run(S, inp, k, mode, H=None):
                                       idx_out=idx, cnt_out=cnt)
         S.read_device_status()
     finally:
-        S.set_option(S.SA_OPT_DECODE_FAST, 1)
+        S.set_option(S.SA_OPT_DECODE_FAST, 0)
     return oc, oh, lc, lh, idx, cnt
 
 
-def _check(S, inp, k, mode, outputs=True):
-    oc, oh, lc, lh, idx, cnt = _run(S, inp, k, mode)
+def _check(S, inp, k, mode, outputs=True, fp8=False):
+    oc, oh, lc, lh, idx, cnt = _run(S, inp, k, mode, fp8=fp8)
+    tol, trel = (TOL_FP8, TOL_REL_FP8) if fp8 else (TOL_BF16, TOL_REL)
     for b in range(inp.B):
         L = int(inp.lengths[b])
-        r = O.hybrid_query(inp.oracle_seq(b), inp.q[b], inp.qI[b], t=L, k=k, scale=SCALE)
+        r = O.hybrid_query(inp.oracle_seq(b, fp8=fp8), inp.q[b], inp.qI[b], t=L, k=k, scale=SCALE)
         assert cnt[b].item() == r["cnt"], b
         assert np.array_equal(idx[b].cpu().numpy(), r["idx"]), b
         if not outputs:
             continue
         for got, ref in ((oc[b], r["out_csa"]), (oh[b], r["out_hca"])):
             mx, rel = out_errors(got, ref)
-            assert mx <= TOL_BF16 and rel <= TOL_REL, (b, mx, rel)
+            assert mx <= tol and rel <= trel, (b, mx, rel)
         if r["cnt"] > 0:
             assert np.abs(lc[b].cpu().numpy() - r["lse_csa"]).max() < 1e-3, b
         else:
@@ -88,6 +89,13 @@ def _check(S, inp, k, mode, outputs=True):
 def test_fast_decode_vs_oracle(S, mode, B, Lcap, H, k, lengths):
     inp = Inputs(4100 + Lcap % 997 + k, B, Lcap, H, lengths=lengths)
     _check(S, inp, k, mode)
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_fast_decode_fp8_ragged(S, mode):
+    # e4m3 cache with per-64-entry scales, ragged lengths (the fp8 workload's shape, smaller)
+    inp = Inputs(4151, 4, 50000, 64, lengths=[50000, 33333, 41001, 16385])
+    _check(S, inp, 1024, mode, fp8=True)
 
 
 @pytest.mark.parametrize("mode", MODES)
@@ -160,15 +168,14 @@ def test_fast_decode_sample_defeated(S, mode):
 
 
 def test_fast_equals_general_path(S):
-    # the same selection on both paths; outputs agree to bf16 rounding
+    # the same selection on both paths, and the same attention kernels after
+    # it: every output agrees bit for bit
     B, Lcap, H, k = 3, 50000, 64, 1024
     inp = Inputs(4701, B, Lcap, H, lengths=[50000, 44443, 20001])
     a = _run(S, inp, k, 1)
     b = _run(S, inp, k, 0)
-    assert torch.equal(a[4], b[4]) and torch.equal(a[5], b[5])
-    for x, y in zip(a[:2], b[:2]):
-        assert (x.float() - y.float()).abs().max().item() <= 2e-3
-    assert (a[2] - b[2]).abs().max().item() < 1e-3
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
 
 
 def test_fast_decode_deterministic(S):

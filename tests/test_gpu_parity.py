@@ -204,18 +204,12 @@ def test_hybrid_decode_vs_oracle(S, B, Lcap, H, k, q_scale, fp8):
 
 
 def test_separate_calls_equal_hybrid(S):
-    # the general kernels (SA_OPT_DECODE_FAST = 0) are the ones the separate
-    # calls run, so their outputs agree bit for bit
     B, Lcap, H, k = 2, 12000, 64, 256
     inp = Inputs(501, B, Lcap, H)
     g = inp.to_device()
     csa, hca = compress_on_gpu(S, g, B, Lcap)
     ws = S.alloc_workspace(S.workspace_size(S.SA_OP_HYBRID_DECODE, B, 1, H, csa.Ncap, hca.Ncap, k))
-    S.set_option(S.SA_OPT_DECODE_FAST, 0)
-    try:
-        oc, oh = S.hybrid_attn_decode(g["q"], g["qI"], csa, hca, k, ws, scale=SCALE)
-    finally:
-        S.set_option(S.SA_OPT_DECODE_FAST, 1)
+    oc, oh = S.hybrid_attn_decode(g["q"], g["qI"], csa, hca, k, ws, scale=SCALE)
     ws2 = S.alloc_workspace(S.workspace_size(S.SA_OP_INDEX_TOPK, B, 1, H, csa.Ncap, 0, k))
     idx, cnt = S.csa_index_topk(g["qI"], csa, k, ws2)
     ws3 = S.alloc_workspace(S.workspace_size(S.SA_OP_SPARSE_ATTN, B, 1, H, csa.Ncap, 0, k))

@@ -1,6 +1,7 @@
 """The profiling build's device timeline: a traced decode step records, for
-every decode-path kernel, its phases in order, with one filter record per
-filter CTA; a traced prefill top-k records every query's selection CTA and
+every decode-path kernel, its phases in order (the general kernels: one
+filter record per filter CTA; the fast path: one bound and one selection
+record set per sequence); a traced prefill top-k records every query's selection CTA and
 its phases, and gives the untraced indices.  Runs in child processes (the
 library variant is chosen per process by SA_TRACE_LIB).
 """
@@ -30,23 +31,40 @@ inp = Inputs(981, B, L, H)
 g = inp.to_device()
 csa, hca = compress_on_gpu(S, g, B, L)
 ws = S.alloc_workspace(S.workspace_size(S.SA_OP_HYBRID_DECODE, B, 1, H, csa.Ncap, hca.Ncap, k))
-S.hybrid_attn_decode(g["q"], g["qI"], csa, hca, k, ws, scale=SCALE)   # warm-up, untraced
-torch.cuda.synchronize()
-buf = trace.install(1 << 15)
-S.hybrid_attn_decode(g["q"], g["qI"], csa, hca, k, ws, scale=SCALE)
-rec = trace.records(buf)
-trace.uninstall()
-S.read_device_status()
-print(trace.format_summary(rec))
-names = {trace.KERNELS[int(x)] for x in np.unique(rec["kernel"])}
+
+def traced_step():
+    S.hybrid_attn_decode(g["q"], g["qI"], csa, hca, k, ws, scale=SCALE)   # warm-up, untraced
+    torch.cuda.synchronize()
+    buf = trace.install(1 << 15)
+    S.hybrid_attn_decode(g["q"], g["qI"], csa, hca, k, ws, scale=SCALE)
+    rec = trace.records(buf)
+    trace.uninstall()
+    S.read_device_status()
+    print(trace.format_summary(rec))
+    return rec, {trace.KERNELS[int(x)] for x in np.unique(rec["kernel"])}
+
+def phases_in_order(rec, kid):
+    r = rec[rec["kernel"] == kid]
+    for cta in np.unique(r["cta"]):
+        ts = r[r["cta"] == cta]
+        order = np.argsort(ts["phase"], kind="stable")
+        assert (np.diff(ts["t"][order].astype(np.int64)) >= 0).all(), (kid, cta)
+
+# the general kernels
+S.set_option(S.SA_OPT_DECODE_FAST, 0)
+rec, names = traced_step()
 assert {"score", "filter", "resolve", "emit", "attn_split"} <= names, names
 nfch = -(-csa.Ncap // 2048)
 assert int(((rec["kernel"] == 2) & (rec["phase"] == 1)).sum()) == nfch * B
-res = rec[rec["kernel"] == 3]
-for cta in np.unique(res["cta"]):
-    ts = res[res["cta"] == cta]
-    order = np.argsort(ts["phase"], kind="stable")
-    assert (np.diff(ts["t"][order].astype(np.int64)) >= 0).all()
+phases_in_order(rec, 3)
+# the fast path: the bound (one "bound found" per sequence), the scan, one
+# selection CTA per sequence through its last phase, the attention
+S.set_option(S.SA_OPT_DECODE_FAST, 1)
+rec, names = traced_step()
+assert {"bound", "score", "select_fast", "attn_split"} <= names and "filter" not in names, names
+assert int(((rec["kernel"] == 12) & (rec["phase"] == 2)).sum()) == B
+assert int(((rec["kernel"] == 13) & (rec["phase"] == 5)).sum()) == B
+phases_in_order(rec, 13)
 print("TRACE_OK")
 """
 
