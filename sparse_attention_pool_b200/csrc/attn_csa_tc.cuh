@@ -1,0 +1,324 @@
+// attn_csa_tc.cuh -- the gathered (CSA) softmax attention of a causal
+// prefill on the 5th-generation tensor cores (tcgen05 + tensor memory),
+// "DeepSeek-V4 ... Review", section 3-2 (2) component table (CSA attends over
+// its sparse top-k of the compressed entries).
+//
+// Every query position has its own list of up to kmax entries, shared by its
+// 64 heads (one KV head).  A query's 64 heads fill only half of a 128-row
+// MMA, so the tiles are transposed: the MMA's 128 rows are list entries,
+//     S^T = K_sel Q^T    (M = 128 entries, N = 64 heads, K = 128 dims)
+//     O^T = V_sel^T P^T  (M = 128 dims,    N = 64 heads, K = 128 entries)
+// with every row of both MMAs used.  Per tile of 128 list entries: the K and
+// V rows are gathered by cp.async into the 128-byte-swizzled canonical
+// layout, S^T lands in tensor memory, the softmax runs per head over the
+// tile's entries (thread = entry, a butterfly exchange per warp gives each
+// lane one head's maximum and sum), P^T goes to shared memory in bf16, and
+// the tile's O^T is folded into registers (thread = dim) with the online
+// rescale of each head.  A persistent grid, two CTAs per SM, walks the
+// queries.  Completion of each MMA group goes through tcgen05.commit on an
+// mbarrier; every wait is bounded.
+#pragma once
+#include "attn_prefill_tc.cuh"
+
+namespace sa {
+
+constexpr int kCtThreads = 256;      // 8 warps
+constexpr int kCtRows = 128;         // list entries per tile
+constexpr int kCtQ = 0;              // Q: 64 heads x 128 dims, K-major SW128, halves 8 KB apart
+constexpr int kCtK = 16384;          // K tile: 128 x 128, K-major SW128, halves 16 KB apart
+constexpr int kCtV = kCtK + 32768;    // V tile (the MN-major A operand of O^T)
+constexpr int kCtP = kCtV + 32768;    // P^T: 128 entries x 64 heads bf16 (the MN-major B operand)
+constexpr int kCtSmem = kCtP + 16384 + 1024;  // + alignment slack
+constexpr uint32_t kCtCols = 128;     // tensor memory: S^T columns [0, 64), the tile's O^T [64, 128)
+
+struct CtArgs {
+    const uint16_t* q;   // [BQ][H][128], BQ = B * T
+    const uint16_t* K;   // [B][Ncap][128] bf16
+    const uint16_t* V;
+    const int32_t* n;    // [B]
+    const int32_t* idx;  // [BQ][kmax]
+    const int32_t* cnt;  // [BQ]
+    long long BQ;
+    int T, H, Ncap, kmax;
+    float scale_log2;    // softmax scale * log2(e)
+    uint16_t* out;       // [BQ][H][128]
+    float* lse;          // [BQ][H] or NULL
+};
+
+// 2^x on the special-function unit (subnormal results flush to zero: a
+// weight below 2^-126 of the row's largest does not change the sum)
+__device__ __forceinline__ float ex2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Transposed reduction of 32 values per lane over the warp's 32 lanes (max
+// or sum per value index): at each of the five butterfly steps a lane keeps
+// one half of its values and sends the other half to its partner, so that
+// lane l ends with the reduction of value index l.
+template <bool MAX>
+__device__ __forceinline__ float warp_transpose_reduce32(float (&v)[32], int lane) {
+#pragma unroll
+    for (int step = 0; step < 5; ++step) {
+        const int half = 16 >> step;
+        const bool upper = (lane & half) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+            const float keep = upper ? v[half + i] : v[i];
+            const float send = upper ? v[i] : v[half + i];
+            const float got = __shfl_xor_sync(0xFFFFFFFFu, send, half);
+            v[i] = MAX ? fmaxf(keep, got) : keep + got;
+        }
+    }
+    return v[0];
+}
+
+// Byte offset of (row r, 16-byte chunk c) in a K-major SW128 operand whose
+// two 64-element halves lie `half` bytes apart.
+__device__ __forceinline__ uint32_t sw128_off(int r, int c, uint32_t half) {
+    return (uint32_t)(c >> 3) * half + (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+// Instruction descriptor, kind::f16 with fp32 D and bf16 A / B: M = 128,
+// N = 64; a_mn / b_mn select MN-major operands.
+__device__ __forceinline__ uint32_t ct_idesc(uint32_t a_mn, uint32_t b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (a_mn << 15) | (b_mn << 16) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
+}
+
+struct CtStatic {
+    float red[8][32];  // per warp: one value per head of its half
+    float m[64];       // running max of scale*log2e*s per head
+    float l[64];       // running sum of 2^(. - m)
+    float alpha[64];   // this tile's rescale of the earlier sums
+    uint32_t tmem;
+    int bad;
+    uint64_t bar_s, bar_o;
+};
+
+// Persistent grid; CTA c takes queries c, c + gridDim.x, ...
+__global__ void __launch_bounds__(kCtThreads, 2) attn_csa_prefill_tc_kernel(CtArgs a) {
+    extern __shared__ uint8_t ct_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ct_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ CtStatic S;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int quarter = warp & 3, hh = warp >> 2;  // TMEM lane quarter; half of the heads
+    const uint32_t sQ = smem_u32(sm + kCtQ), sK = smem_u32(sm + kCtK), sV = smem_u32(sm + kCtV),
+                   sP = smem_u32(sm + kCtP);
+    pdl_wait();
+    pdl_release();
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&S.tmem)),
+                     "r"(kCtCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    if (tid == 0) {
+        mbar_init(&S.bar_s, 1);
+        mbar_init(&S.bar_o, 1);
+        fence_barrier_init();
+        S.bad = 0;
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem;
+    const uint32_t t_s = tmem, t_pv = tmem + 64;
+    const uint32_t lane_q = (uint32_t)(quarter * 32) << 16;
+    const uint32_t id_s = ct_idesc(0, 0), id_o = ct_idesc(1, 1);
+    uint32_t ph_s = 0, ph_o = 0;
+    int pend_s = 0, pend_o = 0;  // (thread 0) commits not yet seen complete
+
+    for (long long bq = blockIdx.x; bq < a.BQ; bq += gridDim.x) {
+        const int b = (int)(bq / a.T);
+        int nb = a.n[b];
+        if (nb < 0 || nb > a.Ncap) {
+            if (tid == 0) flag(DEV_LEN);
+            nb = nb < 0 ? 0 : a.Ncap;
+        }
+        int R = a.cnt[bq];
+        if (R < 0 || R > a.kmax) {
+            if (tid == 0) flag(DEV_LEN);
+            R = R < 0 ? 0 : a.kmax;
+        }
+        // Q: 64 rows of 16 chunks, rows at or past H zero
+        {
+            const int h = tid >> 2, c0 = (tid & 3) * 4;
+            const bool ok = h < a.H;
+            const uint16_t* src = a.q + ((size_t)bq * a.H + (ok ? h : 0)) * 128;
+#pragma unroll
+            for (int c = c0; c < c0 + 4; ++c) cp_async16_zfill(sm + kCtQ + sw128_off(h, c, 8192), src + c * 8, ok);
+        }
+        if (tid < 64) {
+            S.m[tid] = -INFINITY;
+            S.l[tid] = 0.f;
+        }
+        float o[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) o[j] = 0.f;
+        const int ntiles = (R + kCtRows - 1) / kCtRows;
+        const int32_t* lidx = a.idx + (size_t)bq * a.kmax;
+        const int r = tid & (kCtRows - 1);  // the tile row this thread gathers (K: tid < 128, V: the rest)
+        const bool isv = tid >= kCtRows;
+        int jn = ntiles > 0 && r < R ? (int)ld_cg_u32(lidx + r) : 0;  // the first tile's entry
+        for (int i = 0; i < ntiles; ++i) {
+            // gather this tile's K and V rows (zero past the list)
+            {
+                const int p = i * kCtRows + r;
+                bool ok = p < R;
+                int j = jn;
+                if (ok && (j < 0 || j >= nb)) {
+                    flag(DEV_INDEX);
+                    ok = false;
+                }
+                const uint16_t* src = (isv ? a.V : a.K) + ((size_t)b * a.Ncap + (ok ? j : 0)) * 128;
+                uint8_t* dst = sm + (isv ? kCtV : kCtK);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) cp_async16_zfill(dst + sw128_off(r, c, 16384), src + c * 8, ok);
+                cp_async_commit();
+                const int pn = (i + 1) * kCtRows + r;  // the next tile's entry, ahead of its use
+                jn = i + 1 < ntiles && pn < R ? (int)ld_cg_u32(lidx + pn) : 0;
+            }
+            cp_async_wait<0>();
+            fence_async_smem();
+            __syncthreads();
+            // S^T = K Q^T over 8 k-steps of 16 dims
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t ka = sK + (ks >> 2) * 16384 + (ks & 3) * 32;
+                    const uint32_t qb = sQ + (ks >> 2) * 8192 + (ks & 3) * 32;
+                    tc_mma(t_s, tc_desc(ka, 16, 1024), tc_desc(qb, 16, 1024), id_s, ks > 0);
+                }
+                tc_commit(&S.bar_s);
+                ++pend_s;
+            }
+            if (mbar_wait(&S.bar_s, ph_s)) {
+                if (tid == 0) --pend_s;
+            } else {
+                S.bad = 1;  // recorded in the status word; this CTA stops below
+            }
+            ph_s ^= 1;
+            tc_fence_after();
+            // softmax of the tile, per head: thread = entry (its 32 heads)
+            const int e = quarter * 32 + lane;
+            const bool valid = i * kCtRows + e < R;
+            float v[32];
+            auto load_s = [&]() {
+                uint32_t rr[32];
+                tc_ld32_nw(t_s + lane_q + 32 * hh, rr);
+                tc_wait_ld();
+#pragma unroll
+                for (int h = 0; h < 32; ++h) v[h] = valid ? __uint_as_float(rr[h]) * a.scale_log2 : -INFINITY;
+            };
+            load_s();
+            S.red[warp][lane] = warp_transpose_reduce32<true>(v, lane);  // head 32 * hh + lane
+            __syncthreads();
+            if (tid < 64) {  // head tid: the four quarters of its half
+                const int w0 = (tid >> 5) * 4;
+                float mt = S.red[w0][tid & 31];
+#pragma unroll
+                for (int q = 1; q < 4; ++q) mt = fmaxf(mt, S.red[w0 + q][tid & 31]);
+                const float mo = S.m[tid], mn = fmaxf(mo, mt);
+                S.alpha[tid] = mo == -INFINITY ? 0.f : ex2_ftz(mo - mn);  // earlier sums are 0 while m is -inf
+                S.m[tid] = mn;
+            }
+            __syncthreads();
+            load_s();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    const int h = c * 8 + w * 2;
+                    const float p0 = valid ? ex2_ftz(v[h] - S.m[32 * hh + h]) : 0.f;  // valid: m is finite
+                    const float p1 = valid ? ex2_ftz(v[h + 1] - S.m[32 * hh + h + 1]) : 0.f;
+                    v[h] = p0;
+                    v[h + 1] = p1;
+                    pk[w] = pack_bf16x2(p0, p1);
+                }
+                const int cc = 4 * hh + c;  // 16-byte chunk of the entry's 128-byte P^T row
+                *reinterpret_cast<uint4*>(sm + kCtP + (e >> 3) * 1024 + (e & 7) * 128 + ((cc ^ (e & 7)) << 4)) =
+                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+            const float ls = warp_transpose_reduce32<false>(v, lane);
+            __syncthreads();  // every read of the maxima in S.red is done
+            S.red[warp][lane] = ls;
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            if (tid < 64) {
+                const int w0 = (tid >> 5) * 4;
+                float sum = 0.f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) sum += S.red[w0 + q][tid & 31];
+                S.l[tid] = S.l[tid] * S.alpha[tid] + sum;
+            }
+            // O^T = V^T P^T over 8 k-steps of 16 entries
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    tc_mma(t_pv, tc_desc(sV + ks * 2048, 16384, 1024), tc_desc(sP + ks * 2048, 16384, 1024), id_o,
+                           ks > 0);
+                tc_commit(&S.bar_o);
+                ++pend_o;
+            }
+            if (mbar_wait(&S.bar_o, ph_o)) {
+                if (tid == 0) --pend_o;
+            } else {
+                S.bad = 1;
+            }
+            ph_o ^= 1;
+            tc_fence_after();
+            // fold the tile's O^T into the row of this thread's dim (its 32 heads)
+            {
+                uint32_t rr[32];
+                tc_ld32_nw(t_pv + lane_q + 32 * hh, rr);
+                tc_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) o[j] = fmaf(o[j], S.alpha[32 * hh + j], __uint_as_float(rr[j]));
+            }
+            tc_fence_before();
+            __syncthreads();  // K, V, P^T and tensor memory are free for the next tile
+            if (S.bad) break;
+        }
+        if (ntiles == 0) {
+            cp_async_wait<0>();  // the Q copies land before the next query's overwrite them
+            __syncthreads();
+        }
+        // this query's output: dim d of each of the thread's 32 heads, and the lse
+        {
+            const int d = quarter * 32 + lane;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int h = 32 * hh + j;
+                if (h < a.H) {
+                    const float L = S.l[h];
+                    const float inv = L > 0.f ? 1.f / L : 0.f;
+                    const __nv_bfloat16 y = __float2bfloat16_rn(o[j] * inv);
+                    a.out[((size_t)bq * a.H + h) * 128 + d] = *reinterpret_cast<const uint16_t*>(&y);
+                }
+            }
+            if (a.lse && tid < a.H && tid < 64) {
+                const float L = S.l[tid];
+                a.lse[(size_t)bq * a.H + tid] = L > 0.f ? (S.m[tid] + __log2f(L)) * 0.6931471805599453f : -INFINITY;
+            }
+        }
+        __syncthreads();  // S.m / S.l are reset by the next query
+        if (S.bad) break;
+    }
+    // an MMA still in flight after a timeout is waited for (bounded) before
+    // its tensor memory is released
+    if (tid == 0) {
+        if (pend_s > 0) mbar_wait(&S.bar_s, ph_s);
+        if (pend_o > 0) mbar_wait(&S.bar_o, ph_o);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCtCols));
+    }
+}
+
+}  // namespace sa

@@ -17,6 +17,7 @@
 
 #include "../../include/sparse_attn.h"
 #include "attn.cuh"
+#include "attn_csa_tc.cuh"
 #include "attn_prefill_tc.cuh"
 #include "compress.cuh"
 #include "cp_decode.cuh"
@@ -473,6 +474,38 @@ sa_status launch_prefill_tc(const sa::AttnArgs& aa, const sa_cache* c, bool gath
     return SA_OK;
 }
 
+// Causal prefill of the gathered (CSA) branch with at most 64 heads over a
+// bf16 cache: the transposed tensor-memory kernel, a persistent grid of two
+// CTAs per SM.
+sa_status launch_csa_prefill_tc(const sa::AttnArgs& aa, const sa_cache* c, long long BQ, cudaStream_t st) {
+    sa::CtArgs a{};
+    a.q = aa.q;
+    a.K = static_cast<const uint16_t*>(c->k);
+    a.V = static_cast<const uint16_t*>(c->v);
+    a.n = c->n;
+    a.idx = aa.idx;
+    a.cnt = aa.cnt;
+    a.BQ = BQ;
+    a.T = aa.Tq;
+    a.H = aa.H;
+    a.Ncap = c->Ncap;
+    a.kmax = aa.kmax;
+    a.scale_log2 = aa.scale_log2;
+    a.out = aa.out;
+    a.lse = aa.lse;
+    static std::atomic<uint64_t> init{0};
+    if (!attr_done(init)) {
+        SA_CUDA(cudaFuncSetAttribute(sa::attn_csa_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     sa::kCtSmem));
+        attr_set(init);
+    }
+    const long long grid = std::min<long long>(BQ, 2LL * num_sms());
+    if (grid < 1) return SA_OK;
+    sa::attn_csa_prefill_tc_kernel<<<(unsigned)grid, sa::kCtThreads, sa::kCtSmem, st>>>(a);
+    SA_LAUNCHED();
+    return SA_OK;
+}
+
 // The merge follows its split kernel on the same stream: always chained.
 sa_status launch_combine(const float* po, const float* pl, int splits, int H, long long BQ, uint16_t* out, float* lse,
                          cudaStream_t st) {
@@ -547,6 +580,8 @@ sa_status run_attn(const void* q, int Tq, int H, const sa_cache* c, bool gather,
     // the 128K-token, 64-head, k = 2048 prefill it took 110-135 ms against
     // 61 ms for the mma.sync kernel
     if (prefill && !gather && win == 0 && H == 64 && c->dtype == SA_BF16 && pos) return launch_prefill_tc(a, c, false, st);
+    // the gathered lists of a prefill (one per query) on the transposed tensor-memory kernel
+    if (prefill && gather && H <= 64 && c->dtype == SA_BF16) return launch_csa_prefill_tc(a, c, BQ, st);
     const int kv = c->dtype == SA_KV_MIXED ? 2 : c->dtype == SA_FP8_E4M3 ? 1 : 0;
     sa_status r = launch_attn(a, gather, kv, BQ, st, chained && pdl_on(), !prefill);
     if (r != SA_OK) return r;

@@ -296,7 +296,8 @@ def test_prefill_vs_oracle_every_row(S, fp8):
 def test_prefill_tensor_core_path_vs_oracle_every_row(S, T, k):
     """64 heads over a bf16 cache: the HCA branch runs on the tcgen05 prefill
     kernel (two query positions per CTA; an odd T leaves one alone), the CSA
-    branch on the mma.sync kernel (k not a multiple of its 64-entry tile)."""
+    branch on the transposed tcgen05 kernel (k not a multiple of its
+    128-entry tile)."""
     B, H = 2, 64
     inp = Inputs(611 + T, B, T, H, Tq=T)
     g = inp.to_device()
