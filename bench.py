@@ -979,7 +979,7 @@ def main():
     ap.add_argument("--decode-fast", type=int, default=0, choices=[0, 1],
                     help="decode only: the indexer + top-k kernels (SA_OPT_DECODE_FAST: 0 the general ones, "
                          "1 the sampled-bound fast path; same indices and outputs)")
-    ap.add_argument("--prefill-select", type=int, default=1, choices=[1, 2, 3],
+    ap.add_argument("--prefill-select", type=int, default=4, choices=[1, 2, 3, 4],
                     help="prefill only: the top-k selection kernel (SA_OPT_PREFILL_SELECT; same indices)")
     ap.add_argument("--trace", default="",
                     help="profiling: load the profiling build of the library and write the per-CTA timeline of "
@@ -993,7 +993,7 @@ def main():
         ap.error("--indexer, --kv and --cp apply to decode workloads")
     if args.cp and (args.indexer != "bf16" or args.kv != "workload" or args.impl != "ours"):
         ap.error("--cp runs the workload's own storage and indexer on our arm")
-    if args.prefill_select != 1 and (w.mode != "prefill" or args.impl != "ours"):
+    if args.prefill_select != 4 and (w.mode != "prefill" or args.impl != "ours"):
         ap.error("--prefill-select applies to prefill workloads on our arm")
     if args.tokens:
         if w.mode != "prefill":

@@ -450,9 +450,9 @@ uint64_t sa_launch_count(void);
  * work, callable without a GPU.
  *   SA_OPT_PREFILL_SELECT  the selection kernel of the causal prefill top-k
  *     (csa_index_topk / csa_index_topk_mxfp4 with Tq > 1, and the hybrid
- *     prefill calls).  Both give the same indices, the exact top-k of
+ *     prefill calls).  Every form gives the same indices, the exact top-k of
  *     section 3-2 (4) of the review with the lowest-index tie-break:
- *       1 (default)  one 1024-thread CTA per query: three radix-digit
+ *       1            one 1024-thread CTA per query: three radix-digit
  *                    passes over the query's keys, a tie pass and an
  *                    ordered block-scan compaction;
  *       2            the first digit over the keys, the second and third
@@ -461,7 +461,13 @@ uint64_t sa_launch_count(void);
  *                    output with the ties taken in the same pass;
  *       3            form 2 in 512-thread CTAs that read the keys from the
  *                    scratch on every pass instead of staging them, so
- *                    that three queries share an SM.
+ *                    that three queries share an SM;
+ *       4 (default)  one 1024-thread CTA per query: the scores' mean and
+ *                    deviation, one pass over 256 linear score bins counted
+ *                    in per-warp histograms, the threshold ranked inside
+ *                    its bin, then one counting pass and an ordered output
+ *                    by contiguous runs (28 ms of selection became 12 ms on
+ *                    the 128K-token prefill with k = 2048).
  *   SA_OPT_DECODE_FAST  the indexer and top-k of the hybrid decode calls
  *     (hybrid_attn_decode, hybrid_attn_decode_swa) with bf16 indexer keys
  *     and k <= 2048.  Every value gives the same indices (the exact top-k)

@@ -435,7 +435,7 @@ def hybrid_attn_prefill(q, q_idx, csa: Cache, hca: Cache, k: int, ws, idx_out, c
 
 def set_option(option: int, value: int):
     """A process-wide library option (host-only; applies to calls made
-    afterwards).  SA_OPT_PREFILL_SELECT: 1, 2 or 3, the prefill top-k's
+    afterwards).  SA_OPT_PREFILL_SELECT: 1 to 4 (default 4), the prefill top-k's
     selection kernel (the same indices in every form)."""
     check("sa_set_option", lib().sa_set_option(int(option), int(value)))
 

@@ -34,7 +34,7 @@ __device__ __forceinline__ void flag(uint32_t f) { atomicOr(&g_status, f); }
 // whole CTA.
 enum : uint32_t {
     TR_SCORE = 1, TR_FILTER = 2, TR_RESOLVE = 3, TR_EMIT = 4, TR_ATTN = 5, TR_COMBINE = 6, TR_SCORE_FP4 = 7,
-    TR_PSCORE = 8, TR_PSELECT = 9, TR_PSCORE_FP4 = 10, TR_PSELECT2 = 11, TR_BOUND = 12, TR_FAST = 13,
+    TR_PSCORE = 8, TR_PSELECT = 9, TR_PSCORE_FP4 = 10, TR_PSELECT2 = 11, TR_BOUND = 12, TR_FAST = 13, TR_PSELECT4 = 14,
 };
 #ifdef SA_TRACE
 struct TraceRec {

@@ -26,13 +26,14 @@
 #include "sa_common.cuh"
 #include "topk_decode.cuh"
 #include "topk_prefill.cuh"
+#include "topk_prefill_fast.cuh"
 
 namespace {
 
 thread_local char g_err[512] = "";
 thread_local uint64_t g_launches = 0;
 thread_local cudaEvent_t g_stage_ev[SA_NUM_STAGES][2] = {};
-std::atomic<int> g_prefill_select{1};  // SA_OPT_PREFILL_SELECT
+std::atomic<int> g_prefill_select{4};  // SA_OPT_PREFILL_SELECT
 std::atomic<int> g_decode_fast{0};      // SA_OPT_DECODE_FAST
 
 // Inside a stream capture the record must become a graph node of its own
@@ -475,8 +476,8 @@ sa_status launch_prefill_tc(const sa::AttnArgs& aa, const sa_cache* c, bool gath
 }
 
 // Causal prefill of the gathered (CSA) branch with at most 64 heads over a
-// bf16 cache: the transposed tensor-memory kernel, a persistent grid of two
-// CTAs per SM.
+// bf16 cache: the transposed tensor-memory kernel, a persistent grid of one
+// CTA per SM.
 sa_status launch_csa_prefill_tc(const sa::AttnArgs& aa, const sa_cache* c, long long BQ, cudaStream_t st) {
     sa::CtArgs a{};
     a.q = aa.q;
@@ -499,7 +500,7 @@ sa_status launch_csa_prefill_tc(const sa::AttnArgs& aa, const sa_cache* c, long 
                                      sa::kCtSmem));
         attr_set(init);
     }
-    const long long grid = std::min<long long>(BQ, 2LL * num_sms());
+    const long long grid = std::min<long long>(BQ, (long long)num_sms());
     if (grid < 1) return SA_OK;
     sa::attn_csa_prefill_tc_kernel<<<(unsigned)grid, sa::kCtThreads, sa::kCtSmem, st>>>(a);
     SA_LAUNCHED();
@@ -838,6 +839,8 @@ sa_status run_topk_prefill(const void* q_idx, int Tq, const int32_t* pos, const 
                                      sa::kPselSmemKeys * 4));
         SA_CUDA(cudaFuncSetAttribute(sa::select_prefill_v2_kernel<sa::kPselThreads, true>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sa::kPsel2Smem));
+        SA_CUDA(cudaFuncSetAttribute(sa::select_prefill_v4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)sa::kP4Smem));
         attr_set(init);
     }
     const int etiles = std::max(1, cdiv(c->Ncap, sa::kPsE));
@@ -855,7 +858,9 @@ sa_status run_topk_prefill(const void* q_idx, int Tq, const int32_t* pos, const 
                 sa::score_prefill_kernel<<<dim3(etiles, cdiv(a.qb, sa::kPsQ)), sa::kPsThreads, sa::kPsSmem, st>>>(a);
                 SA_LAUNCHED();
             }
-            if (select_form == 2)
+            if (select_form == 4)
+                sa::select_prefill_v4_kernel<<<a.qb, sa::kP4Threads, sa::kP4Smem, st>>>(a);
+            else if (select_form == 2)
                 sa::select_prefill_v2_kernel<sa::kPselThreads, true><<<a.qb, sa::kPselThreads, sa::kPsel2Smem, st>>>(a);
             else if (select_form == 3)
                 sa::select_prefill_v2_kernel<sa::kPsel3Threads, false>
@@ -922,7 +927,7 @@ uint64_t sa_launch_count(void) { return g_launches; }
 sa_status sa_set_option(int32_t option, int64_t value) {
     switch (option) {
         case SA_OPT_PREFILL_SELECT:
-            SA_CHECK(value >= 1 && value <= 3, "sa_set_option: SA_OPT_PREFILL_SELECT=%lld (1, 2 or 3)",
+            SA_CHECK(value >= 1 && value <= 4, "sa_set_option: SA_OPT_PREFILL_SELECT=%lld (1 to 4)",
                      (long long)value);
             g_prefill_select.store((int)value);
             return SA_OK;

@@ -271,11 +271,11 @@ def test_selftest_rejects_bad_arguments(L):
 def test_options_on_the_host(L):
     import sparse_attention_pool_b200 as S
     v = ctypes.c_int64(-1)
-    assert L.sa_get_option(_lib.SA_OPT_PREFILL_SELECT, ctypes.byref(v)) == _lib.SA_OK and v.value == 1  # default
+    assert L.sa_get_option(_lib.SA_OPT_PREFILL_SELECT, ctypes.byref(v)) == _lib.SA_OK and v.value == 4  # default
     try:
         S.set_option(S.SA_OPT_PREFILL_SELECT, 2)
         assert S.get_option(S.SA_OPT_PREFILL_SELECT) == 2
-        assert L.sa_set_option(_lib.SA_OPT_PREFILL_SELECT, 4) == _lib.SA_ERR_INVALID_ARG
+        assert L.sa_set_option(_lib.SA_OPT_PREFILL_SELECT, 5) == _lib.SA_ERR_INVALID_ARG
         assert "SA_OPT_PREFILL_SELECT" in L.sa_last_error().decode()
         assert S.get_option(S.SA_OPT_PREFILL_SELECT) == 2  # a refused value changes nothing
         assert L.sa_set_option(99, 1) == _lib.SA_ERR_INVALID_ARG
@@ -284,7 +284,7 @@ def test_options_on_the_host(L):
         with pytest.raises(S.SparseAttnError):
             S.set_option(S.SA_OPT_PREFILL_SELECT, 0)
     finally:
-        S.set_option(S.SA_OPT_PREFILL_SELECT, 1)
+        S.set_option(S.SA_OPT_PREFILL_SELECT, 4)
     assert L.sa_get_option(_lib.SA_OPT_DECODE_FAST, ctypes.byref(v)) == _lib.SA_OK and v.value == 0  # default
     try:
         for val in (1, 2, 0):

@@ -1,5 +1,5 @@
-"""The second and third forms of the prefill selection
-(SA_OPT_PREFILL_SELECT = 2, 3) against the oracle and against the first form: the exact top-k of every
+"""The second, third and fourth forms of the prefill selection
+(SA_OPT_PREFILL_SELECT = 2, 3, 4) against the oracle and against the first form: the exact top-k of every
 query row, ties at the threshold by lowest index, ascending output.  Cases:
 every row of a short prefill; equal scores (one crowded bin, larger than
 the in-shared-memory list, and ties at the threshold); rows that see more
@@ -31,11 +31,11 @@ def S():
 
 
 def _topk_forms(S, qI, csa, k, pos, fp4=None):
-    """(idx, cnt) under the first, second and third selection forms."""
+    """(idx, cnt) under every selection form (1 to 4)."""
     Tq = qI.shape[1]
     ws = S.alloc_workspace(S.workspace_size(S.SA_OP_INDEX_TOPK, csa.B, Tq, 8, csa.Ncap, 0, k))
     out = []
-    for form in (1, 2, 3):
+    for form in (1, 2, 3, 4):
         S.set_option(S.SA_OPT_PREFILL_SELECT, form)
         try:
             if fp4 is None:
@@ -44,7 +44,7 @@ def _topk_forms(S, qI, csa, k, pos, fp4=None):
                 i, c = S.csa_index_topk_mxfp4(qI, csa, fp4[0], fp4[1], k, ws, q_pos=pos)
             S.read_device_status()
         finally:
-            S.set_option(S.SA_OPT_PREFILL_SELECT, 1)
+            S.set_option(S.SA_OPT_PREFILL_SELECT, 4)
         out.append((i.clone(), c.clone()))
     return out
 
@@ -120,7 +120,7 @@ def test_hybrid_prefill_identical_under_both_forms(S):
     csa, hca = compress_on_gpu(S, g, B, T)
     ws = S.alloc_workspace(S.workspace_size(S.SA_OP_HYBRID_PREFILL, B, T, H, csa.Ncap, hca.Ncap, k))
     res = []
-    for form in (1, 2, 3):
+    for form in (1, 2, 3, 4):
         idx = torch.empty(B, T, k, dtype=torch.int32, device="cuda")
         cnt = torch.empty(B, T, dtype=torch.int32, device="cuda")
         S.set_option(S.SA_OPT_PREFILL_SELECT, form)
@@ -128,7 +128,7 @@ def test_hybrid_prefill_identical_under_both_forms(S):
             oc, oh = S.hybrid_attn_prefill(g["q"], g["qI"], csa, hca, k, ws, idx, cnt, scale=SCALE)
             S.read_device_status()
         finally:
-            S.set_option(S.SA_OPT_PREFILL_SELECT, 1)
+            S.set_option(S.SA_OPT_PREFILL_SELECT, 4)
         res.append((oc, oh, idx, cnt))
     for other in res[1:]:
         for a, b in zip(res[0], other):
