@@ -51,6 +51,17 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def measured_tensor_peak():
+    """Dense bf16 tensor peak for kernels timed inside a long step (TFLOP/s)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if d.get("bf16_tflops_sustained"):
+            return float(d["bf16_tflops_sustained"]), "measured (sustained)"
+    return 1400.0, "fallback (sustained)"
+
+
 def kernel_source_hash(kernel):
     """Hash of the named kernel's own source (its __global__ function) and of the
     shared device helpers: recorded ncu counters stay valid until these change."""
@@ -105,6 +116,7 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
+        self._summary = None
         self.path = f"/tmp/sa_clocks_{os.getpid()}.csv"
 
     def __enter__(self):
@@ -145,6 +157,9 @@ class ClockSampler:
                 self.proc.wait()
 
     def summary(self):
+        """The samples' median SM clock and the throttle reasons seen (read once)."""
+        if self._summary is not None:
+            return self._summary
         if not self.proc or not os.path.exists(self.path):
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         sm, smax, reasons = [], None, set()
@@ -163,8 +178,9 @@ class ClockSampler:
                     if v.lower() == "active":
                         reasons.add(n)
         os.unlink(self.path)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        self._summary = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                         "reasons": sorted(reasons), "samples": len(sm)}
+        return self._summary
 
 
 def decode_bytes(w, lengths, indexer="bf16", kv="workload"):
@@ -431,6 +447,17 @@ def run_ours(args, w, rank, world, dev):
             graph_score.replay()
             stage_ev[0][1].synchronize()
             score_ms.append(stage_ev[0][0].elapsed_time(stage_ev[0][1]))
+        # the same kernel between the same two events in eager calls: queued
+        # behind the flush (far longer than the host's submission), so the
+        # events bracket the kernel alone, without a graph's event nodes
+        L.sa_set_stage_events(0, stage_ev[0][0].cuda_event, stage_ev[0][1].cuda_event)
+        score_eager_ms = []
+        for i in range(args.steps):
+            flush_l2()
+            step()
+            stage_ev[0][1].synchronize()
+            score_eager_ms.append(stage_ev[0][0].elapsed_time(stage_ev[0][1]))
+        L.sa_set_stage_events(0, None, None)
         clk.keep_busy(lambda: (flush_l2(), graph.replay()), min_samples=2)
     torch.cuda.synchronize()
     S.read_device_status()
@@ -447,21 +474,32 @@ def run_ours(args, w, rank, world, dev):
     qi_dev = torch.empty(B, 64, dtype=torch.int16, device=dev)
     h2d = q_pin.numel() * 2 + qi_pin.numel() * 2
     d2h = oc_pin.numel() * 2 * 2 + lc_pin.numel() * 4 * 2
-    # the public API a serving loop uses: the step captured once (CapturedDecode),
-    # queries copied in and outputs out every step; checked bit for bit against
-    # the eager call first, else the eager call is timed instead
+    # the public API a serving loop uses: the step captured once by the library
+    # together with its packed host copies (DecodeGraph: one H2D copy of the
+    # queries, the outputs and lse copied back inside the graph, one launch per
+    # step); checked bit for bit against the eager call first, else the eager
+    # call with separate copies is timed instead
     api_name = "hybrid_attn_decode_mxfp4" if fp4 else "hybrid_attn_decode"
     e2e_api = f"{api_name} (eager) + pinned-host copies"
     cap = None
     try:
-        cap = S.CapturedDecode(csa, hca, k, H, scale=SCALE, codes=codes4, scales=scales4)
-        cap.step(q, qI)
+        cap = S.DecodeGraph(csa, hca, k, H, scale=SCALE, codes=codes4, scales=scales4, flags=args.e2e_io)
+        cap.q.view(torch.int16).copy_(q_pin)
+        cap.q_idx.view(torch.int16).copy_(qi_pin)
+        cap.step()
         decode(q, qI)
         torch.cuda.synchronize()
-        if not (torch.equal(cap.out_csa, out_c) and torch.equal(cap.out_hca, out_h) and torch.equal(cap.idx, idx)
-                and torch.equal(cap.lse_csa, lse_c) and torch.equal(cap.lse_hca, lse_h)):
+        if not (torch.equal(cap.out_csa.view(torch.int16), out_c.view(torch.int16).cpu())
+                and torch.equal(cap.out_hca.view(torch.int16), out_h.view(torch.int16).cpu())
+                and torch.equal(cap.idx, idx) and torch.equal(cap.lse_csa, lse_c.cpu())
+                and torch.equal(cap.lse_hca, lse_h.cpu())):
             raise RuntimeError("the captured step differs from the eager call")
-        e2e_api = f"CapturedDecode (CUDA graph of {api_name}) + pinned-host copies"
+        h2d, d2h = cap.h2d_bytes, cap.d2h_bytes
+        io_in = "a kernel reading the mapped pinned queries" if cap.flags & 1 else "one packed H2D copy"
+        io_out = ("the kernels writing outputs + lse into mapped pinned memory" if cap.flags & 2
+                  else "the outputs + lse copied back by the copy engine")
+        e2e_api = (f"sa_decode_graph_step (C ABI: {api_name} captured with {io_in} and {io_out}, "
+                   f"all inside the graph; one launch per step; flags {cap.flags})")
     except Exception as ex:  # noqa: BLE001 -- recorded in the JSON line
         cap = None
         e2e_api += f"; captured step not used: {str(ex)[:120]}"
@@ -472,7 +510,7 @@ def run_ours(args, w, rank, world, dev):
         flush_l2()
         ev0[i].record(stream)
         if cap is not None:
-            cap.step(q_pin, qi_pin, oc_pin, oh_pin, lc_pin, lh_pin)
+            cap.step(stream)
         else:
             q_dev.copy_(q_pin, non_blocking=True)
             qi_dev.copy_(qi_pin, non_blocking=True)
@@ -491,7 +529,8 @@ def run_ours(args, w, rank, world, dev):
     value = job_throughput(B * args.steps, world, total_ms)
     step_bytes, score_bytes = decode_bytes(w, lengths, args.indexer, args.kv)
     peak, peak_kind = measured_peaks()
-    score_avg = statistics.mean(score_ms)
+    score_avg = statistics.mean(score_eager_ms)
+    score_avg_graph = statistics.mean(score_ms)
     achieved = score_bytes / (score_avg / 1e3) / 1e9
     step_gbs = step_bytes / (total_ms / args.steps / 1e3) / 1e9
     result = {
@@ -521,6 +560,9 @@ def run_ours(args, w, rank, world, dev):
                      "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                      "bytes_per_launch": score_bytes, "avg_launch_ms": score_avg,
+                     "timing": "CUDA events on the launching stream around the kernel in eager calls queued "
+                               "behind the L2 flush",
+                     "avg_launch_ms_graph_events": score_avg_graph,
                      "traffic": None if fp4 else recorded_traffic("score_decode_kernel", w.name)},
         "stages_ms": {n: statistics.mean(v) for n, v in zip(stage_names, stage_ms)},
         "compress": compress_info,
@@ -959,6 +1001,44 @@ def run_reference(args, w, rank, world):
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+EXTRA_DECODE = ["decode_b1_t4k_h8_k64", "decode_b16_t64k_h64_k512", "ragged_fp8_b32_t64k-256k_h64_k1024"]
+EXTRA_PREFILL = "prefill_b1_t128k_h64_k2048"
+
+
+def run_extras(args, dev):
+    """The other workloads, each briefly (10 timed steps, 3 warm-up; the
+    prefill 3 and 3), on the same GPU after the headline: their own step
+    times, throughputs and stage times for the same JSON line."""
+    sub = argparse.Namespace(**vars(args))
+    sub.steps, sub.warmup, sub.no_cpu_baseline, sub.trace = 10, 3, True, ""
+    out = {}
+    for name in EXTRA_DECODE:
+        try:
+            r = run_ours(sub, configs.BY_NAME[name], 0, 1, dev)
+            out[name] = {"ms_per_step": r["ms_per_step"], "value": r["value"], "unit": r["unit"],
+                         "steps": sub.steps, "warmup": sub.warmup, "dtype": r["dtype"],
+                         "hbm_step_frac": r["hbm"]["step_frac"], "step_bytes": r["hbm"]["step_bytes"],
+                         "score_frac": r["roofline"]["frac"], "stages_ms": r["stages_ms"],
+                         "e2e": r["e2e"]["value"], "sm_mhz": r["clocks"].get("sm_mhz"),
+                         "reasons": r["clocks"].get("reasons")}
+        except Exception as ex:  # noqa: BLE001 -- recorded in the JSON line
+            out[name] = {"error": str(ex)[:200]}
+    sub.steps = 3
+    try:
+        r = run_prefill(sub, configs.BY_NAME[EXTRA_PREFILL], 0, 1, dev)
+        peak, kind = measured_tensor_peak()
+        pre = {"workload": EXTRA_PREFILL, "value": r["value"], "unit": r["unit"], "ms_per_step": r["ms_per_step"],
+               "steps": sub.steps, "warmup": sub.warmup, "stages_ms": r["stages_ms"],
+               "attn_tflops": r["attn_tflops"],
+               "tensor_frac": {n: v / peak for n, v in r["attn_tflops"].items()},
+               "tensor_peak": peak, "tensor_peak_kind": kind,
+               "indexer_fp64_frac": r["roofline"]["frac"], "sm_mhz": r["clocks"].get("sm_mhz"),
+               "reasons": r["clocks"].get("reasons")}
+    except Exception as ex:  # noqa: BLE001 -- recorded in the JSON line
+        pre = {"workload": EXTRA_PREFILL, "error": str(ex)[:200]}
+    return out, pre
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -967,6 +1047,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=[x.name for x in configs.WORKLOADS])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="default workload only: skip the brief runs of the other workloads (prefill and the "
+                         "other decode configurations) that the JSON line carries under other_workloads / prefill")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--indexer", default="bf16", choices=["bf16", "mxfp4"],
                     help="decode only: the CSA indexer keys in bf16 (the workload) or FP4 (MXFP4)")
@@ -976,6 +1059,10 @@ def main():
                     help="decode only: context-parallel mode, one batch sharded by context over the ranks")
     ap.add_argument("--tokens", type=int, default=0,
                     help="prefill only: a shorter sequence than the workload's (small cases for profiling)")
+    ap.add_argument("--e2e-io", type=int, default=None, choices=[0, 1, 2, 3],
+                    help="decode only: the I/O mode of the e2e leg's captured step (sa_decode_graph_create flags: "
+                         "1 a kernel copies the queries in, 2 the kernels write the outputs to host memory; "
+                         "default: DecodeGraph.DEFAULT_FLAGS)")
     ap.add_argument("--decode-fast", type=int, default=0, choices=[0, 1],
                     help="decode only: the indexer + top-k kernels (SA_OPT_DECODE_FAST: 0 the general ones, "
                          "1 the sampled-bound fast path; same indices and outputs)")
@@ -1022,6 +1109,9 @@ def main():
             res = run_cp(args, w, rank, world, dev)
         else:
             res = run_ours(args, w, rank, world, dev) if w.mode == "decode" else run_prefill(args, w, rank, world, dev)
+            if (world == 1 and not args.no_extras and args.workload == DEFAULT_WORKLOAD and not args.trace
+                    and args.indexer == "bf16" and args.kv == "workload"):
+                res["other_workloads"], res["prefill"] = run_extras(args, dev)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

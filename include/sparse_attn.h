@@ -248,6 +248,74 @@ sa_status hybrid_attn_prefill_mxfp4(const void* q, const void* q_idx, int32_t T,
                                     int32_t* idx_out, int32_t* cnt_out,
                                     void* ws, size_t ws_bytes, void* stream);
 
+/* A hybrid decode step captured once into a CUDA graph together with its
+ * host copies, for a serving loop that decodes the same batch step after
+ * step: one cudaGraphLaunch per step copies the new queries in from pinned
+ * host memory, runs hybrid_attn_decode (or hybrid_attn_decode_mxfp4) and
+ * copies both outputs and both lse back to pinned host memory.  The review
+ * (section 3-2 (2)) defines the step; the graph and the packed copies are
+ * this library's own serving form of it, with no counterpart on the page.
+ *
+ * Packed I/O, the same layout on the host and on the device (byte offsets
+ * from sa_decode_io_layout, each a multiple of 256):
+ *   in:  q_idx [B][d_idx] bf16 at q_idx_off, q [B][H][d] bf16 at q_off;
+ *   out: out_hca [B][H][d] bf16, lse_hca [B][H] fp32, out_csa, lse_csa.
+ * The HCA half of `out` (out_hca, lse_hca) is copied back as soon as the
+ * HCA branch ends, overlapping the CSA branch; the CSA half at the end.     */
+typedef struct {
+    size_t in_bytes, q_idx_off, q_off;
+    size_t out_bytes, out_hca_off, lse_hca_off, out_csa_off, lse_csa_off;
+} sa_decode_io;
+
+/* Fills *io for B sequences and H heads (B >= 1, H 1..128).                */
+sa_status sa_decode_io_layout(int32_t B, int32_t H, sa_decode_io* io);
+
+typedef struct sa_decode_graph sa_decode_graph;
+
+/* How the step moves its I/O (flags of sa_decode_graph_create):
+ *   0                    copy-engine copies: host_in -> dev_in before the
+ *                        step, dev_out -> host_out after each branch;
+ *   SA_DG_KERNEL_IN      the queries are copied by a kernel that reads
+ *                        host_in through its device mapping;
+ *   SA_DG_DIRECT_OUT     the attention kernels write both outputs and both
+ *                        lse straight into host_out through its device
+ *                        mapping (no copy after the step; dev_out unused).
+ * The mapped forms need host buffers that the device can address (pinned
+ * memory on a system with unified addressing, where cudaHostAlloc memory is
+ * mapped); otherwise SA_ERR_INVALID_ARG.                                     */
+#define SA_DG_KERNEL_IN 1u
+#define SA_DG_DIRECT_OUT 2u
+
+/* Captures the step.  The caller owns every buffer and keeps it alive (and
+ * at the same address) until sa_decode_graph_destroy:
+ *   host_in, host_out: PINNED host memory (cudaHostAlloc or
+ *     cudaHostRegister) of io.in_bytes / io.out_bytes; pageable memory is
+ *     rejected with SA_ERR_INVALID_ARG;
+ *   dev_in, dev_out: device memory of the same sizes (dev_out may be NULL
+ *     with SA_DG_DIRECT_OUT);
+ *   idx_out [B][k] / cnt_out [B] int32 device, or both NULL;
+ *   ws / ws_bytes as for hybrid_attn_decode;
+ *   codes / scales: the MXFP4 indexer (as for hybrid_attn_decode_mxfp4), or
+ *     both NULL for the bf16 indexer keys;
+ *   flags: 0 or an OR of SA_DG_KERNEL_IN and SA_DG_DIRECT_OUT.
+ * The caches are read in place at every step, so appends between steps are
+ * seen; their struct fields (pointers, capacities) are fixed at capture, and
+ * so are the library options.  Unlike the other calls, this one runs the
+ * step once eagerly and synchronises the device before capturing (on a
+ * stream of its own).  On success *graph receives the handle.               */
+sa_status sa_decode_graph_create(const sa_cache* csa, const sa_cache* hca, int32_t H, int32_t k, float scale,
+                                 const uint8_t* codes, const uint8_t* scales, void* host_in, void* host_out,
+                                 void* dev_in, void* dev_out, int32_t* idx_out, int32_t* cnt_out, void* ws,
+                                 size_t ws_bytes, uint32_t flags, sa_decode_graph** graph);
+
+/* Launches one captured step on `stream`.  host_in must hold the step's
+ * queries when the launch runs; host_out holds the results once `stream`
+ * has reached the end of the step (synchronise or wait on an event).       */
+sa_status sa_decode_graph_step(sa_decode_graph* graph, void* stream);
+
+/* Frees the graph (not the caller's buffers).  NULL is accepted.           */
+sa_status sa_decode_graph_destroy(sa_decode_graph* graph);
+
 /* hybrid_attn_decode with the sliding-window branch of both layers: the
  * review (section 3-2 (2)) adds a window of recent uncompressed tokens to CSA
  * and to HCA alike.  out_csa is the attention over the CSA selection joined

@@ -3,7 +3,8 @@
 The compute path is the CUDA library; ``api`` only marshals torch tensors
 into its C ABI and ``synth`` only generates seeded inputs.
 """
-from .api import (Cache, CapturedDecode, alloc_cache, alloc_workspace, attn_lse_merge, csa_append, csa_compress,  # noqa: F401
+from .api import (Cache, CapturedDecode, DecodeGraph, alloc_cache, alloc_workspace, attn_lse_merge,  # noqa: F401
+                  csa_append, csa_compress, decode_io_layout,
                   csa_index_topk, csa_index_topk_noalloc, hca_append, swa_attn,
                   csa_index_quantize_mxfp4, csa_index_topk_mxfp4, hybrid_attn_decode_mxfp4, hybrid_attn_decode_swa,
                   hybrid_attn_prefill_mxfp4,

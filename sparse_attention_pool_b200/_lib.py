@@ -28,11 +28,13 @@ EXPORTS = ["csa_compress", "hca_compress", "csa_index_topk", "csa_sparse_attn", 
            "csa_index_quantize_mxfp4", "csa_index_topk_mxfp4", "hybrid_attn_decode_mxfp4",
            "cp_decode_candidates", "cp_decode_merge_select", "attn_lse_merge_n", "hybrid_attn_decode_swa",
            "sa_selftest_wait_timeout", "sa_trace_install", "sa_trace_count", "hybrid_attn_prefill_mxfp4",
-           "sa_set_option", "sa_get_option"]
+           "sa_set_option", "sa_get_option", "sa_decode_io_layout", "sa_decode_graph_create",
+           "sa_decode_graph_step", "sa_decode_graph_destroy"]
 SA_NOALLOC_SCRATCH_BYTES = 32 << 20
 SA_STAGE_INDEX_SCORE, SA_STAGE_TOPK_SELECT, SA_STAGE_CSA_ATTN, SA_STAGE_HCA_ATTN = 0, 1, 2, 3
 SA_OPT_PREFILL_SELECT = 1
 SA_OPT_DECODE_FAST = 2
+SA_DG_KERNEL_IN, SA_DG_DIRECT_OUT = 1, 2
 
 P = ctypes.c_void_p
 I32 = ctypes.c_int32
@@ -48,6 +50,11 @@ class SaRaw(ctypes.Structure):
 class SaCache(ctypes.Structure):
     _fields_ = [("k", P), ("v", P), ("k_scale", P), ("v_scale", P), ("kidx", P), ("n", P),
                 ("B", I32), ("Ncap", I32), ("d", I32), ("d_idx", I32), ("m", I32), ("dtype", I32)]
+
+
+class SaDecodeIO(ctypes.Structure):
+    _fields_ = [(n, SZ) for n in ("in_bytes", "q_idx_off", "q_off", "out_bytes", "out_hca_off", "lse_hca_off",
+                                  "out_csa_off", "lse_csa_off")]
 
 
 class SparseAttnError(RuntimeError):
@@ -104,6 +111,11 @@ def lib():
         L.sa_set_option.argtypes = [I32, ctypes.c_int64]
         L.sa_get_option.argtypes = [I32, ctypes.POINTER(ctypes.c_int64)]
         L.sa_launch_count.argtypes = []
+        L.sa_decode_io_layout.argtypes = [I32, I32, ctypes.POINTER(SaDecodeIO)]
+        L.sa_decode_graph_create.argtypes = [CP, CP, I32, I32, F32, P, P, P, P, P, P, P, P, P, SZ,
+                                             ctypes.c_uint32, ctypes.POINTER(P)]
+        L.sa_decode_graph_step.argtypes = [P, P]
+        L.sa_decode_graph_destroy.argtypes = [P]
         L.sa_launch_count.restype = ctypes.c_uint64
         for name in EXPORTS:
             if name not in ("sa_workspace_size", "sa_last_error", "sa_abi_version", "sa_launch_count"):

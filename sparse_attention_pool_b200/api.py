@@ -512,3 +512,84 @@ class CapturedDecode:
                          (lse_hca, self.lse_hca)):
             if dst is not None:
                 dst.copy_(src.view(dst.dtype) if dst.dtype != src.dtype else src, non_blocking=True)
+
+
+def decode_io_layout(B: int, H: int) -> _lib.SaDecodeIO:
+    """Byte offsets of the packed decode I/O (sa_decode_io_layout)."""
+    io = _lib.SaDecodeIO()
+    check("sa_decode_io_layout", lib().sa_decode_io_layout(B, H, ctypes.byref(io)))
+    return io
+
+
+class DecodeGraph:
+    """sa_decode_graph_*: a hybrid decode step captured by the library into a
+    CUDA graph together with its host copies (one H2D copy of the packed
+    queries, the HCA outputs copied back from the HCA branch, the CSA outputs
+    at the end), launched by one call per step.
+
+    The pinned host buffers are exposed as views: write ``q`` [B][H][128] and
+    ``q_idx`` [B][64] (bf16) before ``step``; read ``out_csa`` / ``out_hca``
+    [B][H][128] (bf16) and ``lse_csa`` / ``lse_hca`` [B][H] (fp32) once the
+    stream has finished the step.  ``idx`` [B][k] / ``cnt`` [B] stay on the
+    device.  All buffers are allocated here (torch) and owned by this object.
+    ``flags`` (SA_DG_KERNEL_IN, SA_DG_DIRECT_OUT) choose how the I/O moves:
+    copy-engine copies (0), a kernel reading the mapped host queries, the
+    kernels writing the outputs straight into the mapped host buffer.
+    """
+
+    DEFAULT_FLAGS = _lib.SA_DG_KERNEL_IN  # measured fastest on a B200 at 1M context
+
+    def __init__(self, csa: Cache, hca: Cache, k: int, H: int, *, scale: float = 0.0, codes=None, scales=None,
+                 flags: int | None = None):
+        dev = csa.k.device
+        B = csa.B
+        self.io = io = decode_io_layout(B, H)
+        self.csa, self.hca, self.k, self.H = csa, hca, k, H
+        self.codes, self.scales = codes, scales
+        self.host_in = torch.zeros(io.in_bytes, dtype=torch.uint8).pin_memory()
+        self.host_out = torch.zeros(io.out_bytes, dtype=torch.uint8).pin_memory()
+        self.dev_in = torch.zeros(io.in_bytes, dtype=torch.uint8, device=dev)
+        self.dev_out = torch.zeros(io.out_bytes, dtype=torch.uint8, device=dev)
+        self.idx = torch.empty(B, k, dtype=torch.int32, device=dev)
+        self.cnt = torch.empty(B, dtype=torch.int32, device=dev)
+        self.ws = alloc_workspace(workspace_size(_lib.SA_OP_HYBRID_DECODE, B, 1, H, csa.Ncap, hca.Ncap, k), device=dev)
+
+        def view(buf, off, shape, dtype):
+            n = 1
+            for x in shape:
+                n *= x
+            nb = n * torch.tensor([], dtype=dtype).element_size()
+            return buf[off:off + nb].view(dtype).view(*shape)
+
+        self.q_idx = view(self.host_in, io.q_idx_off, (B, D_IDX), torch.bfloat16)
+        self.q = view(self.host_in, io.q_off, (B, H, D), torch.bfloat16)
+        self.out_hca = view(self.host_out, io.out_hca_off, (B, H, D), torch.bfloat16)
+        self.lse_hca = view(self.host_out, io.lse_hca_off, (B, H), torch.float32)
+        self.out_csa = view(self.host_out, io.out_csa_off, (B, H, D), torch.bfloat16)
+        self.lse_csa = view(self.host_out, io.lse_csa_off, (B, H), torch.float32)
+        self.h2d_bytes, self.d2h_bytes = io.in_bytes, io.out_bytes
+        self.flags = self.DEFAULT_FLAGS if flags is None else flags
+        self._cs, self._hs = csa.struct(), hca.struct()
+        handle = ctypes.c_void_p()
+        torch.cuda.synchronize(dev)
+        check("sa_decode_graph_create",
+              lib().sa_decode_graph_create(ctypes.byref(self._cs), ctypes.byref(self._hs), H, k, scale, _ptr(codes),
+                                           _ptr(scales), _ptr(self.host_in), _ptr(self.host_out), _ptr(self.dev_in),
+                                           _ptr(self.dev_out), _ptr(self.idx), _ptr(self.cnt), _ptr(self.ws),
+                                           self.ws.numel(), self.flags, ctypes.byref(handle)))
+        self._handle = handle
+
+    def step(self, stream=None):
+        """Launch one captured step on the stream (asynchronous)."""
+        check("sa_decode_graph_step", lib().sa_decode_graph_step(self._handle, _stream(stream)))
+
+    def close(self):
+        if getattr(self, "_handle", None) is not None and self._handle.value:
+            check("sa_decode_graph_destroy", lib().sa_decode_graph_destroy(self._handle))
+            self._handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # noqa: BLE001 -- interpreter shutdown
+            pass

@@ -176,7 +176,9 @@ __global__ void __launch_bounds__(NW * EG * 32) attn_split_kernel(AttnArgs a) {
     const int rowBytes = FP8 ? 128 : 256;
     const size_t seqBase = (size_t)b * a.Ncap * rowBytes;
 
-    // each thread copies CPT 16-byte chunks of one row; a gathered row costs one index load
+    // each thread copies CPT 16-byte chunks of one row, TPR apart, so that the
+    // row's TPR threads read consecutive chunks in each instruction; a
+    // gathered row costs one index load
     constexpr int cpr = FP8 ? 8 : 16;            // 16-byte chunks per row
     constexpr int CPT = cpr / TPR;               // chunks per thread
     static_assert(TPR >= 1 && CPT >= 1 && CPT * TPR == cpr, "tile mapping");
@@ -198,7 +200,7 @@ __global__ void __launch_bounds__(NW * EG * 32) attn_split_kernel(AttnArgs a) {
         const size_t rowOff = seqBase + (size_t)(ok ? j : 0) * rowBytes;
 #pragma unroll
         for (int c = 0; c < CPT; ++c) {
-            const int ch = c0 + c;
+            const int ch = tid % TPR + c * TPR;
             const uint32_t doff = FP8 ? (uint32_t)(r * 128 + ch * 16) : swz(r, ch);
             if (!MIXED) cp_async16_zfill(rk + doff, Kb + rowOff + ch * 16, ok);
             cp_async16_zfill(rv + doff, Vb + rowOff + ch * 16, ok);

@@ -150,8 +150,13 @@ __global__ void __launch_bounds__(kCtThreads, 1) attn_csa_prefill_tc_kernel(CtAr
     const uint32_t id_s = ct_idesc(0, 0), id_o = ct_idesc(1, 1);
     uint32_t ph_s = 0, ph_o = 0;
     int pend_s = 0, pend_o = 0;  // (thread 0) commits not yet seen complete
-    const int r = tid & (kCtRows - 1);  // the tile row this thread gathers (K: tid < 128, V: the rest)
-    const bool isv = tid >= kCtRows;
+    // The gather: warp w copies tile rows 16w .. 16w + 15, one row per
+    // instruction, lanes 0-15 the row's 16 K chunks and lanes 16-31 its V
+    // chunks (512 contiguous bytes per instruction); lane l holds the entry
+    // of row 16w + (l & 15).
+    const int grow = warp * 16 + (lane & 15);
+    const int gchunk = lane & 15;
+    const bool isv = lane >= 16;
 
     for (long long bq = blockIdx.x; bq < a.BQ; bq += gridDim.x) {
         const int b = (int)(bq / a.T);
@@ -167,30 +172,35 @@ __global__ void __launch_bounds__(kCtThreads, 1) attn_csa_prefill_tc_kernel(CtAr
         }
         const int ntiles = (R + kCtRows - 1) / kCtRows;
         const int32_t* lidx = a.idx + (size_t)bq * a.kmax;
-        // Q: 64 rows of 16 chunks, rows at or past H zero
-        {
-            const int h = tid >> 2, c0 = (tid & 3) * 4;
-            const bool ok = h < a.H;
-            const uint16_t* src = a.q + ((size_t)bq * a.H + (ok ? h : 0)) * 128;
+        // Q: 64 rows of 16 chunks, rows at or past H zero; 16 threads a row,
+        // two consecutive (contiguous) rows per instruction
 #pragma unroll
-            for (int c = c0; c < c0 + 4; ++c) cp_async16_zfill(sm + kCtQ + sw128_off(h, c, 8192), src + c * 8, ok);
+        for (int u = 0; u < 4; ++u) {
+            const int h = u * 16 + (tid >> 4), c = tid & 15;
+            const bool ok = h < a.H;
+            const uint16_t* src = a.q + ((size_t)bq * a.H + (ok ? h : 0)) * 128 + c * 8;
+            cp_async16_zfill(sm + kCtQ + sw128_off(h, c, 8192), src, ok);
         }
         // the gather of tile t's rows into buffer t & 1 (zero past the list);
-        // jn holds this thread's entry of that tile, loaded a tile ahead
-        int jn = ntiles > 0 && r < R ? (int)ld_cg_u32(lidx + r) : 0;
+        // jn holds the entry of this lane's row of that tile, loaded a tile ahead
+        int jn = ntiles > 0 && grow < R ? (int)ld_cg_u32(lidx + grow) : 0;
         auto gather = [&](int t) {
-            const int p = t * kCtRows + r;
-            bool ok = p < R;
-            int j = jn;
-            if (ok && (j < 0 || j >= nb)) {
-                flag(DEV_INDEX);
-                ok = false;
+            int jo = -1;  // this lane's row: its entry, or -1 past the list or when out of range (flagged)
+            if (t * kCtRows + grow < R) {
+                if (jn >= 0 && jn < nb)
+                    jo = jn;
+                else if (!isv)
+                    flag(DEV_INDEX);
             }
-            const uint16_t* src = (isv ? a.V : a.K) + ((size_t)b * a.Ncap + (ok ? j : 0)) * 128;
+            const uint16_t* src = (isv ? a.V : a.K) + (size_t)b * a.Ncap * 128 + gchunk * 8;
             uint8_t* dst = sm + (isv ? kCtV : kCtK) + (t & 1) * 32768;
 #pragma unroll
-            for (int c = 0; c < 16; ++c) cp_async16_zfill(dst + sw128_off(r, c, 16384), src + c * 8, ok);
-            const int pn = (t + 1) * kCtRows + r;
+            for (int p = 0; p < 16; ++p) {
+                const int j = __shfl_sync(0xFFFFFFFFu, jo, p);  // lane p holds row 16w + p
+                cp_async16_zfill(dst + sw128_off(warp * 16 + p, gchunk, 16384), src + (size_t)(j >= 0 ? j : 0) * 128,
+                                 j >= 0);
+            }
+            const int pn = (t + 1) * kCtRows + grow;
             jn = t + 1 < ntiles && pn < R ? (int)ld_cg_u32(lidx + pn) : 0;
         };
         if (ntiles > 0) gather(0);

@@ -161,20 +161,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_prefill_tc_kernel(TcArgs a
     const int rmax = max(R[0], R[1]);
     const int ntiles = (rmax + per_tile - 1) / per_tile;
 
+    // Copies of 128-row operands: warp w takes rows 32w .. 32w + 31, two
+    // rows per instruction (16 lanes a row, 512 contiguous bytes when the
+    // rows are consecutive).
+    const int lane = tid & 31, gchunk = lane & 15;
     // Q: row (qq * 64 + h), 16 chunks of 8 dims; rows of a missing second query are zero
-    {
-        const int r = tid;  // one row per thread
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+        const int r = 32 * warp + 2 * p + (lane >> 4);
         const int qq = r >> 6, h = r & 63;
         const bool ok = t0 + qq < a.T;
-        const uint16_t* src = a.q + (((size_t)b * a.T + (ok ? t0 + qq : t0)) * 64 + h) * 128;
-#pragma unroll
-        for (int c = 0; c < 16; ++c) cp_async16_zfill(sm + kTcQ + tc_off(r, c), src + c * 8, ok);
+        const uint16_t* src = a.q + (((size_t)b * a.T + (ok ? t0 + qq : t0)) * 64 + h) * 128 + gchunk * 8;
+        cp_async16_zfill(sm + kTcQ + tc_off(r, gchunk), src, ok);
     }
     cp_async_commit();
 
-    // one tile of K and V: thread = tile row, 16 chunks each
-    // a gathered row's list entry is fetched one tile ahead (ld_idx), so the
-    // copies of a tile never wait for it
+    // one tile of K and V; thread tid knows the entry of tile row tid (a
+    // gathered row's list entry is fetched one tile ahead by ld_idx, so the
+    // copies of a tile never wait for it) and hands it to the lanes copying it
     auto ld_idx = [&](int i) -> int {
         if (!GATHER) return 0;
         const int qq = tid >> 6;
@@ -184,30 +188,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_prefill_tc_kernel(TcArgs a
                    : 0;
     };
     auto load_tile = [&](int i, int stage, int jg) {
-        const int r = tid;
-        int j;
-        bool ok;
+        int jo;  // tile row tid: its entry, or -1 (past the list, or out of range and flagged)
         if (GATHER) {
-            const int qq = r >> 6;
-            const int p = i * per_tile + (r & 63);
-            ok = t0 + qq < a.T && p < R[qq];
-            j = jg;
-            if (ok && (j < 0 || j >= nb)) {
+            const int qq = tid >> 6;
+            const int p = i * per_tile + (tid & 63);
+            bool ok = t0 + qq < a.T && p < R[qq];
+            if (ok && (jg < 0 || jg >= nb)) {
                 flag(DEV_INDEX);
                 ok = false;
             }
+            jo = ok ? jg : -1;
         } else {
-            j = i * per_tile + r;
-            ok = j < rmax;
+            const int j = i * per_tile + tid;
+            jo = j < rmax ? j : -1;
         }
-        const uint16_t* kr = a.K + ((size_t)b * a.Ncap + (ok ? j : 0)) * 128;
-        const uint16_t* vr = a.V + ((size_t)b * a.Ncap + (ok ? j : 0)) * 128;
         uint8_t* dk = sm + kTcK + stage * kTcOpBytes;
         uint8_t* dv = sm + kTcV + stage * kTcOpBytes;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            cp_async16_zfill(dk + tc_off(r, c), kr + c * 8, ok);
-            cp_async16_zfill(dv + tc_off(r, c), vr + c * 8, ok);
+        for (int p = 0; p < 16; ++p) {
+            const int r = 32 * warp + 2 * p + (lane >> 4);
+            const int j = __shfl_sync(0xFFFFFFFFu, jo, 2 * p + (lane >> 4));  // the lane of row r
+            const bool ok = j >= 0;
+            const size_t off = ((size_t)b * a.Ncap + (ok ? j : 0)) * 128 + gchunk * 8;
+            cp_async16_zfill(dk + tc_off(r, gchunk), a.K + off, ok);
+            cp_async16_zfill(dv + tc_off(r, gchunk), a.V + off, ok);
         }
     };
     const int j0 = ld_idx(0);

@@ -13,6 +13,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <new>
 #include <utility>
 
 #include "../../include/sparse_attn.h"
@@ -917,6 +918,14 @@ __global__ void selftest_wait_kernel(uint32_t limit) {
 }
 }  // namespace sa
 
+namespace sa {
+// Copies n 16-byte words from a pinned host buffer (read through its device
+// mapping, fetched again every time: no stale cached line of it is used).
+__global__ void __launch_bounds__(256) copy_in_kernel(const uint4* src, uint4* __restrict__ dst, uint32_t n) {
+    for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) dst[i] = __ldcv(src + i);
+}
+}  // namespace sa
+
 // =========================================================== public ABI ====
 extern "C" {
 
@@ -1563,6 +1572,166 @@ sa_status hybrid_attn_decode_mxfp4(const void* q, const void* q_idx, int32_t H, 
     SA_CHECK(codes && scales, "hybrid_attn_decode_mxfp4: codes and scales must be non-NULL");
     return hybrid_decode_impl("hybrid_attn_decode_mxfp4", q, q_idx, H, csa, hca, codes, scales, k, scale, out_csa,
                               out_hca, lse_csa, lse_hca, idx_out, cnt_out, ws, ws_bytes, stream);
+}
+
+sa_status sa_decode_io_layout(int32_t B, int32_t H, sa_decode_io* io) {
+    SA_CHECK(io != nullptr, "sa_decode_io_layout: io must be non-NULL");
+    SA_CHECK(B >= 1 && H >= 1 && H <= 128, "sa_decode_io_layout: B=%d H=%d outside B >= 1, H 1..128", B, H);
+    const size_t rows = (size_t)B * H;
+    io->q_idx_off = 0;
+    io->q_off = up256((size_t)B * 64 * 2);
+    io->in_bytes = io->q_off + up256(rows * 128 * 2);
+    io->out_hca_off = 0;
+    io->lse_hca_off = up256(rows * 128 * 2);
+    io->out_csa_off = io->lse_hca_off + up256(rows * 4);
+    io->lse_csa_off = io->out_csa_off + up256(rows * 128 * 2);
+    io->out_bytes = io->lse_csa_off + up256(rows * 4);
+    return SA_OK;
+}
+
+struct sa_decode_graph {
+    cudaGraphExec_t exec = nullptr;
+    uint64_t kernels = 0;  // kernels one step launches (for sa_launch_count)
+};
+
+// The device's view of a pinned host buffer (NULL when it has none), after
+// checking that `p` is pinned host memory.
+static sa_status host_mapping(const void* p, const char* what, const char* name, void** dev_view) {
+    cudaPointerAttributes a{};
+    SA_CUDA(cudaPointerGetAttributes(&a, p));
+    SA_CHECK(a.type == cudaMemoryTypeHost, "%s: %s must be pinned host memory", what, name);
+    *dev_view = a.devicePointer;
+    return SA_OK;
+}
+
+static sa_status check_device_mem(const void* p, const char* what, const char* name) {
+    cudaPointerAttributes a{};
+    SA_CUDA(cudaPointerGetAttributes(&a, p));
+    SA_CHECK(a.type == cudaMemoryTypeDevice, "%s: %s must be device memory", what, name);
+    return SA_OK;
+}
+
+sa_status sa_decode_graph_create(const sa_cache* csa, const sa_cache* hca, int32_t H, int32_t k, float scale,
+                                 const uint8_t* codes, const uint8_t* scales, void* host_in, void* host_out,
+                                 void* dev_in, void* dev_out, int32_t* idx_out, int32_t* cnt_out, void* ws,
+                                 size_t ws_bytes, uint32_t flags, sa_decode_graph** graph) {
+    const char* what = "sa_decode_graph_create";
+    SA_CHECK(graph != nullptr, "%s: graph must be non-NULL", what);
+    *graph = nullptr;
+    SA_CHECK(csa != nullptr && hca != nullptr, "%s: caches must be non-NULL", what);
+    SA_CHECK((codes == nullptr) == (scales == nullptr), "%s: give both codes and scales or neither", what);
+    SA_CHECK((flags & ~(SA_DG_KERNEL_IN | SA_DG_DIRECT_OUT)) == 0, "%s: unknown flags 0x%x", what, flags);
+    const bool kin = flags & SA_DG_KERNEL_IN, dout_direct = flags & SA_DG_DIRECT_OUT;
+    sa_decode_io io;
+    sa_status r = sa_decode_io_layout(csa->B, H, &io);
+    if (r != SA_OK) return r;
+    SA_CHECK(host_in && host_out && dev_in && (dev_out || dout_direct), "%s: I/O buffers must be non-NULL", what);
+    SA_CHECK(aligned16(host_in) && aligned16(host_out) && aligned16(dev_in) && aligned16(dev_out),
+             "%s: I/O buffers must be 16-byte aligned", what);
+    void *map_in = nullptr, *map_out = nullptr;
+    if ((r = host_mapping(host_in, what, "host_in", &map_in)) != SA_OK) return r;
+    if ((r = host_mapping(host_out, what, "host_out", &map_out)) != SA_OK) return r;
+    SA_CHECK(!kin || (map_in && aligned16(map_in)), "%s: SA_DG_KERNEL_IN needs host_in mapped into the device", what);
+    SA_CHECK(!dout_direct || (map_out && aligned16(map_out)),
+             "%s: SA_DG_DIRECT_OUT needs host_out mapped into the device", what);
+    if ((r = check_device_mem(dev_in, what, "dev_in")) != SA_OK) return r;
+    if (!dout_direct && (r = check_device_mem(dev_out, what, "dev_out")) != SA_OK) return r;
+    const bool fp4 = codes != nullptr;
+    uint8_t* di = static_cast<uint8_t*>(dev_in);
+    uint8_t* hout = static_cast<uint8_t*>(host_out);
+    // where the kernels write the outputs: the device buffer, or the host
+    // buffer's device mapping
+    uint8_t* dout = static_cast<uint8_t*>(dout_direct ? map_out : dev_out);
+    // One step: the packed queries in, both branches, the HCA half of the
+    // outputs back from the HCA branch (overlapping the CSA branch), the CSA
+    // half at the end.  The eager pass (kernel attributes, the side stream)
+    // zeroes the queries instead of copying them and copies nothing back.
+    auto body = [&](cudaStream_t cs, bool eager) -> sa_status {
+        if (eager) {
+            SA_CUDA(cudaMemsetAsync(di, 0, io.in_bytes, cs));
+        } else if (kin) {
+            const uint32_t n16 = (uint32_t)(io.in_bytes / 16);
+            sa::copy_in_kernel<<<std::min(cdiv(n16, 256), 2 * num_sms()), 256, 0, cs>>>(
+                static_cast<const uint4*>(map_in), reinterpret_cast<uint4*>(di), n16);
+            SA_LAUNCHED();
+        } else {
+            SA_CUDA(cudaMemcpyAsync(di, host_in, io.in_bytes, cudaMemcpyHostToDevice, cs));
+        }
+        const bool copy_back = !eager && !dout_direct;
+        std::function<sa_status(cudaStream_t)> hca_back = nullptr;
+        if (copy_back)
+            hca_back = [&](cudaStream_t s) -> sa_status {
+                SA_CUDA(cudaMemcpyAsync(hout, dout, io.out_csa_off, cudaMemcpyDeviceToHost, s));
+                return SA_OK;
+            };
+        // the eager pass writes to the device buffer when there is one
+        uint8_t* o = eager && dev_out ? static_cast<uint8_t*>(dev_out) : dout;
+        sa_status rr = hybrid_decode_impl(fp4 ? "hybrid_attn_decode_mxfp4" : "hybrid_attn_decode", di + io.q_off,
+                                          di + io.q_idx_off, H, csa, hca, codes, scales, k, scale,
+                                          o + io.out_csa_off, o + io.out_hca_off,
+                                          reinterpret_cast<float*>(o + io.lse_csa_off),
+                                          reinterpret_cast<float*>(o + io.lse_hca_off), idx_out, cnt_out, ws,
+                                          ws_bytes, cs, hca_back);
+        if (rr != SA_OK) return rr;
+        if (copy_back)
+            SA_CUDA(cudaMemcpyAsync(hout + io.out_csa_off, dout + io.out_csa_off, io.out_bytes - io.out_csa_off,
+                                    cudaMemcpyDeviceToHost, cs));
+        return SA_OK;
+    };
+    cudaStream_t cs = nullptr;
+    SA_CUDA(cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking));
+    cudaGraph_t g = nullptr;
+    cudaGraphExec_t exec = nullptr;
+    uint64_t kernels = 0;
+    r = body(cs, true);
+    cudaError_t e = cudaStreamSynchronize(cs);
+    if (r == SA_OK && e != cudaSuccess) r = fail(SA_ERR_CUDA, "%s: eager step: %s", what, cudaGetErrorString(e));
+    if (r == SA_OK) {
+        e = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal);
+        if (e != cudaSuccess) {
+            r = fail(SA_ERR_CUDA, "%s: begin capture: %s", what, cudaGetErrorString(e));
+        } else {
+            const uint64_t n0 = g_launches;
+            r = body(cs, false);
+            kernels = g_launches - n0;
+            e = cudaStreamEndCapture(cs, &g);  // always ends the capture, also after an error
+            if (r == SA_OK && e != cudaSuccess) r = fail(SA_ERR_CUDA, "%s: end capture: %s", what, cudaGetErrorString(e));
+        }
+    }
+    if (r == SA_OK) {
+        e = cudaGraphInstantiate(&exec, g, 0);
+        if (e != cudaSuccess) r = fail(SA_ERR_CUDA, "%s: instantiate: %s", what, cudaGetErrorString(e));
+    }
+    if (g) cudaGraphDestroy(g);
+    cudaStreamDestroy(cs);
+    if (r != SA_OK) {
+        if (exec) cudaGraphExecDestroy(exec);
+        return r;
+    }
+    sa_decode_graph* h = new (std::nothrow) sa_decode_graph;
+    if (!h) {
+        cudaGraphExecDestroy(exec);
+        return fail(SA_ERR_UNSUPPORTED, "%s: out of host memory", what);
+    }
+    h->exec = exec;
+    h->kernels = kernels;
+    *graph = h;
+    return SA_OK;
+}
+
+sa_status sa_decode_graph_step(sa_decode_graph* graph, void* stream) {
+    SA_CHECK(graph != nullptr && graph->exec != nullptr, "sa_decode_graph_step: graph must be a created graph");
+    SA_CUDA(cudaGraphLaunch(graph->exec, static_cast<cudaStream_t>(stream)));
+    g_launches += graph->kernels;
+    return SA_OK;
+}
+
+sa_status sa_decode_graph_destroy(sa_decode_graph* graph) {
+    if (!graph) return SA_OK;
+    const cudaError_t e = graph->exec ? cudaGraphExecDestroy(graph->exec) : cudaSuccess;
+    delete graph;
+    if (e != cudaSuccess) return fail(SA_ERR_CUDA, "sa_decode_graph_destroy: %s", cudaGetErrorString(e));
+    return SA_OK;
 }
 
 // Causal prefill of both branches; with MXFP4 indexer keys (codes4 /

@@ -369,3 +369,48 @@ def test_workspace_sizes_are_monotone(L, op):
     for key, bigger in (("B", 4), ("Nc", 262144), ("Nh", 8192), ("k", 2048), ("H", 128)):
         assert size(**{key: bigger}) >= s0, key
     assert ws(8, 4, 1, 64, 262144, 8192, 2048) >= ws(4, 4, 1, 64, 262144, 8192, 2048)
+
+
+def test_decode_io_layout_on_the_host(L):
+    io = _lib.SaDecodeIO()
+    assert L.sa_decode_io_layout(4, 64, ctypes.byref(io)) == _lib.SA_OK
+    rows = 4 * 64
+    # q_idx then q; out_hca, lse_hca, out_csa, lse_csa: every region 256-byte aligned and large enough
+    assert io.q_idx_off == 0 and io.q_off == 512 and io.in_bytes == 512 + rows * 256
+    assert io.out_hca_off == 0 and io.lse_hca_off == rows * 256
+    assert io.out_csa_off == io.lse_hca_off + rows * 4 and io.lse_csa_off == io.out_csa_off + rows * 256
+    assert io.out_bytes == io.lse_csa_off + rows * 4
+    assert L.sa_decode_io_layout(3, 5, ctypes.byref(io)) == _lib.SA_OK
+    offs = [io.q_idx_off, io.q_off, io.out_hca_off, io.lse_hca_off, io.out_csa_off, io.lse_csa_off]
+    assert all(o % 256 == 0 for o in offs)
+    assert io.q_off >= 3 * 64 * 2 and io.in_bytes - io.q_off >= 15 * 256
+    assert io.lse_hca_off >= 15 * 256 and io.out_csa_off - io.lse_hca_off >= 15 * 4
+    assert io.out_bytes - io.lse_csa_off >= 15 * 4
+    for B, H in ((0, 64), (4, 0), (4, 129)):
+        assert L.sa_decode_io_layout(B, H, ctypes.byref(io)) == _lib.SA_ERR_INVALID_ARG
+    assert L.sa_decode_io_layout(4, 64, None) == _lib.SA_ERR_INVALID_ARG
+
+
+def test_decode_graph_rejects_bad_arguments(L):
+    g = ctypes.c_void_p()
+    c = _lib.SaCache()
+    args = [ctypes.byref(c), ctypes.byref(c), 64, 512, 0.0, None, None, None, None, None, None, None, None, None, 0,
+            0]
+    assert L.sa_decode_graph_create(*args, None) == _lib.SA_ERR_INVALID_ARG
+    assert "graph" in L.sa_last_error().decode()
+    args2 = list(args)
+    args2[0] = None
+    assert L.sa_decode_graph_create(*args2, ctypes.byref(g)) == _lib.SA_ERR_INVALID_ARG and not g.value
+    args3 = list(args)
+    args3[5] = ctypes.c_void_p(16)  # codes without scales
+    assert L.sa_decode_graph_create(*args3, ctypes.byref(g)) == _lib.SA_ERR_INVALID_ARG
+    assert "codes" in L.sa_last_error().decode()
+    args4 = list(args)
+    args4[15] = 8  # an unknown flag
+    assert L.sa_decode_graph_create(*args4, ctypes.byref(g)) == _lib.SA_ERR_INVALID_ARG
+    assert "flags" in L.sa_last_error().decode()
+    c.B = 2
+    assert L.sa_decode_graph_create(*args, ctypes.byref(g)) == _lib.SA_ERR_INVALID_ARG  # NULL buffers
+    assert "I/O buffers" in L.sa_last_error().decode()
+    assert L.sa_decode_graph_step(None, None) == _lib.SA_ERR_INVALID_ARG
+    assert L.sa_decode_graph_destroy(None) == _lib.SA_OK
