@@ -743,6 +743,7 @@ def run_prefill(args, w, rank, world, dev):
     L = _lib.lib()
     stream = torch.cuda.current_stream()
     S.set_option(S.SA_OPT_PREFILL_SELECT, args.prefill_select)
+    S.set_option(S.SA_OPT_HCA_PREFILL, args.hca_prefill)
 
     def step():
         S.hybrid_attn_prefill(q, qI, csa, hca, k, ws, idx, cnt, scale=SCALE, out_csa=out_c, out_hca=out_h)
@@ -814,7 +815,8 @@ def run_prefill(args, w, rank, world, dev):
         "data": "synthetic",
         "config": {"workload": w.name, "B_per_gpu": B, "tokens": T, "heads": H, "head_dim": 128, "topk": k,
                    "l2": "inputs larger than L2 (q alone is %.1f GB)" % (q.numel() * 2 / 1e9),
-                   "launch": "eager (one call per step)", "prefill_select": args.prefill_select},
+                   "launch": "eager (one call per step)", "prefill_select": args.prefill_select,
+                   "hca_prefill": args.hca_prefill},
         "stages_ms": stages,
         "roofline": {"kernel": "csa_index_topk prefill stage: score_prefill_kernel + the selection kernel",
                      "bound": "alu", "achieved": idx_tflops, "peak": fp64_peak, "unit": "TFLOP/s (fp64)",
@@ -1066,6 +1068,9 @@ def main():
     ap.add_argument("--decode-fast", type=int, default=0, choices=[0, 1],
                     help="decode only: the indexer + top-k kernels (SA_OPT_DECODE_FAST: 0 the general ones, "
                          "1 the sampled-bound fast path; same indices and outputs)")
+    ap.add_argument("--hca-prefill", type=int, default=0, choices=[0, 1],
+                    help="prefill only: the HCA attention kernel (SA_OPT_HCA_PREFILL: 0 transposed tiles, "
+                         "1 two queries per MMA)")
     ap.add_argument("--prefill-select", type=int, default=4, choices=[1, 2, 3, 4],
                     help="prefill only: the top-k selection kernel (SA_OPT_PREFILL_SELECT; same indices)")
     ap.add_argument("--trace", default="",
@@ -1082,6 +1087,8 @@ def main():
         ap.error("--cp runs the workload's own storage and indexer on our arm")
     if args.prefill_select != 4 and (w.mode != "prefill" or args.impl != "ours"):
         ap.error("--prefill-select applies to prefill workloads on our arm")
+    if args.hca_prefill != 0 and (w.mode != "prefill" or args.impl != "ours"):
+        ap.error("--hca-prefill applies to prefill workloads on our arm")
     if args.tokens:
         if w.mode != "prefill":
             ap.error("--tokens applies to prefill workloads")

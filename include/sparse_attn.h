@@ -551,9 +551,17 @@ uint64_t sa_launch_count(void);
  *       0 (default)  the general kernels (scan, filter, resolve, emit), as
  *                    for csa_index_topk; on a B200 they measured faster
  *                    at a 1M-token context (64 us per step against 67).
+ *   SA_OPT_HCA_PREFILL  the kernel of the dense (HCA) causal prefill with
+ *     query positions and a bf16 cache (hca_dense_attn with q_pos, the
+ *     hybrid prefill calls).  Same outputs up to the order of the fp32
+ *     sums (both within the bf16 tolerance of the definition):
+ *       0 (default)  the transposed tensor-memory kernel (128 entries x the
+ *                    query's heads per MMA, one query at a time; <= 64 heads);
+ *       1            the two-query kernel (2 queries x 64 heads per 128-row
+ *                    MMA; exactly 64 heads).
  * sa_set_option returns SA_ERR_INVALID_ARG for an unknown option or value;
  * sa_get_option writes the current value to *value.                        */
-typedef enum { SA_OPT_PREFILL_SELECT = 1, SA_OPT_DECODE_FAST = 2 } sa_option;
+typedef enum { SA_OPT_PREFILL_SELECT = 1, SA_OPT_DECODE_FAST = 2, SA_OPT_HCA_PREFILL = 3 } sa_option;
 sa_status sa_set_option(int32_t option, int64_t value);
 sa_status sa_get_option(int32_t option, int64_t* value);
 

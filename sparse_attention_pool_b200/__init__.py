@@ -16,5 +16,5 @@ from .api import (Cache, CapturedDecode, DecodeGraph, alloc_cache, alloc_workspa
                   workspace_size)
 from ._lib import (SA_OP_DENSE_ATTN, SA_OP_HYBRID_DECODE, SA_OP_HYBRID_PREFILL, SA_OP_INDEX_TOPK,  # noqa: F401
                    SA_OP_SPARSE_ATTN, SA_OP_WINDOW_ATTN, SA_OP_CP_CANDIDATES,
-                   SA_OP_HYBRID_DECODE_SWA, SA_OPT_DECODE_FAST, SA_OPT_PREFILL_SELECT,
+                   SA_OP_HYBRID_DECODE_SWA, SA_OPT_DECODE_FAST, SA_OPT_HCA_PREFILL, SA_OPT_PREFILL_SELECT,
                    SparseAttnError)

@@ -34,6 +34,7 @@ SA_NOALLOC_SCRATCH_BYTES = 32 << 20
 SA_STAGE_INDEX_SCORE, SA_STAGE_TOPK_SELECT, SA_STAGE_CSA_ATTN, SA_STAGE_HCA_ATTN = 0, 1, 2, 3
 SA_OPT_PREFILL_SELECT = 1
 SA_OPT_DECODE_FAST = 2
+SA_OPT_HCA_PREFILL = 3
 SA_DG_KERNEL_IN, SA_DG_DIRECT_OUT = 1, 2
 
 P = ctypes.c_void_p

@@ -18,8 +18,8 @@
 
 #include "../../include/sparse_attn.h"
 #include "attn.cuh"
-#include "attn_csa_tc.cuh"
 #include "attn_prefill_tc.cuh"
+#include "attn_prefill_tr.cuh"
 #include "compress.cuh"
 #include "cp_decode.cuh"
 #include "decode_fast.cuh"
@@ -36,6 +36,7 @@ thread_local uint64_t g_launches = 0;
 thread_local cudaEvent_t g_stage_ev[SA_NUM_STAGES][2] = {};
 std::atomic<int> g_prefill_select{4};  // SA_OPT_PREFILL_SELECT
 std::atomic<int> g_decode_fast{0};      // SA_OPT_DECODE_FAST
+std::atomic<int> g_hca_prefill{0};      // SA_OPT_HCA_PREFILL
 
 // Inside a stream capture the record must become a graph node of its own
 // (an "external" record), so that replays re-record the event.
@@ -476,10 +477,10 @@ sa_status launch_prefill_tc(const sa::AttnArgs& aa, const sa_cache* c, bool gath
     return SA_OK;
 }
 
-// Causal prefill of the gathered (CSA) branch with at most 64 heads over a
-// bf16 cache: the transposed tensor-memory kernel, a persistent grid of one
-// CTA per SM.
-sa_status launch_csa_prefill_tc(const sa::AttnArgs& aa, const sa_cache* c, long long BQ, cudaStream_t st) {
+// Causal prefill with at most 64 heads over a bf16 cache on the transposed
+// tensor-memory kernel, a persistent grid of one CTA per SM: the gathered
+// lists (CSA) or every visible entry (HCA, needs the query positions).
+sa_status launch_prefill_tr(const sa::AttnArgs& aa, const sa_cache* c, bool gather, long long BQ, cudaStream_t st) {
     sa::CtArgs a{};
     a.q = aa.q;
     a.K = static_cast<const uint16_t*>(c->k);
@@ -487,6 +488,8 @@ sa_status launch_csa_prefill_tc(const sa::AttnArgs& aa, const sa_cache* c, long 
     a.n = c->n;
     a.idx = aa.idx;
     a.cnt = aa.cnt;
+    a.pos = aa.pos;
+    a.m = c->m;
     a.BQ = BQ;
     a.T = aa.Tq;
     a.H = aa.H;
@@ -497,13 +500,18 @@ sa_status launch_csa_prefill_tc(const sa::AttnArgs& aa, const sa_cache* c, long 
     a.lse = aa.lse;
     static std::atomic<uint64_t> init{0};
     if (!attr_done(init)) {
-        SA_CUDA(cudaFuncSetAttribute(sa::attn_csa_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        SA_CUDA(cudaFuncSetAttribute(sa::attn_prefill_tr_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     sa::kCtSmem));
+        SA_CUDA(cudaFuncSetAttribute(sa::attn_prefill_tr_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      sa::kCtSmem));
         attr_set(init);
     }
     const long long grid = std::min<long long>(BQ, (long long)num_sms());
     if (grid < 1) return SA_OK;
-    sa::attn_csa_prefill_tc_kernel<<<(unsigned)grid, sa::kCtThreads, sa::kCtSmem, st>>>(a);
+    if (gather)
+        sa::attn_prefill_tr_kernel<true><<<(unsigned)grid, sa::kCtThreads, sa::kCtSmem, st>>>(a);
+    else
+        sa::attn_prefill_tr_kernel<false><<<(unsigned)grid, sa::kCtThreads, sa::kCtSmem, st>>>(a);
     SA_LAUNCHED();
     return SA_OK;
 }
@@ -576,14 +584,16 @@ sa_status run_attn(const void* q, int Tq, int H, const sa_cache* c, bool gather,
         a.part_o = reinterpret_cast<float*>(base);
         a.part_lse = reinterpret_cast<float*>(base + up256((size_t)BQ * sp.splits * H * 128 * 4));
     }
-    // dense causal prefill (HCA) on the tensor-memory kernel.  The gathered
-    // (CSA) variant of that kernel is not dispatched: its block-diagonal tiles
-    // (two queries' lists in one 128-row MMA) waste half of every MMA, and on
-    // the 128K-token, 64-head, k = 2048 prefill it took 110-135 ms against
-    // 61 ms for the mma.sync kernel
-    if (prefill && !gather && win == 0 && H == 64 && c->dtype == SA_BF16 && pos) return launch_prefill_tc(a, c, false, st);
-    // the gathered lists of a prefill (one per query) on the transposed tensor-memory kernel
-    if (prefill && gather && H <= 64 && c->dtype == SA_BF16) return launch_csa_prefill_tc(a, c, BQ, st);
+    // causal prefill on the tensor cores: the gathered lists (CSA) on the
+    // transposed kernel; the dense branch (HCA) on it too, or, with
+    // SA_OPT_HCA_PREFILL = 1, on the two-query kernel.  (The gathered variant
+    // of the two-query kernel is not dispatched: its block-diagonal tiles,
+    // two queries' lists in one 128-row MMA, waste half of every MMA.)
+    if (prefill && !gather && win == 0 && c->dtype == SA_BF16 && pos) {
+        if (g_hca_prefill.load() == 1 && H == 64) return launch_prefill_tc(a, c, false, st);
+        if (H <= 64) return launch_prefill_tr(a, c, false, BQ, st);
+    }
+    if (prefill && gather && H <= 64 && c->dtype == SA_BF16) return launch_prefill_tr(a, c, true, BQ, st);
     const int kv = c->dtype == SA_KV_MIXED ? 2 : c->dtype == SA_FP8_E4M3 ? 1 : 0;
     sa_status r = launch_attn(a, gather, kv, BQ, st, chained && pdl_on(), !prefill);
     if (r != SA_OK) return r;
@@ -944,6 +954,10 @@ sa_status sa_set_option(int32_t option, int64_t value) {
             SA_CHECK(value >= 0 && value <= 2, "sa_set_option: SA_OPT_DECODE_FAST=%lld (0, 1 or 2)", (long long)value);
             g_decode_fast.store((int)value);
             return SA_OK;
+        case SA_OPT_HCA_PREFILL:
+            SA_CHECK(value >= 0 && value <= 1, "sa_set_option: SA_OPT_HCA_PREFILL=%lld (0 or 1)", (long long)value);
+            g_hca_prefill.store((int)value);
+            return SA_OK;
         default:
             return fail(SA_ERR_INVALID_ARG, "sa_set_option: unknown option %d", option);
     }
@@ -957,6 +971,9 @@ sa_status sa_get_option(int32_t option, int64_t* value) {
             return SA_OK;
         case SA_OPT_DECODE_FAST:
             *value = g_decode_fast.load();
+            return SA_OK;
+        case SA_OPT_HCA_PREFILL:
+            *value = g_hca_prefill.load();
             return SA_OK;
         default:
             return fail(SA_ERR_INVALID_ARG, "sa_get_option: unknown option %d", option);

@@ -296,6 +296,15 @@ def test_options_on_the_host(L):
         assert S.get_option(S.SA_OPT_DECODE_FAST) == 0
     finally:
         S.set_option(S.SA_OPT_DECODE_FAST, 0)
+    assert L.sa_get_option(_lib.SA_OPT_HCA_PREFILL, ctypes.byref(v)) == _lib.SA_OK and v.value == 0  # default
+    try:
+        S.set_option(S.SA_OPT_HCA_PREFILL, 1)
+        assert S.get_option(S.SA_OPT_HCA_PREFILL) == 1
+        assert L.sa_set_option(_lib.SA_OPT_HCA_PREFILL, 2) == _lib.SA_ERR_INVALID_ARG
+        assert "SA_OPT_HCA_PREFILL" in L.sa_last_error().decode()
+        assert S.get_option(S.SA_OPT_HCA_PREFILL) == 1
+    finally:
+        S.set_option(S.SA_OPT_HCA_PREFILL, 0)
 
 
 def test_trace_calls_need_the_profiling_build(L):

@@ -158,6 +158,25 @@ def test_decode_topk_all_equal_scores_overflow_paths(S, k):
     assert (idx == np.arange(k)[None, :]).all() and (cnt == k).all()
 
 
+def test_decode_topk_mixed_batch(S):
+    # 37 sequences of every kind in one call: the score kernel hands its
+    # 128-row tiles out dynamically, skipping sequences with n <= k and the
+    # tiles past each length, and finishes each sequence when its last tile
+    # is counted (whichever CTA scanned it)
+    B, Lcap, k = 37, 9000, 300
+    rng = np.random.default_rng(17)
+    fixed = [0, 3, 4 * k, 4 * k + 4, 4 * (k + 1) + 3, 512 * 4, 512 * 4 + 4, Lcap, Lcap - 1, 128 * 4 * 7]
+    lengths = fixed + rng.integers(0, Lcap + 1, size=B - len(fixed)).tolist()
+    inp = Inputs(306, B, Lcap, 8, lengths=lengths)
+    _, _, _, idx, cnt = _topk_case(S, inp, k)
+    for b in range(B):
+        cs = inp.oracle_seq(b)
+        s = O.index_scores(inp.qI[b], cs.cidx)
+        ridx, rcnt = O.topk(s, k)
+        assert cnt[b] == rcnt, b
+        assert np.array_equal(idx[b], ridx), b
+
+
 def test_decode_topk_short_and_empty(S):
     B, Lcap, k = 3, 512, 200
     inp = Inputs(303, B, Lcap, 8, lengths=[512, 3, 0])         # 128, 0, 0 entries
