@@ -105,6 +105,9 @@ struct CtStatic {
     float l[64];       // the query's sums, at its end
     uint32_t tmem;
     uint64_t bar_s[2], bar_o[2];  // S^T(t) and O^T(t) complete on barrier t & 1
+#ifdef SA_TRACE
+    unsigned long long tt[kCtRows / 8][6];  // profiling build: thread 0's step times of one query's tiles
+#endif
 };
 
 // 16 consecutive fp32 columns of this thread's TMEM lane: loaded without
@@ -276,10 +279,22 @@ __global__ void __launch_bounds__(kCtThreads, 1) attn_prefill_tr_kernel(CtArgs a
         }
         int jn = load_idx(2);  // the entries of tile i + 2, loaded a tile ahead
 
+        // profiling build: thread 0's step times for the gathered lists of
+        // CTA 0's last two queries (full lists), written after each query
+        const bool traced = GATHER && blockIdx.x == 0 && bq / gridDim.x + 2 >= a.BQ / gridDim.x;
+        auto tnow = [&](int i, int step) {
+#ifdef SA_TRACE
+            if (traced && tid == 0 && i < kCtRows / 8) S.tt[i][step] = SA_TRACE_NOW();
+#else
+            (void)traced, (void)i, (void)step;
+#endif
+        };
         for (int i = 0; i < ntiles; ++i) {
             const int bi = i & 1;
+            tnow(i, 0);
             // 1. S^T(i) complete; K(i + 2) into the buffer it has read
             wait_s(i);
+            tnow(i, 1);
             tc_fence_after();
             const int j2 = entry(i + 2, jn);
             if (i + 2 < ntiles) copy_rows(Kb, sm + kCtK + bi * 32768, j2);
@@ -363,6 +378,7 @@ __global__ void __launch_bounds__(kCtThreads, 1) attn_prefill_tr_kernel(CtArgs a
                 *reinterpret_cast<uint4*>(sm + kCtP + bi * 16384 + (e >> 3) * 1024 + (e & 7) * 128 +
                                           ((cc ^ (e & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
+            tnow(i, 2);
             // 3. V(i) and K(i + 1) landed (the two newest groups, K(i + 2) and
             // V(i + 1), may still be in flight)
             cp_async_wait<2>();
@@ -372,6 +388,7 @@ __global__ void __launch_bounds__(kCtThreads, 1) attn_prefill_tr_kernel(CtArgs a
                 bad = true;
                 break;
             }
+            tnow(i, 3);
             // 4. S^T(i + 1) (the next softmax waits for it), then O^T += V(i)^T P^T(i)
             if (tid == 0) {
                 tc_fence_after();
@@ -391,11 +408,19 @@ __global__ void __launch_bounds__(kCtThreads, 1) attn_prefill_tr_kernel(CtArgs a
                 tc_commit(&S.bar_o[bi]);
                 ++(bi ? io1 : io0);
             }
+            tnow(i, 4);
             // 5. O^T(i - 1) complete: V(i + 2) into the buffer it has read
             if (i > 0) wait_o_until(i - 1);
             if (i + 2 < ntiles) copy_rows(Vb, sm + kCtV + ((i + 2) % 3) * 32768, j2);
             cp_async_commit();
+            tnow(i, 5);
         }
+#ifdef SA_TRACE
+        if (traced && tid == 0)
+            for (int i = 0; i < min(ntiles, kCtRows / 8); ++i)
+                for (int step = 0; step < 6; ++step)
+                    SA_TRACE_PUT(S.tt[i][step], TR_PATTN, step, (uint32_t)((bq / gridDim.x) % 2) * 16 + i);
+#endif
         if (ntiles > 0 && !bad) wait_o_until(ntiles - 1);  // the query's last O^T group
         cp_async_wait<0>();
         tc_fence_after();

@@ -35,6 +35,7 @@ __device__ __forceinline__ void flag(uint32_t f) { atomicOr(&g_status, f); }
 enum : uint32_t {
     TR_SCORE = 1, TR_FILTER = 2, TR_RESOLVE = 3, TR_EMIT = 4, TR_ATTN = 5, TR_COMBINE = 6, TR_SCORE_FP4 = 7,
     TR_PSCORE = 8, TR_PSELECT = 9, TR_PSCORE_FP4 = 10, TR_PSELECT2 = 11, TR_BOUND = 12, TR_FAST = 13, TR_PSELECT4 = 14,
+    TR_PATTN = 15,
 };
 #ifdef SA_TRACE
 struct TraceRec {
@@ -61,8 +62,27 @@ __device__ __forceinline__ void trace_mark(uint32_t kernel, uint32_t phase) {
     __syncwarp();
 }
 #define SA_TRACE_MARK(kernel, phase) ::sa::trace_mark((kernel), (phase))
+// Marks inside a tight loop: the time is read into a register or shared
+// memory (SA_TRACE_NOW) and the record is written later by one thread
+// (SA_TRACE_PUT), with `unit` in the record's CTA field (a tile, say).
+__device__ __forceinline__ unsigned long long trace_now() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void trace_put(unsigned long long t, uint32_t kernel, uint32_t phase, uint32_t unit) {
+    if (g_trace_buf == nullptr) return;
+    uint32_t sm;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+    const uint32_t i = atomicAdd(&g_trace_n, 1u);
+    if (i < g_trace_cap) g_trace_buf[i] = {t, (uint16_t)kernel, (uint16_t)phase, (uint16_t)sm, (uint16_t)unit};
+}
+#define SA_TRACE_NOW() ::sa::trace_now()
+#define SA_TRACE_PUT(t, kernel, phase, unit) ::sa::trace_put((t), (kernel), (phase), (unit))
 #else
 #define SA_TRACE_MARK(kernel, phase) ((void)0)
+#define SA_TRACE_NOW() 0ull
+#define SA_TRACE_PUT(t, kernel, phase, unit) ((void)0)
 #endif
 
 // Iteration limit of every spin on an mbarrier: each try_wait may itself

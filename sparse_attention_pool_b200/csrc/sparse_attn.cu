@@ -512,7 +512,17 @@ sa_status launch_prefill_tr(const sa::AttnArgs& aa, const sa_cache* c, bool gath
         sa::attn_prefill_tr_kernel<true><<<(unsigned)grid, sa::kCtThreads, sa::kCtSmem, st>>>(a);
     else
         sa::attn_prefill_tr_kernel<false><<<(unsigned)grid, sa::kCtThreads, sa::kCtSmem, st>>>(a);
-    SA_LAUNCHED();
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        cudaFuncAttributes fa{};
+        cudaFuncGetAttributes(&fa, gather ? (const void*)sa::attn_prefill_tr_kernel<true>
+                                          : (const void*)sa::attn_prefill_tr_kernel<false>);
+        return fail(SA_ERR_CUDA, "kernel launch: %s (transposed prefill kernel: %d threads, %d registers, "
+                    "%zu + %d bytes of shared memory; the kernel allows %d threads, %d bytes dynamic)",
+                    cudaGetErrorString(e), sa::kCtThreads, fa.numRegs, fa.sharedSizeBytes, sa::kCtSmem,
+                    fa.maxThreadsPerBlock, fa.maxDynamicSharedSizeBytes);
+    }
+    ++g_launches;
     return SA_OK;
 }
 

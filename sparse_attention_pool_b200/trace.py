@@ -28,7 +28,7 @@ from ._lib import check, lib
 
 KERNELS = {1: "score", 2: "filter", 3: "resolve", 4: "emit", 5: "attn_split", 6: "attn_merge", 7: "score_fp4",
            8: "prefill_score", 9: "prefill_select", 10: "prefill_score_fp4", 11: "prefill_select2", 12: "bound",
-           13: "select_fast", 14: "prefill_select4"}
+           13: "select_fast", 14: "prefill_select4", 15: "prefill_attn"}
 PHASES = {
     "score": ["start", "scan done", "threshold found"],
     "score_fp4": ["start", "scan done", "threshold found"],
@@ -50,6 +50,8 @@ PHASES = {
     "select_fast": ["start", "list loaded", "t~ known", "band rescored", "cut done", "selected"],
     # prefill selection, fourth form: one CTA per query
     "prefill_select4": ["start", "keys staged", "threshold found", "runs counted", "end"],
+    # per tile of a query's list (the record's CTA field holds the tile)
+    "prefill_attn": ["tile start", "S ready", "softmax done", "copies landed", "MMAs issued", "V copies out"],
 }
 RECORD = np.dtype([("t", "<u8"), ("kernel", "<u2"), ("phase", "<u2"), ("sm", "<u2"), ("cta", "<u2")])
 

@@ -91,6 +91,7 @@ g = inp.to_device()
 csa, _ = compress_on_gpu(S, g, B, T)
 pos = torch.arange(T, dtype=torch.int32, device="cuda").view(1, T).contiguous()
 ws = S.alloc_workspace(S.workspace_size(S.SA_OP_INDEX_TOPK, B, T, 8, csa.Ncap, 0, k))
+S.set_option(S.SA_OPT_PREFILL_SELECT, 1)   # the first selection form's phases
 i0, c0 = S.csa_index_topk(g["qI"], csa, k, ws, q_pos=pos)   # untraced
 i0, c0 = i0.clone(), c0.clone()
 torch.cuda.synchronize()
@@ -111,6 +112,20 @@ rows = trace.cta_phase_durations(rec, "prefill_select")
 assert len(rows) == 6 and all(r["runs"] == full for r in rows), rows
 for r in rows + trace.cta_phase_durations(rec, "prefill_score"):
     print(r)
+# the default (fourth) form: its own phases, the same indices
+S.set_option(S.SA_OPT_PREFILL_SELECT, 4)
+buf = trace.install(1 << 17)
+i4, c4 = S.csa_index_topk(g["qI"], csa, k, ws, q_pos=pos)
+rec = trace.records(buf)
+trace.uninstall()
+S.read_device_status()
+assert torch.equal(i0, i4) and torch.equal(c0, c4)
+sel = rec[rec["kernel"] == 14]
+assert int((sel["phase"] == 0).sum()) == T, int((sel["phase"] == 0).sum())
+for ph in range(1, 5):
+    assert int((sel["phase"] == ph).sum()) == full, (ph, int((sel["phase"] == ph).sum()))
+rows = trace.cta_phase_durations(rec, "prefill_select4")
+assert len(rows) == 4 and all(r["runs"] == full for r in rows), rows
 print("TRACE_PREFILL_OK")
 """
 
