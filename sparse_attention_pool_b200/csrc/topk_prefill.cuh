@@ -68,30 +68,36 @@ __global__ void __launch_bounds__(kPsThreads, 2) score_prefill_kernel(TopkPrefil
     if (e0 >= s_maxvis) return;  // no query of this tile sees these entries
     SA_TRACE_MARK(TR_PSCORE, 0);
 
-    {  // queries: q * 2^768 as fp64, dim-major
+    {  // every load of the tile goes out at once, then the stores:
+       // queries as q * 2^768 in fp64, dim-major; keys as packed bf16 pairs, [dim pair][entry]
         const int ql = tid & 63;
-        const bool ok = ql0 + ql < a.qb;
-        const uint4* src = reinterpret_cast<const uint4*>(a.q_idx + ((size_t)a.b * a.Tq + a.t0 + ql0 + ql) * 64);
-        for (int c = tid >> 6; c < 8; c += kPsThreads / 64) {
-            const uint4 w = ok ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        const bool okq = ql0 + ql < a.qb;
+        const uint4* srcq = reinterpret_cast<const uint4*>(a.q_idx + ((size_t)a.b * a.Tq + a.t0 + ql0 + ql) * 64);
+        const int e = tid & 127;
+        const bool okk = e0 + e < a.Ncap;
+        const uint4* srck = reinterpret_cast<const uint4*>(a.kidx + ((size_t)a.b * a.Ncap + e0 + e) * 64);
+        uint4 wq[2], wk[4];
+#pragma unroll
+        for (int v = 0; v < 2; ++v) wq[v] = okq ? __ldg(srcq + (tid >> 6) + 4 * v) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) wk[v] = okk ? __ldg(srck + (tid >> 7) + 2 * v) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+            const int c = (tid >> 6) + 4 * v;
+            const uint32_t ws[4] = {wq[v].x, wq[v].y, wq[v].z, wq[v].w};
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 sQ[(8 * c + 2 * u) * kPsQ + ql] = (double)bf16lo_f32(ws[u]) * 0x1p768;
                 sQ[(8 * c + 2 * u + 1) * kPsQ + ql] = (double)bf16hi_f32(ws[u]) * 0x1p768;
             }
         }
-    }
-    {  // keys: packed bf16 pairs, [dim pair][entry]
-        const int e = tid & 127;
-        const bool ok = e0 + e < a.Ncap;
-        const uint4* src = reinterpret_cast<const uint4*>(a.kidx + ((size_t)a.b * a.Ncap + e0 + e) * 64);
-        for (int c = tid >> 7; c < 8; c += kPsThreads / 128) {
-            const uint4 w = ok ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
-            sK[(4 * c + 0) * kPsE + e] = w.x;
-            sK[(4 * c + 1) * kPsE + e] = w.y;
-            sK[(4 * c + 2) * kPsE + e] = w.z;
-            sK[(4 * c + 3) * kPsE + e] = w.w;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            const int c = (tid >> 7) + 2 * v;
+            sK[(4 * c + 0) * kPsE + e] = wk[v].x;
+            sK[(4 * c + 1) * kPsE + e] = wk[v].y;
+            sK[(4 * c + 2) * kPsE + e] = wk[v].z;
+            sK[(4 * c + 3) * kPsE + e] = wk[v].w;
         }
     }
     __syncthreads();

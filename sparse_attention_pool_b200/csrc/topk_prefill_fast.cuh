@@ -57,16 +57,27 @@ __global__ void __launch_bounds__(kP4Threads, 1) select_prefill_v4_kernel(TopkPr
     float s1 = 0.f, s2 = 0.f;
     if (nv <= kP4Keys) {
         const int n4 = (nv + 3) >> 2;
-        for (int i = tid; i < n4; i += kP4Threads) {
-            const uint4 w = reinterpret_cast<const uint4*>(grow)[i];
-            reinterpret_cast<uint4*>(skeys)[i] = w;
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        // four 16-byte loads in flight per thread, then their stores and sums
+        for (int i0 = tid; i0 < n4; i0 += 4 * kP4Threads) {
+            uint4 w[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                if (4 * i + u < nv) {
-                    const float x = key_to_float(ws[u]);
-                    s1 += x;
-                    s2 = fmaf(x, x, s2);
+            for (int v = 0; v < 4; ++v) {
+                const int i = i0 + v * kP4Threads;
+                w[v] = i < n4 ? reinterpret_cast<const uint4*>(grow)[i] : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const int i = i0 + v * kP4Threads;
+                if (i >= n4) break;
+                reinterpret_cast<uint4*>(skeys)[i] = w[v];
+                const uint32_t ws[4] = {w[v].x, w[v].y, w[v].z, w[v].w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if (4 * i + u < nv) {
+                        const float x = key_to_float(ws[u]);
+                        s1 += x;
+                        s2 = fmaf(x, x, s2);
+                    }
                 }
             }
         }
