@@ -387,14 +387,21 @@ sa_status sa_selftest_wait_timeout(uint32_t wait_tries, void* stream);
  * kernel: 1 indexer score, 2 filter, 3 resolve, 4 emit, 5 attention split,
  * 6 split merge, 7 FP4 indexer score, 8 prefill indexer score, 9 prefill
  * selection, 10 FP4 prefill indexer score, 11 prefill selection (second
- * form, SA_OPT_PREFILL_SELECT = 2).  Phases: score 0 start, 1 scan
+ * form, SA_OPT_PREFILL_SELECT = 2), 12 sampled bound and 13 fast selection
+ * (SA_OPT_DECODE_FAST = 1), 14 prefill selection (fourth form, the
+ * default), 15 prefill attention on the transposed kernel (per tile of the
+ * gathered lists of CTA 0's last two queries; the record's cta field holds
+ * the tile: 16 * (query parity) + tile).  Phases: score 0 start, 1 scan
  * done, 2 threshold found (last CTA); filter 0 start, 1 rows done; resolve 0
  * start, 1 counts scanned, 2 candidates gathered, 3 t~ known, 4 band done,
  * 5 cut done, 6 positions written; emit, attention 0 start, 1 end; merge 0;
  * prefill scores (CTAs whose tile some query sees) 0 start, 1 operands
  * staged, 2 end; prefill selection (one CTA per query) 0 start, then, when
  * the query sees more than k entries, 1 keys staged, 2..4 digits 1..3
- * found, 5 ties resolved (second form: per-warp counts done), 6 end.
+ * found, 5 ties resolved (second form: per-warp counts done), 6 end;
+ * fourth form 0 start, 1 keys staged, 2 threshold found, 3 runs counted,
+ * 4 end; prefill attention 0 tile start, 1 scores ready, 2 softmax done,
+ * 3 copies landed (barrier), 4 MMAs issued, 5 next copies out.
  * sa_trace_install(buf, capacity) waits for `stream`, then makes buf (device
  * memory, 16-byte aligned, capacity records) the destination and resets the
  * count; capacity 0 switches tracing off.  sa_trace_count waits for `stream`

@@ -491,15 +491,19 @@ __global__ void __launch_bounds__(kScThreads, 3)
 
     // The last CTA of the sequence to finish finds, once for every filter
     // CTA, the bin d1 of the k-th largest key, the count of keys above it
-    // and the sequence's bound E.  (Ticket pattern: no CTA waits.)
+    // and the sequence's bound E.  (Ticket pattern: no CTA waits.  The
+    // ticket is an acquire-release add after a barrier: it publishes this
+    // CTA's histogram and bound, and the last CTA sees every other CTA's.)
     uint32_t* tot = a.totals + (size_t)b * kTotals;
-    __threadfence();
     __syncthreads();
     SA_TRACE_MARK(TR_SCORE, 1);
-    if (tid == 0) s_last = atomicAdd(tot + kTotTicket, 1u) == gridDim.x - 1;
+    if (tid == 0) {
+        uint32_t old;
+        asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(old) : "l"(tot + kTotTicket) : "memory");
+        s_last = old == gridDim.x - 1;
+    }
     __syncthreads();
     if (!s_last) return;
-    __threadfence();
     constexpr int NPT = kBins / kScThreads;  // 16 bins per thread
     uint32_t hb[NPT];
     {
