@@ -537,12 +537,13 @@ uint64_t sa_launch_count(void);
  *       3            form 2 in 512-thread CTAs that read the keys from the
  *                    scratch on every pass instead of staging them, so
  *                    that three queries share an SM;
- *       4 (default)  one 1024-thread CTA per query: the scores' mean and
- *                    deviation, one pass over 256 linear score bins counted
- *                    in per-warp histograms, the threshold ranked inside
- *                    its bin, then one counting pass and an ordered output
- *                    by contiguous runs (28 ms of selection became 12 ms on
- *                    the 128K-token prefill with k = 2048).
+ *       4 (default)  one 512-thread CTA per query, two per SM: the
+ *                    scores' mean and deviation, one pass over 256 linear
+ *                    score bins counted in per-warp histograms, the
+ *                    threshold ranked inside its bin, then one counting
+ *                    pass and an ordered output by contiguous runs (28 ms
+ *                    of selection became 12 ms on the 128K-token prefill
+ *                    with k = 2048).
  *   SA_OPT_DECODE_FAST  the indexer and top-k of the hybrid decode calls
  *     (hybrid_attn_decode, hybrid_attn_decode_swa) with bf16 indexer keys
  *     and k <= 2048.  Every value gives the same indices (the exact top-k)

@@ -5,7 +5,8 @@
 // is the same as every other form: the k largest, ties at the threshold by
 // lowest index, indices ascending.
 //
-// One CTA of 1024 threads per query, the keys staged in shared memory:
+// One CTA of 512 threads per query (two per SM), the keys staged in shared
+// memory (the first 24K; a longer row is read from the scratch past them):
 //   1. mean and standard deviation of the scores (one block reduction);
 //   2. one histogram pass over 256 linear bins of the score on
 //      [mean - 4 sd, mean + 4 sd] (clamped at both ends), counted in
@@ -25,14 +26,14 @@
 
 namespace sa {
 
-constexpr int kP4Threads = 1024;
-constexpr int kP4Keys = 40 * 1024;  // keys staged in shared memory (160 KB); more are read from the scratch
+constexpr int kP4Threads = 512;     // two CTAs (queries) per SM
+constexpr int kP4Keys = 24 * 1024;  // keys staged in shared memory (96 KB); the rest are read from the scratch
 constexpr int kP4Bins = 256;        // linear score bins of the first pass
-constexpr int kP4List = 1024;       // keys of the threshold's bin ranked pairwise
+constexpr int kP4List = kP4Threads; // keys of the threshold's bin ranked pairwise (one per thread)
 constexpr size_t kP4Smem = (size_t)kP4Keys * 4 + (size_t)(kP4Threads / 32) * kP4Bins * 4;
 
-__global__ void __launch_bounds__(kP4Threads, 1) select_prefill_v4_kernel(TopkPrefillArgs a) {
-    extern __shared__ __align__(16) uint32_t p4_sm[];  // [kP4Keys] keys, [32 warps][kP4Bins] histograms
+__global__ void __launch_bounds__(kP4Threads, 2) select_prefill_v4_kernel(TopkPrefillArgs a) {
+    extern __shared__ __align__(16) uint32_t p4_sm[];  // [kP4Keys] keys, [16 warps][kP4Bins] histograms
     uint32_t* skeys = p4_sm;
     uint32_t* whist = p4_sm + kP4Keys;
     __shared__ float sf[2][32];
@@ -52,11 +53,12 @@ __global__ void __launch_bounds__(kP4Threads, 1) select_prefill_v4_kernel(TopkPr
         return;
     }
     const uint32_t* grow = a.keys + (size_t)ql * a.KS;
-    const uint32_t* kp = grow;
+    // the query's keys: the first kP4Keys staged in shared memory, the rest from the scratch
+    auto kp = [&](int i) -> uint32_t { return i < kP4Keys ? skeys[i] : __ldg(grow + i); };
     // 1. stage the keys (16-byte rows: KS is a multiple of 128) and sum the scores
     float s1 = 0.f, s2 = 0.f;
-    if (nv <= kP4Keys) {
-        const int n4 = (nv + 3) >> 2;
+    {
+        const int n4 = (min(nv, kP4Keys) + 3) >> 2;
         // four 16-byte loads in flight per thread, then their stores and sums
         for (int i0 = tid; i0 < n4; i0 += 4 * kP4Threads) {
             uint4 w[4];
@@ -81,9 +83,7 @@ __global__ void __launch_bounds__(kP4Threads, 1) select_prefill_v4_kernel(TopkPr
                 }
             }
         }
-        kp = skeys;
-    } else {
-        for (int i = tid; i < nv; i += kP4Threads) {
+        for (int i = kP4Keys + tid; i < nv; i += kP4Threads) {
             const float x = key_to_float(__ldg(grow + i));
             s1 += x;
             s2 = fmaf(x, x, s2);
@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(kP4Threads, 1) select_prefill_v4_kernel(TopkPr
             return f <= 0.f ? 0 : f >= (float)(kP4Bins - 1) ? kP4Bins - 1 : (int)f;
         };
         uint32_t* wh = whist + warp * kP4Bins;
-        for (int i = tid; i < nv; i += kP4Threads) red_add_shared(&wh[bin_of(kp[i])], 1u);
+        for (int i = tid; i < nv; i += kP4Threads) red_add_shared(&wh[bin_of(kp(i))], 1u);
         __syncthreads();
         // bins summed over the warps, the highest bin on thread 0; the bin d of the k-th largest
         uint32_t c = 0;
@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(kP4Threads, 1) select_prefill_v4_kernel(TopkPr
         uint32_t* list = whist;
         if (d >= 0) {
             for (int i = tid; i < nv; i += kP4Threads) {
-                const uint32_t key = kp[i];
+                const uint32_t key = kp(i);
                 if (bin_of(key) == d) {
                     const uint32_t q = atom_add_shared(&s_nd, 1u);
                     if (q < (uint32_t)kP4List) list[q] = key;
@@ -170,14 +170,14 @@ __global__ void __launch_bounds__(kP4Threads, 1) select_prefill_v4_kernel(TopkPr
     SA_TRACE_MARK(TR_PSELECT4, 2);
     if (!found) {  // byte-digit passes over every key
         __syncthreads();
-        T = kth_largest([&](uint32_t i) { return kp[i]; }, (uint32_t)nv, (uint32_t)k, whist, sh64, res);
+        T = kth_largest([&](uint32_t i) { return kp((int)i); }, (uint32_t)nv, (uint32_t)k, whist, sh64, res);
     }
     // 4. ordered output: each thread's contiguous run of keys
     const int per = (nv + kP4Threads - 1) / kP4Threads;
     const int j0 = min(nv, tid * per), j1 = min(nv, j0 + per);
     uint32_t n_above = 0, n_tie = 0;
     for (int j = j0; j < j1; ++j) {
-        const uint32_t key = kp[j];
+        const uint32_t key = kp(j);
         n_above += key > T;
         n_tie += key == T;
     }
@@ -190,7 +190,7 @@ __global__ void __launch_bounds__(kP4Threads, 1) select_prefill_v4_kernel(TopkPr
     uint32_t o = pa + min(pt, take);
     uint32_t ties_before = pt;
     for (int j = j0; j < j1; ++j) {
-        const uint32_t key = kp[j];
+        const uint32_t key = kp(j);
         bool sel = key > T;
         if (key == T) {
             sel = ties_before < take;
