@@ -1068,9 +1068,10 @@ def main():
     ap.add_argument("--decode-fast", type=int, default=0, choices=[0, 1],
                     help="decode only: the indexer + top-k kernels (SA_OPT_DECODE_FAST: 0 the general ones, "
                          "1 the sampled-bound fast path; same indices and outputs)")
-    ap.add_argument("--hca-prefill", type=int, default=0, choices=[0, 1],
-                    help="prefill only: the HCA attention kernel (SA_OPT_HCA_PREFILL: 0 transposed tiles, "
-                         "1 two queries per MMA)")
+    ap.add_argument("--hca-prefill", type=int, default=0, choices=[0, 1, 2],
+                    help="prefill only: the HCA attention kernel (SA_OPT_HCA_PREFILL: 0 transposed tiles, two "
+                         "query positions per tile with 64 heads; 1 the two-query kernel; 2 transposed tiles, one "
+                         "query at a time)")
     ap.add_argument("--prefill-select", type=int, default=4, choices=[1, 2, 3, 4],
                     help="prefill only: the top-k selection kernel (SA_OPT_PREFILL_SELECT; same indices)")
     ap.add_argument("--trace", default="",

@@ -563,10 +563,13 @@ uint64_t sa_launch_count(void);
  *     query positions and a bf16 cache (hca_dense_attn with q_pos, the
  *     hybrid prefill calls).  Same outputs up to the order of the fp32
  *     sums (both within the bf16 tolerance of the definition):
- *       0 (default)  the transposed tensor-memory kernel (128 entries x the
- *                    query's heads per MMA, one query at a time; <= 64 heads);
+ *       0 (default)  the transposed tensor-memory kernel (128 entries per
+ *                    MMA): with exactly 64 heads and an even m, two query
+ *                    positions per tile (2 x 64 heads as the MMA's N);
+ *                    otherwise one query at a time (<= 64 heads);
  *       1            the two-query kernel (2 queries x 64 heads per 128-row
- *                    MMA; exactly 64 heads).
+ *                    MMA; exactly 64 heads);
+ *       2            the transposed kernel one query at a time.
  * sa_set_option returns SA_ERR_INVALID_ARG for an unknown option or value;
  * sa_get_option writes the current value to *value.                        */
 typedef enum { SA_OPT_PREFILL_SELECT = 1, SA_OPT_DECODE_FAST = 2, SA_OPT_HCA_PREFILL = 3 } sa_option;

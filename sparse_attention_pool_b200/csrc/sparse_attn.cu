@@ -504,7 +504,18 @@ sa_status launch_prefill_tr(const sa::AttnArgs& aa, const sa_cache* c, bool gath
                                      sa::kCtSmem));
         SA_CUDA(cudaFuncSetAttribute(sa::attn_prefill_tr_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      sa::kCtSmem));
+        SA_CUDA(cudaFuncSetAttribute(sa::attn_prefill_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     sa::kPrSmem));
         attr_set(init);
+    }
+    if (!gather && aa.H == 64 && (c->m & 1) == 0 && g_hca_prefill.load() == 0) {
+        // dense, 64 heads: two query positions per tile
+        const long long pairs = (long long)c->B * ((aa.Tq + 1) / 2);
+        const long long grid = std::min<long long>(pairs, (long long)num_sms());
+        if (grid < 1) return SA_OK;
+        sa::attn_prefill_pair_kernel<<<(unsigned)grid, sa::kPrThreads, sa::kPrSmem, st>>>(a);
+        SA_LAUNCHED();
+        return SA_OK;
     }
     const long long grid = std::min<long long>(BQ, (long long)num_sms());
     if (grid < 1) return SA_OK;
@@ -965,7 +976,7 @@ sa_status sa_set_option(int32_t option, int64_t value) {
             g_decode_fast.store((int)value);
             return SA_OK;
         case SA_OPT_HCA_PREFILL:
-            SA_CHECK(value >= 0 && value <= 1, "sa_set_option: SA_OPT_HCA_PREFILL=%lld (0 or 1)", (long long)value);
+            SA_CHECK(value >= 0 && value <= 2, "sa_set_option: SA_OPT_HCA_PREFILL=%lld (0, 1 or 2)", (long long)value);
             g_hca_prefill.store((int)value);
             return SA_OK;
         default:

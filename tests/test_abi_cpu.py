@@ -300,7 +300,10 @@ def test_options_on_the_host(L):
     try:
         S.set_option(S.SA_OPT_HCA_PREFILL, 1)
         assert S.get_option(S.SA_OPT_HCA_PREFILL) == 1
-        assert L.sa_set_option(_lib.SA_OPT_HCA_PREFILL, 2) == _lib.SA_ERR_INVALID_ARG
+        S.set_option(S.SA_OPT_HCA_PREFILL, 2)
+        assert S.get_option(S.SA_OPT_HCA_PREFILL) == 2
+        S.set_option(S.SA_OPT_HCA_PREFILL, 1)
+        assert L.sa_set_option(_lib.SA_OPT_HCA_PREFILL, 3) == _lib.SA_ERR_INVALID_ARG
         assert "SA_OPT_HCA_PREFILL" in L.sa_last_error().decode()
         assert S.get_option(S.SA_OPT_HCA_PREFILL) == 1
     finally:
