@@ -23,6 +23,12 @@ on, checked against the oracle and against plain sorting:
   per-warp runs counted and written with the ties at the threshold taken in
   index order -- the model's indices must equal the oracle's top-k.
 
+* the query pairs of the dense prefill kernel (attn_prefill_pair_kernel):
+  with m even, positions 2p and 2p + 1 see the same entries under the causal
+  rule (c + 1) m <= t, so one tile of rows serves both; and the fourth
+  selection form's run split (per-thread contiguous runs, ties taken in
+  index order from the runs' exclusive prefixes) equals plain sorting.
+
 The models restate the kernels' schemes in Python; the CUDA kernels
 themselves are checked against the oracle by the GPU tests.
 """
@@ -431,3 +437,52 @@ def test_fp4_scores_of_huge_blocks_match_the_oracle():
         assert _f2u(got) == _f2u(ref[j]), j
         slow += max(int(ks[j][b]) + int(qe[b]) - 256 for b in range(2)) > 114
     assert slow > n // 4  # the fp64 routine's range is exercised
+
+
+def test_query_pairs_see_the_same_entries():
+    # entry c is visible at position t iff (c + 1) * m <= t, i.e. the count is t // m
+    for m in (2, 4, 8, 128, 1024):
+        for t0 in range(0, 4 * m + 7, 2):
+            assert t0 // m == (t0 + 1) // m, (m, t0)
+    # an odd m breaks it (the kernel takes the pair path only for even m)
+    assert any(t0 // 3 != (t0 + 1) // 3 for t0 in range(0, 12, 2))
+
+
+def _runs_select(keys, k, threads):
+    """The fourth selection form's output stage: T = the k-th largest key;
+    per thread, a contiguous run of keys; counts of keys above and equal to
+    T per run; exclusive prefixes; each run writes its keys above T and its
+    share of the ties (lowest indices first) from its prefix."""
+    n = len(keys)
+    T = sorted(keys, reverse=True)[k - 1]
+    per = (n + threads - 1) // threads
+    runs = [(min(n, t * per), min(n, t * per + per)) for t in range(threads)]
+    above = [sum(1 for j in range(a, b) if keys[j] > T) for a, b in runs]
+    ties = [sum(1 for j in range(a, b) if keys[j] == T) for a, b in runs]
+    tot_a = sum(above)
+    take = k - tot_a
+    out = [None] * k
+    pa = pt = 0
+    for (a, b), na, nt in zip(runs, above, ties):
+        o = pa + min(pt, take)
+        tb = pt
+        for j in range(a, b):
+            sel = keys[j] > T
+            if keys[j] == T:
+                sel = tb < take
+                tb += 1
+            if sel:
+                out[o] = j
+                o += 1
+        pa += na
+        pt += nt
+    return out
+
+
+def test_prefill_select_v4_runs_match_sorting():
+    rng = np.random.default_rng(41)
+    for n, k, threads, levels in ((5000, 300, 512, 40), (2049, 2048, 512, 3), (700, 1, 64, 5), (3000, 2999, 512, 1)):
+        keys = rng.integers(0, levels, size=n).tolist()   # heavy ties
+        got = _runs_select(keys, k, threads)
+        order = sorted(range(n), key=lambda j: (-keys[j], j))[:k]
+        assert got == sorted(order), (n, k, threads)
